@@ -1,0 +1,401 @@
+"""Pins of the fp64 oracle against what the SparseLoRA pages and the mathematics fix:
+worked examples computed by hand (tests/golden/worked_examples.json), closed forms
+(Eckart-Young, full-rank estimator), special cases (keep ratio 1 = dense LoRA, equal
+head counts = MHA formula), brute force on tiny inputs and central finite differences.
+No GPU is needed."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from contextual_sparsity_lora_b200 import inputs
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+def arr(x):
+    return np.asarray([[float(v) for v in row] for row in x]) if isinstance(x[0], list) else \
+        np.asarray([float(v) for v in x])
+
+
+# --------------------------------------------------------------------------- worked examples
+
+def test_l2_norm_worked_example():
+    g = GOLD["l2_norm"]
+    np.testing.assert_allclose(oracle.score_l2(arr(g["Y"])), g["scores"], rtol=0, atol=1e-15)
+
+
+def test_qk_norm_worked_example_mha():
+    g = GOLD["qk_norm"]
+    s = oracle.score_qk(arr(g["Q"]), arr(g["K"]), n_q_heads=1, n_kv_heads=1, head_dim=2)
+    np.testing.assert_allclose(s, g["scores"], rtol=0, atol=1e-15)
+
+
+def test_qk_norm_worked_example_gqa():
+    g = GOLD["qk_norm_gqa"]
+    s = oracle.score_qk(arr(g["Q"]), arr(g["K"]), g["n_q_heads"], g["n_kv_heads"], g["head_dim"])
+    np.testing.assert_allclose(s, g["scores"], rtol=0, atol=1e-15)
+
+
+def test_silu_values():
+    g = GOLD["silu"]
+    np.testing.assert_allclose(oracle.silu(np.array(g["z"])), g["value"], rtol=1e-15, atol=0)
+
+
+def test_select_worked_example():
+    g = GOLD["select_top"]
+    s = np.array([float(v) for v in g["scores"]])
+    for n, want in g["cases"]:
+        assert oracle.select_top(s, n).tolist() == want
+
+
+def test_keep_count_worked_examples():
+    for ratio, n, want in GOLD["keep_count"]["cases"]:
+        assert oracle.keep_count(ratio, n) == want
+
+
+@pytest.mark.parametrize("name", ["linear_out_slice", "linear_in_slice"])
+def test_linear_worked_example(name):
+    g = GOLD[name]
+    kind = "out" if name == "linear_out_slice" else "in"
+    X, W, A, B = (arr(g[k]) for k in ("X", "W", "A", "B"))
+    ctx = np.array(g["ctx"])
+    Y = oracle.sparse_linear_fwd(X, W, A, B, g["scale"], ctx, g["idx"], kind)
+    np.testing.assert_allclose(Y, arr(g["Y"]), rtol=0, atol=1e-14)
+    if "dY" in g:
+        dX, dA, dB = oracle.sparse_linear_bwd(X, arr(g["dY"]), W, A, B, g["scale"], ctx, g["idx"], kind)
+        np.testing.assert_allclose(dX, arr(g["dX"]), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dA, arr(g["dA"]), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dB, arr(g["dB"]), rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- estimator / factors
+
+def _f64_weight(d_out, d_in, alpha, k, seed):
+    gen = inputs.generator(seed)
+    return inputs.spectral_weight(d_out, d_in, alpha, k, gen, "cpu", torch.float64, torch.float64,
+                                  keep_factors=True)
+
+
+@pytest.mark.parametrize("shape", [(96, 40), (40, 96), (64, 64)])
+def test_svd_factors_recover_known_spectrum(shape):
+    d_out, d_in = shape
+    k = 8
+    w = _f64_weight(d_out, d_in, 0.7, k, seed=3)
+    W_A, W_B, S = oracle.svd_factors(w.W, k)
+    s = w.s.numpy()
+    np.testing.assert_allclose(S, s, rtol=1e-12, atol=1e-14)
+    # W_A W_B is the rank-k truncation U_k S_k V_k^T (sign flips of singular vectors cancel)
+    Uk, Vk = w.U.numpy()[:, :k], w.V.numpy()[:, :k]
+    np.testing.assert_allclose(W_A @ W_B, (Uk * s[:k]) @ Vk.T, rtol=0, atol=1e-12)
+    # the generator's emitted factors give the same product
+    np.testing.assert_allclose(w.W_A.numpy() @ w.W_B.numpy(), W_A @ W_B, rtol=0, atol=1e-12)
+    # Eckart-Young: squared Frobenius error of the truncation = sum of the discarded s_i^2
+    err = np.sum((oracle.f64(w.W).T - W_A @ W_B) ** 2)
+    assert err == pytest.approx(np.sum(s[k:] ** 2), rel=1e-10)
+
+
+def test_full_rank_estimator_equals_dense_output():
+    """With k = min(D_in, D_out) the estimate is x W exactly, so estimated scores are the
+    oracle criterion on true activations."""
+    d_out, d_in = 48, 32
+    w = _f64_weight(d_out, d_in, 0.5, min(d_in, d_out), seed=5)
+    x = np.random.default_rng(1).standard_normal((20, d_in))
+    Y = x @ oracle.f64(w.W).T
+    Yh = oracle.estimate(x, w.W_A, w.W_B)
+    np.testing.assert_allclose(Yh, Y, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.score_l2(Yh), oracle.score_l2(Y), rtol=1e-12)
+
+
+def test_estimate_order_is_associative_product():
+    rng = np.random.default_rng(2)
+    x, wa, wb = rng.standard_normal((7, 11)), rng.standard_normal((11, 3)), rng.standard_normal((3, 13))
+    np.testing.assert_allclose(oracle.estimate(x, wa, wb), x @ (wa @ wb), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- criteria
+
+def test_l2_closed_form_constant_columns():
+    c = np.array([0.0, -2.0, 3.5, 1e-3])
+    T = 37
+    Y = np.ones((T, 1)) * c[None, :]
+    np.testing.assert_allclose(oracle.score_l2(Y), np.abs(c) * math.sqrt(T), rtol=1e-14)
+
+
+def test_swiglu_criterion_special_cases():
+    T = 9
+    G = np.zeros((T, 3))
+    G[:, 1] = 50.0       # SiLU(50) = 50 to fp64 precision
+    G[:, 2] = -50.0      # SiLU(-50) ~ -50 e^-50
+    U = np.full((T, 3), 2.0)
+    s = oracle.score_swiglu(G, U)
+    assert s[0] == 0.0
+    assert s[1] == pytest.approx(100.0 * math.sqrt(T), rel=1e-14)
+    assert s[2] == pytest.approx(100.0 * math.exp(-50.0) * math.sqrt(T), rel=1e-10)
+
+
+def test_qk_group_size_one_is_mha_formula():
+    rng = np.random.default_rng(4)
+    Q, K = rng.standard_normal((15, 12)), rng.standard_normal((15, 12))
+    s = oracle.score_qk(Q, K, n_q_heads=3, n_kv_heads=3, head_dim=4)
+    q = np.sqrt((Q ** 2).sum(0))
+    k = np.sqrt((K ** 2).sum(0))
+    np.testing.assert_allclose(s, q * k, rtol=1e-14)
+
+
+def test_qk_gqa_is_sum_over_group():
+    rng = np.random.default_rng(6)
+    nq, nkv, hd = 4, 2, 3
+    Q, K = rng.standard_normal((10, nq * hd)), rng.standard_normal((10, nkv * hd))
+    s = oracle.score_qk(Q, K, nq, nkv, hd)
+    for g in range(nkv):
+        for d in range(hd):
+            qs = sum(np.linalg.norm(Q[:, h * hd + d]) for h in range(g * 2, g * 2 + 2))
+            assert s[g * hd + d] == pytest.approx(qs * np.linalg.norm(K[:, g * hd + d]), rel=1e-13)
+
+
+def test_gram_identity_for_linear_criteria():
+    """sum_t (Z b_i)_t^2 = b_i^T (Z^T Z) b_i: the token reduction of a linear criterion
+    collapses to a k x k Gram matrix (exact algebra)."""
+    rng = np.random.default_rng(7)
+    Z, Wb = rng.standard_normal((50, 8)), rng.standard_normal((8, 30))
+    G = Z.T @ Z
+    quad = np.einsum("ki,kl,li->i", Wb, G, Wb)
+    np.testing.assert_allclose(np.sqrt(quad), oracle.score_l2(Z @ Wb), rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- selection
+
+def _brute_force_valid(scores, n, idx):
+    """Every kept score beats every dropped one under (score desc, index asc, NaN last)."""
+    def key(i):
+        v = scores[i]
+        return (1, 0.0, i) if math.isnan(v) else (0, -v, i)
+    kept = set(idx.tolist())
+    assert len(kept) == n == len(idx)
+    assert list(idx) == sorted(idx)
+    worst_kept = max(key(i) for i in kept)
+    for j in range(len(scores)):
+        if j not in kept:
+            assert key(j) > worst_kept
+
+
+def test_select_brute_force_tiny_exhaustive():
+    vals = [0.0, 1.0, 1.0, float("nan"), -float("inf"), 2.5]
+    for perm in set(itertools.permutations(vals)):
+        s = np.array(perm)
+        for n in range(1, len(s) + 1):
+            _brute_force_valid(s, n, oracle.select_top(s, n))
+
+
+def test_select_brute_force_random_with_duplicates():
+    rng = np.random.default_rng(8)
+    for trial in range(200):
+        N = int(rng.integers(1, 40))
+        s = rng.integers(0, 5, N).astype(float)     # many ties
+        n = int(rng.integers(1, N + 1))
+        idx = oracle.select_top(s, n)
+        _brute_force_valid(s, n, idx)
+        # reference by full sort on (score desc, index asc)
+        order = sorted(range(N), key=lambda i: (-s[i], i))[:n]
+        assert idx.tolist() == sorted(order)
+
+
+def test_expand_units_mha_identity_and_gqa():
+    u = np.array([0, 3, 5])
+    np.testing.assert_array_equal(oracle.expand_units(u, 2, 2, 3), u)
+    # 4 query heads over 2 KV heads, head_dim 3: unit (g=0, d=0) -> heads 0,1 at d=0; (1, 2) -> heads 2,3 at d=2
+    got = oracle.expand_units(np.array([0, 5]), 4, 2, 3)
+    assert got.tolist() == [0, 3, 8, 11]
+
+
+# --------------------------------------------------------------------------- sparse linear
+
+def _rand_linear(rng, T, d_in, d_out, r):
+    return (rng.standard_normal((T, d_in)), rng.standard_normal((d_out, d_in)),
+            rng.standard_normal((r, d_in)), rng.standard_normal((d_out, r)), rng.standard_normal((T, d_out)))
+
+
+@pytest.mark.parametrize("kind", ["out", "in"])
+def test_sliced_equals_compact_submatrix_product(kind):
+    """Kept channels form a dense submatrix: compute it on the compact submatrix and
+    compare with the masked-weight definition."""
+    rng = np.random.default_rng(9)
+    T, d_in, d_out, r = 12, 10, 14, 3
+    X, W, A, B, dY = _rand_linear(rng, T, d_in, d_out, r)
+    ctx = np.ones(T, dtype=bool)
+    n_side = d_out if kind == "out" else d_in
+    idx = np.sort(rng.choice(n_side, 5, replace=False))
+    Y = oracle.sparse_linear_fwd(X, W, A, B, 0.0, ctx, idx, kind)
+    Wm = W.T
+    if kind == "out":
+        want = np.zeros((T, d_out))
+        want[:, idx] = X @ Wm[:, idx]
+    else:
+        want = X[:, idx] @ Wm[idx, :]
+    np.testing.assert_allclose(Y, want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["out", "in"])
+def test_output_rows_do_not_depend_on_index_set(kind):
+    rng = np.random.default_rng(10)
+    T, d_in, d_out, r = 16, 9, 11, 2
+    X, W, A, B, dY = _rand_linear(rng, T, d_in, d_out, r)
+    ctx = rng.random(T) < 0.6
+    n_side = d_out if kind == "out" else d_in
+    i1, i2 = np.array([0, 1]), np.arange(n_side)
+    y1 = oracle.sparse_linear_fwd(X, W, A, B, 1.5, ctx, i1, kind)
+    y2 = oracle.sparse_linear_fwd(X, W, A, B, 1.5, ctx, i2, kind)
+    np.testing.assert_array_equal(y1[~ctx], y2[~ctx])
+    g1 = oracle.sparse_linear_bwd(X, dY, W, A, B, 1.5, ctx, i1, kind)[0]
+    g2 = oracle.sparse_linear_bwd(X, dY, W, A, B, 1.5, ctx, i2, kind)[0]
+    np.testing.assert_array_equal(g1[~ctx], g2[~ctx])
+
+
+def test_keep_ratio_one_is_dense_lora():
+    rng = np.random.default_rng(11)
+    T, d_in, d_out, r = 13, 8, 6, 2
+    X, W, A, B, dY = _rand_linear(rng, T, d_in, d_out, r)
+    ctx = rng.random(T) < 0.5
+    Y, dX, dA, dB = oracle.dense_lora_reference(X, dY, W, A, B, 2.0)
+    for kind, n in (("out", d_out), ("in", d_in)):
+        idx = np.arange(n)
+        np.testing.assert_allclose(oracle.sparse_linear_fwd(X, W, A, B, 2.0, ctx, idx, kind), Y, rtol=1e-13)
+        got = oracle.sparse_linear_bwd(X, dY, W, A, B, 2.0, ctx, idx, kind)
+        for a, b in zip(got, (dX, dA, dB)):
+            np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-13)
+
+
+def _fd(f, x, eps=1e-6):
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + eps
+        fp = f()
+        x[i] = old - eps
+        fm = f()
+        x[i] = old
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+@pytest.mark.parametrize("kind", ["out", "in"])
+def test_linear_backward_matches_finite_differences(kind):
+    rng = np.random.default_rng(12)
+    T, d_in, d_out, r = 6, 5, 7, 2
+    X, W, A, B, dY = _rand_linear(rng, T, d_in, d_out, r)
+    ctx = np.array([True, True, False, True, False, True])
+    n_side = d_out if kind == "out" else d_in
+    idx = np.array([1, 3, 4])
+    assert idx.max() < n_side
+
+    def loss():
+        return float(np.sum(dY * oracle.sparse_linear_fwd(X, W, A, B, 0.7, ctx, idx, kind)))
+    dX, dA, dB = oracle.sparse_linear_bwd(X, dY, W, A, B, 0.7, ctx, idx, kind)
+    np.testing.assert_allclose(dX, _fd(loss, X), rtol=1e-7, atol=1e-7)
+    np.testing.assert_allclose(dA, _fd(loss, A), rtol=1e-7, atol=1e-7)
+    np.testing.assert_allclose(dB, _fd(loss, B), rtol=1e-7, atol=1e-7)
+
+
+def test_silu_grad_matches_finite_differences():
+    z = np.linspace(-8, 8, 33)
+    fd = (oracle.silu(z + 1e-6) - oracle.silu(z - 1e-6)) / 2e-6
+    np.testing.assert_allclose(oracle.silu_grad(z), fd, rtol=1e-7, atol=1e-9)
+
+
+# --------------------------------------------------------------------------- FFN block
+
+def _tiny_ffn(seed=0, T=10, D=6, F=9, r=2):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((T, D))
+    Wg, Wu, Wd = rng.standard_normal((F, D)), rng.standard_normal((F, D)), rng.standard_normal((D, F))
+    lg = (rng.standard_normal((r, D)), rng.standard_normal((F, r)))
+    lu = (rng.standard_normal((r, D)), rng.standard_normal((F, r)))
+    ld = (rng.standard_normal((r, F)), rng.standard_normal((D, r)))
+    ctx = rng.random(T) < 0.6
+    dY = rng.standard_normal((T, D))
+    return X, Wg, Wu, Wd, lg, lu, ld, ctx, dY
+
+
+def test_ffn_keep_ratio_one_is_dense_swiglu_lora():
+    X, Wg, Wu, Wd, lg, lu, ld, ctx, dY = _tiny_ffn()
+    s = 1.3
+    out = oracle.ffn_fwd(X, ctx, Wg, Wu, Wd, lg, lu, ld, s, np.arange(Wg.shape[0]))
+    G = X @ Wg.T + s * (X @ lg[0].T) @ lg[1].T
+    U = X @ Wu.T + s * (X @ lu[0].T) @ lu[1].T
+    H = G / (1 + np.exp(-G)) * U
+    Y = H @ Wd.T + s * (H @ ld[0].T) @ ld[1].T
+    np.testing.assert_allclose(out["Y"], Y, rtol=1e-12, atol=1e-12)
+
+
+def test_ffn_index_coupling():
+    """One index set: gate/up keep idx output channels, down keeps idx input channels;
+    on context rows the dropped intermediate channels carry only the LoRA terms, and
+    down's frozen branch reads only H[:, idx] while its LoRA reads the full H."""
+    X, Wg, Wu, Wd, lg, lu, ld, ctx, dY = _tiny_ffn(1)
+    s = 0.9
+    idx = np.array([0, 2, 3, 7])
+    drop = oracle.complement(idx, Wg.shape[0])
+    out = oracle.ffn_fwd(X, ctx, Wg, Wu, Wd, lg, lu, ld, s, idx)
+    G, H, Y = out["G"], out["H"], out["Y"]
+    np.testing.assert_allclose(G[ctx][:, drop], (s * (X @ lg[0].T) @ lg[1].T)[ctx][:, drop], rtol=1e-12)
+    want = H[ctx][:, idx] @ Wd.T[idx, :] + s * (H[ctx] @ ld[0].T) @ ld[1].T
+    np.testing.assert_allclose(Y[ctx], want, rtol=1e-12, atol=1e-12)
+
+
+def test_ffn_backward_matches_finite_differences():
+    X, Wg, Wu, Wd, lg, lu, ld, ctx, dY = _tiny_ffn(2, T=5, D=4, F=6, r=2)
+    s = 0.8
+    idx = np.array([1, 2, 5])
+
+    def loss():
+        return float(np.sum(dY * oracle.ffn_fwd(X, ctx, Wg, Wu, Wd, lg, lu, ld, s, idx)["Y"]))
+    g = oracle.ffn_bwd(X, dY, ctx, Wg, Wu, Wd, lg, lu, ld, s, idx)
+    np.testing.assert_allclose(g["dX"], _fd(loss, X), rtol=1e-6, atol=1e-7)
+    for name, arrs in (("g", lg), ("u", lu), ("d", ld)):
+        np.testing.assert_allclose(g["dA_" + name], _fd(loss, arrs[0]), rtol=1e-6, atol=1e-7)
+        np.testing.assert_allclose(g["dB_" + name], _fd(loss, arrs[1]), rtol=1e-6, atol=1e-7)
+
+
+def test_ffn_select_on_tiny_config_is_valid():
+    cfg = inputs.TINY_FFN
+    d = inputs.make_ffn_inputs(cfg, seed=0)
+    s, idx = oracle.ffn_select(d["x"], d["ctx_mask"], (d["gate"].W_A, d["gate"].W_B),
+                               (d["up"].W_A, d["up"].W_B), cfg.ratio)
+    assert idx.shape[0] == oracle.keep_count(cfg.ratio, cfg.inter) == 344
+    _brute_force_valid(s, 344, idx)
+
+
+def test_context_first_permutation_equivalence():
+    """Linear layers are row-independent: running on the context-first row order and
+    un-permuting gives the sequence-order result."""
+    X, Wg, Wu, Wd, lg, lu, ld, ctx, dY = _tiny_ffn(3)
+    idx = np.array([0, 4, 5])
+    perm = np.concatenate([np.nonzero(ctx)[0], np.nonzero(~ctx)[0]])
+    a = oracle.ffn_fwd(X, ctx, Wg, Wu, Wd, lg, lu, ld, 1.0, idx)["Y"]
+    b = oracle.ffn_fwd(X[perm], ctx[perm], Wg, Wu, Wd, lg, lu, ld, 1.0, idx)["Y"]
+    inv = np.argsort(perm)
+    np.testing.assert_allclose(b[inv], a, rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- attention projections
+
+def test_attn_select_mha_reduces_to_plain_qk():
+    rng = np.random.default_rng(13)
+    T, D, h, hd, k = 20, 16, 2, 4, 3
+    X = rng.standard_normal((T, D))
+    ctx = np.ones(T, dtype=bool)
+    fs = [(rng.standard_normal((D, k)), rng.standard_normal((k, h * hd))) for _ in range(3)]
+    out = oracle.attn_select(X, ctx, *fs, h, h, hd, 0.5)
+    Q, K = X @ fs[0][0] @ fs[0][1], X @ fs[1][0] @ fs[1][1]
+    s = np.linalg.norm(Q, axis=0) * np.linalg.norm(K, axis=0)
+    np.testing.assert_allclose(out["s_qk"], s, rtol=1e-12)
+    np.testing.assert_array_equal(out["idx_q"], out["idx_k"])
+    np.testing.assert_array_equal(out["idx_o"], out["idx_v"])
