@@ -1,0 +1,233 @@
+"""ctypes binding of libsparselora.so. Same names as the C ABI (include/sparselora.h);
+argument marshalling only: tensors are passed as device pointers, the stream is
+torch's current stream, and every computation happens in the library's kernels.
+
+The library must have been built in-tree (``python -m contextual_sparsity_lora_b200.build``);
+there is no fallback: a missing library raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int32, c_int64, c_size_t, c_void_p
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparselora.so")
+
+SL_OK, SL_ERR_INVALID_ARG, SL_ERR_SHAPE, SL_ERR_ALIGNMENT, SL_ERR_WORKSPACE, SL_ERR_UNSUPPORTED, SL_ERR_CUDA, \
+    SL_ERR_DEVICE_FLAG = range(8)
+SL_CRIT_L2, SL_CRIT_SWIGLU_L2, SL_CRIT_QK = 0, 1, 2
+SL_DT_BF16, SL_DT_F32 = 0, 1
+SL_SLICE_OUT, SL_SLICE_IN = 0, 1
+SL_LAYOUT_NATURAL, SL_LAYOUT_SIGMA = 0, 1
+SL_EPI_NONE, SL_EPI_SWIGLU = 0, 1
+SL_LORA_FWD, SL_LORA_BWD = 0, 1
+
+EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_init", "sl_read_device_flag",
+            "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
+            "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read")
+
+
+class SlWorkspaceC(ctypes.Structure):
+    _fields_ = [("ptr", c_void_p), ("bytes", c_size_t), ("needed", c_size_t)]
+
+
+class SlLinearC(ctypes.Structure):
+    _fields_ = [("w", c_void_p), ("w_t", c_void_p), ("d_in", c_int64), ("d_out", c_int64), ("slice", c_int32),
+                ("r", c_int32), ("lora_a", c_void_p), ("lora_b", c_void_p), ("lora_scale", c_float),
+                ("pad_", c_int32)]
+
+
+class SlChannelsC(ctypes.Structure):
+    _fields_ = [("sigma", c_void_p), ("n_side", c_int64), ("n_keep", c_int64)]
+
+
+class SparseLoRAError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)} (status {code})")
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m contextual_sparsity_lora_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = c_void_p
+        L.sl_status_string.restype = c_char_p
+        L.sl_status_string.argtypes = [c_int32]
+        L.sl_version.restype = c_int32
+        L.sl_keep_count.restype = c_int64
+        L.sl_keep_count.argtypes = [c_double, c_int64]
+        L.sl_workspace_init.argtypes = [POINTER(SlWorkspaceC), P]
+        L.sl_read_device_flag.argtypes = [POINTER(SlWorkspaceC), POINTER(c_int32), P]
+        L.sl_svd_estimate.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p),
+                                      POINTER(c_void_p), POINTER(c_int64), c_int32, c_int32, c_int32, c_int32, P, P,
+                                      POINTER(SlWorkspaceC), P]
+        L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
+        L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
+                                      POINTER(SlChannelsC), P, P, c_int64, POINTER(c_void_p), POINTER(c_int64),
+                                      c_int32, POINTER(SlChannelsC), POINTER(c_void_p), POINTER(c_void_p),
+                                      POINTER(c_void_p), POINTER(c_void_p), POINTER(SlWorkspaceC), P]
+        L.sl_sparse_linear_fwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32, P, c_int64,
+                                           c_int64, c_int64, c_int32, c_int32, P, c_int64, POINTER(c_void_p),
+                                           POINTER(c_int64), POINTER(SlWorkspaceC), P]
+        L.sl_sparse_linear_bwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32,
+                                           POINTER(c_void_p), POINTER(c_int64), c_int64, c_int64, c_int32, c_int32,
+                                           POINTER(c_void_p), P, c_int64, POINTER(c_void_p), POINTER(c_void_p),
+                                           POINTER(SlWorkspaceC), P]
+        L.sl_prepare_weight.argtypes = [P, c_int64, c_int64, P, P]
+        L.sl_profile_enable.argtypes = [c_int32]
+        L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
+        L.sl_permute_rows.argtypes = [P, c_int64, P, c_int64, c_int64, P, c_int64, P]
+        for n in EXPORTED:
+            if n not in ("sl_status_string", "sl_version", "sl_keep_count"):
+                getattr(L, n).restype = c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().sl_status_string(int(code)).decode()
+
+
+def _check(fn, code):
+    if code != SL_OK:
+        raise SparseLoRAError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream():
+    return c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptrs(ts):
+    return (c_void_p * max(1, len(ts)))(*[None if t is None else t.data_ptr() for t in ts])
+
+
+def _i64s(vs):
+    return (c_int64 * max(1, len(vs)))(*[int(v) for v in vs])
+
+
+class Workspace:
+    """Caller-owned scratch memory for the library (a torch byte buffer that grows on demand)."""
+
+    def __init__(self, device="cuda", nbytes: int = 1 << 20):
+        self.device = device
+        self.buf = None
+        self._alloc(nbytes)
+
+    def _alloc(self, nbytes):
+        self.buf = torch.empty(int(nbytes), dtype=torch.uint8, device=self.device)
+        self.c = SlWorkspaceC(self.buf.data_ptr(), self.buf.numel(), 0)
+        _check("sl_workspace_init", lib().sl_workspace_init(ctypes.byref(self.c), _stream()))
+
+    def call(self, fn_name, *args):
+        """Run one library call with this workspace, growing it once if the call asks for more."""
+        fn = getattr(lib(), fn_name)
+        code = fn(*args, ctypes.byref(self.c), _stream())
+        if code == SL_ERR_WORKSPACE and self.c.needed > self.c.bytes:
+            self._alloc(self.c.needed + (1 << 20))
+            code = fn(*args, ctypes.byref(self.c), _stream())
+        _check(fn_name, code)
+
+    def read_device_flag(self) -> int:
+        v = c_int32(0)
+        code = lib().sl_read_device_flag(ctypes.byref(self.c), ctypes.byref(v), _stream())
+        if code not in (SL_OK, SL_ERR_DEVICE_FLAG):
+            _check("sl_read_device_flag", code)
+        return int(v.value)
+
+
+def linear_desc(w, lora_a, lora_b, lora_scale, slice_kind, w_t=None) -> SlLinearC:
+    d_out, d_in = w.shape
+    return SlLinearC(w.data_ptr(), None if w_t is None else w_t.data_ptr(), d_in, d_out, slice_kind,
+                     lora_a.shape[0], lora_a.data_ptr(), lora_b.data_ptr(), float(lora_scale), 0)
+
+
+def channels_desc(sigma, n_keep) -> SlChannelsC:
+    return SlChannelsC(sigma.data_ptr(), sigma.numel(), int(n_keep))
+
+
+def _arr(cls, items):
+    return (cls * max(1, len(items)))(*items)
+
+
+# ---------------------------------------------------------------------------- entry points
+
+def sl_version() -> int:
+    return int(lib().sl_version())
+
+
+def sl_keep_count(ratio: float, n: int) -> int:
+    return int(lib().sl_keep_count(float(ratio), int(n)))
+
+
+def sl_svd_estimate(ws: Workspace, crit, x, n_ctx, w_a, w_b, k, scores, scores_v=None, n_q_heads=0,
+                    n_kv_heads=0, head_dim=0):
+    dtype = SL_DT_F32 if x.dtype == torch.float32 else SL_DT_BF16
+    d_out = [t.shape[1] for t in w_b]
+    ws.call("sl_svd_estimate", crit, dtype, _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w_a), _ptrs(w_a),
+            _ptrs(w_b), _i64s(d_out), int(k), int(n_q_heads), int(n_kv_heads), int(head_dim), _ptr(scores),
+            _ptr(scores_v))
+
+
+def sl_select_channels(scores, n_keep, sigma, heads_per_group=0, head_dim=0, sigma_wide=None):
+    _check("sl_select_channels",
+           lib().sl_select_channels(_ptr(scores), scores.numel(), int(n_keep), _ptr(sigma), int(heads_per_group),
+                                    int(head_dim), _ptr(sigma_wide), _stream()))
+
+
+def sl_lora_fwd_bwd(ws: Workspace, mode, lins, x, n_ctx, xa_s, xa=None, in_layout=SL_LAYOUT_NATURAL, in_ch=None,
+                    dy=(), out_layout=SL_LAYOUT_NATURAL, out_ch=(), dya=(), dya_s=(), dA=(), dB=()):
+    lin_arr = _arr(SlLinearC, list(lins))
+    in_c = ctypes.byref(in_ch) if in_ch is not None else None
+    out_arr = _arr(SlChannelsC, list(out_ch)) if out_ch else None
+    ws.call("sl_lora_fwd_bwd", mode, len(lins), lin_arr, _ptr(x), x.stride(0), x.shape[0], int(n_ctx), in_layout,
+            in_c, _ptr(xa), _ptr(xa_s), xa_s.stride(0), _ptrs(list(dy)), _i64s([t.stride(0) for t in dy]),
+            out_layout, out_arr, _ptrs(list(dya)), _ptrs(list(dya_s)), _ptrs(list(dA)), _ptrs(list(dB)))
+
+
+def sl_sparse_linear_fwd(ws: Workspace, lins, chans, epi, x, n_ctx, xa_s, ys, in_layout=SL_LAYOUT_NATURAL,
+                         out_layout=SL_LAYOUT_NATURAL):
+    ws.call("sl_sparse_linear_fwd", len(lins), _arr(SlLinearC, list(lins)), _arr(SlChannelsC, list(chans)), epi,
+            _ptr(x), x.stride(0), x.shape[0], int(n_ctx), in_layout, out_layout, _ptr(xa_s), xa_s.stride(0),
+            _ptrs(list(ys)), _i64s([t.stride(0) for t in ys]))
+
+
+def sl_sparse_linear_bwd(ws: Workspace, lins, chans, epi, dys, n_ctx, dya_s, dx=None, in_layout=SL_LAYOUT_NATURAL,
+                         out_layout=SL_LAYOUT_NATURAL, aux=(), aux_out=()):
+    ld = dx.stride(0) if dx is not None else aux_out[0].stride(0)
+    ws.call("sl_sparse_linear_bwd", len(lins), _arr(SlLinearC, list(lins)), _arr(SlChannelsC, list(chans)), epi,
+            _ptrs(list(dys)), _i64s([t.stride(0) for t in dys]), dys[0].shape[0], int(n_ctx), in_layout,
+            out_layout, _ptrs(list(dya_s)), _ptr(dx), ld, _ptrs(list(aux)), _ptrs(list(aux_out)))
+
+
+def sl_prepare_weight(w, w_t):
+    d_out, d_in = w.shape
+    _check("sl_prepare_weight", lib().sl_prepare_weight(_ptr(w), d_out, d_in, _ptr(w_t), _stream()))
+
+
+def sl_permute_rows(src, perm, dst):
+    _check("sl_permute_rows", lib().sl_permute_rows(_ptr(src), src.stride(0), _ptr(perm), perm.numel(),
+                                                    src.shape[1], _ptr(dst), dst.stride(0), _stream()))
+
+
+def sl_profile_enable(on: bool):
+    _check("sl_profile_enable", lib().sl_profile_enable(1 if on else 0))
+
+
+def sl_profile_read():
+    """(kernel launches, GEMM-engine launches, GEMM-engine milliseconds) since the last read."""
+    a, b, c = c_int64(0), c_int64(0), c_double(0.0)
+    _check("sl_profile_read", lib().sl_profile_read(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return int(a.value), int(b.value), float(c.value)

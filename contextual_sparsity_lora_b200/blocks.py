@@ -1,0 +1,213 @@
+"""One fine-tuning step of a SparseLoRA FFN block or attention-projection block,
+composed from the C ABI calls (no arithmetic here: buffers are allocated with torch,
+every stage runs in libsparselora's kernels).
+
+Rows are in context-first order (context rows [0, n_ctx), then output rows).
+Dense mode (keep ratio 1, no estimator) is the dense-LoRA baseline on the same kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(*shape, dtype=dtype, device=device)
+
+
+class FFNBlock:
+    """SwiGLU FFN: gate/up (output channels sliced), down (input channels sliced), one
+    index set shared by all three; L2 criterion on the estimated SiLU(gate) * up."""
+
+    def __init__(self, gate, up, down, lora_gate, lora_up, lora_down, lora_scale, k, n_tok, n_ctx, ratio,
+                 device="cuda", dense=False):
+        bf = torch.bfloat16
+        self.device = device
+        self.D = gate.W.shape[1]
+        self.F = gate.W.shape[0]
+        self.k = k
+        self.n_tok, self.n_ctx = n_tok, n_ctx
+        self.dense = dense or ratio >= 1.0
+        self.n_keep = self.F if self.dense else B.sl_keep_count(ratio, self.F)
+        dev = lambda t: t.to(device=device, dtype=bf).contiguous()
+        self.Wg, self.Wu, self.Wd = dev(gate.W), dev(up.W), dev(down.W)
+        self.est_dtype = torch.float32 if gate.W_A.dtype == torch.float32 else bf
+        ed = lambda t: t.to(device=device, dtype=self.est_dtype).contiguous()
+        self.WAg, self.WBg, self.WAu, self.WBu = ed(gate.W_A), ed(gate.W_B), ed(up.W_A), ed(up.W_B)
+        self.Ag, self.Bg = dev(lora_gate[0]), dev(lora_gate[1])
+        self.Au, self.Bu = dev(lora_up[0]), dev(lora_up[1])
+        self.Ad, self.Bd = dev(lora_down[0]), dev(lora_down[1])
+        self.r = self.Ag.shape[0]
+        self.scale = float(lora_scale)
+        self.Wd_t = _empty((self.F, self.D), bf, device)
+        B.sl_prepare_weight(self.Wd, self.Wd_t)
+        self.ws = B.Workspace(device)
+        T, D, F, r = n_tok, self.D, self.F, self.r
+        f32 = torch.float32
+        self.scores = _empty((F,), f32, device)
+        self.sigma = torch.arange(F, dtype=torch.int32, device=device)
+        self.xa_gu, self.xa_s_gu = _empty((T, 2 * r), f32, device), _empty((T, 2 * r), bf, device)
+        self.g, self.u, self.h = (_empty((T, F), bf, device) for _ in range(3))
+        self.xa_d, self.xa_s_d = _empty((T, r), f32, device), _empty((T, r), bf, device)
+        self.y = _empty((T, D), bf, device)
+        self.dya_d, self.dya_s_d = _empty((T, r), f32, device), _empty((T, r), bf, device)
+        self.dA_d, self.dB_d = _empty((r, F), f32, device), _empty((D, r), f32, device)
+        self.dg, self.du = _empty((T, F), bf, device), _empty((T, F), bf, device)
+        self.dya_g, self.dya_s_g = _empty((T, r), f32, device), _empty((T, r), bf, device)
+        self.dya_u, self.dya_s_u = _empty((T, r), f32, device), _empty((T, r), bf, device)
+        self.dA_g, self.dB_g = _empty((r, D), f32, device), _empty((F, r), f32, device)
+        self.dA_u, self.dB_u = _empty((r, D), f32, device), _empty((F, r), f32, device)
+        self.dx = _empty((T, D), bf, device)
+        self._descs()
+
+    def _descs(self):
+        s = self.scale
+        self.lin_g = B.linear_desc(self.Wg, self.Ag, self.Bg, s, B.SL_SLICE_OUT)
+        self.lin_u = B.linear_desc(self.Wu, self.Au, self.Bu, s, B.SL_SLICE_OUT)
+        self.lin_d = B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t)
+        self.ch = B.channels_desc(self.sigma, self.n_keep)
+
+    def select(self, x):
+        """a1 + a2 + a3 on the context rows of x (writes self.scores, self.sigma)."""
+        xe = x if self.est_dtype == torch.bfloat16 else self.x_est
+        B.sl_svd_estimate(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx, [self.WAg, self.WAu],
+                          [self.WBg, self.WBu], self.k, self.scores)
+        B.sl_select_channels(self.scores, self.n_keep, self.sigma)
+
+    def forward(self, x, x_est=None):
+        """x: bf16 [n_tok, D] context-first. x_est: optional fp32 copy for an fp32 estimator."""
+        self.x = x
+        self.x_est = x_est
+        C = self.n_ctx
+        if not self.dense and C > 0:  # no context rows: nothing to score, every row is dense
+            self.select(x)
+        lay = B.SL_LAYOUT_NATURAL if self.dense else B.SL_LAYOUT_SIGMA
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu, xa=self.xa_gu)
+        B.sl_sparse_linear_fwd(self.ws, [self.lin_g, self.lin_u], [self.ch], B.SL_EPI_SWIGLU, x, C, self.xa_s_gu,
+                               [self.g, self.u, self.h], out_layout=B.SL_LAYOUT_SIGMA)
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_d], self.h, C, self.xa_s_d, xa=self.xa_d,
+                          in_layout=lay, in_ch=self.ch)
+        B.sl_sparse_linear_fwd(self.ws, [self.lin_d], [self.ch], B.SL_EPI_NONE, self.h, C, self.xa_s_d, [self.y],
+                               in_layout=B.SL_LAYOUT_SIGMA)
+        return self.y
+
+    def backward(self, dy):
+        C = self.n_ctx
+        lay = B.SL_LAYOUT_NATURAL if self.dense else B.SL_LAYOUT_SIGMA
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [self.lin_d], self.h, C, self.xa_s_d, in_layout=lay,
+                          in_ch=self.ch, dy=[dy], dya=[self.dya_d], dya_s=[self.dya_s_d], dA=[self.dA_d],
+                          dB=[self.dB_d])
+        B.sl_sparse_linear_bwd(self.ws, [self.lin_d], [self.ch], B.SL_EPI_SWIGLU, [dy], C, [self.dya_s_d],
+                               aux=[self.g, self.u], aux_out=[self.dg, self.du], out_layout=B.SL_LAYOUT_SIGMA)
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [self.lin_g, self.lin_u], self.x, C, self.xa_s_gu,
+                          dy=[self.dg, self.du], out_layout=lay, out_ch=[self.ch, self.ch],
+                          dya=[self.dya_g, self.dya_u], dya_s=[self.dya_s_g, self.dya_s_u],
+                          dA=[self.dA_g, self.dA_u], dB=[self.dB_g, self.dB_u])
+        B.sl_sparse_linear_bwd(self.ws, [self.lin_g, self.lin_u], [self.ch, self.ch], B.SL_EPI_NONE,
+                               [self.dg, self.du], C, [self.dya_s_g, self.dya_s_u], dx=self.dx,
+                               in_layout=B.SL_LAYOUT_SIGMA)
+        return self.dx
+
+    def step(self, x, dy, x_est=None):
+        self.forward(x, x_est)
+        return self.backward(dy)
+
+
+class AttnProjBlock:
+    """q, k, v (output channels sliced) and o (input channels sliced). QK criterion over
+    KV units for q/k, L2 criterion on the estimated V for v/o. The attention core is not
+    part of the path: its output x_o and its gradients dq, dk, dv are inputs."""
+
+    def __init__(self, q, k, v, o, lora_q, lora_k, lora_v, lora_o, lora_scale, est_k, n_q_heads, n_kv_heads,
+                 head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False):
+        bf, f32 = torch.bfloat16, torch.float32
+        dev = lambda t: t.to(device=device, dtype=bf).contiguous()
+        self.device = device
+        self.D = q.W.shape[1]
+        self.hq, self.hkv, self.hd = n_q_heads, n_kv_heads, head_dim
+        self.hpg = n_q_heads // n_kv_heads
+        self.Dq, self.Dkv = n_q_heads * head_dim, n_kv_heads * head_dim
+        self.k = est_k
+        self.n_tok, self.n_ctx = n_tok, n_ctx
+        self.dense = dense or ratio >= 1.0
+        self.n_units = self.Dkv
+        self.n_keep_u = self.n_units if self.dense else B.sl_keep_count(ratio, self.n_units)
+        self.Wq, self.Wk, self.Wv, self.Wo = dev(q.W), dev(k.W), dev(v.W), dev(o.W)
+        self.WA = [dev(q.W_A), dev(k.W_A), dev(v.W_A)]
+        self.WB = [dev(q.W_B), dev(k.W_B), dev(v.W_B)]
+        self.L = {n: (dev(a), dev(b)) for n, (a, b) in zip("qkvo", (lora_q, lora_k, lora_v, lora_o))}
+        self.r = self.L["q"][0].shape[0]
+        self.scale = float(lora_scale)
+        self.Wo_t = _empty((self.Dq, self.D), bf, device)
+        B.sl_prepare_weight(self.Wo, self.Wo_t)
+        self.ws = B.Workspace(device)
+        T, D, r = n_tok, self.D, self.r
+        self.s_qk, self.s_v = _empty((self.n_units,), f32, device), _empty((self.n_units,), f32, device)
+        ar = lambda n: torch.arange(n, dtype=torch.int32, device=device)
+        self.sig_k, self.sig_q = ar(self.Dkv), ar(self.Dq)
+        self.sig_v, self.sig_o = ar(self.Dkv), ar(self.Dq)
+        self.xa_qkv, self.xa_s_qkv = _empty((T, 3 * r), f32, device), _empty((T, 3 * r), bf, device)
+        self.q, self.kk, self.vv = _empty((T, self.Dq), bf, device), _empty((T, self.Dkv), bf, device), \
+            _empty((T, self.Dkv), bf, device)
+        self.xa_o, self.xa_s_o = _empty((T, r), f32, device), _empty((T, r), bf, device)
+        self.y = _empty((T, D), bf, device)
+        self.dya = {n: (_empty((T, r), f32, device), _empty((T, r), bf, device)) for n in "qkvo"}
+        d_ins = {"q": D, "k": D, "v": D, "o": self.Dq}
+        d_outs = {"q": self.Dq, "k": self.Dkv, "v": self.Dkv, "o": D}
+        self.dA = {n: _empty((r, d_ins[n]), f32, device) for n in "qkvo"}
+        self.dB = {n: _empty((d_outs[n], r), f32, device) for n in "qkvo"}
+        self.dx_o = _empty((T, self.Dq), bf, device)
+        self.dx = _empty((T, D), bf, device)
+        s = self.scale
+        self.lin = {
+            "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT),
+            "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT),
+            "v": B.linear_desc(self.Wv, *self.L["v"], s, B.SL_SLICE_OUT),
+            "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t),
+        }
+        self.ch = {
+            "q": B.channels_desc(self.sig_q, self.n_keep_u * self.hpg),
+            "k": B.channels_desc(self.sig_k, self.n_keep_u),
+            "v": B.channels_desc(self.sig_v, self.n_keep_u),
+            "o": B.channels_desc(self.sig_o, self.n_keep_u * self.hpg),
+        }
+
+    def select(self, x):
+        C = self.n_ctx
+        B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
+                          n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+        B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
+        B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+
+    def forward(self, x, x_o):
+        C = self.n_ctx
+        self.x, self.x_o = x, x_o
+        if not self.dense and C > 0:
+            self.select(x)
+        lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
+        B.sl_sparse_linear_fwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, x, C,
+                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=B.SL_LAYOUT_NATURAL)
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+        B.sl_sparse_linear_fwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, x_o, C, self.xa_s_o, [self.y],
+                               in_layout=B.SL_LAYOUT_NATURAL)
+        return self.y
+
+    def backward(self, dy, dq, dk, dv):
+        C = self.n_ctx
+        lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
+                          dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
+        B.sl_sparse_linear_bwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
+                               dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
+                          dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
+                          dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
+        B.sl_sparse_linear_bwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
+                               [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
+        return self.dx, self.dx_o
+
+    def step(self, x, x_o, dy, dq, dk, dv):
+        self.forward(x, x_o)
+        return self.backward(dy, dq, dk, dv)

@@ -1,0 +1,795 @@
+// C ABI of libsparselora.so (declared in include/sparselora.h): argument checks,
+// workspace carving, and the grouped tcgen05 GEMM problem lists of each stage.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/sparselora.h"
+#include "sl_internal.h"
+
+using namespace sl;
+
+// ------------------------------------------------------------------ profiling hook state
+namespace {
+std::atomic<bool> g_prof{false};
+std::atomic<long long> g_launches{0};
+std::mutex g_ev_mu;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_events;
+size_t g_ev_used = 0;
+}  // namespace
+
+namespace sl {
+void note_launch(int n) {
+  if (g_prof.load(std::memory_order_relaxed)) g_launches.fetch_add(n, std::memory_order_relaxed);
+}
+bool profiling_on() { return g_prof.load(std::memory_order_relaxed); }
+void gemm_events(cudaStream_t s, bool start) {
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  if (start) {
+    if (g_ev_used == g_events.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess) return;
+      if (cudaEventCreate(&b) != cudaSuccess) return;
+      g_events.emplace_back(a, b);
+    }
+    cudaEventRecord(g_events[g_ev_used].first, s);
+  } else {
+    cudaEventRecord(g_events[g_ev_used].second, s);
+    ++g_ev_used;
+  }
+}
+}  // namespace sl
+
+namespace {
+
+constexpr int32_t kVersion = 1;
+constexpr int kBig = 1 << 30;  // "segment always active"
+
+inline cudaStream_t cs(sl_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Two-pass carving of the caller's workspace: the first pass (base == nullptr)
+// only measures. The first 256 bytes are the device error word.
+struct Carver {
+  uint8_t* base;
+  size_t off = 256;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+inline sl_status ws_check(sl_workspace* ws, size_t needed) {
+  if (!ws) return SL_ERR_WORKSPACE;
+  ws->needed = needed;
+  if (!ws->ptr || ws->bytes < needed || !al16(ws->ptr)) return SL_ERR_WORKSPACE;
+  return SL_OK;
+}
+
+inline int* err_word(sl_workspace* ws) { return static_cast<int*>(ws->ptr); }
+
+inline sl_status from_builder(int rc) {
+  switch (rc) {
+    case 0: return SL_OK;
+    case 2: return SL_ERR_ALIGNMENT;
+    case 1: case 4: return SL_ERR_SHAPE;
+    default: return SL_ERR_CUDA;
+  }
+}
+inline sl_status from_kernel(int rc) { return rc == 0 ? SL_OK : (rc == 1 ? SL_ERR_SHAPE : SL_ERR_CUDA); }
+
+inline int64_t rup(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+bool linear_ok(const sl_linear& L) {
+  return L.w && L.d_in > 0 && L.d_out > 0 && L.lora_a && L.lora_b && L.r >= 8 && L.r <= 64 && L.r % 8 == 0 &&
+         L.d_in % 8 == 0 && L.d_out % 8 == 0 && al16(L.w) && al16(L.lora_a) && al16(L.lora_b) &&
+         (L.slice == SL_SLICE_OUT || L.slice == SL_SLICE_IN);
+}
+
+bool channels_ok(const sl_channels& c, int64_t n_side) {
+  return c.sigma && c.n_side == n_side && c.n_keep >= 1 && c.n_keep <= n_side;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sl_status_string(sl_status s) {
+  switch (s) {
+    case SL_OK: return "ok";
+    case SL_ERR_INVALID_ARG: return "invalid argument";
+    case SL_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case SL_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case SL_ERR_WORKSPACE: return "workspace missing or too small";
+    case SL_ERR_UNSUPPORTED: return "unsupported request";
+    case SL_ERR_CUDA: return "CUDA error";
+    case SL_ERR_DEVICE_FLAG: return "device-side timeout reported";
+  }
+  return "unknown status";
+}
+
+int32_t sl_version(void) { return kVersion; }
+
+int64_t sl_keep_count(double ratio, int64_t n) {
+  if (n <= 0) return 0;
+  int64_t c = (int64_t)std::ceil(ratio * (double)n - 1e-9);
+  if (c < 1) c = 1;
+  if (c > n) c = n;
+  return c;
+}
+
+sl_status sl_workspace_init(sl_workspace* ws, sl_stream stream) {
+  if (!ws || !ws->ptr || ws->bytes < 256) return SL_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws->ptr, 0, 256, cs(stream)) == cudaSuccess ? SL_OK : SL_ERR_CUDA;
+}
+
+sl_status sl_read_device_flag(const sl_workspace* ws, int32_t* code, sl_stream stream) {
+  if (!ws || !ws->ptr || !code) return SL_ERR_INVALID_ARG;
+  if (cudaMemcpyAsync(code, ws->ptr, sizeof(int32_t), cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess)
+    return SL_ERR_CUDA;
+  if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return SL_ERR_CUDA;
+  return *code ? SL_ERR_DEVICE_FLAG : SL_OK;
+}
+
+// ------------------------------------------------------------------ a1 + a2
+sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx,
+                          int32_t n_proj, const void* const* w_a, const void* const* w_b, const int64_t* d_out,
+                          int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float* scores,
+                          float* scores_v, sl_workspace* ws, sl_stream stream) {
+  if (!x || !w_a || !w_b || !d_out || !scores) return SL_ERR_INVALID_ARG;
+  if (dtype != SL_DT_BF16 && dtype != SL_DT_F32) return SL_ERR_INVALID_ARG;
+  if (n_ctx <= 0 || d_in <= 0 || ldx < d_in || k <= 0 || k > 16 || n_proj < 1 || n_proj * k > 64)
+    return SL_ERR_SHAPE;
+  if (d_in % 8 || ldx % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+  for (int j = 0; j < n_proj; ++j)
+    if (!w_a[j] || !w_b[j] || d_out[j] <= 0) return SL_ERR_INVALID_ARG;
+  const int fp32 = dtype == SL_DT_F32;
+  int64_t n_units = 0;
+  switch (crit) {
+    case SL_CRIT_L2:
+      if (n_proj != 1) return SL_ERR_INVALID_ARG;
+      n_units = d_out[0];
+      break;
+    case SL_CRIT_SWIGLU_L2:
+      if (n_proj != 2 || d_out[0] != d_out[1]) return SL_ERR_INVALID_ARG;
+      if (k != 4 && k != 8 && k != 16) return SL_ERR_UNSUPPORTED;
+      n_units = d_out[0];
+      break;
+    case SL_CRIT_QK:
+      if (n_proj != 2 && n_proj != 3) return SL_ERR_INVALID_ARG;
+      if (n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || n_q_heads % n_kv_heads) return SL_ERR_SHAPE;
+      if (d_out[0] != (int64_t)n_q_heads * head_dim || d_out[1] != (int64_t)n_kv_heads * head_dim)
+        return SL_ERR_SHAPE;
+      if (n_proj == 3 && !scores_v) return SL_ERR_INVALID_ARG;
+      n_units = (int64_t)n_kv_heads * head_dim;
+      break;
+    default:
+      return SL_ERR_INVALID_ARG;
+  }
+  const int mk = n_proj * k;
+  const int n_split = est1_splits(d_in);
+  const int n_chunks = (int)((n_ctx + kGramChunk - 1) / kGramChunk);
+  auto carve = [&](Carver& c, float** zp, double** gp) {
+    *zp = c.take<float>((size_t)n_split * n_ctx * mk);
+    *gp = c.take<double>((size_t)n_chunks * mk * mk);
+  };
+  float* zp;
+  double* gp;
+  {
+    Carver c(nullptr);
+    carve(c, &zp, &gp);
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  carve(c, &zp, &gp);
+  cudaStream_t s = cs(stream);
+  int rc = est_stage1(x, fp32, n_ctx, d_in, ldx, n_proj, w_a, fp32, k, zp, n_split, s);
+  if (rc) return from_kernel(rc);
+  if (crit == SL_CRIT_SWIGLU_L2) {
+    rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, s);
+    return from_kernel(rc);
+  }
+  rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s);
+  if (rc) return from_kernel(rc);
+  if (crit == SL_CRIT_L2) {
+    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
+    return from_kernel(rc);
+  }
+  rc = est_linear_scores(gp, n_chunks, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
+                         scores, s);
+  if (rc) return from_kernel(rc);
+  if (n_proj == 3)
+    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
+  return from_kernel(rc);
+}
+
+// ------------------------------------------------------------------ a3
+sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int32_t heads_per_group,
+                             int32_t head_dim, int32_t* sigma_wide, sl_stream stream) {
+  if (!scores || !sigma) return SL_ERR_INVALID_ARG;
+  if (n <= 0 || n > 40960 || n_keep < 1 || n_keep > n) return SL_ERR_SHAPE;
+  if (heads_per_group > 0 && (!sigma_wide || head_dim <= 0 || n % head_dim)) return SL_ERR_INVALID_ARG;
+  const int64_t n_wide = heads_per_group > 0 ? n * heads_per_group : 0;
+  return from_kernel(select_channels(scores, n, n_keep, sigma, heads_per_group, head_dim, n_wide,
+                                     heads_per_group > 0 ? sigma_wide : nullptr, nullptr, cs(stream)));
+}
+
+// ------------------------------------------------------------------ a6
+sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx,
+                          int64_t n_tok, int64_t n_ctx, int32_t in_layout, const sl_channels* in_ch, float* xa,
+                          void* xa_s, int64_t ld_xa, const void* const* dy, const int64_t* ld_dy, int32_t out_layout,
+                          const sl_channels* out_ch, float* const* dya, void* const* dya_s, float* const* dA,
+                          float* const* dB, sl_workspace* ws, sl_stream stream) {
+  if (!lin || !x || n_ad < 1 || n_ad > 4) return SL_ERR_INVALID_ARG;
+  if (n_tok <= 0 || n_ctx < 0 || n_ctx > n_tok) return SL_ERR_SHAPE;
+  const int64_t d_in = lin[0].d_in;
+  int R = 0;
+  for (int i = 0; i < n_ad; ++i) {
+    if (!linear_ok(lin[i]) || lin[i].d_in != d_in) return SL_ERR_INVALID_ARG;
+    R += lin[i].r;
+  }
+  if (ldx < d_in || ldx % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+  const bool in_sig = in_layout == SL_LAYOUT_SIGMA && n_ctx > 0;
+  if (in_sig && (!in_ch || !channels_ok(*in_ch, d_in))) return SL_ERR_INVALID_ARG;
+  if (!xa_s || ld_xa < R || ld_xa % 8 || !al16(xa_s)) return SL_ERR_ALIGNMENT;
+  cudaStream_t s = cs(stream);
+  const int64_t C = n_ctx, T = n_tok, O = T - C;
+
+  if (mode == SL_LORA_FWD) {
+    if (!xa) return SL_ERR_INVALID_ARG;
+    if (R > 256) return SL_ERR_SHAPE;
+    for (int i = 1; i < n_ad; ++i)
+      if (lin[i].lora_scale != lin[0].lora_scale) return SL_ERR_UNSUPPORTED;
+    auto carve = [&](Carver& c, void** asig) {
+      for (int i = 0; i < n_ad; ++i) asig[i] = in_sig ? c.take<uint16_t>((size_t)lin[i].r * d_in) : nullptr;
+    };
+    void* asig[4];
+    {
+      Carver c(nullptr);
+      carve(c, asig);
+      if (sl_status st = ws_check(ws, c.off)) return st;
+    }
+    Carver c(ws->ptr);
+    carve(c, asig);
+    if (in_sig)
+      for (int i = 0; i < n_ad; ++i)
+        if (int rc = gather_cols_bf16(lin[i].lora_a, d_in, lin[i].r, in_ch->sigma, d_in, asig[i], d_in, s))
+          return from_kernel(rc);
+    GemmBuilder gb;
+    const int mx = gb.map(x, T, d_in, ldx, kBM);
+    const int n_mma = (int)rup(R, 16);
+    auto add_prob = [&](int64_t M, int64_t row0, bool sig) {
+      Prob* p = gb.add((int)M, R, kBN, n_mma);
+      Seg* sg = gb.seg(p, mx, 0, (int)row0, 0, 0, 0, (int)d_in, kBig);
+      int off = 0;
+      for (int i = 0; i < n_ad; ++i) {
+        const int mb = gb.map(sig ? asig[i] : lin[i].lora_a, lin[i].r, d_in, d_in, lin[i].r);
+        gb.bsrc(sg, mb, off, lin[i].r, 0, 0);
+        off += lin[i].r;
+      }
+      if (!p) return;
+      p->epi = EPI_XA;
+      p->out_row0 = (int)row0;
+      p->out0 = xa;
+      p->ld0 = ld_xa;
+      p->out1 = xa_s;
+      p->ld1 = ld_xa;
+      p->a0 = 1.f;
+      p->a1 = lin[0].lora_scale;
+    };
+    if (in_sig) {
+      add_prob(C, 0, true);
+      add_prob(O, C, false);
+    } else {
+      add_prob(T, 0, false);
+    }
+    return from_builder(gb.launch(err_word(ws), s));
+  }
+
+  if (mode != SL_LORA_BWD) return SL_ERR_INVALID_ARG;
+  if (!dy || !ld_dy || !dya || !dya_s || !dA || !dB) return SL_ERR_INVALID_ARG;
+  const bool out_sig = out_layout == SL_LAYOUT_SIGMA && n_ctx > 0;
+  if (out_sig && !out_ch) return SL_ERR_INVALID_ARG;
+  for (int i = 0; i < n_ad; ++i) {
+    if (!dy[i] || !dya[i] || !dya_s[i] || !dA[i] || !dB[i]) return SL_ERR_INVALID_ARG;
+    if (ld_dy[i] < lin[i].d_out || ld_dy[i] % 8 || !al16(dy[i]) || !al16(dya_s[i])) return SL_ERR_ALIGNMENT;
+    if (out_sig && !channels_ok(out_ch[i], lin[i].d_out)) return SL_ERR_INVALID_ARG;
+  }
+  auto carve = [&](Carver& c, void** bsig) {
+    for (int i = 0; i < n_ad; ++i) bsig[i] = out_sig ? c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r) : nullptr;
+  };
+  void* bsig[4];
+  {
+    Carver c(nullptr);
+    carve(c, bsig);
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  carve(c, bsig);
+  if (out_sig)
+    for (int i = 0; i < n_ad; ++i)
+      if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i],
+                                    lin[i].r, 0, s))
+        return from_kernel(rc);
+  // launch 1: dya = scale * dy B
+  {
+    GemmBuilder gb;
+    for (int i = 0; i < n_ad; ++i) {
+      const sl_linear& L = lin[i];
+      const int mdy = gb.map(dy[i], T, L.d_out, ld_dy[i], kBM);
+      const int mbn = gb.map(L.lora_b, L.d_out, L.r, L.r, 64);
+      const int mbs = out_sig ? gb.map(bsig[i], L.d_out, L.r, L.r, 64) : -1;
+      auto add_prob = [&](int64_t M, int64_t row0, int mb) {
+        Prob* p = gb.add((int)M, L.r, kBN, (int)rup(L.r, 16));
+        Seg* sg = gb.seg(p, mdy, 0, (int)row0, 0, 1, 0, (int)L.d_out, kBig);
+        gb.bsrc(sg, mb, 0, 64, 0, 0);
+        if (!p) return;
+        p->epi = EPI_XA;
+        p->out_row0 = (int)row0;
+        p->out0 = dya[i];
+        p->ld0 = L.r;
+        p->out1 = dya_s[i];
+        p->ld1 = L.r;
+        p->a0 = L.lora_scale;
+        p->a1 = L.lora_scale;
+      };
+      if (out_sig) {
+        add_prob(C, 0, mbs);
+        add_prob(O, C, mbn);
+      } else {
+        add_prob(T, 0, mbn);
+      }
+    }
+    if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
+  }
+  // launch 2: dB = dy^T xa_s, dA = (x^T dya)^T over the natural part; launch 3: sigma parts (accumulate)
+  for (int pass = 0; pass < 2; ++pass) {
+    GemmBuilder gb;
+    bool any = false;
+    for (int i = 0; i < n_ad; ++i) {
+      const sl_linear& L = lin[i];
+      int64_t koff = 0;
+      for (int i2 = 0; i2 < i; ++i2) koff += lin[i2].r;
+      const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
+      // dB
+      const bool split_b = out_sig;
+      if (pass == 0 || split_b) {
+        const bool ctx_part = pass == 1;
+        const int64_t rows = ctx_part ? C : T;   // map extents zero-fill past the part
+        const int64_t k0 = (split_b && !ctx_part) ? C : 0;
+        const int64_t K = split_b ? (ctx_part ? C : O) : T;
+        if (K > 0) {
+          const int ma = gb.map(dy[i], rows, L.d_out, ld_dy[i], 64);
+          const int mb = gb.map(xa_blk, rows, L.r, ld_xa, 64);
+          Prob* p = gb.add((int)L.d_out, L.r, kBN, (int)rup(L.r, 16));
+          Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
+          gb.bsrc(sg, mb, 0, 64, 0, 0);
+          if (p) {
+            p->epi = EPI_F32;
+            p->out0 = dB[i];
+            p->ld0 = L.r;
+            p->beta = ctx_part ? 1 : 0;
+            p->row_map = ctx_part ? out_ch[i].sigma : nullptr;
+          }
+          any = true;
+        } else if (!ctx_part) {
+          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s);
+        }
+      }
+      // dA
+      const bool split_a = in_sig;
+      if (pass == 0 || split_a) {
+        const bool ctx_part = pass == 1;
+        const int64_t rows = ctx_part ? C : T;
+        const int64_t k0 = (split_a && !ctx_part) ? C : 0;
+        const int64_t K = split_a ? (ctx_part ? C : O) : T;
+        if (K > 0) {
+          const int ma = gb.map(x, rows, d_in, ldx, 64);
+          const int mb = gb.map(dya_s[i], rows, L.r, L.r, 64);
+          Prob* p = gb.add((int)d_in, L.r, kBN, (int)rup(L.r, 16));
+          Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
+          gb.bsrc(sg, mb, 0, 64, 0, 0);
+          if (p) {
+            p->epi = EPI_F32_T;
+            p->out0 = dA[i];
+            p->ld0 = d_in;
+            p->beta = ctx_part ? 1 : 0;
+            p->row_map = ctx_part ? in_ch->sigma : nullptr;
+          }
+          any = true;
+        } else if (!ctx_part) {
+          cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s);
+        }
+      }
+    }
+    if (any)
+      if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
+  }
+  return SL_OK;
+}
+
+// ------------------------------------------------------------------ a4
+sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_channels* ch, int32_t epi, const void* x,
+                               int64_t ldx, int64_t n_tok, int64_t n_ctx, int32_t in_layout, int32_t out_layout,
+                               const void* xa_s, int64_t ld_xa, void* const* y, const int64_t* ldy, sl_workspace* ws,
+                               sl_stream stream) {
+  if (!lin || !ch || !x || !xa_s || !y || !ldy || n_lin < 1 || n_lin > 4) return SL_ERR_INVALID_ARG;
+  if (n_tok <= 0 || n_ctx < 0 || n_ctx > n_tok) return SL_ERR_SHAPE;
+  const int64_t T = n_tok, C = n_ctx, O = T - C;
+  const int slice = lin[0].slice;
+  int R = 0;
+  for (int i = 0; i < n_lin; ++i) {
+    if (!linear_ok(lin[i]) || lin[i].slice != slice || lin[i].d_in != lin[0].d_in) return SL_ERR_INVALID_ARG;
+    if (!channels_ok(ch[i], slice == SL_SLICE_OUT ? lin[i].d_out : lin[i].d_in)) return SL_ERR_INVALID_ARG;
+    R += lin[i].r;
+  }
+  const int64_t d_in = lin[0].d_in;
+  if (ldx < d_in || ldx % 8 || !al16(x) || ld_xa < R || ld_xa % 8 || !al16(xa_s)) return SL_ERR_ALIGNMENT;
+  cudaStream_t s = cs(stream);
+
+  if (slice == SL_SLICE_OUT && epi == SL_EPI_NONE) {
+    for (int i = 0; i < n_lin; ++i)
+      if (!y[i] || ldy[i] < lin[i].d_out || ldy[i] % 8 || !al16(y[i])) return SL_ERR_ALIGNMENT;
+    auto carve = [&](Carver& c, void** wc, void** bs) {
+      for (int i = 0; i < n_lin; ++i) {
+        wc[i] = c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        bs[i] = c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r);
+      }
+    };
+    void *wc[4], *bs[4];
+    {
+      Carver c(nullptr);
+      carve(c, wc, bs);
+      if (sl_status st = ws_check(ws, c.off)) return st;
+    }
+    Carver c(ws->ptr);
+    carve(c, wc, bs);
+    for (int i = 0; i < n_lin; ++i) {
+      if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
+        return from_kernel(rc);
+      if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r, 0, s))
+        return from_kernel(rc);
+    }
+    GemmBuilder gb;
+    const int mx = gb.map(x, T, d_in, ldx, kBM);
+    int koff = 0;
+    for (int i = 0; i < n_lin; ++i) {
+      const sl_linear& L = lin[i];
+      const int mxa = gb.map(static_cast<const uint16_t*>(xa_s) + koff, T, L.r, ld_xa, kBM);
+      koff += L.r;
+      if (C > 0) {
+        const int mwc = gb.map(wc[i], ch[i].n_keep, d_in, d_in, kBN);
+        const int mbs = gb.map(bs[i], L.d_out, L.r, L.r, kBN);
+        Prob* p = gb.add((int)C, (int)L.d_out, kBN, kBN);
+        gb.bsrc(gb.seg(p, mx, 0, 0, 0, 0, 0, (int)d_in, (int)ch[i].n_keep), mwc, 0, kBN, 0, kBN);
+        gb.bsrc(gb.seg(p, mxa, 0, 0, 0, 0, 0, L.r, kBig), mbs, 0, kBN, 0, kBN);
+        if (p) {
+          p->epi = EPI_BF16;
+          p->out0 = y[i];
+          p->ld0 = ldy[i];
+          p->col_map = out_layout == SL_LAYOUT_NATURAL ? ch[i].sigma : nullptr;
+        }
+      }
+      if (O > 0) {
+        const int mw = gb.map(L.w, L.d_out, d_in, d_in, kBN);
+        const int mb = gb.map(L.lora_b, L.d_out, L.r, L.r, kBN);
+        Prob* p = gb.add((int)O, (int)L.d_out, kBN, kBN);
+        gb.bsrc(gb.seg(p, mx, 0, (int)C, 0, 0, 0, (int)d_in, kBig), mw, 0, kBN, 0, kBN);
+        gb.bsrc(gb.seg(p, mxa, 0, (int)C, 0, 0, 0, L.r, kBig), mb, 0, kBN, 0, kBN);
+        if (p) {
+          p->epi = EPI_BF16;
+          p->out0 = y[i];
+          p->ld0 = ldy[i];
+          p->out_row0 = (int)C;
+        }
+      }
+    }
+    return from_builder(gb.launch(err_word(ws), s));
+  }
+
+  if (slice == SL_SLICE_OUT && epi == SL_EPI_SWIGLU) {
+    if (n_lin != 2 || lin[0].d_out != lin[1].d_out || lin[0].r + lin[1].r > 64) return SL_ERR_INVALID_ARG;
+    if (lin[0].lora_scale != lin[1].lora_scale) return SL_ERR_UNSUPPORTED;
+    const int64_t F = lin[0].d_out;
+    for (int i = 0; i < 3; ++i)
+      if (!y[i] || ldy[i] < F || ldy[i] % 8 || !al16(y[i]) || ldy[i] != ldy[0]) return SL_ERR_ALIGNMENT;
+    const int64_t nt = (F + 127) / 128;  // paired tiles: 128 channels each
+    auto carve = [&](Carver& c, void** wc, void** pk) {
+      wc[0] = c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      wc[1] = c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      pk[0] = c.take<uint16_t>((size_t)nt * 256 * 64);  // sigma order
+      pk[1] = c.take<uint16_t>((size_t)nt * 256 * 64);  // natural order
+    };
+    void *wc[2], *pk[2];
+    {
+      Carver c(nullptr);
+      carve(c, wc, pk);
+      if (sl_status st = ws_check(ws, c.off)) return st;
+    }
+    Carver c(ws->ptr);
+    carve(c, wc, pk);
+    const int32_t* sig = ch[0].sigma;
+    for (int i = 0; i < 2; ++i)
+      if (int rc = gather_rows_bf16(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in, 0, s)) return from_kernel(rc);
+    // LoRA B operand of a paired tile t: rows 256 t + j = [B_gate[c_j] | 0], rows 256 t + 128 + j = [0 | B_up[c_j]]
+    cudaMemsetAsync(pk[0], 0, (size_t)nt * 256 * 64 * 2, s);
+    cudaMemsetAsync(pk[1], 0, (size_t)nt * 256 * 64 * 2, s);
+    for (int v = 0; v < 2; ++v) {
+      const int32_t* idx = v == 0 ? sig : nullptr;
+      if (int rc = gather_rows_bf16(lin[0].lora_b, lin[0].r, idx, F, lin[0].r, pk[v], 64, 0, s, 128, 256, 0))
+        return from_kernel(rc);
+      if (int rc = gather_rows_bf16(lin[1].lora_b, lin[1].r, idx, F, lin[1].r, pk[v], 64, lin[0].r, s, 128, 256, 128))
+        return from_kernel(rc);
+    }
+    GemmBuilder gb;
+    const int mx = gb.map(x, T, d_in, ldx, kBM);
+    const int mxa = gb.map(xa_s, T, lin[0].r + lin[1].r, ld_xa, kBM);
+    auto add_prob = [&](int64_t M, int64_t row0, int mg, int mu, int mp, int n_limit) {
+      Prob* p = gb.add((int)M, (int)F, 128, kBN);
+      Seg* sg = gb.seg(p, mx, 0, (int)row0, 0, 0, 0, (int)d_in, n_limit);
+      gb.bsrc(sg, mg, 0, 128, 0, 128);
+      gb.bsrc(sg, mu, 128, 128, 0, 128);
+      gb.bsrc(gb.seg(p, mxa, 0, (int)row0, 0, 0, 0, 64, kBig), mp, 0, kBN, 0, kBN);
+      if (!p) return;
+      p->epi = EPI_SWIGLU;
+      p->out0 = y[0];
+      p->out1 = y[1];
+      p->out2 = y[2];
+      p->ld0 = ldy[0];
+      p->out_row0 = (int)row0;
+    };
+    if (C > 0)
+      add_prob(C, 0, gb.map(wc[0], ch[0].n_keep, d_in, d_in, 128), gb.map(wc[1], ch[0].n_keep, d_in, d_in, 128),
+               gb.map(pk[0], nt * 256, 64, 64, kBN), (int)ch[0].n_keep);
+    if (O > 0)
+      add_prob(O, C, gb.map(lin[0].w, F, d_in, d_in, 128), gb.map(lin[1].w, F, d_in, d_in, 128),
+               gb.map(pk[1], nt * 256, 64, 64, kBN), kBig);
+    return from_builder(gb.launch(err_word(ws), s));
+  }
+
+  if (slice == SL_SLICE_IN && epi == SL_EPI_NONE) {
+    if (n_lin != 1) return SL_ERR_INVALID_ARG;
+    const sl_linear& L = lin[0];
+    if (!L.w_t || !al16(L.w_t)) return SL_ERR_INVALID_ARG;
+    if (!y[0] || ldy[0] < L.d_out || ldy[0] % 8 || !al16(y[0])) return SL_ERR_ALIGNMENT;
+    const int64_t nk = ch[0].n_keep;
+    const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
+    const int64_t ldc = rup(nk, 8);
+    auto carve = [&](Carver& c, void** wtc, void** xc) {
+      *wtc = c.take<uint16_t>((size_t)nk * L.d_out);
+      *xc = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * ldc) : nullptr;
+    };
+    void *wtc, *xc;
+    {
+      Carver c(nullptr);
+      carve(c, &wtc, &xc);
+      if (sl_status st = ws_check(ws, c.off)) return st;
+    }
+    Carver c(ws->ptr);
+    carve(c, &wtc, &xc);
+    if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s)) return from_kernel(rc);
+    if (xc)
+      if (int rc = gather_cols_bf16(x, ldx, C, ch[0].sigma, nk, xc, ldc, s)) return from_kernel(rc);
+    GemmBuilder gb;
+    const int mxa = gb.map(xa_s, T, L.r, ld_xa, kBM);
+    const int mb = gb.map(L.lora_b, L.d_out, L.r, L.r, kBN);
+    if (C > 0) {
+      const int ma = in_sig ? gb.map(x, C, nk, ldx, kBM) : gb.map(xc, C, nk, ldc, kBM);
+      const int mw = gb.map(wtc, nk, L.d_out, L.d_out, 64);
+      Prob* p = gb.add((int)C, (int)L.d_out, kBN, kBN);
+      gb.bsrc(gb.seg(p, ma, 0, 0, 0, 1, 0, (int)nk, kBig), mw, 0, kBN, 0, kBN);
+      gb.bsrc(gb.seg(p, mxa, 0, 0, 0, 0, 0, L.r, kBig), mb, 0, kBN, 0, kBN);
+      if (p) {
+        p->epi = EPI_BF16;
+        p->out0 = y[0];
+        p->ld0 = ldy[0];
+      }
+    }
+    if (O > 0) {
+      const int ma = gb.map(x, T, d_in, ldx, kBM);
+      const int mw = gb.map(L.w, L.d_out, d_in, d_in, kBN);
+      Prob* p = gb.add((int)O, (int)L.d_out, kBN, kBN);
+      gb.bsrc(gb.seg(p, ma, 0, (int)C, 0, 0, 0, (int)d_in, kBig), mw, 0, kBN, 0, kBN);
+      gb.bsrc(gb.seg(p, mxa, 0, (int)C, 0, 0, 0, L.r, kBig), mb, 0, kBN, 0, kBN);
+      if (p) {
+        p->epi = EPI_BF16;
+        p->out0 = y[0];
+        p->ld0 = ldy[0];
+        p->out_row0 = (int)C;
+      }
+    }
+    return from_builder(gb.launch(err_word(ws), s));
+  }
+  return SL_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ a5
+sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_channels* ch, int32_t epi,
+                               const void* const* dy, const int64_t* ld_dy, int64_t n_tok, int64_t n_ctx,
+                               int32_t in_layout, int32_t out_layout, const void* const* dya_s, void* dx,
+                               int64_t lddx, const void* const* aux, void* const* aux_out, sl_workspace* ws,
+                               sl_stream stream) {
+  if (!lin || !ch || !dy || !ld_dy || !dya_s || n_lin < 1 || n_lin > 3) return SL_ERR_INVALID_ARG;
+  if (n_tok <= 0 || n_ctx < 0 || n_ctx > n_tok) return SL_ERR_SHAPE;
+  const int64_t T = n_tok, C = n_ctx, O = T - C;
+  const int slice = lin[0].slice;
+  const int64_t d_in = lin[0].d_in;
+  for (int i = 0; i < n_lin; ++i) {
+    if (!linear_ok(lin[i]) || lin[i].slice != slice || lin[i].d_in != d_in) return SL_ERR_INVALID_ARG;
+    if (!channels_ok(ch[i], slice == SL_SLICE_OUT ? lin[i].d_out : lin[i].d_in)) return SL_ERR_INVALID_ARG;
+    if (!dy[i] || !dya_s[i]) return SL_ERR_INVALID_ARG;
+    if (ld_dy[i] < lin[i].d_out || ld_dy[i] % 8 || !al16(dy[i]) || !al16(dya_s[i])) return SL_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = cs(stream);
+
+  if (slice == SL_SLICE_OUT) {
+    if (epi != SL_EPI_NONE) return SL_ERR_UNSUPPORTED;
+    if (!dx || lddx < d_in || lddx % 8 || !al16(dx)) return SL_ERR_ALIGNMENT;
+    const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
+    auto carve = [&](Carver& c, void** wc, void** dyc) {
+      for (int i = 0; i < n_lin; ++i) {
+        wc[i] = c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        dyc[i] = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * rup(ch[i].n_keep, 8)) : nullptr;
+      }
+    };
+    void *wc[3], *dyc[3];
+    {
+      Carver c(nullptr);
+      carve(c, wc, dyc);
+      if (sl_status st = ws_check(ws, c.off)) return st;
+    }
+    Carver c(ws->ptr);
+    carve(c, wc, dyc);
+    for (int i = 0; i < n_lin; ++i) {
+      if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
+        return from_kernel(rc);
+      if (dyc[i])
+        if (int rc = gather_cols_bf16(dy[i], ld_dy[i], C, ch[i].sigma, ch[i].n_keep, dyc[i], rup(ch[i].n_keep, 8), s))
+          return from_kernel(rc);
+    }
+    GemmBuilder gb;
+    Prob* pc = C > 0 ? gb.add((int)C, (int)d_in, kBN, kBN) : nullptr;
+    Prob* po = O > 0 ? gb.add((int)O, (int)d_in, kBN, kBN) : nullptr;
+    for (int i = 0; i < n_lin; ++i) {
+      const sl_linear& L = lin[i];
+      const int mya = gb.map(dya_s[i], T, L.r, L.r, kBM);
+      const int mam = gb.map(L.lora_a, L.r, d_in, d_in, 64);
+      if (pc) {
+        const int64_t nk = ch[i].n_keep;
+        const int ma = dyc[i] ? gb.map(dyc[i], C, nk, rup(nk, 8), kBM) : gb.map(dy[i], C, nk, ld_dy[i], kBM);
+        const int mw = gb.map(wc[i], nk, d_in, d_in, 64);
+        gb.bsrc(gb.seg(pc, ma, 0, 0, 0, 1, 0, (int)nk, kBig), mw, 0, kBN, 0, kBN);
+        gb.bsrc(gb.seg(pc, mya, 0, 0, 0, 1, 0, L.r, kBig), mam, 0, kBN, 0, kBN);
+      }
+      if (po) {
+        const int ma = gb.map(dy[i], T, L.d_out, ld_dy[i], kBM);
+        const int mw = gb.map(L.w, L.d_out, d_in, d_in, 64);
+        gb.bsrc(gb.seg(po, ma, 0, (int)C, 0, 1, 0, (int)L.d_out, kBig), mw, 0, kBN, 0, kBN);
+        gb.bsrc(gb.seg(po, mya, 0, (int)C, 0, 1, 0, L.r, kBig), mam, 0, kBN, 0, kBN);
+      }
+    }
+    for (Prob* p : {pc, po}) {
+      if (!p) continue;
+      p->epi = EPI_BF16;
+      p->out0 = dx;
+      p->ld0 = lddx;
+      p->out_row0 = p == po ? (int)C : 0;
+    }
+    return from_builder(gb.launch(err_word(ws), s));
+  }
+
+  // SL_SLICE_IN
+  if (n_lin != 1) return SL_ERR_INVALID_ARG;
+  const sl_linear& L = lin[0];
+  if (!L.w_t || !al16(L.w_t)) return SL_ERR_INVALID_ARG;
+  const bool swiglu = epi == SL_EPI_SWIGLU;
+  if (swiglu) {
+    if (!aux || !aux_out || !aux[0] || !aux[1] || !aux_out[0] || !aux_out[1]) return SL_ERR_INVALID_ARG;
+    if (lddx < d_in || lddx % 8) return SL_ERR_ALIGNMENT;
+    for (int i = 0; i < 2; ++i)
+      if (!al16(aux[i]) || !al16(aux_out[i])) return SL_ERR_ALIGNMENT;
+  } else {
+    if (epi != SL_EPI_NONE) return SL_ERR_INVALID_ARG;
+    if (!dx || lddx < d_in || lddx % 8 || !al16(dx)) return SL_ERR_ALIGNMENT;
+  }
+  const int64_t nk = ch[0].n_keep;
+  auto carve = [&](Carver& c, void** wtc, void** at, void** ats) {
+    *wtc = c.take<uint16_t>((size_t)nk * L.d_out);
+    *at = c.take<uint16_t>((size_t)d_in * L.r);
+    *ats = c.take<uint16_t>((size_t)d_in * L.r);
+  };
+  void *wtc, *at, *ats;
+  {
+    Carver c(nullptr);
+    carve(c, &wtc, &at, &ats);
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  carve(c, &wtc, &at, &ats);
+  if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s)) return from_kernel(rc);
+  if (int rc = transpose_bf16(L.lora_a, L.r, d_in, d_in, at, L.r, s)) return from_kernel(rc);
+  if (int rc = gather_rows_bf16(at, L.r, ch[0].sigma, d_in, L.r, ats, L.r, 0, s)) return from_kernel(rc);
+  GemmBuilder gb;
+  const int mdy = gb.map(dy[0], T, L.d_out, ld_dy[0], kBM);
+  const int mya = gb.map(dya_s[0], T, L.r, L.r, kBM);
+  auto set_epi = [&](Prob* p, int64_t row0, bool natural_ctx) {
+    if (!p) return;
+    p->out_row0 = (int)row0;
+    if (swiglu) {
+      p->epi = EPI_DSWIGLU;
+      p->out0 = aux_out[0];
+      p->out1 = aux_out[1];
+      p->aux0 = aux[0];
+      p->aux1 = aux[1];
+      p->ld0 = lddx;
+      p->ld_aux = lddx;
+    } else {
+      p->epi = EPI_BF16;
+      p->out0 = dx;
+      p->ld0 = lddx;
+      p->col_map = natural_ctx ? ch[0].sigma : nullptr;
+    }
+  };
+  if (C > 0) {
+    const int mw = gb.map(wtc, nk, L.d_out, L.d_out, kBN);
+    const int mat = gb.map(ats, d_in, L.r, L.r, kBN);
+    Prob* p = gb.add((int)C, (int)d_in, kBN, kBN);
+    gb.bsrc(gb.seg(p, mdy, 0, 0, 0, 0, 0, (int)L.d_out, (int)nk), mw, 0, kBN, 0, kBN);
+    gb.bsrc(gb.seg(p, mya, 0, 0, 0, 0, 0, L.r, kBig), mat, 0, kBN, 0, kBN);
+    set_epi(p, 0, !swiglu && out_layout == SL_LAYOUT_NATURAL);
+  }
+  if (O > 0) {
+    const int mw = gb.map(L.w, L.d_out, d_in, d_in, 64);
+    const int mam = gb.map(L.lora_a, L.r, d_in, d_in, 64);
+    Prob* p = gb.add((int)O, (int)d_in, kBN, kBN);
+    gb.bsrc(gb.seg(p, mdy, 0, (int)C, 0, 1, 0, (int)L.d_out, kBig), mw, 0, kBN, 0, kBN);
+    gb.bsrc(gb.seg(p, mya, 0, (int)C, 0, 1, 0, L.r, kBig), mam, 0, kBN, 0, kBN);
+    set_epi(p, C, false);
+  }
+  return from_builder(gb.launch(err_word(ws), s));
+}
+
+sl_status sl_profile_enable(int32_t on) {
+  g_prof.store(on != 0);
+  return SL_OK;
+}
+
+sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launches, double* gemm_ms) {
+  if (!kernel_launches || !gemm_launches || !gemm_ms) return SL_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  double ms = 0.0;
+  for (size_t i = 0; i < g_ev_used; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, g_events[i].first, g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
+    ms += t;
+  }
+  *gemm_ms = ms;
+  *gemm_launches = (int64_t)g_ev_used;
+  *kernel_launches = (int64_t)g_launches.exchange(0);
+  g_ev_used = 0;
+  return SL_OK;
+}
+
+sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream) {
+  if (!w || !w_t) return SL_ERR_INVALID_ARG;
+  if (d_out <= 0 || d_in <= 0) return SL_ERR_SHAPE;
+  return from_kernel(transpose_bf16(w, d_out, d_in, d_in, w_t, d_out, cs(stream)));
+}
+
+sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
+                          void* dst, int64_t ld_dst, sl_stream stream) {
+  if (!src || !perm || !dst) return SL_ERR_INVALID_ARG;
+  if (n_rows <= 0 || n_cols <= 0 || ld_src < n_cols || ld_dst < n_cols) return SL_ERR_SHAPE;
+  return from_kernel(permute_rows_bf16(src, ld_src, perm, n_rows, n_cols, dst, ld_dst, cs(stream)));
+}
+
+}  // extern "C"

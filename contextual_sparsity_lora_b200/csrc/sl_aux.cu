@@ -1,0 +1,118 @@
+// Data-movement helpers: row gathers (weight rows of kept channels, token
+// permutation), column gathers (kept columns of activations), transposes of
+// frozen weights and LoRA matrices, and small fp32 adds. All bf16 traffic moves
+// in 16-byte vectors where the layout allows it.
+#include <cuda_bf16.h>
+
+#include "sl_internal.h"
+
+namespace sl {
+
+namespace {
+
+// dst[drow(i), col0 + c] = src[idx ? idx[i] : i, c], c < n_cols, where
+// drow(i) = (i / blk) * blk_stride + blk_off + i % blk (blk = 0: drow(i) = i).
+// One warp per row.
+__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src,
+                                   const int32_t* __restrict__ idx, int64_t n_rows, int64_t n_cols,
+                                   __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int64_t col0, int vec, int blk,
+                                   int blk_stride, int blk_off) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int64_t sr = idx ? (int64_t)idx[row] : row;
+  const int64_t drow = blk ? (row / blk) * blk_stride + blk_off + row % blk : row;
+  const __nv_bfloat16* s = src + sr * ld_src;
+  __nv_bfloat16* d = dst + drow * ld_dst + col0;
+  if (vec) {
+    const int64_t nv = n_cols / 8;
+    for (int64_t c = lane; c < nv; c += 32)
+      reinterpret_cast<uint4*>(d)[c] = __ldg(reinterpret_cast<const uint4*>(s) + c);
+  } else {
+    for (int64_t c = lane; c < n_cols; c += 32) d[c] = s[c];
+  }
+}
+
+// dst[t, j] = src[t, idx[j]]
+__global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t n_rows,
+                                   const int32_t* __restrict__ idx, int64_t n_idx, __nv_bfloat16* __restrict__ dst,
+                                   int64_t ld_dst) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n_idx) return;
+  const int64_t c = idx[j];
+  for (int64_t t = blockIdx.y; t < n_rows; t += gridDim.y) dst[t * ld_dst + j] = src[t * ld_src + c];
+}
+
+// dst[c, r] = src[r, c] with a 32 x 32 shared-memory tile.
+__global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols, int64_t ld_src,
+                                 __nv_bfloat16* __restrict__ dst, int64_t ld_dst) {
+  __shared__ __nv_bfloat16 tile[32][34];
+  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[r * ld_src + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[c * ld_dst + r] = tile[threadIdx.x][i];
+  }
+}
+
+__global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] += src[i];
+}
+
+}  // namespace
+
+int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
+                     int64_t ld_dst, int64_t dst_col0, cudaStream_t s, int blk, int blk_stride, int blk_off) {
+  if (n_rows <= 0 || n_cols <= 0) return 0;
+  const int vec = (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (dst_col0 % 8 == 0) &&
+                  ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
+  const int rows_per_block = 8;
+  gather_rows_kernel<<<(unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s>>>(
+      (const __nv_bfloat16*)src, ld_src, idx, n_rows, n_cols, (__nv_bfloat16*)dst, ld_dst, dst_col0, vec, blk,
+      blk_stride, blk_off);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int32_t* idx, int64_t n_idx, void* dst,
+                     int64_t ld_dst, cudaStream_t s) {
+  if (n_rows <= 0 || n_idx <= 0) return 0;
+  dim3 grid((unsigned)((n_idx + 255) / 256), (unsigned)(n_rows < 1024 ? n_rows : 1024));
+  gather_cols_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)src, ld_src, n_rows, idx, n_idx,
+                                          (__nv_bfloat16*)dst, ld_dst);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,
+                   cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return 0;
+  dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
+  transpose_kernel<<<grid, dim3(32, 8), 0, s>>>((const __nv_bfloat16*)src, rows, cols, ld_src, (__nv_bfloat16*)dst,
+                                                ld_dst);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols, void* dst,
+                      int64_t ld_dst, cudaStream_t s) {
+  return gather_rows_bf16(src, ld_src, perm, n_rows, n_cols, dst, ld_dst, 0, s);
+}
+
+int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s) {
+  if (n <= 0) return 0;
+  add_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dst, src, n);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+}  // namespace sl

@@ -1,0 +1,372 @@
+// SVD sparsity estimator and criterion reductions on CUDA cores (fp32 products,
+// fixed-order reductions; no floating-point atomics, so results are
+// run-to-run identical).
+//
+// Stage 1: Z = X_ctx [W_A^(1) ... W_A^(m)]  (split over the input dimension;
+//          partial sums per split, then a fixed-order sum).
+// Stage 2 (SwiGLU L2): s_i = sqrt(sum_t (SiLU(g_ti) u_ti)^2) with
+//          g = Z_gate W_B^gate, u = Z_up W_B^up evaluated per (token, channel).
+// Stage 2 (linear criteria, V and QK): the token reduction of a linear map
+//          collapses to a Gram matrix, sum_t (Z b_i)_t^2 = b_i^T (Z^T Z) b_i,
+//          formed and contracted in fp64.
+#include <cuda_bf16.h>
+
+#include "sl_internal.h"
+
+namespace sl {
+
+namespace {
+
+constexpr int kE1Rows = 128;   // tokens per CTA
+constexpr int kE1Chunk = 32;   // input channels staged per step
+constexpr int kE1Threads = 256;
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[8]) {
+  uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 v = __bfloat1622float2(h[j]);
+    f[2 * j] = v.x;
+    f[2 * j + 1] = v.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&f)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ float ld_any(const void* p, int64_t i, int fp32) {
+  return fp32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+struct WaPtrs {
+  const void* p[4];
+};
+
+// grid: (ceil(n_ctx / 128), n_split). Thread = (row group of 4 tokens, column group of CPG outputs).
+template <typename T, int CPG>
+__global__ void __launch_bounds__(kE1Threads) est1_kernel(const T* __restrict__ x, int64_t n_ctx, int64_t d_in,
+                                                          int64_t ldx, WaPtrs wa, int wa_fp32, int k, int mk,
+                                                          int64_t d_per_split, float* __restrict__ zpart) {
+  constexpr int MKP = 8 * CPG;  // padded column count
+  extern __shared__ float e1_smem[];
+  float* xs = e1_smem;                              // [kE1Chunk][kE1Rows + 4]
+  float* ws = xs + kE1Chunk * (kE1Rows + 4);        // [d_per_split][MKP]
+  const int tid = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * kE1Rows;
+  const int64_t d0 = (int64_t)blockIdx.y * d_per_split;
+  const int64_t dn = min(d_per_split, d_in - d0);
+
+  for (int64_t e = tid; e < dn * MKP; e += kE1Threads) {
+    const int64_t d = e / MKP;
+    const int j = (int)(e % MKP);
+    float w = 0.f;
+    if (j < mk) {
+      const int pj = j / k, c = j % k;
+      w = ld_any(wa.p[pj], (d0 + d) * k + c, wa_fp32);
+    }
+    ws[e] = w;
+  }
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const int rg = warp * 4 + (lane >> 3);  // 0..31
+  const int cg = lane & 7;
+  float acc[4][CPG];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CPG; ++c) acc[r][c] = 0.f;
+
+  for (int64_t dc = 0; dc < dn; dc += kE1Chunk) {
+    __syncthreads();
+    // stage X[t0 .. t0+128, d0+dc .. +32] transposed into xs[d][row]
+    for (int e = tid; e < kE1Rows * (kE1Chunk / 8); e += kE1Threads) {
+      const int row = e % kE1Rows;
+      const int dq = (e / kE1Rows) * 8;
+      float f[8];
+      const int64_t t = t0 + row;
+      const int64_t d = d0 + dc + dq;
+      if (t < n_ctx && d + 8 <= d0 + dn) {
+        load8<T>(x + t * ldx + d, f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        if (t < n_ctx)
+          for (int i = 0; i < 8; ++i)
+            if (d + i < d0 + dn) f[i] = (float)x[t * ldx + d + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xs[(dq + i) * (kE1Rows + 4) + row] = f[i];
+    }
+    __syncthreads();
+    const int dlen = (int)min64(kE1Chunk, dn - dc);
+    for (int dd = 0; dd < dlen; ++dd) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[dd * (kE1Rows + 4) + rg * 4]);
+      const float* wrow = &ws[(dc + dd) * MKP + cg * CPG];
+      float w[CPG];
+#pragma unroll
+      for (int c = 0; c < CPG; ++c) w[c] = wrow[c];
+#pragma unroll
+      for (int c = 0; c < CPG; ++c) {
+        acc[0][c] = fmaf(xv.x, w[c], acc[0][c]);
+        acc[1][c] = fmaf(xv.y, w[c], acc[1][c]);
+        acc[2][c] = fmaf(xv.z, w[c], acc[2][c]);
+        acc[3][c] = fmaf(xv.w, w[c], acc[3][c]);
+      }
+    }
+  }
+  float* zp = zpart + (int64_t)blockIdx.y * n_ctx * mk;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int64_t t = t0 + rg * 4 + r;
+    if (t >= n_ctx) continue;
+#pragma unroll
+    for (int c = 0; c < CPG; ++c) {
+      const int j = cg * CPG + c;
+      if (j < mk) zp[t * mk + j] = acc[r][c];
+    }
+  }
+}
+
+// Z[t][j] = sum_s zpart[s][t][j], s in increasing order. Written into split slot 0.
+__global__ void est_reduce_kernel(float* zpart, int n_split, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = zpart[i];
+  for (int s = 1; s < n_split; ++s) acc += zpart[(int64_t)s * n + i];
+  zpart[i] = acc;
+}
+
+constexpr int kE2Threads = 256;  // 8 warps; each lane owns 2 channels of a 64-channel block
+constexpr int kE2Tok = 128;      // tokens staged per step
+
+template <int K>
+__global__ void __launch_bounds__(kE2Threads) est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx,
+                                                                const void* wb_g, const void* wb_u, int wb_fp32,
+                                                                int64_t n_ch, float* __restrict__ scores) {
+  __shared__ float zs[kE2Tok][2 * K];
+  __shared__ double part[8][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ch0 = (int64_t)blockIdx.x * 64 + lane;
+  const int64_t ch1 = ch0 + 32;
+  float wg0[K], wu0[K], wg1[K], wu1[K];
+#pragma unroll
+  for (int c = 0; c < K; ++c) {
+    wg0[c] = ch0 < n_ch ? ld_any(wb_g, c * n_ch + ch0, wb_fp32) : 0.f;
+    wu0[c] = ch0 < n_ch ? ld_any(wb_u, c * n_ch + ch0, wb_fp32) : 0.f;
+    wg1[c] = ch1 < n_ch ? ld_any(wb_g, c * n_ch + ch1, wb_fp32) : 0.f;
+    wu1[c] = ch1 < n_ch ? ld_any(wb_u, c * n_ch + ch1, wb_fp32) : 0.f;
+  }
+  double acc0 = 0.0, acc1 = 0.0;
+  for (int64_t tb = 0; tb < n_ctx; tb += kE2Tok) {
+    __syncthreads();
+    const int tn = (int)min64(kE2Tok, n_ctx - tb);
+    for (int e = threadIdx.x; e < tn * 2 * K; e += kE2Threads) zs[e / (2 * K)][e % (2 * K)] = z[tb * 2 * K + e];
+    __syncthreads();
+    float s0 = 0.f, s1 = 0.f;
+    for (int t = warp; t < tn; t += 8) {
+      float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < K; ++c) {
+        const float zg = zs[t][c], zu = zs[t][K + c];
+        g0 = fmaf(zg, wg0[c], g0);
+        u0 = fmaf(zu, wu0[c], u0);
+        g1 = fmaf(zg, wg1[c], g1);
+        u1 = fmaf(zu, wu1[c], u1);
+      }
+      const float h0 = __fdividef(g0, 1.0f + __expf(fminf(-g0, 80.f))) * u0;
+      const float h1 = __fdividef(g1, 1.0f + __expf(fminf(-g1, 80.f))) * u1;
+      s0 = fmaf(h0, h0, s0);
+      s1 = fmaf(h1, h1, s1);
+    }
+    acc0 += (double)s0;
+    acc1 += (double)s1;
+  }
+  part[warp][lane] = acc0;
+  part[warp][lane + 32] = acc1;
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    double s = 0.0;
+    for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
+    const int64_t ch = (int64_t)blockIdx.x * 64 + threadIdx.x;
+    if (ch < n_ch) scores[ch] = (float)sqrt(s);
+  }
+}
+
+constexpr int kGramTok = 128;
+
+// gram_part[chunk][a][b] = sum_{t in chunk} z[t][a] z[t][b], fp64.
+__global__ void __launch_bounds__(256) est_gram_kernel(const float* __restrict__ z, int64_t n_ctx, int mk,
+                                                       double* __restrict__ gram_part) {
+  __shared__ float zs[kGramTok][64];
+  const int64_t t0 = (int64_t)blockIdx.x * kGramTok;
+  const int tn = (int)min64(kGramTok, n_ctx - t0);
+  for (int e = threadIdx.x; e < tn * mk; e += blockDim.x) zs[e / mk][e % mk] = z[t0 * mk + e];
+  __syncthreads();
+  double* g = gram_part + (int64_t)blockIdx.x * mk * mk;
+  for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
+    const int a = e / mk, b = e % mk;
+    double s = 0.0;
+    for (int t = 0; t < tn; ++t) s = fma((double)zs[t][a], (double)zs[t][b], s);
+    g[e] = s;
+  }
+}
+
+struct WbPtrs {
+  const void* p[3];
+  int64_t n[3];
+};
+
+// One thread per unit. crit 0 (L2): units are the output channels of projection
+// `proj`; crit 2 (QK): units are KV channels (g, d), projections 0 = q, 1 = k.
+__global__ void __launch_bounds__(256) est_linear_scores_kernel(const double* __restrict__ gram_part, int n_chunks,
+                                                                int mk, int k, int crit, int proj0, int proj1,
+                                                                WbPtrs wb,
+                                                                int wb_fp32, int n_q_heads, int n_kv_heads,
+                                                                int head_dim, int64_t n_units,
+                                                                float* __restrict__ scores) {
+  extern __shared__ double gs[];  // [mk][mk]
+  for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
+    double s = 0.0;
+    for (int c = 0; c < n_chunks; ++c) s += gram_part[(int64_t)c * mk * mk + e];
+    gs[e] = s;
+  }
+  __syncthreads();
+  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= n_units) return;
+  // pj indexes wb (0 or 1); blk is the projection's column block in Z.
+  auto quad = [&](int pj, int blk, int64_t col) -> double {
+    const int off = blk * k;
+    double b[16];
+    for (int c = 0; c < k; ++c) b[c] = (double)ld_any(wb.p[pj], c * wb.n[pj] + col, wb_fp32);
+    double s = 0.0;
+    for (int a = 0; a < k; ++a) {
+      double row = 0.0;
+      for (int c = 0; c < k; ++c) row = fma(gs[(off + a) * mk + off + c], b[c], row);
+      s = fma(b[a], row, s);
+    }
+    return s > 0.0 ? s : 0.0;
+  };
+  double score;
+  if (crit == 0) {
+    score = sqrt(quad(0, proj0, u));
+  } else {
+    const int g = (int)(u / head_dim), d = (int)(u % head_dim);
+    const int hpg = n_q_heads / n_kv_heads;
+    double qs = 0.0;
+    for (int h = g * hpg; h < (g + 1) * hpg; ++h) qs += sqrt(quad(0, proj0, (int64_t)h * head_dim + d));
+    score = qs * sqrt(quad(1, proj1, u));
+  }
+  scores[u] = (float)score;
+}
+
+}  // namespace
+
+int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
+               const void* const* wa, int wa_fp32, int k, float* zpart, int n_split, cudaStream_t s) {
+  const int mk = n_proj * k;
+  if (mk > 64 || n_proj > 4 || n_ctx <= 0) return 1;
+  WaPtrs w{};
+  for (int i = 0; i < n_proj; ++i) w.p[i] = wa[i];
+  int64_t dps = (d_in + n_split - 1) / n_split;
+  dps = (dps + kE1Chunk - 1) / kE1Chunk * kE1Chunk;
+  const int cpg = (mk + 7) / 8;
+  const size_t smem = (size_t)kE1Chunk * (kE1Rows + 4) * 4 + (size_t)dps * 8 * cpg * 4;
+  dim3 grid((unsigned)((n_ctx + kE1Rows - 1) / kE1Rows), (unsigned)((d_in + dps - 1) / dps));
+  if ((int)grid.y > n_split || smem > 200 * 1024) return 1;
+#define SL_E1(C)                                                                                              \
+  case C: {                                                                                                   \
+    if (x_fp32) {                                                                                             \
+      auto kern = est1_kernel<float, C>;                                                                      \
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
+      kern<<<grid, kE1Threads, smem, s>>>((const float*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, zpart);  \
+    } else {                                                                                                  \
+      auto kern = est1_kernel<__nv_bfloat16, C>;                                                              \
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
+      kern<<<grid, kE1Threads, smem, s>>>((const __nv_bfloat16*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, \
+                                          zpart);                                                             \
+    }                                                                                                         \
+    break;                                                                                                    \
+  }
+  switch (cpg) {
+    SL_E1(1) SL_E1(2) SL_E1(3) SL_E1(4) SL_E1(5) SL_E1(6) SL_E1(7) SL_E1(8)
+    default:
+      return 1;
+  }
+#undef SL_E1
+  const int used = (int)grid.y;
+  if (used > 1) {
+    const int64_t n = n_ctx * mk;
+    est_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(zpart, used, n);
+  }
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, const void* wb_gate, const void* wb_up,
+                      int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s) {
+  const unsigned grid = (unsigned)((n_ch + 63) / 64);
+  switch (k) {
+    case 8: est_swiglu_kernel<8><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 16: est_swiglu_kernel<16><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 4: est_swiglu_kernel<4><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    default: return 1;
+  }
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gram_part, int n_chunks, cudaStream_t s) {
+  if (mk > 64 || n_chunks != (int)((n_ctx + kGramTok - 1) / kGramTok)) return 1;
+  est_gram_kernel<<<n_chunks, 256, 0, s>>>(z, n_ctx, mk, gram_part);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int crit, int proj0, int proj1,
+                      const void* wb0, const void* wb1, int wb_fp32, int n_q_heads, int n_kv_heads, int head_dim,
+                      int64_t n_units, float* scores, cudaStream_t s) {
+  // crit 0 (L2): units = output channels of the projection whose Z columns start at proj0 * k; W_B = wb0.
+  // crit 2 (QK): units = KV channels; q at Z block proj0 (W_B = wb0), k at Z block proj1 (W_B = wb1).
+  if (k > 16 || mk > 64) return 1;
+  WbPtrs w{};
+  if (crit == 0) {
+    w.p[0] = wb0;
+    w.n[0] = n_units;
+  } else {
+    w.p[0] = wb0;
+    w.n[0] = (int64_t)n_q_heads * head_dim;
+    w.p[1] = wb1;
+    w.n[1] = (int64_t)n_kv_heads * head_dim;
+  }
+  const unsigned grid = (unsigned)((n_units + 255) / 256);
+  est_linear_scores_kernel<<<grid, 256, (size_t)mk * mk * sizeof(double), s>>>(
+      gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
+      crit == 0 ? 1 : head_dim, n_units, scores);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  note_launch();
+  return 0;
+}
+
+int est1_splits(int64_t d_in) {
+  int ns = (int)((d_in + 255) / 256);
+  if (ns > 64) ns = 64;
+  if (ns < 1) ns = 1;
+  int64_t dps = (d_in + ns - 1) / ns;
+  dps = (dps + 31) / 32 * 32;
+  return (int)((d_in + dps - 1) / dps);
+}
+
+}  // namespace sl

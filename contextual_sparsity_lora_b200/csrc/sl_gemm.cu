@@ -1,0 +1,512 @@
+// Persistent, warp-specialised tcgen05 GEMM engine for sm_100a (see sl_gemm.h).
+//
+// Roles per CTA (192 threads, one CTA per SM):
+//   warp 0      one thread issues TMA tile loads into a kStages-deep ring
+//   warp 1      allocates 512 TMEM columns (two 256-column fp32 accumulators);
+//               one thread issues tcgen05.mma (M = 128, N = n_mma, K = 16 each)
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread), fused elementwise work, global stores
+// Tiles are handed out round-robin over the problem list; the two accumulators
+// let the epilogue of tile i overlap the main loop of tile i+1.
+#include <cuda_bf16.h>
+
+#include "sl_gemm.h"
+#include "sl_internal.h"
+#include "sl_ptx.cuh"
+
+namespace sl {
+
+struct TileInfo {
+  int prob, tm, tn;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
+  int pi = 0;
+  for (int i = 0; i < p.nprob; ++i)
+    if (t >= p.probs[i].tile_begin) pi = i;
+  const Prob& pr = p.probs[pi];
+  const int local = t - pr.tile_begin;
+  return {pi, local % pr.tiles_m, local / pr.tiles_m};
+}
+
+__device__ __forceinline__ uint32_t seg_tx_bytes(const Seg& sg) {
+  uint32_t bytes = kStageABytes;
+  for (int i = 0; i < sg.nb; ++i) bytes += sg.b_mn ? (uint32_t)(sg.b[i].rows / 64) * 8192u : (uint32_t)sg.b[i].rows * 128u;
+  return bytes;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* dst, const float* v, int n, bool vec_ok) {
+  if (vec_ok && n == 32) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      d4[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < n) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* v, int n, bool vec_ok) {
+  if (vec_ok && n == 32) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 w = s4[i];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 f = __bfloat1622float2(h[j]);
+        v[8 * i + 2 * j] = f.x;
+        v[8 * i + 2 * j + 1] = f.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = i < n ? __bfloat162float(src[i]) : 0.f;
+  }
+}
+
+// Epilogue of one tile for one thread (one output row). All tcgen05.ld are
+// executed by every lane of the warp (they are warp-collective).
+__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb) {
+  const int row = m0 + r;
+  const bool rv = row < pr.M;
+  const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
+  float v[32];
+  uint32_t raw[32];
+
+  if (pr.epi == EPI_SWIGLU) {
+    const int ncols = min(128, pr.N - n0);
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      if (c0 >= ncols) break;
+      float g[32];
+      __syncwarp();
+      tmem_ld32(tb + c0, raw);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = __uint_as_float(raw[i]);
+      __syncwarp();
+      tmem_ld32(tb + 128 + c0, raw);
+      tmem_ld_wait();
+      if (!rv) continue;
+      const int n = min(32, ncols - c0);
+      const int64_t off = orow * pr.ld0 + n0 + c0;
+      const bool vec = ((off & 7) == 0);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);  // u
+      store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out0) + off, g, n, vec);
+      store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out1) + off, v, n, vec);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = silu_f(g[i]) * v[i];
+      store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out2) + off, v, n, vec);
+    }
+    return;
+  }
+
+  const int ncols = min(pr.tile_cols, pr.N - n0);
+  for (int c0 = 0; c0 < pr.n_mma; c0 += 32) {
+    if (c0 >= ncols) break;
+    __syncwarp();
+    tmem_ld32(tb + c0, raw);
+    tmem_ld_wait();
+    if (!rv) continue;
+    const int n = min(32, ncols - c0);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+    switch (pr.epi) {
+      case EPI_BF16: {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= pr.a0;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out0);
+        if (pr.col_map) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < n) out[orow * pr.ld0 + pr.col_map[n0 + c0 + i]] = __float2bfloat16_rn(v[i]);
+        } else {
+          const int64_t off = orow * pr.ld0 + n0 + c0;
+          store_bf16_row(out + off, v, n, (off & 7) == 0);
+        }
+        break;
+      }
+      case EPI_F32: {
+        float* out = reinterpret_cast<float*>(pr.out0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i >= n) break;
+          const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
+          float* d = out + orow * pr.ld0 + col;
+          *d = pr.a0 * v[i] + (pr.beta ? *d : 0.f);
+        }
+        break;
+      }
+      case EPI_F32_T: {
+        float* out = reinterpret_cast<float*>(pr.out0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i >= n) break;
+          const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
+          float* d = out + col * pr.ld0 + orow;
+          *d = pr.a0 * v[i] + (pr.beta ? *d : 0.f);
+        }
+        break;
+      }
+      case EPI_XA: {
+        float* o0 = reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + n0 + c0;
+        __nv_bfloat16* o1 = reinterpret_cast<__nv_bfloat16*>(pr.out1) + orow * pr.ld1 + n0 + c0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i >= n) break;
+          o0[i] = pr.a0 * v[i];
+          o1[i] = __float2bfloat16_rn(pr.a1 * v[i]);
+        }
+        break;
+      }
+      case EPI_DSWIGLU: {
+        float g[32], u[32];
+        const int64_t aoff = orow * pr.ld_aux + n0 + c0;
+        const bool vec = (aoff & 7) == 0;
+        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux0) + aoff, g, n, vec);
+        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux1) + aoff, u, n, vec);
+        float dg[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float s = 1.0f / (1.0f + __expf(-g[i]));
+          const float dh = v[i];
+          dg[i] = dh * u[i] * (s * (1.0f + g[i] * (1.0f - s)));
+          v[i] = dh * g[i] * s;  // du = dh * SiLU(g)
+        }
+        const int64_t off = orow * pr.ld0 + n0 + c0;
+        store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out0) + off, dg, n, (off & 7) == 0);
+        store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out1) + off, v, n, (off & 7) == 0);
+        break;
+      }
+      default:
+        break;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem_a = smem;
+  uint8_t* smem_b = smem + kStages * kStageABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + kStages * kStageBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_par = 0;
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(p, t);
+        const Prob& pr = p.probs[ti.prob];
+        const int n0 = ti.tn * pr.tile_cols;
+        for (int s = 0; s < pr.nseg; ++s) {
+          const Seg& sg = pr.seg[s];
+          if (n0 >= sg.n_limit) continue;
+          const uint32_t bytes = seg_tx_bytes(sg);
+          for (int kb = 0; kb < sg.nk; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            issued_mask |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            uint8_t* sa = smem_a + stage * kStageABytes;
+            uint8_t* sb = smem_b + stage * kStageBBytes;
+            const int kc = kb * kBK;
+            if (!sg.a_mn) {
+              tma_load_2d(sa, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, sg.a_row0 + ti.tm * kBM);
+            } else {
+              tma_load_2d(sa, &p.maps[sg.a_map], &full[stage], sg.a_row0 + ti.tm * kBM, sg.a_k0 + kc);
+              tma_load_2d(sa + 8192, &p.maps[sg.a_map], &full[stage], sg.a_row0 + ti.tm * kBM + 64, sg.a_k0 + kc);
+            }
+            for (int i = 0; i < sg.nb; ++i) {
+              const BSrc& b = sg.b[i];
+              const int coord = b.row0 + b.row_step * ti.tn;
+              if (!sg.b_mn) {
+                tma_load_2d(sb + b.tile_off * 128, &p.maps[b.map], &full[stage], sg.b_k0 + kc, coord);
+              } else {
+                for (int c = 0; c < b.rows / 64; ++c)
+                  tma_load_2d(sb + (b.tile_off / 64 + c) * 8192, &p.maps[b.map], &full[stage], coord + 64 * c,
+                              sg.b_k0 + kc);
+              }
+            }
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+      }
+    producer_done:
+      // Every issued copy must land before the CTA may exit.
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(p, t);
+        const Prob& pr = p.probs[ti.prob];
+        const int n0 = ti.tn * pr.tile_cols;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+        uint32_t accumulate = 0;
+        for (int s = 0; s < pr.nseg; ++s) {
+          const Seg& sg = pr.seg[s];
+          if (n0 >= sg.n_limit) continue;
+          const uint32_t idesc = idesc_bf16(kBM, pr.n_mma, sg.a_mn, sg.b_mn);
+          for (int kb = 0; kb < sg.nk; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEV_TIMEOUT_MMA)) goto mma_done;
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem_a + stage * kStageABytes);
+            const uint32_t sb = smem_u32(smem_b + stage * kStageBBytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t ad = sg.a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bd = sg.b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sb + k * 32, 16, 1024);
+              umma_bf16(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1;
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    mma_done:
+      // Wait for every issued MMA before TMEM is released.
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      const TileInfo ti = decode_tile(p, t);
+      const Prob& pr = p.probs[ti.prob];
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb);
+      __syncwarp();
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+int GemmBuilder::map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  if (status != 0) return 0;
+  if (nmaps >= kMaxMaps) {
+    status = 1;
+    return 0;
+  }
+  if (!ptr || rows <= 0 || cols <= 0 || ld < cols || (reinterpret_cast<uintptr_t>(ptr) & 15) || (ld % 8) ||
+      box_rows <= 0 || box_rows > 256) {
+    status = 2;
+    return 0;
+  }
+  auto enc = get_encode();
+  if (!enc) {
+    status = 3;
+    return 0;
+  }
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&params.maps[nmaps], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    status = 2;
+    return 0;
+  }
+  return nmaps++;
+}
+
+Prob* GemmBuilder::add(int M, int N, int tile_cols, int n_mma) {
+  if (status != 0) return nullptr;
+  if (nprob >= kMaxProbs) {
+    status = 1;
+    return nullptr;
+  }
+  Prob* pr = &params.probs[nprob++];
+  memset(pr, 0, sizeof(Prob));
+  pr->M = M;
+  pr->N = N;
+  pr->tile_cols = tile_cols;
+  pr->n_mma = n_mma;
+  pr->a0 = 1.f;
+  pr->a1 = 1.f;
+  return pr;
+}
+
+Seg* GemmBuilder::seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b_mn, int b_k0, int K, int n_limit) {
+  if (!pr || status != 0) return nullptr;
+  if (pr->nseg >= kMaxSegs) {
+    status = 1;
+    return nullptr;
+  }
+  Seg* s = &pr->seg[pr->nseg++];
+  memset(s, 0, sizeof(Seg));
+  s->a_map = (int16_t)a_map;
+  s->a_mn = (int16_t)a_mn;
+  s->a_row0 = a_row0;
+  s->a_k0 = a_k0;
+  s->b_mn = (int16_t)b_mn;
+  s->b_k0 = b_k0;
+  s->nk = (K + kBK - 1) / kBK;
+  s->n_limit = n_limit;
+  return s;
+}
+
+void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int row_step) {
+  if (!s || status != 0) return;
+  if (s->nb >= kMaxBSrc) {
+    status = 1;
+    return;
+  }
+  BSrc& b = s->b[s->nb++];
+  b.map = (int16_t)map;
+  b.tile_off = (int16_t)tile_off;
+  b.rows = (int16_t)rows;
+  b.row0 = row0;
+  b.row_step = row_step;
+}
+
+int GemmBuilder::launch(int* err, cudaStream_t stream) {
+  if (status != 0) return status;
+  int total = 0;
+  for (int i = 0; i < nprob; ++i) {
+    Prob& pr = params.probs[i];
+    // Every problem needs at least one segment active on every tile, a valid MMA
+    // shape, and segment sources inside the B tile.
+    if (pr.n_mma < 16 || pr.n_mma > kBN || pr.n_mma % 16 || pr.nseg == 0) return 4;
+    if (pr.epi == EPI_SWIGLU && (pr.tile_cols != 128 || pr.n_mma != 256)) return 4;
+    bool always = false;
+    for (int s = 0; s < pr.nseg; ++s) {
+      const Seg& sg = pr.seg[s];
+      if (sg.n_limit >= pr.N) always = true;
+      for (int b = 0; b < sg.nb; ++b) {
+        const BSrc& bs = sg.b[b];
+        if (bs.tile_off + bs.rows > kBN || bs.tile_off % 8) return 4;
+        if (sg.b_mn && (bs.rows % 64 || bs.tile_off % 64)) return 4;
+      }
+    }
+    if (!always) return 4;
+    pr.tiles_m = pr.M > 0 ? (pr.M + kBM - 1) / kBM : 0;
+    pr.tiles_n = pr.N > 0 ? (pr.N + pr.tile_cols - 1) / pr.tile_cols : 0;
+    pr.tile_begin = total;
+    total += pr.tiles_m * pr.tiles_n;
+  }
+  params.nprob = nprob;
+  params.total_tiles = total;
+  params.err = err;
+  if (total == 0) return 0;
+  static int smem_set = 0;
+  if (!smem_set) {
+    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+        cudaSuccess)
+      return 5;
+    smem_set = 1;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = total < sms ? total : sms;
+  const bool prof = profiling_on();
+  if (prof) gemm_events(stream, true);
+  gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (prof) gemm_events(stream, false);
+  note_launch();
+  return 0;
+}
+
+}  // namespace sl

@@ -1,0 +1,86 @@
+// Grouped, persistent tcgen05 GEMM engine: the description of one launch.
+//
+// One launch runs a list of problems. A problem computes an output block
+//   C[M, N] = sum over K-segments of A_seg[M, K_seg] * B_seg[N, K_seg]^T
+// with bf16 operands staged by TMA (128-byte swizzle) and fp32 accumulation in
+// TMEM, followed by a fused epilogue. Operands can be K-major (K contiguous) or
+// MN-major (M or N contiguous); a segment can be switched off for the output
+// tiles at or beyond a channel limit (the kept prefix of a channel-ordered
+// output). The B tile of a segment can be assembled from up to four sources
+// (e.g. the gate and up weights for the two halves of a paired SwiGLU tile).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+namespace sl {
+
+constexpr int kBM = 128;          // rows per tile (TMEM lanes)
+constexpr int kBN = 256;          // max accumulator columns per tile
+constexpr int kBK = 64;           // K per stage (one 128-byte swizzle atom of bf16)
+constexpr int kStages = 4;
+constexpr int kMaxMaps = 48;
+constexpr int kMaxProbs = 12;
+constexpr int kMaxSegs = 6;
+constexpr int kMaxBSrc = 4;
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kStageABytes = kBM * kBK * 2;
+constexpr int kStageBBytes = kBN * kBK * 2;
+constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 256;
+
+enum Epi : int32_t {
+  EPI_BF16 = 0,     // out0 bf16 = a0 * acc
+  EPI_F32 = 1,      // out0 fp32 = a0 * acc (+ out0 when beta)
+  EPI_XA = 2,       // out0 fp32 = a0 * acc, out1 bf16 = a1 * acc
+  EPI_SWIGLU = 3,   // paired tile: g = acc[:, 0:128], u = acc[:, 128:256]; out0 g, out1 u, out2 h = SiLU(g) u
+  EPI_DSWIGLU = 4,  // dh = acc; reads g (aux0), u (aux1); out0 dg = dh u SiLU'(g), out1 du = dh SiLU(g)
+  EPI_F32_T = 5,    // out0[col, row] fp32 = a0 * acc (+ old when beta): transposed store
+};
+
+struct BSrc {
+  int16_t map;       // tensor map index
+  int16_t tile_off;  // first row of the B tile (K-major) / first N column (MN-major) this source fills
+  int16_t rows;      // rows (K-major, = box height) / N columns (MN-major, multiple of 64) it fills
+  int16_t pad_;
+  int32_t row0;      // coordinate of that first row / column for output tile 0
+  int32_t row_step;  // coordinate advance per output tile along N
+};
+
+struct Seg {
+  int16_t a_map, a_mn;  // A tensor map, 1 = MN-major
+  int16_t b_mn, nb;     // B majorness, number of B sources
+  int32_t a_row0;       // A coordinate along M of the problem's first row
+  int32_t a_k0, b_k0;   // K coordinate offsets
+  int32_t nk;           // number of kBK blocks
+  int32_t n_limit;      // segment runs only for tiles whose first output column < n_limit
+  BSrc b[kMaxBSrc];
+};
+
+struct Prob {
+  int32_t M, N;         // output rows, output columns (channels)
+  int32_t tile_cols;    // output columns per tile: 256 (plain) or 128 (paired SwiGLU)
+  int32_t n_mma;        // accumulator columns produced by the MMA (<= 256, multiple of 16)
+  int32_t tiles_m, tiles_n, tile_begin;
+  int32_t nseg;
+  Seg seg[kMaxSegs];
+  int32_t epi, beta;
+  int32_t out_row0;     // first output row
+  int32_t pad_;
+  int64_t ld0, ld1, ld2, ld_aux;
+  void* out0;
+  void* out1;
+  void* out2;
+  const void* aux0;
+  const void* aux1;
+  const int32_t* col_map;  // optional: output column j -> col_map[j]
+  const int32_t* row_map;  // optional: output row i (problem-local) -> row_map[i]
+  float a0, a1;
+};
+
+struct GemmParams {
+  CUtensorMap maps[kMaxMaps];
+  Prob probs[kMaxProbs];
+  int32_t nprob, total_tiles;
+  int* err;
+};
+
+}  // namespace sl

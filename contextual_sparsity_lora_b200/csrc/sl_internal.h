@@ -1,0 +1,63 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "sl_gemm.h"
+
+namespace sl {
+
+// Launch accounting for the optional profiling hook (sl_profile_enable / sl_profile_read).
+void note_launch(int n = 1);
+bool profiling_on();
+void gemm_events(cudaStream_t s, bool start);
+
+// Builds the parameter block of one grouped GEMM launch on the host.
+struct GemmBuilder {
+  GemmParams params;
+  int nmaps = 0;
+  int nprob = 0;
+  int status = 0;  // 0 ok, 1 too many maps/problems/segments, 2 bad tensor, 3 no driver entry, 4 bad problem, 5 launch
+
+  GemmBuilder() { memset(&params, 0, sizeof(params)); }
+  // bf16 row-major matrix [rows, cols] with leading dimension ld (elements);
+  // the TMA box is 64 columns x box_rows rows, 128-byte swizzled, zero fill.
+  int map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows);
+  Prob* add(int M, int N, int tile_cols, int n_mma);
+  // K is the segment's K extent; n_limit = output column limit (use N or more for "always").
+  Seg* seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b_mn, int b_k0, int K, int n_limit);
+  void bsrc(Seg* s, int map, int tile_off, int rows, int row0, int row_step);
+  int launch(int* err, cudaStream_t stream);
+};
+
+// ---- estimator (sl_estimator.cu)
+int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
+               const void* const* wa, int wa_fp32, int k, float* zpart, int n_split, cudaStream_t s);
+int est_swiglu_scores(const float* zpart, int n_split, int64_t n_ctx, int k, const void* wb_gate,
+                      const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s);
+int est_gram(const float* zpart, int n_split, int64_t n_ctx, int mk, double* gram_part, int n_chunks,
+             cudaStream_t s);
+int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int crit, int proj0, int proj1,
+                      const void* wb0, const void* wb1, int wb_fp32, int n_q_heads, int n_kv_heads, int head_dim,
+                      int64_t n_units, float* scores, cudaStream_t s);
+int est1_splits(int64_t d_in);
+constexpr int kGramChunk = 128;
+
+// ---- selection (sl_select.cu)
+int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group,
+                    int head_dim, int64_t n_wide, int32_t* sigma_wide, int64_t* n_keep_wide_out, cudaStream_t s);
+
+// ---- helpers (sl_aux.cu)
+int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols,
+                     void* dst, int64_t ld_dst, int64_t dst_col0, cudaStream_t s, int blk = 0, int blk_stride = 0,
+                     int blk_off = 0);
+int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                     void* dst, int64_t ld_dst, cudaStream_t s);
+int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,
+                   cudaStream_t s);
+int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
+                      void* dst, int64_t ld_dst, cudaStream_t s);
+int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s);
+
+}  // namespace sl

@@ -1,0 +1,236 @@
+/*
+ * sparselora.h - C ABI of libsparselora.so, a B200 (sm_100a) implementation of the
+ * hot path of SparseLoRA: the contextually sparse frozen-main-branch linear layer of
+ * a LoRA fine-tuning step.
+ *
+ * Sources (cited by page title and section):
+ *   [WT] "SparseLoRA: Accelerating LLM Fine-Tuning with Contextual Sparsity",
+ *        paper-graph-ui walkthrough: section 3.2 "Big-Picture Architecture" and
+ *        section 3.4 parts "Oracle Sparse Neuron Selection Criteria", "SVD
+ *        Sparsity Estimator" (Algorithm 1), "Token Sensitivity and
+ *        Context-Output Aware Sparsity" (Figure 8), "Putting It All Together".
+ *   [PN] zhaoyang97 Paper-Notes page on SparseLoRA, section 方法详解
+ *        (selection criteria, SVD sparsity estimator).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are CUDA device pointers owned by the caller. The library
+ *   never allocates device memory, never synchronises the stream and keeps no
+ *   global state besides lazily set kernel attributes. Scratch memory comes from
+ *   the caller's sl_workspace.
+ * - Matrices are row-major with an explicit leading dimension in elements.
+ *   Frozen weights use nn.Linear storage order W[d_out, d_in] (the pages' math
+ *   convention is y = x W_math with W_math = W^T). LoRA: A[r, d_in], B[d_out, r],
+ *   y += scale * (x A^T) B^T.
+ * - Token rows are in context-first order: rows [0, n_ctx) are context tokens and
+ *   rows [n_ctx, n_tok) are output (loss-target) tokens. Linear layers act on rows
+ *   independently, so this is the pages' in-place context/output split (Figure 8)
+ *   after one permutation of the batch (sl_permute_rows).
+ * - A channel set for one projection is a permutation sigma of [0, n_side):
+ *   sigma[0, n_keep) are the kept channels in ascending order, sigma[n_keep,
+ *   n_side) the dropped ones in ascending order (sl_select_channels writes it).
+ * - "sigma layout" of an activation with n_side columns: its context rows store
+ *   channel sigma[p] in column p (kept channels first); its output rows store
+ *   channel c in column c. The SwiGLU path writes g, u, h (and the backward dg,
+ *   du) in this layout so every GEMM operand of the sparse path is contiguous.
+ * - bf16 for activations, frozen weights, estimator factors and LoRA parameters;
+ *   fp32 for scores, x A^T, dy B and LoRA gradients; int32 for channel indices.
+ * - Alignment: every bf16 matrix consumed by a tensor-core GEMM needs a 16-byte
+ *   aligned base and a leading dimension that is a multiple of 8 elements.
+ * - Errors: arguments are checked on the host before any launch and reported as a
+ *   status; nothing is launched on an error. Launch failures give SL_ERR_CUDA. All
+ *   device-side waits are bounded; a wait that runs out writes a non-zero code
+ *   into the workspace's error word (read it with sl_read_device_flag).
+ */
+#ifndef SPARSELORA_H_
+#define SPARSELORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SL_API __attribute__((visibility("default")))
+#else
+#define SL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sl_stream; /* cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  SL_OK = 0,
+  SL_ERR_INVALID_ARG = 1, /* null pointer, bad enum, inconsistent counts */
+  SL_ERR_SHAPE = 2,       /* sizes out of the supported range */
+  SL_ERR_ALIGNMENT = 3,   /* base address or leading dimension not aligned for TMA */
+  SL_ERR_WORKSPACE = 4,   /* workspace missing or too small; ws->needed holds the size */
+  SL_ERR_UNSUPPORTED = 5, /* a valid request this build does not implement */
+  SL_ERR_CUDA = 6,        /* a CUDA launch or driver call failed */
+  SL_ERR_DEVICE_FLAG = 7  /* a kernel reported a device-side timeout */
+} sl_status;
+
+typedef enum {
+  SL_CRIT_L2 = 0,        /* s_i = ||Y_hat[:, i]||_2                 ([WT] VO criterion, [PN] L2 Norm) */
+  SL_CRIT_SWIGLU_L2 = 1, /* s_i = ||SiLU(G_hat) * U_hat [:, i]||_2  ([WT] FFN criterion)            */
+  SL_CRIT_QK = 2         /* s = ||Q_hat||_2 * ||K_hat||_2            ([WT] QK norm, [PN] QK Norm)    */
+} sl_criterion;
+
+typedef enum { SL_DT_BF16 = 0, SL_DT_F32 = 1 } sl_dtype;
+typedef enum { SL_SLICE_OUT = 0, SL_SLICE_IN = 1 } sl_slice;
+typedef enum { SL_LAYOUT_NATURAL = 0, SL_LAYOUT_SIGMA = 1 } sl_layout;
+typedef enum { SL_EPI_NONE = 0, SL_EPI_SWIGLU = 1 } sl_epilogue;
+typedef enum { SL_LORA_FWD = 0, SL_LORA_BWD = 1 } sl_lora_mode;
+
+/* Caller-owned scratch memory. When ptr is NULL or bytes < the size a call needs, the
+ * call stores the size in `needed` and returns SL_ERR_WORKSPACE without launching.
+ * The first 256 bytes hold the device error word; zero them once with
+ * sl_workspace_init before first use. Calls that share a workspace must be ordered
+ * on one stream. */
+typedef struct {
+  void* ptr;
+  size_t bytes;
+  size_t needed;
+} sl_workspace;
+
+/* One frozen projection with its LoRA adapter. */
+typedef struct {
+  const void* w;      /* bf16 [d_out, d_in], frozen */
+  const void* w_t;    /* bf16 [d_in, d_out] = w^T (sl_prepare_weight); required for SL_SLICE_IN */
+  int64_t d_in, d_out;
+  int32_t slice;      /* sl_slice: which side the channel set indexes */
+  int32_t r;          /* LoRA rank, multiple of 8, <= 64 */
+  const void* lora_a; /* bf16 [r, d_in] */
+  const void* lora_b; /* bf16 [d_out, r] */
+  float lora_scale;   /* alpha / r */
+  int32_t pad_;
+} sl_linear;
+
+/* The channel set applied to one projection's sliced side. */
+typedef struct {
+  const int32_t* sigma; /* [n_side] kept (ascending) then dropped (ascending) */
+  int64_t n_side;       /* d_out for SL_SLICE_OUT, d_in for SL_SLICE_IN */
+  int64_t n_keep;       /* 1 <= n_keep <= n_side */
+} sl_channels;
+
+SL_API const char* sl_status_string(sl_status s);
+SL_API int32_t sl_version(void);
+
+/* n_keep = ceil(ratio * n) with a 1e-9 guard against binary rounding, clamped to
+ * [1, n] ([WT] Algorithm 1: the top ceil(r * D_out) channels). Host only. */
+SL_API int64_t sl_keep_count(double ratio, int64_t n);
+
+/* Zero the workspace error word (asynchronous memset on `stream`). */
+SL_API sl_status sl_workspace_init(sl_workspace* ws, sl_stream stream);
+/* Copy the error word to the host (synchronises `stream`). *code = 0: no error. */
+SL_API sl_status sl_read_device_flag(const sl_workspace* ws, int32_t* code, sl_stream stream);
+
+/* a1 + a2: SVD sparsity estimator and criterion ([WT] "SVD Sparsity Estimator",
+ * Algorithm 1, and the criteria of "Oracle Sparse Neuron Selection Criteria";
+ * [PN] SVD 稀疏估计器).
+ *   x: [n_ctx, d_in] (ld ldx), the context rows of the layer input, dtype `dtype`.
+ *   w_a[j]: [d_in, k], w_b[j]: [k, d_out[j]] - offline rank-k factors of projection j
+ *           (same dtype as x).
+ *   crit SL_CRIT_L2:        n_proj = 1; scores[d_out[0]] = ||x W_A W_B||_2 per column.
+ *   crit SL_CRIT_SWIGLU_L2: n_proj = 2 (gate, up); scores[d_out[0]] from SiLU(G_hat) * U_hat.
+ *   crit SL_CRIT_QK:        n_proj = 2 (q, k) or 3 (q, k, v); scores over the
+ *                           n_kv_heads * head_dim KV units (g, d): ||K_hat[:, (g,d)]|| *
+ *                           sum_{h in group g} ||Q_hat[:, (h,d)]|| (equal head counts give
+ *                           s = q * k exactly). With n_proj = 3, scores_v[d_out[2]] receives
+ *                           the L2 scores of v from the same pass over x.
+ * Sums over tokens run in a fixed order (bit-identical across runs). k <= 16,
+ * n_proj * k <= 64, d_in % 8 == 0. */
+SL_API sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in,
+                          int64_t ldx, int32_t n_proj, const void* const* w_a, const void* const* w_b,
+                          const int64_t* d_out, int32_t k, int32_t n_q_heads, int32_t n_kv_heads,
+                          int32_t head_dim, float* scores, float* scores_v, sl_workspace* ws,
+                          sl_stream stream);
+
+/* a3: top-n selection ([WT] Algorithm 1; [PN] top-n). Keeps exactly n_keep of the n
+ * scores: larger score first, ties to the lower index, NaN below every number.
+ * Writes sigma[n] (kept ascending, then dropped ascending). When heads_per_group > 0
+ * the n scores are KV units (g, d) with d < head_dim, and sigma_wide[n *
+ * heads_per_group] receives the matching query-side set: channel (h, d) is kept iff
+ * unit (h / heads_per_group, d) is (the kept count is n_keep * heads_per_group).
+ * n <= 40960. */
+SL_API sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma,
+                             int32_t heads_per_group, int32_t head_dim, int32_t* sigma_wide, sl_stream stream);
+
+/* a6: the dense LoRA branch ([WT] Algorithm 1 "computed densely and added"; section 3.2:
+ * LoRA gradients are always dense).
+ * SL_LORA_FWD: for n_ad adapters sharing the input x [n_tok, d_in] (ld ldx), with
+ *   R = sum r_i and equal scales:  xa[n_tok, R] (fp32, ld ld_xa) = x A_i^T per block,
+ *   xa_s[n_tok, R] (bf16, ld ld_xa) = scale * xa (the operand the sparse GEMMs fuse).
+ *   in_layout SL_LAYOUT_SIGMA: x's context rows are in the sigma layout of in_ch.
+ * SL_LORA_BWD: for each adapter i with output gradient dy[i] [n_tok, d_out_i] (ld ld_dy[i]):
+ *   dya[i] (fp32 [n_tok, r_i], ld r_i) = scale * dy B;  dya_s[i] (bf16, same) = dya;
+ *   dB[i] (fp32 [d_out_i, r_i]) = scale * dy^T xa = dy^T xa_s;
+ *   dA[i] (fp32 [r_i, d_in]) = dya^T x.
+ *   xa_s is the forward's bf16 block for adapter i (ld ld_xa, column offset = sum of
+ *   earlier r). out_layout SL_LAYOUT_SIGMA: dy's context rows are in the sigma layout
+ *   of out_ch[i]; in_layout SL_LAYOUT_SIGMA: x's context rows are in the sigma layout
+ *   of in_ch. */
+SL_API sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx,
+                          int64_t n_tok, int64_t n_ctx, int32_t in_layout, const sl_channels* in_ch, float* xa,
+                          void* xa_s, int64_t ld_xa, const void* const* dy, const int64_t* ld_dy,
+                          int32_t out_layout, const sl_channels* out_ch, float* const* dya, void* const* dya_s,
+                          float* const* dA, float* const* dB, sl_workspace* ws, sl_stream stream);
+
+/* a4: sparse frozen branch forward plus the fused LoRA add ([WT] Algorithm 1, Figure 8;
+ * "Preliminary: what channel sparsity means structurally").
+ * Context rows go through the weight sliced to the kept channels; output rows through
+ * the dense weight; every row adds scale * xa B^T (xa_s from sl_lora_fwd_bwd).
+ *   SL_SLICE_OUT, epi SL_EPI_NONE: n_lin projections sharing x; y[i] [n_tok, d_out_i]:
+ *     kept channels = main + LoRA, dropped context channels = LoRA only. out_layout
+ *     NATURAL scatters to the natural columns; SIGMA writes the sigma layout.
+ *   SL_SLICE_OUT, epi SL_EPI_SWIGLU: n_lin = 2 (gate, up) with one channel set; writes
+ *     y[0] = g, y[1] = u, y[2] = h = SiLU(g) * u, all [n_tok, d_out] in the sigma layout.
+ *   SL_SLICE_IN: n_lin = 1 (down, o). The kept input channels of x's context rows feed
+ *     w_t[kept] (w_t required); x's context rows are in the sigma layout (in_layout
+ *     SIGMA, e.g. h from the SwiGLU path) or natural (gathered into the workspace).
+ *     y[0] [n_tok, d_out] natural.
+ * xa_s: bf16 [n_tok, sum r] (ld ld_xa), the adapters' blocks in the order of lin.
+ * Never forms a frozen-weight gradient. */
+SL_API sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_channels* ch, int32_t epi,
+                               const void* x, int64_t ldx, int64_t n_tok, int64_t n_ctx, int32_t in_layout,
+                               int32_t out_layout, const void* xa_s, int64_t ld_xa, void* const* y,
+                               const int64_t* ldy, sl_workspace* ws, sl_stream stream);
+
+/* a5: input-gradient backward through the same slicing, plus the fused LoRA term
+ * scale * (dy B) A ([WT] section 3.2 backward pass, "Putting It All Together": no
+ * frozen-weight gradient).
+ *   SL_SLICE_OUT: n_lin projections whose input gradients sum into dx [n_tok, d_in]
+ *     (ld lddx); dy[i] [n_tok, d_out_i] in in_layout (SIGMA: context rows in the sigma
+ *     layout of ch[i]; NATURAL: kept columns gathered into the workspace).
+ *   SL_SLICE_IN: n_lin = 1; dy [n_tok, d_out] natural; dx [n_tok, d_in] written in
+ *     out_layout (NATURAL scatters kept channels, dropped context channels carry only
+ *     the LoRA term). epi SL_EPI_SWIGLU fuses the SwiGLU backward: with g = aux[0],
+ *     u = aux[1] (sigma layout, from the forward) it writes aux_out[0] = dg = dh u
+ *     SiLU'(g) and aux_out[1] = du = dh SiLU(g) instead of dx (out_layout SIGMA).
+ * dya_s[i]: bf16 [n_tok, r_i] (ld r_i) from sl_lora_fwd_bwd(BWD). */
+SL_API sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_channels* ch, int32_t epi,
+                               const void* const* dy, const int64_t* ld_dy, int64_t n_tok, int64_t n_ctx,
+                               int32_t in_layout, int32_t out_layout, const void* const* dya_s, void* dx,
+                               int64_t lddx, const void* const* aux, void* const* aux_out, sl_workspace* ws,
+                               sl_stream stream);
+
+/* Optional measurement of the library's own kernels (host-side counters, off by default).
+ * While enabled, every kernel the library launches is counted, and every launch of the
+ * grouped tensor-core GEMM engine is bracketed by CUDA events on its stream.
+ * sl_profile_read waits for those events, returns the totals since the last read (or
+ * since enabling) and resets them. Not thread-safe across concurrent callers. */
+SL_API sl_status sl_profile_enable(int32_t on);
+SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launches, double* gemm_ms);
+
+/* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
+SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream);
+
+/* dst[i, :] = src[perm[i], :] for bf16 rows (context-first reordering of a batch). */
+SL_API sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
+                          void* dst, int64_t ld_dst, sl_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSELORA_H_ */

@@ -1,0 +1,269 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on seeded inputs.
+
+Sizes span several 128-row / 256-column tiles and end in ragged tails. Tolerances:
+relative Frobenius error <= 1e-5 for fp32 quantities computed from exact inputs
+(estimator scores), <= 2e-2 for values that pass through bf16 tensor-core GEMMs;
+channel indices bit-exact when both sides select from the same fp32 scores.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from contextual_sparsity_lora_b200 import binding as B
+from contextual_sparsity_lora_b200 import inputs
+from gpu_helpers import BF16_TOL, FP32_TOL, attn_problem, ffn_problem, rel_fro, unsigma
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def cu(t, dtype=torch.bfloat16):
+    return t.to(device=DEV, dtype=dtype).contiguous()
+
+
+def sigma_from(idx, n):
+    idx = np.asarray(idx, dtype=np.int64)
+    return torch.tensor(np.concatenate([idx, oracle.complement(idx, n)]), dtype=torch.int32, device=DEV)
+
+
+def rand_idx(n, n_keep, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(n, n_keep, replace=False))
+
+
+# ------------------------------------------------------------------------------------------ LoRA
+
+@pytest.mark.parametrize("T,n_ctx,D,rs", [(424, 300, 512, (32,)), (424, 300, 512, (32, 32, 32)),
+                                           (130, 0, 264, (8, 16))])
+def test_lora_fwd_xa(T, n_ctx, D, rs):
+    gen = inputs.generator(1)
+    x = inputs.activations_student_t(T, D, 4, 0.01, 30.0, gen)
+    As = [inputs.lora_pair(64, D, r, 0.02, gen) for r in rs]
+    ws = B.Workspace()
+    R = sum(rs)
+    xa = torch.empty(T, R, device=DEV)
+    xa_s = torch.empty(T, R, device=DEV, dtype=torch.bfloat16)
+    w0 = cu(torch.zeros(64, D))
+    dev_ab = [(cu(a), cu(b)) for a, b in As]   # device copies stay alive for the call
+    lins = [B.linear_desc(w0, a, b, 2.0, B.SL_SLICE_OUT) for a, b in dev_ab]
+    xg = cu(x)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, lins, xg, n_ctx, xa_s, xa=xa)
+    want = oracle.f64(x) @ np.concatenate([oracle.f64(a) for a, b in As], 0).T
+    assert rel_fro(xa, want) < FP32_TOL
+    assert rel_fro(xa_s, 2.0 * want) < BF16_TOL
+
+
+def test_lora_bwd_natural_and_sigma():
+    T, C, D, Do, r = 424, 300, 512, 1000, 32
+    gen = inputs.generator(2)
+    x = inputs.activations_student_t(T, D, 4, 0.01, 30.0, gen)
+    A, Bm = inputs.lora_pair(Do, D, r, 0.02, gen)
+    dy = torch.randn(T, Do, generator=gen).to(torch.bfloat16)
+    s = 2.0
+    xg, Ag, Bg, dyg = cu(x), cu(A), cu(Bm), cu(dy)
+    ws = B.Workspace()
+    lin = B.linear_desc(cu(torch.zeros(Do, D)), Ag, Bg, s, B.SL_SLICE_OUT)
+    xa = torch.empty(T, r, device=DEV)
+    xa_s = torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lin], xg, C, xa_s, xa=xa)
+    X, dY, A64, B64 = (oracle.f64(t) for t in (x, dy, A, Bm))
+    # natural layout
+    dya, dya_s = torch.empty(T, r, device=DEV), torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    dA, dB = torch.empty(r, D, device=DEV), torch.empty(Do, r, device=DEV)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lin], xg, C, xa_s, dy=[dyg], dya=[dya], dya_s=[dya_s], dA=[dA], dB=[dB])
+    assert rel_fro(dya, s * dY @ B64) < FP32_TOL * 10
+    assert rel_fro(dB, s * dY.T @ (X @ A64.T)) < BF16_TOL
+    assert rel_fro(dA, (s * dY @ B64).T @ X) < BF16_TOL
+    # sigma layout on the output side: dy's context rows permuted by sigma
+    idx = rand_idx(Do, 437, 3)
+    sig = sigma_from(idx, Do)
+    dy_sig = dy.clone()
+    dy_sig[:C] = dy[:C][:, sig.cpu().long()]
+    ch = B.channels_desc(sig, 437)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lin], xg, C, xa_s, dy=[cu(dy_sig)], out_layout=B.SL_LAYOUT_SIGMA,
+                      out_ch=[ch], dya=[dya], dya_s=[dya_s], dA=[dA], dB=[dB])
+    assert rel_fro(dya, s * dY @ B64) < FP32_TOL * 10
+    assert rel_fro(dB, s * dY.T @ (X @ A64.T)) < BF16_TOL
+    assert rel_fro(dA, (s * dY @ B64).T @ X) < BF16_TOL
+
+
+# ------------------------------------------------------------------------------------------ sparse linear
+
+@pytest.mark.parametrize("layout", [B.SL_LAYOUT_NATURAL, B.SL_LAYOUT_SIGMA])
+@pytest.mark.parametrize("zero_b", [False, True])
+def test_sparse_linear_out_slice_fwd_bwd(layout, zero_b):
+    T, C, D, Do, r, nk = 424, 300, 512, 1000, 32, 437
+    gen = inputs.generator(4)
+    w = inputs.spectral_weight(Do, D, 0.5, 8, gen, "cpu", torch.float64, torch.bfloat16)
+    A, Bm = inputs.lora_pair(Do, D, r, 0.02, gen)
+    if zero_b:
+        Bm = torch.zeros_like(Bm)
+    x = inputs.activations_student_t(T, D, 4, 0.01, 30.0, gen)
+    dy = torch.randn(T, Do, generator=gen).to(torch.bfloat16)
+    s, ctx = 2.0, np.arange(T) < C
+    idx = rand_idx(Do, nk, 5)
+    sig = sigma_from(idx, Do)
+    ws = B.Workspace()
+    Wg, Ag, Bg, xg = cu(w.W), cu(A), cu(Bm), cu(x)
+    lin = B.linear_desc(Wg, Ag, Bg, s, B.SL_SLICE_OUT)
+    ch = B.channels_desc(sig, nk)
+    xa, xa_s = torch.empty(T, r, device=DEV), torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lin], xg, C, xa_s, xa=xa)
+    y = torch.full((T, Do), float("nan"), device=DEV, dtype=torch.bfloat16)
+    B.sl_sparse_linear_fwd(ws, [lin], [ch], B.SL_EPI_NONE, xg, C, xa_s, [y], out_layout=layout)
+    want = oracle.sparse_linear_fwd(x, w.W, A, Bm, s, ctx, idx, "out")
+    got = oracle.f64(y) if layout == B.SL_LAYOUT_NATURAL else unsigma(y, sig, C)
+    assert np.isfinite(got).all()
+    assert rel_fro(got, want) < BF16_TOL
+    # backward: dy given in the same layout
+    dy_in = dy.clone()
+    if layout == B.SL_LAYOUT_SIGMA:
+        dy_in[:C] = dy[:C][:, sig.cpu().long()]
+    dya, dya_s = torch.empty(T, r, device=DEV), torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    dA, dB = torch.empty(r, D, device=DEV), torch.empty(Do, r, device=DEV)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lin], xg, C, xa_s, dy=[cu(dy_in)], out_layout=layout, out_ch=[ch],
+                      dya=[dya], dya_s=[dya_s], dA=[dA], dB=[dB])
+    dx = torch.full((T, D), float("nan"), device=DEV, dtype=torch.bfloat16)
+    B.sl_sparse_linear_bwd(ws, [lin], [ch], B.SL_EPI_NONE, [cu(dy_in)], C, [dya_s], dx=dx, in_layout=layout)
+    dX, dA_w, dB_w = oracle.sparse_linear_bwd(x, dy, w.W, A, Bm, s, ctx, idx, "out")
+    assert rel_fro(dx, dX) < BF16_TOL
+    assert rel_fro(dA, dA_w) < BF16_TOL
+    if not zero_b:
+        assert rel_fro(dB, dB_w) < BF16_TOL
+
+
+@pytest.mark.parametrize("layout", [B.SL_LAYOUT_NATURAL, B.SL_LAYOUT_SIGMA])
+def test_sparse_linear_in_slice_fwd_bwd(layout):
+    T, C, Di, Do, r, nk = 424, 300, 1000, 512, 32, 437
+    gen = inputs.generator(6)
+    w = inputs.spectral_weight(Do, Di, 0.5, 8, gen, "cpu", torch.float64, torch.bfloat16)
+    A, Bm = inputs.lora_pair(Do, Di, r, 0.02, gen)
+    x = inputs.activations_student_t(T, Di, 4, 0.01, 30.0, gen)
+    dy = torch.randn(T, Do, generator=gen).to(torch.bfloat16)
+    s, ctx = 2.0, np.arange(T) < C
+    idx = rand_idx(Di, nk, 7)
+    sig = sigma_from(idx, Di)
+    ws = B.Workspace()
+    Wg, Ag, Bg = cu(w.W), cu(A), cu(Bm)
+    Wt = torch.empty(Di, Do, device=DEV, dtype=torch.bfloat16)
+    B.sl_prepare_weight(Wg, Wt)
+    assert torch.equal(Wt, Wg.t())
+    lin = B.linear_desc(Wg, Ag, Bg, s, B.SL_SLICE_IN, w_t=Wt)
+    ch = B.channels_desc(sig, nk)
+    x_in = x.clone()
+    if layout == B.SL_LAYOUT_SIGMA:
+        x_in[:C] = x[:C][:, sig.cpu().long()]
+    xg = cu(x_in)
+    xa, xa_s = torch.empty(T, r, device=DEV), torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lin], xg, C, xa_s, xa=xa, in_layout=layout, in_ch=ch)
+    assert rel_fro(xa, oracle.f64(x) @ oracle.f64(A).T) < FP32_TOL
+    y = torch.full((T, Do), float("nan"), device=DEV, dtype=torch.bfloat16)
+    B.sl_sparse_linear_fwd(ws, [lin], [ch], B.SL_EPI_NONE, xg, C, xa_s, [y], in_layout=layout)
+    assert rel_fro(y, oracle.sparse_linear_fwd(x, w.W, A, Bm, s, ctx, idx, "in")) < BF16_TOL
+    dyg = cu(dy)
+    dya, dya_s = torch.empty(T, r, device=DEV), torch.empty(T, r, device=DEV, dtype=torch.bfloat16)
+    dA, dB = torch.empty(r, Di, device=DEV), torch.empty(Do, r, device=DEV)
+    B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lin], xg, C, xa_s, in_layout=layout, in_ch=ch, dy=[dyg], dya=[dya],
+                      dya_s=[dya_s], dA=[dA], dB=[dB])
+    dx = torch.full((T, Di), float("nan"), device=DEV, dtype=torch.bfloat16)
+    B.sl_sparse_linear_bwd(ws, [lin], [ch], B.SL_EPI_NONE, [dyg], C, [dya_s], dx=dx, out_layout=layout)
+    dX, dA_w, dB_w = oracle.sparse_linear_bwd(x, dy, w.W, A, Bm, s, ctx, idx, "in")
+    got = oracle.f64(dx) if layout == B.SL_LAYOUT_NATURAL else unsigma(dx, sig, C)
+    assert rel_fro(got, dX) < BF16_TOL
+    assert rel_fro(dA, dA_w) < BF16_TOL
+    assert rel_fro(dB, dB_w) < BF16_TOL
+
+
+# ------------------------------------------------------------------------------------------ estimator / select
+
+def test_estimator_swiglu_scores_and_select():
+    T, C, D, F, k = 424, 300, 512, 1000, 8
+    p = ffn_problem(T, C, D, F, 32, k, seed=8)
+    ws = B.Workspace()
+    xg = cu(p["x"])
+    scores = torch.empty(F, device=DEV)
+    B.sl_svd_estimate(ws, B.SL_CRIT_SWIGLU_L2, xg[:C], C, [cu(p["gate"].W_A), cu(p["up"].W_A)],
+                      [cu(p["gate"].W_B), cu(p["up"].W_B)], k, scores)
+    s_w, idx_w = oracle.ffn_select(p["x"], p["ctx"], (p["gate"].W_A, p["gate"].W_B), (p["up"].W_A, p["up"].W_B), 0.5)
+    assert rel_fro(scores, s_w) < FP32_TOL
+    nk = oracle.keep_count(0.5, F)
+    sig = torch.empty(F, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(scores, nk, sig)
+    got = sig.cpu().numpy()
+    sc = scores.cpu().numpy().astype(np.float64)
+    want = oracle.select_top(sc, nk)
+    np.testing.assert_array_equal(got[:nk], want)
+    np.testing.assert_array_equal(got[nk:], oracle.complement(want, F))
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 4)])
+def test_estimator_qk_and_v_scores(hq, hkv):
+    T, C, D, hd, k = 424, 300, 512, 64, 8
+    p = attn_problem(T, C, D, hq, hkv, hd, 32, k, seed=9)
+    ws = B.Workspace()
+    xg = cu(p["x"])
+    nu = hkv * hd
+    s_qk, s_v = torch.empty(nu, device=DEV), torch.empty(nu, device=DEV)
+    w = p["w"]
+    B.sl_svd_estimate(ws, B.SL_CRIT_QK, xg[:C], C, [cu(w[n].W_A) for n in "qkv"], [cu(w[n].W_B) for n in "qkv"], k,
+                      s_qk, scores_v=s_v, n_q_heads=hq, n_kv_heads=hkv, head_dim=hd)
+    want = oracle.attn_select(p["x"], p["ctx"], (w["q"].W_A, w["q"].W_B), (w["k"].W_A, w["k"].W_B),
+                              (w["v"].W_A, w["v"].W_B), hq, hkv, hd, 0.5)
+    assert rel_fro(s_qk, want["s_qk"]) < FP32_TOL
+    assert rel_fro(s_v, want["s_v"]) < FP32_TOL
+    nk = oracle.keep_count(0.5, nu)
+    sk, sq = torch.empty(nu, dtype=torch.int32, device=DEV), torch.empty(hq * hd, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(s_qk, nk, sk, hq // hkv, hd, sq)
+    units = oracle.select_top(s_qk.cpu().numpy().astype(np.float64), nk)
+    np.testing.assert_array_equal(sk.cpu().numpy()[:nk], units)
+    qi = oracle.expand_units(units, hq, hkv, hd)
+    np.testing.assert_array_equal(sq.cpu().numpy()[: len(qi)], qi)
+    np.testing.assert_array_equal(sq.cpu().numpy()[len(qi):], oracle.complement(qi, hq * hd))
+
+
+def test_estimator_l2_fp32_inputs():
+    """The tiny fp32 configuration's estimator path (fp32 x and factors)."""
+    T, C, D, Do, k = 128, 96, 256, 688, 8
+    gen = inputs.generator(10)
+    w = inputs.spectral_weight(Do, D, 0.7, k, gen, "cpu", torch.float64, torch.float32)
+    x = inputs.activations_gaussian_outliers(T, D, 4, 20.0, gen)
+    ws = B.Workspace()
+    s = torch.empty(Do, device=DEV)
+    B.sl_svd_estimate(ws, B.SL_CRIT_L2, cu(x, torch.float32)[:C], C, [cu(w.W_A, torch.float32)],
+                      [cu(w.W_B, torch.float32)], k, s)
+    want = oracle.score_l2(oracle.estimate(oracle.f64(x)[:C], w.W_A, w.W_B))
+    assert rel_fro(s, want) < FP32_TOL
+
+
+@pytest.mark.parametrize("n,n_keep", [(1, 1), (7, 3), (1000, 1), (1000, 1000), (14336, 7168), (40960, 12345)])
+def test_select_edge_cases_bit_exact(n, n_keep):
+    rng = np.random.default_rng(n + n_keep)
+    s = rng.integers(0, 50, n).astype(np.float32)          # heavy ties
+    s[rng.random(n) < 0.05] = np.nan
+    s[rng.random(n) < 0.02] = -np.inf
+    s[rng.random(n) < 0.02] = -0.0
+    s[rng.random(n) < 0.02] = 0.0
+    sc = torch.tensor(s, device=DEV)
+    sig = torch.empty(n, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(sc, n_keep, sig)
+    want = oracle.select_top(s.astype(np.float64), n_keep)
+    got = sig.cpu().numpy()
+    np.testing.assert_array_equal(got[:n_keep], want)
+    np.testing.assert_array_equal(got[n_keep:], oracle.complement(want, n))
+
+
+def test_select_and_estimate_are_deterministic():
+    T, C, D, F, k = 424, 300, 512, 1000, 8
+    p = ffn_problem(T, C, D, F, 32, k, seed=11)
+    ws = B.Workspace()
+    xg = cu(p["x"])
+    outs = []
+    for _ in range(2):
+        sc = torch.empty(F, device=DEV)
+        B.sl_svd_estimate(ws, B.SL_CRIT_SWIGLU_L2, xg[:C], C, [cu(p["gate"].W_A), cu(p["up"].W_A)],
+                          [cu(p["gate"].W_B), cu(p["up"].W_B)], k, sc)
+        sig = torch.empty(F, dtype=torch.int32, device=DEV)
+        B.sl_select_channels(sc, 500, sig)
+        outs.append((sc.cpu(), sig.cpu()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
