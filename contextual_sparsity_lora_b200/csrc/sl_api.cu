@@ -428,7 +428,8 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   int R = 0;
   for (int i = 0; i < n_lin; ++i) {
     if (!linear_ok(lin[i]) || lin[i].slice != slice || lin[i].d_in != lin[0].d_in) return SL_ERR_INVALID_ARG;
-    if (!channels_ok(ch[i], slice == SL_SLICE_OUT ? lin[i].d_out : lin[i].d_in)) return SL_ERR_INVALID_ARG;
+    const sl_channels& c = epi == SL_EPI_SWIGLU ? ch[0] : ch[i];  // the paired SwiGLU call shares one set
+    if (!channels_ok(c, slice == SL_SLICE_OUT ? lin[i].d_out : lin[i].d_in)) return SL_ERR_INVALID_ARG;
     R += lin[i].r;
   }
   const int64_t d_in = lin[0].d_in;
