@@ -1,0 +1,378 @@
+"""Benchmark: SparseLoRA layer fine-tuning step (forward + backward) tokens/s at LLaMA3-8B shapes.
+
+One step = every stage of the hot path for one LLaMA3-8B decoder layer's seven
+projections over one batch of 8 x 512 tokens (last 128 of each sequence are output
+tokens): the attention projections q/k/v/o (QK criterion for q/k, L2 criterion on
+the estimated V for v/o, GQA 32/8 heads x 128) and the SwiGLU FFN gate/up/down
+(L2 criterion on the estimated SiLU(gate) * up), keep ratio 0.5, LoRA rank 32 on
+all seven, estimator rank 8. The attention core between q/k/v and o is not part of
+the path; its output and gradients are synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sparselora|reference]
+
+Multi-GPU (torchrun, one rank per GPU): each rank runs the step on its own batch
+(weak scaling, no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from contextual_sparsity_lora_b200 import flops, inputs  # noqa: E402
+
+METRIC = "sparse-LoRA layer fwd+bwd tokens/s at LLaMA3-8B shapes"
+UNIT = "tokens/s"
+WORKLOAD = "llama3-8b-layer-7proj-b8s512-keep0.5"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sparselora", choices=["sparselora", "reference"])
+    ap.add_argument("--ratio", type=float, default=0.5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-LoRA companion measurement")
+    return ap.parse_args()
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = sorted(float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit())
+        mx = max(float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for i, n in enumerate(names):
+                if s[5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+def make_layer(ratio, seed_w, seed_x, device, dense=False):
+    """The two blocks of one LLaMA3-8B layer plus their per-step inputs (context-first rows)."""
+    from contextual_sparsity_lora_b200 import blocks
+    ac = inputs.LLAMA3_8B_ATTN
+    fc = inputs.LLAMA3_8B_FFN
+    da = inputs.make_attn_inputs(ac, seed_w, device=device)
+    df = inputs.make_ffn_inputs(fc, seed_w + 1, device=device)
+    perm = inputs.context_first_order(da["ctx_mask"])
+    C = int(da["ctx_mask"].sum())
+    attn = blocks.AttnProjBlock(da["q"], da["k"], da["v"], da["o"], da["lora_q"], da["lora_k"], da["lora_v"],
+                                da["lora_o"], ac.lora_scale, ac.k, ac.n_q_heads, ac.n_kv_heads, ac.head_dim,
+                                ac.n_tok, C, ratio, device, dense=dense)
+    ffn = blocks.FFNBlock(df["gate"], df["up"], df["down"], df["lora_gate"], df["lora_up"], df["lora_down"],
+                          fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense)
+    if seed_x != seed_w:  # per-rank batches
+        dx = inputs.make_attn_inputs(ac, seed_x, device=device)
+        for key in ("x", "x_o", "dq", "dk", "dv", "dy"):
+            da[key] = dx[key]
+        df["x"], df["dy"] = dx["x"], dx["dy"]
+    step_in = {k: da[k][perm].contiguous() for k in ("x", "x_o", "dq", "dk", "dv", "dy")}
+    step_in["ffn_x"] = df["x"][perm].contiguous()
+    step_in["ffn_dy"] = df["dy"][perm].contiguous()
+    return attn, ffn, step_in, C, (ac, fc), (da, df, perm)
+
+
+def run_step(attn, ffn, s):
+    attn.step(s["x"], s["x_o"], s["dy"], s["dq"], s["dk"], s["dv"])
+    ffn.step(s["ffn_x"], s["ffn_dy"])
+
+
+def algorithmic_flops(ac, fc, C, ratio, dense):
+    T = ac.n_tok
+    nu = ac.n_kv_heads * ac.head_dim
+    nk_u = nu if dense else inputs_keep(ratio, nu)
+    nk_f = fc.inter if dense else inputs_keep(ratio, fc.inter)
+    a = flops.attn_proj_block(ac.hidden, ac.n_q_heads, ac.n_kv_heads, ac.head_dim, T, C, nk_u, nk_u, ac.r, ac.k,
+                              with_estimator=not dense)
+    f = flops.ffn_block(fc.hidden, fc.inter, T, C, nk_f, fc.r, fc.k, with_estimator=not dense)
+    return {k: a[k] + f[k] for k in a}
+
+
+def inputs_keep(ratio, n):
+    from contextual_sparsity_lora_b200 import binding as B
+    return B.sl_keep_count(ratio, n)
+
+
+def time_steps(fn, K, W, world, device):
+    for _ in range(W):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    barrier(world)
+    return max_over_ranks(ms, world, device)
+
+
+def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
+    """The fp64 oracle on the host cores over a bounded sample: the last ``n_tokens``
+    tokens of the first sequence (context and output tokens in the workload's proportion
+    when n_tokens = 512 or 128) through both blocks, estimator to LoRA gradients."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    ac, fc = inputs.LLAMA3_8B_ATTN, inputs.LLAMA3_8B_FFN
+    S = int(n_tokens)
+    sl = slice(ac.seq - S, ac.seq)                 # tail of the first sequence, sequence order
+    ctx = da["ctx_mask"][sl].cpu().numpy()
+    f64 = oracle.f64
+    X = f64(da["x"][sl]); XO = f64(da["x_o"][sl]); dq = f64(da["dq"][sl]); dk = f64(da["dk"][sl])
+    dv = f64(da["dv"][sl]); dyo = f64(da["dy"][sl]); Xf = f64(df["x"][sl]); dyf = f64(df["dy"][sl])
+    W = {n: f64(da[n].W) for n in "qkvo"}
+    F = {n: (f64(da[n].W_A), f64(da[n].W_B)) for n in "qkv"}
+    L = {n: (f64(da["lora_" + n][0]), f64(da["lora_" + n][1])) for n in "qkvo"}
+    Wf = {n: f64(df[n].W) for n in ("gate", "up", "down")}
+    Ff = {n: (f64(df[n].W_A), f64(df[n].W_B)) for n in ("gate", "up")}
+    Lf = {n: (f64(df["lora_" + n][0]), f64(df["lora_" + n][1])) for n in ("gate", "up", "down")}
+    s = ac.lora_scale
+    t0 = time.perf_counter()
+    for _ in range(n_seqs):
+        _oracle_layer(oracle, X, XO, dq, dk, dv, dyo, Xf, dyf, ctx, W, F, L, Wf, Ff, Lf, s, ac, ratio)
+    dt = time.perf_counter() - t0
+    S = S * n_seqs
+    return {"value": S / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{S} tokens ({n_seqs} x {S // n_seqs} of one sequence, {int(ctx.sum())} context + "
+                      f"{S // n_seqs - int(ctx.sum())} output each) through both blocks, fp64 NumPy, {dt:.1f} s",
+            "seconds": dt, "host_cpus": os.cpu_count()}
+
+
+def _oracle_layer(oracle, X, XO, dq, dk, dv, dyo, Xf, dyf, ctx, W, F, L, Wf, Ff, Lf, s, ac, ratio):
+    sel = oracle.attn_select(X, ctx, F["q"], F["k"], F["v"], ac.n_q_heads, ac.n_kv_heads, ac.head_dim, ratio)
+    for n, xin, kind in (("q", X, "out"), ("k", X, "out"), ("v", X, "out"), ("o", XO, "in")):
+        oracle.sparse_linear_fwd(xin, W[n], *L[n], s, ctx, sel["idx_" + n], kind)
+    for n, xin, g, kind in (("q", X, dq, "out"), ("k", X, dk, "out"), ("v", X, dv, "out"), ("o", XO, dyo, "in")):
+        oracle.sparse_linear_bwd(xin, g, W[n], *L[n], s, ctx, sel["idx_" + n], kind)
+    _, idx = oracle.ffn_select(Xf, ctx, Ff["gate"], Ff["up"], ratio)
+    fwd = oracle.ffn_fwd(Xf, ctx, Wf["gate"], Wf["up"], Wf["down"], Lf["gate"], Lf["up"], Lf["down"], s, idx)
+    oracle.ffn_bwd(Xf, dyf, ctx, Wf["gate"], Wf["up"], Wf["down"], Lf["gate"], Lf["up"], Lf["down"], s, idx, fwd=fwd)
+
+
+def e2e_measure(attn, ffn, step_in, K, W, world, device):
+    """Same step through the public API with host buffers: every step copies that step's
+    inputs from pinned host memory and reads the LoRA gradients back."""
+    host = {k: v.cpu().pin_memory() for k, v in step_in.items()}
+    dev_in = {k: torch.empty_like(v) for k, v in step_in.items()}
+    grads = [attn.dA[n] for n in "qkvo"] + [attn.dB[n] for n in "qkvo"] + \
+        [ffn.dA_g, ffn.dB_g, ffn.dA_u, ffn.dB_u, ffn.dA_d, ffn.dB_d]
+    host_out = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(g.numel() * g.element_size() for g in grads)
+
+    def step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        run_step(attn, ffn, dev_in)
+        for h, g in zip(host_out, grads):
+            h.copy_(g, non_blocking=True)
+
+    ms = time_steps(step, K, W, world, device)
+    return ms / K, h2d, d2h
+
+
+def reference_arm(args, rank, world):
+    """The oracle timed on this machine's host cores (rank 0 only) over bounded samples."""
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    ac = inputs.LLAMA3_8B_ATTN
+    da = inputs.make_attn_inputs(ac, 0, device=device)
+    df = inputs.make_ffn_inputs(inputs.LLAMA3_8B_FFN, 1, device=device)
+    n_tok = 128
+    times = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(da, df, args.ratio, n_tokens=n_tok)
+        if i >= args.warmup:
+            times.append(cb["seconds"])
+    per = sum(times) / len(times)
+    value = n_tok / per
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "seq_len": ac.seq, "sample_tokens_per_step": n_tok},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    from contextual_sparsity_lora_b200 import binding as B
+    B.lib()
+    attn, ffn, step_in, C, (ac, fc), (da, df, perm) = make_layer(args.ratio, 0, 1000 + rank, device)
+    T = ac.n_tok
+    fn = lambda: run_step(attn, ffn, step_in)
+    B.sl_profile_enable(False)
+    # timed region: clocks sampled, library kernels counted and GEMM-engine launches event-timed
+    for _ in range(max(args.warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    B.sl_profile_read()
+    B.sl_profile_enable(True)
+    with ClockSampler(local) as clk:
+        ms = time_steps(fn, args.steps, 0, world, device)
+    torch.cuda.synchronize()
+    n_launch, n_gemm, gemm_ms = B.sl_profile_read()
+    B.sl_profile_enable(False)
+    ms_step = ms / args.steps
+    value = world * T / (ms_step / 1e3)
+    fl = algorithmic_flops(ac, fc, C, args.ratio, dense=False)
+    gemm_flops = (fl["main"] + fl["lora"]) * args.steps
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 8 * world, "seq_len": ac.seq, "tokens_per_rank": T,
+                   "context_tokens_per_rank": C, "keep_ratio": args.ratio, "lora_rank": ac.r,
+                   "estimator_rank": ac.k, "parallelism": f"replicas{world}",
+                   "l2": "per-step working set ~1.4 GB > 126 MB L2; no flush"},
+        "roofline": {"bound": "tensor", "kernel": "sl::gemm_kernel (grouped tcgen05 GEMM engine)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "peak_source": f"{src} bf16_tflops_sustained",
+                     "gemm_ms_per_step": gemm_ms / args.steps, "gemm_launches_per_step": n_gemm / args.steps,
+                     "algorithmic_tflop_per_step": (fl["main"] + fl["lora"]) / 1e12},
+        "gpu_launches": n_launch,
+        "gpu_launches_per_step": n_launch / args.steps,
+        "effective_tflops": fl["total"] / (ms_step / 1e3) / 1e12,
+        "clocks": clk.summary(),
+    }
+    # dense LoRA on the same kernels (keep ratio 1, no estimator): context, not the headline
+    if not args.no_dense:
+        d_attn, d_ffn, _, _, _, _ = make_layer(1.0, 0, 1000 + rank, device, dense=True)
+        d_ms = time_steps(lambda: run_step(d_attn, d_ffn, step_in), args.steps, max(args.warmup, 3), world, device)
+        d_fl = algorithmic_flops(ac, fc, C, 1.0, dense=True)
+        line["dense_lora"] = {"value": world * T / (d_ms / args.steps / 1e3), "unit": UNIT,
+                              "ms_per_step": d_ms / args.steps,
+                              "effective_tflops": d_fl["total"] / (d_ms / args.steps / 1e3) / 1e12}
+        line["speedup_vs_dense_lora"] = line["dense_lora"]["ms_per_step"] / ms_step
+        del d_attn, d_ffn
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_measure(attn, ffn, step_in, args.steps, max(args.warmup, 3), world, device)
+        line["e2e"] = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(da, df, args.ratio, n_tokens=512, n_seqs=3).items()
+                                if k != "seconds"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
