@@ -1,5 +1,6 @@
 // C ABI of libsparselora.so (declared in include/sparselora.h): argument checks,
 // workspace carving, and the grouped tcgen05 GEMM problem lists of each stage.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -98,6 +99,19 @@ bool channels_ok(const sl_channels& c, int64_t n_side) {
   return c.sigma && c.n_side == n_side && c.n_keep >= 1 && c.n_keep <= n_side;
 }
 
+// Split-K plan of one skinny problem: partial floats needed (0 when unsplit).
+inline int64_t split_floats(int64_t M, int64_t N, int64_t K) {
+  const int S = choose_ksplit(M, (K + kBK - 1) / kBK);
+  return S > 1 ? (int64_t)S * M * N : 0;
+}
+// Marks a skinny problem for split-K, taking its partials from `region` at `*off`.
+inline void maybe_split(GemmBuilder& gb, Prob* p, int64_t M, int64_t N, int64_t K, float* region, int64_t* off) {
+  const int S = choose_ksplit(M, (K + kBK - 1) / kBK);
+  if (!p || S <= 1 || M <= 0) return;
+  gb.split(p, S, region + *off);
+  *off += (int64_t)S * M * N;
+}
+
 }  // namespace
 
 extern "C" {
@@ -175,24 +189,50 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
       return SL_ERR_INVALID_ARG;
   }
   const int mk = n_proj * k;
-  const int n_split = est1_splits(d_in);
+  // bf16 inputs: stage 1 runs on the tensor-core engine (exact bf16 products, fp32
+  // accumulation, fixed-order split-K); fp32 inputs: CUDA-core fp32 FMA kernel.
+  const bool tc = !fp32 && k % 8 == 0;
+  const int n_split = tc ? 1 : est1_splits(d_in);
   const int n_chunks = (int)((n_ctx + kGramChunk - 1) / kGramChunk);
-  auto carve = [&](Carver& c, float** zp, double** gp) {
+  const int64_t red = tc ? split_floats(n_ctx, mk, d_in) : 0;
+  auto carve = [&](Carver& c, float** zp, double** gp, void** wat, float** region) {
     *zp = c.take<float>((size_t)n_split * n_ctx * mk);
     *gp = c.take<double>((size_t)n_chunks * mk * mk);
+    for (int j = 0; j < n_proj; ++j) wat[j] = tc ? c.take<uint16_t>((size_t)k * d_in) : nullptr;
+    *region = c.take<float>((size_t)red);
   };
   float* zp;
   double* gp;
+  void* wat[4];
+  float* region;
   {
     Carver c(nullptr);
-    carve(c, &zp, &gp);
+    carve(c, &zp, &gp, wat, &region);
     if (sl_status st = ws_check(ws, c.off)) return st;
   }
   Carver c(ws->ptr);
-  carve(c, &zp, &gp);
+  carve(c, &zp, &gp, wat, &region);
   cudaStream_t s = cs(stream);
-  int rc = est_stage1(x, fp32, n_ctx, d_in, ldx, n_proj, w_a, fp32, k, zp, n_split, s);
-  if (rc) return from_kernel(rc);
+  int rc = 0;
+  if (tc) {
+    GemmBuilder gb;
+    int64_t off = 0;
+    for (int j = 0; j < n_proj; ++j)
+      if ((rc = transpose_bf16(w_a[j], d_in, k, k, wat[j], d_in, s))) return from_kernel(rc);
+    Prob* p = gb.add((int)n_ctx, mk, kBN, (int)rup(mk, 16));
+    Seg* sg = gb.seg(p, gb.map(x, n_ctx, d_in, ldx, kBM), 0, 0, 0, 0, 0, (int)d_in, kBig);
+    for (int j = 0; j < n_proj; ++j) gb.bsrc(sg, gb.map(wat[j], k, d_in, d_in, k), j * k, k, 0, 0);
+    if (p) {
+      p->epi = EPI_F32;
+      p->out0 = zp;
+      p->ld0 = mk;
+      maybe_split(gb, p, n_ctx, mk, d_in, region, &off);
+    }
+    if ((rc = gb.launch(err_word(ws), s))) return from_builder(rc);
+  } else {
+    rc = est_stage1(x, fp32, n_ctx, d_in, ldx, n_proj, w_a, fp32, k, zp, n_split, s);
+    if (rc) return from_kernel(rc);
+  }
   if (crit == SL_CRIT_SWIGLU_L2) {
     rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, s);
     return from_kernel(rc);
@@ -200,14 +240,14 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
   rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s);
   if (rc) return from_kernel(rc);
   if (crit == SL_CRIT_L2) {
-    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
+    rc = est_linear_scores(gp, 1, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
     return from_kernel(rc);
   }
-  rc = est_linear_scores(gp, n_chunks, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
+  rc = est_linear_scores(gp, 1, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
                          scores, s);
   if (rc) return from_kernel(rc);
   if (n_proj == 3)
-    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
+    rc = est_linear_scores(gp, 1, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
   return from_kernel(rc);
 }
 
@@ -248,32 +288,36 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     if (R > 256) return SL_ERR_SHAPE;
     for (int i = 1; i < n_ad; ++i)
       if (lin[i].lora_scale != lin[0].lora_scale) return SL_ERR_UNSUPPORTED;
-    auto carve = [&](Carver& c, void** asig) {
+    const int64_t red = in_sig ? split_floats(C, R, d_in) + split_floats(O, R, d_in) : split_floats(T, R, d_in);
+    auto carve = [&](Carver& c, void** asig, float** region) {
       for (int i = 0; i < n_ad; ++i) asig[i] = in_sig ? c.take<uint16_t>((size_t)lin[i].r * d_in) : nullptr;
+      *region = c.take<float>((size_t)red);
     };
     void* asig[4];
+    float* region;
     {
       Carver c(nullptr);
-      carve(c, asig);
+      carve(c, asig, &region);
       if (sl_status st = ws_check(ws, c.off)) return st;
     }
     Carver c(ws->ptr);
-    carve(c, asig);
+    carve(c, asig, &region);
     if (in_sig)
       for (int i = 0; i < n_ad; ++i)
         if (int rc = gather_cols_bf16(lin[i].lora_a, d_in, lin[i].r, in_ch->sigma, d_in, asig[i], d_in, s))
           return from_kernel(rc);
     GemmBuilder gb;
+    int64_t off = 0;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     const int n_mma = (int)rup(R, 16);
     auto add_prob = [&](int64_t M, int64_t row0, bool sig) {
       Prob* p = gb.add((int)M, R, kBN, n_mma);
       Seg* sg = gb.seg(p, mx, 0, (int)row0, 0, 0, 0, (int)d_in, kBig);
-      int off = 0;
+      int toff = 0;
       for (int i = 0; i < n_ad; ++i) {
         const int mb = gb.map(sig ? asig[i] : lin[i].lora_a, lin[i].r, d_in, d_in, lin[i].r);
-        gb.bsrc(sg, mb, off, lin[i].r, 0, 0);
-        off += lin[i].r;
+        gb.bsrc(sg, mb, toff, lin[i].r, 0, 0);
+        toff += lin[i].r;
       }
       if (!p) return;
       p->epi = EPI_XA;
@@ -284,6 +328,7 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
       p->ld1 = ld_xa;
       p->a0 = 1.f;
       p->a1 = lin[0].lora_scale;
+      maybe_split(gb, p, M, R, d_in, region, &off);
     };
     if (in_sig) {
       add_prob(C, 0, true);
@@ -303,17 +348,32 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     if (ld_dy[i] < lin[i].d_out || ld_dy[i] % 8 || !al16(dy[i]) || !al16(dya_s[i])) return SL_ERR_ALIGNMENT;
     if (out_sig && !channels_ok(out_ch[i], lin[i].d_out)) return SL_ERR_INVALID_ARG;
   }
-  auto carve = [&](Carver& c, void** bsig) {
+  // K extents of the dB / dA parts: pass 0 = natural part (all rows, or output rows when the
+  // operand is in the sigma layout), pass 1 = context rows of a sigma-layout operand.
+  auto kpart = [&](bool sig, int pass) -> int64_t { return sig ? (pass ? C : O) : (pass ? 0 : T); };
+  int64_t red1 = 0, red2[2] = {0, 0};
+  for (int i = 0; i < n_ad; ++i) {
+    const sl_linear& L = lin[i];
+    red1 += out_sig ? split_floats(C, L.r, L.d_out) + split_floats(O, L.r, L.d_out) : split_floats(T, L.r, L.d_out);
+    for (int pass = 0; pass < 2; ++pass) {
+      red2[pass] += kpart(out_sig, pass) > 0 ? split_floats(L.d_out, L.r, kpart(out_sig, pass)) : 0;
+      red2[pass] += kpart(in_sig, pass) > 0 ? split_floats(d_in, L.r, kpart(in_sig, pass)) : 0;
+    }
+  }
+  const int64_t red = std::max(red1, std::max(red2[0], red2[1]));
+  auto carve = [&](Carver& c, void** bsig, float** region) {
     for (int i = 0; i < n_ad; ++i) bsig[i] = out_sig ? c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r) : nullptr;
+    *region = c.take<float>((size_t)red);
   };
   void* bsig[4];
+  float* region;
   {
     Carver c(nullptr);
-    carve(c, bsig);
+    carve(c, bsig, &region);
     if (sl_status st = ws_check(ws, c.off)) return st;
   }
   Carver c(ws->ptr);
-  carve(c, bsig);
+  carve(c, bsig, &region);
   if (out_sig)
     for (int i = 0; i < n_ad; ++i)
       if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i],
@@ -322,6 +382,7 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   // launch 1: dya = scale * dy B
   {
     GemmBuilder gb;
+    int64_t off = 0;
     for (int i = 0; i < n_ad; ++i) {
       const sl_linear& L = lin[i];
       const int mdy = gb.map(dy[i], T, L.d_out, ld_dy[i], kBM);
@@ -340,6 +401,7 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
         p->ld1 = L.r;
         p->a0 = L.lora_scale;
         p->a1 = L.lora_scale;
+        maybe_split(gb, p, M, L.r, L.d_out, region, &off);
       };
       if (out_sig) {
         add_prob(C, 0, mbs);
@@ -350,64 +412,45 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     }
     if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
   }
-  // launch 2: dB = dy^T xa_s, dA = (x^T dya)^T over the natural part; launch 3: sigma parts (accumulate)
+  // launch 2: dB = dy^T xa_s and dA = (x^T dya)^T over the natural parts; launch 3: the
+  // context parts of sigma-layout operands, accumulated onto launch 2's results.
   for (int pass = 0; pass < 2; ++pass) {
     GemmBuilder gb;
+    int64_t off = 0;
     bool any = false;
     for (int i = 0; i < n_ad; ++i) {
       const sl_linear& L = lin[i];
       int64_t koff = 0;
       for (int i2 = 0; i2 < i; ++i2) koff += lin[i2].r;
       const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
-      // dB
-      const bool split_b = out_sig;
-      if (pass == 0 || split_b) {
+      for (int which = 0; which < 2; ++which) {  // 0: dB, 1: dA
+        const bool sig = which == 0 ? out_sig : in_sig;
+        const int64_t K = kpart(sig, pass);
         const bool ctx_part = pass == 1;
-        const int64_t rows = ctx_part ? C : T;   // map extents zero-fill past the part
-        const int64_t k0 = (split_b && !ctx_part) ? C : 0;
-        const int64_t K = split_b ? (ctx_part ? C : O) : T;
-        if (K > 0) {
-          const int ma = gb.map(dy[i], rows, L.d_out, ld_dy[i], 64);
-          const int mb = gb.map(xa_blk, rows, L.r, ld_xa, 64);
-          Prob* p = gb.add((int)L.d_out, L.r, kBN, (int)rup(L.r, 16));
-          Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
-          gb.bsrc(sg, mb, 0, 64, 0, 0);
-          if (p) {
-            p->epi = EPI_F32;
-            p->out0 = dB[i];
-            p->ld0 = L.r;
-            p->beta = ctx_part ? 1 : 0;
-            p->row_map = ctx_part ? out_ch[i].sigma : nullptr;
+        if (K <= 0) {
+          if (!ctx_part) {
+            if (which == 0) cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s);
+            else cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s);
           }
-          any = true;
-        } else if (!ctx_part) {
-          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s);
+          continue;
         }
-      }
-      // dA
-      const bool split_a = in_sig;
-      if (pass == 0 || split_a) {
-        const bool ctx_part = pass == 1;
-        const int64_t rows = ctx_part ? C : T;
-        const int64_t k0 = (split_a && !ctx_part) ? C : 0;
-        const int64_t K = split_a ? (ctx_part ? C : O) : T;
-        if (K > 0) {
-          const int ma = gb.map(x, rows, d_in, ldx, 64);
-          const int mb = gb.map(dya_s[i], rows, L.r, L.r, 64);
-          Prob* p = gb.add((int)d_in, L.r, kBN, (int)rup(L.r, 16));
-          Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
-          gb.bsrc(sg, mb, 0, 64, 0, 0);
-          if (p) {
-            p->epi = EPI_F32_T;
-            p->out0 = dA[i];
-            p->ld0 = d_in;
-            p->beta = ctx_part ? 1 : 0;
-            p->row_map = ctx_part ? in_ch->sigma : nullptr;
-          }
-          any = true;
-        } else if (!ctx_part) {
-          cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s);
+        const int64_t rows = ctx_part ? C : T;  // map extents zero-fill past the part
+        const int64_t k0 = (sig && !ctx_part) ? C : 0;
+        const int64_t M = which == 0 ? L.d_out : d_in;
+        const int ma = which == 0 ? gb.map(dy[i], rows, L.d_out, ld_dy[i], 64) : gb.map(x, rows, d_in, ldx, 64);
+        const int mb = which == 0 ? gb.map(xa_blk, rows, L.r, ld_xa, 64) : gb.map(dya_s[i], rows, L.r, L.r, 64);
+        Prob* p = gb.add((int)M, L.r, kBN, (int)rup(L.r, 16));
+        Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
+        gb.bsrc(sg, mb, 0, 64, 0, 0);
+        if (p) {
+          p->epi = which == 0 ? EPI_F32 : EPI_F32_T;
+          p->out0 = which == 0 ? (void*)dB[i] : (void*)dA[i];
+          p->ld0 = which == 0 ? L.r : d_in;
+          p->beta = ctx_part ? 1 : 0;
+          p->row_map = ctx_part ? (which == 0 ? out_ch[i].sigma : in_ch->sigma) : nullptr;
+          maybe_split(gb, p, M, L.r, K, region, &off);
         }
+        any = true;
       }
     }
     if (any)

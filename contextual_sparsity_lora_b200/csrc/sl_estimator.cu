@@ -9,9 +9,12 @@
 // Stage 2 (linear criteria, V and QK): the token reduction of a linear map
 //          collapses to a Gram matrix, sum_t (Z b_i)_t^2 = b_i^T (Z^T Z) b_i,
 //          formed and contracted in fp64.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "sl_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace sl {
 
@@ -148,13 +151,19 @@ __global__ void est_reduce_kernel(float* zpart, int n_split, int64_t n) {
 
 constexpr int kE2Threads = 256;  // 8 warps; each lane owns 2 channels of a 64-channel block
 constexpr int kE2Tok = 128;      // tokens staged per step
+constexpr int kE2Split = 4;      // token ranges per channel block = CTAs per cluster
 
+// SwiGLU criterion. Grid (F / 64, kE2Split) in clusters of (1, kE2Split): the CTAs of a
+// cluster share a 64-channel block and split the context tokens; their fp64 partial sums
+// are combined by cluster rank 0 through distributed shared memory in rank order.
 template <int K>
-__global__ void __launch_bounds__(kE2Threads) est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx,
-                                                                const void* wb_g, const void* wb_u, int wb_fp32,
-                                                                int64_t n_ch, float* __restrict__ scores) {
-  __shared__ float zs[kE2Tok][2 * K];
+__global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
+    est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx, const void* wb_g, const void* wb_u, int wb_fp32,
+                      int64_t n_ch, float* __restrict__ scores) {
+  __shared__ __align__(16) float zs[kE2Tok][2 * K];
   __shared__ double part[8][64];
+  __shared__ double cta_sum[64];
+  cg::cluster_group cluster = cg::this_cluster();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ch0 = (int64_t)blockIdx.x * 64 + lane;
   const int64_t ch1 = ch0 + 32;
@@ -166,22 +175,30 @@ __global__ void __launch_bounds__(kE2Threads) est_swiglu_kernel(const float* __r
     wg1[c] = ch1 < n_ch ? ld_any(wb_g, c * n_ch + ch1, wb_fp32) : 0.f;
     wu1[c] = ch1 < n_ch ? ld_any(wb_u, c * n_ch + ch1, wb_fp32) : 0.f;
   }
+  const int64_t per = (n_ctx + kE2Split - 1) / kE2Split;
+  const int64_t t_beg = min64(n_ctx, (int64_t)blockIdx.y * per), t_end = min64(n_ctx, t_beg + per);
   double acc0 = 0.0, acc1 = 0.0;
-  for (int64_t tb = 0; tb < n_ctx; tb += kE2Tok) {
+  for (int64_t tb = t_beg; tb < t_end; tb += kE2Tok) {
     __syncthreads();
-    const int tn = (int)min64(kE2Tok, n_ctx - tb);
-    for (int e = threadIdx.x; e < tn * 2 * K; e += kE2Threads) zs[e / (2 * K)][e % (2 * K)] = z[tb * 2 * K + e];
+    const int tn = (int)min64(kE2Tok, t_end - tb);
+    for (int e = threadIdx.x; e < tn * 2 * K / 4; e += kE2Threads)
+      reinterpret_cast<float4*>(&zs[0][0])[e] = reinterpret_cast<const float4*>(z + tb * 2 * K)[e];
     __syncthreads();
     float s0 = 0.f, s1 = 0.f;
     for (int t = warp; t < tn; t += 8) {
       float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
+      const float4* zr = reinterpret_cast<const float4*>(&zs[t][0]);
 #pragma unroll
-      for (int c = 0; c < K; ++c) {
-        const float zg = zs[t][c], zu = zs[t][K + c];
-        g0 = fmaf(zg, wg0[c], g0);
-        u0 = fmaf(zu, wu0[c], u0);
-        g1 = fmaf(zg, wg1[c], g1);
-        u1 = fmaf(zu, wu1[c], u1);
+      for (int c4 = 0; c4 < K / 4; ++c4) {
+        const float4 zg = zr[c4], zu = zr[K / 4 + c4];
+        g0 = fmaf(zg.x, wg0[4 * c4], g0); g0 = fmaf(zg.y, wg0[4 * c4 + 1], g0);
+        g0 = fmaf(zg.z, wg0[4 * c4 + 2], g0); g0 = fmaf(zg.w, wg0[4 * c4 + 3], g0);
+        g1 = fmaf(zg.x, wg1[4 * c4], g1); g1 = fmaf(zg.y, wg1[4 * c4 + 1], g1);
+        g1 = fmaf(zg.z, wg1[4 * c4 + 2], g1); g1 = fmaf(zg.w, wg1[4 * c4 + 3], g1);
+        u0 = fmaf(zu.x, wu0[4 * c4], u0); u0 = fmaf(zu.y, wu0[4 * c4 + 1], u0);
+        u0 = fmaf(zu.z, wu0[4 * c4 + 2], u0); u0 = fmaf(zu.w, wu0[4 * c4 + 3], u0);
+        u1 = fmaf(zu.x, wu1[4 * c4], u1); u1 = fmaf(zu.y, wu1[4 * c4 + 1], u1);
+        u1 = fmaf(zu.z, wu1[4 * c4 + 2], u1); u1 = fmaf(zu.w, wu1[4 * c4 + 3], u1);
       }
       const float h0 = __fdividef(g0, 1.0f + __expf(fminf(-g0, 80.f))) * u0;
       const float h1 = __fdividef(g1, 1.0f + __expf(fminf(-g1, 80.f))) * u1;
@@ -197,28 +214,66 @@ __global__ void __launch_bounds__(kE2Threads) est_swiglu_kernel(const float* __r
   if (threadIdx.x < 64) {
     double s = 0.0;
     for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
+    cta_sum[threadIdx.x] = s;
+  }
+  cluster.sync();
+  if (cluster.block_rank() == 0 && threadIdx.x < 64) {
+    double s = 0.0;
+    for (int rnk = 0; rnk < kE2Split; ++rnk) s += cluster.map_shared_rank(cta_sum, rnk)[threadIdx.x];
     const int64_t ch = (int64_t)blockIdx.x * 64 + threadIdx.x;
     if (ch < n_ch) scores[ch] = (float)sqrt(s);
   }
+  cluster.sync();  // peers keep their shared memory alive until rank 0 has read it
 }
 
-constexpr int kGramTok = 128;
+constexpr int kGramTok = 48;
+constexpr int kGramCluster = 8;
 
-// gram_part[chunk][a][b] = sum_{t in chunk} z[t][a] z[t][b], fp64.
-__global__ void __launch_bounds__(256) est_gram_kernel(const float* __restrict__ z, int64_t n_ctx, int mk,
-                                                       double* __restrict__ gram_part) {
+// Gram matrix G[a][b] = sum_t z[t][a] z[t][b] in fp64. One cluster of kGramCluster CTAs
+// splits the tokens; rank 0 adds the CTAs' partial matrices in rank order (distributed
+// shared memory) and writes G.
+__global__ void __cluster_dims__(kGramCluster, 1, 1) __launch_bounds__(256)
+    est_gram_kernel(const float* __restrict__ z, int64_t n_ctx, int mk, double* __restrict__ gram) {
   __shared__ float zs[kGramTok][64];
-  const int64_t t0 = (int64_t)blockIdx.x * kGramTok;
-  const int tn = (int)min64(kGramTok, n_ctx - t0);
-  for (int e = threadIdx.x; e < tn * mk; e += blockDim.x) zs[e / mk][e % mk] = z[t0 * mk + e];
-  __syncthreads();
-  double* g = gram_part + (int64_t)blockIdx.x * mk * mk;
-  for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
-    const int a = e / mk, b = e % mk;
-    double s = 0.0;
-    for (int t = 0; t < tn; ++t) s = fma((double)zs[t][a], (double)zs[t][b], s);
-    g[e] = s;
+  __shared__ double gpart[64 * 64];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int64_t per = (n_ctx + kGramCluster - 1) / kGramCluster;
+  const int64_t t_beg = min64(n_ctx, rank * per), t_end = min64(n_ctx, t_beg + per);
+  const int ne = mk * mk;
+  double acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.0;
+  for (int64_t tb = t_beg; tb < t_end; tb += kGramTok) {
+    __syncthreads();
+    const int tn = (int)min64(kGramTok, t_end - tb);
+    for (int e = threadIdx.x; e < tn * mk; e += blockDim.x) zs[e / mk][e % mk] = z[tb * mk + e];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int e = threadIdx.x + j * 256;
+      if (e < ne) {
+        const int a = e / mk, b = e % mk;
+        double sum = acc[j];
+        for (int t = 0; t < tn; ++t) sum = fma((double)zs[t][a], (double)zs[t][b], sum);
+        acc[j] = sum;
+      }
+    }
   }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int e = threadIdx.x + j * 256;
+    if (e < ne) gpart[e] = acc[j];
+  }
+  cluster.sync();
+  if (rank == 0) {
+    for (int e = threadIdx.x; e < ne; e += blockDim.x) {
+      double sum = 0.0;
+      for (int r = 0; r < kGramCluster; ++r) sum += cluster.map_shared_rank(gpart, r)[e];
+      gram[e] = sum;
+    }
+  }
+  cluster.sync();
 }
 
 struct WbPtrs {
@@ -237,6 +292,7 @@ __global__ void __launch_bounds__(256) est_linear_scores_kernel(const double* __
   extern __shared__ double gs[];  // [mk][mk]
   for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
     double s = 0.0;
+#pragma unroll 8
     for (int c = 0; c < n_chunks; ++c) s += gram_part[(int64_t)c * mk * mk + e];
     gs[e] = s;
   }
@@ -315,7 +371,7 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
 
 int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, const void* wb_gate, const void* wb_up,
                       int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s) {
-  const unsigned grid = (unsigned)((n_ch + 63) / 64);
+  const dim3 grid((unsigned)((n_ch + 63) / 64), kE2Split);
   switch (k) {
     case 8: est_swiglu_kernel<8><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
     case 16: est_swiglu_kernel<16><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
@@ -327,9 +383,10 @@ int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, con
   return 0;
 }
 
-int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gram_part, int n_chunks, cudaStream_t s) {
-  if (mk > 64 || n_chunks != (int)((n_ctx + kGramTok - 1) / kGramTok)) return 1;
-  est_gram_kernel<<<n_chunks, 256, 0, s>>>(z, n_ctx, mk, gram_part);
+int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gram, int /*n_chunks*/,
+             cudaStream_t s) {
+  if (mk > 64 || n_ctx <= 0) return 1;
+  est_gram_kernel<<<kGramCluster, 256, 0, s>>>(z, n_ctx, mk, gram);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
   return 0;
@@ -351,8 +408,8 @@ int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int 
     w.p[1] = wb1;
     w.n[1] = (int64_t)n_kv_heads * head_dim;
   }
-  const unsigned grid = (unsigned)((n_units + 255) / 256);
-  est_linear_scores_kernel<<<grid, 256, (size_t)mk * mk * sizeof(double), s>>>(
+  const unsigned grid = (unsigned)((n_units + 63) / 64);
+  est_linear_scores_kernel<<<grid, 64, (size_t)mk * mk * sizeof(double), s>>>(
       gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
       crit == 0 ? 1 : head_dim, n_units, scores);
   if (cudaGetLastError() != cudaSuccess) return 5;

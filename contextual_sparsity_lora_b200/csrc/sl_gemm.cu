@@ -10,6 +10,8 @@
 // let the epilogue of tile i overlap the main loop of tile i+1.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "sl_gemm.h"
 #include "sl_internal.h"
 #include "sl_ptx.cuh"
@@ -17,7 +19,7 @@
 namespace sl {
 
 struct TileInfo {
-  int prob, tm, tn;
+  int prob, tm, tn, ks, kb0, kb1;  // ks: split-K index; [kb0, kb1): k-block range (over all segments)
 };
 
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
@@ -26,7 +28,14 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
     if (t >= p.probs[i].tile_begin) pi = i;
   const Prob& pr = p.probs[pi];
   const int local = t - pr.tile_begin;
-  return {pi, local % pr.tiles_m, local / pr.tiles_m};
+  const int per = pr.tiles_m * pr.tiles_n;
+  const int ks = local / per, rem = local % per;
+  TileInfo ti{pi, rem % pr.tiles_m, rem / pr.tiles_m, ks, 0, 1 << 30};
+  if (pr.ksplit > 1) {
+    ti.kb0 = (int)((long long)ks * pr.kblocks / pr.ksplit);
+    ti.kb1 = (int)((long long)(ks + 1) * pr.kblocks / pr.ksplit);
+  }
+  return ti;
 }
 
 __device__ __forceinline__ uint32_t seg_tx_bytes(const Seg& sg) {
@@ -78,7 +87,7 @@ __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* v
 
 // Epilogue of one tile for one thread (one output row). All tcgen05.ld are
 // executed by every lane of the warp (they are warp-collective).
-__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb) {
+__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb, float* stage) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
@@ -119,8 +128,29 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
     __syncwarp();
     tmem_ld32(tb + c0, raw);
     tmem_ld_wait();
-    if (!rv) continue;
     const int n = min(32, ncols - c0);
+    if (pr.epi == EPI_BF16 && pr.col_map) {
+      // Scatter through a 32 x 33 shared-memory transpose: each store instruction then
+      // writes 32 columns of one row (a few sectors) instead of one column of 32 rows.
+      const int lane = r & 31;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(raw[i]) * pr.a0;
+      __syncwarp();
+      const bool cv = lane < n;
+      const int64_t ocol = cv ? (int64_t)pr.col_map[n0 + c0 + lane] : 0;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out0);
+      const int wrow0 = m0 + r - lane;
+      for (int rr = 0; rr < 32; ++rr) {
+        const int row2 = wrow0 + rr;
+        if (cv && row2 < pr.M) {
+          const int64_t o2 = pr.row_map ? (int64_t)pr.row_map[row2] : (int64_t)pr.out_row0 + row2;
+          out[o2 * pr.ld0 + ocol] = __float2bfloat16_rn(stage[rr * 33 + lane]);
+        }
+      }
+      __syncwarp();
+      continue;
+    }
+    if (!rv) continue;
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
     switch (pr.epi) {
@@ -196,6 +226,62 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
   }
 }
 
+// Split-K tile: the raw fp32 accumulator goes to part[ks][row][col]; the reduce kernel
+// sums the splits in a fixed order and applies the problem's epilogue.
+__device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t tb) {
+  const int row = m0 + r;
+  const bool rv = row < pr.M;
+  uint32_t raw[32];
+  float* dst = pr.part + ((int64_t)ks * pr.M + row) * pr.N;
+  for (int c0 = 0; c0 < pr.n_mma; c0 += 32) {
+    if (c0 >= pr.N) break;
+    __syncwarp();
+    tmem_ld32(tb + c0, raw);
+    tmem_ld_wait();
+    if (!rv) continue;
+    const int n = min(32, pr.N - c0);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < n) dst[c0 + i] = __uint_as_float(raw[i]);
+  }
+}
+
+struct RedProb {
+  int32_t M, N, ksplit, epi, beta, out_row0;
+  int64_t ld0, ld1;
+  void* out0;
+  void* out1;
+  const int32_t* row_map;
+  const int32_t* col_map;
+  const float* part;
+  float a0, a1;
+};
+struct RedParams {
+  RedProb p[kMaxProbs];
+};
+
+// Fixed-order sum of split-K partials + the problem's epilogue (EPI_XA, EPI_F32, EPI_F32_T).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ RedParams rp) {
+  const RedProb& pr = rp.p[blockIdx.y];
+  const int64_t total = (int64_t)pr.M * pr.N;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    // transposed stores walk rows fastest so that consecutive threads write consecutive addresses
+    const int64_t row = pr.epi == EPI_F32_T ? e % pr.M : e / pr.N;
+    const int64_t col = pr.epi == EPI_F32_T ? e / pr.M : e % pr.N;
+    float acc = 0.f;
+    for (int s = 0; s < pr.ksplit; ++s) acc += pr.part[((int64_t)s * pr.M + row) * pr.N + col];
+    const int64_t orow = pr.row_map ? (int64_t)pr.row_map[row] : pr.out_row0 + row;
+    const int64_t ocol = pr.col_map ? (int64_t)pr.col_map[col] : col;
+    if (pr.epi == EPI_XA) {
+      reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + ocol] = pr.a0 * acc;
+      reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + ocol] = __float2bfloat16_rn(pr.a1 * acc);
+    } else {
+      float* d = reinterpret_cast<float*>(pr.out0) + (pr.epi == EPI_F32_T ? ocol * pr.ld0 + orow : orow * pr.ld0 + ocol);
+      *d = pr.a0 * acc + (pr.beta ? *d : 0.f);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -209,6 +295,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // 4 x [32][33]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -244,11 +331,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const TileInfo ti = decode_tile(p, t);
         const Prob& pr = p.probs[ti.prob];
         const int n0 = ti.tn * pr.tile_cols;
+        int g = 0;  // k-blocks of earlier active segments
         for (int s = 0; s < pr.nseg; ++s) {
           const Seg& sg = pr.seg[s];
           if (n0 >= sg.n_limit) continue;
           const uint32_t bytes = seg_tx_bytes(sg);
-          for (int kb = 0; kb < sg.nk; ++kb) {
+          const int kb_lo = max(0, ti.kb0 - g), kb_hi = min(sg.nk, ti.kb1 - g);
+          g += sg.nk;
+          for (int kb = kb_lo; kb < kb_hi; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
             mbar_arrive_expect_tx(&full[stage], bytes);
             issued_mask |= 1u << stage;
@@ -299,11 +389,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
         uint32_t accumulate = 0;
+        int g = 0;
         for (int s = 0; s < pr.nseg; ++s) {
           const Seg& sg = pr.seg[s];
           if (n0 >= sg.n_limit) continue;
           const uint32_t idesc = idesc_bf16(kBM, pr.n_mma, sg.a_mn, sg.b_mn);
-          for (int kb = 0; kb < sg.nk; ++kb) {
+          const int kb_lo = max(0, ti.kb0 - g), kb_hi = min(sg.nk, ti.kb1 - g);
+          g += sg.nk;
+          for (int kb = kb_lo; kb < kb_hi; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEV_TIMEOUT_MMA)) goto mma_done;
             tc_fence_after();
             const uint32_t sa = smem_u32(smem_a + stage * kStageABytes);
@@ -344,7 +437,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
-      epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb);
+      if (pr.ksplit > 1)
+        epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb);
+      else
+        epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -446,6 +542,21 @@ Seg* GemmBuilder::seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b
   return s;
 }
 
+int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles) {
+  const int64_t tm = (M + kBM - 1) / kBM;
+  int64_t s = (target_tiles + tm - 1) / tm;
+  const int64_t smax = kblocks / 2;
+  if (s > smax) s = smax;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : (int)s;
+}
+
+void GemmBuilder::split(Prob* pr, int ksplit, float* part) {
+  if (!pr || status != 0) return;
+  pr->ksplit = ksplit;
+  pr->part = part;
+}
+
 void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int row_step) {
   if (!s || status != 0) return;
   if (s->nb >= kMaxBSrc) {
@@ -482,8 +593,20 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     if (!always) return 4;
     pr.tiles_m = pr.M > 0 ? (pr.M + kBM - 1) / kBM : 0;
     pr.tiles_n = pr.N > 0 ? (pr.N + pr.tile_cols - 1) / pr.tile_cols : 0;
+    pr.kblocks = 0;
+    for (int s = 0; s < pr.nseg; ++s) pr.kblocks += pr.seg[s].nk;
+    if (pr.ksplit > 1) {
+      // split-K: skinny problems only; every segment active on every tile; partial buffer set
+      if (pr.tiles_n != 1 || !pr.part || pr.ksplit > pr.kblocks ||
+          (pr.epi != EPI_XA && pr.epi != EPI_F32 && pr.epi != EPI_F32_T))
+        return 4;
+      for (int s = 0; s < pr.nseg; ++s)
+        if (pr.seg[s].n_limit < pr.N) return 4;
+    } else {
+      pr.ksplit = 1;
+    }
     pr.tile_begin = total;
-    total += pr.tiles_m * pr.tiles_n;
+    total += pr.tiles_m * pr.tiles_n * pr.ksplit;
   }
   params.nprob = nprob;
   params.total_tiles = total;
@@ -506,6 +629,26 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   if (cudaGetLastError() != cudaSuccess) return 5;
   if (prof) gemm_events(stream, false);
   note_launch();
+  // reduce the split-K problems (one launch for all of them)
+  RedParams rp;
+  memset(&rp, 0, sizeof(rp));
+  int nred = 0;
+  int64_t maxmn = 0;
+  for (int i = 0; i < nprob; ++i) {
+    const Prob& pr = params.probs[i];
+    if (pr.ksplit <= 1 || pr.M <= 0 || pr.N <= 0) continue;
+    RedProb& q = rp.p[nred++];
+    q.M = pr.M; q.N = pr.N; q.ksplit = pr.ksplit; q.epi = pr.epi; q.beta = pr.beta; q.out_row0 = pr.out_row0;
+    q.ld0 = pr.ld0; q.ld1 = pr.ld1; q.out0 = pr.out0; q.out1 = pr.out1; q.row_map = pr.row_map;
+    q.col_map = pr.col_map; q.part = pr.part; q.a0 = pr.a0; q.a1 = pr.a1;
+    maxmn = std::max<int64_t>(maxmn, (int64_t)pr.M * pr.N);
+  }
+  if (nred) {
+    const unsigned gx = (unsigned)std::min<int64_t>((maxmn + 255) / 256, 1184);
+    splitk_reduce_kernel<<<dim3(gx, nred), 256, 0, stream>>>(rp);
+    if (cudaGetLastError() != cudaSuccess) return 5;
+    note_launch();
+  }
   return 0;
 }
 

@@ -25,7 +25,8 @@ constexpr int kMaxBSrc = 4;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kStageABytes = kBM * kBK * 2;
 constexpr int kStageBBytes = kBN * kBK * 2;
-constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 256;
+constexpr int kEpiStageBytes = 4 * 32 * 33 * 4;  // per-epilogue-warp transpose buffers
+constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 256 + kEpiStageBytes;
 
 enum Epi : int32_t {
   EPI_BF16 = 0,     // out0 bf16 = a0 * acc
@@ -60,6 +61,8 @@ struct Prob {
   int32_t tile_cols;    // output columns per tile: 256 (plain) or 128 (paired SwiGLU)
   int32_t n_mma;        // accumulator columns produced by the MMA (<= 256, multiple of 16)
   int32_t tiles_m, tiles_n, tile_begin;
+  int32_t ksplit;       // K ranges computed as separate tiles (1 = none); partials go to `part`
+  int32_t kblocks;      // total kBK blocks over all segments (all segments must be always-active)
   int32_t nseg;
   Seg seg[kMaxSegs];
   int32_t epi, beta;
@@ -74,6 +77,7 @@ struct Prob {
   const int32_t* col_map;  // optional: output column j -> col_map[j]
   const int32_t* row_map;  // optional: output row i (problem-local) -> row_map[i]
   float a0, a1;
+  float* part;          // split-K partials [ksplit][M][N] fp32 (workspace)
 };
 
 struct GemmParams {

@@ -28,8 +28,14 @@ struct GemmBuilder {
   // K is the segment's K extent; n_limit = output column limit (use N or more for "always").
   Seg* seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b_mn, int b_k0, int K, int n_limit);
   void bsrc(Seg* s, int map, int tile_off, int rows, int row0, int row_step);
+  // Compute a skinny problem as `ksplit` K ranges; `part` holds ksplit * M * N floats.
+  void split(Prob* pr, int ksplit, float* part);
   int launch(int* err, cudaStream_t stream);
 };
+
+// Split-K factor for a skinny problem with M rows and `kblocks` 64-wide K blocks, aiming
+// at about `target_tiles` tiles; 1 = no split.
+int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 296);
 
 // ---- estimator (sl_estimator.cu)
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,

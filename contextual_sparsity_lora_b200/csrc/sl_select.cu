@@ -76,9 +76,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     if (threadIdx.x < 256) hist[threadIdx.x] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int i = threadIdx.x; i < n; i += kSelThreads) {
-      const uint32_t k = keys[i];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+    // Scores concentrate in few exponent bins: aggregate equal bins within a warp so each
+    // bin takes one shared-memory atomic per warp instead of one per lane.
+    const int n_round = (n + kSelThreads - 1) / kSelThreads * kSelThreads;
+    for (int i = threadIdx.x; i < n_round; i += kSelThreads) {
+      const uint32_t k = i < n ? keys[i] : 0u;
+      const bool active = i < n && (k & mask) == prefix;
+      const uint32_t bin = active ? ((k >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (active && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (threadIdx.x < 32) {

@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the in-tree library loads, exports every function the header
+declares, and rejects invalid arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from contextual_sparsity_lora_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparselora.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SL_API\s+[\w\s\*]+?\b(sl_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from contextual_sparsity_lora_b200 import build
+        build.build()
+    return B.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTED)
+
+
+def test_status_strings_and_version(lib):
+    assert B.status_string(B.SL_OK) == "ok"
+    assert "workspace" in B.status_string(B.SL_ERR_WORKSPACE)
+    assert B.sl_version() >= 1
+
+
+@pytest.mark.parametrize("ratio,n,want", [(0.7, 14336, 10036), (0.3, 14336, 4301), (0.5, 1024, 512),
+                                          (0.4, 13824, 5530), (1.0, 7, 7), (1e-6, 10, 1), (0.5, 0, 0)])
+def test_keep_count_host(lib, ratio, n, want):
+    assert B.sl_keep_count(ratio, n) == want
+
+
+def _ws(ptr=None, nbytes=0):
+    return B.SlWorkspaceC(ptr, nbytes, 0)
+
+
+def test_estimate_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    fake = 0x10000  # never dereferenced: validation fails first
+    wa = (P * 2)(fake, fake)
+    wb = (P * 2)(fake, fake)
+    dout = (ctypes.c_int64 * 2)(64, 64)
+    ws = _ws()
+    f = lib.sl_svd_estimate
+    # null x
+    assert f(B.SL_CRIT_L2, B.SL_DT_BF16, None, 8, 64, 64, 1, wa, wb, dout, 8, 0, 0, 0, P(fake), None,
+             ctypes.byref(ws), None) == B.SL_ERR_INVALID_ARG
+    # misaligned leading dimension
+    assert f(B.SL_CRIT_L2, B.SL_DT_BF16, P(fake), 8, 64, 66, 1, wa, wb, dout, 8, 0, 0, 0, P(fake), None,
+             ctypes.byref(ws), None) == B.SL_ERR_ALIGNMENT
+    # rank too large
+    assert f(B.SL_CRIT_L2, B.SL_DT_BF16, P(fake), 8, 64, 64, 1, wa, wb, dout, 32, 0, 0, 0, P(fake), None,
+             ctypes.byref(ws), None) == B.SL_ERR_SHAPE
+    # QK with inconsistent heads
+    assert f(B.SL_CRIT_QK, B.SL_DT_BF16, P(fake), 8, 64, 64, 2, wa, wb, dout, 8, 3, 2, 32, P(fake), None,
+             ctypes.byref(ws), None) == B.SL_ERR_SHAPE
+    # missing workspace: reports the size it needs
+    assert f(B.SL_CRIT_SWIGLU_L2, B.SL_DT_BF16, P(fake), 8, 64, 64, 2, wa, wb, dout, 8, 0, 0, 0, P(fake), None,
+             ctypes.byref(ws), None) == B.SL_ERR_WORKSPACE
+    assert ws.needed > 256
+
+
+def test_select_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    f = lib.sl_select_channels
+    assert f(None, 10, 5, P(0x10000), 0, 0, None, None) == B.SL_ERR_INVALID_ARG
+    assert f(P(0x10000), 10, 0, P(0x10000), 0, 0, None, None) == B.SL_ERR_SHAPE
+    assert f(P(0x10000), 10, 11, P(0x10000), 0, 0, None, None) == B.SL_ERR_SHAPE
+    assert f(P(0x10000), 1 << 20, 5, P(0x10000), 0, 0, None, None) == B.SL_ERR_SHAPE
+    assert f(P(0x10000), 12, 5, P(0x10000), 2, 5, None, None) == B.SL_ERR_INVALID_ARG
+
+
+def _linear(fake, d_in=64, d_out=64, r=8, slice_kind=B.SL_SLICE_OUT, w_t=None):
+    return B.SlLinearC(fake, w_t, d_in, d_out, slice_kind, r, fake, fake, 2.0, 0)
+
+
+def test_linear_calls_reject_bad_arguments(lib):
+    fake = 0x10000
+    P = ctypes.c_void_p
+    ch = B.SlChannelsC(fake, 64, 32)
+    ys = (P * 1)(fake)
+    ld = (ctypes.c_int64 * 1)(64)
+    ws = _ws()
+    fwd = lib.sl_sparse_linear_fwd
+    lin = (B.SlLinearC * 1)(_linear(fake))
+    chs = (B.SlChannelsC * 1)(ch)
+    # context rows beyond the token count
+    assert fwd(1, lin, chs, B.SL_EPI_NONE, P(fake), 64, 10, 11, 0, 0, P(fake), 8, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_SHAPE
+    # LoRA rank not a multiple of 8
+    bad = (B.SlLinearC * 1)(_linear(fake, r=12))
+    assert fwd(1, bad, chs, B.SL_EPI_NONE, P(fake), 64, 10, 5, 0, 0, P(fake), 16, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_INVALID_ARG
+    # channel count larger than the sliced side
+    chs_bad = (B.SlChannelsC * 1)(B.SlChannelsC(fake, 64, 65))
+    assert fwd(1, lin, chs_bad, B.SL_EPI_NONE, P(fake), 64, 10, 5, 0, 0, P(fake), 8, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_INVALID_ARG
+    # misaligned pointer
+    assert fwd(1, lin, chs, B.SL_EPI_NONE, P(fake + 2), 64, 10, 5, 0, 0, P(fake), 8, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_ALIGNMENT
+    # input-sliced layer without its transposed weight
+    lin_in = (B.SlLinearC * 1)(_linear(fake, slice_kind=B.SL_SLICE_IN))
+    assert fwd(1, lin_in, chs, B.SL_EPI_NONE, P(fake), 64, 10, 5, 0, 0, P(fake), 8, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_INVALID_ARG
+    # workspace query for a valid call
+    assert fwd(1, lin, chs, B.SL_EPI_NONE, P(fake), 64, 10, 5, 0, 0, P(fake), 8, ys, ld, ctypes.byref(ws),
+               None) == B.SL_ERR_WORKSPACE
+    assert ws.needed > 256
+    bwd = lib.sl_sparse_linear_bwd
+    dys = (P * 1)(fake)
+    assert bwd(4, lin, chs, B.SL_EPI_NONE, dys, ld, 10, 5, 0, 0, (P * 1)(fake), P(fake), 64, None, None,
+               ctypes.byref(ws), None) == B.SL_ERR_INVALID_ARG
+    lora = lib.sl_lora_fwd_bwd
+    assert lora(B.SL_LORA_FWD, 0, lin, P(fake), 64, 10, 5, 0, None, P(fake), P(fake), 8, None, None, 0, None,
+                None, None, None, None, ctypes.byref(ws), None) == B.SL_ERR_INVALID_ARG
+
+
+def test_workspace_init_and_profile_hooks_host_side(lib):
+    ws = _ws()
+    assert lib.sl_workspace_init(ctypes.byref(ws), None) == B.SL_ERR_WORKSPACE
+    assert lib.sl_profile_enable(0) == B.SL_OK
+    a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_double()
+    assert lib.sl_profile_read(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == B.SL_OK
+    assert lib.sl_profile_read(None, None, None) == B.SL_ERR_INVALID_ARG
