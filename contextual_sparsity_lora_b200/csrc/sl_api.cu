@@ -29,6 +29,11 @@ void note_launch(int n) {
 bool profiling_on() { return g_prof.load(std::memory_order_relaxed); }
 void gemm_events(cudaStream_t s, bool start) {
   std::lock_guard<std::mutex> lk(g_ev_mu);
+  // Under stream capture the records become event nodes of the graph, re-recorded by
+  // every replay (external records); otherwise they are plain stream records.
+  cudaStreamCaptureStatus cst = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cst);
+  const unsigned flags = cst == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
   if (start) {
     if (g_ev_used == g_events.size()) {
       cudaEvent_t a, b;
@@ -36,9 +41,9 @@ void gemm_events(cudaStream_t s, bool start) {
       if (cudaEventCreate(&b) != cudaSuccess) return;
       g_events.emplace_back(a, b);
     }
-    cudaEventRecord(g_events[g_ev_used].first, s);
+    cudaEventRecordWithFlags(g_events[g_ev_used].first, s, flags);
   } else {
-    cudaEventRecord(g_events[g_ev_used].second, s);
+    cudaEventRecordWithFlags(g_events[g_ev_used].second, s, flags);
     ++g_ev_used;
   }
 }

@@ -543,6 +543,7 @@ Seg* GemmBuilder::seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b
 }
 
 int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles) {
+  if (M <= 0 || kblocks <= 1) return 1;
   const int64_t tm = (M + kBM - 1) / kBM;
   int64_t s = (target_tiles + tm - 1) / tm;
   const int64_t smax = kblocks / 2;
