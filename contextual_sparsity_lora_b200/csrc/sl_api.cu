@@ -59,10 +59,10 @@ inline cudaStream_t cs(sl_stream s) { return reinterpret_cast<cudaStream_t>(s); 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Two-pass carving of the caller's workspace: the first pass (base == nullptr)
-// only measures. The first 256 bytes are the device error word.
+// only measures. The header (error word, split-tile counters) comes first.
 struct Carver {
   uint8_t* base;
-  size_t off = 256;
+  size_t off = kWorkspaceHeaderBytes;
   explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
   template <typename T>
   T* take(size_t count) {
@@ -146,8 +146,10 @@ int64_t sl_keep_count(double ratio, int64_t n) {
 }
 
 sl_status sl_workspace_init(sl_workspace* ws, sl_stream stream) {
-  if (!ws || !ws->ptr || ws->bytes < 256) return SL_ERR_WORKSPACE;
-  return cudaMemsetAsync(ws->ptr, 0, 256, cs(stream)) == cudaSuccess ? SL_OK : SL_ERR_CUDA;
+  if (!ws) return SL_ERR_WORKSPACE;
+  ws->needed = kWorkspaceHeaderBytes;
+  if (!ws->ptr || ws->bytes < (size_t)kWorkspaceHeaderBytes) return SL_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws->ptr, 0, kWorkspaceHeaderBytes, cs(stream)) == cudaSuccess ? SL_OK : SL_ERR_CUDA;
 }
 
 sl_status sl_read_device_flag(const sl_workspace* ws, int32_t* code, sl_stream stream) {
@@ -198,7 +200,7 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
   // accumulation, fixed-order split-K); fp32 inputs: CUDA-core fp32 FMA kernel.
   const bool tc = !fp32 && k % 8 == 0;
   const int n_split = tc ? 1 : est1_splits(d_in);
-  const int n_chunks = (int)((n_ctx + kGramChunk - 1) / kGramChunk);
+  const int n_chunks = gram_groups(n_ctx);
   const int64_t red = tc ? split_floats(n_ctx, mk, d_in) : 0;
   auto carve = [&](Carver& c, float** zp, double** gp, void** wat, float** region) {
     *zp = c.take<float>((size_t)n_split * n_ctx * mk);
@@ -245,14 +247,14 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
   rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s);
   if (rc) return from_kernel(rc);
   if (crit == SL_CRIT_L2) {
-    rc = est_linear_scores(gp, 1, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
+    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
     return from_kernel(rc);
   }
-  rc = est_linear_scores(gp, 1, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
+  rc = est_linear_scores(gp, n_chunks, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
                          scores, s);
   if (rc) return from_kernel(rc);
   if (n_proj == 3)
-    rc = est_linear_scores(gp, 1, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
+    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
   return from_kernel(rc);
 }
 

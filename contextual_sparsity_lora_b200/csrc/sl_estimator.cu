@@ -238,8 +238,10 @@ __global__ void __cluster_dims__(kGramCluster, 1, 1) __launch_bounds__(256)
   __shared__ double gpart[64 * 64];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
-  const int64_t per = (n_ctx + kGramCluster - 1) / kGramCluster;
-  const int64_t t_beg = min64(n_ctx, rank * per), t_end = min64(n_ctx, t_beg + per);
+  // cluster c covers tokens [c * 8 * kGramTok, (c + 1) * 8 * kGramTok); its rank r the r-th kGramTok slice
+  const int64_t per = kGramTok;
+  const int64_t t_beg = min64(n_ctx, ((int64_t)blockIdx.x / kGramCluster * kGramCluster + rank) * per),
+                t_end = min64(n_ctx, t_beg + per);
   const int ne = mk * mk;
   double acc[16];
 #pragma unroll
@@ -270,7 +272,7 @@ __global__ void __cluster_dims__(kGramCluster, 1, 1) __launch_bounds__(256)
     for (int e = threadIdx.x; e < ne; e += blockDim.x) {
       double sum = 0.0;
       for (int r = 0; r < kGramCluster; ++r) sum += cluster.map_shared_rank(gpart, r)[e];
-      gram[e] = sum;
+      gram[(int64_t)(blockIdx.x / kGramCluster) * ne + e] = sum;
     }
   }
   cluster.sync();
@@ -386,7 +388,7 @@ int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, con
 int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gram, int /*n_chunks*/,
              cudaStream_t s) {
   if (mk > 64 || n_ctx <= 0) return 1;
-  est_gram_kernel<<<kGramCluster, 256, 0, s>>>(z, n_ctx, mk, gram);
+  est_gram_kernel<<<gram_groups(n_ctx) * kGramCluster, 256, 0, s>>>(z, n_ctx, mk, gram);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
   return 0;

@@ -264,7 +264,32 @@ struct RedParams {
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ RedParams rp) {
   const RedProb& pr = rp.p[blockIdx.y];
   const int64_t total = (int64_t)pr.M * pr.N;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if (pr.epi != EPI_F32_T && pr.N % 4 == 0 && !pr.col_map) {
+    // four consecutive columns per thread: 16-byte partial loads
+    for (int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; e < total; e += stride * 4) {
+      const int64_t row = e / pr.N, col = e % pr.N;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < pr.ksplit; ++s) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(pr.part + (int64_t)s * total + e));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const int64_t orow = pr.row_map ? (int64_t)pr.row_map[row] : pr.out_row0 + row;
+      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (pr.epi == EPI_XA) {
+          reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + col + j] = pr.a0 * a[j];
+          reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + col + j] = __float2bfloat16_rn(pr.a1 * a[j]);
+        } else {
+          float* d = reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + col + j;
+          *d = pr.a0 * a[j] + (pr.beta ? *d : 0.f);
+        }
+      }
+    }
+    return;
+  }
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
     // transposed stores walk rows fastest so that consecutive threads write consecutive addresses
     const int64_t row = pr.epi == EPI_F32_T ? e % pr.M : e / pr.N;
     const int64_t col = pr.epi == EPI_F32_T ? e / pr.M : e % pr.N;

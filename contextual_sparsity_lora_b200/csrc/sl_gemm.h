@@ -22,6 +22,10 @@ constexpr int kMaxMaps = 48;
 constexpr int kMaxProbs = 12;
 constexpr int kMaxSegs = 6;
 constexpr int kMaxBSrc = 4;
+// Workspace header: error word at byte 0, split-tile finish counters from byte 256.
+constexpr int kWorkspaceHeaderBytes = 65536;
+constexpr int kCounterOffsetInts = 64;
+constexpr int kMaxSplitCounters = (kWorkspaceHeaderBytes - 256) / 4;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kStageABytes = kBM * kBK * 2;
 constexpr int kStageBBytes = kBN * kBK * 2;
@@ -62,6 +66,7 @@ struct Prob {
   int32_t n_mma;        // accumulator columns produced by the MMA (<= 256, multiple of 16)
   int32_t tiles_m, tiles_n, tile_begin;
   int32_t ksplit;       // K ranges computed as separate tiles (1 = none); partials go to `part`
+  int32_t cnt_base;     // first finish counter of this problem's split tiles (4 per row tile)
   int32_t kblocks;      // total kBK blocks over all segments (all segments must be always-active)
   int32_t nseg;
   Seg seg[kMaxSegs];
@@ -85,6 +90,7 @@ struct GemmParams {
   Prob probs[kMaxProbs];
   int32_t nprob, total_tiles;
   int* err;
+  int* counters;        // split-tile finish counters (zero between launches)
 };
 
 }  // namespace sl

@@ -34,8 +34,8 @@ struct GemmBuilder {
 };
 
 // Split-K factor for a skinny problem with M rows and `kblocks` 64-wide K blocks, aiming
-// at about `target_tiles` tiles; 1 = no split.
-int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 296);
+// at about `target_tiles` tiles (about one wave); 1 = no split.
+int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 160);
 
 // ---- estimator (sl_estimator.cu)
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
@@ -48,7 +48,9 @@ int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int 
                       const void* wb0, const void* wb1, int wb_fp32, int n_q_heads, int n_kv_heads, int head_dim,
                       int64_t n_units, float* scores, cudaStream_t s);
 int est1_splits(int64_t d_in);
-constexpr int kGramChunk = 128;
+// The Gram kernel runs clusters of 8 CTAs over 48 context tokens each; one fp64 partial
+// Gram matrix per cluster is left for the score kernel to add.
+inline int gram_groups(int64_t n_ctx) { return (int)((n_ctx + 8 * 48 - 1) / (8 * 48)); }
 
 // ---- selection (sl_select.cu)
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group,

@@ -85,9 +85,10 @@ typedef enum { SL_LORA_FWD = 0, SL_LORA_BWD = 1 } sl_lora_mode;
 
 /* Caller-owned scratch memory. When ptr is NULL or bytes < the size a call needs, the
  * call stores the size in `needed` and returns SL_ERR_WORKSPACE without launching.
- * The first 256 bytes hold the device error word; zero them once with
- * sl_workspace_init before first use. Calls that share a workspace must be ordered
- * on one stream. */
+ * The first 64 KiB are a header: the device error word (byte 0) and the finish counters
+ * of split-K GEMM tiles (which the kernels return to zero). Zero the header once with
+ * sl_workspace_init before first use. Calls that share a workspace must be ordered on
+ * one stream (they reuse the same scratch and counters). */
 typedef struct {
   void* ptr;
   size_t bytes;
