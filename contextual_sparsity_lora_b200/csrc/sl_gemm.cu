@@ -87,7 +87,9 @@ __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* v
 
 // Epilogue of one tile for one thread (one output row). All tcgen05.ld are
 // executed by every lane of the warp (they are warp-collective).
-__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb, float* stage) {
+// `half` selects the 32-column chunks this warp handles (even or odd); the other epilogue
+// warp on the same TMEM lane quarter takes the rest.
+__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb, float* stage, int half) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
@@ -96,7 +98,7 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
 
   if (pr.epi == EPI_SWIGLU) {
     const int ncols = min(128, pr.N - n0);
-    for (int c0 = 0; c0 < 128; c0 += 32) {
+    for (int c0 = 32 * half; c0 < 128; c0 += 64) {
       if (c0 >= ncols) break;
       float g[32];
       __syncwarp();
@@ -123,7 +125,7 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
   }
 
   const int ncols = min(pr.tile_cols, pr.N - n0);
-  for (int c0 = 0; c0 < pr.n_mma; c0 += 32) {
+  for (int c0 = 32 * half; c0 < pr.n_mma; c0 += 64) {
     if (c0 >= ncols) break;
     __syncwarp();
     tmem_ld32(tb + c0, raw);
@@ -228,12 +230,12 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
 
 // Split-K tile: the raw fp32 accumulator goes to part[ks][row][col]; the reduce kernel
 // sums the splits in a fixed order and applies the problem's epilogue.
-__device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t tb) {
+__device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t tb, int half) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   uint32_t raw[32];
   float* dst = pr.part + ((int64_t)ks * pr.M + row) * pr.N;
-  for (int c0 = 0; c0 < pr.n_mma; c0 += 32) {
+  for (int c0 = 32 * half; c0 < pr.n_mma; c0 += 64) {
     if (c0 >= pr.N) break;
     __syncwarp();
     tmem_ld32(tb + c0, raw);
@@ -332,7 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -452,7 +454,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;   // which 32-column chunks of the tile
     const int r = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -463,9 +466,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
       if (pr.ksplit > 1)
-        epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb);
+        epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb, half);
       else
-        epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33);
+        epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33, half);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

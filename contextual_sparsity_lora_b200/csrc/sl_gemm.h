@@ -26,10 +26,11 @@ constexpr int kMaxBSrc = 4;
 constexpr int kWorkspaceHeaderBytes = 65536;
 constexpr int kCounterOffsetInts = 64;
 constexpr int kMaxSplitCounters = (kWorkspaceHeaderBytes - 256) / 4;
-constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEpiWarps = 8;       // two epilogue warps per TMEM lane quarter, splitting the columns
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
 constexpr int kStageABytes = kBM * kBK * 2;
 constexpr int kStageBBytes = kBN * kBK * 2;
-constexpr int kEpiStageBytes = 4 * 32 * 33 * 4;  // per-epilogue-warp transpose buffers
+constexpr int kEpiStageBytes = kEpiWarps * 32 * 33 * 4;  // per-epilogue-warp transpose buffers
 constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 256 + kEpiStageBytes;
 
 enum Epi : int32_t {
