@@ -486,6 +486,207 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair variant
+//
+// Same roles and problem list, but a cluster of two CTAs (two SMs) computes one
+// 256-row x 256-column tile with cta_group::2 MMAs: each CTA stages its own 128 rows of
+// A and its half (128 rows) of the B tile, the even CTA issues the MMAs for both, and
+// each CTA's TMEM holds the accumulator of its 128 rows. Per SM this halves the B bytes
+// per FLOP of the one-CTA kernel. Only full-width tiles (n_mma = 256) use it.
+constexpr int kStages2 = 6;
+constexpr int kStageB2Bytes = 128 * kBK * 2;
+
+__device__ __forceinline__ void pair_b_loads(const GemmParams& p, const Seg& sg, int tn, uint32_t rank, uint8_t* sb,
+                                             uint64_t* full, int kc) {
+  for (int i = 0; i < sg.nb; ++i) {
+    const BSrc& b = sg.b[i];
+    const int coord = b.row0 + b.row_step * tn;
+    if (!sg.b_mn) {
+      if (b.rows == 256)
+        tma_load_2d_pair(sb, &p.maps[b.map], full, sg.b_k0 + kc, coord + 128 * (int)rank);
+      else if (b.tile_off / 128 == (int)rank)
+        tma_load_2d_pair(sb, &p.maps[b.map], full, sg.b_k0 + kc, coord);
+    } else {
+      for (int c = 0; c < 2; ++c)
+        tma_load_2d_pair(sb + c * 8192, &p.maps[b.map], full, coord + 128 * (int)rank + 64 * c, sg.b_k0 + kc);
+    }
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem_a = smem;
+  uint8_t* smem_b = smem + kStages2 * kStageABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + kStages2 * kStageB2Bytes);
+  uint64_t* full = bars;              // used in the even CTA: both CTAs' copies count here
+  uint64_t* empty = bars + kStages2;  // both CTAs: armed by the even CTA's MMA commits
+  uint64_t* tfull = bars + 2 * kStages2;
+  uint64_t* tempty = tfull + 2;       // used in the even CTA: both CTAs' epilogue threads arrive
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cl = blockIdx.x >> 1, n_cl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * 32 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before any copy or arrive targets them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_par = 0;
+      for (int t = cl; t < p.total_tiles && !*abort_flag; t += n_cl) {
+        const TileInfo ti = decode_tile(p, t);
+        const Prob& pr = p.probs[ti.prob];
+        const int n0 = ti.tn * pr.tile_cols;
+        for (int s = 0; s < pr.nseg; ++s) {
+          const Seg& sg = pr.seg[s];
+          if (n0 >= sg.n_limit) continue;
+          for (int kb = 0; kb < sg.nk; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
+            if (leader) {
+              mbar_arrive_expect_tx(&full[stage], 2u * (kStageABytes + kStageB2Bytes));
+              issued_mask |= 1u << stage;
+              issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            }
+            uint8_t* sa = smem_a + stage * kStageABytes;
+            uint8_t* sb = smem_b + stage * kStageB2Bytes;
+            const int kc = kb * kBK;
+            const int arow = sg.a_row0 + ti.tm * 256 + 128 * (int)rank;
+            if (!sg.a_mn) {
+              tma_load_2d_pair(sa, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, arow);
+            } else {
+              tma_load_2d_pair(sa, &p.maps[sg.a_map], &full[stage], arow, sg.a_k0 + kc);
+              tma_load_2d_pair(sa + 8192, &p.maps[sg.a_map], &full[stage], arow + 64, sg.a_k0 + kc);
+            }
+            pair_b_loads(p, sg, ti.tn, rank, sb, &full[stage], kc);
+            if (++stage == kStages2) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+      }
+    producer_done:
+      // The even CTA's barriers count both CTAs' copies: wait for every stage it armed.
+      for (int s = 0; s < kStages2; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = cl; t < p.total_tiles && !*abort_flag; t += n_cl) {
+        const TileInfo ti = decode_tile(p, t);
+        const Prob& pr = p.probs[ti.prob];
+        const int n0 = ti.tn * pr.tile_cols;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+        uint32_t accumulate = 0;
+        for (int s = 0; s < pr.nseg; ++s) {
+          const Seg& sg = pr.seg[s];
+          if (n0 >= sg.n_limit) continue;
+          const uint32_t idesc = idesc_bf16(256, pr.n_mma, sg.a_mn, sg.b_mn);
+          for (int kb = 0; kb < sg.nk; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEV_TIMEOUT_MMA)) goto mma_done;
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem_a + stage * kStageABytes);
+            const uint32_t sb = smem_u32(smem_b + stage * kStageB2Bytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t ad = sg.a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bd = sg.b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sb + k * 32, 16, 1024);
+              umma_bf16_pair(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1;
+            }
+            umma_commit_pair_mc(&empty[stage], 0x3);
+            if (++stage == kStages2) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+        umma_commit_pair_mc(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    mma_done:
+      umma_commit_pair(drain);
+      mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = cl; t < p.total_tiles; t += n_cl) {
+      const TileInfo ti = decode_tile(p, t);
+      const Prob& pr = p.probs[ti.prob];
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      epilogue_tile(pr, ti.tm * 256 + 128 * (int)rank, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33,
+                    half);
+      __syncwarp();
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && !leader) {
+    // copies of this CTA signal the even CTA's barriers: give any in flight time to land
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while its peer may still read its shared memory or TMEM
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -531,7 +732,29 @@ int GemmBuilder::map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, in
     status = 2;
     return 0;
   }
+  specs[nmaps] = MapSpec{ptr, rows, cols, ld, box_rows};
   return nmaps++;
+}
+
+bool GemmBuilder::pair_eligible() const {
+  static const bool disabled = [] {
+    const char* e = getenv("SL_GEMM_1CTA");
+    return e && e[0] == '1';
+  }();
+  if (disabled || nprob == 0) return false;
+  for (int i = 0; i < nprob; ++i) {
+    const Prob& pr = params.probs[i];
+    if (pr.ksplit > 1 || pr.n_mma != kBN) return false;
+    for (int s = 0; s < pr.nseg; ++s) {
+      const Seg& sg = pr.seg[s];
+      // each CTA must stage exactly 128 rows (or 128 N columns) of every B tile
+      const bool full_one = sg.nb == 1 && sg.b[0].tile_off == 0 && sg.b[0].rows == 256;
+      const bool split_two = !sg.b_mn && sg.nb == 2 && sg.b[0].tile_off == 0 && sg.b[0].rows == 128 &&
+                             sg.b[1].tile_off == 128 && sg.b[1].rows == 128;
+      if (!full_one && !split_two) return false;
+    }
+  }
+  return true;
 }
 
 Prob* GemmBuilder::add(int M, int N, int tile_cols, int n_mma) {
@@ -602,6 +825,29 @@ void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int ro
 
 int GemmBuilder::launch(int* err, cudaStream_t stream) {
   if (status != 0) return status;
+  const bool pair = pair_eligible();
+  const int tile_m = pair ? 2 * kBM : kBM;
+  if (pair) {
+    // each CTA of a pair stages 128 rows of a 256-row K-major B source: re-encode those
+    // maps with a 128-row box (shared by every source that uses the same map)
+    int remap[kMaxMaps];
+    for (int m = 0; m < kMaxMaps; ++m) remap[m] = -1;
+    for (int i = 0; i < nprob; ++i)
+      for (int s = 0; s < params.probs[i].nseg; ++s) {
+        Seg& sg = params.probs[i].seg[s];
+        if (sg.b_mn) continue;
+        for (int b = 0; b < sg.nb; ++b) {
+          BSrc& bs = sg.b[b];
+          if (bs.rows != 256) continue;
+          if (remap[bs.map] < 0) {
+            const MapSpec sp = specs[bs.map];
+            remap[bs.map] = map(sp.ptr, sp.rows, sp.cols, sp.ld, 128);
+            if (status != 0) return status;
+          }
+          bs.map = (int16_t)remap[bs.map];
+        }
+      }
+  }
   int total = 0;
   for (int i = 0; i < nprob; ++i) {
     Prob& pr = params.probs[i];
@@ -620,7 +866,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
       }
     }
     if (!always) return 4;
-    pr.tiles_m = pr.M > 0 ? (pr.M + kBM - 1) / kBM : 0;
+    pr.tiles_m = pr.M > 0 ? (pr.M + tile_m - 1) / tile_m : 0;
     pr.tiles_n = pr.N > 0 ? (pr.N + pr.tile_cols - 1) / pr.tile_cols : 0;
     pr.kblocks = 0;
     for (int s = 0; s < pr.nseg; ++s) pr.kblocks += pr.seg[s].nk;
@@ -646,15 +892,23 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
         cudaSuccess)
       return 5;
+    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+        cudaSuccess)
+      return 5;
     smem_set = 1;
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = total < sms ? total : sms;
   const bool prof = profiling_on();
   if (prof) gemm_events(stream, true);
-  gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+  if (pair) {
+    const int clusters = std::min(total, sms / 2);
+    gemm_pair_kernel<<<2 * clusters, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+  } else {
+    const int grid = total < sms ? total : sms;
+    gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+  }
   if (cudaGetLastError() != cudaSuccess) return 5;
   if (prof) gemm_events(stream, false);
   note_launch();

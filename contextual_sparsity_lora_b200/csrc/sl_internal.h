@@ -15,12 +15,20 @@ void gemm_events(cudaStream_t s, bool start);
 
 // Builds the parameter block of one grouped GEMM launch on the host.
 struct GemmBuilder {
+  struct MapSpec {
+    const void* ptr;
+    int64_t rows, cols, ld;
+    int box_rows;
+  };
   GemmParams params;
+  MapSpec specs[kMaxMaps];
   int nmaps = 0;
   int nprob = 0;
   int status = 0;  // 0 ok, 1 too many maps/problems/segments, 2 bad tensor, 3 no driver entry, 4 bad problem, 5 launch
 
   GemmBuilder() { memset(&params, 0, sizeof(params)); }
+  // True when every problem can run as 256 x 256 tiles on CTA pairs.
+  bool pair_eligible() const;
   // bf16 row-major matrix [rows, cols] with leading dimension ld (elements);
   // the TMA box is 64 columns x box_rows rows, 128-byte swizzled, zero fill.
   int map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows);
