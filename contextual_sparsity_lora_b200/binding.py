@@ -27,7 +27,8 @@ SL_LORA_FWD, SL_LORA_BWD = 0, 1
 
 EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_init", "sl_read_device_flag",
             "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
-            "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read")
+            "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
+            "sl_svd_estimate_noalloc")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -179,6 +180,22 @@ def sl_svd_estimate(ws: Workspace, crit, x, n_ctx, w_a, w_b, k, scores, scores_v
     ws.call("sl_svd_estimate", crit, dtype, _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w_a), _ptrs(w_a),
             _ptrs(w_b), _i64s(d_out), int(k), int(n_q_heads), int(n_kv_heads), int(head_dim), _ptr(scores),
             _ptr(scores_v))
+
+
+def sl_svd_estimate_noalloc(crit, x, n_ctx, w_a, w_b, k, scores, scores_v=None, n_q_heads=0, n_kv_heads=0,
+                            head_dim=0, device_flag=None):
+    """sl_svd_estimate on the library's fixed scratch array (no workspace, no allocation).
+    Returns the scratch bytes the call needed; device_flag: optional int32 CUDA tensor that
+    receives the call's device error word."""
+    dtype = SL_DT_F32 if x.dtype == torch.float32 else SL_DT_BF16
+    d_out = [t.shape[1] for t in w_b]
+    needed = c_int64(0)
+    _check("sl_svd_estimate_noalloc",
+           lib().sl_svd_estimate_noalloc(crit, dtype, _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w_a),
+                                         _ptrs(w_a), _ptrs(w_b), _i64s(d_out), int(k), int(n_q_heads),
+                                         int(n_kv_heads), int(head_dim), _ptr(scores), _ptr(scores_v),
+                                         ctypes.byref(needed), _ptr(device_flag), _stream()))
+    return int(needed.value)
 
 
 def sl_select_channels(scores, n_keep, sigma, heads_per_group=0, head_dim=0, sigma_wide=None):

@@ -148,6 +148,29 @@ SL_API sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* 
                           int32_t head_dim, float* scores, float* scores_v, sl_workspace* ws,
                           sl_stream stream);
 
+/* sl_svd_estimate without a workspace: the method itself has no counterpart of this entry;
+ * it exists for callers that cannot supply device scratch (a host with no device allocator
+ * of its own, or code where cudaMalloc/cudaFree must not run because cudaFree synchronises
+ * the whole device). Same arguments, layouts and results as sl_svd_estimate (bit-identical
+ * scores), with the scratch taken from a fixed 8 MiB array inside the library, one per
+ * device; the call allocates nothing.
+ *   scratch_needed: optional host int64; receives the bytes the call needs whenever the
+ *     arguments are valid.
+ *   device_flag: optional device int32; receives, on `stream` after the estimator's
+ *     kernels, the call's device error word (0 = no device-side timeout).
+ * Errors: argument errors as sl_svd_estimate; SL_ERR_WORKSPACE when the shapes need more
+ * than the 8 MiB (nothing is launched); SL_ERR_CUDA when the array's address cannot be
+ * looked up. The first call on a device (with that device current) looks the address up
+ * and should precede any stream capture there. All calls share the array and leave their
+ * contents in it; the header is cleared at the start of each call. Calls that may execute
+ * at the same time (different streams, unordered threads) race on it: serialise them. */
+SL_API sl_status sl_svd_estimate_noalloc(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx,
+                                         int64_t d_in, int64_t ldx, int32_t n_proj, const void* const* w_a,
+                                         const void* const* w_b, const int64_t* d_out, int32_t k,
+                                         int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float* scores,
+                                         float* scores_v, int64_t* scratch_needed, int32_t* device_flag,
+                                         sl_stream stream);
+
 /* a3: top-n selection ([WT] Algorithm 1; [PN] top-n). Keeps exactly n_keep of the n
  * scores: larger score first, ties to the lower index, NaN below every number.
  * Writes sigma[n] (kept ascending, then dropped ascending). When heads_per_group > 0
