@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "../../include/sparselora.h"
@@ -20,6 +21,9 @@ std::atomic<long long> g_launches{0};
 std::mutex g_ev_mu;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_events;
 size_t g_ev_used = 0;
+#ifdef SL_PROFILE_DUMP
+std::vector<std::string> g_notes;
+#endif
 }  // namespace
 
 namespace sl {
@@ -27,6 +31,20 @@ void note_launch(int n) {
   if (g_prof.load(std::memory_order_relaxed)) g_launches.fetch_add(n, std::memory_order_relaxed);
 }
 bool profiling_on() { return g_prof.load(std::memory_order_relaxed); }
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SL_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+#ifdef SL_PROFILE_DUMP
+void gemm_note(const char* desc) {
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  if (g_notes.size() <= g_ev_used) g_notes.resize(g_ev_used + 1);
+  g_notes[g_ev_used] = desc;
+}
+#endif
 void gemm_events(cudaStream_t s, bool start) {
   std::lock_guard<std::mutex> lk(g_ev_mu);
   // Under stream capture the records become event nodes of the graph, re-recorded by
@@ -822,6 +840,9 @@ sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launches, doub
     if (cudaEventSynchronize(g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
     if (cudaEventElapsedTime(&t, g_events[i].first, g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
     ms += t;
+#ifdef SL_PROFILE_DUMP
+    fprintf(stderr, "[sl gemm %zu] %.4f ms %s\n", i, t, i < g_notes.size() ? g_notes[i].c_str() : "");
+#endif
   }
   *gemm_ms = ms;
   *gemm_launches = (int64_t)g_ev_used;

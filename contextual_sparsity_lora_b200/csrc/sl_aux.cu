@@ -17,6 +17,7 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int64_
                                    const int32_t* __restrict__ idx, int64_t n_rows, int64_t n_cols,
                                    __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int64_t col0, int vec, int blk,
                                    int blk_stride, int blk_off) {
+  pdl_wait();
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= n_rows) return;
@@ -37,6 +38,7 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int64_
 __global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t n_rows,
                                    const int32_t* __restrict__ idx, int64_t n_idx, __nv_bfloat16* __restrict__ dst,
                                    int64_t ld_dst) {
+  pdl_wait();
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n_idx) return;
   const int64_t c = idx[j];
@@ -46,6 +48,7 @@ __global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_
 // dst[c, r] = src[r, c] with a 32 x 32 shared-memory tile.
 __global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols, int64_t ld_src,
                                  __nv_bfloat16* __restrict__ dst, int64_t ld_dst) {
+  pdl_wait();
   __shared__ __nv_bfloat16 tile[32][34];
   const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -60,6 +63,7 @@ __global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t 
 }
 
 __global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, int64_t n) {
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) dst[i] += src[i];
 }
@@ -72,7 +76,7 @@ int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_
   const int vec = (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (dst_col0 % 8 == 0) &&
                   ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
   const int rows_per_block = 8;
-  gather_rows_kernel<<<(unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s>>>(
+  launch_kernel(gather_rows_kernel, (unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s, 
       (const __nv_bfloat16*)src, ld_src, idx, n_rows, n_cols, (__nv_bfloat16*)dst, ld_dst, dst_col0, vec, blk,
       blk_stride, blk_off);
   if (cudaGetLastError() != cudaSuccess) return 5;
@@ -84,7 +88,7 @@ int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int3
                      int64_t ld_dst, cudaStream_t s) {
   if (n_rows <= 0 || n_idx <= 0) return 0;
   dim3 grid((unsigned)((n_idx + 255) / 256), (unsigned)(n_rows < 1024 ? n_rows : 1024));
-  gather_cols_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)src, ld_src, n_rows, idx, n_idx,
+  launch_kernel(gather_cols_kernel, grid, 256, 0, s, (const __nv_bfloat16*)src, ld_src, n_rows, idx, n_idx,
                                           (__nv_bfloat16*)dst, ld_dst);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
@@ -95,7 +99,7 @@ int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, 
                    cudaStream_t s) {
   if (rows <= 0 || cols <= 0) return 0;
   dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
-  transpose_kernel<<<grid, dim3(32, 8), 0, s>>>((const __nv_bfloat16*)src, rows, cols, ld_src, (__nv_bfloat16*)dst,
+  launch_kernel(transpose_kernel, grid, dim3(32, 8), 0, s, (const __nv_bfloat16*)src, rows, cols, ld_src, (__nv_bfloat16*)dst,
                                                 ld_dst);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
@@ -109,7 +113,7 @@ int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int6
 
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s) {
   if (n <= 0) return 0;
-  add_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dst, src, n);
+  launch_kernel(add_f32_kernel, (unsigned)((n + 255) / 256), 256, 0, s, dst, src, n);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
   return 0;

@@ -60,6 +60,7 @@ template <typename T, int CPG>
 __global__ void __launch_bounds__(kE1Threads) est1_kernel(const T* __restrict__ x, int64_t n_ctx, int64_t d_in,
                                                           int64_t ldx, WaPtrs wa, int wa_fp32, int k, int mk,
                                                           int64_t d_per_split, float* __restrict__ zpart) {
+  pdl_wait();
   constexpr int MKP = 8 * CPG;  // padded column count
   extern __shared__ float e1_smem[];
   float* xs = e1_smem;                              // [kE1Chunk][kE1Rows + 4]
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(kE1Threads) est1_kernel(const T* __restrict__ 
 
 // Z[t][j] = sum_s zpart[s][t][j], s in increasing order. Written into split slot 0.
 __global__ void est_reduce_kernel(float* zpart, int n_split, int64_t n) {
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float acc = zpart[i];
@@ -160,6 +162,7 @@ template <int K>
 __global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
     est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx, const void* wb_g, const void* wb_u, int wb_fp32,
                       int64_t n_ch, float* __restrict__ scores) {
+  pdl_wait();
   __shared__ __align__(16) float zs[kE2Tok][2 * K];
   __shared__ double part[8][64];
   __shared__ double cta_sum[64];
@@ -234,6 +237,7 @@ constexpr int kGramCluster = 8;
 // shared memory) and writes G.
 __global__ void __cluster_dims__(kGramCluster, 1, 1) __launch_bounds__(256)
     est_gram_kernel(const float* __restrict__ z, int64_t n_ctx, int mk, double* __restrict__ gram) {
+  pdl_wait();
   __shared__ float zs[kGramTok][64];
   __shared__ double gpart[64 * 64];
   cg::cluster_group cluster = cg::this_cluster();
@@ -291,6 +295,7 @@ __global__ void __launch_bounds__(256) est_linear_scores_kernel(const double* __
                                                                 int wb_fp32, int n_q_heads, int n_kv_heads,
                                                                 int head_dim, int64_t n_units,
                                                                 float* __restrict__ scores) {
+  pdl_wait();
   extern __shared__ double gs[];  // [mk][mk]
   for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
     double s = 0.0;
@@ -346,11 +351,11 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
     if (x_fp32) {                                                                                             \
       auto kern = est1_kernel<float, C>;                                                                      \
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      kern<<<grid, kE1Threads, smem, s>>>((const float*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, zpart);  \
+      launch_kernel(kern, grid, kE1Threads, smem, s, (const float*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, zpart);  \
     } else {                                                                                                  \
       auto kern = est1_kernel<__nv_bfloat16, C>;                                                              \
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      kern<<<grid, kE1Threads, smem, s>>>((const __nv_bfloat16*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, \
+      launch_kernel(kern, grid, kE1Threads, smem, s, (const __nv_bfloat16*)x, n_ctx, d_in, ldx, w, wa_fp32, k, mk, dps, \
                                           zpart);                                                             \
     }                                                                                                         \
     break;                                                                                                    \
@@ -364,7 +369,7 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
   const int used = (int)grid.y;
   if (used > 1) {
     const int64_t n = n_ctx * mk;
-    est_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(zpart, used, n);
+    launch_kernel(est_reduce_kernel, (unsigned)((n + 255) / 256), 256, 0, s, zpart, used, n);
   }
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
@@ -375,9 +380,9 @@ int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, con
                       int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s) {
   const dim3 grid((unsigned)((n_ch + 63) / 64), kE2Split);
   switch (k) {
-    case 8: est_swiglu_kernel<8><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
-    case 16: est_swiglu_kernel<16><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
-    case 4: est_swiglu_kernel<4><<<grid, kE2Threads, 0, s>>>(z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 8: launch_kernel(est_swiglu_kernel<8>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 16: launch_kernel(est_swiglu_kernel<16>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
     default: return 1;
   }
   if (cudaGetLastError() != cudaSuccess) return 5;
@@ -388,7 +393,7 @@ int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, con
 int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gram, int /*n_chunks*/,
              cudaStream_t s) {
   if (mk > 64 || n_ctx <= 0) return 1;
-  est_gram_kernel<<<gram_groups(n_ctx) * kGramCluster, 256, 0, s>>>(z, n_ctx, mk, gram);
+  launch_kernel(est_gram_kernel, gram_groups(n_ctx) * kGramCluster, 256, 0, s, z, n_ctx, mk, gram);
   if (cudaGetLastError() != cudaSuccess) return 5;
   note_launch();
   return 0;
@@ -411,7 +416,7 @@ int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int 
     w.n[1] = (int64_t)n_kv_heads * head_dim;
   }
   const unsigned grid = (unsigned)((n_units + 63) / 64);
-  est_linear_scores_kernel<<<grid, 64, (size_t)mk * mk * sizeof(double), s>>>(
+  launch_kernel(est_linear_scores_kernel, grid, 64, (size_t)mk * mk * sizeof(double), s, 
       gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
       crit == 0 ? 1 : head_dim, n_units, scores);
   if (cudaGetLastError() != cudaSuccess) return 5;

@@ -11,6 +11,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdio>
+#include <vector>
 
 #include "sl_gemm.h"
 #include "sl_internal.h"
@@ -264,6 +266,7 @@ struct RedParams {
 
 // Fixed-order sum of split-K partials + the problem's epilogue (EPI_XA, EPI_F32, EPI_F32_T).
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ RedParams rp) {
+  pdl_wait();
   const RedProb& pr = rp.p[blockIdx.y];
   const int64_t total = (int64_t)pr.M * pr.N;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -348,6 +351,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above overlaps the previous kernel's tail
 
   if (warp == 0) {
     if (lane == 0) {
@@ -488,13 +492,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ CTA-pair variant
 //
-// Same roles and problem list, but a cluster of two CTAs (two SMs) computes one
-// 256-row x 256-column tile with cta_group::2 MMAs: each CTA stages its own 128 rows of
-// A and its half (128 rows) of the B tile, the even CTA issues the MMAs for both, and
-// each CTA's TMEM holds the accumulator of its 128 rows. Per SM this halves the B bytes
-// per FLOP of the one-CTA kernel. Only full-width tiles (n_mma = 256) use it.
-constexpr int kStages2 = 6;
+// Same roles and problem list, but a cluster of two CTAs (two SMs) computes one tile of
+// 256 * MH rows x 256 columns with cta_group::2 MMAs: each CTA stages its own 128 * MH
+// rows of A and its half (128 rows) of the B tile, the even CTA issues the MMAs for both,
+// and each CTA's TMEM holds the accumulators of its rows. Only full-width tiles
+// (n_mma = 256) use it.
+//   MH = 1: 256 x 256 tiles, two accumulator buffers (the epilogue of one tile overlaps
+//           the main loop of the next), six 32 KB stages.
+//   MH = 2: 512 x 256 tiles: per K step two M = 256 MMAs share the B tile, so operand
+//           bytes per FLOP drop by a quarter; one accumulator fills all 512 TMEM columns
+//           (the epilogue is not overlapped), four 48 KB stages.
 constexpr int kStageB2Bytes = 128 * kBK * 2;
+template <int MH>
+struct PairCfg {
+  static constexpr int kStages = MH == 1 ? 6 : 4;
+  static constexpr int kStageA = MH * kStageABytes;
+  static constexpr int kAccBufs = MH == 1 ? 2 : 1;
+  static constexpr int kTileM = 256 * MH;
+};
+static_assert(PairCfg<1>::kStages * (PairCfg<1>::kStageA + kStageB2Bytes) <= kStages * (kStageABytes + kStageBBytes),
+              "pair stages exceed the shared-memory budget");
+static_assert(PairCfg<2>::kStages * (PairCfg<2>::kStageA + kStageB2Bytes) <= kStages * (kStageABytes + kStageBBytes),
+              "pair stages exceed the shared-memory budget");
 
 __device__ __forceinline__ void pair_b_loads(const GemmParams& p, const Seg& sg, int tn, uint32_t rank, uint8_t* sb,
                                              uint64_t* full, int kc) {
@@ -513,16 +532,18 @@ __device__ __forceinline__ void pair_b_loads(const GemmParams& p, const Seg& sg,
   }
 }
 
+template <int MH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  using C = PairCfg<MH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smem_a = smem;
-  uint8_t* smem_b = smem + kStages2 * kStageABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + kStages2 * kStageB2Bytes);
+  uint8_t* smem_b = smem + C::kStages * C::kStageA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + C::kStages * kStageB2Bytes);
   uint64_t* full = bars;              // used in the even CTA: both CTAs' copies count here
-  uint64_t* empty = bars + kStages2;  // both CTAs: armed by the even CTA's MMA commits
-  uint64_t* tfull = bars + 2 * kStages2;
+  uint64_t* empty = bars + C::kStages;  // both CTAs: armed by the even CTA's MMA commits
+  uint64_t* tfull = bars + 2 * C::kStages;
   uint64_t* tempty = tfull + 2;       // used in the even CTA: both CTAs' epilogue threads arrive
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -536,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int cl = blockIdx.x >> 1, n_cl = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages2; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -557,6 +578,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync_all();  // the peer's barriers exist before any copy or arrive targets them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above overlaps the previous kernel's tail
 
   if (warp == 0) {
     if (lane == 0) {
@@ -573,22 +595,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int kb = 0; kb < sg.nk; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
             if (leader) {
-              mbar_arrive_expect_tx(&full[stage], 2u * (kStageABytes + kStageB2Bytes));
+              mbar_arrive_expect_tx(&full[stage], 2u * (C::kStageA + kStageB2Bytes));
               issued_mask |= 1u << stage;
               issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
             }
-            uint8_t* sa = smem_a + stage * kStageABytes;
+            uint8_t* sa = smem_a + stage * C::kStageA;
             uint8_t* sb = smem_b + stage * kStageB2Bytes;
             const int kc = kb * kBK;
-            const int arow = sg.a_row0 + ti.tm * 256 + 128 * (int)rank;
-            if (!sg.a_mn) {
-              tma_load_2d_pair(sa, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, arow);
-            } else {
-              tma_load_2d_pair(sa, &p.maps[sg.a_map], &full[stage], arow, sg.a_k0 + kc);
-              tma_load_2d_pair(sa + 8192, &p.maps[sg.a_map], &full[stage], arow + 64, sg.a_k0 + kc);
+            const int arow = sg.a_row0 + ti.tm * C::kTileM + 128 * MH * (int)rank;
+#pragma unroll
+            for (int h = 0; h < MH; ++h) {
+              uint8_t* sah = sa + h * kStageABytes;
+              if (!sg.a_mn) {
+                tma_load_2d_pair(sah, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, arow + 128 * h);
+              } else {
+                tma_load_2d_pair(sah, &p.maps[sg.a_map], &full[stage], arow + 128 * h, sg.a_k0 + kc);
+                tma_load_2d_pair(sah + 8192, &p.maps[sg.a_map], &full[stage], arow + 128 * h + 64, sg.a_k0 + kc);
+              }
             }
             pair_b_loads(p, sg, ti.tn, rank, sb, &full[stage], kc);
-            if (++stage == kStages2) {
+            if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1;
             }
@@ -597,7 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     producer_done:
       // The even CTA's barriers count both CTAs' copies: wait for every stage it armed.
-      for (int s = 0; s < kStages2; ++s)
+      for (int s = 0; s < C::kStages; ++s)
         if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
@@ -612,7 +638,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int n0 = ti.tn * pr.tile_cols;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN * MH);
         uint32_t accumulate = 0;
         for (int s = 0; s < pr.nseg; ++s) {
           const Seg& sg = pr.seg[s];
@@ -621,27 +647,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int kb = 0; kb < sg.nk; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEV_TIMEOUT_MMA)) goto mma_done;
             tc_fence_after();
-            const uint32_t sa = smem_u32(smem_a + stage * kStageABytes);
+            const uint32_t sa = smem_u32(smem_a + stage * C::kStageA);
             const uint32_t sb = smem_u32(smem_b + stage * kStageB2Bytes);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t ad = sg.a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024)
-                                          : smem_desc_sw128(sa + k * 32, 16, 1024);
               const uint64_t bd = sg.b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024)
                                           : smem_desc_sw128(sb + k * 32, 16, 1024);
-              umma_bf16_pair(d_tmem, ad, bd, idesc, accumulate);
+#pragma unroll
+              for (int h = 0; h < MH; ++h) {
+                const uint32_t sah = sa + h * kStageABytes;
+                const uint64_t ad = sg.a_mn ? smem_desc_sw128(sah + k * 2048, 8192, 1024)
+                                            : smem_desc_sw128(sah + k * 32, 16, 1024);
+                umma_bf16_pair(d_tmem + h * kBN, ad, bd, idesc, accumulate);
+              }
               accumulate = 1;
             }
             umma_commit_pair_mc(&empty[stage], 0x3);
-            if (++stage == kStages2) {
+            if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1;
             }
           }
         }
         umma_commit_pair_mc(&tfull[acc], 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
       }
     mma_done:
       umma_commit_pair(drain);
@@ -660,14 +692,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const Prob& pr = p.probs[ti.prob];
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
-      epilogue_tile(pr, ti.tm * 256 + 128 * (int)rank, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33,
-                    half);
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN * MH);
+#pragma unroll 1
+      for (int h = 0; h < MH; ++h)
+        epilogue_tile(pr, ti.tm * C::kTileM + 128 * MH * (int)rank + 128 * h, ti.tn * pr.tile_cols, r,
+                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half);
       __syncwarp();
       tc_fence_before();
       mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
     }
   }
 
@@ -795,8 +831,15 @@ Seg* GemmBuilder::seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b
 
 int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles) {
   if (M <= 0 || kblocks <= 1) return 1;
+  if (target_tiles <= 0) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+    target_tiles = sms;
+  }
   const int64_t tm = (M + kBM - 1) / kBM;
-  int64_t s = (target_tiles + tm - 1) / tm;
+  // the largest split that still fits one wave of `target_tiles` tiles
+  int64_t s = target_tiles / tm;
   const int64_t smax = kblocks / 2;
   if (s > smax) s = smax;
   if (s > 32) s = 32;
@@ -823,10 +866,57 @@ void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int ro
   b.row_step = row_step;
 }
 
+// Rows per CTA pair (256 or 512) for a pair-eligible launch: the one with the smaller
+// estimated makespan of the round-robin persistent schedule over `pairs` CTA pairs. Cost
+// of a tile in 64-wide k-block units of a 256 x 256 tile: a 512-row tile moves 1.5x the
+// operand bytes of a 256-row tile for twice the FLOPs, and its epilogue is not
+// overlapped; a 256-row tile's epilogue overlaps the next tile's main loop and only shows
+// when that main loop is shorter. Epilogue weights (same units, measured on B200): plain
+// stores 4 per 256 rows; column scatter 8; the SwiGLU backward, which reads g and u from
+// global memory row by row, 20. SL_PAIR_MH=1|2 forces the choice.
+static int choose_pair_mh(const GemmParams& P, int nprob, int pairs) {
+  static const int forced = [] {
+    const char* e = getenv("SL_PAIR_MH");
+    return e ? atoi(e) : 0;
+  }();
+  if (forced == 1 || forced == 2) return forced;
+  double best = 0.0;
+  int best_mh = 1;
+  std::vector<double> load((size_t)pairs);
+  for (int mh = 1; mh <= 2; ++mh) {
+    std::fill(load.begin(), load.end(), 0.0);
+    long long t = 0;
+    for (int i = 0; i < nprob; ++i) {
+      const Prob& pr = P.probs[i];
+      if (pr.M <= 0 || pr.N <= 0) continue;
+      const int tm = (pr.M + 256 * mh - 1) / (256 * mh);
+      const int tn = (pr.N + pr.tile_cols - 1) / pr.tile_cols;
+      const double epi = pr.epi == EPI_DSWIGLU ? 20.0 : (pr.col_map ? 8.0 : 4.0);
+      for (int n = 0; n < tn; ++n) {
+        int kb = 0;
+        for (int sg = 0; sg < pr.nseg; ++sg)
+          if (n * pr.tile_cols < pr.seg[sg].n_limit) kb += pr.seg[sg].nk;
+        const double cost = mh == 1 ? std::max<double>(kb, epi) : 1.5 * kb + 2.0 * epi;
+        for (int m = 0; m < tm; ++m) load[(size_t)(t++ % pairs)] += cost;
+      }
+    }
+    const double span = *std::max_element(load.begin(), load.end());
+    if (mh == 1 || span < best) {
+      best = span;
+      best_mh = mh;
+    }
+  }
+  return best_mh;
+}
+
 int GemmBuilder::launch(int* err, cudaStream_t stream) {
   if (status != 0) return status;
   const bool pair = pair_eligible();
-  const int tile_m = pair ? 2 * kBM : kBM;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int mh = pair ? choose_pair_mh(params, nprob, std::max(1, sms / 2)) : 1;
+  const int tile_m = pair ? 256 * mh : kBM;
   if (pair) {
     // each CTA of a pair stages 128 rows of a 256-row K-major B source: re-encode those
     // maps with a 128-row box (shared by every source that uses the same map)
@@ -892,22 +982,41 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
         cudaSuccess)
       return 5;
-    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+    if (cudaFuncSetAttribute(gemm_pair_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+        cudaSuccess)
+      return 5;
+    if (cudaFuncSetAttribute(gemm_pair_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
         cudaSuccess)
       return 5;
     smem_set = 1;
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const bool prof = profiling_on();
+#ifdef SL_PROFILE_DUMP
+  if (prof) {
+    // per-launch description for the profiling dump: problem shapes and MMA work issued
+    char buf[1024];
+    int o = snprintf(buf, sizeof(buf), "%s%d tiles=%d", pair ? "pair" : "1cta", mh, total);
+    double issued = 0.0;
+    for (int i = 0; i < nprob && o < (int)sizeof(buf) - 96; ++i) {
+      const Prob& pr = params.probs[i];
+      o += snprintf(buf + o, sizeof(buf) - o, " | M=%d N=%d nmma=%d tc=%d kb=%d ks=%d epi=%d segs=%d", pr.M, pr.N,
+                    pr.n_mma, pr.tile_cols, pr.kblocks, pr.ksplit, pr.epi, pr.nseg);
+      issued += 2.0 * pr.tiles_m * tile_m * pr.tiles_n * pr.n_mma * (double)pr.kblocks * kBK;
+    }
+    snprintf(buf + o, sizeof(buf) - o, " | issued_gflop=%.2f", issued / 1e9);
+    gemm_note(buf);
+  }
+#endif
   if (prof) gemm_events(stream, true);
   if (pair) {
     const int clusters = std::min(total, sms / 2);
-    gemm_pair_kernel<<<2 * clusters, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+    if (mh == 2)
+      launch_kernel(gemm_pair_kernel<2>, 2 * clusters, kGemmThreads, kGemmSmemBytes, stream, params);
+    else
+      launch_kernel(gemm_pair_kernel<1>, 2 * clusters, kGemmThreads, kGemmSmemBytes, stream, params);
   } else {
     const int grid = total < sms ? total : sms;
-    gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(params);
+    launch_kernel(gemm_kernel, grid, kGemmThreads, kGemmSmemBytes, stream, params);
   }
   if (cudaGetLastError() != cudaSuccess) return 5;
   if (prof) gemm_events(stream, false);
@@ -928,7 +1037,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   }
   if (nred) {
     const unsigned gx = (unsigned)std::min<int64_t>((maxmn + 255) / 256, 1184);
-    splitk_reduce_kernel<<<dim3(gx, nred), 256, 0, stream>>>(rp);
+    launch_kernel(splitk_reduce_kernel, dim3(gx, nred), 256, 0, stream, rp);
     if (cudaGetLastError() != cudaSuccess) return 5;
     note_launch();
   }

@@ -1,17 +1,50 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "sl_gemm.h"
 
 namespace sl {
 
+// ---- programmatic dependent launch
+// Every library kernel is launched with programmatic stream serialisation: the launch of
+// the next kernel in the stream is already in flight when the kernel before it retires, and
+// its CTAs run their prologue (barrier set-up, tensor-memory allocation) before waiting in
+// pdl_wait() until that kernel has completed and its memory writes are visible. pdl_wait()
+// therefore comes before the first global-memory read or write of every kernel. No kernel
+// signals its dependents early (that measured slower: the waiting CTAs compete with the
+// running grid). SL_PDL=0 in the environment turns it off.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Launch accounting for the optional profiling hook (sl_profile_enable / sl_profile_read).
 void note_launch(int n = 1);
 bool profiling_on();
 void gemm_events(cudaStream_t s, bool start);
+#ifdef SL_PROFILE_DUMP
+// Description of the next GEMM-engine launch, printed with its time by sl_profile_read.
+void gemm_note(const char* desc);
+#endif
 
 // Builds the parameter block of one grouped GEMM launch on the host.
 struct GemmBuilder {
@@ -41,9 +74,10 @@ struct GemmBuilder {
   int launch(int* err, cudaStream_t stream);
 };
 
-// Split-K factor for a skinny problem with M rows and `kblocks` 64-wide K blocks, aiming
-// at about `target_tiles` tiles (about one wave); 1 = no split.
-int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 160);
+// Split-K factor for a skinny problem with M rows and `kblocks` 64-wide K blocks: the
+// largest split whose tiles fit one wave of `target_tiles` CTAs (default: the current
+// device's SM count); 1 = no split.
+int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 0);
 
 // ---- estimator (sl_estimator.cu)
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,

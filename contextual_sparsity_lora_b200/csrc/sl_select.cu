@@ -55,6 +55,7 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores, int n, int n_keep,
                                                              int32_t* __restrict__ sigma, int hpg, int head_dim,
                                                              int n_wide, int32_t* __restrict__ sigma_wide) {
+  pdl_wait();
   extern __shared__ uint32_t sel_smem[];
   uint32_t* keys = sel_smem;                                    // [n]
   uint8_t* keep = reinterpret_cast<uint8_t*>(keys + n);         // [n]
@@ -175,7 +176,7 @@ int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sig
     cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxN * 5 + 64);
     attr = true;
   }
-  select_kernel<<<1, kSelThreads, (smem + 15) / 16 * 16, s>>>(scores, (int)n, (int)n_keep, sigma,
+  launch_kernel(select_kernel, 1, kSelThreads, (smem + 15) / 16 * 16, s, scores, (int)n, (int)n_keep, sigma,
                                                                sigma_wide ? heads_per_group : 0, head_dim,
                                                                (int)n_wide, sigma_wide);
   if (n_keep_wide_out) *n_keep_wide_out = sigma_wide ? n_keep * heads_per_group : 0;
