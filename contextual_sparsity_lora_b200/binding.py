@@ -38,7 +38,7 @@ class SlWorkspaceC(ctypes.Structure):
 class SlLinearC(ctypes.Structure):
     _fields_ = [("w", c_void_p), ("w_t", c_void_p), ("d_in", c_int64), ("d_out", c_int64), ("slice", c_int32),
                 ("r", c_int32), ("lora_a", c_void_p), ("lora_b", c_void_p), ("lora_scale", c_float),
-                ("pad_", c_int32)]
+                ("pad_", c_int32), ("w_kept", c_void_p)]
 
 
 class SlChannelsC(ctypes.Structure):
@@ -149,10 +149,11 @@ class Workspace:
         return int(v.value)
 
 
-def linear_desc(w, lora_a, lora_b, lora_scale, slice_kind, w_t=None) -> SlLinearC:
+def linear_desc(w, lora_a, lora_b, lora_scale, slice_kind, w_t=None, w_kept=None) -> SlLinearC:
     d_out, d_in = w.shape
     return SlLinearC(w.data_ptr(), None if w_t is None else w_t.data_ptr(), d_in, d_out, slice_kind,
-                     lora_a.shape[0], lora_a.data_ptr(), lora_b.data_ptr(), float(lora_scale), 0)
+                     lora_a.shape[0], lora_a.data_ptr(), lora_b.data_ptr(), float(lora_scale), 0,
+                     None if w_kept is None else w_kept.data_ptr())
 
 
 def channels_desc(sigma, n_keep) -> SlChannelsC:

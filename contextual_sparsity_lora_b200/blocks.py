@@ -59,21 +59,33 @@ class FFNBlock:
         self.dA_g, self.dB_g = _empty((r, D), f32, device), _empty((F, r), f32, device)
         self.dA_u, self.dB_u = _empty((r, D), f32, device), _empty((F, r), f32, device)
         self.dx = _empty((T, D), bf, device)
+        # kept rows of the sliced weights, rebuilt once per step and shared by the forward
+        # and backward calls (the weights themselves when nothing is dropped)
+        if self.dense:
+            self.Wg_k, self.Wu_k, self.Wd_k = self.Wg, self.Wu, self.Wd_t
+        else:
+            nk = self.n_keep
+            self.Wg_k, self.Wu_k, self.Wd_k = (_empty((nk, D), bf, device) for _ in range(3))
         self._descs()
 
     def _descs(self):
         s = self.scale
-        self.lin_g = B.linear_desc(self.Wg, self.Ag, self.Bg, s, B.SL_SLICE_OUT)
-        self.lin_u = B.linear_desc(self.Wu, self.Au, self.Bu, s, B.SL_SLICE_OUT)
-        self.lin_d = B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t)
+        self.lin_g = B.linear_desc(self.Wg, self.Ag, self.Bg, s, B.SL_SLICE_OUT, w_kept=self.Wg_k)
+        self.lin_u = B.linear_desc(self.Wu, self.Au, self.Bu, s, B.SL_SLICE_OUT, w_kept=self.Wu_k)
+        self.lin_d = B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t, w_kept=self.Wd_k)
         self.ch = B.channels_desc(self.sigma, self.n_keep)
 
     def select(self, x):
-        """a1 + a2 + a3 on the context rows of x (writes self.scores, self.sigma)."""
+        """a1 + a2 + a3 on the context rows of x (writes self.scores, self.sigma), then the
+        kept weight rows of gate, up (rows of W) and down (rows of W^T)."""
         xe = x if self.est_dtype == torch.bfloat16 else self.x_est
         B.sl_svd_estimate(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx, [self.WAg, self.WAu],
                           [self.WBg, self.WBu], self.k, self.scores)
         B.sl_select_channels(self.scores, self.n_keep, self.sigma)
+        kept = self.sigma[: self.n_keep]
+        B.sl_permute_rows(self.Wg, kept, self.Wg_k)
+        B.sl_permute_rows(self.Wu, kept, self.Wu_k)
+        B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
 
     def forward(self, x, x_est=None):
         """x: bf16 [n_tok, D] context-first. x_est: optional fp32 copy for an fp32 estimator."""
@@ -160,11 +172,19 @@ class AttnProjBlock:
         self.dx_o = _empty((T, self.Dq), bf, device)
         self.dx = _empty((T, D), bf, device)
         s = self.scale
+        # kept rows of the sliced weights (rows of W for q, k, v; rows of W^T for o), rebuilt
+        # once per step after the selection and shared by the forward and backward calls
+        nq, nu = self.n_keep_u * self.hpg, self.n_keep_u
+        if self.dense:
+            self.W_k = {"q": self.Wq, "k": self.Wk, "v": self.Wv, "o": self.Wo_t}
+        else:
+            self.W_k = {"q": _empty((nq, D), bf, device), "k": _empty((nu, D), bf, device),
+                        "v": _empty((nu, D), bf, device), "o": _empty((nq, D), bf, device)}
         self.lin = {
-            "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT),
-            "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT),
-            "v": B.linear_desc(self.Wv, *self.L["v"], s, B.SL_SLICE_OUT),
-            "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t),
+            "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT, w_kept=self.W_k["q"]),
+            "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT, w_kept=self.W_k["k"]),
+            "v": B.linear_desc(self.Wv, *self.L["v"], s, B.SL_SLICE_OUT, w_kept=self.W_k["v"]),
+            "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t, w_kept=self.W_k["o"]),
         }
         self.ch = {
             "q": B.channels_desc(self.sig_q, self.n_keep_u * self.hpg),
@@ -179,6 +199,9 @@ class AttnProjBlock:
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
         B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
         B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+        for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k), ("v", self.Wv, self.sig_v),
+                          ("o", self.Wo_t, self.sig_o)):
+            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
 
     def forward(self, x, x_o):
         C = self.n_ctx

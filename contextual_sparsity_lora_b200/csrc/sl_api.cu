@@ -114,7 +114,7 @@ inline int64_t rup(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 bool linear_ok(const sl_linear& L) {
   return L.w && L.d_in > 0 && L.d_out > 0 && L.lora_a && L.lora_b && L.r >= 8 && L.r <= 64 && L.r % 8 == 0 &&
-         L.d_in % 8 == 0 && L.d_out % 8 == 0 && al16(L.w) && al16(L.lora_a) && al16(L.lora_b) &&
+         L.d_in % 8 == 0 && L.d_out % 8 == 0 && al16(L.w) && al16(L.lora_a) && al16(L.lora_b) && al16(L.w_kept) &&
          (L.slice == SL_SLICE_OUT || L.slice == SL_SLICE_IN);
 }
 
@@ -509,7 +509,7 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       if (!y[i] || ldy[i] < lin[i].d_out || ldy[i] % 8 || !al16(y[i])) return SL_ERR_ALIGNMENT;
     auto carve = [&](Carver& c, void** wc, void** bs) {
       for (int i = 0; i < n_lin; ++i) {
-        wc[i] = c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        wc[i] = lin[i].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
         bs[i] = c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r);
       }
     };
@@ -522,7 +522,9 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     Carver c(ws->ptr);
     carve(c, wc, bs);
     for (int i = 0; i < n_lin; ++i) {
-      if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
+      if (lin[i].w_kept)
+        wc[i] = const_cast<void*>(lin[i].w_kept);
+      else if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
         return from_kernel(rc);
       if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r, 0, s))
         return from_kernel(rc);
@@ -572,8 +574,8 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       if (!y[i] || ldy[i] < F || ldy[i] % 8 || !al16(y[i]) || ldy[i] != ldy[0]) return SL_ERR_ALIGNMENT;
     const int64_t nt = (F + 127) / 128;  // paired tiles: 128 channels each
     auto carve = [&](Carver& c, void** wc, void** pk) {
-      wc[0] = c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
-      wc[1] = c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      wc[0] = lin[0].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      wc[1] = lin[1].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
       pk[0] = c.take<uint16_t>((size_t)nt * 256 * 64);  // sigma order
       pk[1] = c.take<uint16_t>((size_t)nt * 256 * 64);  // natural order
     };
@@ -586,8 +588,12 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     Carver c(ws->ptr);
     carve(c, wc, pk);
     const int32_t* sig = ch[0].sigma;
-    for (int i = 0; i < 2; ++i)
-      if (int rc = gather_rows_bf16(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in, 0, s)) return from_kernel(rc);
+    for (int i = 0; i < 2; ++i) {
+      if (lin[i].w_kept)
+        wc[i] = const_cast<void*>(lin[i].w_kept);
+      else if (int rc = gather_rows_bf16(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in, 0, s))
+        return from_kernel(rc);
+    }
     // LoRA B operand of a paired tile t: rows 256 t + j = [B_gate[c_j] | 0], rows 256 t + 128 + j = [0 | B_up[c_j]]
     cudaMemsetAsync(pk[0], 0, (size_t)nt * 256 * 64 * 2, s);
     cudaMemsetAsync(pk[1], 0, (size_t)nt * 256 * 64 * 2, s);
@@ -633,7 +639,7 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
     const int64_t ldc = rup(nk, 8);
     auto carve = [&](Carver& c, void** wtc, void** xc) {
-      *wtc = c.take<uint16_t>((size_t)nk * L.d_out);
+      *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : c.take<uint16_t>((size_t)nk * L.d_out);
       *xc = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * ldc) : nullptr;
     };
     void *wtc, *xc;
@@ -644,7 +650,9 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
     Carver c(ws->ptr);
     carve(c, &wtc, &xc);
-    if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s)) return from_kernel(rc);
+    if (!L.w_kept)
+      if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s))
+        return from_kernel(rc);
     if (xc)
       if (int rc = gather_cols_bf16(x, ldx, C, ch[0].sigma, nk, xc, ldc, s)) return from_kernel(rc);
     GemmBuilder gb;
@@ -705,7 +713,7 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
     auto carve = [&](Carver& c, void** wc, void** dyc) {
       for (int i = 0; i < n_lin; ++i) {
-        wc[i] = c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        wc[i] = lin[i].w_kept ? const_cast<void*>(lin[i].w_kept) : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
         dyc[i] = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * rup(ch[i].n_keep, 8)) : nullptr;
       }
     };
@@ -718,8 +726,9 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     Carver c(ws->ptr);
     carve(c, wc, dyc);
     for (int i = 0; i < n_lin; ++i) {
-      if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
-        return from_kernel(rc);
+      if (!lin[i].w_kept)
+        if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
+          return from_kernel(rc);
       if (dyc[i])
         if (int rc = gather_cols_bf16(dy[i], ld_dy[i], C, ch[i].sigma, ch[i].n_keep, dyc[i], rup(ch[i].n_keep, 8), s))
           return from_kernel(rc);
@@ -771,7 +780,7 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   }
   const int64_t nk = ch[0].n_keep;
   auto carve = [&](Carver& c, void** wtc, void** at, void** ats) {
-    *wtc = c.take<uint16_t>((size_t)nk * L.d_out);
+    *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : c.take<uint16_t>((size_t)nk * L.d_out);
     *at = c.take<uint16_t>((size_t)d_in * L.r);
     *ats = c.take<uint16_t>((size_t)d_in * L.r);
   };
@@ -783,7 +792,9 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   }
   Carver c(ws->ptr);
   carve(c, &wtc, &at, &ats);
-  if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s)) return from_kernel(rc);
+  if (!L.w_kept)
+    if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s))
+      return from_kernel(rc);
   if (int rc = transpose_bf16(L.lora_a, L.r, d_in, d_in, at, L.r, s)) return from_kernel(rc);
   if (int rc = gather_rows_bf16(at, L.r, ch[0].sigma, d_in, L.r, ats, L.r, 0, s)) return from_kernel(rc);
   GemmBuilder gb;

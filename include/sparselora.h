@@ -16,8 +16,8 @@
  * ---------------------------------------
  * - All tensor pointers are CUDA device pointers owned by the caller. The library
  *   never allocates device memory, never synchronises the stream and keeps no
- *   global state besides lazily set kernel attributes. Scratch memory comes from
- *   the caller's sl_workspace.
+ *   global state besides lazily set kernel attributes (and the fixed scratch array
+ *   of sl_svd_estimate_noalloc). Scratch memory comes from the caller's sl_workspace.
  * - Matrices are row-major with an explicit leading dimension in elements.
  *   Frozen weights use nn.Linear storage order W[d_out, d_in] (the pages' math
  *   convention is y = x W_math with W_math = W^T). LoRA: A[r, d_in], B[d_out, r],
@@ -106,6 +106,14 @@ typedef struct {
   const void* lora_b; /* bf16 [d_out, r] */
   float lora_scale;   /* alpha / r */
   int32_t pad_;
+  /* Optional (may be NULL): the kept rows of the sliced weight for the channel set passed
+   * with the call, row-major and dense: SL_SLICE_OUT: w[sigma[j], :] for j < n_keep
+   * ([n_keep, d_in]); SL_SLICE_IN: w_t[sigma[j], :] ([n_keep, d_out]). The forward and
+   * the backward of one step use the same rows, so a caller that builds them once per
+   * step (sl_permute_rows with the first n_keep entries of sigma) saves both calls their
+   * own gather into the workspace. With keep ratio 1 and the identity sigma it is w
+   * (w_t) itself. The caller keeps it consistent with sigma; 16-byte aligned. */
+  const void* w_kept;
 } sl_linear;
 
 /* The channel set applied to one projection's sliced side. */
