@@ -87,16 +87,49 @@ __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* v
   }
 }
 
+// Bulk-store path of the bf16 epilogues: the warp's 32 rows x 32 columns of one output go
+// through one of the warp's two 2 KB shared-memory boxes (row-major bf16, lane = row) and
+// leave with one bulk tensor store issued by lane 0, so the warp moves on while the copy
+// drains and every write is a whole line. Rows and columns outside the problem are clipped
+// by the tensor map (it covers exactly the problem's M x N block). Lane 0 waits, before a
+// box is rewritten, until at most one of its bulk groups (the other box) is still reading.
+// Warp-collective; the caller skips warps whose rows all lie outside the problem.
+__device__ __forceinline__ void bulk_store_chunk(const CUtensorMap* map, uint8_t* bufs, int& sb, const float* v,
+                                                 int col, int row0) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  uint8_t* buf = bufs + sb * 2048;
+  uint4* d = reinterpret_cast<uint4*>(buf + lane * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, buf, col, row0);
+    bulk_commit();
+  }
+  sb ^= 1;
+}
+
 // Epilogue of one tile for one thread (one output row). All tcgen05.ld are
 // executed by every lane of the warp (they are warp-collective).
 // `half` selects the 32-column chunks this warp handles (even or odd); the other epilogue
 // warp on the same TMEM lane quarter takes the rest.
-__device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb, float* stage, int half) {
+__device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, int n0, int r, uint32_t tb,
+                              float* stage, int half, int& sb) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
   float v[32];
   uint32_t raw[32];
+  // bulk tensor stores: warp-uniform; rows of this warp start at wrow0 (problem-local)
+  const bool bulk = pr.omap[0] >= 0;
+  const int wrow0 = m0 + (r & ~31);
+  const bool wlive = wrow0 < pr.M;
+  uint8_t* bufs = reinterpret_cast<uint8_t*>(stage);
 
   if (pr.epi == EPI_SWIGLU) {
     const int ncols = min(128, pr.N - n0);
@@ -111,12 +144,21 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
       __syncwarp();
       tmem_ld32(tb + 128 + c0, raw);
       tmem_ld_wait();
-      if (!rv) continue;
       const int n = min(32, ncols - c0);
-      const int64_t off = orow * pr.ld0 + n0 + c0;
-      const bool vec = ((off & 7) == 0);
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);  // u
+      if (bulk) {
+        if (!wlive) continue;
+        bulk_store_chunk(&maps[pr.omap[0]], bufs, sb, g, n0 + c0, wrow0);
+        bulk_store_chunk(&maps[pr.omap[1]], bufs, sb, v, n0 + c0, wrow0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = silu_f(g[i]) * v[i];
+        bulk_store_chunk(&maps[pr.omap[2]], bufs, sb, v, n0 + c0, wrow0);
+        continue;
+      }
+      if (!rv) continue;
+      const int64_t off = orow * pr.ld0 + n0 + c0;
+      const bool vec = ((off & 7) == 0);
       store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out0) + off, g, n, vec);
       store_bf16_row(reinterpret_cast<__nv_bfloat16*>(pr.out1) + off, v, n, vec);
 #pragma unroll
@@ -136,7 +178,10 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
     if (pr.epi == EPI_BF16 && pr.col_map) {
       // Scatter through a 32 x 33 shared-memory transpose: each store instruction then
       // writes 32 columns of one row (a few sectors) instead of one column of 32 rows.
+      // (The transpose buffer is also the bulk-store boxes: let pending bulk reads finish.)
       const int lane = r & 31;
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
 #pragma unroll
       for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(raw[i]) * pr.a0;
       __syncwarp();
@@ -154,9 +199,40 @@ __device__ void epilogue_tile(const Prob& pr, int m0, int n0, int r, uint32_t tb
       __syncwarp();
       continue;
     }
-    if (!rv) continue;
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+    if (bulk && pr.epi == EPI_BF16) {
+      if (!wlive) continue;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= pr.a0;
+      bulk_store_chunk(&maps[pr.omap[0]], bufs, sb, v, n0 + c0, wrow0);
+      continue;
+    }
+    if (bulk && pr.epi == EPI_DSWIGLU) {
+      if (!wlive) continue;
+      float g[32], u[32];
+      if (rv) {
+        const int64_t aoff = orow * pr.ld_aux + n0 + c0;
+        const bool vec = (aoff & 7) == 0;
+        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux0) + aoff, g, n, vec);
+        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux1) + aoff, u, n, vec);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) g[i] = u[i] = 0.f;
+      }
+      float dg[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float sg = 1.0f / (1.0f + __expf(-g[i]));
+        const float dh = v[i];
+        dg[i] = dh * u[i] * (sg * (1.0f + g[i] * (1.0f - sg)));
+        v[i] = dh * g[i] * sg;  // du = dh * SiLU(g)
+      }
+      bulk_store_chunk(&maps[pr.omap[0]], bufs, sb, dg, n0 + c0, wrow0);
+      bulk_store_chunk(&maps[pr.omap[1]], bufs, sb, v, n0 + c0, wrow0);
+      continue;
+    }
+    if (!rv) continue;
     switch (pr.epi) {
       case EPI_BF16: {
 #pragma unroll
@@ -461,7 +537,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;   // which 32-column chunks of the tile
     const int r = q * 32 + lane;
-    int acc = 0;
+    int acc = 0, sbuf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
       const TileInfo ti = decode_tile(p, t);
@@ -472,13 +548,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       if (pr.ksplit > 1)
         epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb, half);
       else
-        epilogue_tile(pr, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33, half);
+        epilogue_tile(pr, p.maps, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33, half,
+                      sbuf);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_all();  // bulk stores complete before the CTA's shared memory goes away
   }
 
   tc_fence_before();
@@ -685,7 +763,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int r = q * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    int acc = 0;
+    int acc = 0, sbuf = 0;
     uint32_t acc_phase = 0;
     for (int t = cl; t < p.total_tiles; t += n_cl) {
       const TileInfo ti = decode_tile(p, t);
@@ -695,8 +773,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN * MH);
 #pragma unroll 1
       for (int h = 0; h < MH; ++h)
-        epilogue_tile(pr, ti.tm * C::kTileM + 128 * MH * (int)rank + 128 * h, ti.tn * pr.tile_cols, r,
-                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half);
+        epilogue_tile(pr, p.maps, ti.tm * C::kTileM + 128 * MH * (int)rank + 128 * h, ti.tn * pr.tile_cols, r,
+                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half, sbuf);
       __syncwarp();
       tc_fence_before();
       mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
@@ -705,6 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_all();  // bulk stores complete before the CTA's shared memory goes away
   }
 
   tc_fence_before();
@@ -770,6 +849,56 @@ int GemmBuilder::map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, in
   }
   specs[nmaps] = MapSpec{ptr, rows, cols, ld, box_rows};
   return nmaps++;
+}
+
+// Tensor map of a bf16 output block [rows, cols] (ld elements) for 32 x 32 bulk stores;
+// -1 when it cannot be encoded (the epilogue then stores per thread).
+int GemmBuilder::map_out(void* ptr, int64_t rows, int64_t cols, int64_t ld) {
+  if (nmaps >= kMaxMaps || !ptr || rows <= 0 || cols <= 0 || ld < cols || (reinterpret_cast<uintptr_t>(ptr) & 15) ||
+      (ld % 8))
+    return -1;
+  auto enc = get_encode();
+  if (!enc) return -1;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&params.maps[nmaps], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, gdim, gstride, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return -1;
+  specs[nmaps] = MapSpec{ptr, rows, cols, ld, 32};
+  return nmaps++;
+}
+
+// bf16 epilogues without row or column maps store through bulk tensor copies unless
+// SL_GEMM_BULK_STORE=0.
+void GemmBuilder::attach_output_maps() {
+  static const bool disabled = [] {
+    const char* e = getenv("SL_GEMM_BULK_STORE");
+    return e && e[0] == '0';
+  }();
+  for (int i = 0; i < nprob; ++i) {
+    Prob& pr = params.probs[i];
+    for (int k = 0; k < 4; ++k) pr.omap[k] = -1;
+    const bool eligible = pr.ksplit <= 1 && !pr.row_map && pr.M > 0 && pr.N > 0 &&
+                          ((pr.epi == EPI_BF16 && !pr.col_map) || pr.epi == EPI_SWIGLU || pr.epi == EPI_DSWIGLU);
+    if (disabled || !eligible) continue;
+    const int nout = pr.epi == EPI_SWIGLU ? 3 : (pr.epi == EPI_DSWIGLU ? 2 : 1);
+    void* outs[3] = {pr.out0, pr.out1, pr.out2};
+    int idx[3] = {-1, -1, -1};
+    const int saved = nmaps;
+    bool ok = true;
+    for (int k = 0; k < nout && ok; ++k) {
+      idx[k] = map_out(static_cast<uint16_t*>(outs[k]) + (int64_t)pr.out_row0 * pr.ld0, pr.M, pr.N, pr.ld0);
+      ok = idx[k] >= 0;
+    }
+    if (!ok) {
+      nmaps = saved;
+      continue;
+    }
+    for (int k = 0; k < nout; ++k) pr.omap[k] = (int8_t)idx[k];
+  }
 }
 
 bool GemmBuilder::pair_eligible() const {
@@ -977,6 +1106,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   params.total_tiles = total;
   params.err = err;
   if (total == 0) return 0;
+  attach_output_maps();
   static int smem_set = 0;
   if (!smem_set) {
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=

@@ -65,6 +65,9 @@ struct GemmBuilder {
   // bf16 row-major matrix [rows, cols] with leading dimension ld (elements);
   // the TMA box is 64 columns x box_rows rows, 128-byte swizzled, zero fill.
   int map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows);
+  // bf16 output block for the epilogue's 32 x 32 bulk tensor stores; -1 if not encodable
+  int map_out(void* ptr, int64_t rows, int64_t cols, int64_t ld);
+  void attach_output_maps();
   Prob* add(int M, int N, int tile_cols, int n_mma);
   // K is the segment's K extent; n_limit = output column limit (use N or more for "always").
   Seg* seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b_mn, int b_k0, int K, int n_limit);
