@@ -217,6 +217,50 @@ def time_steps(fn, K, W, world, device):
     return max_over_ranks(ms, world, device)
 
 
+def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
+    """Device time of the selection stages of both blocks, each captured alone in a CUDA
+    graph and replayed `reps` times: a1 (estimator stage 1, the tensor-core launch of
+    sl_svd_estimate, event-timed in a profiled copy), a2 (the rest of sl_svd_estimate: the
+    criterion), a3 (sl_select_channels) and the per-step compaction of the kept weight rows."""
+    from contextual_sparsity_lora_b200 import binding as B
+
+    def graph_us(fn):
+        fn()
+        g = capture_graph(fn, warm=False)
+        return time_steps(g.replay, reps, 3, 1, device) / reps * 1e3
+
+    def a1_us(fn):
+        B.sl_profile_read()
+        B.sl_profile_enable(True)
+        g = capture_graph(fn, warm=False)
+        B.sl_profile_enable(False)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        _, n_gemm, ms = B.sl_profile_read()
+        del g
+        return ms * 1e3 if n_gemm == 1 else None
+
+    out = {}
+    total = 0.0
+    for name, blk, x in (("attn", attn, s["x"]), ("ffn", ffn, s["ffn_x"])):
+        C, D = blk.n_ctx, x.shape[1]
+        est = graph_us(lambda: blk.estimate(x))
+        a1 = a1_us(lambda: blk.estimate(x))
+        sel = graph_us(blk.choose)
+        comp = graph_us(blk.compact)
+        n_proj = 3 if name == "attn" else 2
+        a1_bytes = C * D * 2 + n_proj * D * blk.k * 2  # X_ctx once, plus the rank-k factors W_A
+        out[name] = {"a1_a2_estimate_us": est, "a1_stage1_us": a1,
+                     "a1_bytes": a1_bytes, "a1_GBs": a1_bytes / (a1 * 1e3) if a1 else None,
+                     "a1_frac_of_hbm": a1_bytes / (a1 * 1e3) / hbm_gbs if a1 else None,
+                     "a2_criterion_us": est - a1 if a1 else None, "a3_select_us": sel, "compact_weights_us": comp}
+        total += est + sel
+    out["estimator_and_select_pct_of_step"] = 100.0 * total / (step_ms * 1e3)
+    out["timing"] = "each stage alone in a CUDA graph, replayed; device time between events"
+    return out
+
+
 def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
     """The fp64 oracle on the host cores over a bounded sample: the last ``n_tokens``
     tokens of the first sequence (context and output tokens in the workload's proportion
@@ -348,17 +392,30 @@ def main():
     prof_ms = time_steps(prof_graph.replay, args.steps, args.warmup, world, device)
     torch.cuda.synchronize()
     # launches counted while the profiled copy was captured (the same kernels as the
-    # headline graph); GEMM-engine durations of its last replay
+    # headline graph); GEMM-engine durations of its last replay, per launch and in total
+    per_launch = B.sl_profile_launches()
     n_launch_step, n_gemm, gemm_ms = B.sl_profile_read()
+    pair_ms = sum(m for m, k in per_launch if k > 0)
+    pair_n = sum(1 for _, k in per_launch if k > 0)
+    skinny_ms = sum(m for m, k in per_launch if k == 0)
     del prof_graph
     n_launch = n_launch_step * args.steps
     ms_step = ms / args.steps
     value = world * T / (ms_step / 1e3)
     fl = algorithmic_flops(ac, fc, C, args.ratio, dense=False)
-    gemm_flops = fl["main"] + fl["lora"]   # per step; gemm_ms is per step
+    # dominant kernel: the CTA-pair GEMM launches (the sliced main-branch products with the
+    # LoRA up-projections fused as K extensions: y += xa_s B^T, dx += dya_s A, i.e. one third
+    # of the LoRA FLOPs); the one-CTA launches (rank-r LoRA products, estimator stage 1)
+    # are HBM-bound and reported apart
+    pair_flops = fl["main"] + fl["lora"] / 3.0
     peaks, src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    achieved = pair_flops / (pair_ms / 1e3) / 1e12 if pair_ms > 0 else None
+    skinny_bytes = flops.lora_skinny_bytes([(T, ac.hidden, (ac.n_q_heads * ac.head_dim, 2 * ac.n_kv_heads * ac.head_dim)),
+                                            (T, ac.n_q_heads * ac.head_dim, (ac.hidden,)),
+                                            (T, fc.hidden, (2 * fc.inter,)), (T, fc.inter, (fc.hidden,))])
+    skinny_bytes += 2 * C * ac.hidden * 2  # estimator stage 1 reads X_ctx once per block
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -367,20 +424,30 @@ def main():
                    "context_tokens_per_rank": C, "keep_ratio": args.ratio, "lora_rank": ac.r,
                    "estimator_rank": ac.k, "parallelism": f"replicas{world}",
                    "l2": "per-step working set ~1.4 GB > 126 MB L2; no flush"},
-        "roofline": {"bound": "tensor", "kernel": "sl::gemm_kernel (grouped tcgen05 GEMM engine)",
+        "roofline": {"bound": "tensor", "kernel": "sl::gemm_pair_kernel (CTA-pair tcgen05 GEMM: sliced products)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": None,
                      "peak_source": f"{src} bf16_tflops_sustained",
-                     "gemm_ms_per_step": gemm_ms, "gemm_launches_per_step": n_gemm,
+                     "algorithmic_tflop_per_launch": pair_flops / 1e12 / max(pair_n, 1),
+                     "launches_per_step": pair_n, "ms_per_launch": pair_ms / max(pair_n, 1),
+                     "gemm_engine_ms_per_step": gemm_ms, "gemm_engine_launches_per_step": n_gemm,
+                     "skinny_lora_and_stage1": {"bound": "hbm", "ms_per_step": skinny_ms,
+                                                "launches_per_step": n_gemm - pair_n,
+                                                "algorithmic_bytes_per_step": skinny_bytes,
+                                                "achieved_GBs": skinny_bytes / (skinny_ms * 1e6) if skinny_ms else None,
+                                                "peak_GBs": hbm,
+                                                "frac": skinny_bytes / (skinny_ms * 1e6) / hbm if skinny_ms else None},
                      "timing": "event pair around each GEMM-engine launch, in a separately captured "
                                "copy of the step replayed over its own timed steps",
                      "profiled_step_ms": prof_ms / args.steps,
-                     "algorithmic_tflop_per_step": (fl["main"] + fl["lora"]) / 1e12},
+                     "algorithmic_tflop_per_step": pair_flops / 1e12},
         "gpu_launches": n_launch,
         "gpu_launches_per_step": n_launch_step, "cuda_graph": True,
         "effective_tflops": fl["total"] / (ms_step / 1e3) / 1e12,
         "clocks": clk.summary(),
     }
+    if rank == 0:
+        line["stages"] = stage_times(attn, ffn, step_in, 50, device, float(peaks.get("hbm_gbs", 6650.0)), ms_step)
     # dense LoRA on the same kernels (keep ratio 1, no estimator): context, not the headline
     if not args.no_dense:
         d_attn, d_ffn, _, _, _, _ = make_layer(1.0, 0, 1000 + rank, device, dense=True)

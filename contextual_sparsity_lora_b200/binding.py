@@ -28,7 +28,7 @@ SL_LORA_FWD, SL_LORA_BWD = 0, 1
 EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_init", "sl_read_device_flag",
             "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
-            "sl_svd_estimate_noalloc")
+            "sl_svd_estimate_noalloc", "sl_profile_launches")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -242,6 +242,16 @@ def sl_permute_rows(src, perm, dst):
 
 def sl_profile_enable(on: bool):
     _check("sl_profile_enable", lib().sl_profile_enable(1 if on else 0))
+
+
+def sl_profile_launches(capacity=4096):
+    """[(milliseconds, kind)] of the GEMM-engine launches recorded since the last read
+    (kind 0: one-CTA, 1: CTA pairs 256-row tiles, 2: CTA pairs 512-row tiles)."""
+    ms = (ctypes.c_double * capacity)()
+    kind = (ctypes.c_int32 * capacity)()
+    n = c_int64(0)
+    _check("sl_profile_launches", lib().sl_profile_launches(capacity, ms, kind, ctypes.byref(n)))
+    return [(float(ms[i]), int(kind[i])) for i in range(min(n.value, capacity))]
 
 
 def sl_profile_read():

@@ -75,17 +75,28 @@ class FFNBlock:
         self.lin_d = B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t, w_kept=self.Wd_k)
         self.ch = B.channels_desc(self.sigma, self.n_keep)
 
-    def select(self, x):
-        """a1 + a2 + a3 on the context rows of x (writes self.scores, self.sigma), then the
-        kept weight rows of gate, up (rows of W) and down (rows of W^T)."""
+    def estimate(self, x):
+        """a1 + a2: SwiGLU-L2 scores of the estimated gate/up outputs on x's context rows."""
         xe = x if self.est_dtype == torch.bfloat16 else self.x_est
         B.sl_svd_estimate(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx, [self.WAg, self.WAu],
                           [self.WBg, self.WBu], self.k, self.scores)
+
+    def choose(self):
+        """a3: the kept channel set (self.sigma) from self.scores."""
         B.sl_select_channels(self.scores, self.n_keep, self.sigma)
+
+    def compact(self):
+        """The kept weight rows of gate, up (rows of W) and down (rows of W^T) for this step."""
         kept = self.sigma[: self.n_keep]
         B.sl_permute_rows(self.Wg, kept, self.Wg_k)
         B.sl_permute_rows(self.Wu, kept, self.Wu_k)
         B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+
+    def select(self, x):
+        """a1 + a2 + a3 on the context rows of x, then the kept weight rows."""
+        self.estimate(x)
+        self.choose()
+        self.compact()
 
     def forward(self, x, x_est=None):
         """x: bf16 [n_tok, D] context-first. x_est: optional fp32 copy for an fp32 estimator."""
@@ -193,15 +204,27 @@ class AttnProjBlock:
             "o": B.channels_desc(self.sig_o, self.n_keep_u * self.hpg),
         }
 
-    def select(self, x):
+    def estimate(self, x):
+        """a1 + a2: QK scores over KV units and V scores from one pass over x's context rows."""
         C = self.n_ctx
         B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+
+    def choose(self):
+        """a3: the q/k set from the QK scores and the v/o set from the V scores."""
         B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
         B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+
+    def compact(self):
+        """The kept weight rows of q, k, v (rows of W) and o (rows of W^T) for this step."""
         for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k), ("v", self.Wv, self.sig_v),
                           ("o", self.Wo_t, self.sig_o)):
             B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+
+    def select(self, x):
+        self.estimate(x)
+        self.choose()
+        self.compact()
 
     def forward(self, x, x_o):
         C = self.n_ctx

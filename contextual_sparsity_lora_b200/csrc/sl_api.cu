@@ -20,6 +20,7 @@ std::atomic<bool> g_prof{false};
 std::atomic<long long> g_launches{0};
 std::mutex g_ev_mu;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_events;
+std::vector<int32_t> g_ev_kind;  // launch kind of each event pair (sl_profile_launches)
 size_t g_ev_used = 0;
 #ifdef SL_PROFILE_DUMP
 std::vector<std::string> g_notes;
@@ -45,7 +46,7 @@ void gemm_note(const char* desc) {
   g_notes[g_ev_used] = desc;
 }
 #endif
-void gemm_events(cudaStream_t s, bool start) {
+void gemm_events(cudaStream_t s, bool start, int kind) {
   std::lock_guard<std::mutex> lk(g_ev_mu);
   // Under stream capture the records become event nodes of the graph, re-recorded by
   // every replay (external records); otherwise they are plain stream records.
@@ -58,7 +59,9 @@ void gemm_events(cudaStream_t s, bool start) {
       if (cudaEventCreate(&a) != cudaSuccess) return;
       if (cudaEventCreate(&b) != cudaSuccess) return;
       g_events.emplace_back(a, b);
+      g_ev_kind.push_back(0);
     }
+    g_ev_kind[g_ev_used] = kind;
     cudaEventRecordWithFlags(g_events[g_ev_used].first, s, flags);
   } else {
     cudaEventRecordWithFlags(g_events[g_ev_used].second, s, flags);
@@ -859,6 +862,20 @@ sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launches, doub
   *gemm_launches = (int64_t)g_ev_used;
   *kernel_launches = (int64_t)g_launches.exchange(0);
   g_ev_used = 0;
+  return SL_OK;
+}
+
+sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count) {
+  if (!count || capacity < 0 || (capacity > 0 && (!ms || !kind))) return SL_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  *count = (int64_t)g_ev_used;
+  for (size_t i = 0; i < g_ev_used && (int64_t)i < capacity; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, g_events[i].first, g_events[i].second) != cudaSuccess) return SL_ERR_CUDA;
+    ms[i] = t;
+    kind[i] = g_ev_kind[i];
+  }
   return SL_OK;
 }
 

@@ -1137,7 +1137,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     gemm_note(buf);
   }
 #endif
-  if (prof) gemm_events(stream, true);
+  if (prof) gemm_events(stream, true, pair ? mh : 0);
   if (pair) {
     const int clusters = std::min(total, sms / 2);
     if (mh == 2)
@@ -1149,7 +1149,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     launch_kernel(gemm_kernel, grid, kGemmThreads, kGemmSmemBytes, stream, params);
   }
   if (cudaGetLastError() != cudaSuccess) return 5;
-  if (prof) gemm_events(stream, false);
+  if (prof) gemm_events(stream, false, pair ? mh : 0);
   note_launch();
   // reduce the split-K problems (one launch for all of them)
   RedParams rp;

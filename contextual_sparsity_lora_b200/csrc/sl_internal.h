@@ -40,7 +40,8 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 // Launch accounting for the optional profiling hook (sl_profile_enable / sl_profile_read).
 void note_launch(int n = 1);
 bool profiling_on();
-void gemm_events(cudaStream_t s, bool start);
+// kind: 0 one-CTA launch, 1 CTA-pair 256-row tiles, 2 CTA-pair 512-row tiles
+void gemm_events(cudaStream_t s, bool start, int kind = 0);
 #ifdef SL_PROFILE_DUMP
 // Description of the next GEMM-engine launch, printed with its time by sl_profile_read.
 void gemm_note(const char* desc);

@@ -67,3 +67,15 @@ def attn_proj_block(hidden: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
         + lora_fwd_bwd(dq, hidden, n_tok, r)
     est = estimator(hidden, (dq, dkv, dkv), n_ctx, k) if with_estimator else 0.0
     return dict(main=main, lora=lora, estimator=est, total=main + lora + est)
+
+
+def lora_skinny_bytes(ops) -> float:
+    """Minimum HBM bytes of the LoRA products that are not fused into the sliced GEMMs
+    (x A^T, dy B, dy^T xa, dya^T x): every large operand read once per direction.
+    ops: (n_tok, d_in, (d_out, ...)) per group of adapters sharing one input; bf16."""
+    total = 0.0
+    for n_tok, d_in, d_outs in ops:
+        total += 2.0 * n_tok * d_in * 2          # x: forward (x A^T) and backward (dya^T x)
+        total += sum(2.0 * n_tok * d for d in d_outs)  # dy: read once for dy B and dy^T xa
+    return total
+

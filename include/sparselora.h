@@ -254,6 +254,11 @@ SL_API sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const
  * since enabling) and resets them. Not thread-safe across concurrent callers. */
 SL_API sl_status sl_profile_enable(int32_t on);
 SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launches, double* gemm_ms);
+/* Per-launch view of the same GEMM-engine event pairs, without resetting them (call it
+ * before sl_profile_read): *count = launches recorded; for the first min(count, capacity)
+ * of them, in launch order, ms[i] = duration and kind[i] = 0 (one-CTA grouped launch),
+ * 1 (CTA pairs, 256-row tiles) or 2 (CTA pairs, 512-row tiles). Waits for the events. */
+SL_API sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count);
 
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
 SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream);

@@ -1,8 +1,10 @@
-"""Full LLaMA3-8B sizes in the launch configuration the benchmark times (8 x 512 tokens,
-3072 context + 1024 output, keep ratio 0.5). The estimator scores and the selection are
-checked in full; the row-independent outputs (g, u, h, y, dx of the FFN; q, k, v, y, dx_o,
-dx of the attention projections) are checked on sampled context and output rows, which
-the oracle can compute one row at a time."""
+"""Full model sizes: LLaMA3-8B in the launch configuration the benchmark times (8 x 512
+tokens, 3072 context + 1024 output, keep ratio 0.5, GQA 32/8, estimator rank 8) and the
+LLaMA2-13B layer (4 x 1024 tokens, 3072 context + 1024 output, keep ratio 0.4, MHA 40 x 128,
+FFN 13824, estimator rank 16). The estimator scores and the selection are checked in full;
+the row-independent outputs (g, u, h, y, dx of the FFN; q, k, v, y, dx_o, dx of the
+attention projections) are checked on sampled context and output rows, which the oracle
+can compute one row at a time."""
 import numpy as np
 import pytest
 import torch
@@ -22,8 +24,8 @@ def sample_rows(T, C, n, seed):
     return np.sort(np.concatenate([ctx, out]))
 
 
-def test_ffn_llama3_8b_full_size():
-    cfg = inputs.LLAMA3_8B_FFN
+@pytest.mark.parametrize("cfg", [inputs.LLAMA3_8B_FFN, inputs.LLAMA2_13B_FFN], ids=lambda c: c.name)
+def test_ffn_full_size(cfg):
     d = inputs.make_ffn_inputs(cfg, seed=1, device=DEV)
     perm = inputs.context_first_order(d["ctx_mask"])
     C = int(d["ctx_mask"].sum())
@@ -64,8 +66,8 @@ def test_ffn_llama3_8b_full_size():
     assert rel_fro(blk.dx[rows], bwd["dX"]) < BF16_TOL
 
 
-def test_attn_llama3_8b_full_size():
-    cfg = inputs.LLAMA3_8B_ATTN
+@pytest.mark.parametrize("cfg", [inputs.LLAMA3_8B_ATTN, inputs.LLAMA2_13B_ATTN], ids=lambda c: c.name)
+def test_attn_full_size(cfg):
     d = inputs.make_attn_inputs(cfg, seed=2, device=DEV)
     perm = inputs.context_first_order(d["ctx_mask"])
     C = int(d["ctx_mask"].sum())
