@@ -388,26 +388,38 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
   }
 }
 
+// The one-CTA kernel's stage ring holds B tiles of BROWS rows (or N columns): skinny
+// launches (the rank-r LoRA products, estimator stage 1) stage only the B rows they use
+// and keep 6 or 8 stages of A in flight instead of 4 in the same shared memory.
+template <int BROWS>
+struct OneCfg {
+  static constexpr int kStageB = BROWS * kBK * 2;
+  static constexpr int kStages = (sl::kStages * (kStageABytes + kStageBBytes)) / (kStageABytes + kStageB);
+};
+static_assert(OneCfg<64>::kStages == 8 && OneCfg<128>::kStages == 6 && OneCfg<256>::kStages == 4, "stage ring");
+
+template <int BROWS>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = OneCfg<BROWS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smem_a = smem;
-  uint8_t* smem_b = smem + kStages * kStageABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + kStages * kStageBBytes);
+  uint8_t* smem_b = smem + C::kStages * kStageABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_b + C::kStages * C::kStageB);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* tfull = bars + 2 * C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // 4 x [32][33]
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // kEpiWarps x [32][33]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -451,7 +463,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             issued_mask |= 1u << stage;
             issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
             uint8_t* sa = smem_a + stage * kStageABytes;
-            uint8_t* sb = smem_b + stage * kStageBBytes;
+            uint8_t* sb = smem_b + stage * C::kStageB;
             const int kc = kb * kBK;
             if (!sg.a_mn) {
               tma_load_2d(sa, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, sg.a_row0 + ti.tm * kBM);
@@ -470,7 +482,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                               sg.b_k0 + kc);
               }
             }
-            if (++stage == kStages) {
+            if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1;
             }
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
     producer_done:
       // Every issued copy must land before the CTA may exit.
-      for (int s = 0; s < kStages; ++s)
+      for (int s = 0; s < C::kStages; ++s)
         if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEV_TIMEOUT_MMA)) goto mma_done;
             tc_fence_after();
             const uint32_t sa = smem_u32(smem_a + stage * kStageABytes);
-            const uint32_t sb = smem_u32(smem_b + stage * kStageBBytes);
+            const uint32_t sb = smem_u32(smem_b + stage * C::kStageB);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
               const uint64_t ad = sg.a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024)
@@ -518,7 +530,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               accumulate = 1;
             }
             umma_commit(&empty[stage]);
-            if (++stage == kStages) {
+            if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1;
             }
@@ -1038,6 +1050,25 @@ static int choose_pair_mh(const GemmParams& P, int nprob, int pairs) {
   return best_mh;
 }
 
+// B-tile height of a one-CTA launch: the smallest stage layout (64, 128 or 256 rows) that
+// holds every problem's B sources and MMA width. SL_GEMM_BROWS=256 forces the widest.
+static int one_cta_brows(const GemmParams& P, int nprob) {
+  static const bool wide = [] {
+    const char* e = getenv("SL_GEMM_BROWS");
+    return e && atoi(e) == 256;
+  }();
+  if (wide) return 256;
+  int need = 0;
+  for (int i = 0; i < nprob; ++i) {
+    const Prob& pr = P.probs[i];
+    need = std::max(need, pr.n_mma);
+    for (int sgi = 0; sgi < pr.nseg; ++sgi)
+      for (int b = 0; b < pr.seg[sgi].nb; ++b)
+        need = std::max(need, (int)pr.seg[sgi].b[b].tile_off + (int)pr.seg[sgi].b[b].rows);
+  }
+  return need <= 64 ? 64 : (need <= 128 ? 128 : 256);
+}
+
 int GemmBuilder::launch(int* err, cudaStream_t stream) {
   if (status != 0) return status;
   const bool pair = pair_eligible();
@@ -1109,8 +1140,12 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   attach_output_maps();
   static int smem_set = 0;
   if (!smem_set) {
-    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+            cudaSuccess)
       return 5;
     if (cudaFuncSetAttribute(gemm_pair_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
         cudaSuccess)
@@ -1146,7 +1181,13 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
       launch_kernel(gemm_pair_kernel<1>, 2 * clusters, kGemmThreads, kGemmSmemBytes, stream, params);
   } else {
     const int grid = total < sms ? total : sms;
-    launch_kernel(gemm_kernel, grid, kGemmThreads, kGemmSmemBytes, stream, params);
+    const int brows = one_cta_brows(params, nprob);
+    if (brows == 64)
+      launch_kernel(gemm_kernel<64>, grid, kGemmThreads, kGemmSmemBytes, stream, params);
+    else if (brows == 128)
+      launch_kernel(gemm_kernel<128>, grid, kGemmThreads, kGemmSmemBytes, stream, params);
+    else
+      launch_kernel(gemm_kernel<256>, grid, kGemmThreads, kGemmSmemBytes, stream, params);
   }
   if (cudaGetLastError() != cudaSuccess) return 5;
   if (prof) gemm_events(stream, false, pair ? mh : 0);
