@@ -32,6 +32,16 @@ void note_launch(int n) {
   if (g_prof.load(std::memory_order_relaxed)) g_launches.fetch_add(n, std::memory_order_relaxed);
 }
 bool profiling_on() { return g_prof.load(std::memory_order_relaxed); }
+bool launch_failed(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return false;
+  static const bool verbose = [] {
+    const char* v = std::getenv("SL_VERBOSE_ERRORS");
+    return v && v[0] == '1';
+  }();
+  if (verbose) fprintf(stderr, "libsparselora: %s launch failed: %s\n", where, cudaGetErrorString(e));
+  return true;
+}
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = std::getenv("SL_PDL");

@@ -79,7 +79,7 @@ int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_
   launch_kernel(gather_rows_kernel, (unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s, 
       (const __nv_bfloat16*)src, ld_src, idx, n_rows, n_cols, (__nv_bfloat16*)dst, ld_dst, dst_col0, vec, blk,
       blk_stride, blk_off);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;
 }
@@ -90,7 +90,7 @@ int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int3
   dim3 grid((unsigned)((n_idx + 255) / 256), (unsigned)(n_rows < 1024 ? n_rows : 1024));
   launch_kernel(gather_cols_kernel, grid, 256, 0, s, (const __nv_bfloat16*)src, ld_src, n_rows, idx, n_idx,
                                           (__nv_bfloat16*)dst, ld_dst);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;
 }
@@ -101,7 +101,7 @@ int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, 
   dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
   launch_kernel(transpose_kernel, grid, dim3(32, 8), 0, s, (const __nv_bfloat16*)src, rows, cols, ld_src, (__nv_bfloat16*)dst,
                                                 ld_dst);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;
 }
@@ -114,7 +114,7 @@ int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int6
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s) {
   if (n <= 0) return 0;
   launch_kernel(add_f32_kernel, (unsigned)((n + 255) / 256), 256, 0, s, dst, src, n);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;
 }

@@ -371,7 +371,7 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
     const int64_t n = n_ctx * mk;
     launch_kernel(est_reduce_kernel, (unsigned)((n + 255) / 256), 256, 0, s, zpart, used, n);
   }
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;
 }
@@ -385,7 +385,7 @@ int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, con
     case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
     default: return 1;
   }
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;
 }
@@ -394,7 +394,7 @@ int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gra
              cudaStream_t s) {
   if (mk > 64 || n_ctx <= 0) return 1;
   launch_kernel(est_gram_kernel, gram_groups(n_ctx) * kGramCluster, 256, 0, s, z, n_ctx, mk, gram);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;
 }
@@ -419,7 +419,7 @@ int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int 
   launch_kernel(est_linear_scores_kernel, grid, 64, (size_t)mk * mk * sizeof(double), s, 
       gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
       crit == 0 ? 1 : head_dim, n_units, scores);
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;
 }

@@ -46,7 +46,10 @@ __device__ __forceinline__ uint32_t seg_tx_bytes(const Seg& sg) {
   return bytes;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU and the logistic function with the fast division intrinsic (the GEMM epilogues round
+// their results to bf16; exp overflow gives a zero quotient, the correct limit).
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -136,14 +139,16 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
     for (int c0 = 32 * half; c0 < 128; c0 += 64) {
       if (c0 >= ncols) break;
       float g[32];
+      uint32_t rawu[32];
       __syncwarp();
-      tmem_ld32(tb + c0, raw);
-      tmem_ld_wait();
+      tmem_ld32(tb + c0, raw);  // g and u in flight together, one wait
+      tmem_ld32(tb + 128 + c0, rawu);
+      tmem_ld_wait_regs(raw);
+      regs_after_wait(rawu);
 #pragma unroll
       for (int i = 0; i < 32; ++i) g[i] = __uint_as_float(raw[i]);
-      __syncwarp();
-      tmem_ld32(tb + 128 + c0, raw);
-      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) raw[i] = rawu[i];
       const int n = min(32, ncols - c0);
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);  // u
@@ -169,11 +174,9 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
   }
 
   const int ncols = min(pr.tile_cols, pr.N - n0);
-  for (int c0 = 32 * half; c0 < pr.n_mma; c0 += 64) {
-    if (c0 >= ncols) break;
-    __syncwarp();
-    tmem_ld32(tb + c0, raw);
-    tmem_ld_wait();
+  const int cend = min(pr.n_mma, ncols);
+  // One 32-column chunk: TMEM values in `raw` (already waited for), columns c0 .. c0 + 31.
+  auto chunk = [&](uint32_t (&raw)[32], int c0) {
     const int n = min(32, ncols - c0);
     if (pr.epi == EPI_BF16 && pr.col_map) {
       // Scatter through a 32 x 33 shared-memory transpose: each store instruction then
@@ -197,19 +200,19 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         }
       }
       __syncwarp();
-      continue;
+      return;
     }
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
     if (bulk && pr.epi == EPI_BF16) {
-      if (!wlive) continue;
+      if (!wlive) return;
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= pr.a0;
       bulk_store_chunk(&maps[pr.omap[0]], bufs, sb, v, n0 + c0, wrow0);
-      continue;
+      return;
     }
     if (bulk && pr.epi == EPI_DSWIGLU) {
-      if (!wlive) continue;
+      if (!wlive) return;
       float g[32], u[32];
       if (rv) {
         const int64_t aoff = orow * pr.ld_aux + n0 + c0;
@@ -223,16 +226,16 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
       float dg[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float sg = 1.0f / (1.0f + __expf(-g[i]));
+        const float sg = sigmoid_f(g[i]);
         const float dh = v[i];
         dg[i] = dh * u[i] * (sg * (1.0f + g[i] * (1.0f - sg)));
         v[i] = dh * g[i] * sg;  // du = dh * SiLU(g)
       }
       bulk_store_chunk(&maps[pr.omap[0]], bufs, sb, dg, n0 + c0, wrow0);
       bulk_store_chunk(&maps[pr.omap[1]], bufs, sb, v, n0 + c0, wrow0);
-      continue;
+      return;
     }
-    if (!rv) continue;
+    if (!rv) return;
     switch (pr.epi) {
       case EPI_BF16: {
 #pragma unroll
@@ -303,6 +306,18 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
       default:
         break;
     }
+    };
+  // Two chunks in flight per TMEM wait (columns c0 and c0 + 64 of this warp's half).
+  uint32_t raw2[32];
+  for (int c0 = 32 * half; c0 < cend; c0 += 128) {
+    const bool two = c0 + 64 < cend;
+    __syncwarp();
+    tmem_ld32(tb + c0, raw);
+    if (two) tmem_ld32(tb + c0 + 64, raw2);
+    tmem_ld_wait_regs(raw);
+    regs_after_wait(raw2);
+    chunk(raw, c0);
+    if (two) chunk(raw2, c0 + 64);
   }
 }
 
@@ -1189,7 +1204,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     else
       launch_kernel(gemm_kernel<256>, grid, kGemmThreads, kGemmSmemBytes, stream, params);
   }
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_gemm")) return 5;
   if (prof) gemm_events(stream, false, pair ? mh : 0);
   note_launch();
   // reduce the split-K problems (one launch for all of them)
@@ -1209,7 +1224,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   if (nred) {
     const unsigned gx = (unsigned)std::min<int64_t>((maxmn + 255) / 256, 1184);
     launch_kernel(splitk_reduce_kernel, dim3(gx, nred), 256, 0, stream, rp);
-    if (cudaGetLastError() != cudaSuccess) return 5;
+    if (launch_failed("sl_gemm")) return 5;
     note_launch();
   }
   return 0;

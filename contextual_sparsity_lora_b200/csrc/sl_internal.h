@@ -21,6 +21,10 @@ namespace sl {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 bool pdl_enabled();
 
+// True when the last launch failed; with SL_VERBOSE_ERRORS=1 in the environment the CUDA
+// error and the failing launch site go to stderr.
+bool launch_failed(const char* where);
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                           Args&&... args) {

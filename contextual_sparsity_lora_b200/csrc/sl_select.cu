@@ -180,7 +180,7 @@ int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sig
                                                                sigma_wide ? heads_per_group : 0, head_dim,
                                                                (int)n_wide, sigma_wide);
   if (n_keep_wide_out) *n_keep_wide_out = sigma_wide ? n_keep * heads_per_group : 0;
-  if (cudaGetLastError() != cudaSuccess) return 5;
+  if (launch_failed("sl_select")) return 5;
   note_launch();
   return 0;
 }
