@@ -272,7 +272,7 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
     if (rc) return from_kernel(rc);
   }
   if (crit == SL_CRIT_SWIGLU_L2) {
-    rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, s);
+    rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, err_word(ws), s);
     return from_kernel(rc);
   }
   rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s);

@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 
 #include "sl_internal.h"
+#include "sl_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -152,20 +153,25 @@ __global__ void est_reduce_kernel(float* zpart, int n_split, int64_t n) {
 }
 
 constexpr int kE2Threads = 256;  // 8 warps; each lane owns 2 channels of a 64-channel block
-constexpr int kE2Tok = 128;      // tokens staged per step
 constexpr int kE2Split = 4;      // token ranges per channel block = CTAs per cluster
+constexpr int kE2Buf = 4096;     // floats per staging buffer (16 KB): 4096 / (2k) tokens per chunk
 
 // SwiGLU criterion. Grid (F / 64, kE2Split) in clusters of (1, kE2Split): the CTAs of a
 // cluster share a 64-channel block and split the context tokens; their fp64 partial sums
-// are combined by cluster rank 0 through distributed shared memory in rank order.
+// are combined by cluster rank 0 through distributed shared memory in rank order. The
+// CTA's Z rows (2k floats per token, contiguous) arrive by bulk copies into two 16 KB
+// buffers, the next chunk in flight while the current one is consumed.
 template <int K>
 __global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
     est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx, const void* wb_g, const void* wb_u, int wb_fp32,
-                      int64_t n_ch, float* __restrict__ scores) {
-  pdl_wait();
-  __shared__ __align__(16) float zs[kE2Tok][2 * K];
+                      int64_t n_ch, float* __restrict__ scores, int* err) {
+  constexpr int kRow = 2 * K;
+  constexpr int kChunk = kE2Buf / kRow;
+  __shared__ __align__(128) float zs[2][kE2Buf];
+  __shared__ __align__(8) uint64_t bars[2];
   __shared__ double part[8][64];
   __shared__ double cta_sum[64];
+  pdl_wait();
   cg::cluster_group cluster = cg::this_cluster();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ch0 = (int64_t)blockIdx.x * 64 + lane;
@@ -180,36 +186,74 @@ __global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
   }
   const int64_t per = (n_ctx + kE2Split - 1) / kE2Split;
   const int64_t t_beg = min64(n_ctx, (int64_t)blockIdx.y * per), t_end = min64(n_ctx, t_beg + per);
+  const int nchunks = (int)((t_end - t_beg + kChunk - 1) / kChunk);
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int c) {  // thread 0: chunk c into buffer c & 1
+    const int64_t t0 = t_beg + (int64_t)c * kChunk;
+    const uint32_t bytes = (uint32_t)(min64(kChunk, t_end - t0) * kRow * 4);
+    mbar_arrive_expect_tx(&bars[c & 1], bytes);
+    bulk_load_g2s(&zs[c & 1][0], z + t0 * kRow, bytes, &bars[c & 1]);
+  };
+  if (threadIdx.x == 0) {
+    if (nchunks > 0) issue(0);
+    if (nchunks > 1) issue(1);
+  }
   double acc0 = 0.0, acc1 = 0.0;
-  for (int64_t tb = t_beg; tb < t_end; tb += kE2Tok) {
-    __syncthreads();
-    const int tn = (int)min64(kE2Tok, t_end - tb);
-    for (int e = threadIdx.x; e < tn * 2 * K / 4; e += kE2Threads)
-      reinterpret_cast<float4*>(&zs[0][0])[e] = reinterpret_cast<const float4*>(z + tb * 2 * K)[e];
-    __syncthreads();
+  int done = 0;  // chunks consumed
+  for (int c = 0; c < nchunks; ++c) {
+    const bool got = mbar_wait(&bars[c & 1], (uint32_t)((c >> 1) & 1), nullptr, err, DEV_TIMEOUT_ESTIMATOR);
+    if (__syncthreads_or(!got)) break;  // uniform: every thread leaves the loop together
+    const int tn = (int)min64(kChunk, t_end - (t_beg + (int64_t)c * kChunk));
+    const float* zc = &zs[c & 1][0];
     float s0 = 0.f, s1 = 0.f;
-    for (int t = warp; t < tn; t += 8) {
-      float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
-      const float4* zr = reinterpret_cast<const float4*>(&zs[t][0]);
+    // four tokens per step (t, t + 8, t + 16, t + 24): independent FMA chains and SiLUs in flight
+    constexpr int kU = 4;
+    for (int tb = warp; tb < tn; tb += 8 * kU) {
+      float g0[kU], u0[kU], g1[kU], u1[kU];
 #pragma unroll
-      for (int c4 = 0; c4 < K / 4; ++c4) {
-        const float4 zg = zr[c4], zu = zr[K / 4 + c4];
-        g0 = fmaf(zg.x, wg0[4 * c4], g0); g0 = fmaf(zg.y, wg0[4 * c4 + 1], g0);
-        g0 = fmaf(zg.z, wg0[4 * c4 + 2], g0); g0 = fmaf(zg.w, wg0[4 * c4 + 3], g0);
-        g1 = fmaf(zg.x, wg1[4 * c4], g1); g1 = fmaf(zg.y, wg1[4 * c4 + 1], g1);
-        g1 = fmaf(zg.z, wg1[4 * c4 + 2], g1); g1 = fmaf(zg.w, wg1[4 * c4 + 3], g1);
-        u0 = fmaf(zu.x, wu0[4 * c4], u0); u0 = fmaf(zu.y, wu0[4 * c4 + 1], u0);
-        u0 = fmaf(zu.z, wu0[4 * c4 + 2], u0); u0 = fmaf(zu.w, wu0[4 * c4 + 3], u0);
-        u1 = fmaf(zu.x, wu1[4 * c4], u1); u1 = fmaf(zu.y, wu1[4 * c4 + 1], u1);
-        u1 = fmaf(zu.z, wu1[4 * c4 + 2], u1); u1 = fmaf(zu.w, wu1[4 * c4 + 3], u1);
+      for (int j = 0; j < kU; ++j) g0[j] = u0[j] = g1[j] = u1[j] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kU; ++j) {
+        const int t = min(tb + 8 * j, tn - 1);  // clamped rows are read but not summed
+        const float4* zr = reinterpret_cast<const float4*>(zc + t * kRow);
+#pragma unroll
+        for (int c4 = 0; c4 < K / 4; ++c4) {
+          const float4 zg = zr[c4], zu = zr[K / 4 + c4];
+          g0[j] = fmaf(zg.x, wg0[4 * c4], g0[j]); g0[j] = fmaf(zg.y, wg0[4 * c4 + 1], g0[j]);
+          g0[j] = fmaf(zg.z, wg0[4 * c4 + 2], g0[j]); g0[j] = fmaf(zg.w, wg0[4 * c4 + 3], g0[j]);
+          g1[j] = fmaf(zg.x, wg1[4 * c4], g1[j]); g1[j] = fmaf(zg.y, wg1[4 * c4 + 1], g1[j]);
+          g1[j] = fmaf(zg.z, wg1[4 * c4 + 2], g1[j]); g1[j] = fmaf(zg.w, wg1[4 * c4 + 3], g1[j]);
+          u0[j] = fmaf(zu.x, wu0[4 * c4], u0[j]); u0[j] = fmaf(zu.y, wu0[4 * c4 + 1], u0[j]);
+          u0[j] = fmaf(zu.z, wu0[4 * c4 + 2], u0[j]); u0[j] = fmaf(zu.w, wu0[4 * c4 + 3], u0[j]);
+          u1[j] = fmaf(zu.x, wu1[4 * c4], u1[j]); u1[j] = fmaf(zu.y, wu1[4 * c4 + 1], u1[j]);
+          u1[j] = fmaf(zu.z, wu1[4 * c4 + 2], u1[j]); u1[j] = fmaf(zu.w, wu1[4 * c4 + 3], u1[j]);
+        }
       }
-      const float h0 = __fdividef(g0, 1.0f + __expf(fminf(-g0, 80.f))) * u0;
-      const float h1 = __fdividef(g1, 1.0f + __expf(fminf(-g1, 80.f))) * u1;
-      s0 = fmaf(h0, h0, s0);
-      s1 = fmaf(h1, h1, s1);
+#pragma unroll
+      for (int j = 0; j < kU; ++j) {
+        if (tb + 8 * j >= tn) break;  // in order: the per-thread sum keeps a fixed token order
+        const float h0 = __fdividef(g0[j], 1.0f + __expf(fminf(-g0[j], 80.f))) * u0[j];
+        const float h1 = __fdividef(g1[j], 1.0f + __expf(fminf(-g1[j], 80.f))) * u1[j];
+        s0 = fmaf(h0, h0, s0);
+        s1 = fmaf(h1, h1, s1);
+      }
     }
     acc0 += (double)s0;
     acc1 += (double)s1;
+    done = c + 1;
+    __syncthreads();  // buffer c & 1 is free again
+    if (threadIdx.x == 0 && c + 2 < nchunks) issue(c + 2);
+  }
+  if (done < nchunks && threadIdx.x == 0) {
+    // a copy did not land in time: wait (bounded) for the ones still in flight to finish
+    // writing this CTA's shared memory before it is released
+    for (int c = done; c < nchunks && c < done + 2; ++c)
+      mbar_wait(&bars[c & 1], (uint32_t)((c >> 1) & 1), nullptr, nullptr, 0);
   }
   part[warp][lane] = acc0;
   part[warp][lane + 32] = acc1;
@@ -377,12 +421,13 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
 }
 
 int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, const void* wb_gate, const void* wb_up,
-                      int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s) {
+                      int wb_fp32, int64_t n_ch, float* scores, int* err, cudaStream_t s) {
+  if (reinterpret_cast<uintptr_t>(z) & 15) return 1;  // bulk copies need 16-byte alignment
   const dim3 grid((unsigned)((n_ch + 63) / 64), kE2Split);
   switch (k) {
-    case 8: launch_kernel(est_swiglu_kernel<8>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
-    case 16: launch_kernel(est_swiglu_kernel<16>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
-    case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores); break;
+    case 8: launch_kernel(est_swiglu_kernel<8>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
+    case 16: launch_kernel(est_swiglu_kernel<16>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
+    case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
     default: return 1;
   }
   if (launch_failed("sl_estimator")) return 5;

@@ -91,7 +91,7 @@ int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 0);
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
                const void* const* wa, int wa_fp32, int k, float* zpart, int n_split, cudaStream_t s);
 int est_swiglu_scores(const float* zpart, int n_split, int64_t n_ctx, int k, const void* wb_gate,
-                      const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, cudaStream_t s);
+                      const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, int* err, cudaStream_t s);
 int est_gram(const float* zpart, int n_split, int64_t n_ctx, int mk, double* gram_part, int n_chunks,
              cudaStream_t s);
 int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int crit, int proj0, int proj1,

@@ -16,6 +16,7 @@ enum : int {
   DEV_TIMEOUT_EPILOGUE = 3,
   DEV_TIMEOUT_DRAIN = 4,
   DEV_BAD_TILE = 5,
+  DEV_TIMEOUT_ESTIMATOR = 6,
 };
 
 // Upper bound of any single wait inside a kernel. Correct kernels wait microseconds.
@@ -89,6 +90,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// Untiled bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // Bulk tensor store of a shared-memory box to global memory (no multicast), tracked in
