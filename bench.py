@@ -383,9 +383,13 @@ def main():
     # with the library's launch counting and an event pair around each GEMM-engine launch,
     # is replayed over its own K timed steps for the roofline's kernel durations.
     graph = capture_graph(lambda: run_step(attn, ffn, step_in), warm=False)
+    # (the profiled copy runs each block's chains in order, so that no concurrent kernel
+    # stretches a GEMM-engine launch's event-timed duration)
+    attn.concurrent = ffn.concurrent = False
     B.sl_profile_enable(True)
     prof_graph = capture_graph(lambda: run_step(attn, ffn, step_in), warm=False)
     B.sl_profile_enable(False)
+    attn.concurrent = ffn.concurrent = True
     with ClockSampler(local) as clk:
         ms = time_steps(graph.replay, args.steps, args.warmup, world, device)
     torch.cuda.synchronize()

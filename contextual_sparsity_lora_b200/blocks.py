@@ -16,6 +16,24 @@ def _empty(shape, dtype, device):
     return torch.empty(*shape, dtype=dtype, device=device)
 
 
+class _Side:
+    """A second stream for a chain of calls that does not depend on the main chain (and the
+    workspace it needs: concurrent calls must not share scratch). `fork` makes the side
+    stream wait for the work queued so far; `join` makes the main stream wait for the side
+    chain. Inside CUDA-graph capture this becomes two parallel branches of the graph."""
+
+    def __init__(self, device):
+        self.stream = torch.cuda.Stream(device=device)
+        self.ws = B.Workspace(device)
+
+    def fork(self):
+        self.stream.wait_stream(torch.cuda.current_stream())
+        return torch.cuda.stream(self.stream)
+
+    def join(self):
+        torch.cuda.current_stream().wait_stream(self.stream)
+
+
 class FFNBlock:
     """SwiGLU FFN: gate/up (output channels sliced), down (input channels sliced), one
     index set shared by all three; L2 criterion on the estimated SiLU(gate) * up."""
@@ -43,6 +61,8 @@ class FFNBlock:
         self.Wd_t = _empty((self.F, self.D), bf, device)
         B.sl_prepare_weight(self.Wd, self.Wd_t)
         self.ws = B.Workspace(device)
+        self.side = _Side(device)
+        self.concurrent = True  # independent chains on a second stream
         T, D, F, r = n_tok, self.D, self.F, self.r
         f32 = torch.float32
         self.scores = _empty((F,), f32, device)
@@ -103,10 +123,20 @@ class FFNBlock:
         self.x = x
         self.x_est = x_est
         C = self.n_ctx
-        if not self.dense and C > 0:  # no context rows: nothing to score, every row is dense
-            self.select(x)
         lay = B.SL_LAYOUT_NATURAL if self.dense else B.SL_LAYOUT_SIGMA
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu, xa=self.xa_gu)
+        if not self.dense and C > 0:  # no context rows: nothing to score, every row is dense
+            if self.concurrent:  # x A^T of gate/up does not depend on the selection
+                with self.side.fork():
+                    B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
+                                      xa=self.xa_gu)
+                self.select(x)
+                self.side.join()
+            else:
+                self.select(x)
+                B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
+                                  xa=self.xa_gu)
+        else:
+            B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu, xa=self.xa_gu)
         B.sl_sparse_linear_fwd(self.ws, [self.lin_g, self.lin_u], [self.ch], B.SL_EPI_SWIGLU, x, C, self.xa_s_gu,
                                [self.g, self.u, self.h], out_layout=B.SL_LAYOUT_SIGMA)
         B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_d], self.h, C, self.xa_s_d, xa=self.xa_d,
@@ -131,6 +161,10 @@ class FFNBlock:
                                [self.dg, self.du], C, [self.dya_s_g, self.dya_s_u], dx=self.dx,
                                in_layout=B.SL_LAYOUT_SIGMA)
         return self.dx
+
+    def read_device_flag(self) -> int:
+        """Device error word of both workspaces (0: no device-side timeout); synchronises."""
+        return self.ws.read_device_flag() or self.side.ws.read_device_flag()
 
     def step(self, x, dy, x_est=None):
         self.forward(x, x_est)
@@ -165,6 +199,8 @@ class AttnProjBlock:
         self.Wo_t = _empty((self.Dq, self.D), bf, device)
         B.sl_prepare_weight(self.Wo, self.Wo_t)
         self.ws = B.Workspace(device)
+        self.side = _Side(device)
+        self.concurrent = True  # independent chains on a second stream
         T, D, r = n_tok, self.D, self.r
         self.s_qk, self.s_v = _empty((self.n_units,), f32, device), _empty((self.n_units,), f32, device)
         ar = lambda n: torch.arange(n, dtype=torch.int32, device=device)
@@ -229,13 +265,24 @@ class AttnProjBlock:
     def forward(self, x, x_o):
         C = self.n_ctx
         self.x, self.x_o = x, x_o
-        if not self.dense and C > 0:
-            self.select(x)
         lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
+        sel = not self.dense and C > 0
+
+        def lora_fwd(ws):  # x A^T for q, k, v and x_o A^T for o: independent of the selection
+            B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
+            B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+
+        if sel and self.concurrent:
+            with self.side.fork():
+                lora_fwd(self.side.ws)
+            self.select(x)
+            self.side.join()
+        else:
+            if sel:
+                self.select(x)
+            lora_fwd(self.ws)
         B.sl_sparse_linear_fwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, x, C,
                                self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=B.SL_LAYOUT_NATURAL)
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
         B.sl_sparse_linear_fwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, x_o, C, self.xa_s_o, [self.y],
                                in_layout=B.SL_LAYOUT_NATURAL)
         return self.y
@@ -243,16 +290,33 @@ class AttnProjBlock:
     def backward(self, dy, dq, dk, dv):
         C = self.n_ctx
         lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
-                          dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
-        B.sl_sparse_linear_bwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
-                               dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
-                          dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
-                          dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
-        B.sl_sparse_linear_bwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
-                               [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
+
+        def o_chain(ws):  # o's LoRA gradients and its input gradient dx_o
+            B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
+                              dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
+            B.sl_sparse_linear_bwd(ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
+                                   dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
+
+        def qkv_chain(ws):  # q, k, v LoRA gradients and dx; independent of the o chain
+            B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
+                              dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
+                              dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
+            B.sl_sparse_linear_bwd(ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
+                                   [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
+
+        if self.concurrent:
+            with self.side.fork():
+                o_chain(self.side.ws)
+            qkv_chain(self.ws)
+            self.side.join()
+        else:
+            o_chain(self.ws)
+            qkv_chain(self.ws)
         return self.dx, self.dx_o
+
+    def read_device_flag(self) -> int:
+        """Device error word of both workspaces (0: no device-side timeout); synchronises."""
+        return self.ws.read_device_flag() or self.side.ws.read_device_flag()
 
     def step(self, x, x_o, dy, dq, dk, dv):
         self.forward(x, x_o)

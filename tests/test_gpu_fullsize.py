@@ -35,7 +35,7 @@ def test_ffn_full_size(cfg):
                           cfg.lora_scale, cfg.k, T, C, cfg.ratio, DEV)
     blk.step(x, dy)
     torch.cuda.synchronize()
-    assert blk.ws.read_device_flag() == 0
+    assert blk.read_device_flag() == 0
     ctx = np.arange(T) < C
     s_w, _ = oracle.ffn_select(x, ctx, (d["gate"].W_A, d["gate"].W_B), (d["up"].W_A, d["up"].W_B), cfg.ratio)
     assert rel_fro(blk.scores, s_w) < FP32_TOL
@@ -78,7 +78,7 @@ def test_attn_full_size(cfg):
                                DEV)
     blk.step(t["x"], t["x_o"], t["dy"], t["dq"], t["dk"], t["dv"])
     torch.cuda.synchronize()
-    assert blk.ws.read_device_flag() == 0
+    assert blk.read_device_flag() == 0
     ctx = np.arange(T) < C
     F = lambda n: (d[n].W_A, d[n].W_B)
     sel = oracle.attn_select(t["x"], ctx, F("q"), F("k"), F("v"), cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim,
