@@ -399,9 +399,10 @@ def main():
     # headline graph); GEMM-engine durations of its last replay, per launch and in total
     per_launch = B.sl_profile_launches()
     n_launch_step, n_gemm, gemm_ms = B.sl_profile_read()
-    pair_ms = sum(m for m, k in per_launch if k > 0)
-    pair_n = sum(1 for _, k in per_launch if k > 0)
-    skinny_ms = sum(m for m, k in per_launch if k == 0)
+    pair_ms = sum(m for m, k in per_launch if k in (1, 2))
+    pair_n = sum(1 for _, k in per_launch if k in (1, 2))
+    skinny_ms = sum(m for m, k in per_launch if k in (0, 3))
+    skinny_n = sum(1 for _, k in per_launch if k in (0, 3))
     del prof_graph
     n_launch = n_launch_step * args.steps
     ms_step = ms / args.steps
@@ -436,7 +437,7 @@ def main():
                      "launches_per_step": pair_n, "ms_per_launch": pair_ms / max(pair_n, 1),
                      "gemm_engine_ms_per_step": gemm_ms, "gemm_engine_launches_per_step": n_gemm,
                      "skinny_lora_and_stage1": {"bound": "hbm", "ms_per_step": skinny_ms,
-                                                "launches_per_step": n_gemm - pair_n,
+                                                "launches_per_step": skinny_n,
                                                 "algorithmic_bytes_per_step": skinny_bytes,
                                                 "achieved_GBs": skinny_bytes / (skinny_ms * 1e6) if skinny_ms else None,
                                                 "peak_GBs": hbm,

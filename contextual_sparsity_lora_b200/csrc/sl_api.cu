@@ -383,7 +383,8 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   if (out_sig && !out_ch) return SL_ERR_INVALID_ARG;
   for (int i = 0; i < n_ad; ++i) {
     if (!dy[i] || !dya[i] || !dya_s[i] || !dA[i] || !dB[i]) return SL_ERR_INVALID_ARG;
-    if (ld_dy[i] < lin[i].d_out || ld_dy[i] % 8 || !al16(dy[i]) || !al16(dya_s[i])) return SL_ERR_ALIGNMENT;
+    if (ld_dy[i] < lin[i].d_out || ld_dy[i] % 8 || !al16(dy[i]) || !al16(dya_s[i]) || !al16(dya[i]) || !al16(dB[i]))
+      return SL_ERR_ALIGNMENT;
     if (out_sig && !channels_ok(out_ch[i], lin[i].d_out)) return SL_ERR_INVALID_ARG;
   }
   // K extents of the dB / dA parts: pass 0 = natural part (all rows, or output rows when the
@@ -417,38 +418,52 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
       if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i],
                                     lin[i].r, 0, s))
         return from_kernel(rc);
-  // launch 1: dya = scale * dy B
+  // dya = scale * dy B and dB = dy^T xa_s from one pass over each dy (fused kernel; context rows
+  // of a sigma-layout dy use the permuted B and land in dB rows sigma[p]), then dya_s = bf16(dya)
   {
-    GemmBuilder gb;
-    int64_t off = 0;
+    DualSpec sp[8];
+    int nsp = 0;
+    const float* csrc[4];
+    void* cdst[4];
+    int64_t ccount[4];
+    int64_t koff = 0;
     for (int i = 0; i < n_ad; ++i) {
       const sl_linear& L = lin[i];
-      const int mdy = gb.map(dy[i], T, L.d_out, ld_dy[i], kBM);
-      const int mbn = gb.map(L.lora_b, L.d_out, L.r, L.r, 64);
-      const int mbs = out_sig ? gb.map(bsig[i], L.d_out, L.r, L.r, 64) : -1;
-      auto add_prob = [&](int64_t M, int64_t row0, int mb) {
-        Prob* p = gb.add((int)M, L.r, kBN, (int)rup(L.r, 16));
-        Seg* sg = gb.seg(p, mdy, 0, (int)row0, 0, 1, 0, (int)L.d_out, kBig);
-        gb.bsrc(sg, mb, 0, 64, 0, 0);
-        if (!p) return;
-        p->epi = EPI_XA;
-        p->out_row0 = (int)row0;
-        p->out0 = dya[i];
-        p->ld0 = L.r;
-        p->out1 = dya_s[i];
-        p->ld1 = L.r;
-        p->a0 = L.lora_scale;
-        p->a1 = L.lora_scale;
-        maybe_split(gb, p, M, L.r, L.d_out, region, &off);
+      if (cudaMemsetAsync(dya[i], 0, sizeof(float) * T * L.r, s) != cudaSuccess ||
+          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s) != cudaSuccess)
+        return SL_ERR_CUDA;
+      const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
+      koff += L.r;
+      auto add = [&](int64_t row0, int64_t rows, const void* Bm, const int32_t* sig) {
+        if (rows <= 0) return;
+        DualSpec& d = sp[nsp++];
+        d.dy = dy[i];
+        d.ld_dy = ld_dy[i];
+        d.B = Bm;
+        d.xa_s = xa_blk;
+        d.ld_xa = ld_xa;
+        d.row0 = row0;
+        d.rows = rows;
+        d.cols = L.d_out;
+        d.r = L.r;
+        d.scale = L.lora_scale;
+        d.dya = dya[i];
+        d.ld_dya = L.r;
+        d.dB = dB[i];
+        d.sigma = sig;
       };
       if (out_sig) {
-        add_prob(C, 0, mbs);
-        add_prob(O, C, mbn);
+        add(0, C, bsig[i], out_ch[i].sigma);
+        add(C, O, L.lora_b, nullptr);
       } else {
-        add_prob(T, 0, mbn);
+        add(0, T, L.lora_b, nullptr);
       }
+      csrc[i] = dya[i];
+      cdst[i] = dya_s[i];
+      ccount[i] = T * L.r;
     }
-    if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
+    if (int rc = lora_dual_launch(sp, nsp, err_word(ws), s)) return from_builder(rc);
+    if (int rc = cast_f32_bf16(csrc, cdst, ccount, n_ad, s)) return from_kernel(rc);
   }
   // launch 2: dB = dy^T xa_s and dA = (x^T dya)^T over the natural parts; launch 3: the
   // context parts of sigma-layout operands, accumulated onto launch 2's results.
@@ -461,7 +476,7 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
       int64_t koff = 0;
       for (int i2 = 0; i2 < i; ++i2) koff += lin[i2].r;
       const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
-      for (int which = 0; which < 2; ++which) {  // 0: dB, 1: dA
+      for (int which = 1; which < 2; ++which) {  // dA (dB came from the fused kernel)
         const bool sig = which == 0 ? out_sig : in_sig;
         const int64_t K = kpart(sig, pass);
         const bool ctx_part = pass == 1;

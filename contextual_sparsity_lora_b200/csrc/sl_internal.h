@@ -44,7 +44,8 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 // Launch accounting for the optional profiling hook (sl_profile_enable / sl_profile_read).
 void note_launch(int n = 1);
 bool profiling_on();
-// kind: 0 one-CTA launch, 1 CTA-pair 256-row tiles, 2 CTA-pair 512-row tiles
+// kind: 0 one-CTA launch, 1 CTA-pair 256-row tiles, 2 CTA-pair 512-row tiles, 3 fused LoRA
+// backward
 void gemm_events(cudaStream_t s, bool start, int kind = 0);
 #ifdef SL_PROFILE_DUMP
 // Description of the next GEMM-engine launch, printed with its time by sl_profile_read.
@@ -101,6 +102,27 @@ int est1_splits(int64_t d_in);
 // The Gram kernel runs clusters of 8 CTAs over 48 context tokens each; one fp64 partial
 // Gram matrix per cluster is left for the score kernel to add.
 inline int gram_groups(int64_t n_ctx) { return (int)((n_ctx + 8 * 48 - 1) / (8 * 48)); }
+
+// ---- fused LoRA backward (sl_lora.cu)
+// One adapter over one row segment of its upstream gradient: adds scale * dy B into dya and
+// dy^T xa_s into dB (rows sigma[p] when sigma is set), reading dy once.
+struct DualSpec {
+  const void* dy;    // bf16, rows [0, row0 + rows) addressable, ld_dy elements
+  int64_t ld_dy;
+  const void* B;     // bf16 [cols, r]: LoRA B, or its rows permuted by sigma for sigma-layout rows
+  const void* xa_s;  // bf16 [row0 + rows, r] block of this adapter (ld_xa)
+  int64_t ld_xa;
+  int64_t row0, rows, cols;
+  int r;
+  float scale;
+  float* dya;        // fp32 [n_tok, ld_dya], 16-byte aligned, zeroed by the caller
+  int64_t ld_dya;
+  float* dB;         // fp32 [cols, r], 16-byte aligned, zeroed by the caller
+  const int32_t* sigma;
+};
+int lora_dual_launch(const DualSpec* specs, int n, int* err, cudaStream_t s);
+// dst[i][k] = bf16(src[i][k]) for k < count[i], i < n (one launch).
+int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* count, int n, cudaStream_t s);
 
 // ---- selection (sl_select.cu)
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group,

@@ -199,6 +199,8 @@ SL_API sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_ke
  *   dya[i] (fp32 [n_tok, r_i], ld r_i) = scale * dy B;  dya_s[i] (bf16, same) = dya;
  *   dB[i] (fp32 [d_out_i, r_i]) = scale * dy^T xa = dy^T xa_s;
  *   dA[i] (fp32 [r_i, d_in]) = dya^T x.
+ *   dya and dB come from one pass over dy whose partial sums meet in fp32 reductions, so
+ *   their last bits may differ between runs; dya and dB must be 16-byte aligned.
  *   xa_s is the forward's bf16 block for adapter i (ld ld_xa, column offset = sum of
  *   earlier r). out_layout SL_LAYOUT_SIGMA: dy's context rows are in the sigma layout
  *   of out_ch[i]; in_layout SL_LAYOUT_SIGMA: x's context rows are in the sigma layout
@@ -257,7 +259,8 @@ SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launche
 /* Per-launch view of the same GEMM-engine event pairs, without resetting them (call it
  * before sl_profile_read): *count = launches recorded; for the first min(count, capacity)
  * of them, in launch order, ms[i] = duration and kind[i] = 0 (one-CTA grouped launch),
- * 1 (CTA pairs, 256-row tiles) or 2 (CTA pairs, 512-row tiles). Waits for the events. */
+ * 1 (CTA pairs, 256-row tiles), 2 (CTA pairs, 512-row tiles) or 3 (fused LoRA backward
+ * stream). Waits for the events. */
 SL_API sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count);
 
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
