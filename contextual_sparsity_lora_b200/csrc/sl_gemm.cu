@@ -121,8 +121,18 @@ __device__ __forceinline__ void bulk_store_chunk(const CUtensorMap* map, uint8_t
 // executed by every lane of the warp (they are warp-collective).
 // `half` selects the 32-column chunks this warp handles (even or odd); the other epilogue
 // warp on the same TMEM lane quarter takes the rest.
+// Aux loads of the SwiGLU backward: per epilogue warp one mbarrier (abar), its phase (aph)
+// and whether a load is still outstanding (apend, drained at the end of the kernel).
+struct AuxWait {
+  uint64_t* bar;
+  uint32_t phase;
+  bool pending;
+  volatile int* abort;
+  int* err;
+};
+
 __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, int n0, int r, uint32_t tb,
-                              float* stage, int half, int& sb) {
+                              float* stage, int half, int& sb, AuxWait& aw) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
@@ -214,15 +224,22 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
     if (bulk && pr.epi == EPI_DSWIGLU) {
       if (!wlive) return;
       float g[32], u[32];
-      if (rv) {
-        const int64_t aoff = orow * pr.ld_aux + n0 + c0;
-        const bool vec = (aoff & 7) == 0;
-        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux0) + aoff, g, n, vec);
-        load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(pr.aux1) + aoff, u, n, vec);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) g[i] = u[i] = 0.f;
+      const int lane = r & 31;
+      // g and u of the warp's 32 rows x 32 columns arrive by two bulk tensor loads into the
+      // warp's two boxes, once its earlier bulk stores have read them; one lane = one row
+      if (lane == 0) {
+        bulk_wait_read<0>();
+        mbar_arrive_expect_tx(aw.bar, 4096);
+        tma_load_2d(bufs, &maps[pr.omap[2]], aw.bar, n0 + c0, wrow0);
+        tma_load_2d(bufs + 2048, &maps[pr.omap[3]], aw.bar, n0 + c0, wrow0);
       }
+      aw.pending = true;
+      if (!mbar_wait(aw.bar, aw.phase, aw.abort, aw.err, DEV_TIMEOUT_EPILOGUE)) return;
+      aw.pending = false;
+      aw.phase ^= 1;
+      load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(bufs) + lane * 32, g, 32, true);
+      load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(bufs + 2048) + lane * 32, u, 32, true);
+      __syncwarp();
       float dg[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -429,6 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // kEpiWarps x [32][33]
+  uint64_t* aux_bars = bars + 24;  // one per epilogue warp (bytes 192..255 of the barrier block)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -443,6 +461,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       mbar_init(&tempty[b], 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&aux_bars[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -565,6 +584,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int half = (warp - 2) >> 2;   // which 32-column chunks of the tile
     const int r = q * 32 + lane;
     int acc = 0, sbuf = 0;
+    AuxWait aw{aux_bars + (warp - 2), 0u, false, abort_flag, p.err};
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
       const TileInfo ti = decode_tile(p, t);
@@ -576,13 +596,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb, half);
       else
         epilogue_tile(pr, p.maps, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33, half,
-                      sbuf);
+                      sbuf, aw);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (aw.pending) mbar_wait(aw.bar, aw.phase, nullptr, nullptr, 0);  // an aux load in flight lands first
     if (lane == 0) bulk_wait_all();  // bulk stores complete before the CTA's shared memory goes away
   }
 
@@ -654,6 +675,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  uint64_t* aux_bars = bars + 24;  // one per epilogue warp (bytes 192..255 of the barrier block)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -671,6 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[b], 2 * 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&aux_bars[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -791,6 +814,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0, sbuf = 0;
+    AuxWait aw{aux_bars + (warp - 2), 0u, false, abort_flag, p.err};
     uint32_t acc_phase = 0;
     for (int t = cl; t < p.total_tiles; t += n_cl) {
       const TileInfo ti = decode_tile(p, t);
@@ -801,7 +825,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int h = 0; h < MH; ++h)
         epilogue_tile(pr, p.maps, ti.tm * C::kTileM + 128 * MH * (int)rank + 128 * h, ti.tn * pr.tile_cols, r,
-                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half, sbuf);
+                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half, sbuf, aw);
       __syncwarp();
       tc_fence_before();
       mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
@@ -810,6 +834,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1;
       }
     }
+    if (aw.pending) mbar_wait(aw.bar, aw.phase, nullptr, nullptr, 0);  // an aux load in flight lands first
     if (lane == 0) bulk_wait_all();  // bulk stores complete before the CTA's shared memory goes away
   }
 
@@ -911,13 +936,16 @@ void GemmBuilder::attach_output_maps() {
     const bool eligible = pr.ksplit <= 1 && !pr.row_map && pr.M > 0 && pr.N > 0 &&
                           ((pr.epi == EPI_BF16 && !pr.col_map) || pr.epi == EPI_SWIGLU || pr.epi == EPI_DSWIGLU);
     if (disabled || !eligible) continue;
-    const int nout = pr.epi == EPI_SWIGLU ? 3 : (pr.epi == EPI_DSWIGLU ? 2 : 1);
-    void* outs[3] = {pr.out0, pr.out1, pr.out2};
-    int idx[3] = {-1, -1, -1};
+    // SwiGLU backward: two outputs (dg, du) and two inputs (g, u) read through the same boxes
+    const int nout = pr.epi == EPI_SWIGLU ? 3 : (pr.epi == EPI_DSWIGLU ? 4 : 1);
+    void* outs[4] = {pr.out0, pr.out1, pr.epi == EPI_DSWIGLU ? const_cast<void*>(pr.aux0) : pr.out2,
+                     const_cast<void*>(pr.aux1)};
+    int idx[4] = {-1, -1, -1, -1};
     const int saved = nmaps;
     bool ok = true;
     for (int k = 0; k < nout && ok; ++k) {
-      idx[k] = map_out(static_cast<uint16_t*>(outs[k]) + (int64_t)pr.out_row0 * pr.ld0, pr.M, pr.N, pr.ld0);
+      const int64_t ld = (pr.epi == EPI_DSWIGLU && k >= 2) ? pr.ld_aux : pr.ld0;
+      idx[k] = map_out(static_cast<uint16_t*>(outs[k]) + (int64_t)pr.out_row0 * ld, pr.M, pr.N, ld);
       ok = idx[k] >= 0;
     }
     if (!ok) {

@@ -73,8 +73,9 @@ struct Prob {
   Seg seg[kMaxSegs];
   int32_t epi, beta;
   int32_t out_row0;     // first output row
-  int8_t omap[4];       // tensor maps (32 x 32 boxes) of out0..out2 rows [out_row0, out_row0 + M) for
-                        // bulk tensor stores from the epilogue; -1: per-thread stores
+  int8_t omap[4];       // tensor maps (32 x 32 boxes) of out0..out2 (SwiGLU backward: dg, du, g, u)
+                        // over rows [out_row0, out_row0 + M), for the epilogue's bulk tensor copies;
+                        // -1: per-thread loads and stores
   int64_t ld0, ld1, ld2, ld_aux;
   void* out0;
   void* out1;
