@@ -460,8 +460,8 @@ int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int 
     w.p[1] = wb1;
     w.n[1] = (int64_t)n_kv_heads * head_dim;
   }
-  const unsigned grid = (unsigned)((n_units + 63) / 64);
-  launch_kernel(est_linear_scores_kernel, grid, 64, (size_t)mk * mk * sizeof(double), s, 
+  const unsigned grid = (unsigned)((n_units + 255) / 256);
+  launch_kernel(est_linear_scores_kernel, grid, 256, (size_t)mk * mk * sizeof(double), s, 
       gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
       crit == 0 ? 1 : head_dim, n_units, scores);
   if (launch_failed("sl_estimator")) return 5;
