@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-LoRA companion measurement")
+    ap.add_argument("--stages-only", action="store_true",
+                    help="time only the selection stages (estimator, criterion, top-n, compaction) of both blocks "
+                         "and print them; no step, no headline line")
     return ap.parse_args()
 
 
@@ -219,15 +222,22 @@ def time_steps(fn, K, W, world, device):
 
 def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
     """Device time of the selection stages of both blocks, each captured alone in a CUDA
-    graph and replayed `reps` times: a1 (estimator stage 1, the tensor-core launch of
-    sl_svd_estimate, event-timed in a profiled copy), a2 (the rest of sl_svd_estimate: the
-    criterion), a3 (sl_select_channels) and the per-step compaction of the kept weight rows."""
+    graph (`inner` back-to-back copies of the stage per graph, so that the host's graph
+    launches do not pace tiny stages) and replayed `reps` times: a1 (estimator stage 1, the
+    tensor-core launch of sl_svd_estimate, event-timed in a profiled copy), a2 (the rest of
+    sl_svd_estimate: the criterion), a3 (sl_select_channels) and the per-step compaction of
+    the kept weight rows."""
     from contextual_sparsity_lora_b200 import binding as B
+    inner = 10
 
     def graph_us(fn):
         fn()
-        g = capture_graph(fn, warm=False)
-        return time_steps(g.replay, reps, 3, 1, device) / reps * 1e3
+
+        def many():
+            for _ in range(inner):
+                fn()
+        g = capture_graph(many, warm=False)
+        return time_steps(g.replay, reps, 3, 1, device) / (reps * inner) * 1e3
 
     def a1_us(fn):
         B.sl_profile_read()
@@ -256,8 +266,10 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
                      "a1_frac_of_hbm": a1_bytes / (a1 * 1e3) / hbm_gbs if a1 else None,
                      "a2_criterion_us": est - a1 if a1 else None, "a3_select_us": sel, "compact_weights_us": comp}
         total += est + sel
-    out["estimator_and_select_pct_of_step"] = 100.0 * total / (step_ms * 1e3)
-    out["timing"] = "each stage alone in a CUDA graph, replayed; device time between events"
+    out["estimator_and_select_us"] = total
+    if step_ms:
+        out["estimator_and_select_pct_of_step"] = 100.0 * total / (step_ms * 1e3)
+    out["timing"] = "each stage alone, 10 copies per CUDA graph, replayed; device time between events"
     return out
 
 
@@ -378,6 +390,10 @@ def main():
         run_step(attn, ffn, step_in)
     torch.cuda.synchronize()
     B.sl_profile_read()
+    if args.stages_only:
+        print(json.dumps({"stages": stage_times(attn, ffn, step_in, 50, device,
+                                                float(load_peaks()[0].get("hbm_gbs", 6650.0)), None)}))
+        return
     # The step is captured once into a CUDA graph and replayed; every replay runs every
     # kernel. The headline graph carries no event nodes. A second capture of the same step,
     # with the library's launch counting and an event pair around each GEMM-engine launch,
@@ -401,8 +417,8 @@ def main():
     n_launch_step, n_gemm, gemm_ms = B.sl_profile_read()
     pair_ms = sum(m for m, k in per_launch if k in (1, 2))
     pair_n = sum(1 for _, k in per_launch if k in (1, 2))
-    skinny_ms = sum(m for m, k in per_launch if k in (0, 3))
-    skinny_n = sum(1 for _, k in per_launch if k in (0, 3))
+    skinny_ms = sum(m for m, k in per_launch if k in (0, 3, 4))
+    skinny_n = sum(1 for _, k in per_launch if k in (0, 3, 4))
     del prof_graph
     n_launch = n_launch_step * args.steps
     ms_step = ms / args.steps

@@ -246,6 +246,16 @@ class AttnProjBlock:
         B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
 
+    def _qk_chain(self):
+        B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
+        for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k)):
+            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+
+    def _vo_chain(self):
+        B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+        for n, w, sig in (("v", self.Wv, self.sig_v), ("o", self.Wo_t, self.sig_o)):
+            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+
     def choose(self):
         """a3: the q/k set from the QK scores and the v/o set from the V scores."""
         B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
@@ -258,9 +268,17 @@ class AttnProjBlock:
             B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
 
     def select(self, x):
+        """a1 + a2, then the q/k and v/o selections with their kept weight rows: two
+        independent chains (the v/o one on the second stream when concurrent)."""
         self.estimate(x)
-        self.choose()
-        self.compact()
+        if self.concurrent:
+            with self.side.fork():
+                self._vo_chain()
+            self._qk_chain()
+            self.side.join()
+        else:
+            self.choose()
+            self.compact()
 
     def forward(self, x, x_o):
         C = self.n_ctx

@@ -227,65 +227,62 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
       return SL_ERR_INVALID_ARG;
   }
   const int mk = n_proj * k;
-  // bf16 inputs: stage 1 runs on the tensor-core engine (exact bf16 products, fp32
-  // accumulation, fixed-order split-K); fp32 inputs: CUDA-core fp32 FMA kernel.
-  const bool tc = !fp32 && k % 8 == 0;
+  // bf16 inputs: stage 1 on the tensor cores (exact bf16 products, fp32 accumulation,
+  // K-range partials summed in a fixed order); fp32 inputs: CUDA-core fp32 FMA kernel.
+  const bool tc = !fp32 && mk % 4 == 0;
+  int z_split = 1, kb_per = 0;
+  if (tc && est_z_plan(n_ctx, d_in, mk, &z_split, &kb_per)) return SL_ERR_SHAPE;
+  const int64_t tiles = (n_ctx + 127) / 128;
+  if (tc && (tiles > kMaxSplitCounters || tiles > 65535 || n_ctx > 2147483647LL)) return SL_ERR_SHAPE;
   const int n_split = tc ? 1 : est1_splits(d_in);
-  const int n_chunks = gram_groups(n_ctx);
-  const int64_t red = tc ? split_floats(n_ctx, mk, d_in) : 0;
-  auto carve = [&](Carver& c, float** zp, double** gp, void** wat, float** region) {
+  const int n_chunks = tc ? (int)tiles : gram_groups(n_ctx);
+  const bool linear = crit != SL_CRIT_SWIGLU_L2;
+  // SwiGLU with bf16 inputs: criterion on the tensor cores from a bf16 expansion of Z
+  const bool swiglu_tc = tc && !linear;
+  auto carve = [&](Carver& c, float** zp, float** zpart, double** gp, uint16_t** zs) {
     *zp = c.take<float>((size_t)n_split * n_ctx * mk);
-    *gp = c.take<double>((size_t)n_chunks * mk * mk);
-    for (int j = 0; j < n_proj; ++j) wat[j] = tc ? c.take<uint16_t>((size_t)k * d_in) : nullptr;
-    *region = c.take<float>((size_t)red);
+    *zpart = tc && z_split > 1 ? c.take<float>((size_t)z_split * n_ctx * mk) : nullptr;
+    *gp = linear ? c.take<double>((size_t)n_chunks * mk * mk) : nullptr;
+    *zs = swiglu_tc ? c.take<uint16_t>((size_t)n_ctx * 128) : nullptr;
   };
   float* zp;
+  float* zpart;
   double* gp;
-  void* wat[4];
-  float* region;
+  uint16_t* zs;
   {
     Carver c(nullptr);
-    carve(c, &zp, &gp, wat, &region);
+    carve(c, &zp, &zpart, &gp, &zs);
     if (sl_status st = ws_check(ws, c.off)) return st;
   }
   Carver c(ws->ptr);
-  carve(c, &zp, &gp, wat, &region);
+  carve(c, &zp, &zpart, &gp, &zs);
   cudaStream_t s = cs(stream);
   int rc = 0;
   if (tc) {
-    GemmBuilder gb;
-    int64_t off = 0;
-    for (int j = 0; j < n_proj; ++j)
-      if ((rc = transpose_bf16(w_a[j], d_in, k, k, wat[j], d_in, s))) return from_kernel(rc);
-    Prob* p = gb.add((int)n_ctx, mk, kBN, (int)rup(mk, 16));
-    Seg* sg = gb.seg(p, gb.map(x, n_ctx, d_in, ldx, kBM), 0, 0, 0, 0, 0, (int)d_in, kBig);
-    for (int j = 0; j < n_proj; ++j) gb.bsrc(sg, gb.map(wat[j], k, d_in, d_in, k), j * k, k, 0, 0);
-    if (p) {
-      p->epi = EPI_F32;
-      p->out0 = zp;
-      p->ld0 = mk;
-      maybe_split(gb, p, n_ctx, mk, d_in, region, &off);
-    }
-    if ((rc = gb.launch(err_word(ws), s))) return from_builder(rc);
+    int* tickets = err_word(ws) + kCounterOffsetInts;
+    rc = est_z_tc(x, n_ctx, d_in, ldx, n_proj, w_a, k, zpart, zp, linear ? gp : nullptr, zs, tickets, err_word(ws),
+                  s);
+    if (rc) return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
   } else {
     rc = est_stage1(x, fp32, n_ctx, d_in, ldx, n_proj, w_a, fp32, k, zp, n_split, s);
     if (rc) return from_kernel(rc);
+  }
+  if (swiglu_tc) {
+    rc = est_swiglu_tc(zs, n_ctx, k, w_b[0], w_b[1], n_units, scores, err_word(ws), s);
+    return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
   }
   if (crit == SL_CRIT_SWIGLU_L2) {
     rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, err_word(ws), s);
     return from_kernel(rc);
   }
-  rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s);
-  if (rc) return from_kernel(rc);
-  if (crit == SL_CRIT_L2) {
-    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 0, 0, w_b[0], nullptr, fp32, 0, 0, 0, n_units, scores, s);
-    return from_kernel(rc);
-  }
-  rc = est_linear_scores(gp, n_chunks, mk, k, 2, 0, 1, w_b[0], w_b[1], fp32, n_q_heads, n_kv_heads, head_dim, n_units,
-                         scores, s);
-  if (rc) return from_kernel(rc);
-  if (n_proj == 3)
-    rc = est_linear_scores(gp, n_chunks, mk, k, 0, 2, 0, w_b[2], nullptr, fp32, 0, 0, 0, d_out[2], scores_v, s);
+  if (!tc && (rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s))) return from_kernel(rc);
+  if (crit == SL_CRIT_L2)
+    rc = est_scores(gp, n_chunks, mk, k, fp32, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0, n_units, scores,
+                    s);
+  else
+    rc = est_scores(gp, n_chunks, mk, k, fp32, w_b[0], w_b[1], 0, 1, n_q_heads, n_kv_heads, head_dim, scores,
+                    n_proj == 3 ? w_b[2] : nullptr, 2, n_proj == 3 ? d_out[2] : 0, n_proj == 3 ? scores_v : nullptr,
+                    s);
   return from_kernel(rc);
 }
 

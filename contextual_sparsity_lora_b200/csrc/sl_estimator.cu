@@ -326,56 +326,6 @@ __global__ void __cluster_dims__(kGramCluster, 1, 1) __launch_bounds__(256)
   cluster.sync();
 }
 
-struct WbPtrs {
-  const void* p[3];
-  int64_t n[3];
-};
-
-// One thread per unit. crit 0 (L2): units are the output channels of projection
-// `proj`; crit 2 (QK): units are KV channels (g, d), projections 0 = q, 1 = k.
-__global__ void __launch_bounds__(256) est_linear_scores_kernel(const double* __restrict__ gram_part, int n_chunks,
-                                                                int mk, int k, int crit, int proj0, int proj1,
-                                                                WbPtrs wb,
-                                                                int wb_fp32, int n_q_heads, int n_kv_heads,
-                                                                int head_dim, int64_t n_units,
-                                                                float* __restrict__ scores) {
-  pdl_wait();
-  extern __shared__ double gs[];  // [mk][mk]
-  for (int e = threadIdx.x; e < mk * mk; e += blockDim.x) {
-    double s = 0.0;
-#pragma unroll 8
-    for (int c = 0; c < n_chunks; ++c) s += gram_part[(int64_t)c * mk * mk + e];
-    gs[e] = s;
-  }
-  __syncthreads();
-  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (u >= n_units) return;
-  // pj indexes wb (0 or 1); blk is the projection's column block in Z.
-  auto quad = [&](int pj, int blk, int64_t col) -> double {
-    const int off = blk * k;
-    double b[16];
-    for (int c = 0; c < k; ++c) b[c] = (double)ld_any(wb.p[pj], c * wb.n[pj] + col, wb_fp32);
-    double s = 0.0;
-    for (int a = 0; a < k; ++a) {
-      double row = 0.0;
-      for (int c = 0; c < k; ++c) row = fma(gs[(off + a) * mk + off + c], b[c], row);
-      s = fma(b[a], row, s);
-    }
-    return s > 0.0 ? s : 0.0;
-  };
-  double score;
-  if (crit == 0) {
-    score = sqrt(quad(0, proj0, u));
-  } else {
-    const int g = (int)(u / head_dim), d = (int)(u % head_dim);
-    const int hpg = n_q_heads / n_kv_heads;
-    double qs = 0.0;
-    for (int h = g * hpg; h < (g + 1) * hpg; ++h) qs += sqrt(quad(0, proj0, (int64_t)h * head_dim + d));
-    score = qs * sqrt(quad(1, proj1, u));
-  }
-  scores[u] = (float)score;
-}
-
 }  // namespace
 
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
@@ -439,31 +389,6 @@ int est_gram(const float* z, int /*n_split*/, int64_t n_ctx, int mk, double* gra
              cudaStream_t s) {
   if (mk > 64 || n_ctx <= 0) return 1;
   launch_kernel(est_gram_kernel, gram_groups(n_ctx) * kGramCluster, 256, 0, s, z, n_ctx, mk, gram);
-  if (launch_failed("sl_estimator")) return 5;
-  note_launch();
-  return 0;
-}
-
-int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int crit, int proj0, int proj1,
-                      const void* wb0, const void* wb1, int wb_fp32, int n_q_heads, int n_kv_heads, int head_dim,
-                      int64_t n_units, float* scores, cudaStream_t s) {
-  // crit 0 (L2): units = output channels of the projection whose Z columns start at proj0 * k; W_B = wb0.
-  // crit 2 (QK): units = KV channels; q at Z block proj0 (W_B = wb0), k at Z block proj1 (W_B = wb1).
-  if (k > 16 || mk > 64) return 1;
-  WbPtrs w{};
-  if (crit == 0) {
-    w.p[0] = wb0;
-    w.n[0] = n_units;
-  } else {
-    w.p[0] = wb0;
-    w.n[0] = (int64_t)n_q_heads * head_dim;
-    w.p[1] = wb1;
-    w.n[1] = (int64_t)n_kv_heads * head_dim;
-  }
-  const unsigned grid = (unsigned)((n_units + 255) / 256);
-  launch_kernel(est_linear_scores_kernel, grid, 256, (size_t)mk * mk * sizeof(double), s, 
-      gram_part, n_chunks, mk, k, crit == 0 ? 0 : 2, proj0, proj1, w, wb_fp32, n_q_heads, n_kv_heads,
-      crit == 0 ? 1 : head_dim, n_units, scores);
   if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;

@@ -95,10 +95,26 @@ int est_swiglu_scores(const float* zpart, int n_split, int64_t n_ctx, int k, con
                       const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, int* err, cudaStream_t s);
 int est_gram(const float* zpart, int n_split, int64_t n_ctx, int mk, double* gram_part, int n_chunks,
              cudaStream_t s);
-int est_linear_scores(const double* gram_part, int n_chunks, int mk, int k, int crit, int proj0, int proj1,
-                      const void* wb0, const void* wb1, int wb_fp32, int n_q_heads, int n_kv_heads, int head_dim,
-                      int64_t n_units, float* scores, cudaStream_t s);
 int est1_splits(int64_t d_in);
+
+// ---- estimator on the tensor cores (sl_est_tc.cu)
+// Stage-1 plan for bf16 inputs: K-range splits per 128-token tile and 64-wide K blocks per split.
+int est_z_plan(int64_t n_ctx, int64_t d_in, int mk, int* n_split, int* kb_per);
+// z[n_ctx][mk] = x[:, :d_in] [W_A^(0) .. W_A^(n_proj-1)] (W_A^(j) bf16 [d_in, k]); zpart holds
+// the K-range partials (n_split * n_ctx * mk floats when n_split > 1); gram_part, when not
+// null, receives each 128-token tile's fp64 Gram matrix [n_tiles][mk][mk]; zsplit, when not
+// null (two projections, 3k <= 64), receives Z as bf16 terms for est_swiglu_tc. tickets: n_tiles
+// finish counters that are zero between calls.
+int est_z_tc(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj, const void* const* wa, int k,
+             float* zpart, float* z, double* gram_part, void* zsplit, int* tickets, int* err, cudaStream_t s);
+// SwiGLU criterion from zsplit ([n_ctx][128] bf16: Z of gate and of up as three bf16 terms,
+// written by est_z_tc) and the bf16 W_B of gate and up [k, F]; scores[F].
+int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, const void* wb_u, int64_t F,
+                  float* scores, int* err, cudaStream_t s);
+// QK units and/or L2 channels from the Gram partials (sum over n_parts in order), one launch.
+int est_scores(const double* gram_part, int n_parts, int mk, int k, int wb_fp32, const void* wb_q, const void* wb_k,
+               int blk_q, int blk_k, int n_q_heads, int n_kv_heads, int head_dim, float* scores_qk, const void* wb_l2,
+               int blk_l2, int64_t n_l2, float* scores_l2, cudaStream_t s);
 // The Gram kernel runs clusters of 8 CTAs over 48 context tokens each; one fp64 partial
 // Gram matrix per cluster is left for the score kernel to add.
 inline int gram_groups(int64_t n_ctx) { return (int)((n_ctx + 8 * 48 - 1) / (8 * 48)); }
@@ -139,5 +155,8 @@ int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, 
 int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
                       void* dst, int64_t ld_dst, cudaStream_t s);
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s);
+// Tensor map of a bf16 matrix [rows, cols] (ld elements) with box_cols x box_rows boxes.
+bool encode_bf16_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols,
+                    int box_rows, bool swizzle128);
 
 }  // namespace sl

@@ -1,12 +1,17 @@
-// Top-n channel selection by radix select over fp32 scores (one CTA per call).
+// Top-n channel selection over fp32 scores (one CTA of 1024 threads per call).
 //
-// Scores become order-preserving 32-bit keys (NaN lowest, -0 == +0). Four 8-bit
-// passes over shared-memory histograms find the n-th largest key K*; every key
-// above K* is kept, and among keys equal to K* the lowest indices are kept, so
-// exactly n channels survive. The output is a permutation sigma of [0, N):
-// sigma[0, n) = kept channels ascending, sigma[n, N) = dropped channels
-// ascending. Optionally the selection over KV units (g, d) is expanded to the
-// query side: query channel (h, d) is kept iff unit (h / heads_per_group, d) is.
+// Scores become order-preserving 32-bit keys (NaN lowest, -0 == +0), held in registers:
+// thread t owns the contiguous index range [t * per, (t + 1) * per). The n-th largest key
+// K* is found bit by bit from the most significant bit on: starting from the bits that all
+// keys share, a candidate bit is kept when at least n keys are >= the threshold with that
+// bit set (one block-wide count per bit; the search stops early when a threshold has
+// exactly n keys at or above it). Every key above K* is kept, and among keys equal to K*
+// the lowest indices are kept, so exactly n channels survive. The output is a permutation
+// sigma of [0, N): sigma[0, n) = kept channels ascending, sigma[n, N) = dropped channels
+// ascending. Optionally the selection over KV units (g, d) is expanded to the query side:
+// query channel (h, d) is kept iff unit (h / heads_per_group, d) is. Scores come in and
+// sigma goes out through shared memory with coalesced global accesses (one CTA issues all of
+// them, so per-thread strided accesses would pay a 32-byte sector per 4-byte element).
 #include "sl_internal.h"
 
 namespace sl {
@@ -14,7 +19,8 @@ namespace sl {
 namespace {
 
 constexpr int kSelThreads = 1024;
-constexpr int kSelMaxN = 40960;  // keys + flags in shared memory
+constexpr int kSelMaxN = 40960;
+constexpr int kSelStageWords = 40960;  // staging words for scores in / sigma out (160 KB)
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -23,8 +29,8 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan of one int per thread (1024 threads). Returns the total.
-__device__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
+// Exclusive block scan of one int per thread (1024 threads). Returns the thread's prefix.
+__device__ int block_exclusive_scan(int v, int* warp_sums) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -35,7 +41,7 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_sums[lane];
+    const int w = warp_sums[lane];
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -43,124 +49,167 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
       if (lane >= o) wi += n;
     }
     warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
-    if (lane == 31) warp_sums[32] = wi;
   }
   __syncthreads();
   const int excl = warp_sums[warp] + incl - v;
-  total = warp_sums[32];
   __syncthreads();
   return excl;
 }
 
+// Block-wide sum of one int per thread; `slot` alternates between calls so that one
+// barrier per call suffices (a slot is rewritten only two calls later, after every
+// thread has passed the barrier of the call in between).
+__device__ __forceinline__ int block_sum(int v, int (*red)[32], int& slot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_add_sync(0xffffffffu, v);
+  if (lane == 0) red[slot][warp] = v;
+  __syncthreads();
+  const int tot = __reduce_add_sync(0xffffffffu, red[slot][lane]);
+  slot ^= 1;
+  return tot;
+}
+
+__host__ __device__ inline int stage_words(int n, int n_wide) {
+  return n_wide <= kSelStageWords && n_wide > n ? n_wide : n;
+}
+
+template <int PER>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores, int n, int n_keep,
                                                              int32_t* __restrict__ sigma, int hpg, int head_dim,
                                                              int n_wide, int32_t* __restrict__ sigma_wide) {
   pdl_wait();
-  extern __shared__ uint32_t sel_smem[];
-  uint32_t* keys = sel_smem;                                    // [n]
-  uint8_t* keep = reinterpret_cast<uint8_t*>(keys + n);         // [n]
-  __shared__ int hist[256];
-  __shared__ int warp_sums[33];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_remaining;
-
-  for (int i = threadIdx.x; i < n; i += kSelThreads) keys[i] = score_key(scores[i]);
-  if (threadIdx.x == 0) {
-    s_prefix = 0;
-    s_mask = 0;
-    s_remaining = n_keep;
-  }
+  // staging words for scores in / sigma out (and sigma_wide when it fits), then [n] kept flags
+  extern __shared__ uint32_t sbuf[];
+  uint8_t* keep = reinterpret_cast<uint8_t*>(sbuf + stage_words(n, n_wide));
+  __shared__ int red[2][32];
+  __shared__ uint32_t s_or[32], s_and[32];
+  __shared__ int warp_sums[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = (n + kSelThreads - 1) / kSelThreads;  // <= PER
+  const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
+  for (int i = threadIdx.x; i < n; i += kSelThreads) sbuf[i] = __float_as_uint(scores[i]);
   __syncthreads();
 
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    // Scores concentrate in few exponent bins: aggregate equal bins within a warp so each
-    // bin takes one shared-memory atomic per warp instead of one per lane.
-    const int n_round = (n + kSelThreads - 1) / kSelThreads * kSelThreads;
-    for (int i = threadIdx.x; i < n_round; i += kSelThreads) {
-      const uint32_t k = i < n ? keys[i] : 0u;
-      const bool active = i < n && (k & mask) == prefix;
-      const uint32_t bin = active ? ((k >> shift) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (active && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      // lane l owns bins [255 - 8l - 7, 255 - 8l], walked from the top
-      const int lane = threadIdx.x;
-      int local = 0;
-      for (int j = 0; j < 8; ++j) local += hist[255 - 8 * lane - j];
-      int incl = local;
+  uint32_t key[PER];
+  uint32_t kor = 0u, kand = 0xffffffffu;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int rem = s_remaining;
-      const int excl = incl - local;
-      const bool here = excl < rem && incl >= rem;
-      const unsigned ball = __ballot_sync(0xffffffffu, here);
-      if (here && lane == __ffs(ball) - 1) {
-        int cum = excl;
-        for (int j = 0; j < 8; ++j) {
-          const int b = 255 - 8 * lane - j;
-          if (cum + hist[b] >= rem) {
-            s_remaining = rem - cum;
-            s_prefix = prefix | ((uint32_t)b << shift);
-            s_mask = mask | (255u << shift);
-            break;
-          }
-          cum += hist[b];
-        }
-      }
+  for (int j = 0; j < PER; ++j) {
+    const int i = i0 + j;
+    key[j] = i < i1 ? score_key(__uint_as_float(sbuf[i])) : 0u;
+    if (i < i1) {
+      kor |= key[j];
+      kand &= key[j];
     }
-    __syncthreads();
   }
-  const uint32_t thr = s_prefix;
-  const int take_eq = s_remaining;
-
-  // Each thread owns a contiguous index range, so block scans give index-order ranks.
-  const int per = (n + kSelThreads - 1) / kSelThreads;
-  const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
-  int n_eq = 0;
-  for (int i = i0; i < i1; ++i) n_eq += keys[i] == thr;
-  int tot;
-  int eq_rank = block_exclusive_scan(n_eq, warp_sums, tot);
+  kor = __reduce_or_sync(0xffffffffu, kor);
+  kand = __reduce_and_sync(0xffffffffu, kand);
+  if (lane == 0) {
+    s_or[warp] = kor;
+    s_and[warp] = kand;
+  }
+  __syncthreads();
+  const uint32_t bor = __reduce_or_sync(0xffffffffu, s_or[lane]);
+  const uint32_t band = __reduce_and_sync(0xffffffffu, s_and[lane]);
+  // Every key carries the bits above the highest bit in which two keys differ: the search
+  // starts below it, from a threshold that all n keys reach.
+  const uint32_t diff = bor ^ band;
+  int b = diff ? 31 - __clz(diff) : -1;
+  uint32_t T = diff ? (band & ~((2u << b) - 1u)) : band;
+  int slot = 0;
+  for (; b >= 0; --b) {
+    const uint32_t Tp = T | (1u << b);
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) c += key[j] >= Tp ? 1 : 0;  // padding keys are 0 < Tp
+    const int tot = block_sum(c, red, slot);
+    if (tot >= n_keep) {
+      T = Tp;
+      if (tot == n_keep) break;  // exactly n keys at or above T
+    }
+  }
+  // Keys above T are kept; keys equal to T fill the remaining places lowest index first.
+  int gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const bool valid = i0 + j < i1;
+    gt += valid && key[j] > T ? 1 : 0;
+    n_eq += valid && key[j] == T ? 1 : 0;
+  }
+  const int take_eq = n_keep - block_sum(gt, red, slot);
+  int eq_rank = block_exclusive_scan(n_eq, warp_sums);
+  uint64_t kmask = 0;
   int n_kept = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t k = keys[i];
-    bool kp = k > thr;
-    if (k == thr) {
-      kp = eq_rank < take_eq;
-      ++eq_rank;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    if (i0 + j >= i1) break;
+    bool kp = key[j] > T;
+    if (key[j] == T) kp = eq_rank++ < take_eq;
+    if (kp) {
+      kmask |= 1ull << j;
+      ++n_kept;
     }
-    keep[i] = kp;
-    n_kept += kp;
   }
-  int kept_before = block_exclusive_scan(n_kept, warp_sums, tot);
+  int kept_before = block_exclusive_scan(n_kept, warp_sums);  // also orders the key reads before the reuse
   int drop_before = i0 - kept_before;
-  for (int i = i0; i < i1; ++i) {
-    if (keep[i]) sigma[kept_before++] = i;
-    else sigma[n_keep + drop_before++] = i;
+  const bool wide = hpg > 0 && sigma_wide != nullptr;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int i = i0 + j;
+    if (i >= i1) break;
+    const bool kp = (kmask >> j) & 1ull;
+    // exactly n_keep keys are kept, so both ranges stay inside [0, n); the checks only
+    // keep a broken invariant from writing past them
+    if (kp) {
+      if (kept_before < n_keep) sbuf[kept_before] = (uint32_t)i;
+      ++kept_before;
+    } else {
+      if (n_keep + drop_before < n) sbuf[n_keep + drop_before] = (uint32_t)i;
+      ++drop_before;
+    }
+    if (wide) keep[i] = kp;
   }
-  if (hpg <= 0 || sigma_wide == nullptr) return;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kSelThreads) sigma[i] = (int32_t)sbuf[i];
+  if (!wide) return;
   __syncthreads();
   // Query-side expansion: channel c = h * head_dim + d follows unit (h / hpg) * head_dim + d.
   const int n_keep_w = n_keep * hpg;
+  const bool staged = n_wide <= kSelStageWords;
   const int perw = (n_wide + kSelThreads - 1) / kSelThreads;
   const int w0 = min(n_wide, (int)threadIdx.x * perw), w1 = min(n_wide, w0 + perw);
   auto unit_of = [&](int c) { return (c / head_dim / hpg) * head_dim + c % head_dim; };
   int nk = 0;
   for (int c = w0; c < w1; ++c) nk += keep[unit_of(c)];
-  int kb = block_exclusive_scan(nk, warp_sums, tot);
+  int kb = block_exclusive_scan(nk, warp_sums);
   int db = w0 - kb;
+  uint32_t* out = staged ? sbuf : reinterpret_cast<uint32_t*>(sigma_wide);
   for (int c = w0; c < w1; ++c) {
-    if (keep[unit_of(c)]) sigma_wide[kb++] = c;
-    else sigma_wide[n_keep_w + db++] = c;
+    if (keep[unit_of(c)]) {
+      if (kb < n_keep_w) out[kb] = (uint32_t)c;
+      ++kb;
+    } else {
+      if (n_keep_w + db < n_wide) out[n_keep_w + db] = (uint32_t)c;
+      ++db;
+    }
   }
+  if (!staged) return;
+  __syncthreads();
+  for (int c = threadIdx.x; c < n_wide; c += kSelThreads) sigma_wide[c] = (int32_t)sbuf[c];
+}
+
+template <int PER>
+void launch_select(const float* scores, int n, int n_keep, int32_t* sigma, int hpg, int head_dim, int n_wide,
+                   int32_t* sigma_wide, cudaStream_t s) {
+  if (!sigma_wide) n_wide = 0;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(select_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kSelStageWords * 4 + kSelMaxN + 16);
+    attr = true;
+  }
+  const size_t smem = (size_t)stage_words(n, sigma_wide ? n_wide : 0) * 4 + (sigma_wide ? ((size_t)n + 15) / 16 * 16 : 0);
+  launch_kernel(select_kernel<PER>, 1, kSelThreads, smem, s, scores, n, n_keep, sigma, hpg, head_dim, n_wide,
+                sigma_wide);
 }
 
 }  // namespace
@@ -170,15 +219,15 @@ int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sig
   if (n <= 0 || n > kSelMaxN || n_keep < 1 || n_keep > n) return 1;
   if (sigma_wide && (heads_per_group <= 0 || head_dim <= 0 || n % head_dim || n_wide != n * heads_per_group))
     return 1;
-  const size_t smem = (size_t)n * 5;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxN * 5 + 64);
-    attr = true;
-  }
-  launch_kernel(select_kernel, 1, kSelThreads, (smem + 15) / 16 * 16, s, scores, (int)n, (int)n_keep, sigma,
-                                                               sigma_wide ? heads_per_group : 0, head_dim,
-                                                               (int)n_wide, sigma_wide);
+  const int hpg = sigma_wide ? heads_per_group : 0;
+  if (n <= kSelThreads)
+    launch_select<1>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  else if (n <= 4 * kSelThreads)
+    launch_select<4>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  else if (n <= 16 * kSelThreads)
+    launch_select<16>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  else
+    launch_select<40>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
   if (n_keep_wide_out) *n_keep_wide_out = sigma_wide ? n_keep * heads_per_group : 0;
   if (launch_failed("sl_select")) return 5;
   note_launch();

@@ -259,8 +259,8 @@ SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launche
 /* Per-launch view of the same GEMM-engine event pairs, without resetting them (call it
  * before sl_profile_read): *count = launches recorded; for the first min(count, capacity)
  * of them, in launch order, ms[i] = duration and kind[i] = 0 (one-CTA grouped launch),
- * 1 (CTA pairs, 256-row tiles), 2 (CTA pairs, 512-row tiles) or 3 (fused LoRA backward
- * stream). Waits for the events. */
+ * 1 (CTA pairs, 256-row tiles), 2 (CTA pairs, 512-row tiles), 3 (fused LoRA backward
+ * stream) or 4 (estimator stage 1). Waits for the events. */
 SL_API sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count);
 
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */

@@ -236,7 +236,8 @@ def test_estimator_l2_fp32_inputs():
     assert rel_fro(s, want) < FP32_TOL
 
 
-@pytest.mark.parametrize("n,n_keep", [(1, 1), (7, 3), (1000, 1), (1000, 1000), (14336, 7168), (40960, 12345)])
+@pytest.mark.parametrize("n,n_keep", [(1, 1), (7, 3), (1000, 1), (1000, 1000), (1025, 513), (4096, 4095),
+                                        (14336, 7168), (16384, 5000), (16385, 8000), (40960, 12345)])
 def test_select_edge_cases_bit_exact(n, n_keep):
     rng = np.random.default_rng(n + n_keep)
     s = rng.integers(0, 50, n).astype(np.float32)          # heavy ties
@@ -244,6 +245,21 @@ def test_select_edge_cases_bit_exact(n, n_keep):
     s[rng.random(n) < 0.02] = -np.inf
     s[rng.random(n) < 0.02] = -0.0
     s[rng.random(n) < 0.02] = 0.0
+    sc = torch.tensor(s, device=DEV)
+    sig = torch.empty(n, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(sc, n_keep, sig)
+    want = oracle.select_top(s.astype(np.float64), n_keep)
+    got = sig.cpu().numpy()
+    np.testing.assert_array_equal(got[:n_keep], want)
+    np.testing.assert_array_equal(got[n_keep:], oracle.complement(want, n))
+
+
+@pytest.mark.parametrize("n,n_keep", [(1024, 512), (4096, 1229), (14336, 4301), (14336, 10036), (20000, 7)])
+def test_select_continuous_scores_bit_exact(n, n_keep):
+    """Distinct scores spread over a narrow range (criterion-like): the threshold search
+    mostly ends on a threshold with exactly n_keep scores at or above it."""
+    rng = np.random.default_rng(7 * n + n_keep)
+    s = (1.0 + rng.standard_normal(n) ** 2).astype(np.float32)
     sc = torch.tensor(s, device=DEV)
     sig = torch.empty(n, dtype=torch.int32, device=DEV)
     B.sl_select_channels(sc, n_keep, sig)
