@@ -387,29 +387,36 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   // K extents of the dB / dA parts: pass 0 = natural part (all rows, or output rows when the
   // operand is in the sigma layout), pass 1 = context rows of a sigma-layout operand.
   auto kpart = [&](bool sig, int pass) -> int64_t { return sig ? (pass ? C : O) : (pass ? 0 : T); };
-  int64_t red1 = 0, red2[2] = {0, 0};
-  for (int i = 0; i < n_ad; ++i) {
-    const sl_linear& L = lin[i];
-    red1 += out_sig ? split_floats(C, L.r, L.d_out) + split_floats(O, L.r, L.d_out) : split_floats(T, L.r, L.d_out);
-    for (int pass = 0; pass < 2; ++pass) {
-      red2[pass] += kpart(out_sig, pass) > 0 ? split_floats(L.d_out, L.r, kpart(out_sig, pass)) : 0;
-      red2[pass] += kpart(in_sig, pass) > 0 ? split_floats(d_in, L.r, kpart(in_sig, pass)) : 0;
-    }
+  // dA of adapters that share x and the rank (up to three, x in the natural layout) come from
+  // one product x^T [dya_1 | dya_2 | ...] over an interleaved bf16 copy of their dya
+  bool merge_da = n_ad >= 2 && n_ad <= 3 && !in_sig && R <= 128;
+  for (int i = 1; i < n_ad; ++i) merge_da = merge_da && lin[i].r == lin[0].r;
+  // split-K partials of the dA products (the two launches reuse them in stream order)
+  int64_t red = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int64_t K = kpart(in_sig, pass);
+    if (K <= 0) continue;
+    int64_t r2 = 0;
+    if (merge_da) r2 = split_floats(d_in, R, K);
+    else
+      for (int i = 0; i < n_ad; ++i) r2 += split_floats(d_in, lin[i].r, K);
+    red = std::max(red, r2);
   }
-  const int64_t red = std::max(red1, std::max(red2[0], red2[1]));
-  auto carve = [&](Carver& c, void** bsig, float** region) {
+  auto carve = [&](Carver& c, void** bsig, void** dcat, float** region) {
     for (int i = 0; i < n_ad; ++i) bsig[i] = out_sig ? c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r) : nullptr;
+    *dcat = merge_da ? c.take<uint16_t>((size_t)T * R) : nullptr;
     *region = c.take<float>((size_t)red);
   };
   void* bsig[4];
+  void* dcat;
   float* region;
   {
     Carver c(nullptr);
-    carve(c, bsig, &region);
+    carve(c, bsig, &dcat, &region);
     if (sl_status st = ws_check(ws, c.off)) return st;
   }
   Carver c(ws->ptr);
-  carve(c, bsig, &region);
+  carve(c, bsig, &dcat, &region);
   if (out_sig)
     for (int i = 0; i < n_ad; ++i)
       if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i],
@@ -423,12 +430,16 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     const float* csrc[4];
     void* cdst[4];
     int64_t ccount[4];
+    int cr[4];
     int64_t koff = 0;
     for (int i = 0; i < n_ad; ++i) {
       const sl_linear& L = lin[i];
+      // dya and dB are sums of reductions into zeroed outputs; dA accumulates its two parts
       if (cudaMemsetAsync(dya[i], 0, sizeof(float) * T * L.r, s) != cudaSuccess ||
-          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s) != cudaSuccess)
+          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s) != cudaSuccess ||
+          cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s) != cudaSuccess)
         return SL_ERR_CUDA;
+      cr[i] = L.r;
       const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
       koff += L.r;
       auto add = [&](int64_t row0, int64_t rows, const void* Bm, const int32_t* sig) {
@@ -460,51 +471,45 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
       ccount[i] = T * L.r;
     }
     if (int rc = lora_dual_launch(sp, nsp, err_word(ws), s)) return from_builder(rc);
-    if (int rc = cast_f32_bf16(csrc, cdst, ccount, n_ad, s)) return from_kernel(rc);
+    if (int rc = cast_f32_bf16(csrc, cdst, ccount, n_ad, s, dcat, cr, R)) return from_kernel(rc);
   }
-  // launch 2: dB = dy^T xa_s and dA = (x^T dya)^T over the natural parts; launch 3: the
-  // context parts of sigma-layout operands, accumulated onto launch 2's results.
+  // dA = (x^T dya)^T, added into the zeroed dA: launch 2 over the natural part of x (all rows,
+  // or the output rows when x is in the sigma layout), launch 3 over the context rows of a
+  // sigma-layout x (rows through sigma). Split-K partials are summed in a fixed order.
   for (int pass = 0; pass < 2; ++pass) {
+    const int64_t K = kpart(in_sig, pass);
+    if (K <= 0) continue;
+    const bool ctx_part = pass == 1;
+    const int64_t rows = ctx_part ? C : T;  // map extents zero-fill past the part
+    const int64_t k0 = (in_sig && !ctx_part) ? C : 0;
     GemmBuilder gb;
     int64_t off = 0;
-    bool any = false;
-    for (int i = 0; i < n_ad; ++i) {
-      const sl_linear& L = lin[i];
-      int64_t koff = 0;
-      for (int i2 = 0; i2 < i; ++i2) koff += lin[i2].r;
-      const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
-      for (int which = 1; which < 2; ++which) {  // dA (dB came from the fused kernel)
-        const bool sig = which == 0 ? out_sig : in_sig;
-        const int64_t K = kpart(sig, pass);
-        const bool ctx_part = pass == 1;
-        if (K <= 0) {
-          if (!ctx_part) {
-            if (which == 0) cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s);
-            else cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s);
-          }
-          continue;
-        }
-        const int64_t rows = ctx_part ? C : T;  // map extents zero-fill past the part
-        const int64_t k0 = (sig && !ctx_part) ? C : 0;
-        const int64_t M = which == 0 ? L.d_out : d_in;
-        const int ma = which == 0 ? gb.map(dy[i], rows, L.d_out, ld_dy[i], 64) : gb.map(x, rows, d_in, ldx, 64);
-        const int mb = which == 0 ? gb.map(xa_blk, rows, L.r, ld_xa, 64) : gb.map(dya_s[i], rows, L.r, L.r, 64);
-        Prob* p = gb.add((int)M, L.r, kBN, (int)rup(L.r, 16));
-        Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
-        gb.bsrc(sg, mb, 0, 64, 0, 0);
-        if (p) {
-          p->epi = which == 0 ? EPI_F32 : EPI_F32_T;
-          p->out0 = which == 0 ? (void*)dB[i] : (void*)dA[i];
-          p->ld0 = which == 0 ? L.r : d_in;
-          p->beta = ctx_part ? 1 : 0;
-          p->row_map = ctx_part ? (which == 0 ? out_ch[i].sigma : in_ch->sigma) : nullptr;
-          maybe_split(gb, p, M, L.r, K, region, &off);
-        }
-        any = true;
+    const int ma = gb.map(x, rows, d_in, ldx, 64);
+    auto add_da = [&](int n, const void* bsrc, int64_t ldb, int i0) {
+      const int bcols = (int)rup(n, 64);
+      const int mb = gb.map(bsrc, rows, n, ldb, 64);
+      Prob* p = gb.add((int)d_in, n, kBN, (int)rup(n, 16));
+      Seg* sg = gb.seg(p, ma, 1, 0, (int)k0, 1, (int)k0, (int)K, kBig);
+      gb.bsrc(sg, mb, 0, bcols, 0, 0);
+      if (!p) return;
+      p->epi = EPI_F32_T;
+      p->out0 = dA[i0];
+      p->ld0 = d_in;
+      p->beta = 1;
+      p->row_map = ctx_part ? in_ch->sigma : nullptr;
+      if (n > lin[i0].r) {
+        p->col_split = lin[i0].r;
+        p->out1 = dA[i0 + 1];
+        p->out2 = n_ad > 2 ? dA[i0 + 2] : nullptr;
       }
+      maybe_split(gb, p, d_in, n, K, region, &off);
+    };
+    if (merge_da) {
+      add_da(R, dcat, R, 0);
+    } else {
+      for (int i = 0; i < n_ad; ++i) add_da(lin[i].r, dya_s[i], lin[i].r, i);
     }
-    if (any)
-      if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
+    if (int rc = gb.launch(err_word(ws), s)) return from_builder(rc);
   }
   return SL_OK;
 }

@@ -24,6 +24,17 @@ struct TileInfo {
   int prob, tm, tn, ks, kb0, kb1;  // ks: split-K index; [kb0, kb1): k-block range (over all segments)
 };
 
+// Row `col` of the transposed fp32 output of an EPI_F32_T problem (col_split: columns in
+// blocks of col_split go to out0, out1, out2).
+__device__ __forceinline__ float* f32t_dst(const Prob& pr, int64_t col) {
+  if (pr.col_split) {
+    const int j = (int)(col / pr.col_split);
+    void* o = j == 0 ? pr.out0 : (j == 1 ? pr.out1 : pr.out2);
+    return reinterpret_cast<float*>(o) + (col - (int64_t)j * pr.col_split) * pr.ld0;
+  }
+  return reinterpret_cast<float*>(pr.out0) + col * pr.ld0;
+}
+
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
   int pi = 0;
   for (int i = 0; i < p.nprob; ++i)
@@ -280,12 +291,11 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         break;
       }
       case EPI_F32_T: {
-        float* out = reinterpret_cast<float*>(pr.out0);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i >= n) break;
           const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
-          float* d = out + col * pr.ld0 + orow;
+          float* d = f32t_dst(pr, col) + orow;
           *d = pr.a0 * v[i] + (pr.beta ? *d : 0.f);
         }
         break;
@@ -338,13 +348,14 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
   }
 }
 
-// Split-K tile: the raw fp32 accumulator goes to part[ks][row][col]; the reduce kernel
+// Split-K tile: the raw fp32 accumulator goes to part[ks][col][row] (column-major, so the
+// threads of a warp, one row each, store 128 contiguous bytes per column); the reduce kernel
 // sums the splits in a fixed order and applies the problem's epilogue.
 __device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t tb, int half) {
   const int row = m0 + r;
   const bool rv = row < pr.M;
   uint32_t raw[32];
-  float* dst = pr.part + ((int64_t)ks * pr.M + row) * pr.N;
+  float* dst = pr.part + (int64_t)ks * pr.N * pr.M + row;
   for (int c0 = 32 * half; c0 < pr.n_mma; c0 += 64) {
     if (c0 >= pr.N) break;
     __syncwarp();
@@ -354,15 +365,16 @@ __device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t
     const int n = min(32, pr.N - c0);
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-      if (i < n) dst[c0 + i] = __uint_as_float(raw[i]);
+      if (i < n) dst[(int64_t)(c0 + i) * pr.M] = __uint_as_float(raw[i]);
   }
 }
 
 struct RedProb {
-  int32_t M, N, ksplit, epi, beta, out_row0;
+  int32_t M, N, ksplit, epi, beta, out_row0, col_split, pad_;
   int64_t ld0, ld1;
   void* out0;
   void* out1;
+  void* out2;
   const int32_t* row_map;
   const int32_t* col_map;
   const float* part;
@@ -372,49 +384,34 @@ struct RedParams {
   RedProb p[kMaxProbs];
 };
 
-// Fixed-order sum of split-K partials + the problem's epilogue (EPI_XA, EPI_F32, EPI_F32_T).
+__device__ __forceinline__ float* f32t_out(const RedProb& pr, int64_t col) {
+  if (pr.col_split) {
+    const int j = (int)(col / pr.col_split);
+    void* o = j == 0 ? pr.out0 : (j == 1 ? pr.out1 : pr.out2);
+    return reinterpret_cast<float*>(o) + (col - (int64_t)j * pr.col_split) * pr.ld0;
+  }
+  return reinterpret_cast<float*>(pr.out0) + col * pr.ld0;
+}
+
+// Fixed-order sum of split-K partials (column-major [ksplit][N][M]) + the problem's epilogue
+// (EPI_XA, EPI_F32, EPI_F32_T). Consecutive threads take consecutive rows of a column, so the
+// partial loads and the transposed stores are contiguous.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ RedParams rp) {
   pdl_wait();
   const RedProb& pr = rp.p[blockIdx.y];
   const int64_t total = (int64_t)pr.M * pr.N;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  if (pr.epi != EPI_F32_T && pr.N % 4 == 0 && !pr.col_map) {
-    // four consecutive columns per thread: 16-byte partial loads
-    for (int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; e < total; e += stride * 4) {
-      const int64_t row = e / pr.N, col = e % pr.N;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s = 0; s < pr.ksplit; ++s) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(pr.part + (int64_t)s * total + e));
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      const int64_t orow = pr.row_map ? (int64_t)pr.row_map[row] : pr.out_row0 + row;
-      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (pr.epi == EPI_XA) {
-          reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + col + j] = pr.a0 * a[j];
-          reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + col + j] = __float2bfloat16_rn(pr.a1 * a[j]);
-        } else {
-          float* d = reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + col + j;
-          *d = pr.a0 * a[j] + (pr.beta ? *d : 0.f);
-        }
-      }
-    }
-    return;
-  }
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
-    // transposed stores walk rows fastest so that consecutive threads write consecutive addresses
-    const int64_t row = pr.epi == EPI_F32_T ? e % pr.M : e / pr.N;
-    const int64_t col = pr.epi == EPI_F32_T ? e / pr.M : e % pr.N;
+    const int64_t row = e % pr.M, col = e / pr.M;
     float acc = 0.f;
-    for (int s = 0; s < pr.ksplit; ++s) acc += pr.part[((int64_t)s * pr.M + row) * pr.N + col];
+    for (int s = 0; s < pr.ksplit; ++s) acc += __ldg(pr.part + (int64_t)s * total + e);
     const int64_t orow = pr.row_map ? (int64_t)pr.row_map[row] : pr.out_row0 + row;
     const int64_t ocol = pr.col_map ? (int64_t)pr.col_map[col] : col;
     if (pr.epi == EPI_XA) {
       reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + ocol] = pr.a0 * acc;
       reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + ocol] = __float2bfloat16_rn(pr.a1 * acc);
     } else {
-      float* d = reinterpret_cast<float*>(pr.out0) + (pr.epi == EPI_F32_T ? ocol * pr.ld0 + orow : orow * pr.ld0 + ocol);
+      float* d = pr.epi == EPI_F32_T ? f32t_out(pr, ocol) + orow : reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + ocol;
       *d = pr.a0 * acc + (pr.beta ? *d : 0.f);
     }
   }
@@ -1245,6 +1242,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     if (pr.ksplit <= 1 || pr.M <= 0 || pr.N <= 0) continue;
     RedProb& q = rp.p[nred++];
     q.M = pr.M; q.N = pr.N; q.ksplit = pr.ksplit; q.epi = pr.epi; q.beta = pr.beta; q.out_row0 = pr.out_row0;
+    q.col_split = pr.col_split; q.out2 = pr.out2;
     q.ld0 = pr.ld0; q.ld1 = pr.ld1; q.out0 = pr.out0; q.out1 = pr.out1; q.row_map = pr.row_map;
     q.col_map = pr.col_map; q.part = pr.part; q.a0 = pr.a0; q.a1 = pr.a1;
     maxmn = std::max<int64_t>(maxmn, (int64_t)pr.M * pr.N);

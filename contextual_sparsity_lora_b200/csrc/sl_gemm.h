@@ -72,6 +72,8 @@ struct Prob {
   int32_t nseg;
   Seg seg[kMaxSegs];
   int32_t epi, beta;
+  int32_t col_split;    // EPI_F32_T: output columns [j * col_split, (j + 1) * col_split) go to
+                        // out_j (j < 3), column c - j * col_split; 0 = all columns to out0
   int32_t out_row0;     // first output row
   int8_t omap[4];       // tensor maps (32 x 32 boxes) of out0..out2 (SwiGLU backward: dg, du, g, u)
                         // over rows [out_row0, out_row0 + M), for the epilogue's bulk tensor copies;
@@ -85,7 +87,7 @@ struct Prob {
   const int32_t* col_map;  // optional: output column j -> col_map[j]
   const int32_t* row_map;  // optional: output row i (problem-local) -> row_map[i]
   float a0, a1;
-  float* part;          // split-K partials [ksplit][M][N] fp32 (workspace)
+  float* part;          // split-K partials [ksplit][N][M] fp32 (workspace, column-major)
 };
 
 struct GemmParams {

@@ -376,11 +376,14 @@ __global__ void __launch_bounds__(kDualThreads, 1) lora_dual_kernel(const __grid
   }
 }
 
-// dya_s = bf16(dya) for every adapter of the call (dya already holds the scale).
+// dya_s = bf16(dya) for every adapter of the call (dya already holds the scale); with `cat`,
+// the same values also go to column block [coff, coff + r) of cat [rows, ld_cat].
 struct CastJob {
   const float* src;
   __nv_bfloat16* dst;
   int64_t n;
+  __nv_bfloat16* cat;
+  int32_t r, coff, ld_cat, pad_;
 };
 struct CastParams {
   CastJob j[kMaxDualJobs];
@@ -390,8 +393,11 @@ struct CastParams {
 __global__ void __launch_bounds__(256) cast_bf16_kernel(const __grid_constant__ CastParams p) {
   pdl_wait();
   const CastJob& c = p.j[blockIdx.y];
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.n; i += (int64_t)gridDim.x * blockDim.x)
-    c.dst[i] = __float2bfloat16_rn(c.src[i]);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.n; i += (int64_t)gridDim.x * blockDim.x) {
+    const __nv_bfloat16 v = __float2bfloat16_rn(c.src[i]);
+    c.dst[i] = v;
+    if (c.cat) c.cat[(i / c.r) * c.ld_cat + c.coff + i % c.r] = v;
+  }
 }
 
 bool encode(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows) {
@@ -462,14 +468,23 @@ int lora_dual_launch(const DualSpec* specs, int n, int* err, cudaStream_t s) {
   return 0;
 }
 
-int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* count, int n, cudaStream_t s) {
+int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* count, int n, cudaStream_t s,
+                  void* cat, const int* r, int ld_cat) {
   if (n <= 0) return 0;
   if (n > kMaxDualJobs) return 1;
   CastParams P;
   memset(&P, 0, sizeof(P));
   int64_t mx = 0;
+  int coff = 0;
   for (int i = 0; i < n; ++i) {
-    P.j[i] = CastJob{src[i], static_cast<__nv_bfloat16*>(dst[i]), count[i]};
+    P.j[i] = CastJob{src[i], static_cast<__nv_bfloat16*>(dst[i]), count[i], nullptr, 1, 0, 0, 0};
+    if (cat) {
+      P.j[i].cat = static_cast<__nv_bfloat16*>(cat);
+      P.j[i].r = r[i];
+      P.j[i].coff = coff;
+      P.j[i].ld_cat = ld_cat;
+      coff += r[i];
+    }
     mx = std::max(mx, count[i]);
   }
   P.n = n;

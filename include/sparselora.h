@@ -198,7 +198,8 @@ SL_API sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_ke
  * SL_LORA_BWD: for each adapter i with output gradient dy[i] [n_tok, d_out_i] (ld ld_dy[i]):
  *   dya[i] (fp32 [n_tok, r_i], ld r_i) = scale * dy B;  dya_s[i] (bf16, same) = dya;
  *   dB[i] (fp32 [d_out_i, r_i]) = scale * dy^T xa = dy^T xa_s;
- *   dA[i] (fp32 [r_i, d_in]) = dya^T x.
+ *   dA[i] (fp32 [r_i, d_in]) = dya^T x (adapters of equal rank that share x in the natural
+ *   layout, up to three, form one product over x).
  *   dya and dB come from one pass over dy whose partial sums meet in fp32 reductions, so
  *   their last bits may differ between runs; dya and dB must be 16-byte aligned.
  *   xa_s is the forward's bf16 block for adapter i (ld ld_xa, column offset = sum of
