@@ -140,8 +140,9 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def make_layer(ratio, seed_w, seed_x, device, dense=False):
-    """The two blocks of one LLaMA3-8B layer plus their per-step inputs (context-first rows)."""
+def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None):
+    """The two blocks of one LLaMA3-8B layer plus their per-step inputs (context-first rows).
+    dp: a blocks.DataParallel over the ranks (one index set per global batch), or None."""
     from contextual_sparsity_lora_b200 import blocks
     ac = inputs.LLAMA3_8B_ATTN
     fc = inputs.LLAMA3_8B_FFN
@@ -151,9 +152,9 @@ def make_layer(ratio, seed_w, seed_x, device, dense=False):
     C = int(da["ctx_mask"].sum())
     attn = blocks.AttnProjBlock(da["q"], da["k"], da["v"], da["o"], da["lora_q"], da["lora_k"], da["lora_v"],
                                 da["lora_o"], ac.lora_scale, ac.k, ac.n_q_heads, ac.n_kv_heads, ac.head_dim,
-                                ac.n_tok, C, ratio, device, dense=dense)
+                                ac.n_tok, C, ratio, device, dense=dense, dp=dp)
     ffn = blocks.FFNBlock(df["gate"], df["up"], df["down"], df["lora_gate"], df["lora_up"], df["lora_down"],
-                          fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense)
+                          fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense, dp=dp)
     if seed_x != seed_w:  # per-rank batches
         dx = inputs.make_attn_inputs(ac, seed_x, device=device)
         for key in ("x", "x_o", "dq", "dk", "dv", "dy"):
@@ -200,6 +201,25 @@ def capture_graph(fn, warm=True):
         fn()
     torch.cuda.synchronize()
     return g
+
+
+def capture_or_eager(fn, world):
+    """A replay callable for one step: its CUDA graph, or with N > 1 (NCCL collectives inside
+    the step), the eager step when the collectives cannot be captured. Returns (callable,
+    captured)."""
+    if world == 1:
+        return capture_graph(fn, warm=False).replay, True
+    try:
+        g = capture_graph(fn, warm=False)
+        _GRAPHS.append(g)  # released before the process group is destroyed
+        return g.replay, True
+    except Exception as e:  # noqa: BLE001 - any capture failure falls back to the eager step
+        print(f"rank step not captured ({type(e).__name__}: {e}); timing the eager step", file=sys.stderr)
+        torch.cuda.synchronize()
+        return fn, False
+
+
+_GRAPHS = []
 
 
 def time_steps(fn, K, W, world, device):
@@ -331,12 +351,14 @@ def e2e_measure(attn, ffn, step_in, K, W, world, device):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(g.numel() * g.element_size() for g in grads)
 
-    graph = capture_graph(lambda: run_step(attn, ffn, dev_in))
+    for _ in range(2):
+        run_step(attn, ffn, dev_in)
+    replay, _ = capture_or_eager(lambda: run_step(attn, ffn, dev_in), world)
 
     def step():
         for k in host:
             dev_in[k].copy_(host[k], non_blocking=True)
-        graph.replay()
+        replay()
         for h, g in zip(host_out, grads):
             h.copy_(g, non_blocking=True)
 
@@ -382,8 +404,12 @@ def main():
     torch.cuda.set_device(local)
     device = f"cuda:{local}"
     from contextual_sparsity_lora_b200 import binding as B
+    from contextual_sparsity_lora_b200 import blocks
     B.lib()
-    attn, ffn, step_in, C, (ac, fc), (da, df, perm) = make_layer(args.ratio, 0, 1000 + rank, device)
+    # N > 1: every rank takes its own 4096-token share of the global batch; the criterion
+    # statistics and the LoRA gradients are summed over the ranks (NCCL all-reduce)
+    dp = blocks.DataParallel() if world > 1 else None
+    attn, ffn, step_in, C, (ac, fc), (da, df, perm) = make_layer(args.ratio, 0, 1000 + rank, device, dp=dp)
     T = ac.n_tok
     B.sl_profile_enable(False)
     for _ in range(max(args.warmup, 3)):   # eager warm-up: sizes every workspace
@@ -391,25 +417,31 @@ def main():
     torch.cuda.synchronize()
     B.sl_profile_read()
     if args.stages_only:
-        print(json.dumps({"stages": stage_times(attn, ffn, step_in, 50, device,
-                                                float(load_peaks()[0].get("hbm_gbs", 6650.0)), None)}))
+        if rank == 0:
+            attn.dp = ffn.dp = None  # rank-local stages only: no collective inside the stage graphs
+            print(json.dumps({"stages": stage_times(attn, ffn, step_in, 50, device,
+                                                    float(load_peaks()[0].get("hbm_gbs", 6650.0)), None)}))
+        barrier(world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
     # The step is captured once into a CUDA graph and replayed; every replay runs every
     # kernel. The headline graph carries no event nodes. A second capture of the same step,
     # with the library's launch counting and an event pair around each GEMM-engine launch,
     # is replayed over its own K timed steps for the roofline's kernel durations.
-    graph = capture_graph(lambda: run_step(attn, ffn, step_in), warm=False)
+    graph, use_graph = capture_or_eager(lambda: run_step(attn, ffn, step_in), world)
     # (the profiled copy runs each block's chains in order, so that no concurrent kernel
     # stretches a GEMM-engine launch's event-timed duration)
     attn.concurrent = ffn.concurrent = False
     B.sl_profile_enable(True)
-    prof_graph = capture_graph(lambda: run_step(attn, ffn, step_in), warm=False)
+    prof_graph, _ = capture_or_eager(lambda: run_step(attn, ffn, step_in), world) if use_graph else (graph, False)
     B.sl_profile_enable(False)
     attn.concurrent = ffn.concurrent = True
     with ClockSampler(local) as clk:
-        ms = time_steps(graph.replay, args.steps, args.warmup, world, device)
+        ms = time_steps(graph, args.steps, args.warmup, world, device)
     torch.cuda.synchronize()
-    prof_ms = time_steps(prof_graph.replay, args.steps, args.warmup, world, device)
+    prof_ms = time_steps(prof_graph, args.steps, args.warmup, world, device)
     torch.cuda.synchronize()
     # launches counted while the profiled copy was captured (the same kernels as the
     # headline graph); GEMM-engine durations of its last replay, per launch and in total
@@ -443,7 +475,9 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": 8 * world, "seq_len": ac.seq, "tokens_per_rank": T,
                    "context_tokens_per_rank": C, "keep_ratio": args.ratio, "lora_rank": ac.r,
-                   "estimator_rank": ac.k, "parallelism": f"replicas{world}",
+                   "estimator_rank": ac.k, "parallelism": f"dp{world}",
+                   "exchange": ("per block: fp64 all-reduce of the criterion statistics (one index set per "
+                                "global batch), fp32 all-reduce of the LoRA gradients") if world > 1 else "none",
                    "l2": "per-step working set ~1.4 GB > 126 MB L2; no flush"},
         "roofline": {"bound": "tensor", "kernel": "sl::gemm_pair_kernel (CTA-pair tcgen05 GEMM: sliced products)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -463,19 +497,23 @@ def main():
                      "profiled_step_ms": prof_ms / args.steps,
                      "algorithmic_tflop_per_step": pair_flops / 1e12},
         "gpu_launches": n_launch,
-        "gpu_launches_per_step": n_launch_step, "cuda_graph": True,
+        "gpu_launches_per_step": n_launch_step, "cuda_graph": use_graph,
         "effective_tflops": fl["total"] / (ms_step / 1e3) / 1e12,
         "clocks": clk.summary(),
     }
     if rank == 0:
+        saved = (attn.dp, ffn.dp)
+        attn.dp = ffn.dp = None  # rank-local stages only: no collective inside the stage graphs
         line["stages"] = stage_times(attn, ffn, step_in, 50, device, float(peaks.get("hbm_gbs", 6650.0)), ms_step)
+        attn.dp, ffn.dp = saved
+    barrier(world)
     # dense LoRA on the same kernels (keep ratio 1, no estimator): context, not the headline
     if not args.no_dense:
-        d_attn, d_ffn, _, _, _, _ = make_layer(1.0, 0, 1000 + rank, device, dense=True)
+        d_attn, d_ffn, _, _, _, _ = make_layer(1.0, 0, 1000 + rank, device, dense=True, dp=dp)
         for _ in range(3):
             run_step(d_attn, d_ffn, step_in)
-        d_graph = capture_graph(lambda: run_step(d_attn, d_ffn, step_in))
-        d_ms = time_steps(d_graph.replay, args.steps, max(args.warmup, 3), world, device)
+        d_graph, _ = capture_or_eager(lambda: run_step(d_attn, d_ffn, step_in), world)
+        d_ms = time_steps(d_graph, args.steps, max(args.warmup, 3), world, device)
         d_fl = algorithmic_flops(ac, fc, C, 1.0, dense=True)
         line["dense_lora"] = {"value": world * T / (d_ms / args.steps / 1e3), "unit": UNIT,
                               "ms_per_step": d_ms / args.steps,
@@ -493,6 +531,9 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
+        del graph, prof_graph
+        _GRAPHS.clear()
+        torch.cuda.synchronize()
         dist.destroy_process_group()
 
 

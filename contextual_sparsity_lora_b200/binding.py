@@ -28,7 +28,8 @@ SL_LORA_FWD, SL_LORA_BWD = 0, 1
 EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_init", "sl_read_device_flag",
             "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
-            "sl_svd_estimate_noalloc", "sl_profile_launches")
+            "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
+            "sl_svd_scores_from_partials")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -71,6 +72,13 @@ def lib():
         L.sl_svd_estimate.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p),
                                       POINTER(c_void_p), POINTER(c_int64), c_int32, c_int32, c_int32, c_int32, P, P,
                                       POINTER(SlWorkspaceC), P]
+        L.sl_svd_partials_count.restype = c_int64
+        L.sl_svd_partials_count.argtypes = [c_int32, c_int32, POINTER(c_int64), c_int32]
+        L.sl_svd_estimate_partials.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32,
+                                               POINTER(c_void_p), POINTER(c_void_p), POINTER(c_int64), c_int32,
+                                               c_int32, c_int32, c_int32, P, POINTER(SlWorkspaceC), P]
+        L.sl_svd_scores_from_partials.argtypes = [c_int32, c_int32, c_int32, POINTER(c_void_p), POINTER(c_int64),
+                                                  c_int32, c_int32, c_int32, c_int32, P, P, P, P]
         L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
         L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
                                       POINTER(SlChannelsC), P, P, c_int64, POINTER(c_void_p), POINTER(c_int64),
@@ -88,7 +96,7 @@ def lib():
         L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
         L.sl_permute_rows.argtypes = [P, c_int64, P, c_int64, c_int64, P, c_int64, P]
         for n in EXPORTED:
-            if n not in ("sl_status_string", "sl_version", "sl_keep_count"):
+            if n not in ("sl_status_string", "sl_version", "sl_keep_count", "sl_svd_partials_count"):
                 getattr(L, n).restype = c_int32
         _lib = L
     return _lib
@@ -197,6 +205,31 @@ def sl_svd_estimate_noalloc(crit, x, n_ctx, w_a, w_b, k, scores, scores_v=None, 
                                          int(n_kv_heads), int(head_dim), _ptr(scores), _ptr(scores_v),
                                          ctypes.byref(needed), _ptr(device_flag), _stream()))
     return int(needed.value)
+
+
+def sl_svd_partials_count(crit, w_b, k):
+    d_out = [t.shape[1] for t in w_b]
+    return int(lib().sl_svd_partials_count(crit, len(w_b), _i64s(d_out), int(k)))
+
+
+def sl_svd_estimate_partials(ws: Workspace, crit, x, n_ctx, w_a, w_b, k, partials, n_q_heads=0, n_kv_heads=0,
+                             head_dim=0):
+    """The rank-local criterion statistics (fp64 `partials`, sl_svd_partials_count elements)."""
+    dtype = SL_DT_F32 if x.dtype == torch.float32 else SL_DT_BF16
+    d_out = [t.shape[1] for t in w_b]
+    ws.call("sl_svd_estimate_partials", crit, dtype, _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w_a),
+            _ptrs(w_a), _ptrs(w_b), _i64s(d_out), int(k), int(n_q_heads), int(n_kv_heads), int(head_dim),
+            _ptr(partials))
+
+
+def sl_svd_scores_from_partials(crit, w_b, k, partials, scores, scores_v=None, n_q_heads=0, n_kv_heads=0,
+                                head_dim=0):
+    dtype = SL_DT_F32 if w_b[0].dtype == torch.float32 else SL_DT_BF16
+    d_out = [t.shape[1] for t in w_b]
+    _check("sl_svd_scores_from_partials",
+           lib().sl_svd_scores_from_partials(crit, dtype, len(w_b), _ptrs(w_b), _i64s(d_out), int(k), int(n_q_heads),
+                                             int(n_kv_heads), int(head_dim), _ptr(partials), _ptr(scores),
+                                             _ptr(scores_v), _stream()))
 
 
 def sl_select_channels(scores, n_keep, sigma, heads_per_group=0, head_dim=0, sigma_wide=None):

@@ -34,12 +34,52 @@ class _Side:
         torch.cuda.current_stream().wait_stream(self.stream)
 
 
+class DataParallel:
+    """Ranks that each hold part of one global batch ([WT] "Oracle Sparse Neuron Selection
+    Criteria": one index set per batch). The criterion statistics of each rank's context rows
+    (sl_svd_estimate_partials) are summed over the ranks before the scores and the top-n, so
+    every rank keeps the same channels; the LoRA gradients (sums over tokens) are summed over
+    the ranks after the backward. One fp64 all-reduce per block for the statistics (the FFN's
+    per-channel sums of squares, or the attention block's Gram matrix) and one fp32 all-reduce
+    per block for its gradients. world == 1 leaves every path as on one GPU."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+
+    @property
+    def active(self) -> bool:
+        return self.world > 1
+
+    def all_reduce(self, t):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.all_reduce(t, group=self.group)
+
+
+class _GradBuffer:
+    """One flat fp32 buffer holding a block's LoRA gradients, so that a single collective sums
+    them over ranks; views start on 64-element boundaries (16-byte alignment and more)."""
+
+    def __init__(self, shapes, device):
+        self.offsets, n = [], 0
+        for sh in shapes:
+            self.offsets.append(n)
+            cnt = 1
+            for d in sh:
+                cnt *= d
+            n += (cnt + 63) // 64 * 64
+        self.flat = torch.zeros(n, dtype=torch.float32, device=device)
+        self.views = [self.flat[o:o + sh[0] * sh[1]].view(*sh) for o, sh in zip(self.offsets, shapes)]
+
+
 class FFNBlock:
     """SwiGLU FFN: gate/up (output channels sliced), down (input channels sliced), one
     index set shared by all three; L2 criterion on the estimated SiLU(gate) * up."""
 
     def __init__(self, gate, up, down, lora_gate, lora_up, lora_down, lora_scale, k, n_tok, n_ctx, ratio,
-                 device="cuda", dense=False):
+                 device="cuda", dense=False, dp=None):
         bf = torch.bfloat16
         self.device = device
         self.D = gate.W.shape[1]
@@ -72,12 +112,13 @@ class FFNBlock:
         self.xa_d, self.xa_s_d = _empty((T, r), f32, device), _empty((T, r), bf, device)
         self.y = _empty((T, D), bf, device)
         self.dya_d, self.dya_s_d = _empty((T, r), f32, device), _empty((T, r), bf, device)
-        self.dA_d, self.dB_d = _empty((r, F), f32, device), _empty((D, r), f32, device)
         self.dg, self.du = _empty((T, F), bf, device), _empty((T, F), bf, device)
         self.dya_g, self.dya_s_g = _empty((T, r), f32, device), _empty((T, r), bf, device)
         self.dya_u, self.dya_s_u = _empty((T, r), f32, device), _empty((T, r), bf, device)
-        self.dA_g, self.dB_g = _empty((r, D), f32, device), _empty((F, r), f32, device)
-        self.dA_u, self.dB_u = _empty((r, D), f32, device), _empty((F, r), f32, device)
+        self.grads = _GradBuffer([(r, F), (D, r), (r, D), (F, r), (r, D), (F, r)], device)
+        self.dA_d, self.dB_d, self.dA_g, self.dB_g, self.dA_u, self.dB_u = self.grads.views
+        self.dp = dp if dp is not None and dp.active else None
+        self.est_part = _empty((F,), torch.float64, device) if self.dp else None
         self.dx = _empty((T, D), bf, device)
         # kept rows of the sliced weights, rebuilt once per step and shared by the forward
         # and backward calls (the weights themselves when nothing is dropped)
@@ -98,6 +139,13 @@ class FFNBlock:
     def estimate(self, x):
         """a1 + a2: SwiGLU-L2 scores of the estimated gate/up outputs on x's context rows."""
         xe = x if self.est_dtype == torch.bfloat16 else self.x_est
+        if self.dp:  # statistics of this rank's context rows, summed over the ranks
+            B.sl_svd_estimate_partials(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx,
+                                       [self.WAg, self.WAu], [self.WBg, self.WBu], self.k, self.est_part)
+            self.dp.all_reduce(self.est_part)
+            B.sl_svd_scores_from_partials(B.SL_CRIT_SWIGLU_L2, [self.WBg, self.WBu], self.k, self.est_part,
+                                          self.scores)
+            return
         B.sl_svd_estimate(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx, [self.WAg, self.WAu],
                           [self.WBg, self.WBu], self.k, self.scores)
 
@@ -124,7 +172,9 @@ class FFNBlock:
         self.x_est = x_est
         C = self.n_ctx
         lay = B.SL_LAYOUT_NATURAL if self.dense else B.SL_LAYOUT_SIGMA
-        if not self.dense and C > 0:  # no context rows: nothing to score, every row is dense
+        # no context rows: nothing to score, every row is dense (data-parallel ranks still take
+        # part in the selection of the batch)
+        if not self.dense and (C > 0 or self.dp):
             if self.concurrent:  # x A^T of gate/up does not depend on the selection
                 with self.side.fork():
                     B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
@@ -168,7 +218,10 @@ class FFNBlock:
 
     def step(self, x, dy, x_est=None):
         self.forward(x, x_est)
-        return self.backward(dy)
+        dx = self.backward(dy)
+        if self.dp:
+            self.dp.all_reduce(self.grads.flat)
+        return dx
 
 
 class AttnProjBlock:
@@ -177,7 +230,7 @@ class AttnProjBlock:
     part of the path: its output x_o and its gradients dq, dk, dv are inputs."""
 
     def __init__(self, q, k, v, o, lora_q, lora_k, lora_v, lora_o, lora_scale, est_k, n_q_heads, n_kv_heads,
-                 head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False):
+                 head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False, dp=None):
         bf, f32 = torch.bfloat16, torch.float32
         dev = lambda t: t.to(device=device, dtype=bf).contiguous()
         self.device = device
@@ -214,8 +267,12 @@ class AttnProjBlock:
         self.dya = {n: (_empty((T, r), f32, device), _empty((T, r), bf, device)) for n in "qkvo"}
         d_ins = {"q": D, "k": D, "v": D, "o": self.Dq}
         d_outs = {"q": self.Dq, "k": self.Dkv, "v": self.Dkv, "o": D}
-        self.dA = {n: _empty((r, d_ins[n]), f32, device) for n in "qkvo"}
-        self.dB = {n: _empty((d_outs[n], r), f32, device) for n in "qkvo"}
+        self.grads = _GradBuffer([(r, d_ins[n]) for n in "qkvo"] + [(d_outs[n], r) for n in "qkvo"], device)
+        self.dA = dict(zip("qkvo", self.grads.views[:4]))
+        self.dB = dict(zip("qkvo", self.grads.views[4:]))
+        self.dp = dp if dp is not None and dp.active else None
+        self.est_part = _empty((B.sl_svd_partials_count(B.SL_CRIT_QK, self.WB, self.k),), torch.float64,
+                               device) if self.dp else None
         self.dx_o = _empty((T, self.Dq), bf, device)
         self.dx = _empty((T, D), bf, device)
         s = self.scale
@@ -243,6 +300,13 @@ class AttnProjBlock:
     def estimate(self, x):
         """a1 + a2: QK scores over KV units and V scores from one pass over x's context rows."""
         C = self.n_ctx
+        if self.dp:  # Gram matrix of this rank's Z, summed over the ranks
+            B.sl_svd_estimate_partials(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.est_part,
+                                       n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+            self.dp.all_reduce(self.est_part)
+            B.sl_svd_scores_from_partials(B.SL_CRIT_QK, self.WB, self.k, self.est_part, self.s_qk, scores_v=self.s_v,
+                                          n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+            return
         B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
 
@@ -284,7 +348,7 @@ class AttnProjBlock:
         C = self.n_ctx
         self.x, self.x_o = x, x_o
         lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
-        sel = not self.dense and C > 0
+        sel = not self.dense and (C > 0 or self.dp is not None)
 
         def lora_fwd(ws):  # x A^T for q, k, v and x_o A^T for o: independent of the selection
             B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
@@ -338,4 +402,7 @@ class AttnProjBlock:
 
     def step(self, x, x_o, dy, dq, dk, dv):
         self.forward(x, x_o)
-        return self.backward(dy, dq, dk, dv)
+        dx = self.backward(dy, dq, dk, dv)
+        if self.dp:
+            self.dp.all_reduce(self.grads.flat)
+        return dx

@@ -191,19 +191,19 @@ sl_status sl_read_device_flag(const sl_workspace* ws, int32_t* code, sl_stream s
   return *code ? SL_ERR_DEVICE_FLAG : SL_OK;
 }
 
+}  // extern "C"
+
 // ------------------------------------------------------------------ a1 + a2
-sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx,
-                          int32_t n_proj, const void* const* w_a, const void* const* w_b, const int64_t* d_out,
-                          int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float* scores,
-                          float* scores_v, sl_workspace* ws, sl_stream stream) {
-  if (!x || !w_a || !w_b || !d_out || !scores) return SL_ERR_INVALID_ARG;
-  if (dtype != SL_DT_BF16 && dtype != SL_DT_F32) return SL_ERR_INVALID_ARG;
-  if (n_ctx <= 0 || d_in <= 0 || ldx < d_in || k <= 0 || k > 16 || n_proj < 1 || n_proj * k > 64)
-    return SL_ERR_SHAPE;
-  if (d_in % 8 || ldx % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+namespace {
+
+// Arguments of the criterion shared by the estimate and the scores-from-partials entries:
+// the unit count, or a status.
+sl_status criterion_units(sl_criterion crit, int32_t n_proj, const void* const* w_b, const int64_t* d_out, int32_t k,
+                          int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, bool need_v, int64_t* units) {
+  if (!w_b || !d_out) return SL_ERR_INVALID_ARG;
+  if (k <= 0 || k > 16 || n_proj < 1 || n_proj * k > 64) return SL_ERR_SHAPE;
   for (int j = 0; j < n_proj; ++j)
-    if (!w_a[j] || !w_b[j] || d_out[j] <= 0) return SL_ERR_INVALID_ARG;
-  const int fp32 = dtype == SL_DT_F32;
+    if (!w_b[j] || d_out[j] <= 0) return SL_ERR_INVALID_ARG;
   int64_t n_units = 0;
   switch (crit) {
     case SL_CRIT_L2:
@@ -220,12 +220,38 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
       if (n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || n_q_heads % n_kv_heads) return SL_ERR_SHAPE;
       if (d_out[0] != (int64_t)n_q_heads * head_dim || d_out[1] != (int64_t)n_kv_heads * head_dim)
         return SL_ERR_SHAPE;
-      if (n_proj == 3 && !scores_v) return SL_ERR_INVALID_ARG;
+      if (n_proj == 3 && need_v) return SL_ERR_INVALID_ARG;
       n_units = (int64_t)n_kv_heads * head_dim;
       break;
     default:
       return SL_ERR_INVALID_ARG;
   }
+  *units = n_units;
+  return SL_OK;
+}
+
+// Rank-local statistics of the criterion: per-channel sums of squares (SwiGLU) or the Gram
+// matrix of Z (linear criteria).
+int64_t partial_count(sl_criterion crit, int32_t n_proj, const int64_t* d_out, int32_t k) {
+  return crit == SL_CRIT_SWIGLU_L2 ? d_out[0] : (int64_t)n_proj * k * n_proj * k;
+}
+
+// Estimator body: scores (and scores_v) when partials is null, else the rank-local statistics.
+sl_status svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx,
+                       int32_t n_proj, const void* const* w_a, const void* const* w_b, const int64_t* d_out,
+                       int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float* scores,
+                       float* scores_v, double* partials, sl_workspace* ws, sl_stream stream) {
+  if (!x || !w_a || (!scores && !partials)) return SL_ERR_INVALID_ARG;
+  if (dtype != SL_DT_BF16 && dtype != SL_DT_F32) return SL_ERR_INVALID_ARG;
+  int64_t n_units = 0;
+  if (sl_status st = criterion_units(crit, n_proj, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim,
+                                     !partials && !scores_v, &n_units))
+    return st;
+  if (n_ctx <= 0 || d_in <= 0 || ldx < d_in) return SL_ERR_SHAPE;
+  if (d_in % 8 || ldx % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+  for (int j = 0; j < n_proj; ++j)
+    if (!w_a[j]) return SL_ERR_INVALID_ARG;
+  const int fp32 = dtype == SL_DT_F32;
   const int mk = n_proj * k;
   // bf16 inputs: stage 1 on the tensor cores (exact bf16 products, fp32 accumulation,
   // K-range partials summed in a fixed order); fp32 inputs: CUDA-core fp32 FMA kernel.
@@ -268,14 +294,15 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
     if (rc) return from_kernel(rc);
   }
   if (swiglu_tc) {
-    rc = est_swiglu_tc(zs, n_ctx, k, w_b[0], w_b[1], n_units, scores, err_word(ws), s);
+    rc = est_swiglu_tc(zs, n_ctx, k, w_b[0], w_b[1], n_units, scores, partials, err_word(ws), s);
     return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
   }
   if (crit == SL_CRIT_SWIGLU_L2) {
-    rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, err_word(ws), s);
+    rc = est_swiglu_scores(zp, 1, n_ctx, k, w_b[0], w_b[1], fp32, n_units, scores, partials, err_word(ws), s);
     return from_kernel(rc);
   }
   if (!tc && (rc = est_gram(zp, 1, n_ctx, mk, gp, n_chunks, s))) return from_kernel(rc);
+  if (partials) return from_kernel(gram_sum(gp, n_chunks, mk, partials, s));
   if (crit == SL_CRIT_L2)
     rc = est_scores(gp, n_chunks, mk, k, fp32, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0, n_units, scores,
                     s);
@@ -284,6 +311,64 @@ sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int6
                     n_proj == 3 ? w_b[2] : nullptr, 2, n_proj == 3 ? d_out[2] : 0, n_proj == 3 ? scores_v : nullptr,
                     s);
   return from_kernel(rc);
+}
+
+}  // namespace
+
+extern "C" {
+
+sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx,
+                          int32_t n_proj, const void* const* w_a, const void* const* w_b, const int64_t* d_out,
+                          int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float* scores,
+                          float* scores_v, sl_workspace* ws, sl_stream stream) {
+  if (!scores) return SL_ERR_INVALID_ARG;
+  return svd_estimate(crit, dtype, x, n_ctx, d_in, ldx, n_proj, w_a, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim,
+                      scores, scores_v, nullptr, ws, stream);
+}
+
+int64_t sl_svd_partials_count(sl_criterion crit, int32_t n_proj, const int64_t* d_out, int32_t k) {
+  if (!d_out || n_proj < 1 || k < 1) return 0;
+  return partial_count(crit, n_proj, d_out, k);
+}
+
+sl_status sl_svd_estimate_partials(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx, int64_t d_in,
+                                   int64_t ldx, int32_t n_proj, const void* const* w_a, const void* const* w_b,
+                                   const int64_t* d_out, int32_t k, int32_t n_q_heads, int32_t n_kv_heads,
+                                   int32_t head_dim, double* partials, sl_workspace* ws, sl_stream stream) {
+  if (!partials || !d_out) return SL_ERR_INVALID_ARG;
+  if (n_ctx == 0) {  // no context rows on this rank: its statistics are zero
+    int64_t units = 0;
+    if (sl_status st = criterion_units(crit, n_proj, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim, false, &units))
+      return st;
+    return cudaMemsetAsync(partials, 0, sizeof(double) * partial_count(crit, n_proj, d_out, k), cs(stream)) ==
+                   cudaSuccess
+               ? SL_OK
+               : SL_ERR_CUDA;
+  }
+  return svd_estimate(crit, dtype, x, n_ctx, d_in, ldx, n_proj, w_a, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim,
+                      nullptr, nullptr, partials, ws, stream);
+}
+
+sl_status sl_svd_scores_from_partials(sl_criterion crit, sl_dtype dtype, int32_t n_proj, const void* const* w_b,
+                                      const int64_t* d_out, int32_t k, int32_t n_q_heads, int32_t n_kv_heads,
+                                      int32_t head_dim, const double* partials, float* scores, float* scores_v,
+                                      sl_stream stream) {
+  if (!partials || !scores) return SL_ERR_INVALID_ARG;
+  if (dtype != SL_DT_BF16 && dtype != SL_DT_F32) return SL_ERR_INVALID_ARG;
+  int64_t n_units = 0;
+  if (sl_status st = criterion_units(crit, n_proj, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim, !scores_v,
+                                     &n_units))
+    return st;
+  cudaStream_t s = cs(stream);
+  const int fp32 = dtype == SL_DT_F32;
+  const int mk = n_proj * k;
+  if (crit == SL_CRIT_SWIGLU_L2) return from_kernel(sqrt_scores(partials, n_units, scores, s));
+  if (crit == SL_CRIT_L2)
+    return from_kernel(est_scores(partials, 1, mk, k, fp32, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0,
+                                  n_units, scores, s));
+  return from_kernel(est_scores(partials, 1, mk, k, fp32, w_b[0], w_b[1], 0, 1, n_q_heads, n_kv_heads, head_dim,
+                                scores, n_proj == 3 ? w_b[2] : nullptr, 2, n_proj == 3 ? d_out[2] : 0,
+                                n_proj == 3 ? scores_v : nullptr, s));
 }
 
 // ------------------------------------------------------------------ a3

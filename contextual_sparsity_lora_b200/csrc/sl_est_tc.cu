@@ -504,6 +504,7 @@ struct SwigluParams {
   const __nv_bfloat16* wb_u;  // W_B of up [k, F]
   int32_t k, n_k16, n_ctx, F, n_blocks, pad_;
   float* scores;
+  double* sumsq;              // when not null: the sums of squares instead of the scores
   int* err;
 };
 
@@ -657,12 +658,35 @@ __global__ void __launch_bounds__(kSwThreads, 1) est_swiglu_tc_kernel(const __gr
     sw_epi_bar();
     if (hc == 0) {
       const int64_t ch = ch0 + row;
-      if (ch < p.F) p.scores[ch] = (float)sqrt(part[row] + part[128 + row]);
+      if (ch < p.F) {
+        const double tot = part[row] + part[128 + row];
+        if (p.sumsq) p.sumsq[ch] = tot;
+        else p.scores[ch] = (float)sqrt(tot);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// out[e] = sum of n_parts matrices in part order (the rank-local Gram matrix).
+__global__ void __launch_bounds__(256) gram_sum_kernel(const double* __restrict__ parts, int n_parts, int ne,
+                                                       double* __restrict__ out) {
+  pdl_wait();
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < ne; e += gridDim.x * blockDim.x) {
+    double s = 0.0;
+    for (int c = 0; c < n_parts; ++c) s += parts[(int64_t)c * ne + e];
+    out[e] = s;
+  }
+}
+
+// scores[i] = sqrt(sumsq[i]) (the SwiGLU criterion from summed squares).
+__global__ void __launch_bounds__(256) sqrt_scores_kernel(const double* __restrict__ sumsq, int64_t n,
+                                                          float* __restrict__ scores) {
+  pdl_wait();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    scores[i] = (float)sqrt(sumsq[i] > 0.0 ? sumsq[i] : 0.0);
 }
 
 }  // namespace
@@ -744,7 +768,7 @@ int est_z_tc(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj
 }
 
 int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, const void* wb_u, int64_t F,
-                  float* scores, int* err, cudaStream_t s) {
+                  float* scores, double* sumsq, int* err, cudaStream_t s) {
   if (k < 1 || 3 * k > 64 || F <= 0 || n_ctx <= 0 || n_ctx > 2147483647LL || F > 2147483647LL) return 1;
   SwigluParams P;
   memset(&P, 0, sizeof(P));
@@ -757,6 +781,7 @@ int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, co
   P.F = (int32_t)F;
   P.n_blocks = (int32_t)((n_ctx + 127) / 128);
   P.scores = scores;
+  P.sumsq = sumsq;
   P.err = err;
   static bool attr = false;
   if (!attr) {
@@ -764,6 +789,24 @@ int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, co
     attr = true;
   }
   launch_kernel(est_swiglu_tc_kernel, (unsigned)((F + 127) / 128), kSwThreads, kSwSmem, s, P);
+  if (launch_failed("sl_estimator")) return 5;
+  note_launch();
+  return 0;
+}
+
+int gram_sum(const double* parts, int n_parts, int mk, double* out, cudaStream_t s) {
+  if (n_parts < 1 || mk < 1 || mk > 64) return 1;
+  const int ne = mk * mk;
+  launch_kernel(gram_sum_kernel, (unsigned)((ne + 255) / 256), 256, 0, s, parts, n_parts, ne, out);
+  if (launch_failed("sl_estimator")) return 5;
+  note_launch();
+  return 0;
+}
+
+int sqrt_scores(const double* sumsq, int64_t n, float* scores, cudaStream_t s) {
+  if (n < 1) return 1;
+  const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 1184);
+  launch_kernel(sqrt_scores_kernel, grid, 256, 0, s, sumsq, n, scores);
   if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;

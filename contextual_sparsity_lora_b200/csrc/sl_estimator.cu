@@ -164,7 +164,7 @@ constexpr int kE2Buf = 4096;     // floats per staging buffer (16 KB): 4096 / (2
 template <int K>
 __global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
     est_swiglu_kernel(const float* __restrict__ z, int64_t n_ctx, const void* wb_g, const void* wb_u, int wb_fp32,
-                      int64_t n_ch, float* __restrict__ scores, int* err) {
+                      int64_t n_ch, float* __restrict__ scores, double* __restrict__ sumsq, int* err) {
   constexpr int kRow = 2 * K;
   constexpr int kChunk = kE2Buf / kRow;
   __shared__ __align__(128) float zs[2][kE2Buf];
@@ -268,7 +268,10 @@ __global__ void __cluster_dims__(1, kE2Split, 1) __launch_bounds__(kE2Threads)
     double s = 0.0;
     for (int rnk = 0; rnk < kE2Split; ++rnk) s += cluster.map_shared_rank(cta_sum, rnk)[threadIdx.x];
     const int64_t ch = (int64_t)blockIdx.x * 64 + threadIdx.x;
-    if (ch < n_ch) scores[ch] = (float)sqrt(s);
+    if (ch < n_ch) {
+      if (sumsq) sumsq[ch] = s;
+      else scores[ch] = (float)sqrt(s);
+    }
   }
   cluster.sync();  // peers keep their shared memory alive until rank 0 has read it
 }
@@ -371,13 +374,13 @@ int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t l
 }
 
 int est_swiglu_scores(const float* z, int /*n_split*/, int64_t n_ctx, int k, const void* wb_gate, const void* wb_up,
-                      int wb_fp32, int64_t n_ch, float* scores, int* err, cudaStream_t s) {
+                      int wb_fp32, int64_t n_ch, float* scores, double* sumsq, int* err, cudaStream_t s) {
   if (reinterpret_cast<uintptr_t>(z) & 15) return 1;  // bulk copies need 16-byte alignment
   const dim3 grid((unsigned)((n_ch + 63) / 64), kE2Split);
   switch (k) {
-    case 8: launch_kernel(est_swiglu_kernel<8>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
-    case 16: launch_kernel(est_swiglu_kernel<16>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
-    case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, err); break;
+    case 8: launch_kernel(est_swiglu_kernel<8>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, sumsq, err); break;
+    case 16: launch_kernel(est_swiglu_kernel<16>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, sumsq, err); break;
+    case 4: launch_kernel(est_swiglu_kernel<4>, grid, kE2Threads, 0, s, z, n_ctx, wb_gate, wb_up, wb_fp32, n_ch, scores, sumsq, err); break;
     default: return 1;
   }
   if (launch_failed("sl_estimator")) return 5;

@@ -92,7 +92,8 @@ int choose_ksplit(int64_t M, int64_t kblocks, int target_tiles = 0);
 int est_stage1(const void* x, int x_fp32, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj,
                const void* const* wa, int wa_fp32, int k, float* zpart, int n_split, cudaStream_t s);
 int est_swiglu_scores(const float* zpart, int n_split, int64_t n_ctx, int k, const void* wb_gate,
-                      const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, int* err, cudaStream_t s);
+                      const void* wb_up, int wb_fp32, int64_t n_ch, float* scores, double* sumsq, int* err,
+                      cudaStream_t s);
 int est_gram(const float* zpart, int n_split, int64_t n_ctx, int mk, double* gram_part, int n_chunks,
              cudaStream_t s);
 int est1_splits(int64_t d_in);
@@ -110,7 +111,10 @@ int est_z_tc(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj
 // SwiGLU criterion from zsplit ([n_ctx][128] bf16: Z of gate and of up as three bf16 terms,
 // written by est_z_tc) and the bf16 W_B of gate and up [k, F]; scores[F].
 int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, const void* wb_u, int64_t F,
-                  float* scores, int* err, cudaStream_t s);
+                  float* scores, double* sumsq, int* err, cudaStream_t s);
+// out[mk][mk] = sum of n_parts Gram matrices in order; scores = sqrt(sumsq).
+int gram_sum(const double* parts, int n_parts, int mk, double* out, cudaStream_t s);
+int sqrt_scores(const double* sumsq, int64_t n, float* scores, cudaStream_t s);
 // QK units and/or L2 channels from the Gram partials (sum over n_parts in order), one launch.
 int est_scores(const double* gram_part, int n_parts, int mk, int k, int wb_fp32, const void* wb_q, const void* wb_k,
                int blk_q, int blk_k, int n_q_heads, int n_kv_heads, int head_dim, float* scores_qk, const void* wb_l2,

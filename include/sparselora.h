@@ -179,6 +179,33 @@ SL_API sl_status sl_svd_estimate_noalloc(sl_criterion crit, sl_dtype dtype, cons
                                          float* scores_v, int64_t* scratch_needed, int32_t* device_flag,
                                          sl_stream stream);
 
+/* a1 + a2 across data-parallel ranks ([WT] "Oracle Sparse Neuron Selection Criteria": the
+ * criterion is a norm over the context tokens of the batch, one index set per batch). A rank
+ * holding part of the batch's context rows computes its rank-local statistics, the caller sums
+ * them over the ranks (an fp64 all-reduce), and every rank turns the sum into the same scores:
+ *   SL_CRIT_SWIGLU_L2: partials[d_out[0]] = sum over the rank's context rows of
+ *                      (SiLU(G_hat) * U_hat)^2 per channel (fp64);
+ *   SL_CRIT_L2, SL_CRIT_QK: partials[(n_proj k)^2] = the Gram matrix Z^T Z of the rank's
+ *                      Z = X_ctx [W_A^(1) ...] (fp64, row-major), from which every linear
+ *                      criterion follows exactly: sum_t (z_t . b)^2 = b^T (Z^T Z) b.
+ * sl_svd_partials_count gives the element count (0 for invalid arguments). Arguments of
+ * sl_svd_estimate_partials are those of sl_svd_estimate, with n_ctx = 0 allowed (zero
+ * statistics); sl_svd_scores_from_partials takes the summed statistics and writes scores (and
+ * scores_v for SL_CRIT_QK with n_proj = 3) exactly as sl_svd_estimate would for the union of the
+ * ranks' context rows (up to the summation order). Sums over tokens run in a fixed order on a
+ * rank; the sum over ranks is the caller's. */
+SL_API int64_t sl_svd_partials_count(sl_criterion crit, int32_t n_proj, const int64_t* d_out, int32_t k);
+SL_API sl_status sl_svd_estimate_partials(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx,
+                                          int64_t d_in, int64_t ldx, int32_t n_proj, const void* const* w_a,
+                                          const void* const* w_b, const int64_t* d_out, int32_t k,
+                                          int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          double* partials, sl_workspace* ws, sl_stream stream);
+SL_API sl_status sl_svd_scores_from_partials(sl_criterion crit, sl_dtype dtype, int32_t n_proj,
+                                             const void* const* w_b, const int64_t* d_out, int32_t k,
+                                             int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                             const double* partials, float* scores, float* scores_v,
+                                             sl_stream stream);
+
 /* a3: top-n selection ([WT] Algorithm 1; [PN] top-n). Keeps exactly n_keep of the n
  * scores: larger score first, ties to the lower index, NaN below every number.
  * Writes sigma[n] (kept ascending, then dropped ascending). When heads_per_group > 0

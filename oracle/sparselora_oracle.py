@@ -135,8 +135,27 @@ def score_qk(Q, K, n_q_heads, n_kv_heads, head_dim):
     attention the unit is a KV channel (g, d) and the query side sums the norms of
     the group's query heads at the same head dimension (reading R5).
     Returns scores over n_kv_heads * head_dim units, unit index g * head_dim + d."""
-    q = score_l2(Q).reshape(n_q_heads, head_dim)
-    k = score_l2(K).reshape(n_kv_heads, head_dim)
+    return qk_from_sumsq(sumsq(Q), sumsq(K), n_q_heads, n_kv_heads, head_dim)
+
+
+# ---------------------------------------------------------------------------
+# Sufficient statistics for ranks that each hold part of the batch's context rows.
+# Every criterion above is built from per-channel sums of squares over the context
+# rows, and a sum over all rows is the sum of the sums over disjoint parts of them:
+# the ranks add their statistics and every rank then derives the scores of the
+# whole batch (one index set per batch, reading R3).
+# ---------------------------------------------------------------------------
+
+def sumsq(Y):
+    """Per-channel sum of squares over rows: sum_t Y[t, i]^2 (score_l2 before the root)."""
+    Y = f64(Y)
+    return np.sum(Y * Y, axis=0)
+
+
+def qk_from_sumsq(q2, k2, n_q_heads, n_kv_heads, head_dim):
+    """The QK scores (reading R5) from the per-channel sums of squares of Q_hat and K_hat."""
+    q = np.sqrt(f64(q2)).reshape(n_q_heads, head_dim)
+    k = np.sqrt(f64(k2)).reshape(n_kv_heads, head_dim)
     group = n_q_heads // n_kv_heads
     q_group = q.reshape(n_kv_heads, group, head_dim).sum(axis=1)
     return (q_group * k).reshape(-1)

@@ -50,3 +50,83 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
     bench.barrier(1)
+
+
+def _dp_rank_main(rank, world, port, out):
+    """Two ranks, each with half of the batch's sequences: the rank-local statistics of the
+    criteria (oracle), summed with the same collective the library's blocks use (an fp64
+    all-reduce), give every rank the scores and the index sets of the whole batch."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from contextual_sparsity_lora_b200 import inputs
+
+    dist.init_process_group("gloo")
+    gen = inputs.generator(3)
+    D, F, hq, hkv, hd, k = 64, 96, 4, 2, 8, 8
+    x = inputs.activations_student_t(8 * 16, D, 4, 0.03, 30.0, gen)  # 8 sequences of 16 tokens
+    ctx = np.tile(np.arange(16) < 12, 8)
+    fac = {n: oracle.svd_factors(inputs.spectral_weight(o, D, 0.5, k, gen, "cpu", torch.float64,
+                                                        torch.float32).W, k)[:2]
+           for n, o in (("gate", F), ("up", F), ("q", hq * hd), ("k", hkv * hd), ("v", hkv * hd))}
+    X = oracle.f64(x)
+
+    def stats(rows):
+        Xc = X[rows & ctx]
+        G, U = oracle.estimate(Xc, *fac["gate"]), oracle.estimate(Xc, *fac["up"])
+        Q, K, V = (oracle.estimate(Xc, *fac[n]) for n in "qkv")
+        return np.concatenate([oracle.sumsq(oracle.silu(G) * U), oracle.sumsq(Q), oracle.sumsq(K),
+                               oracle.sumsq(V)])
+
+    mine = np.arange(8 * 16) // 64 == rank  # rank r holds sequences 4r .. 4r + 3
+    t = torch.tensor(stats(mine), dtype=torch.float64)
+    dist.all_reduce(t)  # sum over the ranks
+    s = t.numpy()
+    f2, q2, k2, v2 = np.split(s, np.cumsum([F, hq * hd, hkv * hd]))
+    s_ffn = np.sqrt(f2)
+    s_qk = oracle.qk_from_sumsq(q2, k2, hq, hkv, hd)
+    s_v = np.sqrt(v2)
+    sel = [oracle.select_top(v, oracle.keep_count(0.5, v.shape[0])) for v in (s_ffn, s_qk, s_v)]
+    out[rank] = (s_ffn, s_qk, s_v, sel)
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_data_parallel_ranks_select_the_batch_index_sets():
+    import numpy as np
+
+    import oracle
+    from contextual_sparsity_lora_b200 import inputs
+    import torch
+
+    ctx_ = mp.get_context("spawn")
+    with ctx_.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_dp_rank_main, args=(2, _free_port(), out), nprocs=2, start_method="spawn", join=True)
+        res = dict(out)
+    # both ranks agree exactly
+    for a, b in zip(res[0][:3], res[1][:3]):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(res[0][3], res[1][3]):
+        np.testing.assert_array_equal(a, b)
+    # and equal the single-process criterion over the whole batch
+    gen = inputs.generator(3)
+    D, F, hq, hkv, hd, k = 64, 96, 4, 2, 8, 8
+    x = inputs.activations_student_t(8 * 16, D, 4, 0.03, 30.0, gen)
+    ctx = np.tile(np.arange(16) < 12, 8)
+    fac = {n: oracle.svd_factors(inputs.spectral_weight(o, D, 0.5, k, gen, "cpu", torch.float64,
+                                                        torch.float32).W, k)[:2]
+           for n, o in (("gate", F), ("up", F), ("q", hq * hd), ("k", hkv * hd), ("v", hkv * hd))}
+    s_ffn, _ = oracle.ffn_select(x, ctx, fac["gate"], fac["up"], 0.5)
+    sel = oracle.attn_select(x, ctx, fac["q"], fac["k"], fac["v"], hq, hkv, hd, 0.5)
+    np.testing.assert_allclose(res[0][0], s_ffn, rtol=1e-12)
+    np.testing.assert_allclose(res[0][1], sel["s_qk"], rtol=1e-12)
+    np.testing.assert_allclose(res[0][2], sel["s_v"], rtol=1e-12)
+    np.testing.assert_array_equal(res[0][3][0], oracle.select_top(s_ffn, oracle.keep_count(0.5, F)))
+    np.testing.assert_array_equal(res[0][3][1], sel["units_qk"])
+    np.testing.assert_array_equal(res[0][3][2], sel["units_v"])

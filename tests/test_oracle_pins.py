@@ -399,3 +399,15 @@ def test_attn_select_mha_reduces_to_plain_qk():
     np.testing.assert_allclose(out["s_qk"], s, rtol=1e-12)
     np.testing.assert_array_equal(out["idx_q"], out["idx_k"])
     np.testing.assert_array_equal(out["idx_o"], out["idx_v"])
+
+
+def test_sum_of_squares_statistics_add_over_row_parts():
+    """The per-channel statistics of data-parallel ranks: the sum over all rows is the sum of
+    the sums over any split of the rows, and the root is the L2 criterion."""
+    rng = np.random.default_rng(5)
+    Y = rng.standard_normal((37, 11))
+    np.testing.assert_allclose(oracle.sumsq(Y), oracle.score_l2(Y) ** 2, rtol=1e-13)
+    for cut in (0, 1, 18, 37):
+        np.testing.assert_allclose(oracle.sumsq(Y[:cut]) + oracle.sumsq(Y[cut:]), oracle.sumsq(Y), rtol=1e-13)
+    # columns of constant value c over n rows: n c^2
+    np.testing.assert_allclose(oracle.sumsq(np.full((6, 3), 2.5)), np.full(3, 6 * 2.5 ** 2), rtol=0)
