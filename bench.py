@@ -203,6 +203,14 @@ def capture_graph(fn, warm=True):
     return g
 
 
+# DRAM bytes (read + write) of gemm_pair_kernel per launch, the mean over the 8 CTA-pair
+# launches of one step of this workload, from the ncu capture whose command and per-launch
+# figures are in profiles/gemm_pair_kernel_traffic_llama3-8b-layer-step.md (3013.8 MB per
+# step). Valid for the kernel as captured; to be set to None when the kernel changes.
+PAIR_DRAM_BYTES_PER_LAUNCH = 3013.8e6 / 8
+PAIR_DRAM_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of the step's 8 launches"
+
+
 def capture_or_eager(fn, world):
     """A replay callable for one step: its CUDA graph, or with N > 1 (NCCL collectives inside
     the step), the eager step when the collectives cannot be captured. Returns (callable,
@@ -481,7 +489,8 @@ def main():
                    "l2": "per-step working set ~1.4 GB > 126 MB L2; no flush"},
         "roofline": {"bound": "tensor", "kernel": "sl::gemm_pair_kernel (CTA-pair tcgen05 GEMM: sliced products)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak) if achieved else None,
+                     "traffic": PAIR_DRAM_BYTES_PER_LAUNCH, "traffic_source": PAIR_DRAM_SOURCE,
                      "peak_source": f"{src} bf16_tflops_sustained",
                      "algorithmic_tflop_per_launch": pair_flops / 1e12 / max(pair_n, 1),
                      "launches_per_step": pair_n, "ms_per_launch": pair_ms / max(pair_n, 1),
