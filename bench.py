@@ -294,6 +294,21 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
                      "a1_frac_of_hbm": a1_bytes / (a1 * 1e3) / hbm_gbs if a1 else None,
                      "a2_criterion_us": est - a1 if a1 else None, "a3_select_us": sel, "compact_weights_us": comp}
         total += est + sel
+    # criterion ablation variants (not on the step's path): the Wanda-style FFN criterion
+    # (reads X_ctx and the gate and up weights once) and the head-level QK selection
+    C, D, F = ffn.n_ctx, ffn.D, ffn.F
+    ws = B.Workspace(device)
+    wanda_sc = torch.empty(F, device=device)
+    xf = s["ffn_x"]
+    w_us = graph_us(lambda: B.sl_wanda_scores(ws, xf[:C], C, [ffn.Wg, ffn.Wu], wanda_sc))
+    w_bytes = C * D * 2 + 2 * F * D * 2
+    sig_k = torch.empty_like(attn.sig_k)
+    sig_q = torch.empty_like(attn.sig_q)
+    h_us = graph_us(lambda: B.sl_select_heads(attn.s_qk, attn.hkv, attn.hd, attn.n_keep_heads, sig_k, attn.hpg,
+                                              sig_q))
+    out["variants"] = {"ffn_wanda_scores_us": w_us, "ffn_wanda_bytes": w_bytes,
+                       "ffn_wanda_GBs": w_bytes / (w_us * 1e3), "ffn_wanda_frac_of_hbm": w_bytes / (w_us * 1e3) / hbm_gbs,
+                       "qk_head_select_us": h_us}
     out["estimator_and_select_us"] = total
     if step_ms:
         out["estimator_and_select_pct_of_step"] = 100.0 * total / (step_ms * 1e3)

@@ -29,7 +29,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
-            "sl_svd_scores_from_partials")
+            "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -80,6 +80,9 @@ def lib():
         L.sl_svd_scores_from_partials.argtypes = [c_int32, c_int32, c_int32, POINTER(c_void_p), POINTER(c_int64),
                                                   c_int32, c_int32, c_int32, c_int32, P, P, P, P]
         L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
+        L.sl_select_heads.argtypes = [P, c_int32, c_int32, c_int32, c_int32, P, P, P]
+        L.sl_wanda_scores.argtypes = [P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p), c_int64, c_int64, P,
+                                      POINTER(SlWorkspaceC), P]
         L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
                                       POINTER(SlChannelsC), P, P, c_int64, POINTER(c_void_p), POINTER(c_int64),
                                       c_int32, POINTER(SlChannelsC), POINTER(c_void_p), POINTER(c_void_p),
@@ -236,6 +239,18 @@ def sl_select_channels(scores, n_keep, sigma, heads_per_group=0, head_dim=0, sig
     _check("sl_select_channels",
            lib().sl_select_channels(_ptr(scores), scores.numel(), int(n_keep), _ptr(sigma), int(heads_per_group),
                                     int(head_dim), _ptr(sigma_wide), _stream()))
+
+
+def sl_select_heads(scores, n_heads, head_dim, n_keep_heads, sigma, heads_per_group=0, sigma_wide=None):
+    _check("sl_select_heads",
+           lib().sl_select_heads(_ptr(scores), int(n_heads), int(head_dim), int(n_keep_heads), int(heads_per_group),
+                                 _ptr(sigma), _ptr(sigma_wide), _stream()))
+
+
+def sl_wanda_scores(ws: Workspace, x, n_ctx, w, scores):
+    """Wanda-style channel scores over the context rows x[:n_ctx] for the weights w (one index set)."""
+    ws.call("sl_wanda_scores", _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w), _ptrs(w), w[0].shape[0],
+            w[0].stride(0), _ptr(scores))
 
 
 def sl_lora_fwd_bwd(ws: Workspace, mode, lins, x, n_ctx, xa_s, xa=None, in_layout=SL_LAYOUT_NATURAL, in_ch=None,

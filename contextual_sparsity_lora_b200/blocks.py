@@ -78,8 +78,20 @@ class FFNBlock:
     """SwiGLU FFN: gate/up (output channels sliced), down (input channels sliced), one
     index set shared by all three; L2 criterion on the estimated SiLU(gate) * up."""
 
+    CRITERIA = ("svd", "wanda", "random")
+
     def __init__(self, gate, up, down, lora_gate, lora_up, lora_down, lora_scale, k, n_tok, n_ctx, ratio,
-                 device="cuda", dense=False, dp=None):
+                 device="cuda", dense=False, dp=None, criterion="svd", seed=0):
+        """criterion: "svd" (SwiGLU L2 of the SVD estimate, the method's criterion), or the
+        criterion ablation's alternatives "wanda" (Wanda-style channel scores of the frozen
+        gate/up weights) and "random" (uniform scores from a generator seeded with `seed`)."""
+        if criterion not in self.CRITERIA:
+            raise ValueError(f"criterion {criterion!r} not in {self.CRITERIA}")
+        if criterion != "svd" and dp is not None and dp.active:
+            raise ValueError("the ablation criteria run on one rank")
+        self.criterion = criterion
+        self.rng = torch.Generator(device=device)
+        self.rng.manual_seed(int(seed))
         bf = torch.bfloat16
         self.device = device
         self.D = gate.W.shape[1]
@@ -137,7 +149,14 @@ class FFNBlock:
         self.ch = B.channels_desc(self.sigma, self.n_keep)
 
     def estimate(self, x):
-        """a1 + a2: SwiGLU-L2 scores of the estimated gate/up outputs on x's context rows."""
+        """a1 + a2: SwiGLU-L2 scores of the estimated gate/up outputs on x's context rows (or
+        the ablation criterion's scores)."""
+        if self.criterion == "wanda":
+            B.sl_wanda_scores(self.ws, x[: self.n_ctx], self.n_ctx, [self.Wg, self.Wu], self.scores)
+            return
+        if self.criterion == "random":
+            self.scores.uniform_(generator=self.rng)
+            return
         xe = x if self.est_dtype == torch.bfloat16 else self.x_est
         if self.dp:  # statistics of this rank's context rows, summed over the ranks
             B.sl_svd_estimate_partials(self.ws, B.SL_CRIT_SWIGLU_L2, xe[: self.n_ctx], self.n_ctx,
@@ -230,7 +249,18 @@ class AttnProjBlock:
     part of the path: its output x_o and its gradients dq, dk, dv are inputs."""
 
     def __init__(self, q, k, v, o, lora_q, lora_k, lora_v, lora_o, lora_scale, est_k, n_q_heads, n_kv_heads,
-                 head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False, dp=None):
+                 head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False, dp=None, qk_criterion="channel",
+                 vo_criterion="l2", seed=0):
+        """qk_criterion: "channel" (the method's QK norm per KV channel), or the criterion
+        ablation's "head" (whole KV heads by the summed QK norm) and "random"; vo_criterion:
+        "l2" (the method's) or "random" (uniform scores from a generator seeded with `seed`)."""
+        if qk_criterion not in ("channel", "head", "random") or vo_criterion not in ("l2", "random"):
+            raise ValueError(f"criteria {qk_criterion!r}, {vo_criterion!r}")
+        if (qk_criterion, vo_criterion) != ("channel", "l2") and dp is not None and dp.active:
+            raise ValueError("the ablation criteria run on one rank")
+        self.qk_criterion, self.vo_criterion = qk_criterion, vo_criterion
+        self.rng = torch.Generator(device=device)
+        self.rng.manual_seed(int(seed))
         bf, f32 = torch.bfloat16, torch.float32
         dev = lambda t: t.to(device=device, dtype=bf).contiguous()
         self.device = device
@@ -243,6 +273,10 @@ class AttnProjBlock:
         self.dense = dense or ratio >= 1.0
         self.n_units = self.Dkv
         self.n_keep_u = self.n_units if self.dense else B.sl_keep_count(ratio, self.n_units)
+        # kept KV units of q/k (whole heads for the head-level criterion) and of v/o
+        self.n_keep_heads = self.hkv if self.dense else B.sl_keep_count(ratio, self.hkv)
+        self.n_keep_qk = self.n_keep_heads * head_dim if qk_criterion == "head" else self.n_keep_u
+        self.n_keep_vo = self.n_keep_u
         self.Wq, self.Wk, self.Wv, self.Wo = dev(q.W), dev(k.W), dev(v.W), dev(o.W)
         self.WA = [dev(q.W_A), dev(k.W_A), dev(v.W_A)]
         self.WB = [dev(q.W_B), dev(k.W_B), dev(v.W_B)]
@@ -278,12 +312,13 @@ class AttnProjBlock:
         s = self.scale
         # kept rows of the sliced weights (rows of W for q, k, v; rows of W^T for o), rebuilt
         # once per step after the selection and shared by the forward and backward calls
-        nq, nu = self.n_keep_u * self.hpg, self.n_keep_u
+        nq, nu = self.n_keep_qk * self.hpg, self.n_keep_qk
+        nv, no = self.n_keep_vo, self.n_keep_vo * self.hpg
         if self.dense:
             self.W_k = {"q": self.Wq, "k": self.Wk, "v": self.Wv, "o": self.Wo_t}
         else:
             self.W_k = {"q": _empty((nq, D), bf, device), "k": _empty((nu, D), bf, device),
-                        "v": _empty((nu, D), bf, device), "o": _empty((nq, D), bf, device)}
+                        "v": _empty((nv, D), bf, device), "o": _empty((no, D), bf, device)}
         self.lin = {
             "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT, w_kept=self.W_k["q"]),
             "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT, w_kept=self.W_k["k"]),
@@ -291,15 +326,25 @@ class AttnProjBlock:
             "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t, w_kept=self.W_k["o"]),
         }
         self.ch = {
-            "q": B.channels_desc(self.sig_q, self.n_keep_u * self.hpg),
-            "k": B.channels_desc(self.sig_k, self.n_keep_u),
-            "v": B.channels_desc(self.sig_v, self.n_keep_u),
-            "o": B.channels_desc(self.sig_o, self.n_keep_u * self.hpg),
+            "q": B.channels_desc(self.sig_q, self.n_keep_qk * self.hpg),
+            "k": B.channels_desc(self.sig_k, self.n_keep_qk),
+            "v": B.channels_desc(self.sig_v, self.n_keep_vo),
+            "o": B.channels_desc(self.sig_o, self.n_keep_vo * self.hpg),
         }
 
     def estimate(self, x):
-        """a1 + a2: QK scores over KV units and V scores from one pass over x's context rows."""
+        """a1 + a2: QK scores over KV units and V scores from one pass over x's context rows
+        (random scores replace them for the ablation's random criteria)."""
         C = self.n_ctx
+        if self.qk_criterion == "random" or self.vo_criterion == "random":
+            if (self.qk_criterion, self.vo_criterion) != ("random", "random"):
+                B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk,
+                                  scores_v=self.s_v, n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+            if self.qk_criterion == "random":
+                self.s_qk.uniform_(generator=self.rng)
+            if self.vo_criterion == "random":
+                self.s_v.uniform_(generator=self.rng)
+            return
         if self.dp:  # Gram matrix of this rank's Z, summed over the ranks
             B.sl_svd_estimate_partials(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.est_part,
                                        n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
@@ -310,20 +355,29 @@ class AttnProjBlock:
         B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
 
+    def _select_qk(self):
+        if self.qk_criterion == "head":
+            B.sl_select_heads(self.s_qk, self.hkv, self.hd, self.n_keep_heads, self.sig_k, self.hpg, self.sig_q)
+        else:
+            B.sl_select_channels(self.s_qk, self.n_keep_qk, self.sig_k, self.hpg, self.hd, self.sig_q)
+
+    def _select_vo(self):
+        B.sl_select_channels(self.s_v, self.n_keep_vo, self.sig_v, self.hpg, self.hd, self.sig_o)
+
     def _qk_chain(self):
-        B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
+        self._select_qk()
         for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k)):
             B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
 
     def _vo_chain(self):
-        B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+        self._select_vo()
         for n, w, sig in (("v", self.Wv, self.sig_v), ("o", self.Wo_t, self.sig_o)):
             B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
 
     def choose(self):
         """a3: the q/k set from the QK scores and the v/o set from the V scores."""
-        B.sl_select_channels(self.s_qk, self.n_keep_u, self.sig_k, self.hpg, self.hd, self.sig_q)
-        B.sl_select_channels(self.s_v, self.n_keep_u, self.sig_v, self.hpg, self.hd, self.sig_o)
+        self._select_qk()
+        self._select_vo()
 
     def compact(self):
         """The kept weight rows of q, k, v (rows of W) and o (rows of W^T) for this step."""

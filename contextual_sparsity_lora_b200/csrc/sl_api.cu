@@ -382,6 +382,37 @@ sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_keep, int
                                      heads_per_group > 0 ? sigma_wide : nullptr, nullptr, cs(stream)));
 }
 
+sl_status sl_select_heads(const float* scores, int32_t n_heads, int32_t head_dim, int32_t n_keep_heads,
+                          int32_t heads_per_group, int32_t* sigma, int32_t* sigma_wide, sl_stream stream) {
+  if (!scores || !sigma) return SL_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_heads > 1024 || head_dim < 1 || n_keep_heads < 1 || n_keep_heads > n_heads)
+    return SL_ERR_SHAPE;
+  if (sigma_wide && heads_per_group < 1) return SL_ERR_INVALID_ARG;
+  return from_kernel(select_heads(scores, n_heads, head_dim, n_keep_heads, heads_per_group, sigma, sigma_wide,
+                                  cs(stream)));
+}
+
+sl_status sl_wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int32_t n_proj,
+                          const void* const* w, int64_t d_out, int64_t ldw, float* scores, sl_workspace* ws,
+                          sl_stream stream) {
+  if (!x || !w || !scores || n_proj < 1 || n_proj > 4) return SL_ERR_INVALID_ARG;
+  if (n_ctx < 1 || d_in < 8 || d_out < 1 || ldx < d_in || ldw < d_in || d_in > 51200) return SL_ERR_SHAPE;
+  if (d_in % 8 || ldx % 8 || ldw % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+  for (int q = 0; q < n_proj; ++q) {
+    if (!w[q]) return SL_ERR_INVALID_ARG;
+    if (!al16(w[q])) return SL_ERR_ALIGNMENT;
+  }
+  float* scratch;
+  {
+    Carver c(nullptr);
+    scratch = c.take<float>((size_t)wanda_scratch_floats(n_ctx, d_in));
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  scratch = c.take<float>((size_t)wanda_scratch_floats(n_ctx, d_in));
+  return from_kernel(wanda_scores(x, n_ctx, d_in, ldx, n_proj, w, d_out, ldw, scores, scratch, cs(stream)));
+}
+
 // ------------------------------------------------------------------ a6
 sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx,
                           int64_t n_tok, int64_t n_ctx, int32_t in_layout, const sl_channels* in_ch, float* xa,

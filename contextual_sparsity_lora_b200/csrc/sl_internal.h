@@ -149,6 +149,16 @@ int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* coun
 // ---- selection (sl_select.cu)
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group,
                     int head_dim, int64_t n_wide, int32_t* sigma_wide, int64_t* n_keep_wide_out, cudaStream_t s);
+int select_heads(const float* scores, int n_heads, int head_dim, int n_keep_heads, int heads_per_group,
+                 int32_t* sigma, int32_t* sigma_wide, cudaStream_t s);
+
+// ---- criterion variants (sl_criteria.cu)
+// Wanda-style channel scores s_i = sum_p sum_j |W_p[i, j]| ||x[:, j]||_2 over n_ctx rows of x
+// (bf16 [n_ctx, d_in], ld ldx) and n_proj bf16 weights [d_out, d_in] (ld ldw); scratch holds
+// wanda_scratch_floats(n_ctx, d_in) floats.
+int64_t wanda_scratch_floats(int64_t n_ctx, int64_t d_in);
+int wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj, const void* const* w,
+                 int64_t d_out, int64_t ldw, float* scores, float* scratch, cudaStream_t s);
 
 // ---- helpers (sl_aux.cu)
 int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols,

@@ -212,6 +212,65 @@ void launch_select(const float* scores, int n, int n_keep, int32_t* sigma, int h
                 sigma_wide);
 }
 
+// Head-level selection: head score H_g = sum_d s[g * head_dim + d] (fp64, d order); the
+// n_keep_heads largest heads are kept (ties to the lower index, NaN below every number),
+// each with all of its head_dim channels. sigma[n_kv * head_dim]: channels of kept heads
+// ascending, then the others ascending; sigma_wide (query side, heads_per_group query heads
+// per KV head): channel (h, d) kept iff head h / heads_per_group is.
+__global__ void __launch_bounds__(kSelThreads) select_heads_kernel(const float* __restrict__ s, int n_heads,
+                                                                   int head_dim, int n_keep_heads, int hpg,
+                                                                   int32_t* __restrict__ sigma,
+                                                                   int32_t* __restrict__ sigma_wide) {
+  pdl_wait();
+  __shared__ uint32_t hkey[kSelThreads];
+  __shared__ uint8_t kept[kSelThreads];
+  __shared__ int kept_before[kSelThreads + 1];
+  const int g = threadIdx.x;
+  if (g < n_heads) {
+    double h = 0.0;
+    for (int d = 0; d < head_dim; ++d) h += (double)s[(int64_t)g * head_dim + d];
+    hkey[g] = score_key((float)h);
+  }
+  __syncthreads();
+  if (g < n_heads) {
+    // rank among the heads: larger keys first, equal keys by index
+    const uint32_t k = hkey[g];
+    int rank = 0;
+    for (int o = 0; o < n_heads; ++o) rank += (hkey[o] > k || (hkey[o] == k && o < g)) ? 1 : 0;
+    kept[g] = rank < n_keep_heads;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // heads are few: a serial prefix count
+    int c = 0;
+    for (int o = 0; o < n_heads; ++o) {
+      kept_before[o] = c;
+      c += kept[o];
+    }
+    kept_before[n_heads] = c;
+  }
+  __syncthreads();
+  // KV side: head g's channels go to its slot among kept or dropped heads
+  for (int64_t c = threadIdx.x; c < (int64_t)n_heads * head_dim; c += kSelThreads) {
+    const int hg = (int)(c / head_dim), d = (int)(c % head_dim);
+    const int kb = kept_before[hg];
+    const int64_t pos = kept[hg] ? (int64_t)kb * head_dim + d
+                                 : (int64_t)n_keep_heads * head_dim + (int64_t)(hg - kb) * head_dim + d;
+    sigma[pos] = (int32_t)c;
+  }
+  if (!sigma_wide) return;
+  // query side: query head h follows KV head h / hpg; kept query heads keep index order
+  const int nq = n_heads * hpg;
+  for (int64_t c = threadIdx.x; c < (int64_t)nq * head_dim; c += kSelThreads) {
+    const int h = (int)(c / head_dim), d = (int)(c % head_dim);
+    const int hg = h / hpg, r = h % hpg;
+    const int kb = kept_before[hg];
+    const int64_t qkb = (int64_t)kb * hpg + r;  // kept query heads before h (kept KV heads are contiguous groups)
+    const int64_t qdb = (int64_t)(hg - kb) * hpg + r;
+    const int64_t pos = kept[hg] ? qkb * head_dim + d : (int64_t)n_keep_heads * hpg * head_dim + qdb * head_dim + d;
+    sigma_wide[pos] = (int32_t)c;
+  }
+}
+
 }  // namespace
 
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group, int head_dim,
@@ -229,6 +288,17 @@ int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sig
   else
     launch_select<40>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
   if (n_keep_wide_out) *n_keep_wide_out = sigma_wide ? n_keep * heads_per_group : 0;
+  if (launch_failed("sl_select")) return 5;
+  note_launch();
+  return 0;
+}
+
+int select_heads(const float* scores, int n_heads, int head_dim, int n_keep_heads, int heads_per_group,
+                 int32_t* sigma, int32_t* sigma_wide, cudaStream_t s) {
+  if (n_heads < 1 || n_heads > kSelThreads || head_dim < 1 || n_keep_heads < 1 || n_keep_heads > n_heads) return 1;
+  if (sigma_wide && heads_per_group < 1) return 1;
+  launch_kernel(select_heads_kernel, 1, kSelThreads, 0, s, scores, n_heads, head_dim, n_keep_heads,
+                sigma_wide ? heads_per_group : 1, sigma, sigma_wide);
   if (launch_failed("sl_select")) return 5;
   note_launch();
   return 0;

@@ -216,6 +216,31 @@ SL_API sl_status sl_svd_scores_from_partials(sl_criterion crit, sl_dtype dtype, 
 SL_API sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma,
                              int32_t heads_per_group, int32_t head_dim, int32_t* sigma_wide, sl_stream stream);
 
+/* Head-level variant of the QK selection ([WT] "Oracle Sparse Neuron Selection Criteria",
+ * why not head-level pruning for QK, and the criterion ablation of Table 10: head-level pruning
+ * with the same metric). scores: the n_heads * head_dim unit scores of sl_svd_estimate
+ * (SL_CRIT_QK); the head score is their sum over the head's head_dim units; the n_keep_heads
+ * largest heads are kept whole (ties to the lower head index, NaN below every number).
+ * sigma[n_heads * head_dim] (KV channels): channels of kept heads ascending, then the others
+ * ascending (kept count n_keep_heads * head_dim); sigma_wide (optional, query side,
+ * [n_heads * heads_per_group * head_dim]): query channel (h, d) is kept iff KV head
+ * h / heads_per_group is. n_heads <= 1024. */
+SL_API sl_status sl_select_heads(const float* scores, int32_t n_heads, int32_t head_dim, int32_t n_keep_heads,
+                                 int32_t heads_per_group, int32_t* sigma, int32_t* sigma_wide, sl_stream stream);
+
+/* Wanda-style channel criterion, the FFN alternative of the criterion ablation ([WT] "Oracle
+ * Sparse Neuron Selection Criteria", Table 10: Wanda against L2 norm and random pruning for the
+ * FFN projections). Wanda's weight importance is |W[i, j]| ||X[:, j]||_2 with the input feature
+ * norm over the context rows; the channel score sums it over the channel's row, and the n_proj
+ * weights that share one index set (gate and up) add theirs:
+ *   scores[i] = sum_p sum_j |w[p][i, j]| * sqrt(sum_t x[t, j]^2),  i < d_out.
+ *   x: bf16 [n_ctx, d_in] (ld ldx), the context rows; w[p]: frozen bf16 [d_out, d_in] (ld ldw),
+ *   16-byte aligned, d_in % 8 == 0, d_in <= 51200, n_proj <= 4. Reads every weight byte once;
+ *   fp32 sums in a fixed order. Workspace: (ceil(n_ctx / 128) + 1) * d_in floats. */
+SL_API sl_status sl_wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int32_t n_proj,
+                                 const void* const* w, int64_t d_out, int64_t ldw, float* scores,
+                                 sl_workspace* ws, sl_stream stream);
+
 /* a6: the dense LoRA branch ([WT] Algorithm 1 "computed densely and added"; section 3.2:
  * LoRA gradients are always dense).
  * SL_LORA_FWD: for n_ad adapters sharing the input x [n_tok, d_in] (ld ldx), with

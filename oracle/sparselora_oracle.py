@@ -44,6 +44,14 @@ Readings where the pages are silent or ambiguous (each is listed in the design doc):
       lower index, NaN below every number; the kept set is returned ascending.
   R9  The index set is a constant for the backward pass.
 
+  R13 Head-level QK variant (criterion ablation, Table 10): a KV head's score is the sum
+      of its head_dim unit scores; whole heads are kept (top n_heads_keep, ties to the lower
+      head index) with every channel of the head.
+  R14 Wanda-style channel criterion (criterion ablation, Table 10; Wanda's importance
+      |W[i, j]| ||X[:, j]||_2): the channel score sums it over the channel's row of the
+      frozen weight, over every projection that shares the index set (gate and up), with the
+      feature norms over the context rows of the layer input.
+
 Parity unpinned (no printed value or closed form pins them):
 the GQA aggregation of R5 and the V-space reading of R4.
 """
@@ -161,6 +169,13 @@ def qk_from_sumsq(q2, k2, n_q_heads, n_kv_heads, head_dim):
     return (q_group * k).reshape(-1)
 
 
+def wanda_scores(X_ctx, Ws):
+    """Wanda-style channel scores (reading R14): s_i = sum_p sum_j |W_p[i, j]| ||X[:, j]||_2,
+    W_p in nn.Linear storage [D_out, D_in], norms over the rows of X_ctx."""
+    n = np.sqrt(np.sum(f64(X_ctx) ** 2, axis=0))
+    return sum(np.abs(f64(W)) @ n for W in Ws)
+
+
 # ---------------------------------------------------------------------------
 # Selection  [WT Algorithm 1: keep the top ceil(r * D_out) channels; PN top-n]
 # ---------------------------------------------------------------------------
@@ -207,6 +222,15 @@ def expand_units(units, n_q_heads, n_kv_heads, head_dim):
 # ---------------------------------------------------------------------------
 # Sparse frozen branch + dense LoRA  [WT Algorithm 1, Figure 8, section 3.2]
 # ---------------------------------------------------------------------------
+
+def select_heads(unit_scores, n_kv_heads, head_dim, n_keep_heads):
+    """Head-level QK selection (reading R13): head score = sum of its unit scores; the
+    n_keep_heads best heads (select_top order) keep all their channels. Returns the kept KV
+    channels ascending."""
+    h = f64(unit_scores).reshape(n_kv_heads, head_dim).sum(axis=1)
+    heads = select_top(h, n_keep_heads)
+    return (heads[:, None] * head_dim + np.arange(head_dim)[None, :]).reshape(-1)
+
 
 def sliced_weight(W, idx, slice_kind):
     """W_math restricted to the kept channels, with dropped channels set to zero:

@@ -411,3 +411,47 @@ def test_sum_of_squares_statistics_add_over_row_parts():
         np.testing.assert_allclose(oracle.sumsq(Y[:cut]) + oracle.sumsq(Y[cut:]), oracle.sumsq(Y), rtol=1e-13)
     # columns of constant value c over n rows: n c^2
     np.testing.assert_allclose(oracle.sumsq(np.full((6, 3), 2.5)), np.full(3, 6 * 2.5 ** 2), rtol=0)
+
+
+# ----------------------------------------------------------------------- criterion variants
+
+def test_wanda_scores_brute_force_tiny():
+    """Wanda-style channel scores (R14) against explicit loops over rows, columns and tokens."""
+    rng = np.random.default_rng(41)
+    X = rng.standard_normal((5, 4))
+    Ws = [rng.standard_normal((3, 4)), rng.standard_normal((3, 4))]
+    want = np.zeros(3)
+    for i in range(3):
+        for W in Ws:
+            for j in range(4):
+                norm = 0.0
+                for t in range(5):
+                    norm += X[t, j] * X[t, j]
+                want[i] += abs(W[i, j]) * norm ** 0.5
+    np.testing.assert_allclose(oracle.wanda_scores(X, Ws), want, rtol=1e-13)
+
+
+def test_wanda_scores_closed_forms():
+    # constant columns c_j over T rows give norms sqrt(T) |c_j|; W = I picks them out
+    T, c = 9, np.array([2.0, -3.0, 0.5])
+    X = np.tile(c, (T, 1))
+    np.testing.assert_allclose(oracle.wanda_scores(X, [np.eye(3)]), np.sqrt(T) * np.abs(c), rtol=1e-14)
+    # homogeneous in |W| and in |X|
+    rng = np.random.default_rng(42)
+    X, W = rng.standard_normal((7, 6)), rng.standard_normal((4, 6))
+    base = oracle.wanda_scores(X, [W])
+    np.testing.assert_allclose(oracle.wanda_scores(-3.0 * X, [W]), 3.0 * base, rtol=1e-13)
+    np.testing.assert_allclose(oracle.wanda_scores(X, [-0.5 * W]), 0.5 * base, rtol=1e-13)
+    np.testing.assert_allclose(oracle.wanda_scores(X, [W, W]), 2.0 * base, rtol=1e-13)
+
+
+def test_select_heads_special_cases():
+    # head_dim 1: whole heads are single units, so this is the plain top-n
+    s = np.array([0.3, 2.0, 1.1, 2.0, -1.0])
+    np.testing.assert_array_equal(oracle.select_heads(s, 5, 1, 2), oracle.select_top(s, 2))
+    # equal head sums: the lower heads
+    np.testing.assert_array_equal(oracle.select_heads(np.ones(12), 3, 4, 2), np.arange(8))
+    # a head with the largest single unit but the smaller sum loses to the head with the larger sum
+    s = np.array([10.0, 0.0, 0.0, 0.0, 3.0, 3.0, 3.0, 3.0])
+    np.testing.assert_array_equal(oracle.select_heads(s, 2, 4, 1), np.arange(4, 8))
+    np.testing.assert_array_equal(oracle.select_top(s, 4), np.array([0, 4, 5, 6]))
