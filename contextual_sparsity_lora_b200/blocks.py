@@ -33,6 +33,13 @@ class _Side:
     def join(self):
         torch.cuda.current_stream().wait_stream(self.stream)
 
+    def mark(self):
+        """An event after the work queued on the side stream so far (wait on it with
+        torch.cuda.current_stream().wait_event to join only that part)."""
+        ev = torch.cuda.Event()
+        ev.record(self.stream)
+        return ev
+
 
 class DataParallel:
     """Ranks that each hold part of one global batch ([WT] "Oracle Sparse Neuron Selection
@@ -193,13 +200,22 @@ class FFNBlock:
         lay = B.SL_LAYOUT_NATURAL if self.dense else B.SL_LAYOUT_SIGMA
         # no context rows: nothing to score, every row is dense (data-parallel ranks still take
         # part in the selection of the batch)
+        down_side = False
         if not self.dense and (C > 0 or self.dp):
             if self.concurrent:  # x A^T of gate/up does not depend on the selection
                 with self.side.fork():
                     B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
                                       xa=self.xa_gu)
-                self.select(x)
-                self.side.join()
+                lora_done = self.side.mark()
+                self.estimate(x)
+                self.choose()
+                kept = self.sigma[: self.n_keep]
+                B.sl_permute_rows(self.Wg, kept, self.Wg_k)
+                B.sl_permute_rows(self.Wu, kept, self.Wu_k)
+                with self.side.fork():  # down's kept rows are needed only by the down product
+                    B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+                torch.cuda.current_stream().wait_event(lora_done)
+                down_side = True
             else:
                 self.select(x)
                 B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
@@ -208,6 +224,8 @@ class FFNBlock:
             B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu, xa=self.xa_gu)
         B.sl_sparse_linear_fwd(self.ws, [self.lin_g, self.lin_u], [self.ch], B.SL_EPI_SWIGLU, x, C, self.xa_s_gu,
                                [self.g, self.u, self.h], out_layout=B.SL_LAYOUT_SIGMA)
+        if down_side:
+            self.side.join()
         B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_d], self.h, C, self.xa_s_d, xa=self.xa_d,
                           in_layout=lay, in_ch=self.ch)
         B.sl_sparse_linear_fwd(self.ws, [self.lin_d], [self.ch], B.SL_EPI_NONE, self.h, C, self.xa_s_d, [self.y],

@@ -548,13 +548,23 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     int64_t ccount[4];
     int cr[4];
     int64_t koff = 0;
+    // dya and dB are sums of reductions into zeroed outputs; dA accumulates its two parts
+    {
+      float* zp[12];
+      int64_t zn[12];
+      int nz = 0;
+      for (int i = 0; i < n_ad; ++i) {
+        zp[nz] = dya[i];
+        zn[nz++] = T * lin[i].r;
+        zp[nz] = dB[i];
+        zn[nz++] = lin[i].d_out * lin[i].r;
+        zp[nz] = dA[i];
+        zn[nz++] = (int64_t)lin[i].r * d_in;
+      }
+      if (int rc = zero_f32(zp, zn, nz, s)) return from_kernel(rc);
+    }
     for (int i = 0; i < n_ad; ++i) {
       const sl_linear& L = lin[i];
-      // dya and dB are sums of reductions into zeroed outputs; dA accumulates its two parts
-      if (cudaMemsetAsync(dya[i], 0, sizeof(float) * T * L.r, s) != cudaSuccess ||
-          cudaMemsetAsync(dB[i], 0, sizeof(float) * L.d_out * L.r, s) != cudaSuccess ||
-          cudaMemsetAsync(dA[i], 0, sizeof(float) * L.r * d_in, s) != cudaSuccess)
-        return SL_ERR_CUDA;
       cr[i] = L.r;
       const void* xa_blk = static_cast<const uint16_t*>(xa_s) + koff;
       koff += L.r;

@@ -145,6 +145,8 @@ int lora_dual_launch(const DualSpec* specs, int n, int* err, cudaStream_t s);
 // [rows, r[i]] and its values also go to columns [sum_{j<i} r[j], ... + r[i]) of cat (ld ld_cat).
 int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* count, int n, cudaStream_t s,
                   void* cat = nullptr, const int* r = nullptr, int ld_cat = 0);
+// Zeroes n <= 12 fp32 buffers (one launch).
+int zero_f32(float* const* ptrs, const int64_t* counts, int n, cudaStream_t s);
 
 // ---- selection (sl_select.cu)
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group,

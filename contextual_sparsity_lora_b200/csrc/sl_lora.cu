@@ -400,6 +400,28 @@ __global__ void __launch_bounds__(256) cast_bf16_kernel(const __grid_constant__ 
   }
 }
 
+// Zeroes up to kMaxZero fp32 buffers in one launch (blockIdx.y = buffer).
+constexpr int kMaxZero = 12;
+struct ZeroParams {
+  float* p[kMaxZero];
+  int64_t n[kMaxZero];
+};
+
+__global__ void __launch_bounds__(256) zero_f32_kernel(const __grid_constant__ ZeroParams z) {
+  pdl_wait();
+  float* p = z.p[blockIdx.y];
+  const int64_t n = z.n[blockIdx.y];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    float4* q = reinterpret_cast<float4*>(p);
+    for (int64_t i = i0; i < n / 4; i += stride) q[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t i = n / 4 * 4 + i0; i < n; i += stride) p[i] = 0.f;
+  } else {
+    for (int64_t i = i0; i < n; i += stride) p[i] = 0.f;
+  }
+}
+
 bool encode(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows) {
   return encode_bf16_2d(m, ptr, rows, cols, ld, box_cols, box_rows, true);
 }
@@ -490,6 +512,24 @@ int cast_f32_bf16(const float* const* src, void* const* dst, const int64_t* coun
   P.n = n;
   const unsigned gx = (unsigned)std::min<int64_t>((mx + 255) / 256, 1184);
   launch_kernel(cast_bf16_kernel, dim3(gx, n), 256, 0, s, P);
+  if (launch_failed("sl_lora")) return 5;
+  note_launch();
+  return 0;
+}
+
+int zero_f32(float* const* ptrs, const int64_t* counts, int n, cudaStream_t s) {
+  if (n <= 0) return 0;
+  if (n > kMaxZero) return 1;
+  ZeroParams Z;
+  memset(&Z, 0, sizeof(Z));
+  int64_t mx = 0;
+  for (int i = 0; i < n; ++i) {
+    Z.p[i] = ptrs[i];
+    Z.n[i] = counts[i];
+    mx = std::max(mx, counts[i]);
+  }
+  const unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((mx / 4 + 255) / 256, 592));
+  launch_kernel(zero_f32_kernel, dim3(gx, n), 256, 0, s, Z);
   if (launch_failed("sl_lora")) return 5;
   note_launch();
   return 0;
