@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-LoRA companion measurement")
+    ap.add_argument("--no-layer", action="store_true", help="skip the whole-decoder-layer measurement")
     ap.add_argument("--stages-only", action="store_true",
                     help="time only the selection stages (estimator, criterion, top-n, compaction) of both blocks "
                          "and print them; no step, no headline line")
@@ -363,6 +364,32 @@ def _oracle_layer(oracle, X, XO, dq, dk, dv, dyo, Xf, dyf, ctx, W, F, L, Wf, Ff,
     oracle.ffn_bwd(Xf, dyf, ctx, Wf["gate"], Wf["up"], Wf["down"], Lf["gate"], Lf["up"], Lf["down"], s, idx, fwd=fwd)
 
 
+def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
+    """The whole decoder layer around the same blocks (RMSNorm, sparse q/k/v, causal GQA
+    attention core, sparse o, residual, RMSNorm, sparse FFN, residual), forward and backward
+    on the step's 8 x 512 tokens: context, not the headline."""
+    from contextual_sparsity_lora_b200.layer import DecoderLayer
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(77)
+    g1 = 1.0 + 0.1 * torch.randn(ac.hidden, generator=gen)
+    g2 = 1.0 + 0.1 * torch.randn(ac.hidden, generator=gen)
+    layer = DecoderLayer(attn, ffn, g1, g2, perm, ac.batch)
+    x, dy = step_in["x"], step_in["dy"]
+    for _ in range(2):
+        layer.step(x, dy)
+    torch.cuda.synchronize()
+    try:  # the attention core's autograd backward inside a captured graph
+        replay, captured = capture_graph(lambda: layer.step(x, dy), warm=False).replay, True
+    except Exception as e:  # noqa: BLE001 - fall back to the eager layer step
+        print(f"layer step not captured ({type(e).__name__}: {e}); timing the eager step", file=sys.stderr)
+        torch.cuda.synchronize()
+        replay, captured = (lambda: layer.step(x, dy)), False
+    ms = time_steps(replay, K, W, 1, device) / K
+    return {"value": ac.n_tok / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "cuda_graph": captured, "attention_core": "torch scaled_dot_product_attention (causal, GQA)",
+            "layer": "RMSNorm, sparse q/k/v, attention, sparse o, residual, RMSNorm, sparse SwiGLU FFN, residual"}
+
+
 def e2e_measure(attn, ffn, step_in, K, W, world, device):
     """Same step through the public API with host buffers: every step copies that step's
     inputs from pinned host memory and reads the LoRA gradients back."""
@@ -544,6 +571,8 @@ def main():
                               "effective_tflops": d_fl["total"] / (d_ms / args.steps / 1e3) / 1e12}
         line["speedup_vs_dense_lora"] = line["dense_lora"]["ms_per_step"] / ms_step
         del d_attn, d_ffn, d_graph
+    if world == 1 and not args.no_layer:
+        line["full_layer"] = full_layer_measure(attn, ffn, step_in, perm, ac, args.steps, max(args.warmup, 3), device)
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_measure(attn, ffn, step_in, args.steps, max(args.warmup, 3), world, device)
         line["e2e"] = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -29,7 +29,8 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_svd_estimate", "sl_select_channels", "sl_lora_fwd_bwd", "sl_sparse_linear_fwd",
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
-            "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores")
+            "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
+            "sl_add_rows")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -81,6 +82,9 @@ def lib():
                                                   c_int32, c_int32, c_int32, c_int32, P, P, P, P]
         L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
         L.sl_select_heads.argtypes = [P, c_int32, c_int32, c_int32, c_int32, P, P, P]
+        L.sl_rmsnorm_fwd.argtypes = [P, c_int64, P, c_int64, P, c_int64, P, c_float, P, c_int64, P, c_int64, c_int64, P]
+        L.sl_rmsnorm_bwd.argtypes = [P, c_int64, P, c_int64, P, P, P, c_int64, P, c_int64, c_int64, c_int64, P]
+        L.sl_add_rows.argtypes = [P, c_int64, P, c_int64, P, c_int64, c_int64, c_int64, P]
         L.sl_wanda_scores.argtypes = [P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p), c_int64, c_int64, P,
                                       POINTER(SlWorkspaceC), P]
         L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
@@ -251,6 +255,25 @@ def sl_wanda_scores(ws: Workspace, x, n_ctx, w, scores):
     """Wanda-style channel scores over the context rows x[:n_ctx] for the weights w (one index set)."""
     ws.call("sl_wanda_scores", _ptr(x), int(n_ctx), x.shape[1], x.stride(0), len(w), _ptrs(w), w[0].shape[0],
             w[0].stride(0), _ptr(scores))
+
+
+def sl_rmsnorm_fwd(x, gamma, eps, y, rstd, res=None, sum_out=None):
+    _check("sl_rmsnorm_fwd",
+           lib().sl_rmsnorm_fwd(_ptr(x), x.stride(0), _ptr(res), res.stride(0) if res is not None else 0,
+                                _ptr(sum_out), sum_out.stride(0) if sum_out is not None else 0, _ptr(gamma),
+                                float(eps), _ptr(y), y.stride(0), _ptr(rstd), x.shape[0], x.shape[1], _stream()))
+
+
+def sl_rmsnorm_bwd(dy, x, gamma, rstd, dx, dres=None):
+    _check("sl_rmsnorm_bwd",
+           lib().sl_rmsnorm_bwd(_ptr(dy), dy.stride(0), _ptr(x), x.stride(0), _ptr(gamma), _ptr(rstd), _ptr(dres),
+                                dres.stride(0) if dres is not None else 0, _ptr(dx), dx.stride(0), x.shape[0],
+                                x.shape[1], _stream()))
+
+
+def sl_add_rows(a, b, out):
+    _check("sl_add_rows", lib().sl_add_rows(_ptr(a), a.stride(0), _ptr(b), b.stride(0), _ptr(out), out.stride(0),
+                                            a.shape[0], a.shape[1], _stream()))
 
 
 def sl_lora_fwd_bwd(ws: Workspace, mode, lins, x, n_ctx, xa_s, xa=None, in_layout=SL_LAYOUT_NATURAL, in_ch=None,

@@ -441,32 +441,75 @@ class AttnProjBlock:
                                in_layout=B.SL_LAYOUT_NATURAL)
         return self.y
 
-    def backward(self, dy, dq, dk, dv):
+    def _o_backward(self, ws, dy):
+        """o's LoRA gradients and its input gradient dx_o."""
+        lo = self.lin["o"]
         C = self.n_ctx
-        lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
+        B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
+                          dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
+        B.sl_sparse_linear_bwd(ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
+                               dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
 
-        def o_chain(ws):  # o's LoRA gradients and its input gradient dx_o
-            B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
-                              dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
-            B.sl_sparse_linear_bwd(ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
-                                   dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
+    def _qkv_backward(self, ws, dq, dk, dv):
+        """q, k, v LoRA gradients and dx."""
+        lq, lk, lv = (self.lin[n] for n in "qkv")
+        C = self.n_ctx
+        B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
+                          dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
+                          dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
+        B.sl_sparse_linear_bwd(ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
+                               [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
 
-        def qkv_chain(ws):  # q, k, v LoRA gradients and dx; independent of the o chain
-            B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
-                              dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
-                              dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
-            B.sl_sparse_linear_bwd(ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
-                                   [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
-
-        if self.concurrent:
+    def backward(self, dy, dq, dk, dv):
+        if self.concurrent:  # the o chain and the q/k/v chain are independent
             with self.side.fork():
-                o_chain(self.side.ws)
-            qkv_chain(self.ws)
+                self._o_backward(self.side.ws, dy)
+            self._qkv_backward(self.ws, dq, dk, dv)
             self.side.join()
         else:
-            o_chain(self.ws)
-            qkv_chain(self.ws)
+            self._o_backward(self.ws, dy)
+            self._qkv_backward(self.ws, dq, dk, dv)
         return self.dx, self.dx_o
+
+    # ---- the same step in the order of a decoder layer, where the attention core sits between
+    # q/k/v and o: forward_qkv, forward_o, then backward_o, backward_qkv
+
+    def forward_qkv(self, x):
+        """The selection on x's context rows and q, k, v (natural column layout)."""
+        C = self.n_ctx
+        self.x = x
+        lq, lk, lv = (self.lin[n] for n in "qkv")
+        sel = not self.dense and (C > 0 or self.dp is not None)
+        if sel and self.concurrent:
+            with self.side.fork():
+                B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
+            self.select(x)
+            self.side.join()
+        else:
+            if sel:
+                self.select(x)
+            B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
+        B.sl_sparse_linear_fwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, x, C,
+                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=B.SL_LAYOUT_NATURAL)
+        return self.q, self.kk, self.vv
+
+    def forward_o(self, x_o):
+        """o of the attention output x_o (its input channels sliced by the v/o selection)."""
+        C = self.n_ctx
+        self.x_o = x_o
+        lo = self.lin["o"]
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+        B.sl_sparse_linear_fwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, x_o, C, self.xa_s_o, [self.y],
+                               in_layout=B.SL_LAYOUT_NATURAL)
+        return self.y
+
+    def backward_o(self, dy):
+        self._o_backward(self.ws, dy)
+        return self.dx_o
+
+    def backward_qkv(self, dq, dk, dv):
+        self._qkv_backward(self.ws, dq, dk, dv)
+        return self.dx
 
     def read_device_flag(self) -> int:
         """Device error word of both workspaces (0: no device-side timeout); synchronises."""

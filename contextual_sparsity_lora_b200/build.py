@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsparselora.so")
-SOURCES = ["sl_api.cu", "sl_gemm.cu", "sl_estimator.cu", "sl_select.cu", "sl_aux.cu", "sl_lora.cu", "sl_noalloc.cu", "sl_est_tc.cu", "sl_criteria.cu"]
+SOURCES = ["sl_api.cu", "sl_gemm.cu", "sl_estimator.cu", "sl_select.cu", "sl_aux.cu", "sl_lora.cu", "sl_noalloc.cu", "sl_est_tc.cu", "sl_criteria.cu", "sl_layer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

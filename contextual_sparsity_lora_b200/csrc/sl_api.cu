@@ -413,6 +413,41 @@ sl_status sl_wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ld
   return from_kernel(wanda_scores(x, n_ctx, d_in, ldx, n_proj, w, d_out, ldw, scores, scratch, cs(stream)));
 }
 
+// ------------------------------------------------------------------ decoder layer pieces
+namespace {
+bool rows_ok(const void* p, int64_t ld, int64_t d) { return p && al16(p) && ld >= d && ld % 8 == 0; }
+}  // namespace
+
+sl_status sl_rmsnorm_fwd(const void* x, int64_t ldx, const void* res, int64_t ldr, void* sum_out, int64_t lds,
+                         const void* gamma, float eps, void* y, int64_t ldy, float* rstd, int64_t n_rows, int64_t d,
+                         sl_stream stream) {
+  if (!x || !gamma || !y || !rstd || (res && !sum_out)) return SL_ERR_INVALID_ARG;
+  if (n_rows < 1 || d < 8 || d % 8 || !(eps >= 0.f)) return SL_ERR_SHAPE;
+  if (!rows_ok(x, ldx, d) || !rows_ok(y, ldy, d) || !al16(gamma) || (res && (!rows_ok(res, ldr, d) ||
+                                                                             !rows_ok(sum_out, lds, d))))
+    return SL_ERR_ALIGNMENT;
+  return from_kernel(rmsnorm_fwd(x, ldx, res, ldr, sum_out, lds, gamma, eps, y, ldy, rstd, n_rows, d, cs(stream)));
+}
+
+sl_status sl_rmsnorm_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx, const void* gamma,
+                         const float* rstd, const void* dres, int64_t ldr, void* dx, int64_t lddx, int64_t n_rows,
+                         int64_t d, sl_stream stream) {
+  if (!dy || !x || !gamma || !rstd || !dx) return SL_ERR_INVALID_ARG;
+  if (n_rows < 1 || d < 8 || d % 8) return SL_ERR_SHAPE;
+  if (!rows_ok(dy, lddy, d) || !rows_ok(x, ldx, d) || !rows_ok(dx, lddx, d) || !al16(gamma) ||
+      (dres && !rows_ok(dres, ldr, d)))
+    return SL_ERR_ALIGNMENT;
+  return from_kernel(rmsnorm_bwd(dy, lddy, x, ldx, gamma, rstd, dres, ldr, dx, lddx, n_rows, d, cs(stream)));
+}
+
+sl_status sl_add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, int64_t ldo, int64_t n_rows,
+                      int64_t d, sl_stream stream) {
+  if (!a || !b || !out) return SL_ERR_INVALID_ARG;
+  if (n_rows < 1 || d < 8 || d % 8) return SL_ERR_SHAPE;
+  if (!rows_ok(a, lda, d) || !rows_ok(b, ldb, d) || !rows_ok(out, ldo, d)) return SL_ERR_ALIGNMENT;
+  return from_kernel(add_rows(a, lda, b, ldb, out, ldo, n_rows, d, cs(stream)));
+}
+
 // ------------------------------------------------------------------ a6
 sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx,
                           int64_t n_tok, int64_t n_ctx, int32_t in_layout, const sl_channels* in_ch, float* xa,

@@ -154,6 +154,15 @@ int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sig
 int select_heads(const float* scores, int n_heads, int head_dim, int n_keep_heads, int heads_per_group,
                  int32_t* sigma, int32_t* sigma_wide, cudaStream_t s);
 
+// ---- decoder layer pieces (sl_layer.cu)
+int rmsnorm_fwd(const void* x, int64_t ldx, const void* res, int64_t ldr, void* sum_out, int64_t lds,
+                const void* gamma, float eps, void* y, int64_t ldy, float* rstd, int64_t n_rows, int64_t d,
+                cudaStream_t s);
+int rmsnorm_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx, const void* gamma, const float* rstd,
+                const void* dres, int64_t ldr, void* dx, int64_t lddx, int64_t n_rows, int64_t d, cudaStream_t s);
+int add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, int64_t ldo, int64_t n_rows, int64_t d,
+             cudaStream_t s);
+
 // ---- criterion variants (sl_criteria.cu)
 // Wanda-style channel scores s_i = sum_p sum_j |W_p[i, j]| ||x[:, j]||_2 over n_ctx rows of x
 // (bf16 [n_ctx, d_in], ld ldx) and n_proj bf16 weights [d_out, d_in] (ld ldw); scratch holds

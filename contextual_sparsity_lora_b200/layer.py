@@ -1,0 +1,102 @@
+"""One LLaMA-style decoder layer around the sparse projections, forward and backward
+([WT] "Putting It All Together": the sparse q/k/v/o and FFN projections inside the model's
+layers; the per-layer context/output split, so output rows attend to context keys and values
+computed with the sparse projections).
+
+    h1 = RMSNorm(x, g1); q, k, v = sparse projections of h1; a = causal GQA attention(q, k, v)
+    x2 = x + o(a); h2 = RMSNorm(x2, g2); y = x2 + FFN(h2)
+
+RMSNorm, the residual adds and every projection run in libsparselora's kernels; the attention
+core (not one of the method's steps) is torch's scaled_dot_product_attention, a library call
+like a cuBLAS GEMM, with its backward through autograd. Rows are in context-first order like
+the blocks' (sl_permute_rows moves q, k, v to sequence order for the attention core and its
+output back). No rotary positional encoding: the pages do not say how it meets channel
+sparsity (a rotation mixes channel pairs that the selection may split)."""
+from __future__ import annotations
+
+import torch
+import torch.nn.functional as Fn
+
+from . import binding as B
+from .blocks import AttnProjBlock, FFNBlock
+
+
+class DecoderLayer:
+    def __init__(self, attn: AttnProjBlock, ffn: FFNBlock, gamma1, gamma2, perm, n_seq: int, eps: float = 1e-5):
+        """attn, ffn: the layer's projection blocks (same n_tok and n_ctx); gamma1, gamma2: frozen
+        RMSNorm gains [D]; perm: int64 [n_tok], context-first position p holds sequence-order row
+        perm[p] (rows of n_seq sequences of equal length)."""
+        dev = attn.device
+        self.attn, self.ffn = attn, ffn
+        self.g1 = gamma1.to(device=dev, dtype=torch.bfloat16).contiguous()
+        self.g2 = gamma2.to(device=dev, dtype=torch.bfloat16).contiguous()
+        self.eps = float(eps)
+        self.n_seq = int(n_seq)
+        T, D = attn.n_tok, attn.D
+        self.T, self.D = T, D
+        self.S = T // self.n_seq
+        perm = torch.as_tensor(perm, dtype=torch.int64, device=dev)
+        inv = torch.empty_like(perm)
+        inv[perm] = torch.arange(T, device=dev)
+        self.perm = perm.to(torch.int32).contiguous()  # sequence-order row of each context-first row
+        self.inv = inv.to(torch.int32).contiguous()    # context-first row of each sequence-order row
+        bf, f32 = torch.bfloat16, torch.float32
+        e = lambda *sh, dt=bf: torch.empty(*sh, dtype=dt, device=dev)
+        self.h1, self.x2, self.h2, self.y = e(T, D), e(T, D), e(T, D), e(T, D)
+        self.rstd1, self.rstd2 = e(T, dt=f32), e(T, dt=f32)
+        Dq, Dkv = attn.Dq, attn.Dkv
+        self.q_nat, self.k_nat, self.v_nat = e(T, Dq), e(T, Dkv), e(T, Dkv)
+        self.a_cf = e(T, Dq)
+        self.da_nat = e(T, Dq)
+        self.dq_cf, self.dk_cf, self.dv_cf = e(T, Dq), e(T, Dkv), e(T, Dkv)
+        self.dx2, self.dx = e(T, D), e(T, D)
+
+    def _to_seq(self, src, dst):
+        B.sl_permute_rows(src, self.inv, dst)
+
+    def _to_cf(self, src, dst):
+        B.sl_permute_rows(src, self.perm, dst)
+
+    def _heads(self, t, n_heads):
+        """[T, n_heads * hd] sequence-order rows -> [n_seq, n_heads, S, hd] view."""
+        return t.view(self.n_seq, self.S, n_heads, self.attn.hd).transpose(1, 2)
+
+    def forward(self, x):
+        at = self.attn
+        B.sl_rmsnorm_fwd(x, self.g1, self.eps, self.h1, self.rstd1)
+        q, k, v = at.forward_qkv(self.h1)
+        for src, dst in ((q, self.q_nat), (k, self.k_nat), (v, self.v_nat)):
+            self._to_seq(src, dst)
+        self._q = self._heads(self.q_nat, at.hq).detach().requires_grad_()
+        self._k = self._heads(self.k_nat, at.hkv).detach().requires_grad_()
+        self._v = self._heads(self.v_nat, at.hkv).detach().requires_grad_()
+        with torch.enable_grad():
+            self._a = Fn.scaled_dot_product_attention(self._q, self._k, self._v, is_causal=True,
+                                                      enable_gqa=at.hq != at.hkv)
+        a_nat = self._a.detach().transpose(1, 2).reshape(self.T, at.Dq)
+        self._to_cf(a_nat.contiguous(), self.a_cf)
+        o = at.forward_o(self.a_cf)
+        # x2 = x + o (the residual stream) and h2 = RMSNorm(x2) in one pass
+        B.sl_rmsnorm_fwd(o, self.g2, self.eps, self.h2, self.rstd2, res=x, sum_out=self.x2)
+        f = self.ffn.forward(self.h2)
+        B.sl_add_rows(self.x2, f, self.y)
+        self.x = x
+        return self.y
+
+    def backward(self, dy):
+        at = self.attn
+        dh2 = self.ffn.backward(dy)
+        B.sl_rmsnorm_bwd(dh2, self.x2, self.g2, self.rstd2, self.dx2, dres=dy)
+        da_cf = at.backward_o(self.dx2)
+        self._to_seq(da_cf, self.da_nat)
+        dq, dk, dv = torch.autograd.grad(self._a, (self._q, self._k, self._v),
+                                         self._heads(self.da_nat, at.hq))
+        for g, n_h, dst in ((dq, at.hq, self.dq_cf), (dk, at.hkv, self.dk_cf), (dv, at.hkv, self.dv_cf)):
+            self._to_cf(g.transpose(1, 2).reshape(self.T, n_h * at.hd).contiguous(), dst)
+        dh1 = at.backward_qkv(self.dq_cf, self.dk_cf, self.dv_cf)
+        B.sl_rmsnorm_bwd(dh1, self.x, self.g1, self.rstd1, self.dx, dres=self.dx2)
+        return self.dx
+
+    def step(self, x, dy):
+        self.forward(x)
+        return self.backward(dy)

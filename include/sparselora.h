@@ -241,6 +241,24 @@ SL_API sl_status sl_wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int
                                  const void* const* w, int64_t d_out, int64_t ldw, float* scores,
                                  sl_workspace* ws, sl_stream stream);
 
+/* Decoder-layer pieces around the sparse projections ([WT] "Putting It All Together": the
+ * projections sit in a LLaMA decoder layer; RMSNorm with a frozen gain). All bf16 rows
+ * [n_rows, d] (ld elements, 16-byte aligned, ld % 8 == 0, d % 8 == 0), fp32 arithmetic.
+ * sl_rmsnorm_fwd: s = x (+ res when res is given, written to sum_out as the new residual
+ *   stream, rounded to bf16); rstd[row] = 1 / sqrt(mean_j s_j^2 + eps); y = s * rstd * gamma.
+ * sl_rmsnorm_bwd: dx = rstd * gamma * dy - s * rstd^3 * (sum_j s_j gamma_j dy_j) / d
+ *   (+ dres when given: the gradient arriving through the residual connection); x is the
+ *   normalised input s of the forward.
+ * sl_add_rows: out = a + b. */
+SL_API sl_status sl_rmsnorm_fwd(const void* x, int64_t ldx, const void* res, int64_t ldr, void* sum_out,
+                                int64_t lds, const void* gamma, float eps, void* y, int64_t ldy, float* rstd,
+                                int64_t n_rows, int64_t d, sl_stream stream);
+SL_API sl_status sl_rmsnorm_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx, const void* gamma,
+                                const float* rstd, const void* dres, int64_t ldr, void* dx, int64_t lddx,
+                                int64_t n_rows, int64_t d, sl_stream stream);
+SL_API sl_status sl_add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, int64_t ldo,
+                             int64_t n_rows, int64_t d, sl_stream stream);
+
 /* a6: the dense LoRA branch ([WT] Algorithm 1 "computed densely and added"; section 3.2:
  * LoRA gradients are always dense).
  * SL_LORA_FWD: for n_ad adapters sharing the input x [n_tok, d_in] (ld ldx), with

@@ -52,6 +52,13 @@ Readings where the pages are silent or ambiguous (each is listed in the design doc):
       frozen weight, over every projection that shares the index set (gate and up), with the
       feature norms over the context rows of the layer input.
 
+  R16 The decoder layer around the projections (NEXT-1): LLaMA's pre-norm layer with RMSNorm
+      (frozen gain), causal grouped-query attention without a positional encoding (the pages
+      do not say how rotary embeddings meet channel sparsity), residual connections; the
+      selections read the normalised layer inputs.
+  R17 In the layer, output rows attend to context keys and values computed with the sparse
+      projections, as the per-layer split implies (R12).
+
 Parity unpinned (no printed value or closed form pins them):
 the GQA aggregation of R5 and the V-space reading of R4.
 """
@@ -340,6 +347,123 @@ def attn_select(X, ctx, q_f, k_f, v_f, n_q_heads, n_kv_heads, head_dim, ratio):
     return dict(s_qk=s_qk, s_v=s_v, units_qk=u_qk, units_v=u_v,
                 idx_q=expand_units(u_qk, n_q_heads, n_kv_heads, head_dim), idx_k=u_qk,
                 idx_v=u_v, idx_o=expand_units(u_v, n_q_heads, n_kv_heads, head_dim))
+
+
+# ---------------------------------------------------------------------------
+# The decoder layer around the sparse projections (NEXT-1): RMSNorm, causal GQA attention,
+# residual connections  [WT "Putting It All Together"; R16, R17]
+# ---------------------------------------------------------------------------
+
+def rmsnorm(X, gamma, eps):
+    """y = x / sqrt(mean_j x_j^2 + eps) * gamma, per row (LLaMA's RMSNorm, frozen gain)."""
+    X = f64(X)
+    r = 1.0 / np.sqrt(np.mean(X * X, axis=1, keepdims=True) + eps)
+    return X * r * f64(gamma)[None, :]
+
+
+def rmsnorm_bwd(dY, X, gamma, eps):
+    """dX of rmsnorm for the upstream gradient dY (the gain is frozen)."""
+    X, dY, g = f64(X), f64(dY), f64(gamma)[None, :]
+    d = X.shape[1]
+    r = 1.0 / np.sqrt(np.mean(X * X, axis=1, keepdims=True) + eps)
+    gd = g * dY
+    return r * gd - X * r ** 3 * np.sum(X * gd, axis=1, keepdims=True) / d
+
+
+def attention(Q, K, V, n_seq, n_q_heads, n_kv_heads, head_dim):
+    """Causal scaled dot-product attention per sequence (rows sequence-major, n_seq sequences
+    of equal length), grouped-query: query head h reads KV head h // (n_q_heads // n_kv_heads).
+    Returns (O, P) with P the attention probabilities [n_seq, n_q_heads, S, S]."""
+    Q, K, V = f64(Q), f64(K), f64(V)
+    T = Q.shape[0]
+    S = T // n_seq
+    hpg = n_q_heads // n_kv_heads
+    O = np.zeros((T, n_q_heads * head_dim))
+    P = np.zeros((n_seq, n_q_heads, S, S))
+    mask = np.tril(np.ones((S, S), dtype=bool))
+    for b in range(n_seq):
+        rows = slice(b * S, (b + 1) * S)
+        for h in range(n_q_heads):
+            g = h // hpg
+            q = Q[rows, h * head_dim:(h + 1) * head_dim]
+            k = K[rows, g * head_dim:(g + 1) * head_dim]
+            v = V[rows, g * head_dim:(g + 1) * head_dim]
+            sc = q @ k.T / math.sqrt(head_dim)
+            sc = np.where(mask, sc, -np.inf)
+            sc = sc - sc.max(axis=1, keepdims=True)
+            e = np.exp(sc)
+            p = e / e.sum(axis=1, keepdims=True)
+            P[b, h] = p
+            O[rows, h * head_dim:(h + 1) * head_dim] = p @ v
+    return O, P
+
+
+def attention_bwd(dO, Q, K, V, P, n_seq, n_q_heads, n_kv_heads, head_dim):
+    """Gradients of attention() for the upstream gradient dO (softmax backward
+    dS = P * (dP - rowsum(dP * P)))."""
+    dO, Q, K, V = f64(dO), f64(Q), f64(K), f64(V)
+    T = Q.shape[0]
+    S = T // n_seq
+    hpg = n_q_heads // n_kv_heads
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for b in range(n_seq):
+        rows = slice(b * S, (b + 1) * S)
+        for h in range(n_q_heads):
+            g = h // hpg
+            qs, ks = slice(h * head_dim, (h + 1) * head_dim), slice(g * head_dim, (g + 1) * head_dim)
+            p = P[b, h]
+            do = dO[rows, qs]
+            dV[rows, ks] += p.T @ do
+            dp = do @ V[rows, ks].T
+            ds = p * (dp - np.sum(dp * p, axis=1, keepdims=True))
+            dQ[rows, qs] = ds @ K[rows, ks] / math.sqrt(head_dim)
+            dK[rows, ks] += ds.T @ Q[rows, qs] / math.sqrt(head_dim)
+    return dQ, dK, dV
+
+
+def decoder_layer(X, dY, ctx, n_seq, w, lora, gammas, eps, scale, heads, ratio, est_k_factors=None, idx=None):
+    """One decoder layer around the sparse projections, forward and backward:
+      h1 = rmsnorm(X, g1); q, k, v = sparse projections of h1 (QK / V criteria on h1's context
+      rows); O = attention(q, k, v); x2 = X + o(O); h2 = rmsnorm(x2, g2); Y = x2 + FFN(h2)
+      (SwiGLU criterion on h2's context rows).
+    w: frozen weights {"q","k","v","o","gate","up","down"} (nn.Linear storage); lora: (A, B)
+    per projection; heads = (n_q_heads, n_kv_heads, head_dim); est_k_factors: (W_A, W_B) per
+    estimated projection (q, k, v, gate, up) for the selection, or idx: fixed index sets
+    {"q","k","v","o","ffn"} (e.g. the ones a GPU run chose). Returns the forward values, the
+    index sets, dX and every LoRA gradient."""
+    hq, hkv, hd = heads
+    X = f64(X)
+    H1 = rmsnorm(X, gammas[0], eps)
+    if idx is None:
+        sel = attn_select(H1, ctx, est_k_factors["q"], est_k_factors["k"], est_k_factors["v"], hq, hkv, hd, ratio)
+        idx = {"q": sel["idx_q"], "k": sel["idx_k"], "v": sel["idx_v"], "o": sel["idx_o"]}
+    Qm = sparse_linear_fwd(H1, w["q"], *lora["q"], scale, ctx, idx["q"], "out")
+    Km = sparse_linear_fwd(H1, w["k"], *lora["k"], scale, ctx, idx["k"], "out")
+    Vm = sparse_linear_fwd(H1, w["v"], *lora["v"], scale, ctx, idx["v"], "out")
+    O, P = attention(Qm, Km, Vm, n_seq, hq, hkv, hd)
+    Om = sparse_linear_fwd(O, w["o"], *lora["o"], scale, ctx, idx["o"], "in")
+    X2 = X + Om
+    H2 = rmsnorm(X2, gammas[1], eps)
+    if "ffn" not in idx:
+        _, idx["ffn"] = ffn_select(H2, ctx, est_k_factors["gate"], est_k_factors["up"], ratio)
+    fwd_f = ffn_fwd(H2, ctx, w["gate"], w["up"], w["down"], lora["gate"], lora["up"], lora["down"], scale, idx["ffn"])
+    Y = X2 + fwd_f["Y"]
+    # backward
+    dY = f64(dY)
+    bf = ffn_bwd(H2, dY, ctx, w["gate"], w["up"], w["down"], lora["gate"], lora["up"], lora["down"], scale,
+                 idx["ffn"], fwd=fwd_f)
+    dX2 = dY + rmsnorm_bwd(bf["dX"], X2, gammas[1], eps)
+    dO, dA_o, dB_o = sparse_linear_bwd(O, dX2, w["o"], *lora["o"], scale, ctx, idx["o"], "in")
+    dQ, dK, dV = attention_bwd(dO, Qm, Km, Vm, P, n_seq, hq, hkv, hd)
+    grads = {"dA_o": dA_o, "dB_o": dB_o, "dA_gate": bf["dA_g"], "dB_gate": bf["dB_g"], "dA_up": bf["dA_u"],
+             "dB_up": bf["dB_u"], "dA_down": bf["dA_d"], "dB_down": bf["dB_d"]}
+    dH1 = np.zeros_like(H1)
+    for n, dm in (("q", dQ), ("k", dK), ("v", dV)):
+        dx, da, db = sparse_linear_bwd(H1, dm, w[n], *lora[n], scale, ctx, idx[n], "out")
+        dH1 += dx
+        grads["dA_" + n], grads["dB_" + n] = da, db
+    dX = dX2 + rmsnorm_bwd(dH1, X, gammas[0], eps)
+    return dict(Y=Y, dX=dX, H1=H1, H2=H2, X2=X2, O=O, Q=Qm, K=Km, V=Vm, idx=idx, **grads)
 
 
 def dense_lora_reference(X, dY, W, A, B, scale):

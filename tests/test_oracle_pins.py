@@ -455,3 +455,126 @@ def test_select_heads_special_cases():
     s = np.array([10.0, 0.0, 0.0, 0.0, 3.0, 3.0, 3.0, 3.0])
     np.testing.assert_array_equal(oracle.select_heads(s, 2, 4, 1), np.arange(4, 8))
     np.testing.assert_array_equal(oracle.select_top(s, 4), np.array([0, 4, 5, 6]))
+
+
+# ----------------------------------------------------------------------- decoder layer (NEXT-1)
+
+def test_rmsnorm_closed_forms():
+    g = np.array([1.0, 2.0, -0.5, 3.0])
+    # a constant row c: mean(x^2) = c^2, so y = c / sqrt(c^2 + eps) * gamma
+    c, eps = 2.5, 1e-6
+    np.testing.assert_allclose(oracle.rmsnorm(np.full((1, 4), c), g, eps)[0], c / np.sqrt(c * c + eps) * g,
+                               rtol=1e-14)
+    # eps = 0: invariant to scaling the row
+    rng = np.random.default_rng(51)
+    X = rng.standard_normal((3, 4))
+    np.testing.assert_allclose(oracle.rmsnorm(7.0 * X, g, 0.0), oracle.rmsnorm(X, g, 0.0), rtol=1e-13)
+    # rows of +-1: y = x * gamma
+    X = np.array([[1.0, -1.0, 1.0, -1.0]])
+    np.testing.assert_allclose(oracle.rmsnorm(X, g, 0.0), X * g, rtol=1e-15)
+
+
+def test_rmsnorm_backward_matches_finite_differences():
+    rng = np.random.default_rng(52)
+    X, dY, g = rng.standard_normal((3, 6)), rng.standard_normal((3, 6)), rng.standard_normal(6)
+    eps, h = 1e-5, 1e-6
+    num = np.zeros_like(X)
+    for i in range(X.shape[0]):
+        for j in range(X.shape[1]):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[i, j] += h
+            Xm[i, j] -= h
+            num[i, j] = (np.sum(dY * oracle.rmsnorm(Xp, g, eps)) - np.sum(dY * oracle.rmsnorm(Xm, g, eps))) / (2 * h)
+    np.testing.assert_allclose(oracle.rmsnorm_bwd(dY, X, g, eps), num, rtol=1e-7, atol=1e-8)
+
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(53)
+    n_seq, S, hq, hkv, hd = 2, 5, 4, 2, 3
+    T = n_seq * S
+    V = rng.standard_normal((T, hkv * hd))
+    # zero queries: causal uniform weights, O[i] = mean of V over positions 0..i of the sequence
+    O, _ = oracle.attention(np.zeros((T, hq * hd)), rng.standard_normal((T, hkv * hd)), V, n_seq, hq, hkv, hd)
+    for b in range(n_seq):
+        for i in range(S):
+            for h in range(hq):
+                g = h // (hq // hkv)
+                want = V[b * S:b * S + i + 1, g * hd:(g + 1) * hd].mean(axis=0)
+                np.testing.assert_allclose(O[b * S + i, h * hd:(h + 1) * hd], want, rtol=1e-13)
+    # the first token of every sequence attends only to itself
+    Q, K = rng.standard_normal((T, hq * hd)), rng.standard_normal((T, hkv * hd))
+    O, _ = oracle.attention(Q, K, V, n_seq, hq, hkv, hd)
+    for b in range(n_seq):
+        for h in range(hq):
+            g = h // (hq // hkv)
+            np.testing.assert_allclose(O[b * S, h * hd:(h + 1) * hd], V[b * S, g * hd:(g + 1) * hd], rtol=1e-14)
+
+
+def test_attention_backward_matches_finite_differences():
+    rng = np.random.default_rng(54)
+    n_seq, S, hq, hkv, hd = 2, 3, 2, 1, 2
+    T = n_seq * S
+    Q, K, V = (rng.standard_normal((T, n * hd)) for n in (hq, hkv, hkv))
+    dO = rng.standard_normal((T, hq * hd))
+    _, P = oracle.attention(Q, K, V, n_seq, hq, hkv, hd)
+    dQ, dK, dV = oracle.attention_bwd(dO, Q, K, V, P, n_seq, hq, hkv, hd)
+    h = 1e-6
+
+    def loss(Q, K, V):
+        return np.sum(dO * oracle.attention(Q, K, V, n_seq, hq, hkv, hd)[0])
+
+    for M, G, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
+        num = np.zeros_like(M)
+        for i in range(M.shape[0]):
+            for j in range(M.shape[1]):
+                args_p = [Q.copy(), K.copy(), V.copy()]
+                args_m = [Q.copy(), K.copy(), V.copy()]
+                args_p[which][i, j] += h
+                args_m[which][i, j] -= h
+                num[i, j] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(G, num, rtol=1e-6, atol=1e-8)
+
+
+def test_decoder_layer_backward_matches_finite_differences():
+    """dX and two LoRA gradients of the whole layer (fixed index sets, R9) against central
+    differences of the layer's output."""
+    rng = np.random.default_rng(55)
+    n_seq, S, D, hq, hkv, hd, F, r = 2, 3, 8, 2, 1, 4, 12, 2
+    T = n_seq * S
+    Dq, Dkv = hq * hd, hkv * hd
+    shapes = {"q": (Dq, D), "k": (Dkv, D), "v": (Dkv, D), "o": (D, Dq), "gate": (F, D), "up": (F, D), "down": (D, F)}
+    w = {n: 0.3 * rng.standard_normal(s) for n, s in shapes.items()}
+    lora = {n: (0.3 * rng.standard_normal((r, s[1])), 0.3 * rng.standard_normal((s[0], r))) for n, s in shapes.items()}
+    gammas = (1.0 + 0.1 * rng.standard_normal(D), 1.0 + 0.1 * rng.standard_normal(D))
+    ctx = np.tile(np.array([True, True, False]), n_seq)
+    idx = {"q": np.array([0, 1, 4, 5]), "k": np.array([0, 1]), "v": np.array([1, 3]), "o": np.array([1, 3, 5, 7]),
+           "ffn": np.array([0, 2, 3, 7, 8, 11])}
+    X, dY = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+    res = oracle.decoder_layer(X, dY, ctx, n_seq, w, lora, gammas, 1e-5, 2.0, (hq, hkv, hd), 0.5, idx=dict(idx))
+
+    def loss(X, lora):
+        out = oracle.decoder_layer(X, np.zeros_like(dY), ctx, n_seq, w, lora, gammas, 1e-5, 2.0, (hq, hkv, hd), 0.5,
+                                   idx=dict(idx))
+        return np.sum(dY * out["Y"])
+
+    h = 1e-6
+    num = np.zeros_like(X)
+    for i in range(T):
+        for j in range(D):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[i, j] += h
+            Xm[i, j] -= h
+            num[i, j] = (loss(Xp, lora) - loss(Xm, lora)) / (2 * h)
+    np.testing.assert_allclose(res["dX"], num, rtol=1e-5, atol=1e-7)
+    for name, which in (("q", 0), ("down", 1)):
+        M = lora[name][which]
+        G = res[("dA_" if which == 0 else "dB_") + name]
+        numg = np.zeros_like(M)
+        for i in range(M.shape[0]):
+            for j in range(M.shape[1]):
+                lp = {k: (a.copy(), b.copy()) for k, (a, b) in lora.items()}
+                lm = {k: (a.copy(), b.copy()) for k, (a, b) in lora.items()}
+                lp[name][which][i, j] += h
+                lm[name][which][i, j] -= h
+                numg[i, j] = (loss(X, lp) - loss(X, lm)) / (2 * h)
+        np.testing.assert_allclose(G, numg, rtol=1e-5, atol=1e-7)
