@@ -30,7 +30,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
-            "sl_add_rows")
+            "sl_add_rows", "sl_adamw_step")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -85,6 +85,7 @@ def lib():
         L.sl_rmsnorm_fwd.argtypes = [P, c_int64, P, c_int64, P, c_int64, P, c_float, P, c_int64, P, c_int64, c_int64, P]
         L.sl_rmsnorm_bwd.argtypes = [P, c_int64, P, c_int64, P, P, P, c_int64, P, c_int64, c_int64, c_int64, P]
         L.sl_add_rows.argtypes = [P, c_int64, P, c_int64, P, c_int64, c_int64, c_int64, P]
+        L.sl_adamw_step.argtypes = [P, P, P, P, P, c_int64, c_float, c_float, c_float, c_float, c_float, c_int32, P]
         L.sl_wanda_scores.argtypes = [P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p), c_int64, c_int64, P,
                                       POINTER(SlWorkspaceC), P]
         L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
@@ -274,6 +275,13 @@ def sl_rmsnorm_bwd(dy, x, gamma, rstd, dx, dres=None):
 def sl_add_rows(a, b, out):
     _check("sl_add_rows", lib().sl_add_rows(_ptr(a), a.stride(0), _ptr(b), b.stride(0), _ptr(out), out.stride(0),
                                             a.shape[0], a.shape[1], _stream()))
+
+
+def sl_adamw_step(params, grads, m, v, step, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+                  params_bf16=None):
+    _check("sl_adamw_step", lib().sl_adamw_step(_ptr(params), _ptr(grads), _ptr(m), _ptr(v), _ptr(params_bf16),
+                                                params.numel(), float(lr), float(beta1), float(beta2), float(eps),
+                                                float(weight_decay), int(step), _stream()))
 
 
 def sl_lora_fwd_bwd(ws: Workspace, mode, lins, x, n_ctx, xa_s, xa=None, in_layout=SL_LAYOUT_NATURAL, in_ch=None,

@@ -66,10 +66,12 @@ class DataParallel:
 
 
 class _GradBuffer:
-    """One flat fp32 buffer holding a block's LoRA gradients, so that a single collective sums
-    them over ranks; views start on 64-element boundaries (16-byte alignment and more)."""
+    """One flat buffer holding a block's LoRA matrices (gradients in fp32, or the parameters'
+    bf16 working copy with initial values), so that one collective or one optimiser launch
+    covers them all; views start on 64-element boundaries (16-byte alignment and more), and the
+    gradient and parameter buffers of a block share the layout."""
 
-    def __init__(self, shapes, device):
+    def __init__(self, shapes, device, dtype=torch.float32, init=None):
         self.offsets, n = [], 0
         for sh in shapes:
             self.offsets.append(n)
@@ -77,8 +79,11 @@ class _GradBuffer:
             for d in sh:
                 cnt *= d
             n += (cnt + 63) // 64 * 64
-        self.flat = torch.zeros(n, dtype=torch.float32, device=device)
+        self.flat = torch.zeros(n, dtype=dtype, device=device)
         self.views = [self.flat[o:o + sh[0] * sh[1]].view(*sh) for o, sh in zip(self.offsets, shapes)]
+        if init is not None:
+            for v, t in zip(self.views, init):
+                v.copy_(t.to(device=device, dtype=dtype))
 
 
 class FFNBlock:
@@ -112,9 +117,12 @@ class FFNBlock:
         self.est_dtype = torch.float32 if gate.W_A.dtype == torch.float32 else bf
         ed = lambda t: t.to(device=device, dtype=self.est_dtype).contiguous()
         self.WAg, self.WBg, self.WAu, self.WBu = ed(gate.W_A), ed(gate.W_B), ed(up.W_A), ed(up.W_B)
-        self.Ag, self.Bg = dev(lora_gate[0]), dev(lora_gate[1])
-        self.Au, self.Bu = dev(lora_up[0]), dev(lora_up[1])
-        self.Ad, self.Bd = dev(lora_down[0]), dev(lora_down[1])
+        r_, D_, F_ = lora_gate[0].shape[0], gate.W.shape[1], gate.W.shape[0]
+        # LoRA matrices in the order and layout of the gradient buffer (A_d, B_d, A_g, B_g, A_u, B_u)
+        self.params = _GradBuffer([(r_, F_), (D_, r_), (r_, D_), (F_, r_), (r_, D_), (F_, r_)], device, torch.bfloat16,
+                                  init=[lora_down[0], lora_down[1], lora_gate[0], lora_gate[1], lora_up[0],
+                                        lora_up[1]])
+        self.Ad, self.Bd, self.Ag, self.Bg, self.Au, self.Bu = self.params.views
         self.r = self.Ag.shape[0]
         self.scale = float(lora_scale)
         self.Wd_t = _empty((self.F, self.D), bf, device)
@@ -150,10 +158,21 @@ class FFNBlock:
 
     def _descs(self):
         s = self.scale
-        self.lin_g = B.linear_desc(self.Wg, self.Ag, self.Bg, s, B.SL_SLICE_OUT, w_kept=self.Wg_k)
-        self.lin_u = B.linear_desc(self.Wu, self.Au, self.Bu, s, B.SL_SLICE_OUT, w_kept=self.Wu_k)
-        self.lin_d = B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t, w_kept=self.Wd_k)
-        self.ch = B.channels_desc(self.sigma, self.n_keep)
+        lin = lambda wk_g, wk_u, wk_d: (
+            B.linear_desc(self.Wg, self.Ag, self.Bg, s, B.SL_SLICE_OUT, w_kept=wk_g),
+            B.linear_desc(self.Wu, self.Au, self.Bu, s, B.SL_SLICE_OUT, w_kept=wk_u),
+            B.linear_desc(self.Wd, self.Ad, self.Bd, s, B.SL_SLICE_IN, w_t=self.Wd_t, w_kept=wk_d))
+        self._sparse = lin(self.Wg_k, self.Wu_k, self.Wd_k) + (B.channels_desc(self.sigma, self.n_keep),)
+        self._sigma_id = torch.arange(self.F, dtype=torch.int32, device=self.device)
+        self._dense = lin(self.Wg, self.Wu, self.Wd_t) + (B.channels_desc(self._sigma_id, self.F),)
+        self._always_dense = self.dense
+        self.lin_g, self.lin_u, self.lin_d, self.ch = self._dense if self.dense else self._sparse
+
+    def set_dense(self, on: bool):
+        """Run the next steps densely (the progressive schedule's first steps, [WT] "Step
+        Sensitivity and Progressive Sparse Fine-Tuning") or back with the block's keep ratio."""
+        self.dense = bool(on) or self._always_dense
+        self.lin_g, self.lin_u, self.lin_d, self.ch = self._dense if self.dense else self._sparse
 
     def estimate(self, x):
         """a1 + a2: SwiGLU-L2 scores of the estimated gate/up outputs on x's context rows (or
@@ -298,7 +317,11 @@ class AttnProjBlock:
         self.Wq, self.Wk, self.Wv, self.Wo = dev(q.W), dev(k.W), dev(v.W), dev(o.W)
         self.WA = [dev(q.W_A), dev(k.W_A), dev(v.W_A)]
         self.WB = [dev(q.W_B), dev(k.W_B), dev(v.W_B)]
-        self.L = {n: (dev(a), dev(b)) for n, (a, b) in zip("qkvo", (lora_q, lora_k, lora_v, lora_o))}
+        loras = dict(zip("qkvo", (lora_q, lora_k, lora_v, lora_o)))
+        # LoRA matrices in the order and layout of the gradient buffer (A_q..A_o, then B_q..B_o)
+        self.params = _GradBuffer([tuple(loras[n][0].shape) for n in "qkvo"] + [tuple(loras[n][1].shape) for n in "qkvo"],
+                                  device, torch.bfloat16, init=[loras[n][0] for n in "qkvo"] + [loras[n][1] for n in "qkvo"])
+        self.L = {n: (self.params.views[i], self.params.views[4 + i]) for i, n in enumerate("qkvo")}
         self.r = self.L["q"][0].shape[0]
         self.scale = float(lora_scale)
         self.Wo_t = _empty((self.Dq, self.D), bf, device)
@@ -337,18 +360,25 @@ class AttnProjBlock:
         else:
             self.W_k = {"q": _empty((nq, D), bf, device), "k": _empty((nu, D), bf, device),
                         "v": _empty((nv, D), bf, device), "o": _empty((no, D), bf, device)}
-        self.lin = {
-            "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT, w_kept=self.W_k["q"]),
-            "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT, w_kept=self.W_k["k"]),
-            "v": B.linear_desc(self.Wv, *self.L["v"], s, B.SL_SLICE_OUT, w_kept=self.W_k["v"]),
-            "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t, w_kept=self.W_k["o"]),
+        lin = lambda wk: {
+            "q": B.linear_desc(self.Wq, *self.L["q"], s, B.SL_SLICE_OUT, w_kept=wk["q"]),
+            "k": B.linear_desc(self.Wk, *self.L["k"], s, B.SL_SLICE_OUT, w_kept=wk["k"]),
+            "v": B.linear_desc(self.Wv, *self.L["v"], s, B.SL_SLICE_OUT, w_kept=wk["v"]),
+            "o": B.linear_desc(self.Wo, *self.L["o"], s, B.SL_SLICE_IN, w_t=self.Wo_t, w_kept=wk["o"]),
         }
-        self.ch = {
+        self._lin_sparse = lin(self.W_k)
+        self._ch_sparse = {
             "q": B.channels_desc(self.sig_q, self.n_keep_qk * self.hpg),
             "k": B.channels_desc(self.sig_k, self.n_keep_qk),
             "v": B.channels_desc(self.sig_v, self.n_keep_vo),
             "o": B.channels_desc(self.sig_o, self.n_keep_vo * self.hpg),
         }
+        self._ids = {"q": ar(self.Dq), "kv": ar(self.Dkv)}
+        self._lin_dense = lin({"q": self.Wq, "k": self.Wk, "v": self.Wv, "o": self.Wo_t})
+        self._ch_dense = {"q": B.channels_desc(self._ids["q"], self.Dq), "k": B.channels_desc(self._ids["kv"], self.Dkv),
+                          "v": B.channels_desc(self._ids["kv"], self.Dkv), "o": B.channels_desc(self._ids["q"], self.Dq)}
+        self._always_dense = self.dense
+        self.lin, self.ch = (self._lin_dense, self._ch_dense) if self.dense else (self._lin_sparse, self._ch_sparse)
 
     def estimate(self, x):
         """a1 + a2: QK scores over KV units and V scores from one pass over x's context rows
@@ -381,6 +411,12 @@ class AttnProjBlock:
 
     def _select_vo(self):
         B.sl_select_channels(self.s_v, self.n_keep_vo, self.sig_v, self.hpg, self.hd, self.sig_o)
+
+    def set_dense(self, on: bool):
+        """Run the next steps densely (the progressive schedule's first steps) or back with the
+        block's keep ratios."""
+        self.dense = bool(on) or self._always_dense
+        self.lin, self.ch = (self._lin_dense, self._ch_dense) if self.dense else (self._lin_sparse, self._ch_sparse)
 
     def _qk_chain(self):
         self._select_qk()

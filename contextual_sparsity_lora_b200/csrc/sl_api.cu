@@ -448,6 +448,15 @@ sl_status sl_add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, vo
   return from_kernel(add_rows(a, lda, b, ldb, out, ldo, n_rows, d, cs(stream)));
 }
 
+sl_status sl_adamw_step(float* params, const float* grads, float* m, float* v, void* params_bf16, int64_t n, float lr,
+                        float beta1, float beta2, float eps, float weight_decay, int32_t step, sl_stream stream) {
+  if (!params || !grads || !m || !v) return SL_ERR_INVALID_ARG;
+  if (n < 1 || step < 1 || !(lr >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+    return SL_ERR_SHAPE;
+  return from_kernel(adamw_step(params, grads, m, v, params_bf16, n, lr, beta1, beta2, eps, weight_decay, step,
+                                cs(stream)));
+}
+
 // ------------------------------------------------------------------ a6
 sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx,
                           int64_t n_tok, int64_t n_ctx, int32_t in_layout, const sl_channels* in_ch, float* xa,

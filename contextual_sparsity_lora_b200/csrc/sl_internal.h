@@ -162,6 +162,8 @@ int rmsnorm_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx, const 
                 const void* dres, int64_t ldr, void* dx, int64_t lddx, int64_t n_rows, int64_t d, cudaStream_t s);
 int add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, int64_t ldo, int64_t n_rows, int64_t d,
              cudaStream_t s);
+int adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, float lr, float b1, float b2,
+               float eps, float wd, int step, cudaStream_t s);
 
 // ---- criterion variants (sl_criteria.cu)
 // Wanda-style channel scores s_i = sum_p sum_j |W_p[i, j]| ||x[:, j]||_2 over n_ctx rows of x

@@ -4,6 +4,9 @@
 // a frozen gamma). One warp per row; fp32 arithmetic on bf16 rows, 16-byte vectors.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <cmath>
+
 #include "sl_internal.h"
 
 namespace sl {
@@ -168,6 +171,49 @@ int add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, 
   launch_kernel(add_rows_kernel, grid, kNormWarps * 32, 0, s, static_cast<const __nv_bfloat16*>(a), lda,
                 static_cast<const __nv_bfloat16*>(b), ldb, static_cast<__nv_bfloat16*>(out), ldo, n_rows, (int)d);
   if (launch_failed("sl_add")) return 5;
+  note_launch();
+  return 0;
+}
+
+}  // namespace sl
+
+// ---- AdamW on the LoRA parameters (the optimiser of a fine-tuning step)
+
+namespace sl {
+
+namespace {
+
+// Decoupled weight decay (AdamW): p -= lr * wd * p; m = b1 m + (1 - b1) g; v = b2 v + (1 - b2) g^2;
+// p -= lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps); the bf16 working copy gets p.
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                                    float* __restrict__ m, float* __restrict__ v,
+                                                    __nv_bfloat16* __restrict__ p_bf16, int64_t n, float lr, float b1,
+                                                    float b2, float eps, float wd, float c1, float c2) {
+  pdl_wait();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float pi = p[i];
+    const float gi = g[i];
+    pi -= lr * wd * pi;
+    const float mi = b1 * m[i] + (1.f - b1) * gi;
+    const float vi = b2 * v[i] + (1.f - b2) * gi * gi;
+    m[i] = mi;
+    v[i] = vi;
+    pi -= lr * (mi / c1) / (sqrtf(vi / c2) + eps);
+    p[i] = pi;
+    if (p_bf16) p_bf16[i] = __float2bfloat16_rn(pi);
+  }
+}
+
+}  // namespace
+
+int adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, float lr, float b1, float b2,
+               float eps, float wd, int step, cudaStream_t s) {
+  if (n < 1 || step < 1) return 1;
+  const float c1 = 1.f - powf(b1, (float)step), c2 = 1.f - powf(b2, (float)step);
+  const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 1184);
+  launch_kernel(adamw_kernel, grid, 256, 0, s, p, g, m, v, static_cast<__nv_bfloat16*>(p_bf16), n, lr, b1, b2, eps, wd,
+                c1, c2);
+  if (launch_failed("sl_adamw")) return 5;
   note_launch();
   return 0;
 }

@@ -259,6 +259,15 @@ SL_API sl_status sl_rmsnorm_bwd(const void* dy, int64_t lddy, const void* x, int
 SL_API sl_status sl_add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, int64_t ldo,
                              int64_t n_rows, int64_t d, sl_stream stream);
 
+/* AdamW step over n fp32 parameters (the LoRA matrices of a fine-tuning step; [WT] §3.2: only
+ * the adapters train): decoupled decay p -= lr * weight_decay * p; m = beta1 m + (1 - beta1) g;
+ * v = beta2 v + (1 - beta2) g^2; p -= lr * m_hat / (sqrt(v_hat) + eps) with the bias corrections
+ * m_hat = m / (1 - beta1^step), v_hat = v / (1 - beta2^step), step >= 1. params_bf16
+ * (optional) receives the updated parameters rounded to bf16 (the working copy the kernels read). */
+SL_API sl_status sl_adamw_step(float* params, const float* grads, float* m, float* v, void* params_bf16, int64_t n,
+                               float lr, float beta1, float beta2, float eps, float weight_decay, int32_t step,
+                               sl_stream stream);
+
 /* a6: the dense LoRA branch ([WT] Algorithm 1 "computed densely and added"; section 3.2:
  * LoRA gradients are always dense).
  * SL_LORA_FWD: for n_ad adapters sharing the input x [n_tok, d_in] (ld ldx), with

@@ -466,6 +466,52 @@ def decoder_layer(X, dY, ctx, n_seq, w, lora, gammas, eps, scale, heads, ratio, 
     return dict(Y=Y, dX=dX, H1=H1, H2=H2, X2=X2, O=O, Q=Qm, K=Km, V=Vm, idx=idx, **grads)
 
 
+def model_step(ids, targets_out, ctx, n_seq, embed, lm_head, gamma_f, layers, eps, scale, heads):
+    """Loss and LoRA gradients of a stack of decoder layers (NEXT-2): X_0 = embed[ids]; each
+    layer as decoder_layer with its index sets; H = rmsnorm(X_L, gamma_f); cross-entropy of
+    H W_lm^T against targets_out on the output rows (mean over them); backward through every
+    layer. layers: list of dicts w, lora, gammas, idx. Rows in sequence order; targets_out in
+    the order of the output rows. Returns (loss, per-layer gradient dicts)."""
+    X = f64(embed)[np.asarray(ids)]
+    xs = []
+    for L in layers:
+        xs.append(X)
+        X = decoder_layer(X, np.zeros_like(X), ctx, n_seq, L["w"], L["lora"], L["gammas"], eps, scale, heads, 0.0,
+                          idx=dict(L["idx"]))["Y"]
+    H = rmsnorm(X, gamma_f, eps)
+    out = ~np.asarray(ctx, dtype=bool)
+    logits = H[out] @ f64(lm_head).T
+    m = logits.max(axis=1, keepdims=True)
+    lse = (m + np.log(np.exp(logits - m).sum(axis=1, keepdims=True)))[:, 0]
+    t = np.asarray(targets_out)
+    loss = float(np.mean(lse - logits[np.arange(len(t)), t]))
+    p = np.exp(logits - lse[:, None])
+    p[np.arange(len(t)), t] -= 1.0
+    p /= len(t)
+    dH = np.zeros_like(H)
+    dH[out] = p @ f64(lm_head)
+    dX = rmsnorm_bwd(dH, X, gamma_f, eps)
+    grads = [None] * len(layers)
+    for l in range(len(layers) - 1, -1, -1):
+        L = layers[l]
+        res = decoder_layer(xs[l], dX, ctx, n_seq, L["w"], L["lora"], L["gammas"], eps, scale, heads, 0.0,
+                            idx=dict(L["idx"]))
+        grads[l] = res
+        dX = res["dX"]
+    return loss, grads
+
+
+def adamw(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
+    """One AdamW update (decoupled weight decay, bias-corrected moments); returns (p, m, v)."""
+    p, g, m, v = f64(p), f64(g), f64(m), f64(v)
+    p = p - lr * weight_decay * p
+    m = beta1 * m + (1 - beta1) * g
+    v = beta2 * v + (1 - beta2) * g * g
+    mh = m / (1 - beta1 ** step)
+    vh = v / (1 - beta2 ** step)
+    return p - lr * mh / (np.sqrt(vh) + eps), m, v
+
+
 def dense_lora_reference(X, dY, W, A, B, scale):
     """Dense LoRA layer (keep ratio 1): y = x W + scale (x A^T) B^T and its backward."""
     X = f64(X)

@@ -578,3 +578,50 @@ def test_decoder_layer_backward_matches_finite_differences():
                 lm[name][which][i, j] -= h
                 numg[i, j] = (loss(X, lp) - loss(X, lm)) / (2 * h)
         np.testing.assert_allclose(G, numg, rtol=1e-5, atol=1e-7)
+
+
+def test_adamw_closed_forms():
+    # first step, no decay: m_hat = g, v_hat = g^2, so p moves by -lr * g / (|g| + eps)
+    p, g = np.array([1.0, -2.0, 0.5]), np.array([0.3, -4.0, 0.0])
+    q, m, v = oracle.adamw(p, g, np.zeros(3), np.zeros(3), 1, 0.1, 0.9, 0.999, 1e-8, 0.0)
+    np.testing.assert_allclose(q, p - 0.1 * g / (np.abs(g) + 1e-8), rtol=1e-12)
+    np.testing.assert_allclose(m, 0.1 * g, rtol=1e-15)
+    # zero gradient, decay only
+    q, _, _ = oracle.adamw(p, np.zeros(3), np.zeros(3), np.zeros(3), 3, 0.01, 0.9, 0.999, 1e-8, 0.1)
+    np.testing.assert_allclose(q, p * (1 - 0.01 * 0.1), rtol=1e-15)
+
+
+def test_model_step_one_layer_equals_layer_and_loss_gradient():
+    """A one-layer stack: the loss gradient reaching the layer is the cross-entropy gradient through
+    the final RMSNorm, checked by central differences of the loss in the layer's output."""
+    rng = np.random.default_rng(56)
+    n_seq, S, D, hq, hkv, hd, F, r, V = 1, 4, 8, 2, 1, 4, 12, 2, 11
+    T = n_seq * S
+    shapes = {"q": (hq * hd, D), "k": (hkv * hd, D), "v": (hkv * hd, D), "o": (D, hq * hd), "gate": (F, D),
+              "up": (F, D), "down": (D, F)}
+    w = {n: 0.3 * rng.standard_normal(s) for n, s in shapes.items()}
+    lora = {n: (0.3 * rng.standard_normal((r, s[1])), 0.3 * rng.standard_normal((s[0], r))) for n, s in shapes.items()}
+    gammas = (1.0 + 0.1 * rng.standard_normal(D), 1.0 + 0.1 * rng.standard_normal(D))
+    ctx = np.array([True, True, False, False])
+    idx = {"q": np.arange(8), "k": np.arange(4), "v": np.arange(4), "o": np.arange(8), "ffn": np.arange(12)}
+    embed, lm_head, gf = rng.standard_normal((V, D)), rng.standard_normal((V, D)), 1.0 + 0.1 * rng.standard_normal(D)
+    ids, tgt = rng.integers(0, V, T), rng.integers(0, V, 2)
+    layers = [dict(w=w, lora=lora, gammas=gammas, idx=idx)]
+    loss, grads = oracle.model_step(ids, tgt, ctx, n_seq, embed, lm_head, gf, layers, 1e-5, 2.0, (hq, hkv, hd))
+
+    def loss_of(lo):
+        L = [dict(w=w, lora=lo, gammas=gammas, idx=idx)]
+        return oracle.model_step(ids, tgt, ctx, n_seq, embed, lm_head, gf, L, 1e-5, 2.0, (hq, hkv, hd))[0]
+
+    h = 1e-6
+    for name in ("q", "down"):
+        M = lora[name][1]
+        num = np.zeros_like(M)
+        for i in range(M.shape[0]):
+            for j in range(M.shape[1]):
+                lp = {k: (a.copy(), b.copy()) for k, (a, b) in lora.items()}
+                lm = {k: (a.copy(), b.copy()) for k, (a, b) in lora.items()}
+                lp[name][1][i, j] += h
+                lm[name][1][i, j] -= h
+                num[i, j] = (loss_of(lp) - loss_of(lm)) / (2 * h)
+        np.testing.assert_allclose(grads[0]["dB_" + name], num, rtol=1e-5, atol=1e-8)
