@@ -16,6 +16,7 @@ Multi-GPU (torchrun, one rank per GPU): each rank runs the step on its own batch
 from __future__ import annotations
 
 import argparse
+import math
 import json
 import os
 import subprocess
@@ -47,6 +48,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-LoRA companion measurement")
     ap.add_argument("--no-layer", action="store_true", help="skip the whole-decoder-layer measurement")
+    ap.add_argument("--no-model", action="store_true", help="skip the 32-layer fine-tuning run")
     ap.add_argument("--stages-only", action="store_true",
                     help="time only the selection stages (estimator, criterion, top-n, compaction) of both blocks "
                          "and print them; no step, no headline line")
@@ -364,6 +366,69 @@ def _oracle_layer(oracle, X, XO, dq, dk, dv, dyo, Xf, dyf, ctx, W, F, L, Wf, Ff,
     oracle.ffn_bwd(Xf, dyf, ctx, Wf["gate"], Wf["up"], Wf["down"], Lf["gate"], Lf["up"], Lf["down"], s, idx, fwd=fwd)
 
 
+def model_measure(da, df, perm, C, ac, fc, device, keep, n_steps=20, vocab=128256, peak_lr=1e-4):
+    """A 20-step fine-tuning run of a 32-layer LLaMA3-8B-shaped model: embedding, 32 decoder
+    layers with the per-layer keep table `keep`, final RMSNorm, LM head with cross-entropy on the
+    output rows, backward, AdamW on every LoRA matrix at the cosine schedule's rate; the first
+    10% of the steps dense (progressive schedule). Each layer's frozen projection weights are a
+    random signed permutation of one decaying-spectrum draw per projection (distinct weights of
+    the same spectrum, exact factors); LoRA matrices and RMSNorm gains are per layer. Each
+    mode's forward + backward is one CUDA graph (captured once); AdamW runs per block between
+    replays, all inside the timed region."""
+    from contextual_sparsity_lora_b200.model import SparseLoRAModel, cosine_lr
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(91)
+    D, n_layers = ac.hidden, len(keep)
+    base = {"q": da["q"], "k": da["k"], "v": da["v"], "o": da["o"], "gate": df["gate"], "up": df["up"],
+            "down": df["down"]}
+    frozen = {"layers": [{n: inputs.signed_permutation(w, gen) for n, w in base.items()} for _ in range(n_layers)]}
+    frozen["embed"] = torch.randn(vocab, D, device=device, dtype=torch.bfloat16)
+    frozen["lm_head"] = 0.02 * torch.randn(vocab, D, device=device, dtype=torch.bfloat16)
+    frozen["gamma_f"] = torch.ones(D, dtype=torch.bfloat16)
+    shapes = {n: tuple(w.W.shape) for n, w in base.items()}
+    loras = [{n: inputs.lora_pair(do, di, ac.r, 0.02, gen) for n, (do, di) in shapes.items()} for _ in range(n_layers)]
+    gammas = [(torch.ones(D, dtype=torch.bfloat16), torch.ones(D, dtype=torch.bfloat16)) for _ in range(n_layers)]
+    model = SparseLoRAModel(frozen, loras, gammas, keep, perm.cpu().numpy(), C, ac.batch,
+                            (ac.n_q_heads, ac.n_kv_heads, ac.head_dim), ac.k, ac.lora_scale, device)
+    del frozen
+    T = ac.n_tok
+    ids_cf = torch.randint(0, vocab, (T,), generator=gen).to(torch.int32).to(device)
+    targets = torch.randint(0, vocab, (T - C,), generator=gen).to(device)
+    graphs = {}
+    for dense in (True, False):
+        model.set_dense(dense)
+        for _ in range(2):
+            model.forward_backward(ids_cf, targets)
+        torch.cuda.synchronize()
+        graphs[dense] = capture_graph(lambda: model.forward_backward(ids_cf, targets), warm=False)
+    n_dense = math.ceil(0.1 * n_steps)
+    times, losses = [], []
+    for step in range(1, n_steps + 1):
+        dense = step <= n_dense
+        model.set_dense(dense)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graphs[dense].replay()
+        model.optimizer_step(step, cosine_lr(step, n_steps, peak_lr))
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        losses.append(float(model.loss))
+    total = sum(times)
+    sparse_ms = sum(times[n_dense:]) / (n_steps - n_dense)
+    dense_ms = sum(times[:n_dense]) / n_dense
+    del graphs, model
+    torch.cuda.synchronize()
+    return {"value": n_steps * T / (total / 1e3), "unit": UNIT, "steps": n_steps, "dense_steps": n_dense,
+            "ms_per_sparse_step": sparse_ms, "ms_per_dense_step": dense_ms,
+            "sparse_vs_dense_speedup": dense_ms / sparse_ms, "run_vs_all_dense_speedup": n_steps * dense_ms / total,
+            "loss_first": losses[0], "loss_last": losses[-1], "layers": n_layers, "vocab": vocab,
+            "lr": f"AdamW, cosine schedule, 4% warm-up, peak {peak_lr}",
+            "frozen_weights": "per layer: a random signed permutation of one decaying-spectrum draw per projection",
+            "lm_head_and_cross_entropy": "torch (library)",
+            "attention_core": "torch scaled_dot_product_attention (library)"}
+
+
 def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
     """The whole decoder layer around the same blocks (RMSNorm, sparse q/k/v, causal GQA
     attention core, sparse o, residual, RMSNorm, sparse FFN, residual), forward and backward
@@ -571,6 +636,13 @@ def main():
                               "effective_tflops": d_fl["total"] / (d_ms / args.steps / 1e3) / 1e12}
         line["speedup_vs_dense_lora"] = line["dense_lora"]["ms_per_step"] / ms_step
         del d_attn, d_ffn, d_graph
+    if world == 1 and not args.no_model:
+        from contextual_sparsity_lora_b200.model import layerwise_keep, llama3_8b_math10k_keep
+        line["model_32_layers"] = model_measure(da, df, perm, C, ac, fc, device, layerwise_keep())
+        line["model_32_layers"]["keep_table"] = "layers 0-7 dense, 8-19 keep 0.6, 20-31 keep 0.35 (attention and FFN)"
+        m10 = model_measure(da, df, perm, C, ac, fc, device, llama3_8b_math10k_keep())
+        m10["keep_table"] = "FFN keep 0.01 on L3-L30, QKVO keep 0.25 on L14-19, L21-23, L25-29, else dense (from 1)"
+        line["model_32_layers_math10k_table"] = m10
     if world == 1 and not args.no_layer:
         line["full_layer"] = full_layer_measure(attn, ffn, step_in, perm, ac, args.steps, max(args.warmup, 3), device)
     if not args.no_e2e:

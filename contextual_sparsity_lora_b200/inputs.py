@@ -82,6 +82,23 @@ def spectral_weight(d_out: int, d_in: int, alpha: float, k: int, gen, device="cp
     return out
 
 
+def signed_permutation(w: SpectralWeight, gen) -> SpectralWeight:
+    """Another weight of the same spectrum: W' = P_out W P_in^T with random signed permutations
+    P_out, P_in (orthogonal), so U' = P_in U and V' = P_out V stay orthonormal and the factors
+    move with them (rows of W_A, columns of W_B), exactly, in any storage dtype. One spectral
+    draw thus gives distinct per-layer weights without a new orthogonalisation."""
+    d_out, d_in = w.W.shape
+    dev = w.W.device
+    po = torch.randperm(d_out, generator=gen).to(dev)
+    pi = torch.randperm(d_in, generator=gen).to(dev)
+    so = (torch.randint(0, 2, (d_out,), generator=gen) * 2 - 1).to(device=dev, dtype=w.W.dtype)
+    si = (torch.randint(0, 2, (d_in,), generator=gen) * 2 - 1).to(device=dev, dtype=w.W.dtype)
+    W = w.W[po][:, pi] * so[:, None] * si[None, :]
+    W_A = w.W_A[pi] * si.to(w.W_A.dtype)[:, None]
+    W_B = w.W_B[:, po] * so.to(w.W_B.dtype)[None, :]
+    return SpectralWeight(W=W.contiguous(), W_A=W_A.contiguous(), W_B=W_B.contiguous(), s=w.s)
+
+
 def lora_pair(d_out: int, d_in: int, r: int, std: float, gen, device="cpu", dtype=torch.bfloat16):
     """LoRA adapter A [r, d_in], B [d_out, r], both i.i.d. N(0, std^2)."""
     A = _randn((r, d_in), gen, device, torch.float32) * std

@@ -34,6 +34,32 @@ def llama3_8b_math10k_keep(n_layers: int = 32):
     return out
 
 
+def layerwise_keep(n_layers: int = 32, dense_layers: int = 8, mid_end: int = 20, mid_keep: float = 0.6,
+                   deep_keep: float = 0.35):
+    """A non-uniform keep table over a 32-layer LLaMA3-8B (layers numbered from 0): layers
+    0-7 dense, 8-19 at keep 0.6, 20-31 at keep 0.35, the same ratio on the attention
+    projections and the FFN ([WT] "Layer Sensitivity Analysis and Non-Uniform Sparsity":
+    deeper layers tolerate more sparsity, so shallow layers stay dense)."""
+    out = []
+    for i in range(n_layers):
+        k = 1.0 if i < dense_layers else (mid_keep if i < mid_end else deep_keep)
+        out.append((k, k))
+    return out
+
+
+def cosine_lr(step: int, n_steps: int, peak: float, warmup_frac: float = 0.04) -> float:
+    """Learning rate of 1-based `step` of `n_steps` ([WT] "Step Sensitivity and Progressive
+    Sparse Fine-Tuning", the schedule of Table 11): linear warm-up to `peak` over the first
+    ceil(warmup_frac * n_steps) steps, then cosine decay to 0 at the last step."""
+    n_warm = math.ceil(warmup_frac * n_steps)
+    if step <= n_warm:
+        return peak * step / n_warm
+    if n_steps == n_warm:
+        return peak
+    t = (step - n_warm) / (n_steps - n_warm)
+    return 0.5 * peak * (1.0 + math.cos(math.pi * t))
+
+
 class SparseLoRAModel:
     def __init__(self, frozen, loras, gammas, keep, perm, n_ctx, n_seq, heads, est_k, lora_scale, device="cuda",
                  eps=1e-5):
@@ -110,10 +136,12 @@ class SparseLoRAModel:
             B.sl_adamw_step(master, blk.grads.flat, m, v, step, lr, betas[0], betas[1], eps, weight_decay,
                             params_bf16=blk.params.flat)
 
-    def step(self, ids_cf, targets_out, step: int, n_steps: int, lr: float, dense_frac: float = 0.1):
+    def step(self, ids_cf, targets_out, step: int, n_steps: int, lr: float, dense_frac: float = 0.1,
+             warmup_frac: float = 0.04):
         """One fine-tuning step (1-based `step` of `n_steps`): dense while step <= ceil(dense_frac *
-        n_steps), then with the per-layer keep ratios."""
+        n_steps), then with the per-layer keep ratios; AdamW at the cosine schedule's rate for
+        this step, peak `lr`."""
         self.set_dense(step <= math.ceil(dense_frac * n_steps))
         loss = self.forward_backward(ids_cf, targets_out)
-        self.optimizer_step(step, lr)
+        self.optimizer_step(step, cosine_lr(step, n_steps, lr, warmup_frac))
         return loss

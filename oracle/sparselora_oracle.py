@@ -58,6 +58,10 @@ Readings where the pages are silent or ambiguous (each is listed in the design doc):
       selections read the normalised layer inputs.
   R17 In the layer, output rows attend to context keys and values computed with the sparse
       projections, as the per-layer split implies (R12).
+  R19 The model step's loss is the mean cross-entropy of the LM head's logits over the output
+      rows only (next-token targets given per output row); the LM head is frozen.
+  R21 Learning rate: cosine decay to 0 at the last step after a linear warm-up over
+      ceil(0.04 n_steps) steps (the warm-up reaches the peak at its last step).
 
 Parity unpinned (no printed value or closed form pins them):
 the GQA aggregation of R5 and the V-space reading of R4.
@@ -510,6 +514,21 @@ def adamw(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
     mh = m / (1 - beta1 ** step)
     vh = v / (1 - beta2 ** step)
     return p - lr * mh / (np.sqrt(vh) + eps), m, v
+
+
+def cosine_lr(step, n_steps, peak, warmup_frac):
+    """Learning rate at 1-based `step` of `n_steps` under a cosine schedule with linear warm-up
+    ([WT] "Step Sensitivity and Progressive Sparse Fine-Tuning", interaction with the learning
+    rate schedule: Table 11's cosine scheduler with a 4% warm-up ratio; reading R21): the rate
+    climbs as a straight line from 0 to `peak` across the first ceil(warmup_frac * n_steps)
+    steps, then follows half a cosine period from `peak` down to 0 at the last step."""
+    n_warm = math.ceil(warmup_frac * n_steps)
+    if step <= n_warm:
+        return peak * (step / n_warm)
+    if n_steps == n_warm:
+        return peak
+    phase = (step - n_warm) / (n_steps - n_warm)  # 0 just after the warm-up, 1 at the last step
+    return peak * (math.cos(math.pi * phase) + 1.0) / 2.0
 
 
 def dense_lora_reference(X, dY, W, A, B, scale):

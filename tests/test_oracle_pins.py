@@ -625,3 +625,20 @@ def test_model_step_one_layer_equals_layer_and_loss_gradient():
                 lm[name][1][i, j] -= h
                 num[i, j] = (loss_of(lp) - loss_of(lm)) / (2 * h)
         np.testing.assert_allclose(grads[0]["dB_" + name], num, rtol=1e-5, atol=1e-8)
+
+
+def test_cosine_lr_closed_forms():
+    # 100 steps, 4% warm-up: 4 warm-up steps reaching the peak at step 4; the cosine half-period
+    # over steps 4..100 is at its midpoint (peak / 2) at step 52 and reaches 0 at step 100
+    f = lambda t: oracle.cosine_lr(t, 100, 2e-4, 0.04)
+    assert f(1) == pytest.approx(0.5e-4, rel=1e-15)
+    assert f(4) == pytest.approx(2e-4, rel=1e-15)
+    assert f(52) == pytest.approx(1e-4, rel=1e-12)
+    assert f(100) == pytest.approx(0.0, abs=1e-20)
+    # a third of the decay: (cos(pi / 3) + 1) / 2 = 3/4 of the peak
+    assert f(4 + 32) == pytest.approx(0.75 * 2e-4, rel=1e-12)
+    rates = [f(t) for t in range(4, 101)]
+    assert all(a >= b for a, b in zip(rates, rates[1:]))
+    # 20 steps: ceil(0.8) = 1 warm-up step, so the first step already runs at the peak
+    assert oracle.cosine_lr(1, 20, 1.0, 0.04) == 1.0
+    assert oracle.cosine_lr(20, 20, 1.0, 0.04) == pytest.approx(0.0, abs=1e-15)
