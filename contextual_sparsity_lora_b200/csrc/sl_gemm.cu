@@ -286,24 +286,37 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         }
         break;
       }
-      case EPI_F32: {
-        float* out = reinterpret_cast<float*>(pr.out0);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i >= n) break;
-          const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
-          float* d = out + orow * pr.ld0 + col;
-          *d = pr.a0 * v[i] + (pr.beta ? *d : 0.f);
-        }
-        break;
-      }
+      case EPI_F32:
       case EPI_F32_T: {
+        // out += a0 v goes out as a reduction in L2 (no load round trip; each element receives
+        // one addition per launch, so the result does not depend on timing). Without a column
+        // map or split, column i of the chunk is base + i * step: a short instruction stream,
+        // which matters when each CTA runs this code once (its first fetch is the cost).
+        if (!pr.col_map && !pr.col_split) {
+          const bool tr = pr.epi == EPI_F32_T;
+          const int64_t step = tr ? pr.ld0 : 1;
+          float* base = reinterpret_cast<float*>(pr.out0) + (tr ? (int64_t)(n0 + c0) * pr.ld0 + orow
+                                                                 : orow * pr.ld0 + n0 + c0);
+          if (pr.beta) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < n) atomicAdd(base + i * step, pr.a0 * v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < n) base[i * step] = pr.a0 * v[i];
+          }
+          break;
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i >= n) break;
           const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
-          float* d = f32t_dst(pr, col) + orow;
-          *d = pr.a0 * v[i] + (pr.beta ? *d : 0.f);
+          float* d = pr.epi == EPI_F32 ? reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + col : f32t_dst(pr, col) + orow;
+          if (pr.beta)
+            atomicAdd(d, pr.a0 * v[i]);
+          else
+            *d = pr.a0 * v[i];
         }
         break;
       }
