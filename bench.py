@@ -319,6 +319,47 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
     return out
 
 
+def rank_sweep(fc, x, C, device, ks=(4, 8, 16), reps=20):
+    """Estimator rank k against cost and fidelity on the LLaMA3-8B FFN (the sweep the pages leave
+    open): for each k, the device time of estimator + selection (10 copies per CUDA graph) and
+    how well the estimated kept set matches the kept set of the exact criterion,
+    ||SiLU(X_ctx W_g^T)[:, i] * (X_ctx W_u^T)[:, i]||_2 computed with full products (torch,
+    evaluation only): the recall of the exact top-n and the share of the exact top-n's squared
+    criterion mass the estimated set holds. One spectral draw with rank-16 factors; ranks 4 and
+    8 are its truncations (the leading singular triplets), so every k sees the same weights."""
+    from contextual_sparsity_lora_b200 import blocks
+    d = inputs.make_ffn_inputs(inputs.scaled(fc, k=max(ks)), 1, device=device)
+    T = fc.n_tok
+    xc = x[:C].float()
+    g = xc @ d["gate"].W.float().t()
+    u = xc @ d["up"].W.float().t()
+    s_true = (torch.nn.functional.silu(g) * u).pow(2).sum(0)
+    del g, u, xc
+    out = {}
+    for k in ks:
+        cut = lambda w: inputs.SpectralWeight(W=w.W, W_A=w.W_A[:, :k].contiguous(), W_B=w.W_B[:k].contiguous(), s=w.s)
+        blk = blocks.FFNBlock(cut(d["gate"]), cut(d["up"]), cut(d["down"]), d["lora_gate"], d["lora_up"],
+                              d["lora_down"], fc.lora_scale, k, T, C, fc.ratio, device)
+
+        def sel():
+            blk.estimate(x)
+            blk.choose()
+        sel()
+        g10 = capture_graph(lambda: [sel() for _ in range(10)], warm=False)
+        us = time_steps(g10.replay, reps, 3, 1, device) / (reps * 10) * 1e3
+        n = blk.n_keep
+        top = torch.topk(s_true, n).indices
+        kept = blk.sigma[:n].long()
+        out[f"k{k}"] = {"estimate_select_us": us,
+                        "recall_of_exact_top_n": float(torch.isin(kept, top).float().mean()),
+                        "exact_mass_share": float(s_true[kept].sum() / s_true[top].sum())}
+        del g10, blk
+        torch.cuda.synchronize()
+    out["workload"] = (f"LLaMA3-8B FFN, {C} context rows, keep {fc.ratio}; synthetic weights with singular "
+                       f"values i^-{fc.alpha}")
+    return out
+
+
 def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
     """The fp64 oracle on the host cores over a bounded sample: the last ``n_tokens``
     tokens of the first sequence (context and output tokens in the workload's proportion
@@ -621,6 +662,8 @@ def main():
         saved = (attn.dp, ffn.dp)
         attn.dp = ffn.dp = None  # rank-local stages only: no collective inside the stage graphs
         line["stages"] = stage_times(attn, ffn, step_in, 50, device, float(peaks.get("hbm_gbs", 6650.0)), ms_step)
+        if world == 1:
+            line["stages"]["estimator_rank_sweep"] = rank_sweep(fc, step_in["ffn_x"], C, device)
         attn.dp, ffn.dp = saved
     barrier(world)
     # dense LoRA on the same kernels (keep ratio 1, no estimator): context, not the headline
