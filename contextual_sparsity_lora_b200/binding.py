@@ -30,7 +30,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
-            "sl_add_rows", "sl_adamw_step")
+            "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -103,6 +103,7 @@ def lib():
         L.sl_profile_enable.argtypes = [c_int32]
         L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
         L.sl_permute_rows.argtypes = [P, c_int64, P, c_int64, c_int64, P, c_int64, P]
+        L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P]
         for n in EXPORTED:
             if n not in ("sl_status_string", "sl_version", "sl_keep_count", "sl_svd_partials_count"):
                 getattr(L, n).restype = c_int32
@@ -317,6 +318,15 @@ def sl_prepare_weight(w, w_t):
 def sl_permute_rows(src, perm, dst):
     _check("sl_permute_rows", lib().sl_permute_rows(_ptr(src), src.stride(0), _ptr(perm), perm.numel(),
                                                     src.shape[1], _ptr(dst), dst.stride(0), _stream()))
+
+
+def sl_gather_rows_batch(srcs, perms, dsts):
+    """dst_q[i, :] = src_q[perm_q[i], :] for every q, in one launch (at most 8 gathers);
+    perm_q holds one int32 index per row of dst_q."""
+    n = len(srcs)
+    _check("sl_gather_rows_batch", lib().sl_gather_rows_batch(
+        n, _ptrs(srcs), _i64s([t.stride(0) for t in srcs]), _ptrs(perms), _i64s([t.numel() for t in perms]),
+        _i64s([t.shape[1] for t in srcs]), _ptrs(dsts), _i64s([t.stride(0) for t in dsts]), _stream()))
 
 
 def sl_profile_enable(on: bool):

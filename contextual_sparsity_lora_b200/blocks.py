@@ -201,9 +201,7 @@ class FFNBlock:
     def compact(self):
         """The kept weight rows of gate, up (rows of W) and down (rows of W^T) for this step."""
         kept = self.sigma[: self.n_keep]
-        B.sl_permute_rows(self.Wg, kept, self.Wg_k)
-        B.sl_permute_rows(self.Wu, kept, self.Wu_k)
-        B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+        B.sl_gather_rows_batch([self.Wg, self.Wu, self.Wd_t], [kept] * 3, [self.Wg_k, self.Wu_k, self.Wd_k])
 
     def select(self, x):
         """a1 + a2 + a3 on the context rows of x, then the kept weight rows."""
@@ -229,8 +227,7 @@ class FFNBlock:
                 self.estimate(x)
                 self.choose()
                 kept = self.sigma[: self.n_keep]
-                B.sl_permute_rows(self.Wg, kept, self.Wg_k)
-                B.sl_permute_rows(self.Wu, kept, self.Wu_k)
+                B.sl_gather_rows_batch([self.Wg, self.Wu], [kept] * 2, [self.Wg_k, self.Wu_k])
                 with self.side.fork():  # down's kept rows are needed only by the down product
                     B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
                 torch.cuda.current_stream().wait_event(lora_done)
@@ -418,15 +415,20 @@ class AttnProjBlock:
         self.dense = bool(on) or self._always_dense
         self.lin, self.ch = (self._lin_dense, self._ch_dense) if self.dense else (self._lin_sparse, self._ch_sparse)
 
+    def _kept_rows(self, names):
+        """The kept weight rows of the named projections (rows of W; for o, rows of W^T), one launch."""
+        src = {"q": (self.Wq, self.sig_q), "k": (self.Wk, self.sig_k), "v": (self.Wv, self.sig_v),
+               "o": (self.Wo_t, self.sig_o)}
+        B.sl_gather_rows_batch([src[n][0] for n in names], [src[n][1][: self.ch[n].n_keep] for n in names],
+                               [self.W_k[n] for n in names])
+
     def _qk_chain(self):
         self._select_qk()
-        for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k)):
-            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+        self._kept_rows("qk")
 
     def _vo_chain(self):
         self._select_vo()
-        for n, w, sig in (("v", self.Wv, self.sig_v), ("o", self.Wo_t, self.sig_o)):
-            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+        self._kept_rows("vo")
 
     def choose(self):
         """a3: the q/k set from the QK scores and the v/o set from the V scores."""
@@ -435,9 +437,7 @@ class AttnProjBlock:
 
     def compact(self):
         """The kept weight rows of q, k, v (rows of W) and o (rows of W^T) for this step."""
-        for n, w, sig in (("q", self.Wq, self.sig_q), ("k", self.Wk, self.sig_k), ("v", self.Wv, self.sig_v),
-                          ("o", self.Wo_t, self.sig_o)):
-            B.sl_permute_rows(w, sig[: self.ch[n].n_keep], self.W_k[n])
+        self._kept_rows("qkvo")
 
     def select(self, x):
         """a1 + a2, then the q/k and v/o selections with their kept weight rows: two

@@ -577,11 +577,12 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   }
   Carver c(ws->ptr);
   carve(c, bsig, &dcat, &region);
-  if (out_sig)
+  if (out_sig) {
+    GatherBatch gat;
     for (int i = 0; i < n_ad; ++i)
-      if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i],
-                                    lin[i].r, 0, s))
-        return from_kernel(rc);
+      gat.add(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i], lin[i].r);
+    if (int rc = gat.launch(s)) return from_kernel(rc);
+  }
   // dya = scale * dy B and dB = dy^T xa_s from one pass over each dy (fused kernel; context rows
   // of a sigma-layout dy use the permuted B and land in dB rows sigma[p]), then dya_s = bf16(dya)
   {
@@ -721,14 +722,15 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
     Carver c(ws->ptr);
     carve(c, wc, bs);
+    GatherBatch gat;  // kept weight rows (when not given) and sigma-ordered LoRA B, one launch
     for (int i = 0; i < n_lin; ++i) {
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
-      else if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
-        return from_kernel(rc);
-      if (int rc = gather_rows_bf16(lin[i].lora_b, lin[i].r, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r, 0, s))
-        return from_kernel(rc);
+      else
+        gat.add(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
+      gat.add(lin[i].lora_b, lin[i].r, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r);
     }
+    if (int rc = gat.launch(s)) return from_kernel(rc);
     GemmBuilder gb;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     int koff = 0;
@@ -788,22 +790,22 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     Carver c(ws->ptr);
     carve(c, wc, pk);
     const int32_t* sig = ch[0].sigma;
+    GatherBatch gat;  // kept weight rows (when not given) and the paired LoRA B packs, one launch
     for (int i = 0; i < 2; ++i) {
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
-      else if (int rc = gather_rows_bf16(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in, 0, s))
-        return from_kernel(rc);
+      else
+        gat.add(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in);
     }
     // LoRA B operand of a paired tile t: rows 256 t + j = [B_gate[c_j] | 0], rows 256 t + 128 + j = [0 | B_up[c_j]]
     cudaMemsetAsync(pk[0], 0, (size_t)nt * 256 * 64 * 2, s);
     cudaMemsetAsync(pk[1], 0, (size_t)nt * 256 * 64 * 2, s);
     for (int v = 0; v < 2; ++v) {
       const int32_t* idx = v == 0 ? sig : nullptr;
-      if (int rc = gather_rows_bf16(lin[0].lora_b, lin[0].r, idx, F, lin[0].r, pk[v], 64, 0, s, 128, 256, 0))
-        return from_kernel(rc);
-      if (int rc = gather_rows_bf16(lin[1].lora_b, lin[1].r, idx, F, lin[1].r, pk[v], 64, lin[0].r, s, 128, 256, 128))
-        return from_kernel(rc);
+      gat.add(lin[0].lora_b, lin[0].r, idx, F, lin[0].r, pk[v], 64, 0, 128, 256, 0);
+      gat.add(lin[1].lora_b, lin[1].r, idx, F, lin[1].r, pk[v], 64, lin[0].r, 128, 256, 128);
     }
+    if (int rc = gat.launch(s)) return from_kernel(rc);
     GemmBuilder gb;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     const int mxa = gb.map(xa_s, T, lin[0].r + lin[1].r, ld_xa, kBM);
@@ -925,10 +927,11 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
     Carver c(ws->ptr);
     carve(c, wc, dyc);
+    GatherBatch gat;
+    for (int i = 0; i < n_lin; ++i)
+      if (!lin[i].w_kept) gat.add(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
+    if (int rc = gat.launch(s)) return from_kernel(rc);
     for (int i = 0; i < n_lin; ++i) {
-      if (!lin[i].w_kept)
-        if (int rc = gather_rows_bf16(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in, 0, s))
-          return from_kernel(rc);
       if (dyc[i])
         if (int rc = gather_cols_bf16(dy[i], ld_dy[i], C, ch[i].sigma, ch[i].n_keep, dyc[i], rup(ch[i].n_keep, 8), s))
           return from_kernel(rc);
@@ -992,11 +995,13 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   }
   Carver c(ws->ptr);
   carve(c, &wtc, &at, &ats);
-  if (!L.w_kept)
-    if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s))
-      return from_kernel(rc);
   if (int rc = transpose_bf16(L.lora_a, L.r, d_in, d_in, at, L.r, s)) return from_kernel(rc);
-  if (int rc = gather_rows_bf16(at, L.r, ch[0].sigma, d_in, L.r, ats, L.r, 0, s)) return from_kernel(rc);
+  {
+    GatherBatch gat;  // kept rows of W^T (when not given) and the permuted A^T, one launch
+    if (!L.w_kept) gat.add(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out);
+    gat.add(at, L.r, ch[0].sigma, d_in, L.r, ats, L.r);
+    if (int rc = gat.launch(s)) return from_kernel(rc);
+  }
   GemmBuilder gb;
   const int mdy = gb.map(dy[0], T, L.d_out, ld_dy[0], kBM);
   const int mya = gb.map(dya_s[0], T, L.r, L.r, kBM);
@@ -1087,6 +1092,22 @@ sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, 
   if (!src || !perm || !dst) return SL_ERR_INVALID_ARG;
   if (n_rows <= 0 || n_cols <= 0 || ld_src < n_cols || ld_dst < n_cols) return SL_ERR_SHAPE;
   return from_kernel(permute_rows_bf16(src, ld_src, perm, n_rows, n_cols, dst, ld_dst, cs(stream)));
+}
+
+sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src, const int32_t* const* perm,
+                               const int64_t* n_rows, const int64_t* n_cols, void* const* dst, const int64_t* ld_dst,
+                               sl_stream stream) {
+  if (n < 1 || n > kMaxGatherJobs || !src || !ld_src || !perm || !n_rows || !n_cols || !dst || !ld_dst)
+    return SL_ERR_INVALID_ARG;
+  GatherBatch gat;
+  for (int q = 0; q < n; ++q) {
+    if (n_rows[q] < 0) return SL_ERR_SHAPE;
+    if (n_rows[q] == 0) continue;
+    if (!src[q] || !perm[q] || !dst[q]) return SL_ERR_INVALID_ARG;
+    if (n_cols[q] <= 0 || ld_src[q] < n_cols[q] || ld_dst[q] < n_cols[q]) return SL_ERR_SHAPE;
+    gat.add(src[q], ld_src[q], perm[q], n_rows[q], n_cols[q], dst[q], ld_dst[q]);
+  }
+  return from_kernel(gat.launch(cs(stream)));
 }
 
 }  // extern "C"

@@ -34,6 +34,27 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int64_
   }
 }
 
+// Several row gathers in one launch: blockIdx.y picks the job, each warp copies one row as in
+// gather_rows_kernel (the grid covers the job with the most rows; shorter jobs return early).
+__global__ void gather_rows_multi_kernel(const __grid_constant__ GatherJobs p) {
+  pdl_wait();
+  const GatherJob& j = p.j[blockIdx.y];
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= j.n_rows) return;
+  const int64_t sr = j.idx ? (int64_t)j.idx[row] : row;
+  const int64_t drow = j.blk ? (row / j.blk) * j.blk_stride + j.blk_off + row % j.blk : row;
+  const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(j.src) + sr * j.ld_src;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(j.dst) + drow * j.ld_dst + j.col0;
+  if (j.vec) {
+    const int64_t nv = j.n_cols / 8;
+    for (int64_t c = lane; c < nv; c += 32)
+      reinterpret_cast<uint4*>(dst)[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+  } else {
+    for (int64_t c = lane; c < j.n_cols; c += 32) dst[c] = src[c];
+  }
+}
+
 // dst[t, j] = src[t, idx[j]]
 __global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t n_rows,
                                    const int32_t* __restrict__ idx, int64_t n_idx, __nv_bfloat16* __restrict__ dst,
@@ -79,6 +100,40 @@ int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_
   launch_kernel(gather_rows_kernel, (unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s, 
       (const __nv_bfloat16*)src, ld_src, idx, n_rows, n_cols, (__nv_bfloat16*)dst, ld_dst, dst_col0, vec, blk,
       blk_stride, blk_off);
+  if (launch_failed("sl_aux")) return 5;
+  note_launch();
+  return 0;
+}
+
+int GatherBatch::add(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
+                     int64_t ld_dst, int64_t dst_col0, int blk, int blk_stride, int blk_off) {
+  if (n_rows <= 0 || n_cols <= 0) return 0;
+  if (jobs.n >= kMaxGatherJobs) return 1;
+  GatherJob& j = jobs.j[jobs.n++];
+  j.src = src;
+  j.ld_src = ld_src;
+  j.idx = idx;
+  j.n_rows = n_rows;
+  j.n_cols = n_cols;
+  j.dst = dst;
+  j.ld_dst = ld_dst;
+  j.col0 = dst_col0;
+  j.blk = blk;
+  j.blk_stride = blk_stride;
+  j.blk_off = blk_off;
+  j.vec = (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (dst_col0 % 8 == 0) &&
+          ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
+  return 0;
+}
+
+int GatherBatch::launch(cudaStream_t s) {
+  if (jobs.n == 0) return 0;
+  int64_t rows = 0;
+  for (int i = 0; i < jobs.n; ++i) rows = rows > jobs.j[i].n_rows ? rows : jobs.j[i].n_rows;
+  const int rows_per_block = 8;
+  const dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), (unsigned)jobs.n);
+  launch_kernel(gather_rows_multi_kernel, grid, 32 * rows_per_block, 0, s, jobs);
+  jobs.n = 0;
   if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;

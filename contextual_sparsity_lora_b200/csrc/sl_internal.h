@@ -177,6 +177,26 @@ int wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_
 int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols,
                      void* dst, int64_t ld_dst, int64_t dst_col0, cudaStream_t s, int blk = 0, int blk_stride = 0,
                      int blk_off = 0);
+// Row gathers batched into one launch (jobs as in gather_rows_bf16).
+constexpr int kMaxGatherJobs = 8;
+struct GatherJob {
+  const void* src;
+  const int32_t* idx;
+  void* dst;
+  int64_t ld_src, n_rows, n_cols, ld_dst, col0;
+  int32_t blk, blk_stride, blk_off, vec;
+};
+struct GatherJobs {
+  GatherJob j[kMaxGatherJobs];
+  int32_t n;
+};
+struct GatherBatch {
+  GatherJobs jobs{};
+  // returns 1 when the batch is full; empty jobs are skipped
+  int add(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
+          int64_t ld_dst, int64_t dst_col0 = 0, int blk = 0, int blk_stride = 0, int blk_off = 0);
+  int launch(cudaStream_t s);  // one launch for every job added, then empty
+};
 int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int32_t* idx, int64_t n_idx,
                      void* dst, int64_t ld_dst, cudaStream_t s);
 int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,

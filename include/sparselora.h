@@ -350,6 +350,19 @@ SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, v
 SL_API sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
                           void* dst, int64_t ld_dst, sl_stream stream);
 
+/* Up to 8 row gathers of bf16 rows in one launch: for each q < n, dst[q][i, :] =
+ * src[q][perm[q][i], :] for i < n_rows[q], n_cols[q] columns, leading dimensions ld_src[q] and
+ * ld_dst[q]. Used to build the kept weight rows of several projections at once (each w_kept
+ * of a step: "SparseLoRA: Accelerating LLM Fine-Tuning with Contextual Sparsity",
+ * walkthrough, "Putting It All Together": the weights sliced to the selected channels).
+ * The arrays are host arrays of length n; every pointer in them is a device pointer. The
+ * destinations must not overlap any source. Errors: SL_ERR_INVALID_ARG for n outside [1, 8]
+ * or a null pointer, SL_ERR_SHAPE for a non-positive size or a leading dimension below
+ * n_cols. A job with zero rows is skipped (its pointers may be NULL). */
+SL_API sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src,
+                                      const int32_t* const* perm, const int64_t* n_rows, const int64_t* n_cols,
+                                      void* const* dst, const int64_t* ld_dst, sl_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

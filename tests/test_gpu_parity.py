@@ -283,3 +283,26 @@ def test_select_and_estimate_are_deterministic():
         B.sl_select_channels(sc, 500, sig)
         outs.append((sc.cpu(), sig.cpu()))
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_gather_rows_batch_is_exact():
+    """Several row gathers in one launch: ragged row counts, a width that is not a multiple of
+    8 (scalar copies), a strided destination and an empty job, against NumPy indexing."""
+    from contextual_sparsity_lora_b200 import binding as B
+    rng = np.random.default_rng(81)
+    shapes = [(300, 64, 120), (77, 203, 77), (5, 13, 0), (1000, 40, 999)]  # (src rows, cols, gathered rows)
+    srcs, perms, dsts, want = [], [], [], []
+    for rows, cols, n in shapes:
+        src = torch.from_numpy(rng.standard_normal((rows, cols)).astype(np.float32)).to(torch.bfloat16)
+        p = rng.permutation(rows)[:n].astype(np.int32)
+        wide = torch.zeros(max(n, 1), cols + 24, dtype=torch.bfloat16, device=DEV)
+        srcs.append(src.to(DEV))
+        perms.append(torch.from_numpy(p).to(DEV))
+        dsts.append(wide[:n, :cols] if n else wide[:0, :cols])
+        want.append(src.view(torch.int16).numpy()[p])
+    B.sl_gather_rows_batch(srcs, perms, dsts)
+    torch.cuda.synchronize()
+    for d, w in zip(dsts, want):
+        np.testing.assert_array_equal(d.cpu().view(torch.int16).numpy(), w)
+    with pytest.raises(RuntimeError):
+        B.sl_gather_rows_batch(srcs * 3, perms * 3, dsts * 3)  # more than 8 jobs
