@@ -361,9 +361,10 @@ def rank_sweep(fc, x, C, device, ks=(4, 8, 16), reps=20):
 
 
 def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
-    """The fp64 oracle on the host cores over a bounded sample: the last ``n_tokens``
-    tokens of the first sequence (context and output tokens in the workload's proportion
-    when n_tokens = 512 or 128) through both blocks, estimator to LoRA gradients."""
+    """The fp64 oracle on the host cores over a bounded sample: ``n_tokens`` consecutive
+    tokens of the first sequence, the window placed so that context and output tokens keep the
+    workload's proportion (the whole sequence at 512: 384 context + 128 output; at 128:
+    96 + 32), through both blocks, estimator to LoRA gradients."""
     import numpy as np
     import oracle
     try:
@@ -373,7 +374,9 @@ def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
         threads = os.cpu_count()
     ac, fc = inputs.LLAMA3_8B_ATTN, inputs.LLAMA3_8B_FFN
     S = int(n_tokens)
-    sl = slice(ac.seq - S, ac.seq)                 # tail of the first sequence, sequence order
+    n_o = round(S * ac.n_out / ac.seq)             # output tokens of the window
+    end = ac.seq - ac.n_out + n_o
+    sl = slice(end - S, end)                       # sequence order, ends n_o tokens into the output part
     ctx = da["ctx_mask"][sl].cpu().numpy()
     f64 = oracle.f64
     X = f64(da["x"][sl]); XO = f64(da["x_o"][sl]); dq = f64(da["dq"][sl]); dk = f64(da["dk"][sl])
