@@ -66,7 +66,7 @@ typedef enum {
   SL_ERR_SHAPE = 2,       /* sizes out of the supported range */
   SL_ERR_ALIGNMENT = 3,   /* base address or leading dimension not aligned for TMA */
   SL_ERR_WORKSPACE = 4,   /* workspace missing or too small; ws->needed holds the size */
-  SL_ERR_UNSUPPORTED = 5, /* a valid request this build does not implement */
+  SL_ERR_UNSUPPORTED = 5, /* a valid request the library does not implement */
   SL_ERR_CUDA = 6,        /* a CUDA launch or driver call failed */
   SL_ERR_DEVICE_FLAG = 7  /* a kernel reported a device-side timeout */
 } sl_status;

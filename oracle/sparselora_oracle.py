@@ -25,7 +25,7 @@ W in R^{D_in x D_out}. This oracle takes weights in nn.Linear storage order,
 ``B[D_out, r]``, y += scale * (x A^T) B^T. Tokens are rows; ``ctx`` is a
 boolean row mask (True = context token, False = output token).
 
-Readings where the pages are silent or ambiguous (each is listed in the design doc):
+Readings where the pages are silent or ambiguous:
   R1  W_B = diag(sqrt(s_k)) V[:, :k]^T with V the right singular vectors, so
       that W_A W_B is the Eckart-Young rank-k truncation.
   R3  Scores are reduced over the context rows of the layer's own input, all
@@ -63,7 +63,7 @@ Readings where the pages are silent or ambiguous (each is listed in the design doc):
   R21 Learning rate: cosine decay to 0 at the last step after a linear warm-up over
       ceil(0.04 n_steps) steps (the warm-up reaches the peak at its last step).
 
-Parity unpinned (no printed value or closed form pins them; see DESIGN.md):
+Parity unpinned (no printed value or closed form pins them):
 the GQA aggregation of R5 and the V-space reading of R4.
 """
 from __future__ import annotations
