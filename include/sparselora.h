@@ -41,6 +41,13 @@
  *   status; nothing is launched on an error. Launch failures give SL_ERR_CUDA. All
  *   device-side waits are bounded; a wait that runs out writes a non-zero code
  *   into the workspace's error word (read it with sl_read_device_flag).
+ * - Environment (read once per process; each changes how a result is computed, never
+ *   which result): SL_PDL=0 launches without programmatic dependent launch;
+ *   SL_VERBOSE_ERRORS=1 prints the CUDA error of a failed launch to stderr;
+ *   SL_PAIR_MH=1|2 forces 256- or 512-row CTA-pair GEMM tiles (default: chosen per
+ *   launch); SL_GEMM_1CTA=1 runs every GEMM on the one-CTA kernel; SL_GEMM_BROWS=256
+ *   forces the one-CTA kernel's widest B stage; SL_GEMM_BULK_STORE=0 stores bf16
+ *   epilogues per thread instead of through bulk tensor copies.
  */
 #ifndef SPARSELORA_H_
 #define SPARSELORA_H_
