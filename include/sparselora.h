@@ -117,7 +117,8 @@ typedef struct {
    * with the call, row-major and dense: SL_SLICE_OUT: w[sigma[j], :] for j < n_keep
    * ([n_keep, d_in]); SL_SLICE_IN: w_t[sigma[j], :] ([n_keep, d_out]). The forward and
    * the backward of one step use the same rows, so a caller that builds them once per
-   * step (sl_permute_rows with the first n_keep entries of sigma) saves both calls their
+   * step (sl_gather_rows_batch or sl_permute_rows with the first n_keep entries of sigma,
+   * several projections per launch with the former) saves both calls their
    * own gather into the workspace. With keep ratio 1 and the identity sigma it is w
    * (w_t) itself. The caller keeps it consistent with sigma; 16-byte aligned. */
   const void* w_kept;
