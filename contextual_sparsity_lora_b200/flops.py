@@ -28,6 +28,13 @@ def dense_warmup_speedup_bound(p: float, s: float) -> float:
     return 1.0 / (p + (1.0 - p) / s)
 
 
+def estimator_factor_bytes(n_layers: int, projections, k: int, bytes_per_param: int = 2) -> int:
+    """Memory of the offline rank-k factors W_A [d_in, k] and W_B [k, d_out]: k (d_in + d_out)
+    parameters per estimated projection (same page, memory overhead), over `n_layers` layers
+    with the (d_in, d_out) pairs in `projections`."""
+    return n_layers * sum(k * (di + do) for di, do in projections) * bytes_per_param
+
+
 def frozen_fwd_bwd(d_in: int, d_out: int, n_tok: int, n_ctx: int, n_kept_of_sliced_side: int,
                    sliced_side_size: int) -> float:
     """Frozen-branch FLOPs of one projection; the kept count is on the sliced side

@@ -34,3 +34,11 @@ def test_attention_projection_totals():
     assert w["main"] / 1e12 == pytest.approx(0.430, abs=2e-3)
     dense = flops.attn_proj_block(4096, 32, 8, 128, 4096, 3072, 1024, 1024, 32, 8)
     assert dense["main"] / 1e12 == pytest.approx(0.687, abs=2e-3)
+
+
+def test_factor_memory_worked_example():
+    """The factors of the estimated projections (q, k, v, gate, up) of LLaMA2-7B at k = 8 in
+    16-bit storage come to the page's approximate total."""
+    g = GOLD["factor_memory"]
+    b = flops.estimator_factor_bytes(g["n_layers"], g["projections"], g["k"], g["bytes_per_param"])
+    assert b / 1e6 == pytest.approx(g["approx_mb"], rel=g["rel_tol"])
