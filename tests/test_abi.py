@@ -137,3 +137,62 @@ def test_workspace_init_and_profile_hooks_host_side(lib):
     a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_double()
     assert lib.sl_profile_read(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == B.SL_OK
     assert lib.sl_profile_read(None, None, None) == B.SL_ERR_INVALID_ARG
+
+
+def test_layer_and_optimizer_entries_reject_bad_arguments(lib):
+    """RMSNorm, residual add, AdamW, head-level selection, Wanda scores and the batched row
+    gather check their arguments before any launch (fake device addresses are never touched)."""
+    P = ctypes.c_void_p
+    a, odd = P(0x10000), P(0x10002)  # 16-byte aligned / not
+    # sl_rmsnorm_fwd(x, ldx, res, ldr, sum_out, lds, gamma, eps, y, ldy, rstd, n_rows, d, stream)
+    f = lib.sl_rmsnorm_fwd
+    assert f(None, 64, None, 0, None, 0, a, 1e-5, a, 64, a, 4, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, a, 64, None, 0, a, 1e-5, a, 64, a, 4, 64, None) == B.SL_ERR_INVALID_ARG  # res without sum_out
+    assert f(a, 64, None, 0, None, 0, a, 1e-5, a, 64, a, 0, 64, None) == B.SL_ERR_SHAPE
+    assert f(a, 64, None, 0, None, 0, a, 1e-5, a, 64, a, 4, 60, None) == B.SL_ERR_SHAPE
+    assert f(a, 64, None, 0, None, 0, a, -1.0, a, 64, a, 4, 64, None) == B.SL_ERR_SHAPE
+    assert f(odd, 64, None, 0, None, 0, a, 1e-5, a, 64, a, 4, 64, None) == B.SL_ERR_ALIGNMENT
+    # sl_rmsnorm_bwd(dy, lddy, x, ldx, gamma, rstd, dres, ldr, dx, lddx, n_rows, d, stream)
+    g = lib.sl_rmsnorm_bwd
+    assert g(a, 64, a, 64, a, None, None, 0, a, 64, 4, 64, None) == B.SL_ERR_INVALID_ARG
+    assert g(a, 64, a, 32, a, a, None, 0, a, 64, 4, 64, None) == B.SL_ERR_ALIGNMENT  # ld below d
+    # sl_add_rows(a, lda, b, ldb, out, ldo, n_rows, d, stream)
+    h = lib.sl_add_rows
+    assert h(a, 64, None, 64, a, 64, 4, 64, None) == B.SL_ERR_INVALID_ARG
+    assert h(a, 64, a, 64, a, 64, 4, 12, None) == B.SL_ERR_SHAPE
+    # sl_adamw_step(p, g, m, v, p_bf16, n, lr, b1, b2, eps, wd, step, stream)
+    w = lib.sl_adamw_step
+    assert w(a, a, None, a, None, 10, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None) == B.SL_ERR_INVALID_ARG
+    assert w(a, a, a, a, None, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None) == B.SL_ERR_SHAPE
+    assert w(a, a, a, a, None, 10, 1e-3, 1.0, 0.999, 1e-8, 0.0, 1, None) == B.SL_ERR_SHAPE
+    assert w(a, a, a, a, None, 10, -1.0, 0.9, 0.999, 1e-8, 0.0, 1, None) == B.SL_ERR_SHAPE
+    assert w(a, a, a, a, None, 10, 1e-3, 0.9, 0.999, 1e-8, 0.0, 0, None) == B.SL_ERR_SHAPE
+    # sl_select_heads(scores, n_heads, head_dim, n_keep_heads, heads_per_group, sigma, sigma_wide, stream)
+    sh = lib.sl_select_heads
+    assert sh(None, 8, 128, 2, 4, a, None, None) == B.SL_ERR_INVALID_ARG
+    assert sh(a, 8, 128, 9, 4, a, None, None) == B.SL_ERR_SHAPE
+    assert sh(a, 0, 128, 1, 4, a, None, None) == B.SL_ERR_SHAPE
+    assert sh(a, 8, 128, 2, 0, a, a, None) == B.SL_ERR_INVALID_ARG  # query side without a group size
+    # sl_wanda_scores(x, n_ctx, d_in, ldx, n_proj, w, d_out, ldw, scores, ws, stream)
+    wa = lib.sl_wanda_scores
+    ws = B.SlWorkspaceC(None, 0, 0)
+    wp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    assert wa(a, 16, 64, 64, 0, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_INVALID_ARG
+    assert wa(a, 0, 64, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_SHAPE
+    assert wa(a, 16, 60, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_ALIGNMENT
+    assert wa(a, 16, 64, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_WORKSPACE
+    # sl_gather_rows_batch(n, src[], ld_src[], perm[], n_rows[], n_cols[], dst[], ld_dst[], stream)
+    gb = lib.sl_gather_rows_batch
+    ptrs = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    ok = dict(src=ptrs(0x10000), ld=i64(64), perm=ptrs(0x20000), rows=i64(4), cols=i64(64), dst=ptrs(0x30000))
+    args = lambda n, **k: [n] + [k.get(x, ok[x]) for x in ("src", "ld", "perm", "rows", "cols", "dst")] + \
+        [k.get("ldd", i64(64)), None]
+    assert gb(*args(0)) == B.SL_ERR_INVALID_ARG
+    assert gb(*args(9)) == B.SL_ERR_INVALID_ARG
+    assert gb(*args(1, perm=ptrs(None))) == B.SL_ERR_INVALID_ARG
+    assert gb(*args(1, rows=i64(-1))) == B.SL_ERR_SHAPE
+    assert gb(*args(1, cols=i64(0))) == B.SL_ERR_SHAPE
+    assert gb(*args(1, ldd=i64(32))) == B.SL_ERR_SHAPE
+    # a job without rows launches nothing, whatever its pointers
+    assert gb(*args(1, rows=i64(0), src=ptrs(None), perm=ptrs(None), dst=ptrs(None))) == B.SL_OK
