@@ -130,3 +130,36 @@ def test_data_parallel_ranks_select_the_batch_index_sets():
     np.testing.assert_array_equal(res[0][3][0], oracle.select_top(s_ffn, oracle.keep_count(0.5, F)))
     np.testing.assert_array_equal(res[0][3][1], sel["units_qk"])
     np.testing.assert_array_equal(res[0][3][2], sel["units_v"])
+
+
+def _ref_rank_main(rank, world, port, out):
+    """One rank of `torchrun ... bench.py --impl reference --gpus 2`: rank 0 prints the line."""
+    import contextlib
+    import io
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+
+    sys.argv = ["bench.py", "--impl", "reference", "--gpus", str(world), "--steps", "1", "--warmup", "1"]
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main()
+    out[rank] = buf.getvalue()
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_under_two_ranks_prints_once():
+    import json
+
+    ctx_ = mp.get_context("spawn")
+    with ctx_.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_ref_rank_main, args=(2, _free_port(), out), nprocs=2, start_method="spawn", join=True)
+        res = dict(out)
+    assert res[1].strip() == ""
+    lines = [l for l in res[0].splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
