@@ -642,3 +642,21 @@ def test_cosine_lr_closed_forms():
     # 20 steps: ceil(0.8) = 1 warm-up step, so the first step already runs at the peak
     assert oracle.cosine_lr(1, 20, 1.0, 0.04) == 1.0
     assert oracle.cosine_lr(20, 20, 1.0, 0.04) == pytest.approx(0.0, abs=1e-15)
+
+
+def test_sigmoid_identities():
+    # sigma(z) + sigma(-z) = 1, sigma(0) = 1/2, no overflow at large |z|, sigma(log 3) = 3/4
+    z = np.array([-800.0, -30.0, -1.5, 0.0, 1.5, 30.0, 800.0, np.log(3.0)])
+    s = oracle.sigmoid(z)
+    assert np.all(np.isfinite(s))
+    np.testing.assert_allclose(s + oracle.sigmoid(-z), 1.0, rtol=0, atol=1e-15)
+    assert s[3] == 0.5 and s[0] == 0.0 and s[6] == 1.0
+    assert s[7] == pytest.approx(0.75, rel=1e-15)
+
+
+def test_sliced_weight_zeroes_the_dropped_channels():
+    W = np.arange(12.0).reshape(3, 4)  # nn.Linear storage [d_out = 3, d_in = 4]; W_math = W.T [4, 3]
+    out = oracle.sliced_weight(W, np.array([0, 2]), "out")
+    np.testing.assert_array_equal(out, np.array([[0, 0, 8], [1, 0, 9], [2, 0, 10], [3, 0, 11]], dtype=float))
+    inn = oracle.sliced_weight(W, np.array([1, 3]), "in")
+    np.testing.assert_array_equal(inn, np.array([[0, 0, 0], [1, 5, 9], [0, 0, 0], [3, 7, 11]], dtype=float))
