@@ -55,16 +55,25 @@ def parse():
     return ap.parse_args()
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, cpu_only=False):
+    """Process group of a torchrun launch (none for one process). The reference arm runs on the
+    host cores only, so it takes gloo even on a GPU machine."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        backend = "nccl" if torch.cuda.is_available() and not cpu_only else "gloo"
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world, local
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
@@ -542,7 +551,7 @@ def reference_arm(args, rank, world):
             times.append(cb["seconds"])
     per = sum(times) / len(times)
     value = n_tok / per
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "seq_len": ac.seq, "sample_tokens_per_step": n_tok},
@@ -554,9 +563,12 @@ def reference_arm(args, rank, world):
 
 def main():
     args = parse()
-    rank, world, local = dist_setup(args.gpus)
+    rank, world, local = dist_setup(args.gpus, cpu_only=args.impl == "reference")
     if args.impl == "reference":
-        reference_arm(args, rank, world)
+        try:
+            reference_arm(args, rank, world)
+        finally:
+            dist_teardown(world)
         return
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device")

@@ -30,7 +30,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
-            "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch")
+            "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -104,6 +104,7 @@ def lib():
         L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
         L.sl_permute_rows.argtypes = [P, c_int64, P, c_int64, c_int64, P, c_int64, P]
         L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P]
+        L.sl_set_pair_tile_rows.argtypes = [c_int32]
         for n in EXPORTED:
             if n not in ("sl_status_string", "sl_version", "sl_keep_count", "sl_svd_partials_count"):
                 getattr(L, n).restype = c_int32
@@ -327,6 +328,26 @@ def sl_gather_rows_batch(srcs, perms, dsts):
     _check("sl_gather_rows_batch", lib().sl_gather_rows_batch(
         n, _ptrs(srcs), _i64s([t.stride(0) for t in srcs]), _ptrs(perms), _i64s([t.numel() for t in perms]),
         _i64s([t.shape[1] for t in srcs]), _ptrs(dsts), _i64s([t.stride(0) for t in dsts]), _stream()))
+
+
+def sl_set_pair_tile_rows(rows: int):
+    """Tile height of the CTA-pair GEMM for later launches: 256, 512, or 0 (chosen per launch)."""
+    _check("sl_set_pair_tile_rows", lib().sl_set_pair_tile_rows(int(rows)))
+
+
+class pair_tile_rows:
+    """Context manager that forces the CTA-pair tile height inside a block of calls (and
+    restores the per-launch choice after it)."""
+
+    def __init__(self, rows: int):
+        self.rows = int(rows)
+
+    def __enter__(self):
+        sl_set_pair_tile_rows(self.rows)
+        return self
+
+    def __exit__(self, *exc):
+        sl_set_pair_tile_rows(0)
 
 
 def sl_profile_enable(on: bool):

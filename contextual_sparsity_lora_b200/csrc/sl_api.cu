@@ -1081,6 +1081,12 @@ sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64
   return SL_OK;
 }
 
+sl_status sl_set_pair_tile_rows(int32_t rows) {
+  if (rows != 0 && rows != 256 && rows != 512) return SL_ERR_INVALID_ARG;
+  set_forced_pair_mh(rows / 256);
+  return SL_OK;
+}
+
 sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream) {
   if (!w || !w_t) return SL_ERR_INVALID_ARG;
   if (d_out <= 0 || d_in <= 0) return SL_ERR_SHAPE;

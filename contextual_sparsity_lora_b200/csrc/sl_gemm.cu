@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <vector>
 
@@ -57,16 +58,17 @@ __device__ __forceinline__ uint32_t seg_tx_bytes(const Seg& sg) {
   return bytes;
 }
 
-// The logistic function as sigma(g) = 1/2 + tanh(g / 2) / 2 with the hardware tanh
-// approximation (one special-function operation instead of an exponential and a reciprocal;
-// its relative error, below 2^-10.9, sits under the bf16 rounding of every epilogue output),
-// and SiLU(g) = g sigma(g). Saturation at large |g| gives the exact limits 0 and 1.
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// The logistic function from one exponential of -|g| (it never overflows) and one division
+// by 1 + e in (1, 2]: sigma(g) = 1 / (1 + e) for g >= 0 and e / (1 + e) for g < 0, with
+// e = exp(-|g|). Neither branch subtracts nearly equal numbers, so the relative error of
+// sigma(g), and of SiLU(g) = g sigma(g), stays at a few ulp of the two approximate operations
+// over the whole range, the far negative tail included (where a form built on 1 + tanh(g/2)
+// cancels: its absolute error, about 2^-12, exceeds sigma(g) itself below g = -8).
+__device__ __forceinline__ float sigmoid_f(float g) {
+  const float e = __expf(-fabsf(g));
+  const float q = __fdividef(1.0f, 1.0f + e);
+  return g >= 0.0f ? q : e * q;
 }
-__device__ __forceinline__ float sigmoid_f(float g) { return fmaf(0.5f, tanh_approx(0.5f * g), 0.5f); }
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -1074,12 +1076,12 @@ void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int ro
 // overlapped; a 256-row tile's epilogue overlaps the next tile's main loop and only shows
 // when that main loop is shorter. Epilogue weights (same units, measured on B200): plain
 // stores 4 per 256 rows; column scatter 8; the SwiGLU backward, which reads g and u from
-// global memory row by row, 20. SL_PAIR_MH=1|2 forces the choice.
+// global memory row by row, 20. sl_set_pair_tile_rows(256 | 512) forces the choice.
+static std::atomic<int> g_forced_mh{0};
+void set_forced_pair_mh(int mh) { g_forced_mh.store(mh, std::memory_order_relaxed); }
+int forced_pair_mh() { return g_forced_mh.load(std::memory_order_relaxed); }
 static int choose_pair_mh(const GemmParams& P, int nprob, int pairs) {
-  static const int forced = [] {
-    const char* e = getenv("SL_PAIR_MH");
-    return e ? atoi(e) : 0;
-  }();
+  const int forced = forced_pair_mh();
   if (forced == 1 || forced == 2) return forced;
   double best = 0.0;
   int best_mh = 1;

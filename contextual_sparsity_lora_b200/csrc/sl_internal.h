@@ -83,6 +83,11 @@ struct GemmBuilder {
   int launch(int* err, cudaStream_t stream);
 };
 
+// Forced CTA-pair tile height of the GEMM engine: 0 = chosen per launch, 1 = 256 rows,
+// 2 = 512 rows (sl_set_pair_tile_rows).
+void set_forced_pair_mh(int mh);
+int forced_pair_mh();
+
 // Split-K factor for a skinny problem with M rows and `kblocks` 64-wide K blocks: the
 // largest split whose tiles fit one wave of `target_tiles` CTAs (default: the current
 // device's SM count); 1 = no split.

@@ -44,8 +44,7 @@
  * - Environment (read once per process; each changes how a result is computed, never
  *   which result): SL_PDL=0 launches without programmatic dependent launch;
  *   SL_VERBOSE_ERRORS=1 prints the CUDA error of a failed launch to stderr;
- *   SL_PAIR_MH=1|2 forces 256- or 512-row CTA-pair GEMM tiles (default: chosen per
- *   launch); SL_GEMM_1CTA=1 runs every GEMM on the one-CTA kernel; SL_GEMM_BROWS=256
+ *   SL_GEMM_1CTA=1 runs every GEMM on the one-CTA kernel; SL_GEMM_BROWS=256
  *   forces the one-CTA kernel's widest B stage; SL_GEMM_BULK_STORE=0 stores bf16
  *   epilogues per thread instead of through bulk tensor copies.
  */
@@ -176,8 +175,11 @@ SL_API sl_status sl_svd_estimate(sl_criterion crit, sl_dtype dtype, const void* 
  *     kernels, the call's device error word (0 = no device-side timeout).
  * Errors: argument errors as sl_svd_estimate; SL_ERR_WORKSPACE when the shapes need more
  * than the 8 MiB (nothing is launched); SL_ERR_CUDA when the array's address cannot be
- * looked up. The first call on a device (with that device current) looks the address up
- * and should precede any stream capture there. All calls share the array and leave their
+ * looked up. The array costs 8 MiB of device memory on every device where the library is
+ * loaded, whether or not this entry is called. The first call on a device (with that device
+ * current) looks the address up and should precede any stream capture there; the address is
+ * kept per device and CUDA context, so the first call after a device reset looks it up again
+ * (and should not be captured either). All calls share the array and leave their
  * contents in it; the header is cleared at the start of each call. Calls that may execute
  * at the same time (different streams, unordered threads) race on it: serialise them. */
 SL_API sl_status sl_svd_estimate_noalloc(sl_criterion crit, sl_dtype dtype, const void* x, int64_t n_ctx,
@@ -350,6 +352,15 @@ SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launche
  * 1 (CTA pairs, 256-row tiles), 2 (CTA pairs, 512-row tiles), 3 (fused LoRA backward
  * stream) or 4 (estimator stage 1). Waits for the events. */
 SL_API sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count);
+
+/* Tile height of the CTA-pair tensor-core GEMM that runs the sliced products (a4, a5):
+ * rows = 256 (each pair of SMs computes 256 x 256 output tiles with two accumulators, so a
+ * tile's epilogue overlaps the next tile's products), 512 (512 x 256 tiles: a quarter fewer
+ * operand bytes per FLOP, epilogue not overlapped), or 0 (the default: chosen per launch by
+ * a makespan model of the persistent schedule). Process-wide; applies to launches issued
+ * (or captured) after the call; changes how a product is tiled, never its result beyond
+ * the fp32 summation order of the tile. Errors: SL_ERR_INVALID_ARG for any other value. */
+SL_API sl_status sl_set_pair_tile_rows(int32_t rows);
 
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
 SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream);

@@ -196,3 +196,12 @@ def test_layer_and_optimizer_entries_reject_bad_arguments(lib):
     assert gb(*args(1, ldd=i64(32))) == B.SL_ERR_SHAPE
     # a job without rows launches nothing, whatever its pointers
     assert gb(*args(1, rows=i64(0), src=ptrs(None), perm=ptrs(None), dst=ptrs(None))) == B.SL_OK
+
+
+def test_pair_tile_rows_setting_host_side(lib):
+    """The tile-height setting accepts 0 (chosen per launch), 256 and 512, and nothing else."""
+    for rows in (256, 512, 0):
+        assert lib.sl_set_pair_tile_rows(rows) == B.SL_OK
+    for rows in (-1, 1, 128, 384, 1024):
+        assert lib.sl_set_pair_tile_rows(rows) == B.SL_ERR_INVALID_ARG
+    assert lib.sl_set_pair_tile_rows(0) == B.SL_OK

@@ -306,3 +306,59 @@ def test_gather_rows_batch_is_exact():
         np.testing.assert_array_equal(d.cpu().view(torch.int16).numpy(), w)
     with pytest.raises(RuntimeError):
         B.sl_gather_rows_batch(srcs * 3, perms * 3, dsts * 3)  # more than 8 jobs
+
+
+# ------------------------------------------------------------- SiLU in the far negative tail
+
+@pytest.mark.parametrize("tile_rows", [256, 512])
+def test_swiglu_epilogues_elementwise_on_negative_gates(tile_rows):
+    """The SwiGLU epilogues evaluate the logistic function on every element. Gate pre-activations
+    spread over [-24, 3] (most of them strongly negative, where SiLU(g) is tiny) are checked
+    element by element at relative error 2e-2: h = SiLU(g) u (formed from the fp32 accumulators)
+    against the oracle's fp64 H, and the backward's dg = dh u SiLU'(g), du = dh SiLU(g) against
+    the oracle's formulas applied to the g, u the forward stored (bf16) and to the oracle's dh.
+    A logistic function with a fixed absolute error (such as one built on 1 + tanh(g/2)) fails
+    this test below g = -8."""
+    T, C, D, F, r, k = 256, 192, 256, 512, 16, 8
+    gen = inputs.generator(71)
+    absn = lambda *s: torch.randn(*s, generator=gen, dtype=torch.float64).abs()
+    x = absn(T, D).to(torch.bfloat16)                       # non-negative inputs: no cancellation in g
+    a = torch.linspace(-30.0, 4.0, F, dtype=torch.float64)[torch.randperm(F, generator=gen)]
+    Wg = (a[:, None] * absn(F, D) * 1.25 / D).to(torch.bfloat16)
+    Wu = (torch.randn(F, D, generator=gen, dtype=torch.float64) / D ** 0.5).to(torch.bfloat16)
+    Wd = (torch.randn(D, F, generator=gen, dtype=torch.float64) / F ** 0.5).to(torch.bfloat16)
+
+    def sw(W):
+        WA = torch.randn(W.shape[1], k, generator=gen, dtype=torch.float64) / 16
+        WB = torch.randn(k, W.shape[0], generator=gen, dtype=torch.float64) / 16
+        return inputs.SpectralWeight(W=W, W_A=WA.to(torch.bfloat16), W_B=WB.to(torch.bfloat16), s=torch.ones(k))
+
+    zl = lambda do, di: (inputs.lora_pair(do, di, r, 0.02, gen)[0], torch.zeros(do, r, dtype=torch.bfloat16))
+    lg, lu, ld = zl(F, D), zl(F, D), zl(D, F)
+    dy = torch.randn(T, D, generator=gen).to(torch.bfloat16)
+    from contextual_sparsity_lora_b200 import blocks
+    with B.pair_tile_rows(tile_rows):
+        blk = blocks.FFNBlock(sw(Wg), sw(Wu), sw(Wd), lg, lu, ld, 2.0, k, T, C, 0.5, DEV)
+        blk.step(cu(x), cu(dy))
+        torch.cuda.synchronize()
+    assert blk.read_device_flag() == 0
+    idx = blk.sigma.cpu().numpy()[: blk.n_keep].astype(np.int64)
+    ctx = np.arange(T) < C
+    fwd = oracle.ffn_fwd(x, ctx, Wg, Wu, Wd, lg, lu, ld, 2.0, idx)
+    G = fwd["G"]
+    live = G != 0.0   # dropped context channels are exactly 0 (LoRA B = 0)
+    assert (G[live] < -8).mean() > 0.5, "most gates in the far negative tail"
+    h = unsigma(blk.h, blk.sigma, C)
+    rel = np.abs(h[live] - fwd["H"][live]) / np.abs(fwd["H"][live])
+    assert rel.max() < 2e-2, f"h: worst relative error {rel.max():.3g}"
+    # backward epilogue: the oracle's SwiGLU backward on the stored bf16 g and u, with the oracle's
+    # dh = dY W_down (sliced on the context rows; LoRA B = 0 adds nothing)
+    g16, u16 = unsigma(blk.g, blk.sigma, C), unsigma(blk.u, blk.sigma, C)
+    dH = oracle.sparse_linear_bwd(fwd["H"], dy, Wd, ld[0], ld[1], 2.0, ctx, idx, "in")[0]
+    rms = np.sqrt(np.mean(dH * dH))
+    for got, fac, name in ((unsigma(blk.dg, blk.sigma, C), u16 * oracle.silu_grad(g16), "dg"),
+                           (unsigma(blk.du, blk.sigma, C), oracle.silu(g16), "du")):
+        want = dH * fac
+        # 2e-2 relative, plus a floor for the fp32 accumulation error of dh where dh itself is ~0
+        bad = live & (np.abs(got - want) > 2e-2 * np.abs(want) + 1e-4 * np.abs(fac) * rms)
+        assert not bad.any(), f"{name}: {int(bad.sum())} elements outside tolerance"

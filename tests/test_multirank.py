@@ -142,11 +142,14 @@ def _ref_rank_main(rank, world, port, out):
     sys.path.insert(0, ROOT)
     import bench
 
-    sys.argv = ["bench.py", "--impl", "reference", "--gpus", str(world), "--steps", "1", "--warmup", "1"]
+    # no --gpus flag: the line's n_gpus is the launch's world size
+    sys.argv = ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"]
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         bench.main()
+    import torch.distributed as dist
     out[rank] = buf.getvalue()
+    out[f"group_left_{rank}"] = not dist.is_initialized()
 
 
 @pytest.mark.timeout(300)
@@ -163,3 +166,4 @@ def test_reference_arm_under_two_ranks_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert res["group_left_0"] and res["group_left_1"], "both ranks destroy the process group"

@@ -660,3 +660,149 @@ def test_sliced_weight_zeroes_the_dropped_channels():
     np.testing.assert_array_equal(out, np.array([[0, 0, 8], [1, 0, 9], [2, 0, 10], [3, 0, 11]], dtype=float))
     inn = oracle.sliced_weight(W, np.array([1, 3]), "in")
     np.testing.assert_array_equal(inn, np.array([[0, 0, 0], [1, 5, 9], [0, 0, 0], [3, 7, 11]], dtype=float))
+
+
+# ---------------------------------------------------------------------------
+# Closed forms of the decoder layer and of the model step: forward values that follow from the
+# layer's structure alone (pre-norm RMSNorm, residual connections from the layer input and from
+# the attention sum, causal attention within each sequence, SwiGLU, loss on the output rows), so
+# that a composition mistake mirrored in the backward still fails.
+# ---------------------------------------------------------------------------
+
+def _sign_rows(rng, T, D):
+    """Rows of +-1 entries: mean square exactly 1, so RMSNorm with eps = 0 and unit gain is the
+    identity on them."""
+    return rng.choice([-1.0, 1.0], size=(T, D))
+
+
+def _layer_weights(D, hq, hkv, hd, F, r, rng, zero=True):
+    Dq, Dkv = hq * hd, hkv * hd
+    shapes = {"q": (Dq, D), "k": (Dkv, D), "v": (Dkv, D), "o": (D, Dq), "gate": (F, D), "up": (F, D), "down": (D, F)}
+    w = {n: np.zeros(s) for n, s in shapes.items()}
+    # LoRA B = 0 (the adapter adds nothing), A random (its input path still runs)
+    lora = {n: (rng.standard_normal((r, s[1])), np.zeros((s[0], r))) for n, s in shapes.items()}
+    full = {"q": np.arange(Dq), "k": np.arange(Dkv), "v": np.arange(Dkv), "o": np.arange(Dq), "ffn": np.arange(F)}
+    return w, lora, full
+
+
+def test_decoder_layer_zero_projections_is_identity():
+    """Every frozen weight zero and every LoRA B zero: each branch adds exactly zero, so the layer
+    passes X through its two residual connections (Y = X) and the gradient through them
+    (dX = dY), for any gains and any index sets."""
+    rng = np.random.default_rng(61)
+    n_seq, S, D, hq, hkv, hd, F, r = 2, 4, 8, 2, 1, 4, 12, 2
+    T = n_seq * S
+    w, lora, _ = _layer_weights(D, hq, hkv, hd, F, r, rng)
+    gammas = (1.0 + 0.3 * rng.standard_normal(D), 1.0 + 0.3 * rng.standard_normal(D))
+    ctx = np.tile(np.array([True, True, True, False]), n_seq)
+    idx = {"q": np.array([1, 2, 5, 6]), "k": np.array([1, 2]), "v": np.array([0, 3]), "o": np.array([0, 3, 4, 7]),
+           "ffn": np.array([0, 1, 5, 6, 9, 10])}
+    X, dY = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+    res = oracle.decoder_layer(X, dY, ctx, n_seq, w, lora, gammas, 1e-5, 2.0, (hq, hkv, hd), 0.5, idx=dict(idx))
+    np.testing.assert_array_equal(res["Y"], X)
+    np.testing.assert_array_equal(res["dX"], dY)
+    for n in ("q", "k", "v", "o", "gate", "up", "down"):
+        np.testing.assert_array_equal(res["dA_" + n], 0.0)
+
+
+def test_decoder_layer_attention_branch_closed_form():
+    """Attention branch alone, MHA with D = heads x head_dim: W_q = W_k = 0 (uniform causal
+    weights), W_v = W_o = I, the FFN zero, every LoRA B zero, all channels kept. On rows of +-1
+    with eps = 0 and unit gains the pre-norm is the identity, so the layer is
+    Y_t = X_t + mean_{s <= t, same sequence} X_s. Its backward: with J_t = I - x_t x_t^T / D the
+    Jacobian of RMSNorm at such a row, dX_t = dY_t + J_t sum_{u >= t, same sequence} dY_u / (pos(u) + 1).
+    A post-norm layer, a residual taken after the norm, a non-causal or cross-sequence mask, or a
+    missing residual gives another Y."""
+    rng = np.random.default_rng(62)
+    n_seq, S, hq, hd, F, r = 2, 5, 2, 3, 4, 2
+    D = hq * hd
+    T = n_seq * S
+    w, lora, full = _layer_weights(D, hq, hq, hd, F, r, rng)
+    w["v"] = np.eye(D)
+    w["o"] = np.eye(D)
+    ones = (np.ones(D), np.ones(D))
+    ctx = np.tile(np.array([True, True, True, False, False]), n_seq)
+    X = _sign_rows(rng, T, D)
+    dY = rng.standard_normal((T, D))
+    res = oracle.decoder_layer(X, dY, ctx, n_seq, w, lora, ones, 0.0, 2.0, (hq, hq, hd), 1.0, idx=dict(full))
+    Y = np.empty_like(X)
+    dX = np.empty_like(X)
+    for b in range(n_seq):
+        for i in range(S):
+            t = b * S + i
+            Y[t] = X[t] + X[b * S:t + 1].sum(axis=0) / (i + 1)
+            acc = sum(dY[b * S + j] / (j + 1) for j in range(i, S))
+            J = np.eye(D) - np.outer(X[t], X[t]) / D
+            dX[t] = dY[t] + J @ acc
+    np.testing.assert_allclose(res["Y"], Y, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(res["dX"], dX, rtol=1e-12, atol=1e-12)
+
+
+def test_decoder_layer_ffn_branch_closed_form():
+    """FFN branch alone: attention weights zero, W_up = I, W_gate = c I, W_down = I (F = D), LoRA
+    B zero, all channels kept; rows of +-1, eps = 0, unit gains. Then Y = X + SiLU(c X) * X, and
+    for x = +-1 that is x + c * sigmoid(c x) (SiLU(c) for x = 1, -SiLU(-c) = c sigmoid(-c) for
+    x = -1)."""
+    rng = np.random.default_rng(63)
+    n_seq, S, D, hq, hkv, hd, r = 2, 3, 6, 2, 1, 3, 2
+    T = n_seq * S
+    c = 1.7
+    w, lora, full = _layer_weights(D, hq, hkv, hd, D, r, rng)
+    w["up"] = np.eye(D)
+    w["gate"] = c * np.eye(D)
+    w["down"] = np.eye(D)
+    ones = (np.ones(D), np.ones(D))
+    ctx = np.tile(np.array([True, True, False]), n_seq)
+    X = _sign_rows(rng, T, D)
+    res = oracle.decoder_layer(X, np.zeros((T, D)), ctx, n_seq, w, lora, ones, 0.0, 2.0, (hq, hkv, hd), 1.0,
+                               idx=dict(full))
+    want = X + c / (1.0 + np.exp(-c * X))
+    np.testing.assert_allclose(res["Y"], want, rtol=1e-14, atol=1e-14)
+
+
+def _identity_model(rng, n_layers, D, hq, hkv, hd, F, r):
+    layers = []
+    for _ in range(n_layers):
+        w, lora, full = _layer_weights(D, hq, hkv, hd, F, r, rng)
+        layers.append(dict(w=w, lora=lora, gammas=(1.0 + 0.2 * rng.standard_normal(D),) * 2, idx=full))
+    return layers
+
+
+def test_model_step_zero_head_loss_is_log_vocab():
+    """A zero LM head gives all-zero logits: the mean cross-entropy over the output rows is ln V
+    exactly, whatever the layers, ids and targets."""
+    rng = np.random.default_rng(64)
+    n_seq, S, D, hq, hkv, hd, F, r, V = 2, 4, 8, 2, 1, 4, 12, 2, 37
+    T = n_seq * S
+    layers = _identity_model(rng, 2, D, hq, hkv, hd, F, r)
+    for L in layers:  # non-trivial layers: the head alone fixes the loss
+        L["w"] = {n: 0.3 * rng.standard_normal(a.shape) for n, a in L["w"].items()}
+    ctx = np.tile(np.array([True, True, True, False]), n_seq)
+    embed = rng.standard_normal((V, D))
+    ids, tgt = rng.integers(0, V, T), rng.integers(0, V, int((~ctx).sum()))
+    loss, _ = oracle.model_step(ids, tgt, ctx, n_seq, embed, np.zeros((V, D)), np.ones(D), layers, 1e-5, 2.0,
+                                (hq, hkv, hd))
+    assert abs(loss - math.log(V)) < 1e-13
+
+
+def test_model_step_signed_one_hot_head_closed_form():
+    """Identity layers (zero weights, zero LoRA B), embedding rows of +-1, eps = 0 and unit final
+    gain make the final hidden state H_t = E[id_t] exactly. With V = 2 D and LM-head rows e_j
+    (v = j) and -e_j (v = D + j), every row's logits are D values +1 and D values -1, so
+    logsumexp = ln D + ln(e + 1/e); the loss is the mean over the output rows (in their order) of
+    that minus the target's logit +-H_t[j]."""
+    rng = np.random.default_rng(65)
+    n_seq, S, D, hq, hkv, hd, F, r = 2, 4, 6, 2, 1, 3, 8, 2
+    V = 2 * D
+    T = n_seq * S
+    layers = _identity_model(rng, 2, D, hq, hkv, hd, F, r)
+    ctx = np.tile(np.array([True, False, True, False]), n_seq)
+    embed = _sign_rows(rng, V, D)
+    head = np.concatenate([np.eye(D), -np.eye(D)])
+    ids = rng.integers(0, V, T)
+    out_rows = np.flatnonzero(~ctx)
+    tgt = rng.integers(0, V, out_rows.size)
+    loss, _ = oracle.model_step(ids, tgt, ctx, n_seq, embed, head, np.ones(D), layers, 0.0, 2.0, (hq, hkv, hd))
+    lse = math.log(D) + math.log(math.e + 1.0 / math.e)
+    want = np.mean([lse - (embed[ids[t], v] if v < D else -embed[ids[t], v - D]) for t, v in zip(out_rows, tgt)])
+    assert abs(loss - want) < 1e-13

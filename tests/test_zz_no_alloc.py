@@ -76,8 +76,35 @@ def _scores(case, fn):
     return outs
 
 
+def _other_library_work():
+    """Kernels of other entries first (a small FFN block step: estimator with a workspace,
+    selection, sparse GEMMs, LoRA backward), so the case where the fixed array follows other
+    work on the device is exercised inside this test, not only through collection order."""
+    import numpy as np  # noqa: F401
+    from contextual_sparsity_lora_b200 import blocks, inputs
+    T, C, D, F, r, k = 256, 192, 256, 512, 16, 8
+    gen = inputs.generator(9)
+    w = [inputs.spectral_weight(a, b, 0.5, k, gen, "cpu", torch.float64) for a, b in ((F, D), (F, D), (D, F))]
+    lo = [inputs.lora_pair(a, b, r, 0.02, gen) for a, b in ((F, D), (F, D), (D, F))]
+    blk = blocks.FFNBlock(*w, *lo, 2.0, k, T, C, 0.5, "cuda")
+    x = inputs.activations_student_t(T, D, 4, 0.01, 30.0, gen).cuda()
+    blk.step(x, torch.randn(T, D, generator=gen).to(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    assert blk.read_device_flag() == 0
+
+
+def _memory_state():
+    torch.cuda.synchronize()
+    free, _ = torch.cuda.mem_get_info()
+    return free, torch.cuda.memory_allocated(), torch.cuda.memory_reserved()
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_on_consecutive_calls():
+    """Scores equal to the workspace entry's, bit for bit, on calls in a row over new inputs and
+    differently sized scratch layouts; and the calls allocate nothing: device free memory (as the
+    driver reports it) and torch's allocator counters are unchanged across them."""
+    _other_library_work()
     ws = B.Workspace()
     flag = torch.full((1,), -1, dtype=torch.int32, device="cuda")
 
@@ -91,18 +118,41 @@ def test_noalloc_matches_workspace_entry_on_consecutive_calls():
         needed.append(B.sl_svd_estimate_noalloc(crit, x, n_ctx, w_a, w_b, k, s, scores_v=sv, n_q_heads=hq,
                                                 n_kv_heads=hkv, head_dim=hd, device_flag=flag))
 
-    # consecutive calls on new inputs and differently sized scratch layouts
     cases = [_ffn_case(1), _attn_case(2), _ffn_case(3), _l2_fp32_case(4), _attn_case(5)]
-    for case in cases:
-        got = _scores(case, no_alloc)
-        torch.cuda.synchronize()
-        assert int(flag.item()) == 0
-        want = _scores(case, with_ws)
-        torch.cuda.synchronize()
-        for g_, w_ in zip(got, want):
-            assert torch.isfinite(g_).all()
-            assert _rel(g_, w_) < FP32_TOL
-            assert torch.equal(g_, w_)  # same kernels, fixed-order sums
-        flag.fill_(-1)
+    wants = [_scores(c, with_ws) for c in cases]
+    outs = [[torch.full((n,), float("nan"), device="cuda") for n in c["outs"]] for c in cases]
+
+    def run(case, out):
+        for o in out:
+            o.fill_(float("nan"))
+        hq, hkv, hd = case["heads"]
+        no_alloc(case["crit"], case["x"], case["n_ctx"], case["w_a"], case["w_b"], case["k"], out[0],
+                 out[1] if len(out) > 1 else None, hq, hkv, hd)
+
+    # first round: every kernel involved has been loaded and run once
+    for case, out in zip(cases, outs):
+        run(case, out)
+    # two more rounds of consecutive calls on the shared array; the results and device flags are
+    # copied into buffers allocated beforehand, and compared only after the second snapshot, so
+    # that nothing in between allocates on the test's side either
+    kept = [[[torch.empty_like(o) for o in out] for out in outs] for _ in range(2)]
+    flags = torch.full((2, len(cases)), -1, dtype=torch.int32, device="cuda")
+    before = _memory_state()
+    for rep in range(2):
+        for i, (case, out) in enumerate(zip(cases, outs)):
+            flag.fill_(-1)
+            run(case, out)
+            flags[rep, i].copy_(flag[0])
+            for dst, src in zip(kept[rep][i], out):
+                dst.copy_(src)
+    after = _memory_state()
+    assert after == before, f"memory changed across the calls: {before} -> {after}"
+    assert bool((flags == 0).all()), f"device flags {flags.tolist()}"
+    for rep in range(2):
+        for got, want in zip(kept[rep], wants):
+            for g_, w_ in zip(got, want):
+                assert torch.isfinite(g_).all()
+                assert _rel(g_, w_) < FP32_TOL
+                assert torch.equal(g_, w_)  # same kernels, fixed-order sums
     assert all(0 < n <= 8 << 20 for n in needed)
     assert len(set(needed)) > 1
