@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-LoRA companion measurement")
     ap.add_argument("--no-layer", action="store_true", help="skip the whole-decoder-layer measurement")
     ap.add_argument("--no-model", action="store_true", help="skip the 32-layer fine-tuning run")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the keep-ratio sweep and the LLaMA2-13B layer")
     ap.add_argument("--stages-only", action="store_true",
                     help="time only the selection stages (estimator, criterion, top-n, compaction) of both blocks "
                          "and print them; no step, no headline line")
@@ -101,63 +102,90 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled every `interval` seconds while the
+    timed region runs, read-only through NVML (nvidia-smi's query loop as the fallback)."""
 
-    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
-             "clocks_event_reasons.sw_power_cap"
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
-    def __init__(self, index):
+    def __init__(self, index, interval=0.005):
         self.index = index
-        self.samples = []
+        self.interval = interval
+        self.samples = []   # (sm_mhz, max_mhz, reasons bitmask)
+        self.source = None
+        self._stop = threading.Event()
+        self.thread = None
         self.proc = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                             int(get_reasons(h))))
+                    except Exception:
+                        pass
+                    self._stop.wait(self.interval)
+            self.source = f"NVML every {self.interval * 1e3:.0f} ms"
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+        except Exception:
+            self._start_smi()
+        return self
+
+    def _start_smi(self):
+        fields = "clocks.sm,clocks.max.sm,clocks_event_reasons.active"
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={fields}",
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi -lms 20"
+
+            def read():
+                for line in self.proc.stdout:
+                    parts = [q.strip() for q in line.split(",")]
+                    try:
+                        self.samples.append((float(parts[0]), float(parts[1]), int(parts[2], 16)))
+                    except Exception:
+                        pass
+            self.thread = threading.Thread(target=read, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
-        return self
-
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
 
     def __exit__(self, *a):
+        self._stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = sorted(float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit())
-        mx = max(float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for s in self.samples:
-            for i, n in enumerate(names):
-                if s[5 + i].lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = sorted(float(x[0]) for x in self.samples)
+        reasons = sorted({name for x in self.samples for bit, name in self.REASONS.items() if x[2] & bit})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_min_mhz": sm[0], "sm_max_mhz": max(float(x[1]) for x in self.samples),
+                "reasons": reasons, "samples": len(self.samples), "source": self.source}
 
 
-def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None):
-    """The two blocks of one LLaMA3-8B layer plus their per-step inputs (context-first rows).
-    dp: a blocks.DataParallel over the ranks (one index set per global batch), or None."""
+def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None, cfgs=None):
+    """The two blocks of one layer (LLaMA3-8B unless `cfgs` = (attention config, FFN config))
+    plus their per-step inputs (context-first rows). dp: a blocks.DataParallel over the ranks
+    (one index set per global batch), or None."""
     from contextual_sparsity_lora_b200 import blocks
-    ac = inputs.LLAMA3_8B_ATTN
-    fc = inputs.LLAMA3_8B_FFN
+    ac, fc = cfgs if cfgs else (inputs.LLAMA3_8B_ATTN, inputs.LLAMA3_8B_FFN)
     da = inputs.make_attn_inputs(ac, seed_w, device=device)
     df = inputs.make_ffn_inputs(fc, seed_w + 1, device=device)
     perm = inputs.context_first_order(da["ctx_mask"])
@@ -219,8 +247,29 @@ def capture_graph(fn, warm=True):
 # launches of one step of this workload, from an ncu capture of one step's CTA-pair launches
 # (dram__bytes_read.sum + dram__bytes_write.sum: 3014.7 MB per step). Valid for the kernel
 # as captured; to be set to None when the kernel changes.
-PAIR_DRAM_BYTES_PER_LAUNCH = 3014.7e6 / 8
+PAIR_DRAM_BYTES_PER_LAUNCH = 3009.4e6 / 8
 PAIR_DRAM_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of the step's 8 launches"
+# SHA-256 (first 16 hex digits) of the sources that define gemm_pair_kernel, as they were when the
+# figure above was captured; when the sources differ the figure is stale and is reported as null.
+PAIR_DRAM_SOURCES = ("sl_gemm.cu", "sl_gemm.h", "sl_ptx.cuh", "sl_internal.h")
+PAIR_DRAM_SOURCE_SHA = "8fb721552cbb1aa7"
+
+
+def pair_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in PAIR_DRAM_SOURCES:
+        with open(os.path.join(ROOT, "contextual_sparsity_lora_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def pair_traffic():
+    """(bytes per launch or None, source note) for the roofline's traffic key."""
+    sha = pair_sources_sha()
+    if sha == PAIR_DRAM_SOURCE_SHA:
+        return PAIR_DRAM_BYTES_PER_LAUNCH, f"{PAIR_DRAM_SOURCE} (sources {sha})"
+    return None, f"no capture of the current kernel sources ({sha}); the last capture was of {PAIR_DRAM_SOURCE_SHA}"
 
 
 def capture_or_eager(fn, world):
@@ -402,7 +451,7 @@ def cpu_baseline(da, df, ratio, n_tokens=512, n_seqs=1):
         _oracle_layer(oracle, X, XO, dq, dk, dv, dyo, Xf, dyf, ctx, W, F, L, Wf, Ff, Lf, s, ac, ratio)
     dt = time.perf_counter() - t0
     S = S * n_seqs
-    return {"value": S / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+    return {"value": S / dt, "unit": UNIT, "cores": int(threads), "blas_threads": int(threads), "kind": "oracle",
             "sample": f"{S} tokens ({n_seqs} x {S // n_seqs} of one sequence, {int(ctx.sum())} context + "
                       f"{S // n_seqs - int(ctx.sum())} output each) through both blocks, fp64 NumPy, {dt:.1f} s",
             "seconds": dt, "host_cpus": os.cpu_count()}
@@ -508,30 +557,161 @@ def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
             "layer": "RMSNorm, sparse q/k/v, attention, sparse o, residual, RMSNorm, sparse SwiGLU FFN, residual"}
 
 
-def e2e_measure(attn, ffn, step_in, K, W, world, device):
-    """Same step through the public API with host buffers: every step copies that step's
-    inputs from pinned host memory and reads the LoRA gradients back."""
+def e2e_measure(attn, ffn, step_in, K, W, world, device, eager=False):
+    """Same step through the public API with host buffers: every step copies that step's inputs
+    from pinned host memory and reads the LoRA gradients back. The copies run on a second stream
+    and are double-buffered: the inputs of step i+1 go into one device buffer while step i
+    computes on the other, and the gradients of step i (snapshotted on the device) return to the
+    host during step i+1. eager=False replays one captured graph of the step per input buffer;
+    eager=True calls the library entries step by step (the host-side cost of every ABI call:
+    argument checks, tensor-map encoding, marshalling, launches) with the same copies.
+    Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
     host = {k: v.cpu().pin_memory() for k, v in step_in.items()}
-    dev_in = {k: torch.empty_like(v) for k, v in step_in.items()}
+    bufs = [{k: torch.empty_like(v) for k, v in step_in.items()} for _ in range(2)]
     grads = [attn.dA[n] for n in "qkvo"] + [attn.dB[n] for n in "qkvo"] + \
         [ffn.dA_g, ffn.dB_g, ffn.dA_u, ffn.dB_u, ffn.dA_d, ffn.dB_d]
+    snap = [torch.empty_like(g) for g in grads]
     host_out = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(g.numel() * g.element_size() for g in grads)
-
+    for b in bufs:
+        for k in host:
+            b[k].copy_(host[k])
     for _ in range(2):
-        run_step(attn, ffn, dev_in)
-    replay, _ = capture_or_eager(lambda: run_step(attn, ffn, dev_in), world)
+        run_step(attn, ffn, bufs[0])
+    torch.cuda.synchronize()
+    if eager:
+        replays = [(lambda b=b: run_step(attn, ffn, b)) for b in bufs]
+    else:
+        replays = [capture_or_eager(lambda b=b: run_step(attn, ffn, b), world)[0] for b in bufs]
+    main = torch.cuda.current_stream()
+    h2d_s = torch.cuda.Stream(device=device)   # inputs in
+    d2h_s = torch.cuda.Stream(device=device)   # gradients out (its own stream: the two directions overlap)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer j have landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # the step that read buffer j has finished
+    ev_snap, ev_out = torch.cuda.Event(), torch.cuda.Event()
+    for e in ev_in + ev_done + [ev_out]:
+        e.record(main)
+    state = {"i": 0}
 
     def step():
-        for k in host:
-            dev_in[k].copy_(host[k], non_blocking=True)
-        replay()
-        for h, g in zip(host_out, grads):
-            h.copy_(g, non_blocking=True)
+        j = state["i"] % 2
+        with torch.cuda.stream(h2d_s):     # step i+1's inputs into the other buffer, during step i
+            h2d_s.wait_event(ev_done[1 - j])   # the buffer is free once the step that read it finished
+            for k in host:
+                bufs[1 - j][k].copy_(host[k], non_blocking=True)
+            ev_in[1 - j].record(h2d_s)
+        main.wait_event(ev_in[j])
+        replays[j]()
+        ev_done[j].record(main)
+        main.wait_event(ev_out)            # the previous step's gradients have left the snapshot
+        for d, g in zip(snap, grads):
+            d.copy_(g)
+        ev_snap.record(main)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_snap)
+            for h, d in zip(host_out, snap):
+                h.copy_(d, non_blocking=True)
+            ev_out.record(d2h_s)
+        state["i"] += 1
 
-    ms = time_steps(step, K, W, world, device)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for _ in range(K):
+        step()
+    main.wait_stream(h2d_s)                # the last step's copies belong to the timed region
+    main.wait_stream(d2h_s)
+    e1.record(main)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    barrier(world)
     return ms / K, h2d, d2h
+
+
+def sweep_measure(device, K, W):
+    """Keep-ratio sweep of the LLaMA3-8B workload (the pages' operating points at several
+    sparsities): for keep 1.0 (dense LoRA on the same kernels, no estimator), 0.7, 0.5 and 0.3,
+    the FFN block alone and the whole 7-projection step, each one CUDA graph replayed K times."""
+    out = {}
+    ac, fc = inputs.LLAMA3_8B_ATTN, inputs.LLAMA3_8B_FFN
+    for ratio in (1.0, 0.7, 0.5, 0.3):
+        attn, ffn, s_in, C, _, _ = make_layer(ratio, 0, 1000, device, dense=ratio >= 1.0)
+        for _ in range(3):
+            run_step(attn, ffn, s_in)
+        torch.cuda.synchronize()
+        g_all = capture_graph(lambda: run_step(attn, ffn, s_in), warm=False)
+        ms_all = time_steps(g_all.replay, K, W, 1, device) / K
+        del g_all
+        g_ffn = capture_graph(lambda: ffn.step(s_in["ffn_x"], s_in["ffn_dy"]), warm=False)
+        ms_ffn = time_steps(g_ffn.replay, K, W, 1, device) / K
+        del g_ffn
+        fl = algorithmic_flops(ac, fc, C, ratio, dense=ratio >= 1.0)
+        nk = fc.inter if ratio >= 1.0 else inputs_keep(ratio, fc.inter)
+        f = flops.ffn_block(fc.hidden, fc.inter, fc.n_tok, C, nk, fc.r, fc.k, with_estimator=ratio < 1.0)
+        out[f"keep{ratio}"] = {"step_ms": ms_all, "step_tokens_per_s": ac.n_tok / (ms_all / 1e3),
+                               "step_effective_tflops": fl["total"] / (ms_all / 1e3) / 1e12,
+                               "ffn_ms": ms_ffn, "ffn_tokens_per_s": fc.n_tok / (ms_ffn / 1e3),
+                               "ffn_effective_tflops": f["total"] / (ms_ffn / 1e3) / 1e12}
+        del attn, ffn, s_in
+        torch.cuda.synchronize()
+    out["workload"] = "LLaMA3-8B, 8 x 512 tokens (last 128 output), LoRA rank 32, estimator rank 8"
+    return out
+
+
+def llama2_13b_measure(device, K, W):
+    """The LLaMA2-13B layer's seven projections (4 x 1024 tokens, last 256 output; MHA 40 x 128,
+    FFN 13824; LoRA rank 32, estimator rank 16) at keep 0.4, and densely (keep 1, no estimator)."""
+    ac, fc = inputs.LLAMA2_13B_ATTN, inputs.LLAMA2_13B_FFN
+    res = {}
+    for name, ratio, dense in (("sparse", ac.ratio, False), ("dense_lora", 1.0, True)):
+        attn, ffn, s_in, C, _, _ = make_layer(ratio, 0, 1000, device, dense=dense, cfgs=(ac, fc))
+        for _ in range(3):
+            run_step(attn, ffn, s_in)
+        torch.cuda.synchronize()
+        g = capture_graph(lambda: run_step(attn, ffn, s_in), warm=False)
+        ms = time_steps(g.replay, K, W, 1, device) / K
+        fl = algorithmic_flops(ac, fc, C, ratio, dense=dense)
+        res[name] = {"ms_per_step": ms, "tokens_per_s": ac.n_tok / (ms / 1e3),
+                     "effective_tflops": fl["total"] / (ms / 1e3) / 1e12,
+                     "algorithmic_tflop_per_step": fl["total"] / 1e12}
+        del g, attn, ffn, s_in
+        torch.cuda.synchronize()
+    res["speedup_vs_dense_lora"] = res["dense_lora"]["ms_per_step"] / res["sparse"]["ms_per_step"]
+    res["workload"] = "llama2-13b-layer-7proj-b4s1024-keep0.4-k16"
+    return res
+
+
+def cpu_tiny_single_core(repeats=3):
+    """The fp64 oracle on one host thread (BLAS limited to one thread) for the tiny fp32 FFN
+    configuration (hidden 256, FFN 688, 2 x 64 tokens, last 16 output, LoRA rank 8, estimator
+    rank 8, keep 0.5): estimator, selection, forward and backward of the block."""
+    import numpy as np
+    import oracle
+    from threadpoolctl import threadpool_limits
+    cfg = inputs.TINY_FFN
+    d = inputs.make_ffn_inputs(cfg, seed=0, device="cpu")
+    ctx = d["ctx_mask"].numpy()
+    X, dY = oracle.f64(d["x"]), oracle.f64(d["dy"])
+    W = {n: oracle.f64(d[n].W) for n in ("gate", "up", "down")}
+    Fa = {n: (oracle.f64(d[n].W_A), oracle.f64(d[n].W_B)) for n in ("gate", "up")}
+    L = {n: (oracle.f64(d["lora_" + n][0]), oracle.f64(d["lora_" + n][1])) for n in ("gate", "up", "down")}
+    times = []
+    with threadpool_limits(limits=1):
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            _, idx = oracle.ffn_select(X, ctx, Fa["gate"], Fa["up"], cfg.ratio)
+            fwd = oracle.ffn_fwd(X, ctx, W["gate"], W["up"], W["down"], L["gate"], L["up"], L["down"],
+                                 cfg.lora_scale, idx)
+            oracle.ffn_bwd(X, dY, ctx, W["gate"], W["up"], W["down"], L["gate"], L["up"], L["down"],
+                           cfg.lora_scale, idx, fwd=fwd)
+            times.append(time.perf_counter() - t0)
+    t = min(times)
+    return {"value": cfg.n_tok / t, "unit": UNIT, "seconds": t, "threads": 1, "blas_threads": 1,
+            "workload": cfg.name, "repeats": repeats, "np_version": np.__version__}
 
 
 def reference_arm(args, rank, world):
@@ -648,7 +828,9 @@ def main():
     # are HBM-bound and reported apart
     pair_flops = fl["main"] + fl["lora"] / 3.0
     peaks, src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak = float(peaks.get("bf16_tflops"))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    traffic, traffic_src = pair_traffic()
     achieved = pair_flops / (pair_ms / 1e3) / 1e12 if pair_ms > 0 else None
     skinny_bytes = flops.lora_skinny_bytes([(T, ac.hidden, (ac.n_q_heads * ac.head_dim, 2 * ac.n_kv_heads * ac.head_dim)),
                                             (T, ac.n_q_heads * ac.head_dim, (ac.hidden,)),
@@ -668,8 +850,10 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "sl::gemm_pair_kernel (CTA-pair tcgen05 GEMM: sliced products)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None,
-                     "traffic": PAIR_DRAM_BYTES_PER_LAUNCH, "traffic_source": PAIR_DRAM_SOURCE,
-                     "peak_source": f"{src} bf16_tflops_sustained",
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "peak_source": f"{src} bf16_tflops (burst: the step's timed region lasts well under the "
+                                    f"seconds-long loop of the sustained figure)",
+                     "frac_of_sustained": (achieved / peak_sus) if achieved else None,
                      "algorithmic_tflop_per_launch": pair_flops / 1e12 / max(pair_n, 1),
                      "launches_per_step": pair_n, "ms_per_launch": pair_ms / max(pair_n, 1),
                      "gemm_engine_ms_per_step": gemm_ms, "gemm_engine_launches_per_step": n_gemm,
@@ -718,13 +902,26 @@ def main():
         line["model_32_layers_math10k_table"] = m10
     if world == 1 and not args.no_layer:
         line["full_layer"] = full_layer_measure(attn, ffn, step_in, perm, ac, args.steps, max(args.warmup, 3), device)
+    if world == 1 and not args.no_sweep:
+        line["sweep"] = sweep_measure(device, args.steps, max(args.warmup, 3))
+        line["llama2_13b_layer"] = llama2_13b_measure(device, args.steps, max(args.warmup, 3))
     if not args.no_e2e:
+        how = ("inputs from pinned host memory on a copy stream into two device buffers (step i+1's copy "
+               "overlaps step i), LoRA gradients snapshotted on the device and read back on a third stream "
+               "during the next step")
         e2e_ms, h2d, d2h = e2e_measure(attn, ffn, step_in, args.steps, max(args.warmup, 3), world, device)
         line["e2e"] = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "copies": how,
+                       "step": "one CUDA graph of the step per input buffer"}
+        ee_ms, _, _ = e2e_measure(attn, ffn, step_in, args.steps, max(args.warmup, 3), world, device, eager=True)
+        line["e2e_eager"] = {"value": world * T / (ee_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                             "d2h_bytes_per_step": d2h, "ms_per_step": ee_ms, "copies": how,
+                             "step": "every library entry called from Python per step (no graph): argument "
+                                     "checks, tensor-map encoding and ctypes marshalling included"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(da, df, args.ratio, n_tokens=512, n_seqs=3).items()
                                 if k != "seconds"}
+        line["cpu_baseline"]["single_core_tiny_ffn"] = cpu_tiny_single_core()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -30,7 +30,8 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_sparse_linear_bwd", "sl_prepare_weight", "sl_permute_rows", "sl_profile_enable", "sl_profile_read",
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
-            "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows")
+            "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows",
+            "sl_debug_bounds_enabled", "sl_read_debug_flag")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -53,63 +54,93 @@ class SparseLoRAError(RuntimeError):
         super().__init__(f"{fn} failed: {status_string(code)} (status {code})")
 
 
+DEBUG_LIB_PATH = os.path.join(_HERE, "libsparselora_debug.so")
+
 _lib = None
 
 
 def lib():
+    """The library every wrapper below calls (the in-tree release build unless `using_library`
+    selected another one)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m contextual_sparsity_lora_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        P = c_void_p
-        L.sl_status_string.restype = c_char_p
-        L.sl_status_string.argtypes = [c_int32]
-        L.sl_version.restype = c_int32
-        L.sl_keep_count.restype = c_int64
-        L.sl_keep_count.argtypes = [c_double, c_int64]
-        L.sl_workspace_init.argtypes = [POINTER(SlWorkspaceC), P]
-        L.sl_read_device_flag.argtypes = [POINTER(SlWorkspaceC), POINTER(c_int32), P]
-        L.sl_svd_estimate.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p),
-                                      POINTER(c_void_p), POINTER(c_int64), c_int32, c_int32, c_int32, c_int32, P, P,
-                                      POINTER(SlWorkspaceC), P]
-        L.sl_svd_partials_count.restype = c_int64
-        L.sl_svd_partials_count.argtypes = [c_int32, c_int32, POINTER(c_int64), c_int32]
-        L.sl_svd_estimate_partials.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32,
-                                               POINTER(c_void_p), POINTER(c_void_p), POINTER(c_int64), c_int32,
-                                               c_int32, c_int32, c_int32, P, POINTER(SlWorkspaceC), P]
-        L.sl_svd_scores_from_partials.argtypes = [c_int32, c_int32, c_int32, POINTER(c_void_p), POINTER(c_int64),
-                                                  c_int32, c_int32, c_int32, c_int32, P, P, P, P]
-        L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
-        L.sl_select_heads.argtypes = [P, c_int32, c_int32, c_int32, c_int32, P, P, P]
-        L.sl_rmsnorm_fwd.argtypes = [P, c_int64, P, c_int64, P, c_int64, P, c_float, P, c_int64, P, c_int64, c_int64, P]
-        L.sl_rmsnorm_bwd.argtypes = [P, c_int64, P, c_int64, P, P, P, c_int64, P, c_int64, c_int64, c_int64, P]
-        L.sl_add_rows.argtypes = [P, c_int64, P, c_int64, P, c_int64, c_int64, c_int64, P]
-        L.sl_adamw_step.argtypes = [P, P, P, P, P, c_int64, c_float, c_float, c_float, c_float, c_float, c_int32, P]
-        L.sl_wanda_scores.argtypes = [P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p), c_int64, c_int64, P,
-                                      POINTER(SlWorkspaceC), P]
-        L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
-                                      POINTER(SlChannelsC), P, P, c_int64, POINTER(c_void_p), POINTER(c_int64),
-                                      c_int32, POINTER(SlChannelsC), POINTER(c_void_p), POINTER(c_void_p),
-                                      POINTER(c_void_p), POINTER(c_void_p), POINTER(SlWorkspaceC), P]
-        L.sl_sparse_linear_fwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32, P, c_int64,
-                                           c_int64, c_int64, c_int32, c_int32, P, c_int64, POINTER(c_void_p),
-                                           POINTER(c_int64), POINTER(SlWorkspaceC), P]
-        L.sl_sparse_linear_bwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32,
-                                           POINTER(c_void_p), POINTER(c_int64), c_int64, c_int64, c_int32, c_int32,
-                                           POINTER(c_void_p), P, c_int64, POINTER(c_void_p), POINTER(c_void_p),
-                                           POINTER(SlWorkspaceC), P]
-        L.sl_prepare_weight.argtypes = [P, c_int64, c_int64, P, P]
-        L.sl_profile_enable.argtypes = [c_int32]
-        L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
-        L.sl_permute_rows.argtypes = [P, c_int64, P, c_int64, c_int64, P, c_int64, P]
-        L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P]
-        L.sl_set_pair_tile_rows.argtypes = [c_int32]
-        for n in EXPORTED:
-            if n not in ("sl_status_string", "sl_version", "sl_keep_count", "sl_svd_partials_count"):
-                getattr(L, n).restype = c_int32
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+class using_library:
+    """Context manager: the wrappers call the library at `path` (e.g. DEBUG_LIB_PATH, the build
+    with device-side bounds checks) inside the block."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = load(self.path)
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+
+
+def load(path):
+    """Load a build of the library and declare its entry points' argument types."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m contextual_sparsity_lora_b200.build`")
+    L = ctypes.CDLL(path)
+    P = c_void_p
+    L.sl_status_string.restype = c_char_p
+    L.sl_status_string.argtypes = [c_int32]
+    L.sl_version.restype = c_int32
+    L.sl_keep_count.restype = c_int64
+    L.sl_keep_count.argtypes = [c_double, c_int64]
+    L.sl_workspace_init.argtypes = [POINTER(SlWorkspaceC), P]
+    L.sl_read_device_flag.argtypes = [POINTER(SlWorkspaceC), POINTER(c_int32), P]
+    L.sl_svd_estimate.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p),
+                                  POINTER(c_void_p), POINTER(c_int64), c_int32, c_int32, c_int32, c_int32, P, P,
+                                  POINTER(SlWorkspaceC), P]
+    L.sl_svd_partials_count.restype = c_int64
+    L.sl_svd_partials_count.argtypes = [c_int32, c_int32, POINTER(c_int64), c_int32]
+    L.sl_svd_estimate_partials.argtypes = [c_int32, c_int32, P, c_int64, c_int64, c_int64, c_int32,
+                                           POINTER(c_void_p), POINTER(c_void_p), POINTER(c_int64), c_int32,
+                                           c_int32, c_int32, c_int32, P, POINTER(SlWorkspaceC), P]
+    L.sl_svd_scores_from_partials.argtypes = [c_int32, c_int32, c_int32, POINTER(c_void_p), POINTER(c_int64),
+                                              c_int32, c_int32, c_int32, c_int32, P, P, P, P]
+    L.sl_select_channels.argtypes = [P, c_int64, c_int64, P, c_int32, c_int32, P, P]
+    L.sl_select_heads.argtypes = [P, c_int32, c_int32, c_int32, c_int32, P, P, P]
+    L.sl_rmsnorm_fwd.argtypes = [P, c_int64, P, c_int64, P, c_int64, P, c_float, P, c_int64, P, c_int64, c_int64, P]
+    L.sl_rmsnorm_bwd.argtypes = [P, c_int64, P, c_int64, P, P, P, c_int64, P, c_int64, c_int64, c_int64, P]
+    L.sl_add_rows.argtypes = [P, c_int64, P, c_int64, P, c_int64, c_int64, c_int64, P]
+    L.sl_adamw_step.argtypes = [P, P, P, P, P, c_int64, c_float, c_float, c_float, c_float, c_float, c_int32, P]
+    L.sl_wanda_scores.argtypes = [P, c_int64, c_int64, c_int64, c_int32, POINTER(c_void_p), c_int64, c_int64, P,
+                                  POINTER(SlWorkspaceC), P]
+    L.sl_lora_fwd_bwd.argtypes = [c_int32, c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, c_int32,
+                                  POINTER(SlChannelsC), P, P, c_int64, POINTER(c_void_p), POINTER(c_int64),
+                                  c_int32, POINTER(SlChannelsC), POINTER(c_void_p), POINTER(c_void_p),
+                                  POINTER(c_void_p), POINTER(c_void_p), POINTER(SlWorkspaceC), P]
+    L.sl_sparse_linear_fwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32, P, c_int64,
+                                       c_int64, c_int64, c_int32, c_int32, P, c_int64, POINTER(c_void_p),
+                                       POINTER(c_int64), POINTER(SlWorkspaceC), P]
+    L.sl_sparse_linear_bwd.argtypes = [c_int32, POINTER(SlLinearC), POINTER(SlChannelsC), c_int32,
+                                       POINTER(c_void_p), POINTER(c_int64), c_int64, c_int64, c_int32, c_int32,
+                                       POINTER(c_void_p), P, c_int64, POINTER(c_void_p), POINTER(c_void_p),
+                                       POINTER(SlWorkspaceC), P]
+    L.sl_prepare_weight.argtypes = [P, c_int64, c_int64, P, P]
+    L.sl_profile_enable.argtypes = [c_int32]
+    L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
+    L.sl_permute_rows.argtypes = [P, c_int64, c_int64, P, c_int64, c_int64, P, c_int64, P]
+    L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P, P]
+    L.sl_debug_bounds_enabled.restype = c_int32
+    L.sl_read_debug_flag.argtypes = [POINTER(c_int32), P]
+    L.sl_set_pair_tile_rows.argtypes = [c_int32]
+    for n in EXPORTED:
+        if n not in ("sl_status_string", "sl_version", "sl_keep_count", "sl_svd_partials_count",
+                     "sl_debug_bounds_enabled"):
+            getattr(L, n).restype = c_int32
+    return L
 
 
 def status_string(code: int) -> str:
@@ -317,7 +348,8 @@ def sl_prepare_weight(w, w_t):
 
 
 def sl_permute_rows(src, perm, dst):
-    _check("sl_permute_rows", lib().sl_permute_rows(_ptr(src), src.stride(0), _ptr(perm), perm.numel(),
+    """dst[i, :] = src[perm[i], :] for i < perm.numel() (src may have more rows than dst)."""
+    _check("sl_permute_rows", lib().sl_permute_rows(_ptr(src), src.stride(0), src.shape[0], _ptr(perm), perm.numel(),
                                                     src.shape[1], _ptr(dst), dst.stride(0), _stream()))
 
 
@@ -326,8 +358,23 @@ def sl_gather_rows_batch(srcs, perms, dsts):
     perm_q holds one int32 index per row of dst_q."""
     n = len(srcs)
     _check("sl_gather_rows_batch", lib().sl_gather_rows_batch(
-        n, _ptrs(srcs), _i64s([t.stride(0) for t in srcs]), _ptrs(perms), _i64s([t.numel() for t in perms]),
-        _i64s([t.shape[1] for t in srcs]), _ptrs(dsts), _i64s([t.stride(0) for t in dsts]), _stream()))
+        n, _ptrs(srcs), _i64s([t.stride(0) for t in srcs]), _i64s([t.shape[0] for t in srcs]), _ptrs(perms),
+        _i64s([t.numel() for t in perms]), _i64s([t.shape[1] for t in srcs]), _ptrs(dsts),
+        _i64s([t.stride(0) for t in dsts]), _stream()))
+
+
+def sl_debug_bounds_enabled() -> bool:
+    return bool(lib().sl_debug_bounds_enabled())
+
+
+def sl_read_debug_flag() -> int:
+    """Code recorded by a failed bounds check of the entries without a workspace (debug build),
+    cleared by the read; 0 when none (always 0 in the release build). Synchronises."""
+    code = c_int32(0)
+    rc = lib().sl_read_debug_flag(ctypes.byref(code), _stream())
+    if rc not in (SL_OK, SL_ERR_DEVICE_FLAG):
+        _check("sl_read_debug_flag", rc)
+    return int(code.value)
 
 
 def sl_set_pair_tile_rows(rows: int):

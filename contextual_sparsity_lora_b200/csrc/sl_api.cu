@@ -499,7 +499,7 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
     carve(c, asig, &region);
     if (in_sig)
       for (int i = 0; i < n_ad; ++i)
-        if (int rc = gather_cols_bf16(lin[i].lora_a, d_in, lin[i].r, in_ch->sigma, d_in, asig[i], d_in, s))
+        if (int rc = gather_cols_bf16(lin[i].lora_a, d_in, d_in, lin[i].r, in_ch->sigma, d_in, asig[i], d_in, err_word(ws), s))
           return from_kernel(rc);
     GemmBuilder gb;
     int64_t off = 0;
@@ -580,8 +580,8 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   if (out_sig) {
     GatherBatch gat;
     for (int i = 0; i < n_ad; ++i)
-      gat.add(lin[i].lora_b, lin[i].r, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i], lin[i].r);
-    if (int rc = gat.launch(s)) return from_kernel(rc);
+      gat.add(lin[i].lora_b, lin[i].r, lin[i].d_out, out_ch[i].sigma, lin[i].d_out, lin[i].r, bsig[i], lin[i].r);
+    if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
   }
   // dya = scale * dy B and dB = dy^T xa_s from one pass over each dy (fused kernel; context rows
   // of a sigma-layout dy use the permuted B and land in dB rows sigma[p]), then dya_s = bf16(dya)
@@ -727,10 +727,10 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
       else
-        gat.add(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
-      gat.add(lin[i].lora_b, lin[i].r, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r);
+        gat.add(lin[i].w, d_in, lin[i].d_out, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
+      gat.add(lin[i].lora_b, lin[i].r, lin[i].d_out, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r);
     }
-    if (int rc = gat.launch(s)) return from_kernel(rc);
+    if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
     GemmBuilder gb;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     int koff = 0;
@@ -795,17 +795,17 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
       else
-        gat.add(lin[i].w, d_in, sig, ch[0].n_keep, d_in, wc[i], d_in);
+        gat.add(lin[i].w, d_in, lin[i].d_out, sig, ch[0].n_keep, d_in, wc[i], d_in);
     }
     // LoRA B operand of a paired tile t: rows 256 t + j = [B_gate[c_j] | 0], rows 256 t + 128 + j = [0 | B_up[c_j]]
     cudaMemsetAsync(pk[0], 0, (size_t)nt * 256 * 64 * 2, s);
     cudaMemsetAsync(pk[1], 0, (size_t)nt * 256 * 64 * 2, s);
     for (int v = 0; v < 2; ++v) {
       const int32_t* idx = v == 0 ? sig : nullptr;
-      gat.add(lin[0].lora_b, lin[0].r, idx, F, lin[0].r, pk[v], 64, 0, 128, 256, 0);
-      gat.add(lin[1].lora_b, lin[1].r, idx, F, lin[1].r, pk[v], 64, lin[0].r, 128, 256, 128);
+      gat.add(lin[0].lora_b, lin[0].r, F, idx, F, lin[0].r, pk[v], 64, 0, 128, 256, 0);
+      gat.add(lin[1].lora_b, lin[1].r, F, idx, F, lin[1].r, pk[v], 64, lin[0].r, 128, 256, 128);
     }
-    if (int rc = gat.launch(s)) return from_kernel(rc);
+    if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
     GemmBuilder gb;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     const int mxa = gb.map(xa_s, T, lin[0].r + lin[1].r, ld_xa, kBM);
@@ -853,10 +853,10 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     Carver c(ws->ptr);
     carve(c, &wtc, &xc);
     if (!L.w_kept)
-      if (int rc = gather_rows_bf16(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, s))
+      if (int rc = gather_rows_bf16(L.w_t, L.d_out, L.d_in, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, err_word(ws), s))
         return from_kernel(rc);
     if (xc)
-      if (int rc = gather_cols_bf16(x, ldx, C, ch[0].sigma, nk, xc, ldc, s)) return from_kernel(rc);
+      if (int rc = gather_cols_bf16(x, ldx, L.d_in, C, ch[0].sigma, nk, xc, ldc, err_word(ws), s)) return from_kernel(rc);
     GemmBuilder gb;
     const int mxa = gb.map(xa_s, T, L.r, ld_xa, kBM);
     const int mb = gb.map(L.lora_b, L.d_out, L.r, L.r, kBN);
@@ -929,11 +929,12 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     carve(c, wc, dyc);
     GatherBatch gat;
     for (int i = 0; i < n_lin; ++i)
-      if (!lin[i].w_kept) gat.add(lin[i].w, d_in, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
-    if (int rc = gat.launch(s)) return from_kernel(rc);
+      if (!lin[i].w_kept) gat.add(lin[i].w, d_in, lin[i].d_out, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
+    if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
     for (int i = 0; i < n_lin; ++i) {
       if (dyc[i])
-        if (int rc = gather_cols_bf16(dy[i], ld_dy[i], C, ch[i].sigma, ch[i].n_keep, dyc[i], rup(ch[i].n_keep, 8), s))
+        if (int rc = gather_cols_bf16(dy[i], ld_dy[i], lin[i].d_out, C, ch[i].sigma, ch[i].n_keep, dyc[i], rup(ch[i].n_keep, 8),
+                                      err_word(ws), s))
           return from_kernel(rc);
     }
     GemmBuilder gb;
@@ -998,9 +999,9 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   if (int rc = transpose_bf16(L.lora_a, L.r, d_in, d_in, at, L.r, s)) return from_kernel(rc);
   {
     GatherBatch gat;  // kept rows of W^T (when not given) and the permuted A^T, one launch
-    if (!L.w_kept) gat.add(L.w_t, L.d_out, ch[0].sigma, nk, L.d_out, wtc, L.d_out);
-    gat.add(at, L.r, ch[0].sigma, d_in, L.r, ats, L.r);
-    if (int rc = gat.launch(s)) return from_kernel(rc);
+    if (!L.w_kept) gat.add(L.w_t, L.d_out, L.d_in, ch[0].sigma, nk, L.d_out, wtc, L.d_out);
+    gat.add(at, L.r, d_in, ch[0].sigma, d_in, L.r, ats, L.r);
+    if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
   }
   GemmBuilder gb;
   const int mdy = gb.map(dy[0], T, L.d_out, ld_dy[0], kBM);
@@ -1093,27 +1094,48 @@ sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_
   return from_kernel(transpose_bf16(w, d_out, d_in, d_in, w_t, d_out, cs(stream)));
 }
 
-sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
-                          void* dst, int64_t ld_dst, sl_stream stream) {
+sl_status sl_permute_rows(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm, int64_t n_rows,
+                          int64_t n_cols, void* dst, int64_t ld_dst, sl_stream stream) {
   if (!src || !perm || !dst) return SL_ERR_INVALID_ARG;
-  if (n_rows <= 0 || n_cols <= 0 || ld_src < n_cols || ld_dst < n_cols) return SL_ERR_SHAPE;
-  return from_kernel(permute_rows_bf16(src, ld_src, perm, n_rows, n_cols, dst, ld_dst, cs(stream)));
+  if (src_rows <= 0 || n_rows <= 0 || n_cols <= 0 || ld_src < n_cols || ld_dst < n_cols) return SL_ERR_SHAPE;
+  return from_kernel(
+      gather_rows_bf16(src, ld_src, src_rows, perm, n_rows, n_cols, dst, ld_dst, 0, aux_debug_word(), cs(stream)));
 }
 
-sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src, const int32_t* const* perm,
-                               const int64_t* n_rows, const int64_t* n_cols, void* const* dst, const int64_t* ld_dst,
-                               sl_stream stream) {
-  if (n < 1 || n > kMaxGatherJobs || !src || !ld_src || !perm || !n_rows || !n_cols || !dst || !ld_dst)
+sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src, const int64_t* src_rows,
+                               const int32_t* const* perm, const int64_t* n_rows, const int64_t* n_cols,
+                               void* const* dst, const int64_t* ld_dst, sl_stream stream) {
+  if (n < 1 || n > kMaxGatherJobs || !src || !ld_src || !src_rows || !perm || !n_rows || !n_cols || !dst || !ld_dst)
     return SL_ERR_INVALID_ARG;
   GatherBatch gat;
   for (int q = 0; q < n; ++q) {
     if (n_rows[q] < 0) return SL_ERR_SHAPE;
     if (n_rows[q] == 0) continue;
     if (!src[q] || !perm[q] || !dst[q]) return SL_ERR_INVALID_ARG;
-    if (n_cols[q] <= 0 || ld_src[q] < n_cols[q] || ld_dst[q] < n_cols[q]) return SL_ERR_SHAPE;
-    gat.add(src[q], ld_src[q], perm[q], n_rows[q], n_cols[q], dst[q], ld_dst[q]);
+    if (n_cols[q] <= 0 || src_rows[q] <= 0 || ld_src[q] < n_cols[q] || ld_dst[q] < n_cols[q]) return SL_ERR_SHAPE;
+    gat.add(src[q], ld_src[q], src_rows[q], perm[q], n_rows[q], n_cols[q], dst[q], ld_dst[q]);
   }
-  return from_kernel(gat.launch(cs(stream)));
+  return from_kernel(gat.launch(aux_debug_word(), cs(stream)));
+}
+
+int32_t sl_debug_bounds_enabled(void) {
+#ifdef SL_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+sl_status sl_read_debug_flag(int32_t* code, sl_stream stream) {
+  if (!code) return SL_ERR_INVALID_ARG;
+  *code = 0;
+  int* w = aux_debug_word();
+  if (!w) return SL_OK;  // release build: no checks, nothing recorded
+  if (cudaMemcpyAsync(code, w, sizeof(int32_t), cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess ||
+      cudaMemsetAsync(w, 0, sizeof(int32_t), cs(stream)) != cudaSuccess ||
+      cudaStreamSynchronize(cs(stream)) != cudaSuccess)
+    return SL_ERR_CUDA;
+  return *code ? SL_ERR_DEVICE_FLAG : SL_OK;
 }
 
 }  // extern "C"

@@ -10,41 +10,15 @@ namespace sl {
 
 namespace {
 
-// dst[drow(i), col0 + c] = src[idx ? idx[i] : i, c], c < n_cols, where
-// drow(i) = (i / blk) * blk_stride + blk_off + i % blk (blk = 0: drow(i) = i).
-// One warp per row.
-__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src,
-                                   const int32_t* __restrict__ idx, int64_t n_rows, int64_t n_cols,
-                                   __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int64_t col0, int vec, int blk,
-                                   int blk_stride, int blk_off) {
-  pdl_wait();
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= n_rows) return;
-  const int64_t sr = idx ? (int64_t)idx[row] : row;
-  const int64_t drow = blk ? (row / blk) * blk_stride + blk_off + row % blk : row;
-  const __nv_bfloat16* s = src + sr * ld_src;
-  __nv_bfloat16* d = dst + drow * ld_dst + col0;
-  if (vec) {
-    const int64_t nv = n_cols / 8;
-    for (int64_t c = lane; c < nv; c += 32)
-      reinterpret_cast<uint4*>(d)[c] = __ldg(reinterpret_cast<const uint4*>(s) + c);
-  } else {
-    for (int64_t c = lane; c < n_cols; c += 32) d[c] = s[c];
-  }
-}
-
-// Several row gathers in one launch: blockIdx.y picks the job, each warp copies one row as in
-// gather_rows_kernel (the grid covers the job with the most rows; shorter jobs return early).
-__global__ void gather_rows_multi_kernel(const __grid_constant__ GatherJobs p) {
-  pdl_wait();
-  const GatherJob& j = p.j[blockIdx.y];
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= j.n_rows) return;
+// One warp copies row i of a gather: dst[drow(i), col0 + c] = src[idx ? idx[i] : i, c], c < n_cols,
+// drow(i) = i, or (i / blk) * blk_stride + blk_off + i % blk when blk > 0.
+// The debug build checks idx[i] against the source's rows first (and skips the row if it is out
+// of range).
+__device__ __forceinline__ void gather_row(const GatherJob& j, int64_t row, int lane, int* err) {
   const int64_t sr = j.idx ? (int64_t)j.idx[row] : row;
-  const int64_t drow = j.blk ? (row / j.blk) * j.blk_stride + j.blk_off + row % j.blk : row;
+  if (!index_ok(sr, j.src_rows, err, DEV_BAD_GATHER_ROW)) return;
   const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(j.src) + sr * j.ld_src;
+  const int64_t drow = j.blk ? (row / j.blk) * j.blk_stride + j.blk_off + row % j.blk : row;
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(j.dst) + drow * j.ld_dst + j.col0;
   if (j.vec) {
     const int64_t nv = j.n_cols / 8;
@@ -55,14 +29,25 @@ __global__ void gather_rows_multi_kernel(const __grid_constant__ GatherJobs p) {
   }
 }
 
+// Row gathers in one launch: blockIdx.y picks the job, each warp copies one row (the grid covers
+// the job with the most rows; shorter jobs return early).
+__global__ void gather_rows_multi_kernel(const __grid_constant__ GatherJobs p) {
+  pdl_wait();
+  const GatherJob& j = p.j[blockIdx.y];
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= j.n_rows) return;
+  gather_row(j, row, threadIdx.x & 31, p.err);
+}
+
 // dst[t, j] = src[t, idx[j]]
-__global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t n_rows,
-                                   const int32_t* __restrict__ idx, int64_t n_idx, __nv_bfloat16* __restrict__ dst,
-                                   int64_t ld_dst) {
+__global__ void gather_cols_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t src_cols,
+                                   int64_t n_rows, const int32_t* __restrict__ idx, int64_t n_idx,
+                                   __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int* err) {
   pdl_wait();
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n_idx) return;
   const int64_t c = idx[j];
+  if (!index_ok(c, src_cols, err, DEV_BAD_GATHER_COL)) return;
   for (int64_t t = blockIdx.y; t < n_rows; t += gridDim.y) dst[t * ld_dst + j] = src[t * ld_src + c];
 }
 
@@ -91,27 +76,27 @@ __global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict_
 
 }  // namespace
 
-int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
-                     int64_t ld_dst, int64_t dst_col0, cudaStream_t s, int blk, int blk_stride, int blk_off) {
-  if (n_rows <= 0 || n_cols <= 0) return 0;
-  const int vec = (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (dst_col0 % 8 == 0) &&
-                  ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
-  const int rows_per_block = 8;
-  launch_kernel(gather_rows_kernel, (unsigned)((n_rows + rows_per_block - 1) / rows_per_block), 32 * rows_per_block, 0, s, 
-      (const __nv_bfloat16*)src, ld_src, idx, n_rows, n_cols, (__nv_bfloat16*)dst, ld_dst, dst_col0, vec, blk,
-      blk_stride, blk_off);
-  if (launch_failed("sl_aux")) return 5;
-  note_launch();
-  return 0;
+static int vec_ok(const void* src, int64_t ld_src, const void* dst, int64_t ld_dst, int64_t n_cols, int64_t col0) {
+  return (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (col0 % 8 == 0) &&
+         ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
 }
 
-int GatherBatch::add(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
-                     int64_t ld_dst, int64_t dst_col0, int blk, int blk_stride, int blk_off) {
+int gather_rows_bf16(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* idx, int64_t n_rows,
+                     int64_t n_cols, void* dst, int64_t ld_dst, int64_t dst_col0, int* err, cudaStream_t s) {
+  GatherBatch b;
+  b.add(src, ld_src, src_rows, idx, n_rows, n_cols, dst, ld_dst, dst_col0);
+  return b.launch(err, s);
+}
+
+int GatherBatch::add(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* idx, int64_t n_rows,
+                     int64_t n_cols, void* dst, int64_t ld_dst, int64_t dst_col0, int blk, int blk_stride,
+                     int blk_off) {
   if (n_rows <= 0 || n_cols <= 0) return 0;
   if (jobs.n >= kMaxGatherJobs) return 1;
   GatherJob& j = jobs.j[jobs.n++];
   j.src = src;
   j.ld_src = ld_src;
+  j.src_rows = src_rows;
   j.idx = idx;
   j.n_rows = n_rows;
   j.n_cols = n_cols;
@@ -121,16 +106,16 @@ int GatherBatch::add(const void* src, int64_t ld_src, const int32_t* idx, int64_
   j.blk = blk;
   j.blk_stride = blk_stride;
   j.blk_off = blk_off;
-  j.vec = (n_cols % 8 == 0) && (ld_src % 8 == 0) && (ld_dst % 8 == 0) && (dst_col0 % 8 == 0) &&
-          ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 == 0);
+  j.vec = vec_ok(src, ld_src, dst, ld_dst, n_cols, dst_col0);
   return 0;
 }
 
-int GatherBatch::launch(cudaStream_t s) {
+int GatherBatch::launch(int* err, cudaStream_t s) {
   if (jobs.n == 0) return 0;
   int64_t rows = 0;
   for (int i = 0; i < jobs.n; ++i) rows = rows > jobs.j[i].n_rows ? rows : jobs.j[i].n_rows;
   const int rows_per_block = 8;
+  jobs.err = err;
   const dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), (unsigned)jobs.n);
   launch_kernel(gather_rows_multi_kernel, grid, 32 * rows_per_block, 0, s, jobs);
   jobs.n = 0;
@@ -139,12 +124,12 @@ int GatherBatch::launch(cudaStream_t s) {
   return 0;
 }
 
-int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int32_t* idx, int64_t n_idx, void* dst,
-                     int64_t ld_dst, cudaStream_t s) {
+int gather_cols_bf16(const void* src, int64_t ld_src, int64_t src_cols, int64_t n_rows, const int32_t* idx,
+                     int64_t n_idx, void* dst, int64_t ld_dst, int* err, cudaStream_t s) {
   if (n_rows <= 0 || n_idx <= 0) return 0;
   dim3 grid((unsigned)((n_idx + 255) / 256), (unsigned)(n_rows < 1024 ? n_rows : 1024));
-  launch_kernel(gather_cols_kernel, grid, 256, 0, s, (const __nv_bfloat16*)src, ld_src, n_rows, idx, n_idx,
-                                          (__nv_bfloat16*)dst, ld_dst);
+  launch_kernel(gather_cols_kernel, grid, 256, 0, s, (const __nv_bfloat16*)src, ld_src, src_cols, n_rows, idx, n_idx,
+                (__nv_bfloat16*)dst, ld_dst, err);
   if (launch_failed("sl_aux")) return 5;
   note_launch();
   return 0;
@@ -161,10 +146,17 @@ int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, 
   return 0;
 }
 
-int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols, void* dst,
-                      int64_t ld_dst, cudaStream_t s) {
-  return gather_rows_bf16(src, ld_src, perm, n_rows, n_cols, dst, ld_dst, 0, s);
+#ifdef SL_DEBUG_BOUNDS
+// The error word of the debug checks in the entries that take no workspace (one per device).
+static __device__ int g_aux_debug_word;
+int* aux_debug_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_aux_debug_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
+#else
+int* aux_debug_word() { return nullptr; }
+#endif
 
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s) {
   if (n <= 0) return 0;

@@ -154,8 +154,9 @@ struct AuxWait {
 __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, int n0, int r, uint32_t tb,
                               float* stage, int half, int& sb, AuxWait& aw) {
   const int row = m0 + r;
-  const bool rv = row < pr.M;
+  bool rv = row < pr.M;
   const int64_t orow = pr.row_map ? (rv ? (int64_t)pr.row_map[row] : 0) : (int64_t)pr.out_row0 + row;
+  if (pr.row_map && rv) rv = index_ok(orow, pr.M, aw.err, DEV_BAD_ROW_MAP);
   float v[32];
   uint32_t raw[32];
   // bulk tensor stores: warp-uniform; rows of this warp start at wrow0 (problem-local)
@@ -218,15 +219,17 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
 #pragma unroll
       for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(raw[i]) * pr.a0;
       __syncwarp();
-      const bool cv = lane < n;
+      bool cv = lane < n;
       const int64_t ocol = cv ? (int64_t)pr.col_map[n0 + c0 + lane] : 0;
+      if (cv) cv = index_ok(ocol, pr.N, aw.err, DEV_BAD_COL_MAP);
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out0);
       const int wrow0 = m0 + r - lane;
       for (int rr = 0; rr < 32; ++rr) {
         const int row2 = wrow0 + rr;
         if (cv && row2 < pr.M) {
           const int64_t o2 = pr.row_map ? (int64_t)pr.row_map[row2] : (int64_t)pr.out_row0 + row2;
-          out[o2 * pr.ld0 + ocol] = __float2bfloat16_rn(stage[rr * 33 + lane]);
+          if (!pr.row_map || index_ok(o2, pr.M, aw.err, DEV_BAD_ROW_MAP))
+            out[o2 * pr.ld0 + ocol] = __float2bfloat16_rn(stage[rr * 33 + lane]);
         }
       }
       __syncwarp();
@@ -281,7 +284,10 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         if (pr.col_map) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (i < n) out[orow * pr.ld0 + pr.col_map[n0 + c0 + i]] = __float2bfloat16_rn(v[i]);
+            if (i < n) {
+              const int64_t oc = pr.col_map[n0 + c0 + i];
+              if (index_ok(oc, pr.N, aw.err, DEV_BAD_COL_MAP)) out[orow * pr.ld0 + oc] = __float2bfloat16_rn(v[i]);
+            }
         } else {
           const int64_t off = orow * pr.ld0 + n0 + c0;
           store_bf16_row(out + off, v, n, (off & 7) == 0);
@@ -314,6 +320,7 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         for (int i = 0; i < 32; ++i) {
           if (i >= n) break;
           const int64_t col = pr.col_map ? pr.col_map[n0 + c0 + i] : n0 + c0 + i;
+          if (pr.col_map && !index_ok(col, pr.N, aw.err, DEV_BAD_COL_MAP)) continue;
           float* d = pr.epi == EPI_F32 ? reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + col : f32t_dst(pr, col) + orow;
           if (pr.beta)
             atomicAdd(d, pr.a0 * v[i]);
@@ -393,6 +400,7 @@ __device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t
 
 struct RedProb {
   int32_t M, N, ksplit, epi, beta, out_row0, col_split, pad_;
+  int* err;
   int64_t ld0, ld1;
   void* out0;
   void* out1;
@@ -429,6 +437,8 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
     for (int s = 0; s < pr.ksplit; ++s) acc += __ldg(pr.part + (int64_t)s * total + e);
     const int64_t orow = pr.row_map ? (int64_t)pr.row_map[row] : pr.out_row0 + row;
     const int64_t ocol = pr.col_map ? (int64_t)pr.col_map[col] : col;
+    if (pr.row_map && !index_ok(orow, pr.M, pr.err, DEV_BAD_ROW_MAP)) continue;
+    if (pr.col_map && !index_ok(ocol, pr.N, pr.err, DEV_BAD_COL_MAP)) continue;
     if (pr.epi == EPI_XA) {
       reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + ocol] = pr.a0 * acc;
       reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + ocol] = __float2bfloat16_rn(pr.a1 * acc);
@@ -1266,7 +1276,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     q.M = pr.M; q.N = pr.N; q.ksplit = pr.ksplit; q.epi = pr.epi; q.beta = pr.beta; q.out_row0 = pr.out_row0;
     q.col_split = pr.col_split; q.out2 = pr.out2;
     q.ld0 = pr.ld0; q.ld1 = pr.ld1; q.out0 = pr.out0; q.out1 = pr.out1; q.row_map = pr.row_map;
-    q.col_map = pr.col_map; q.part = pr.part; q.a0 = pr.a0; q.a1 = pr.a1;
+    q.col_map = pr.col_map; q.part = pr.part; q.a0 = pr.a0; q.a1 = pr.a1; q.err = err;
     maxmn = std::max<int64_t>(maxmn, (int64_t)pr.M * pr.N);
   }
   if (nred) {

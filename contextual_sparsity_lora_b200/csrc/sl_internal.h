@@ -41,6 +41,38 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// ---- debug bounds checks
+// A debug build (-DSL_DEBUG_BOUNDS; python -m contextual_sparsity_lora_b200.build --debug writes
+// libsparselora_debug.so) checks every index read from a channel set or a row map against the
+// extent it indexes, before the access that index drives: gathered rows and columns against the
+// source's rows or columns, scattered output columns and rows against the problem's columns and
+// rows, dB rows against the adapter's output channels. A failing check skips that access and
+// records its code in the error word (first writer wins): the caller's workspace error word, or,
+// for the entries that take no workspace, the library's debug word (sl_read_debug_flag). In the
+// release build index_ok is `true` and compiles away.
+enum : int {
+  DEV_BAD_GATHER_ROW = 0x101,  // row gather: source row index out of range
+  DEV_BAD_GATHER_COL = 0x102,  // column gather: source column index out of range
+  DEV_BAD_COL_MAP = 0x103,     // GEMM epilogue or split-K reduce: output column map out of range
+  DEV_BAD_ROW_MAP = 0x104,     // GEMM epilogue or split-K reduce: output row map out of range
+  DEV_BAD_DB_ROW = 0x105,      // fused LoRA backward: dB row (sigma) out of range
+};
+#ifdef __CUDACC__
+__device__ __forceinline__ bool index_ok(int64_t i, int64_t n, int* err, int code) {
+#ifdef SL_DEBUG_BOUNDS
+  if (i >= 0 && i < n) return true;
+  if (err) atomicCAS(err, 0, code);
+  return false;
+#else
+  (void)i; (void)n; (void)err; (void)code;
+  return true;
+#endif
+}
+#endif
+// Device address of the library's debug word (debug builds; null in release builds), the error
+// word of the checks in entries that take no workspace.
+int* aux_debug_word();
+
 // Launch accounting for the optional profiling hook (sl_profile_enable / sl_profile_read).
 void note_launch(int n = 1);
 bool profiling_on();
@@ -179,35 +211,38 @@ int wanda_scores(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_
                  int64_t d_out, int64_t ldw, float* scores, float* scratch, cudaStream_t s);
 
 // ---- helpers (sl_aux.cu)
-int gather_rows_bf16(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols,
-                     void* dst, int64_t ld_dst, int64_t dst_col0, cudaStream_t s, int blk = 0, int blk_stride = 0,
-                     int blk_off = 0);
+// dst[i, :] = src[idx[i], :]; src_rows: rows of src (the debug build checks idx against it);
+// err: error word of the debug checks.
+int gather_rows_bf16(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* idx, int64_t n_rows,
+                     int64_t n_cols, void* dst, int64_t ld_dst, int64_t dst_col0, int* err, cudaStream_t s);
 // Row gathers batched into one launch (jobs as in gather_rows_bf16).
 constexpr int kMaxGatherJobs = 8;
 struct GatherJob {
   const void* src;
   const int32_t* idx;
   void* dst;
-  int64_t ld_src, n_rows, n_cols, ld_dst, col0;
-  int32_t blk, blk_stride, blk_off, vec;
+  int64_t ld_src, src_rows, n_rows, n_cols, ld_dst, col0;
+  int32_t blk, blk_stride, blk_off, vec;  // destination row of row i: (i / blk) * blk_stride + blk_off + i % blk
 };
 struct GatherJobs {
   GatherJob j[kMaxGatherJobs];
   int32_t n;
+  int* err;  // error word of the debug checks
 };
 struct GatherBatch {
   GatherJobs jobs{};
-  // returns 1 when the batch is full; empty jobs are skipped
-  int add(const void* src, int64_t ld_src, const int32_t* idx, int64_t n_rows, int64_t n_cols, void* dst,
-          int64_t ld_dst, int64_t dst_col0 = 0, int blk = 0, int blk_stride = 0, int blk_off = 0);
-  int launch(cudaStream_t s);  // one launch for every job added, then empty
+  // dst[drow(i), col0 + c] = src[idx[i], c] (src has src_rows rows), drow(i) = i, or with blk > 0
+  // (i / blk) * blk_stride + blk_off + i % blk; returns 1 when the batch is full; empty jobs are
+  // skipped
+  int add(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* idx, int64_t n_rows, int64_t n_cols,
+          void* dst, int64_t ld_dst, int64_t dst_col0 = 0, int blk = 0, int blk_stride = 0, int blk_off = 0);
+  int launch(int* err, cudaStream_t s);  // one launch for every job added, then empty
 };
-int gather_cols_bf16(const void* src, int64_t ld_src, int64_t n_rows, const int32_t* idx, int64_t n_idx,
-                     void* dst, int64_t ld_dst, cudaStream_t s);
+// dst[t, j] = src[t, idx[j]] for t < n_rows, j < n_idx; src_cols: columns of src (debug checks).
+int gather_cols_bf16(const void* src, int64_t ld_src, int64_t src_cols, int64_t n_rows, const int32_t* idx,
+                     int64_t n_idx, void* dst, int64_t ld_dst, int* err, cudaStream_t s);
 int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,
                    cudaStream_t s);
-int permute_rows_bf16(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
-                      void* dst, int64_t ld_dst, cudaStream_t s);
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s);
 // Tensor map of a bf16 matrix [rows, cols] (ld elements) with box_cols x box_rows boxes.
 bool encode_bf16_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols,

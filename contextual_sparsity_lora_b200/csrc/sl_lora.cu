@@ -349,6 +349,7 @@ __global__ void __launch_bounds__(kDualThreads, 1) lora_dual_kernel(const __grid
         const int col = (cb0 + c) * 128 + r;
         if (col < jb.cols) {
           const int dst = jb.sigma ? jb.sigma[col] : col;
+          if (jb.sigma && !index_ok(dst, jb.cols, p.err, DEV_BAD_DB_ROW)) continue;
           float* d = jb.dB + (int64_t)dst * nr;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)

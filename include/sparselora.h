@@ -365,22 +365,46 @@ SL_API sl_status sl_set_pair_tile_rows(int32_t rows);
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
 SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, void* w_t, sl_stream stream);
 
-/* dst[i, :] = src[perm[i], :] for bf16 rows (context-first reordering of a batch). */
-SL_API sl_status sl_permute_rows(const void* src, int64_t ld_src, const int32_t* perm, int64_t n_rows, int64_t n_cols,
-                          void* dst, int64_t ld_dst, sl_stream stream);
+/* dst[i, :] = src[perm[i], :] for i < n_rows, bf16 rows of n_cols columns: the context-first
+ * reordering of a batch, or any row gather (an embedding lookup, kept weight rows). src has
+ * src_rows rows; every perm entry must lie in [0, src_rows) (the debug build checks it).
+ * Errors: SL_ERR_INVALID_ARG for a null pointer, SL_ERR_SHAPE for a non-positive size or a
+ * leading dimension below n_cols. */
+SL_API sl_status sl_permute_rows(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm,
+                                 int64_t n_rows, int64_t n_cols, void* dst, int64_t ld_dst, sl_stream stream);
 
 /* Up to 8 row gathers of bf16 rows in one launch: for each q < n, dst[q][i, :] =
  * src[q][perm[q][i], :] for i < n_rows[q], n_cols[q] columns, leading dimensions ld_src[q] and
- * ld_dst[q]. Used to build the kept weight rows of several projections at once (each w_kept
+ * ld_dst[q]; src[q] has src_rows[q] rows (every perm entry must lie in [0, src_rows[q]); the debug
+ * build checks it). Used to build the kept weight rows of several projections at once (each w_kept
  * of a step: "SparseLoRA: Accelerating LLM Fine-Tuning with Contextual Sparsity",
  * walkthrough, "Putting It All Together": the weights sliced to the selected channels).
  * The arrays are host arrays of length n; every pointer in them is a device pointer. The
  * destinations must not overlap any source. Errors: SL_ERR_INVALID_ARG for n outside [1, 8]
- * or a null pointer, SL_ERR_SHAPE for a non-positive size or a leading dimension below
- * n_cols. A job with zero rows is skipped (its pointers may be NULL). */
+ * or a null pointer, SL_ERR_SHAPE for a non-positive size (src_rows, n_cols) or a leading
+ * dimension below n_cols. A job with zero rows is skipped (its pointers may be NULL). */
 SL_API sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src,
-                                      const int32_t* const* perm, const int64_t* n_rows, const int64_t* n_cols,
-                                      void* const* dst, const int64_t* ld_dst, sl_stream stream);
+                                      const int64_t* src_rows, const int32_t* const* perm, const int64_t* n_rows,
+                                      const int64_t* n_cols, void* const* dst, const int64_t* ld_dst,
+                                      sl_stream stream);
+
+/* Debug bounds checks. A library built with them (python -m contextual_sparsity_lora_b200.build
+ * --debug writes libsparselora_debug.so; the release library has none) checks, on the device,
+ * every index it reads from a channel set (sigma), a row permutation or a gather list against the
+ * extent it indexes, before the access that index drives: gathered weight rows against the source's
+ * rows (src_rows above, d_out or d_in of a projection), gathered activation and LoRA columns
+ * against their columns, scattered output columns and rows against the product's extent, dB rows
+ * against the adapter's output channels. A failing check skips that access (nothing outside the
+ * caller's buffers is read or written) and records a code, first writer wins: 0x101 row gather,
+ * 0x102 column gather, 0x103 output column map, 0x104 output row map, 0x105 dB row. Entries with a
+ * workspace record it in the workspace error word (sl_read_device_flag); sl_gather_rows_batch and
+ * sl_permute_rows record it in the library's debug word, one per device.
+ * sl_debug_bounds_enabled: 1 in a debug build, else 0.
+ * sl_read_debug_flag: copies the debug word of the current device to *code and clears it
+ * (synchronises `stream`); SL_ERR_DEVICE_FLAG when it was set. In the release build *code = 0 and
+ * SL_OK. */
+SL_API int32_t sl_debug_bounds_enabled(void);
+SL_API sl_status sl_read_debug_flag(int32_t* code, sl_stream stream);
 
 #ifdef __cplusplus
 }

@@ -181,18 +181,21 @@ def test_layer_and_optimizer_entries_reject_bad_arguments(lib):
     assert wa(a, 0, 64, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_SHAPE
     assert wa(a, 16, 60, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_ALIGNMENT
     assert wa(a, 16, 64, 64, 2, wp, 32, 64, a, ctypes.byref(ws), None) == B.SL_ERR_WORKSPACE
-    # sl_gather_rows_batch(n, src[], ld_src[], perm[], n_rows[], n_cols[], dst[], ld_dst[], stream)
+    # sl_gather_rows_batch(n, src[], ld_src[], src_rows[], perm[], n_rows[], n_cols[], dst[], ld_dst[], stream)
     gb = lib.sl_gather_rows_batch
     ptrs = lambda *v: (ctypes.c_void_p * len(v))(*v)
     i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)
-    ok = dict(src=ptrs(0x10000), ld=i64(64), perm=ptrs(0x20000), rows=i64(4), cols=i64(64), dst=ptrs(0x30000))
-    args = lambda n, **k: [n] + [k.get(x, ok[x]) for x in ("src", "ld", "perm", "rows", "cols", "dst")] + \
+    ok = dict(src=ptrs(0x10000), ld=i64(64), srows=i64(16), perm=ptrs(0x20000), rows=i64(4), cols=i64(64),
+              dst=ptrs(0x30000))
+    args = lambda n, **k: [n] + [k.get(x, ok[x]) for x in ("src", "ld", "srows", "perm", "rows", "cols", "dst")] + \
         [k.get("ldd", i64(64)), None]
     assert gb(*args(0)) == B.SL_ERR_INVALID_ARG
     assert gb(*args(9)) == B.SL_ERR_INVALID_ARG
     assert gb(*args(1, perm=ptrs(None))) == B.SL_ERR_INVALID_ARG
+    assert gb(*args(1, srows=None)) == B.SL_ERR_INVALID_ARG
     assert gb(*args(1, rows=i64(-1))) == B.SL_ERR_SHAPE
     assert gb(*args(1, cols=i64(0))) == B.SL_ERR_SHAPE
+    assert gb(*args(1, srows=i64(0))) == B.SL_ERR_SHAPE
     assert gb(*args(1, ldd=i64(32))) == B.SL_ERR_SHAPE
     # a job without rows launches nothing, whatever its pointers
     assert gb(*args(1, rows=i64(0), src=ptrs(None), perm=ptrs(None), dst=ptrs(None))) == B.SL_OK
@@ -205,3 +208,32 @@ def test_pair_tile_rows_setting_host_side(lib):
     for rows in (-1, 1, 128, 384, 1024):
         assert lib.sl_set_pair_tile_rows(rows) == B.SL_ERR_INVALID_ARG
     assert lib.sl_set_pair_tile_rows(0) == B.SL_OK
+
+
+def test_debug_build_exports_and_flags_host_side():
+    """The debug build exports the same entry points and says it checks bounds; the release build
+    says it does not, and its debug word always reads 0."""
+    if not os.path.exists(B.DEBUG_LIB_PATH):
+        pytest.skip("debug library not built")
+    dbg = B.load(B.DEBUG_LIB_PATH)
+    for name in B.EXPORTED:
+        getattr(dbg, name)
+    assert dbg.sl_debug_bounds_enabled() == 1
+    rel = B.load(B.LIB_PATH)
+    assert rel.sl_debug_bounds_enabled() == 0
+    code = ctypes.c_int32(-1)
+    assert rel.sl_read_debug_flag(ctypes.byref(code), None) == B.SL_OK and code.value == 0
+    assert rel.sl_read_debug_flag(None, None) == B.SL_ERR_INVALID_ARG
+
+
+def test_permute_rows_rejects_bad_arguments(lib):
+    """sl_permute_rows(src, ld_src, src_rows, perm, n_rows, n_cols, dst, ld_dst, stream): host checks
+    only; nothing is launched."""
+    P = ctypes.c_void_p
+    f = lib.sl_permute_rows
+    a = P(0x10000)
+    assert f(None, 64, 8, a, 4, 64, a, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, 8, None, 4, 64, a, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, 0, a, 4, 64, a, 64, None) == B.SL_ERR_SHAPE
+    assert f(a, 64, 8, a, 0, 64, a, 64, None) == B.SL_ERR_SHAPE
+    assert f(a, 32, 8, a, 4, 64, a, 64, None) == B.SL_ERR_SHAPE
