@@ -528,7 +528,7 @@ def model_measure(da, df, perm, C, ac, fc, device, keep, n_steps=20, vocab=12825
             "lr": f"AdamW, cosine schedule, 4% warm-up, peak {peak_lr}",
             "frozen_weights": "per layer: a random signed permutation of one decaying-spectrum draw per projection",
             "lm_head_and_cross_entropy": "torch (library)",
-            "attention_core": "torch scaled_dot_product_attention (library)"}
+            "attention_core": "sl_attention_fwd / sl_attention_bwd (tcgen05, causal GQA)"}
 
 
 def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
@@ -545,16 +545,44 @@ def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
     for _ in range(2):
         layer.step(x, dy)
     torch.cuda.synchronize()
-    try:  # the attention core's autograd backward inside a captured graph
-        replay, captured = capture_graph(lambda: layer.step(x, dy), warm=False).replay, True
-    except Exception as e:  # noqa: BLE001 - fall back to the eager layer step
-        print(f"layer step not captured ({type(e).__name__}: {e}); timing the eager step", file=sys.stderr)
-        torch.cuda.synchronize()
-        replay, captured = (lambda: layer.step(x, dy)), False
+    replay = capture_graph(lambda: layer.step(x, dy), warm=False).replay
     ms = time_steps(replay, K, W, 1, device) / K
-    return {"value": ac.n_tok / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
-            "cuda_graph": captured, "attention_core": "torch scaled_dot_product_attention (causal, GQA)",
+    return {"value": ac.n_tok / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "cuda_graph": True,
+            "attention_core": attention_core_measure(layer, ac, K, W, device),
             "layer": "RMSNorm, sparse q/k/v, attention, sparse o, residual, RMSNorm, sparse SwiGLU FFN, residual"}
+
+
+def attention_core_measure(layer, ac, K, W, device):
+    """The layer's attention core alone (sl_attention_fwd, sl_attention_bwd on the layer's own q, k,
+    v, o, do buffers after a step), each captured in a CUDA graph of 10 calls: device time per call
+    and TFLOP/s of the causal products (forward Q K^T and P V, backward the recomputed Q K^T, dO V^T,
+    P^T dO, dS^T Q and dS K: 2 and 5 products of 2 hd FLOP per visible (query, key) pair)."""
+    from contextual_sparsity_lora_b200 import binding as B
+    at = layer.attn
+    n_seq, S = layer.n_seq, layer.S
+    pairs = n_seq * at.hq * S * (S + 1) / 2
+
+    def fwd():
+        B.sl_attention_fwd(layer.ws, layer.q_nat, layer.k_nat, layer.v_nat, n_seq, at.hq, at.hkv, at.hd,
+                           layer.a_nat, layer.lse)
+
+    def bwd():
+        B.sl_attention_bwd(layer.ws, layer.q_nat, layer.k_nat, layer.v_nat, layer.a_nat, layer.da_nat, layer.lse,
+                           n_seq, at.hq, at.hkv, at.hd, layer.dq_nat, layer.dk_nat, layer.dv_nat)
+
+    out = {"kernels": "attn_fwd_kernel, attn_bwd_kernel (tcgen05, TMEM accumulators)",
+           "shape": f"{n_seq} x {S} tokens, {at.hq} query / {at.hkv} key-value heads of {at.hd}, causal"}
+    peak = float(load_peaks()[0].get("bf16_tflops", 1590.0))
+    for name, fn, n_prod in (("fwd", fwd, 2), ("bwd", bwd, 5)):
+        fn()
+        g = capture_graph(lambda: [fn() for _ in range(10)], warm=False)
+        us = time_steps(g.replay, K, W, 1, device) / (10 * K) * 1e3
+        del g
+        tf = n_prod * 2.0 * at.hd * pairs / (us * 1e-6) / 1e12
+        out[f"{name}_us"] = us
+        out[f"{name}_tflops"] = tf
+        out[f"{name}_frac_of_bf16_peak"] = tf / peak
+    return out
 
 
 def e2e_measure(attn, ffn, step_in, K, W, world, device, eager=False):

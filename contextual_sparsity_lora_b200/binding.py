@@ -31,7 +31,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
             "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows",
-            "sl_debug_bounds_enabled", "sl_read_debug_flag")
+            "sl_debug_bounds_enabled", "sl_read_debug_flag", "sl_attention_fwd", "sl_attention_bwd")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -134,6 +134,10 @@ def load(path):
     L.sl_permute_rows.argtypes = [P, c_int64, c_int64, P, c_int64, c_int64, P, c_int64, P]
     L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P, P]
     L.sl_debug_bounds_enabled.restype = c_int32
+    L.sl_attention_fwd.argtypes = [P, P, P, c_int64, c_int64, c_int32, c_int32, c_int32, c_int32, c_int32, P, P,
+                                   POINTER(SlWorkspaceC), P]
+    L.sl_attention_bwd.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                   P, P, P, POINTER(SlWorkspaceC), P]
     L.sl_read_debug_flag.argtypes = [POINTER(c_int32), P]
     L.sl_set_pair_tile_rows.argtypes = [c_int32]
     for n in EXPORTED:
@@ -375,6 +379,19 @@ def sl_read_debug_flag() -> int:
     if rc not in (SL_OK, SL_ERR_DEVICE_FLAG):
         _check("sl_read_debug_flag", rc)
     return int(code.value)
+
+
+def sl_attention_fwd(ws: Workspace, q, k, v, n_seq, n_q_heads, n_kv_heads, head_dim, o, lse):
+    """Causal GQA attention over n_seq equal-length sequences (rows in sequence order): o and the
+    per-row log-sum-exp lse [n_q_heads, T] for the backward."""
+    ws.call("sl_attention_fwd", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), int(n_seq),
+            q.shape[0] // int(n_seq), int(n_q_heads), int(n_kv_heads), int(head_dim), _ptr(o), _ptr(lse))
+
+
+def sl_attention_bwd(ws: Workspace, q, k, v, o, d_o, lse, n_seq, n_q_heads, n_kv_heads, head_dim, dq, dk, dv):
+    ws.call("sl_attention_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), q.stride(0), k.stride(0),
+            int(n_seq), q.shape[0] // int(n_seq), int(n_q_heads), int(n_kv_heads), int(head_dim), _ptr(dq), _ptr(dk),
+            _ptr(dv))
 
 
 def sl_set_pair_tile_rows(rows: int):

@@ -20,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsparselora.so")
 DEBUG_LIB = os.path.join(HERE, "libsparselora_debug.so")
-SOURCES = ["sl_api.cu", "sl_gemm.cu", "sl_estimator.cu", "sl_select.cu", "sl_aux.cu", "sl_lora.cu", "sl_noalloc.cu", "sl_est_tc.cu", "sl_criteria.cu", "sl_layer.cu"]
+SOURCES = ["sl_api.cu", "sl_gemm.cu", "sl_estimator.cu", "sl_select.cu", "sl_aux.cu", "sl_lora.cu", "sl_noalloc.cu", "sl_est_tc.cu", "sl_criteria.cu", "sl_layer.cu", "sl_attention.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

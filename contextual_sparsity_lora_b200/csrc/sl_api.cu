@@ -1082,6 +1082,50 @@ sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64
   return SL_OK;
 }
 
+// ------------------------------------------------------------------ attention core
+namespace {
+sl_status attention_args(const void* const* ptrs, int n_ptrs, int64_t ldq, int64_t ldkv, int32_t n_seq,
+                         int32_t seq_len, int32_t hq, int32_t hkv, int32_t hd) {
+  for (int i = 0; i < n_ptrs; ++i)
+    if (!ptrs[i]) return SL_ERR_INVALID_ARG;
+  if (n_seq < 1 || seq_len < 1 || hq < 1 || hkv < 1 || hq % hkv || hd < 8 || hd > 128 || hd % 8) return SL_ERR_SHAPE;
+  if ((int64_t)n_seq * seq_len > (int64_t)1 << 31 || seq_len > (1 << 24) || hq > 65535 || hkv > 65535)
+    return SL_ERR_SHAPE;
+  if (ldq < (int64_t)hq * hd || ldkv < (int64_t)hkv * hd) return SL_ERR_SHAPE;
+  if (ldq % 8 || ldkv % 8) return SL_ERR_ALIGNMENT;
+  for (int i = 0; i < n_ptrs; ++i)
+    if (!al16(ptrs[i])) return SL_ERR_ALIGNMENT;
+  return SL_OK;
+}
+}  // namespace
+
+sl_status sl_attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int64_t ldkv, int32_t n_seq,
+                           int32_t seq_len, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, void* o,
+                           float* lse, sl_workspace* ws, sl_stream stream) {
+  const void* ptrs[5] = {q, k, v, o, lse};
+  if (sl_status st = attention_args(ptrs, 5, ldq, ldkv, n_seq, seq_len, n_q_heads, n_kv_heads, head_dim)) return st;
+  if (sl_status st = ws_check(ws, kWorkspaceHeaderBytes)) return st;
+  const int rc = attention_fwd(q, k, v, ldq, ldkv, n_seq, seq_len, n_q_heads, n_kv_heads, head_dim, o, ldq, lse,
+                               err_word(ws), cs(stream));
+  return rc == 0 ? SL_OK : (rc == 2 ? SL_ERR_ALIGNMENT : SL_ERR_CUDA);
+}
+
+sl_status sl_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                           const float* lse, int64_t ldq, int64_t ldkv, int32_t n_seq, int32_t seq_len,
+                           int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, void* dq, void* dk, void* dv,
+                           sl_workspace* ws, sl_stream stream) {
+  const void* ptrs[9] = {q, k, v, o, d_o, lse, dq, dk, dv};
+  if (sl_status st = attention_args(ptrs, 9, ldq, ldkv, n_seq, seq_len, n_q_heads, n_kv_heads, head_dim)) return st;
+  Carver c(nullptr);
+  c.take<uint8_t>(attention_bwd_scratch(n_seq, seq_len, n_q_heads, head_dim));
+  if (sl_status st = ws_check(ws, c.off)) return st;
+  Carver c2(ws->ptr);
+  void* scratch = c2.take<uint8_t>(attention_bwd_scratch(n_seq, seq_len, n_q_heads, head_dim));
+  const int rc = attention_bwd(q, k, v, o, d_o, lse, ldq, ldkv, n_seq, seq_len, n_q_heads, n_kv_heads, head_dim, dq,
+                               dk, dv, scratch, err_word(ws), cs(stream));
+  return rc == 0 ? SL_OK : (rc == 2 ? SL_ERR_ALIGNMENT : SL_ERR_CUDA);
+}
+
 sl_status sl_set_pair_tile_rows(int32_t rows) {
   if (rows != 0 && rows != 256 && rows != 512) return SL_ERR_INVALID_ARG;
   set_forced_pair_mh(rows / 256);

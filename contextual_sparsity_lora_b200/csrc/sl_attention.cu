@@ -1,0 +1,709 @@
+// Causal grouped-query attention core of the decoder layer, forward and backward, on the
+// tcgen05 tensor cores ("SparseLoRA: Accelerating LLM Fine-Tuning with Contextual Sparsity",
+// walkthrough, "Putting It All Together": the sparse q/k/v and o projections sit around the
+// layer's attention; output rows attend to the context keys and values the sparse projections
+// computed).
+//
+//   S = Q K^T / sqrt(d) per query head h (key/value head h / (Hq / Hkv)), keys k <= query q of the
+//   same sequence; P = softmax_row(S); O = P V; LSE_q = log sum_k exp(S_qk).
+//   Backward with D_q = sum_d dO_qd O_qd: dV = P^T dO, dP = dO V^T, dS = P (dP - D), dQ = dS K / sqrt(d),
+//   dK = dS^T Q / sqrt(d).
+//
+// Rows are tokens in sequence order: n_seq sequences of seq_len tokens. Operand tiles (128 tokens
+// x 64 head-dimension elements, 128-byte swizzle) come from 4-D tensor maps [head_dim, heads,
+// seq_len, n_seq]: positions past a sequence's end and head-dimension elements past head_dim read
+// as zeros, so ragged sequence lengths and head_dim < 64 need no padding copies. One tile in shared
+// memory serves both operand majors: loaded with tokens as rows, it is K-major when the head
+// dimension is the contraction (Q K^T, dO V^T) and MN-major when the tokens are (P V, P^T dO,
+// dS^T Q, dS K).
+//
+// Forward: one CTA per (128-query tile, query head, sequence). Warp 0 loads Q once and the K/V
+// tiles through a two-stage ring; warp 1 issues the MMAs (S into two alternating TMEM buffers, so
+// S of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-5
+// run the online softmax, one query row per thread (its TMEM lane): row maximum, exponentials,
+// rescaling of O in TMEM when the maximum grows, P (bf16) into shared memory for the P V MMA.
+// Backward: one CTA per (128-key tile, key/value head, sequence), looping over the query heads of
+// the group and the query tiles at or after the key tile: S^T and dP^T by MMA, P^T and dS^T by the
+// compute warps (one key row per thread), then dV += P^T dO, dK += dS^T Q and dQ = dS K by MMA;
+// dK and dV stay in TMEM for the whole loop and are stored once, dQ leaves every iteration through
+// fp32 reductions into a workspace accumulator (several key tiles add to the same query rows).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "sl_internal.h"
+#include "sl_ptx.cuh"
+
+namespace sl {
+
+namespace {
+
+constexpr int kAttnThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 softmax / epilogue
+constexpr int kTile = 128;           // tokens per tile (TMEM lanes)
+constexpr int kChunk = 128 * 64 * 2;  // one 128-token x 64-element bf16 tile chunk (16 KB)
+
+struct AttnFwdParams {
+  CUtensorMap qmap, kmap, vmap;  // [head_dim, heads, seq_len, n_seq], boxes 64 x 1 x 128 x 1
+  __nv_bfloat16* o;
+  int64_t ldo;
+  float* lse;                    // [n_q_heads][n_seq * seq_len]
+  int32_t n_seq, S, hq, hkv, hd, nd;
+  float scale, scale_log2;       // 1 / sqrt(hd); log2(e) / sqrt(hd)
+  int* err;
+};
+
+struct AttnBwdParams {
+  CUtensorMap qmap, kmap, vmap, domap;
+  const float* lse;              // [hq][T]
+  const float* delta;            // [hq][T]: sum_d dO O per query row
+  float* dq_acc;                 // [T][hq * hd] fp32, zero on entry
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int64_t ldkv;
+  int32_t n_seq, S, hq, hkv, hd, nd;
+  float scale, scale_log2;
+  int* err;
+};
+
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m, uint64_t* bar, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Each thread of the warp writes 32 consecutive fp32 columns of its TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Shared-memory descriptors of a tile stored as nc chunks (16 KB apart) of 128 token rows x 128 B.
+// K-major use (contraction over the head dimension, or over the 128 columns of a P-like tile):
+// 16-element step t lies in chunk t / 4 at byte 32 (t % 4) of each row.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int t) {
+  return smem_desc_sw128(base + (uint32_t)(t >> 2) * kChunk + (uint32_t)(t & 3) * 32, 16, 1024);
+}
+// MN-major use (contraction over the 128 token rows): step t covers rows 16 t .. 16 t + 15; the
+// 64-wide chunks of the other dimension are 16 KB apart.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int t) {
+  return smem_desc_sw128(base + (uint32_t)t * 2048, kChunk, 1024);
+}
+
+// Writes 32 bf16 values (v[0..31] as 16 packed pairs) of row r into a 128-byte-swizzled K-major
+// tile (the layout the tensor maps produce): element c of the row sits in chunk c / 64, 16-byte
+// unit ((c % 64) / 8) ^ (r % 8).
+__device__ __forceinline__ void st_swizzled_row32(uint8_t* tile, int r, int c0, const uint32_t (&w)[16]) {
+  uint8_t* row = tile + (c0 >> 6) * kChunk + r * 128;
+  const int u0 = (c0 & 63) >> 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int u = (u0 + q) ^ (r & 7);
+    *reinterpret_cast<uint4*>(row + u * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
+__device__ __forceinline__ void named_bar_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------ forward
+
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnFwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nd = p.nd;
+  uint8_t* sq = smem;                          // Q: nd chunks
+  uint8_t* skv = sq + nd * kChunk;             // stage s: K (nd chunks) then V (nd chunks)
+  uint8_t* sp = skv + 2 * 2 * nd * kChunk;     // P: 2 chunks (128 keys)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sp + 2 * kChunk);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;  // longest (most key tiles) first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (p.hq / p.hkv);
+  const int n_kv = qt + 1;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S buffers at columns 0 and 128, O at 256
+  pdl_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, nd * kChunk);
+      for (int c = 0; c < nd; ++c) tma_load_4d(sq + c * kChunk, &p.qmap, q_full, 64 * c, h, qt * kTile, b);
+      uint32_t issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * nd * kChunk);
+        issued |= 1u << s;
+        uint8_t* st = skv + s * 2 * nd * kChunk;
+        for (int c = 0; c < nd; ++c) {
+          tma_load_4d(st + c * kChunk, &p.kmap, &kv_full[s], 64 * c, g, j * kTile, b);
+          tma_load_4d(st + (nd + c) * kChunk, &p.vmap, &kv_full[s], 64 * c, g, j * kTile, b);
+        }
+      }
+      // every copy lands before the CTA may exit
+      mbar_wait(q_full, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      for (int j = max(0, n_kv - 2); j < n_kv; ++j)
+        if (issued & (1u << (j & 1))) mbar_wait(&kv_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(128, 128, 0, 0);          // S = Q K^T: both K-major over d
+      const uint32_t id_pv = idesc_bf16(128, 64 * nd, 0, 1);     // O += P V: P K-major, V MN-major
+      const uint32_t aq = smem_u32(sq), ap = smem_u32(sp);
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.err, DEV_TIMEOUT_MMA);
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(p_full, j & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t bv = smem_u32(skv + (j & 1) * 2 * nd * kChunk + nd * kChunk);
+        for (int t = 0; t < 8; ++t)
+          umma_bf16(tmem + 256, kmajor_desc(ap, t), mnmajor_desc(bv, t), id_pv, (j > 0 || t > 0) ? 1u : 0u);
+        umma_commit(pv_done);
+        umma_commit(&kv_empty[j & 1]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&s_free[s], ((j - 2) >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t bk = smem_u32(skv + s * 2 * nd * kChunk);
+        for (int t = 0; t < 4 * nd; ++t)
+          umma_bf16(tmem + 128 * s, kmajor_desc(aq, t), kmajor_desc(bk, t), id_s, t > 0 ? 1u : 0u);
+        umma_commit(&s_full[s]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(n_kv - 1);
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;               // query row in the tile = TMEM lane
+    const int qpos = qt * kTile + r;                 // position in the sequence
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait(&s_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128 * s + 32 * c, sv[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[s]);
+      // causal mask within the sequence: key k is visible to query q when k <= q and k < S
+      const int kbase = j * kTile;
+      const int kmax = min(qpos, p.S - 1) - kbase;   // last visible column of this tile
+      float mj = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * c + i <= kmax) mj = fmaxf(mj, __uint_as_float(sv[c][i]));
+      const float m_new = fmaxf(m, mj);
+      const float mb = m_new * p.scale_log2;
+      const float corr = (m == -INFINITY) ? 0.f : ex2(m * p.scale_log2 - mb);
+      float rs = 0.f;
+      uint32_t pw[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float e0 = (32 * c + i <= kmax) ? ex2(__uint_as_float(sv[c][i]) * p.scale_log2 - mb) : 0.f;
+          const float e1 = (32 * c + i + 1 <= kmax) ? ex2(__uint_as_float(sv[c][i + 1]) * p.scale_log2 - mb) : 0.f;
+          rs += e0 + e1;
+          pw[c][i / 2] = pack2(e0, e1);
+        }
+      l = l * corr + rs;
+      if (j >= 1) {
+        // the previous P V has landed in O (and read P): rescale O when the maximum grew
+        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+          for (int c = 0; c < 2 * nd; ++c) {
+            uint32_t ov[32];
+            __syncwarp();
+            tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
+            tmem_ld_wait_regs(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+            tmem_st32(tmem + lane_off + 256 + 32 * c, ov);
+          }
+          tmem_st_wait();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) st_swizzled_row32(sp, r, 32 * c, pw[c]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      m = m_new;
+    }
+    if (ok && mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool store = qpos < p.S;
+      __nv_bfloat16* orow = p.o + ((int64_t)b * p.S + qpos) * p.ldo + (int64_t)h * p.hd;
+      for (int c = 0; c < 2 * nd; ++c) {
+        uint32_t ov[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
+        tmem_ld_wait_regs(ov);
+        if (!store || 32 * c >= p.hd) continue;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        const int nv = min(32, p.hd - 32 * c) / 8;
+        for (int v = 0; v < nv; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+      if (store) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(l);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------------------------- backward pieces
+
+// delta[h][t] = sum_d dO[t, h hd + d] O[t, h hd + d]; one warp per (token, head).
+__global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ d_o,
+                                  int64_t ld, int64_t T, int hq, int hd, float* __restrict__ delta) {
+  pdl_wait();
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= T * hq) return;
+  const int64_t t = item / hq;
+  const int h = (int)(item % hq);
+  const __nv_bfloat16* a = o + t * ld + (int64_t)h * hd;
+  const __nv_bfloat16* c = d_o + t * ld + (int64_t)h * hd;
+  float acc = 0.f;
+  for (int d = lane; d < hd; d += 32) acc += __bfloat162float(a[d]) * __bfloat162float(c[d]);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) delta[(int64_t)h * T + t] = acc;
+}
+
+// dq[t * ldq + c] = bf16(acc[t * n + c]) for a [T, n] fp32 accumulator (n % 4 == 0), four
+// columns per thread.
+__global__ void attn_dq_cast_kernel(const float* __restrict__ acc, int64_t T, int64_t n, __nv_bfloat16* __restrict__ dq,
+                                    int64_t ldq) {
+  pdl_wait();
+  const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= T * n) return;
+  const int64_t t = i / n, c = i % n;
+  const float4 v = *reinterpret_cast<const float4*>(acc + i);
+  *reinterpret_cast<uint2*>(dq + t * ldq + c) = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
+}
+
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// ----------------------------------------------------------------------------------- backward
+
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nd = p.nd;
+  uint8_t* sk = smem;                  // K_j: nd chunks
+  uint8_t* sv = sk + nd * kChunk;      // V_j
+  uint8_t* sq = sv + nd * kChunk;      // Q_i
+  uint8_t* sdo = sq + nd * kChunk;     // dO_i
+  uint8_t* spt = sdo + nd * kChunk;    // P^T: 2 chunks (128 queries)
+  uint8_t* sdst = spt + 2 * kChunk;    // dS^T: 2 chunks
+  float* s_lse = reinterpret_cast<float*>(sdst + 2 * kChunk);  // [128]
+  float* s_delta = s_lse + 128;                                // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_delta + 128);
+  uint64_t* kv_full = bars;
+  uint64_t* qd_full = bars + 1;
+  uint64_t* qd_empty = bars + 2;
+  uint64_t* s_full = bars + 3;
+  uint64_t* p_full = bars + 4;
+  uint64_t* mma2_done = bars + 5;
+  uint64_t* dq_free = bars + 6;
+  uint64_t* drain = bars + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int hpg = p.hq / p.hkv;
+  const int n_qt = (p.S + kTile - 1) / kTile;
+  const int n_it = hpg * (n_qt - kt);  // (query head of the group, query tile >= kt)
+  const int64_t T = (int64_t)p.n_seq * p.S;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(qd_full, 1);
+    mbar_init(qd_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(mma2_done, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // TMEM: S^T, then dQ, at 0; dP^T at 128; dV at 256; dK at 256 + 64 nd
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_dv = 256, t_dk = 256 + 64 * nd;
+  pdl_wait();
+
+  auto it_head = [&](int it) { return g * hpg + it % hpg; };
+  auto it_qtile = [&](int it) { return kt + it / hpg; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * nd * kChunk);
+      for (int c = 0; c < nd; ++c) {
+        tma_load_4d(sk + c * kChunk, &p.kmap, kv_full, 64 * c, g, kt * kTile, b);
+        tma_load_4d(sv + c * kChunk, &p.vmap, kv_full, 64 * c, g, kt * kTile, b);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        if (it > 0 && !mbar_wait(qd_empty, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(qd_full, 2 * nd * kChunk);
+        const int h = it_head(it), qt = it_qtile(it);
+        for (int c = 0; c < nd; ++c) {
+          tma_load_4d(sq + c * kChunk, &p.qmap, qd_full, 64 * c, h, qt * kTile, b);
+          tma_load_4d(sdo + c * kChunk, &p.domap, qd_full, 64 * c, h, qt * kTile, b);
+        }
+        issued = it + 1;
+      }
+      mbar_wait(kv_full, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      if (issued > 0) mbar_wait(qd_full, (issued - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_kq = idesc_bf16(128, 128, 0, 0);       // S^T = K Q^T, dP^T = V dO^T
+      const uint32_t id_kd = idesc_bf16(128, 64 * nd, 0, 1);   // dV += P^T dO, dK += dS^T Q
+      const uint32_t id_qd = idesc_bf16(128, 64 * nd, 1, 1);   // dQ = dS K (dS read MN-major from dS^T)
+      const uint32_t ak = smem_u32(sk), av = smem_u32(sv), bq = smem_u32(sq), bdo = smem_u32(sdo);
+      const uint32_t apt = smem_u32(spt), adst = smem_u32(sdst);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, p.err, DEV_TIMEOUT_MMA);
+      for (int it = 0; ok && it < n_it; ++it) {
+        if (!mbar_wait(qd_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < 4 * nd; ++t) {
+          umma_bf16(tmem, kmajor_desc(ak, t), kmajor_desc(bq, t), id_kq, t > 0 ? 1u : 0u);
+          umma_bf16(tmem + 128, kmajor_desc(av, t), kmajor_desc(bdo, t), id_kq, t > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        if (!mbar_wait(p_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < 8; ++t) {
+          const uint32_t acc = (it > 0 || t > 0) ? 1u : 0u;
+          umma_bf16(tmem + t_dv, kmajor_desc(apt, t), mnmajor_desc(bdo, t), id_kd, acc);
+          umma_bf16(tmem + t_dk, kmajor_desc(adst, t), mnmajor_desc(bq, t), id_kd, acc);
+          umma_bf16(tmem, mnmajor_desc(adst, t), mnmajor_desc(ak, t), id_qd, t > 0 ? 1u : 0u);
+        }
+        umma_commit(mma2_done);
+        umma_commit(qd_empty);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;           // key row of the tile (S^T, dP^T, dV, dK) or query row (dQ)
+    const int kpos = kt * kTile + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float log2e = 1.4426950408889634f;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int h = it_head(it), qt = it_qtile(it);
+      const int qpos_r = qt * kTile + r;
+      // this tile's LSE and delta (the previous iteration's readers passed the barrier below)
+      named_bar_compute();
+      s_lse[r] = qpos_r < p.S ? p.lse[(int64_t)h * T + (int64_t)b * p.S + qpos_r] * log2e : 0.f;
+      s_delta[r] = qpos_r < p.S ? p.delta[(int64_t)h * T + (int64_t)b * p.S + qpos_r] : 0.f;
+      named_bar_compute();
+      if (!mbar_wait(s_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+      tc_fence_after();
+      // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S
+      const int cmin = kpos - qt * kTile;            // first visible query column
+      const int cmax = p.S - 1 - qt * kTile;         // last query column inside the sequence
+      for (int c = 0; c < 4; ++c) {
+        uint32_t st[32], dp[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + 32 * c, st);
+        tmem_ld32(tmem + lane_off + 128 + 32 * c, dp);
+        tmem_ld_wait_regs(st);
+        regs_after_wait(dp);
+        uint32_t pw[16], dw[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 32 * c + i + e;
+            const bool vis = col >= cmin && col <= cmax && kpos < p.S;
+            const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - s_lse[col]) : 0.f;
+            pv[e] = pe;
+            dv2[e] = pe * (__uint_as_float(dp[i + e]) - s_delta[col]);
+          }
+          pw[i / 2] = pack2(pv[0], pv[1]);
+          dw[i / 2] = pack2(dv2[0], dv2[1]);
+        }
+        st_swizzled_row32(spt, r, 32 * c, pw);
+        st_swizzled_row32(sdst, r, 32 * c, dw);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // dQ of this (head, query tile): lane r = query row qt * 128 + r
+      if (!mbar_wait(mma2_done, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+      tc_fence_after();
+      const bool qok = qpos_r < p.S;
+      float* dqrow = p.dq_acc + ((int64_t)b * p.S + qpos_r) * ((int64_t)p.hq * p.hd) + (int64_t)h * p.hd;
+      for (int c = 0; c < 2 * nd; ++c) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + 32 * c, v);
+        tmem_ld_wait_regs(v);
+        if (!qok || 32 * c >= p.hd) continue;
+        const int n = min(32, p.hd - 32 * c);
+        for (int i = 0; i < n; i += 4)
+          red_add_v4(dqrow + 32 * c + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
+                     __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+    // dK, dV of this key tile: the MMAs of the last iteration have completed (mma2_done); every lane
+    // takes part in the (warp-collective) loads, rows past the sequence store nothing
+    if (ok) {
+      tc_fence_after();
+      const bool kok = kpos < p.S;
+      const int64_t row = (int64_t)b * p.S + kpos;
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* out = (which ? p.dk : p.dv) + row * p.ldkv + (int64_t)g * p.hd;
+        const float mul = which ? p.scale : 1.f;
+        for (int c = 0; c < 2 * nd; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_off + (which ? t_dk : t_dv) + 32 * c, v);
+          tmem_ld_wait_regs(v);
+          if (!kok || 32 * c >= p.hd) continue;
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
+          uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
+          const int nv = min(32, p.hd - 32 * c) / 8;
+          for (int q = 0; q < nv; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [hd, heads, S, n_seq] view of a [n_seq * S, ld] bf16 matrix whose head h occupies columns
+// [h hd, (h + 1) hd); boxes of 64 x 1 x 128 x 1, 128-byte swizzle, zero fill outside.
+bool head_map(CUtensorMap* m, const void* ptr, int64_t ld, int n_seq, int S, int heads, int hd) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)S, (cuuint64_t)n_seq};
+  cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)ld * 2, (cuuint64_t)S * ld * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shared memory of a launch: sized for head_dim 128 whatever the head dimension, which also keeps
+// one CTA per SM (each CTA allocates all 512 TMEM columns).
+int fwd_smem() { return 1024 + 2 * kChunk + 8 * kChunk + 2 * kChunk + 256; }
+int bwd_smem() { return 1024 + 8 * kChunk + 4 * kChunk + 2 * 128 * 4 + 256; }
+
+}  // namespace
+
+int attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int64_t ldkv, int n_seq, int S, int hq,
+                  int hkv, int hd, void* o, int64_t ldo, float* lse, int* err, cudaStream_t s) {
+  AttnFwdParams p;
+  memset(&p, 0, sizeof(p));
+  if (!head_map(&p.qmap, q, ldq, n_seq, S, hq, hd) || !head_map(&p.kmap, k, ldkv, n_seq, S, hkv, hd) ||
+      !head_map(&p.vmap, v, ldkv, n_seq, S, hkv, hd))
+    return 2;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.ldo = ldo;
+  p.lse = lse;
+  p.n_seq = n_seq;
+  p.S = S;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.hd = hd;
+  p.nd = (hd + 63) / 64;
+  p.scale = 1.0f / std::sqrt((float)hd);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.err = err;
+  const int smem = fwd_smem();
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem()) != cudaSuccess)
+      return 5;
+    attr = true;
+  }
+  const dim3 grid((unsigned)((S + kTile - 1) / kTile), (unsigned)hq, (unsigned)n_seq);
+  launch_kernel(attn_fwd_kernel, grid, kAttnThreads, smem, s, p);
+  if (launch_failed("sl_attention")) return 5;
+  note_launch();
+  return 0;
+}
+
+size_t attention_bwd_scratch(int n_seq, int S, int hq, int hd) {
+  const size_t T = (size_t)n_seq * S;
+  return T * hq * hd * 4 + 256 + T * hq * 4;  // dQ accumulator, then delta
+}
+
+int attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                  int64_t ldq, int64_t ldkv, int n_seq, int S, int hq, int hkv, int hd, void* dq, void* dk, void* dv,
+                  void* scratch, int* err, cudaStream_t s) {
+  AttnBwdParams p;
+  memset(&p, 0, sizeof(p));
+  if (!head_map(&p.qmap, q, ldq, n_seq, S, hq, hd) || !head_map(&p.kmap, k, ldkv, n_seq, S, hkv, hd) ||
+      !head_map(&p.vmap, v, ldkv, n_seq, S, hkv, hd) || !head_map(&p.domap, d_o, ldq, n_seq, S, hq, hd))
+    return 2;
+  const int64_t T = (int64_t)n_seq * S;
+  float* dq_acc = static_cast<float*>(scratch);
+  float* delta = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + ((T * hq * hd * 4 + 255) & ~int64_t(255)));
+  if (cudaMemsetAsync(dq_acc, 0, (size_t)T * hq * hd * 4, s) != cudaSuccess) return 5;
+  {
+    const int64_t items = T * hq;
+    launch_kernel(attn_delta_kernel, (unsigned)((items + 7) / 8), 256, 0, s, static_cast<const __nv_bfloat16*>(o),
+                  static_cast<const __nv_bfloat16*>(d_o), ldq, T, hq, hd, delta);
+    if (launch_failed("sl_attention")) return 5;
+    note_launch();
+  }
+  p.lse = lse;
+  p.delta = delta;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.ldkv = ldkv;
+  p.n_seq = n_seq;
+  p.S = S;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.hd = hd;
+  p.nd = (hd + 63) / 64;
+  p.scale = 1.0f / std::sqrt((float)hd);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.err = err;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd_smem()) != cudaSuccess)
+      return 5;
+    attr = true;
+  }
+  const dim3 grid((unsigned)((S + kTile - 1) / kTile), (unsigned)hkv, (unsigned)n_seq);
+  launch_kernel(attn_bwd_kernel, grid, kAttnThreads, bwd_smem(), s, p);
+  if (launch_failed("sl_attention")) return 5;
+  note_launch();
+  // dQ: the dense [T, hq hd] accumulator to bf16 rows of leading dimension ldq
+  const int64_t n = (int64_t)hq * hd;
+  launch_kernel(attn_dq_cast_kernel, (unsigned)((T * n / 4 + 255) / 256), 256, 0, s, dq_acc, T, n,
+                static_cast<__nv_bfloat16*>(dq), ldq);
+  if (launch_failed("sl_attention")) return 5;
+  note_launch();
+  return 0;
+}
+
+}  // namespace sl

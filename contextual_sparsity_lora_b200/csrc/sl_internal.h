@@ -202,6 +202,19 @@ int add_rows(const void* a, int64_t lda, const void* b, int64_t ldb, void* out, 
 int adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, float lr, float b1, float b2,
                float eps, float wd, int step, cudaStream_t s);
 
+// ---- attention core of the decoder layer (sl_attention.cu)
+// Causal GQA attention over n_seq sequences of S tokens (rows in sequence order): o [T, hq hd]
+// (ld ldo), lse [hq][T] (natural log of each query row's softmax denominator, scores scaled by
+// 1 / sqrt(hd)). Returns 0, 2 (tensor map), 5 (launch).
+int attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int64_t ldkv, int n_seq, int S, int hq,
+                  int hkv, int hd, void* o, int64_t ldo, float* lse, int* err, cudaStream_t s);
+// Scratch bytes of attention_bwd: the fp32 dQ accumulator and the per-row delta = sum dO O.
+size_t attention_bwd_scratch(int n_seq, int S, int hq, int hd);
+// dq [T, hq hd] (ld ldq), dk, dv [T, hkv hd] (ld ldkv) from q, k, v, o, d_o and the forward's lse.
+int attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                  int64_t ldq, int64_t ldkv, int n_seq, int S, int hq, int hkv, int hd, void* dq, void* dk, void* dv,
+                  void* scratch, int* err, cudaStream_t s);
+
 // ---- criterion variants (sl_criteria.cu)
 // Wanda-style channel scores s_i = sum_p sum_j |W_p[i, j]| ||x[:, j]||_2 over n_ctx rows of x
 // (bf16 [n_ctx, d_in], ld ldx) and n_proj bf16 weights [d_out, d_in] (ld ldw); scratch holds

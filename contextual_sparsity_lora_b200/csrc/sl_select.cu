@@ -2,10 +2,9 @@
 //
 // Scores become order-preserving 32-bit keys (NaN lowest, -0 == +0), held in registers:
 // thread t owns the contiguous index range [t * per, (t + 1) * per). The n-th largest key
-// K* is found bit by bit from the most significant bit on: starting from the bits that all
-// keys share, a candidate bit is kept when at least n keys are >= the threshold with that
-// bit set (one block-wide count per bit; the search stops early when a threshold has
-// exactly n keys at or above it). Every key above K* is kept, and among keys equal to K*
+// K* is found by radix selection a byte at a time from the most significant byte in which two
+// keys differ (a shared-memory histogram of 256 bins per pass, at most four passes). Every key
+// above K* is kept, and among keys equal to K*
 // the lowest indices are kept, so exactly n channels survive. The output is a permutation
 // sigma of [0, N): sigma[0, n) = kept channels ascending, sigma[n, N) = dropped channels
 // ascending. Optionally the selection over KV units (g, d) is expanded to the query side:
@@ -84,6 +83,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   __shared__ int red[2][32];
   __shared__ uint32_t s_or[32], s_and[32];
   __shared__ int warp_sums[32];
+  __shared__ int hist[256];
+  __shared__ int sel_state[2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per = (n + kSelThreads - 1) / kSelThreads;  // <= PER
   const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
@@ -110,23 +111,68 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   __syncthreads();
   const uint32_t bor = __reduce_or_sync(0xffffffffu, s_or[lane]);
   const uint32_t band = __reduce_and_sync(0xffffffffu, s_and[lane]);
-  // Every key carries the bits above the highest bit in which two keys differ: the search
-  // starts below it, from a threshold that all n keys reach.
+  // The n-th largest key K* by radix selection, 8 bits per pass from the byte holding the highest
+  // bit in which two keys differ (every key shares the bits above it): per pass, a 256-bin
+  // histogram of the next byte over the keys that match the bytes chosen so far; the chosen byte is
+  // the one where the count of matching keys with a larger byte stops falling short of the places
+  // still to fill. After the last pass T = K* exactly, and `need` keys equal to T are to be kept.
   const uint32_t diff = bor ^ band;
-  int b = diff ? 31 - __clz(diff) : -1;
-  uint32_t T = diff ? (band & ~((2u << b) - 1u)) : band;
-  int slot = 0;
-  for (; b >= 0; --b) {
-    const uint32_t Tp = T | (1u << b);
-    int c = 0;
+  const int top = diff ? 31 - __clz(diff) : -1;  // highest bit in which two keys differ
+  uint32_t T = band;                              // every byte at or above top's is decided below
+  uint32_t tmask = 0u;
+  int need = n_keep;
+  if (top >= 0) {
+    const int first = (top / 8) * 8;
+    tmask = first + 8 < 32 ? ~((1u << (first + 8)) - 1u) : 0u;  // bytes above the first pass
+    T &= tmask;
+    for (int shift = first; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
 #pragma unroll
-    for (int j = 0; j < PER; ++j) c += key[j] >= Tp ? 1 : 0;  // padding keys are 0 < Tp
-    const int tot = block_sum(c, red, slot);
-    if (tot >= n_keep) {
-      T = Tp;
-      if (tot == n_keep) break;  // exactly n keys at or above T
+      for (int j = 0; j < PER; ++j)
+        if (i0 + j < i1 && (key[j] & tmask) == T) atomicAdd(&hist[(key[j] >> shift) & 255u], 1);
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds bins 255 - 8 l .. 248 - 8 l (descending); counts from the top
+        int c[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[255 - 8 * lane - e];
+          tot += c[e];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += nb;
+        }
+        int above = incl - tot;  // matching keys whose byte lies above this lane's bins
+        int pick = -1, above_pick = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (pick < 0 && above < need && above + c[e] >= need) {
+            pick = 255 - 8 * lane - e;
+            above_pick = above;
+          }
+          above += c[e];
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, pick >= 0);  // one lane holds the crossing
+        const int src = who ? __ffs(who) - 1 : 0;
+        pick = __shfl_sync(0xffffffffu, pick, src);
+        above_pick = __shfl_sync(0xffffffffu, above_pick, src);
+        if (lane == 0) {
+          sel_state[0] = pick < 0 ? 0 : pick;
+          sel_state[1] = above_pick;
+        }
+      }
+      __syncthreads();
+      T |= (uint32_t)sel_state[0] << shift;
+      need -= sel_state[1];
+      tmask |= 255u << shift;
+      __syncthreads();  // sel_state and hist are rewritten by the next pass
     }
   }
+  int slot = 0;
   // Keys above T are kept; keys equal to T fill the remaining places lowest index first.
   int gt = 0, n_eq = 0;
 #pragma unroll

@@ -6,16 +6,14 @@ computed with the sparse projections).
     h1 = RMSNorm(x, g1); q, k, v = sparse projections of h1; a = causal GQA attention(q, k, v)
     x2 = x + o(a); h2 = RMSNorm(x2, g2); y = x2 + FFN(h2)
 
-RMSNorm, the residual adds and every projection run in libsparselora's kernels; the attention
-core (not one of the method's steps) is torch's scaled_dot_product_attention, a library call
-like a cuBLAS GEMM, with its backward through autograd. Rows are in context-first order like
-the blocks' (sl_permute_rows moves q, k, v to sequence order for the attention core and its
-output back). No rotary positional encoding: the pages do not say how it meets channel
-sparsity (a rotation mixes channel pairs that the selection may split)."""
+RMSNorm, the residual adds, every projection and the causal grouped-query attention core
+(sl_attention_fwd / sl_attention_bwd, tcgen05 kernels) run in libsparselora's kernels. Rows are
+in context-first order like the blocks' (sl_permute_rows moves q, k, v to sequence order for the
+attention core and its output back). No rotary positional encoding: the pages do not say how it
+meets channel sparsity (a rotation mixes channel pairs that the selection may split)."""
 from __future__ import annotations
 
 import torch
-import torch.nn.functional as Fn
 
 from . import binding as B
 from .blocks import AttnProjBlock, FFNBlock
@@ -46,10 +44,13 @@ class DecoderLayer:
         self.rstd1, self.rstd2 = e(T, dt=f32), e(T, dt=f32)
         Dq, Dkv = attn.Dq, attn.Dkv
         self.q_nat, self.k_nat, self.v_nat = e(T, Dq), e(T, Dkv), e(T, Dkv)
-        self.a_cf = e(T, Dq)
+        self.a_nat, self.a_cf = e(T, Dq), e(T, Dq)
+        self.lse = e(attn.hq, T, dt=f32)
         self.da_nat = e(T, Dq)
+        self.dq_nat, self.dk_nat, self.dv_nat = e(T, Dq), e(T, Dkv), e(T, Dkv)
         self.dq_cf, self.dk_cf, self.dv_cf = e(T, Dq), e(T, Dkv), e(T, Dkv)
         self.dx2, self.dx = e(T, D), e(T, D)
+        self.ws = B.Workspace(dev)  # the attention core's scratch (the dq accumulator) and error word
 
     def _to_seq(self, src, dst):
         B.sl_permute_rows(src, self.inv, dst)
@@ -57,24 +58,15 @@ class DecoderLayer:
     def _to_cf(self, src, dst):
         B.sl_permute_rows(src, self.perm, dst)
 
-    def _heads(self, t, n_heads):
-        """[T, n_heads * hd] sequence-order rows -> [n_seq, n_heads, S, hd] view."""
-        return t.view(self.n_seq, self.S, n_heads, self.attn.hd).transpose(1, 2)
-
     def forward(self, x):
         at = self.attn
         B.sl_rmsnorm_fwd(x, self.g1, self.eps, self.h1, self.rstd1)
         q, k, v = at.forward_qkv(self.h1)
         for src, dst in ((q, self.q_nat), (k, self.k_nat), (v, self.v_nat)):
             self._to_seq(src, dst)
-        self._q = self._heads(self.q_nat, at.hq).detach().requires_grad_()
-        self._k = self._heads(self.k_nat, at.hkv).detach().requires_grad_()
-        self._v = self._heads(self.v_nat, at.hkv).detach().requires_grad_()
-        with torch.enable_grad():
-            self._a = Fn.scaled_dot_product_attention(self._q, self._k, self._v, is_causal=True,
-                                                      enable_gqa=at.hq != at.hkv)
-        a_nat = self._a.detach().transpose(1, 2).reshape(self.T, at.Dq)
-        self._to_cf(a_nat.contiguous(), self.a_cf)
+        B.sl_attention_fwd(self.ws, self.q_nat, self.k_nat, self.v_nat, self.n_seq, at.hq, at.hkv, at.hd, self.a_nat,
+                           self.lse)
+        self._to_cf(self.a_nat, self.a_cf)
         o = at.forward_o(self.a_cf)
         # x2 = x + o (the residual stream) and h2 = RMSNorm(x2) in one pass
         B.sl_rmsnorm_fwd(o, self.g2, self.eps, self.h2, self.rstd2, res=x, sum_out=self.x2)
@@ -89,13 +81,17 @@ class DecoderLayer:
         B.sl_rmsnorm_bwd(dh2, self.x2, self.g2, self.rstd2, self.dx2, dres=dy)
         da_cf = at.backward_o(self.dx2)
         self._to_seq(da_cf, self.da_nat)
-        dq, dk, dv = torch.autograd.grad(self._a, (self._q, self._k, self._v),
-                                         self._heads(self.da_nat, at.hq))
-        for g, n_h, dst in ((dq, at.hq, self.dq_cf), (dk, at.hkv, self.dk_cf), (dv, at.hkv, self.dv_cf)):
-            self._to_cf(g.transpose(1, 2).reshape(self.T, n_h * at.hd).contiguous(), dst)
+        B.sl_attention_bwd(self.ws, self.q_nat, self.k_nat, self.v_nat, self.a_nat, self.da_nat, self.lse, self.n_seq,
+                           at.hq, at.hkv, at.hd, self.dq_nat, self.dk_nat, self.dv_nat)
+        for src, dst in ((self.dq_nat, self.dq_cf), (self.dk_nat, self.dk_cf), (self.dv_nat, self.dv_cf)):
+            self._to_cf(src, dst)
         dh1 = at.backward_qkv(self.dq_cf, self.dk_cf, self.dv_cf)
         B.sl_rmsnorm_bwd(dh1, self.x, self.g1, self.rstd1, self.dx, dres=self.dx2)
         return self.dx
+
+    def read_device_flag(self) -> int:
+        """Device error word of the attention core's workspace (0: no device-side timeout); synchronises."""
+        return self.ws.read_device_flag()
 
     def step(self, x, dy):
         self.forward(x)

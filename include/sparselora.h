@@ -353,6 +353,35 @@ SL_API sl_status sl_profile_read(int64_t* kernel_launches, int64_t* gemm_launche
  * stream) or 4 (estimator stage 1). Waits for the events. */
 SL_API sl_status sl_profile_launches(int64_t capacity, double* ms, int32_t* kind, int64_t* count);
 
+/* The decoder layer's attention core between the sparse q/k/v and o projections ("SparseLoRA:
+ * Accelerating LLM Fine-Tuning with Contextual Sparsity", walkthrough, "Putting It All Together":
+ * output rows attend to the context keys and values the sparse projections computed). Causal,
+ * grouped-query, no positional rotation, scores scaled by 1 / sqrt(head_dim), on the tcgen05
+ * tensor cores (S = Q K^T and O = P V per 128-query tile with the softmax between them; the
+ * backward recomputes P from the forward's row log-sum-exp).
+ *   Rows are tokens in sequence order: n_seq sequences of seq_len tokens, T = n_seq * seq_len.
+ *   q, o, d_o, dq: bf16 [T, n_q_heads * head_dim], leading dimension ldq (query head h in columns
+ *     [h head_dim, (h + 1) head_dim)); k, v, dk, dv: bf16 [T, n_kv_heads * head_dim], leading
+ *     dimension ldkv. Query head h attends with key/value head h / (n_q_heads / n_kv_heads).
+ *   lse: fp32 [n_q_heads][T], written by the forward (natural log of sum_k exp(score)) and read by
+ *     the backward.
+ *   sl_attention_fwd: o[t] = sum over keys s <= t of the same sequence of softmax(q k^T) v.
+ *   sl_attention_bwd: dq, dk, dv of the loss whose gradient at o is d_o. dq is summed across key
+ *     tiles in fp32 reductions whose order varies between runs (last bits of dq may differ); dk and
+ *     dv are run-to-run identical. Workspace: 4 n_q_heads head_dim T + 4 n_q_heads T bytes past
+ *     the header (fp32 dq accumulator, per-row sum of d_o o).
+ * head_dim in [8, 128], a multiple of 8; n_q_heads a multiple of n_kv_heads; every pointer 16-byte
+ * aligned, ldq and ldkv multiples of 8. Errors: SL_ERR_INVALID_ARG (null pointer), SL_ERR_SHAPE,
+ * SL_ERR_ALIGNMENT, SL_ERR_WORKSPACE (backward: ws->needed holds the size; the forward needs only
+ * the header, whose error word receives device-side timeouts of both). */
+SL_API sl_status sl_attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int64_t ldkv,
+                                  int32_t n_seq, int32_t seq_len, int32_t n_q_heads, int32_t n_kv_heads,
+                                  int32_t head_dim, void* o, float* lse, sl_workspace* ws, sl_stream stream);
+SL_API sl_status sl_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                                  const float* lse, int64_t ldq, int64_t ldkv, int32_t n_seq, int32_t seq_len,
+                                  int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, void* dq, void* dk,
+                                  void* dv, sl_workspace* ws, sl_stream stream);
+
 /* Tile height of the CTA-pair tensor-core GEMM that runs the sliced products (a4, a5):
  * rows = 256 (each pair of SMs computes 256 x 256 output tiles with two accumulators, so a
  * tile's epilogue overlaps the next tile's products), 512 (512 x 256 tiles: a quarter fewer
