@@ -310,12 +310,14 @@ def time_steps(fn, K, W, world, device):
 
 
 def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
-    """Device time of the selection stages of both blocks, each captured alone in a CUDA
-    graph (`inner` back-to-back copies of the stage per graph, so that the host's graph
-    launches do not pace tiny stages) and replayed `reps` times: a1 (estimator stage 1, the
-    tensor-core launch of sl_svd_estimate, event-timed in a profiled copy), a2 (the rest of
-    sl_svd_estimate: the criterion), a3 (sl_select_channels) and the per-step compaction of
-    the kept weight rows."""
+    """Device time of the selection stages of both blocks, each captured alone in a CUDA graph
+    (`inner` back-to-back copies of the stage per graph, so that the host's graph launches do not
+    pace tiny stages) and replayed `reps` times. The step runs the estimator's stage 1 (a1, Z =
+    X_ctx W_A) as extra columns of the LoRA x A^T launch that streams the same rows
+    (sl_lora_fwd_estimate): its cost is the difference between that launch and the x A^T launch
+    alone. Then a2 (sl_svd_scores_from_z: the criterion from Z), a3 (sl_select_channels) and the
+    per-step compaction of the kept weight rows. The standalone estimator (sl_svd_estimate: its own
+    pass over X_ctx, then the criterion) is timed beside it for reference."""
     from contextual_sparsity_lora_b200 import binding as B
     inner = 10
 
@@ -328,33 +330,36 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
         g = capture_graph(many, warm=False)
         return time_steps(g.replay, reps, 3, 1, device) / (reps * inner) * 1e3
 
-    def a1_us(fn):
-        B.sl_profile_read()
-        B.sl_profile_enable(True)
-        g = capture_graph(fn, warm=False)
-        B.sl_profile_enable(False)
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        _, n_gemm, ms = B.sl_profile_read()
-        del g
-        return ms * 1e3 if n_gemm == 1 else None
-
     out = {}
     total = 0.0
     for name, blk, x in (("attn", attn, s["x"]), ("ffn", ffn, s["ffn_x"])):
         C, D = blk.n_ctx, x.shape[1]
-        est = graph_us(lambda: blk.estimate(x))
-        a1 = a1_us(lambda: blk.estimate(x))
+        T = x.shape[0]
+        if name == "attn":
+            lins = [blk.lin[n] for n in "qkv"]
+            xa, xa_s, crit, n_proj = blk.xa_qkv, blk.xa_s_qkv, B.SL_CRIT_QK, 3
+            kw = dict(scores_v=blk.s_v, n_q_heads=blk.hq, n_kv_heads=blk.hkv, head_dim=blk.hd)
+            sc, WB = blk.s_qk, blk.WB
+        else:
+            lins = [blk.lin_g, blk.lin_u]
+            xa, xa_s, crit, n_proj = blk.xa_gu, blk.xa_s_gu, B.SL_CRIT_SWIGLU_L2, 2
+            kw = {}
+            sc, WB = blk.scores, [blk.WBg, blk.WBu]
+        lora_us = graph_us(lambda: B.sl_lora_fwd_bwd(blk.ws, B.SL_LORA_FWD, lins, x, C, xa_s, xa=xa))
+        fused_us = graph_us(lambda: B.sl_lora_fwd_estimate(blk.ws, lins, x, C, xa_s, xa, n_proj, blk.k, blk.WAt,
+                                                          blk.z))
+        a2 = graph_us(lambda: B.sl_svd_scores_from_z(blk.ws, crit, WB, blk.k, blk.z, C, sc, **kw))
         sel = graph_us(blk.choose)
         comp = graph_us(blk.compact)
-        n_proj = 3 if name == "attn" else 2
-        a1_bytes = C * D * 2 + n_proj * D * blk.k * 2  # X_ctx once, plus the rank-k factors W_A
-        out[name] = {"a1_a2_estimate_us": est, "a1_stage1_us": a1,
-                     "a1_bytes": a1_bytes, "a1_GBs": a1_bytes / (a1 * 1e3) if a1 else None,
-                     "a1_frac_of_hbm": a1_bytes / (a1 * 1e3) / hbm_gbs if a1 else None,
-                     "a2_criterion_us": est - a1 if a1 else None, "a3_select_us": sel, "compact_weights_us": comp}
-        total += est + sel
+        standalone = graph_us(lambda: blk.estimate(x))
+        a1 = max(fused_us - lora_us, 0.0)
+        fused_bytes = T * D * 2 + (sum(l.r for l in lins) + n_proj * blk.k) * D * 2
+        out[name] = {"a1_marginal_us": a1, "lora_x_at_us": lora_us, "lora_x_at_with_z_us": fused_us,
+                     "fused_launch_bytes": fused_bytes, "fused_launch_GBs": fused_bytes / (fused_us * 1e3),
+                     "fused_launch_frac_of_hbm": fused_bytes / (fused_us * 1e3) / hbm_gbs,
+                     "a2_criterion_us": a2, "a3_select_us": sel, "compact_weights_us": comp,
+                     "standalone_estimator_us": standalone}
+        total += a1 + a2 + sel
     # criterion ablation variants (not on the step's path): the Wanda-style FFN criterion
     # (reads X_ctx and the gate and up weights once) and the head-level QK selection
     C, D, F = ffn.n_ctx, ffn.D, ffn.F
@@ -373,7 +378,8 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
     out["estimator_and_select_us"] = total
     if step_ms:
         out["estimator_and_select_pct_of_step"] = 100.0 * total / (step_ms * 1e3)
-    out["timing"] = "each stage alone, 10 copies per CUDA graph, replayed; device time between events"
+    out["timing"] = ("each stage alone, 10 copies per CUDA graph, replayed; device time between events; "
+                     "a1 = the x A^T launch with Z minus the x A^T launch alone")
     return out
 
 
@@ -863,7 +869,7 @@ def main():
     skinny_bytes = flops.lora_skinny_bytes([(T, ac.hidden, (ac.n_q_heads * ac.head_dim, 2 * ac.n_kv_heads * ac.head_dim)),
                                             (T, ac.n_q_heads * ac.head_dim, (ac.hidden,)),
                                             (T, fc.hidden, (2 * fc.inter,)), (T, fc.inter, (fc.hidden,))])
-    skinny_bytes += 2 * C * ac.hidden * 2  # estimator stage 1 reads X_ctx once per block
+    # (the estimator's stage 1 rides in the x A^T launches of q/k/v and gate/up: no bytes of its own)
     hbm = float(peaks.get("hbm_gbs", 6650.0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -886,6 +892,8 @@ def main():
                      "launches_per_step": pair_n, "ms_per_launch": pair_ms / max(pair_n, 1),
                      "gemm_engine_ms_per_step": gemm_ms, "gemm_engine_launches_per_step": n_gemm,
                      "skinny_lora_and_stage1": {"bound": "hbm", "ms_per_step": skinny_ms,
+                                                "what": "one-CTA rank-r launches (x A^T with the estimator's Z, "
+                                                        "dA = dya^T x) and the fused LoRA backward",
                                                 "launches_per_step": skinny_n,
                                                 "algorithmic_bytes_per_step": skinny_bytes,
                                                 "achieved_GBs": skinny_bytes / (skinny_ms * 1e6) if skinny_ms else None,

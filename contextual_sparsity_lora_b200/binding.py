@@ -31,7 +31,8 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_svd_estimate_noalloc", "sl_profile_launches", "sl_svd_partials_count", "sl_svd_estimate_partials",
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
             "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows",
-            "sl_debug_bounds_enabled", "sl_read_debug_flag", "sl_attention_fwd", "sl_attention_bwd")
+            "sl_debug_bounds_enabled", "sl_read_debug_flag", "sl_attention_fwd", "sl_attention_bwd",
+            "sl_lora_fwd_estimate", "sl_svd_scores_from_z")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -134,6 +135,10 @@ def load(path):
     L.sl_permute_rows.argtypes = [P, c_int64, c_int64, P, c_int64, c_int64, P, c_int64, P]
     L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P, P]
     L.sl_debug_bounds_enabled.restype = c_int32
+    L.sl_lora_fwd_estimate.argtypes = [c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, P, P, c_int64,
+                                       c_int32, c_int32, P, c_int64, P, c_int64, POINTER(SlWorkspaceC), P]
+    L.sl_svd_scores_from_z.argtypes = [c_int32, c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, c_int32, c_int32,
+                                       c_int32, P, c_int64, c_int64, P, P, POINTER(SlWorkspaceC), P]
     L.sl_attention_fwd.argtypes = [P, P, P, c_int64, c_int64, c_int32, c_int32, c_int32, c_int32, c_int32, P, P,
                                    POINTER(SlWorkspaceC), P]
     L.sl_attention_bwd.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int32, c_int32, c_int32, c_int32, c_int32,
@@ -250,6 +255,21 @@ def sl_svd_estimate_noalloc(crit, x, n_ctx, w_a, w_b, k, scores, scores_v=None, 
                                          int(n_kv_heads), int(head_dim), _ptr(scores), _ptr(scores_v),
                                          ctypes.byref(needed), _ptr(device_flag), _stream()))
     return int(needed.value)
+
+
+def sl_lora_fwd_estimate(ws: Workspace, lins, x, n_ctx, xa_s, xa, n_proj, k, w_a_t, z):
+    """x A^T of the adapters (xa, xa_s) and the estimator's Z = X_ctx W_A (z [n_ctx, n_proj k] fp32)
+    from one pass over x; w_a_t [n_proj k, d_in] bf16 stacks the transposed factors."""
+    ws.call("sl_lora_fwd_estimate", len(lins), _arr(SlLinearC, list(lins)), _ptr(x), x.stride(0), x.shape[0],
+            int(n_ctx), _ptr(xa), _ptr(xa_s), xa_s.stride(0), int(n_proj), int(k), _ptr(w_a_t), w_a_t.stride(0),
+            _ptr(z), z.stride(0))
+
+
+def sl_svd_scores_from_z(ws: Workspace, crit, w_b, k, z, n_ctx, scores, scores_v=None, n_q_heads=0, n_kv_heads=0,
+                         head_dim=0):
+    ws.call("sl_svd_scores_from_z", int(crit), len(w_b), _ptrs(list(w_b)), _i64s([t.shape[1] for t in w_b]), int(k),
+            int(n_q_heads), int(n_kv_heads), int(head_dim), _ptr(z), z.stride(0), int(n_ctx), _ptr(scores),
+            _ptr(scores_v))
 
 
 def sl_svd_partials_count(crit, w_b, k):

@@ -147,6 +147,15 @@ class FFNBlock:
         self.dp = dp if dp is not None and dp.active else None
         self.est_part = _empty((F,), torch.float64, device) if self.dp else None
         self.dx = _empty((T, D), bf, device)
+        # the estimator's stage 1 inside the gate/up x A^T launch (one pass over x): single rank,
+        # the method's criterion, bf16 factors
+        self.fold = (criterion == "svd" and self.dp is None and self.est_dtype == bf and self.k in (4, 8, 16)
+                     and n_ctx > 0 and not self.dense)
+        if self.fold:
+            self.WAt = _empty((2 * self.k, D), bf, device)  # [W_A(gate)^T; W_A(up)^T]
+            B.sl_prepare_weight(self.WAg, self.WAt[: self.k])
+            B.sl_prepare_weight(self.WAu, self.WAt[self.k:])
+            self.z = _empty((n_ctx, 2 * self.k), f32, device)
         # kept rows of the sliced weights, rebuilt once per step and shared by the forward
         # and backward calls (the weights themselves when nothing is dropped)
         if self.dense:
@@ -218,7 +227,23 @@ class FFNBlock:
         # no context rows: nothing to score, every row is dense (data-parallel ranks still take
         # part in the selection of the batch)
         down_side = False
-        if not self.dense and (C > 0 or self.dp):
+        if not self.dense and self.fold and x_est is None:
+            # x A^T of gate/up and the estimator's Z from one pass over x, then the criterion
+            # from Z, the selection and the kept rows (down's on the second stream)
+            B.sl_lora_fwd_estimate(self.ws, [self.lin_g, self.lin_u], x, C, self.xa_s_gu, self.xa_gu, 2, self.k,
+                                   self.WAt, self.z)
+            B.sl_svd_scores_from_z(self.ws, B.SL_CRIT_SWIGLU_L2, [self.WBg, self.WBu], self.k, self.z, C,
+                                   self.scores)
+            self.choose()
+            kept = self.sigma[: self.n_keep]
+            B.sl_gather_rows_batch([self.Wg, self.Wu], [kept] * 2, [self.Wg_k, self.Wu_k])
+            if self.concurrent:
+                with self.side.fork():
+                    B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+                down_side = True
+            else:
+                B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+        elif not self.dense and (C > 0 or self.dp):
             if self.concurrent:  # x A^T of gate/up does not depend on the selection
                 with self.side.fork():
                     B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
@@ -347,6 +372,15 @@ class AttnProjBlock:
                                device) if self.dp else None
         self.dx_o = _empty((T, self.Dq), bf, device)
         self.dx = _empty((T, D), bf, device)
+        # the estimator's stage 1 inside the q/k/v x A^T launch (one pass over x): single rank, the
+        # method's criteria, factor widths the fused product takes
+        self.fold = ((qk_criterion, vo_criterion) == ("channel", "l2") and self.dp is None and est_k % 4 == 0
+                     and 3 * est_k <= 64 and n_ctx > 0 and not self.dense)
+        if self.fold:
+            self.WAt = _empty((3 * est_k, D), bf, device)  # [W_A(q)^T; W_A(k)^T; W_A(v)^T]
+            for j in range(3):
+                B.sl_prepare_weight(self.WA[j], self.WAt[j * est_k:(j + 1) * est_k])
+            self.z = _empty((n_ctx, 3 * est_k), f32, device)
         s = self.scale
         # kept rows of the sliced weights (rows of W for q, k, v; rows of W^T for o), rebuilt
         # once per step after the selection and shared by the forward and backward calls
@@ -399,6 +433,27 @@ class AttnProjBlock:
             return
         B.sl_svd_estimate(self.ws, B.SL_CRIT_QK, x[:C], C, self.WA, self.WB, self.k, self.s_qk, scores_v=self.s_v,
                           n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+
+    def _estimate_fused(self, x, ws):
+        """x A^T of q, k, v together with the estimator's Z (one pass over x), then the QK and V
+        scores from Z."""
+        C = self.n_ctx
+        lq, lk, lv = (self.lin[n] for n in "qkv")
+        B.sl_lora_fwd_estimate(ws, [lq, lk, lv], x, C, self.xa_s_qkv, self.xa_qkv, 3, self.k, self.WAt, self.z)
+        B.sl_svd_scores_from_z(ws, B.SL_CRIT_QK, self.WB, self.k, self.z, C, self.s_qk, scores_v=self.s_v,
+                               n_q_heads=self.hq, n_kv_heads=self.hkv, head_dim=self.hd)
+
+    def _choose_and_compact(self):
+        """The q/k and v/o selections with their kept weight rows: two independent chains (the
+        v/o one on the second stream when concurrent)."""
+        if self.concurrent:
+            with self.side.fork():
+                self._vo_chain()
+            self._qk_chain()
+            self.side.join()
+        else:
+            self.choose()
+            self.compact()
 
     def _select_qk(self):
         if self.qk_criterion == "head":
@@ -462,7 +517,19 @@ class AttnProjBlock:
             B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
             B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
 
-        if sel and self.concurrent:
+        if sel and self.fold:
+            if self.concurrent:
+                with self.side.fork():  # x_o A^T does not depend on the selection
+                    B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+                o_done = self.side.mark()
+                self._estimate_fused(x, self.ws)
+                self._choose_and_compact()
+                torch.cuda.current_stream().wait_event(o_done)
+            else:
+                B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+                self._estimate_fused(x, self.ws)
+                self._choose_and_compact()
+        elif sel and self.concurrent:
             with self.side.fork():
                 lora_fwd(self.side.ws)
             self.select(x)
@@ -516,7 +583,10 @@ class AttnProjBlock:
         self.x = x
         lq, lk, lv = (self.lin[n] for n in "qkv")
         sel = not self.dense and (C > 0 or self.dp is not None)
-        if sel and self.concurrent:
+        if sel and self.fold:
+            self._estimate_fused(x, self.ws)
+            self._choose_and_compact()
+        elif sel and self.concurrent:
             with self.side.fork():
                 B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
             self.select(x)

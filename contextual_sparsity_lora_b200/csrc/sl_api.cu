@@ -685,6 +685,109 @@ sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linear* lin,
   return SL_OK;
 }
 
+// a1 inside the LoRA forward: x A^T of the adapters and Z = X_ctx W_A of the estimator from one pass
+// over x (the factors W_A^T as extra B rows of the same skinny product).
+sl_status sl_lora_fwd_estimate(int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx, int64_t n_tok,
+                               int64_t n_ctx, float* xa, void* xa_s, int64_t ld_xa, int32_t n_proj, int32_t k,
+                               const void* w_a_t, int64_t ld_wat, float* z, int64_t ld_z, sl_workspace* ws,
+                               sl_stream stream) {
+  if (!lin || !x || !xa || !w_a_t || !z || n_ad < 1 || n_ad > kMaxBSrc - 1) return SL_ERR_INVALID_ARG;
+  if (n_tok <= 0 || n_ctx < 0 || n_ctx > n_tok) return SL_ERR_SHAPE;
+  if (k < 1 || k > 16 || n_proj < 1) return SL_ERR_SHAPE;
+  const int mk = n_proj * k;
+  const int64_t d_in = lin[0].d_in;
+  int R = 0;
+  for (int i = 0; i < n_ad; ++i) {
+    if (!linear_ok(lin[i]) || lin[i].d_in != d_in) return SL_ERR_INVALID_ARG;
+    if (lin[i].lora_scale != lin[0].lora_scale) return SL_ERR_UNSUPPORTED;
+    R += lin[i].r;
+  }
+  if (mk > 64 || mk % 4 || R + mk > 256) return SL_ERR_SHAPE;
+  if (ld_z < mk) return SL_ERR_SHAPE;
+  if (ldx < d_in || ldx % 8 || !al16(x)) return SL_ERR_ALIGNMENT;
+  if (ld_wat < d_in || ld_wat % 8 || !al16(w_a_t)) return SL_ERR_ALIGNMENT;
+  if (!xa_s || ld_xa < R || ld_xa % 8 || !al16(xa_s)) return SL_ERR_ALIGNMENT;
+  const int64_t T = n_tok;
+  const int N = R + mk;
+  const int64_t red = split_floats(T, N, d_in);
+  {
+    Carver c(nullptr);
+    c.take<float>((size_t)red);
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  float* region = c.take<float>((size_t)red);
+  GemmBuilder gb;
+  int64_t off = 0;
+  const int mx = gb.map(x, T, d_in, ldx, kBM);
+  Prob* p = gb.add((int)T, N, kBN, (int)rup(N, 16));
+  Seg* sg = gb.seg(p, mx, 0, 0, 0, 0, 0, (int)d_in, kBig);
+  int toff = 0;
+  for (int i = 0; i < n_ad; ++i) {
+    gb.bsrc(sg, gb.map(lin[i].lora_a, lin[i].r, d_in, d_in, lin[i].r), toff, lin[i].r, 0, 0);
+    toff += lin[i].r;
+  }
+  gb.bsrc(sg, gb.map(w_a_t, mk, d_in, ld_wat, mk), toff, mk, 0, 0);
+  if (p) {
+    p->epi = EPI_XA;
+    p->out0 = xa;
+    p->ld0 = ld_xa;
+    p->out1 = xa_s;
+    p->ld1 = ld_xa;
+    p->a0 = 1.f;
+    p->a1 = lin[0].lora_scale;
+    p->z_col0 = R;
+    p->z_rows = (int32_t)n_ctx;
+    p->out2 = z;
+    p->ld2 = ld_z;
+  }
+  maybe_split(gb, p, T, N, d_in, region, &off);
+  return from_builder(gb.launch(err_word(ws), cs(stream)));
+}
+
+// a2 from a Z computed by sl_lora_fwd_estimate.
+sl_status sl_svd_scores_from_z(sl_criterion crit, int32_t n_proj, const void* const* w_b, const int64_t* d_out,
+                               int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, const float* z,
+                               int64_t ld_z, int64_t n_ctx, float* scores, float* scores_v, sl_workspace* ws,
+                               sl_stream stream) {
+  if (!z || !scores) return SL_ERR_INVALID_ARG;
+  int64_t n_units = 0;
+  if (sl_status st = criterion_units(crit, n_proj, w_b, d_out, k, n_q_heads, n_kv_heads, head_dim, !scores_v,
+                                     &n_units))
+    return st;
+  const int mk = n_proj * k;
+  if (n_ctx <= 0 || ld_z < mk || mk % 4) return SL_ERR_SHAPE;
+  const int64_t tiles = (n_ctx + 127) / 128;
+  const bool linear = crit != SL_CRIT_SWIGLU_L2;
+  auto carve = [&](Carver& c, double** gp, uint16_t** zs) {
+    *gp = linear ? c.take<double>((size_t)tiles * mk * mk) : nullptr;
+    *zs = linear ? nullptr : c.take<uint16_t>((size_t)n_ctx * 128);
+  };
+  double* gp;
+  uint16_t* zs;
+  {
+    Carver c(nullptr);
+    carve(c, &gp, &zs);
+    if (sl_status st = ws_check(ws, c.off)) return st;
+  }
+  Carver c(ws->ptr);
+  carve(c, &gp, &zs);
+  cudaStream_t s = cs(stream);
+  if (int rc = z_finish(z, ld_z, n_ctx, mk, k, gp, zs, s)) return from_kernel(rc);
+  int rc;
+  if (!linear) {
+    rc = est_swiglu_tc(zs, n_ctx, k, w_b[0], w_b[1], n_units, scores, nullptr, err_word(ws), s);
+    return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
+  }
+  if (crit == SL_CRIT_L2)
+    rc = est_scores(gp, (int)tiles, mk, k, 0, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0, n_units, scores, s);
+  else
+    rc = est_scores(gp, (int)tiles, mk, k, 0, w_b[0], w_b[1], 0, 1, n_q_heads, n_kv_heads, head_dim, scores,
+                    n_proj == 3 ? w_b[2] : nullptr, 2, n_proj == 3 ? d_out[2] : 0, n_proj == 3 ? scores_v : nullptr,
+                    s);
+  return from_kernel(rc);
+}
+
 // ------------------------------------------------------------------ a4
 sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_channels* ch, int32_t epi, const void* x,
                                int64_t ldx, int64_t n_tok, int64_t n_ctx, int32_t in_layout, int32_t out_layout,

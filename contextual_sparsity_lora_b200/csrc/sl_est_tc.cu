@@ -68,13 +68,14 @@ __device__ __forceinline__ void stage_bar() { asm volatile("bar.sync 2, 160;" ::
 // each difference is exact in fp32 and the residual stays below 2^-24 |z| (8 significant
 // bits per term).
 template <int K>
-__device__ void write_zsplit(const EstZParams& p, const float* zr, int64_t row0) {
+__device__ void write_zsplit_rows(const float* zr, int mk, int64_t row0, int64_t n_ctx, __nv_bfloat16* zsplit,
+                                  int nthreads) {
   static_assert(3 * K <= 64 && K % 2 == 0, "three terms of k values fill at most 64 elements");
-  for (int it = threadIdx.x; it < 256; it += kZThreads) {
+  for (int it = threadIdx.x; it < 256; it += nthreads) {
     const int rr = it >> 1, pj = it & 1;
     const int64_t row = row0 + rr;
-    if (row >= p.n_ctx) continue;
-    const float* z = zr + rr * (p.mk + 1) + pj * K;
+    if (row >= n_ctx) continue;
+    const float* z = zr + rr * (mk + 1) + pj * K;
     uint32_t w[32];  // 64 bf16, element part * K + c
 #pragma unroll
     for (int i = 0; i < 32; ++i) w[i] = 0u;
@@ -91,9 +92,57 @@ __device__ void write_zsplit(const EstZParams& p, const float* zr, int64_t row0)
       w[(K + c) / 2] = *reinterpret_cast<const uint32_t*>(&t2);
       w[(2 * K + c) / 2] = *reinterpret_cast<const uint32_t*>(&t3);
     }
-    uint4* dst = reinterpret_cast<uint4*>(p.zsplit + row * 128 + pj * 64);
+    uint4* dst = reinterpret_cast<uint4*>(zsplit + row * 128 + pj * 64);
 #pragma unroll
     for (int q = 0; q < 8; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
+__device__ void write_zsplit_k(int k, const float* zr, int mk, int64_t row0, int64_t n_ctx, __nv_bfloat16* zsplit,
+                               int nthreads) {
+  switch (k) {
+    case 4: write_zsplit_rows<4>(zr, mk, row0, n_ctx, zsplit, nthreads); break;
+    case 8: write_zsplit_rows<8>(zr, mk, row0, n_ctx, zsplit, nthreads); break;
+    case 16: write_zsplit_rows<16>(zr, mk, row0, n_ctx, zsplit, nthreads); break;
+  }
+}
+
+// The Gram share of one 128-row tile, G[a][b] = sum over its rows of z[a] z[b] in fp64 (products
+// of fp32 values are exact), from the tile's rows staged as fp64 [128][mk] in shared memory (rows
+// past the context hold zeros). Work items (row group, 4 x 4 block of G): each sums its rows in
+// order into 16 registers; the row-group partials (gp, shared memory [RG][mk][mk]) are then added
+// in row-group order into out [mk][mk]. Block-wide (every thread calls it).
+__device__ void gram_tile(const double* zs, int mk, double* gp, double* out, int nthreads) {
+  const int nb4 = mk / 4, blocks = nb4 * nb4;
+  const int RG = gram_row_groups(mk), rows_per = 128 / RG;
+  for (int it = threadIdx.x; it < blocks * RG; it += nthreads) {
+    const int rg = it / blocks, blk = it - rg * blocks;
+    const int ba = blk / nb4, bb = blk - ba * nb4;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int t = rg * rows_per; t < (rg + 1) * rows_per; ++t) {
+      const double2* ra = reinterpret_cast<const double2*>(zs + t * mk + ba * 4);
+      const double2* rb = reinterpret_cast<const double2*>(zs + t * mk + bb * 4);
+      const double2 a01 = ra[0], a23 = ra[1], b01 = rb[0], b23 = rb[1];
+      const double va[4] = {a01.x, a01.y, a23.x, a23.y}, vb[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(va[i], vb[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) gp[((int64_t)rg * mk + ba * 4 + i) * mk + bb * 4 + j] = acc[i][j];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < mk * mk; e += nthreads) {
+    double sum = gp[e];
+    for (int rg = 1; rg < RG; ++rg) sum += gp[(int64_t)rg * mk * mk + e];
+    out[e] = sum;
   }
 }
 
@@ -355,55 +404,47 @@ __global__ void __launch_bounds__(kZThreads, 1) est_z_kernel(const __grid_consta
     // Z rows of the two projections (gate, up) as three bf16 terms each, for the SwiGLU
     // criterion's tensor-core products: row t holds 128 bf16, [proj * 64 + part * k + c] =
     // part `part` of Z[t][proj * k + c], zero past 3k. Work items (row, 8 outputs).
-    switch (p.k) {
-      case 4: write_zsplit<4>(p, reinterpret_cast<const float*>(sa), row0); break;
-      case 8: write_zsplit<8>(p, reinterpret_cast<const float*>(sa), row0); break;
-      case 16: write_zsplit<16>(p, reinterpret_cast<const float*>(sa), row0); break;
-    }
+    write_zsplit_k(p.k, reinterpret_cast<const float*>(sa), p.mk, row0, p.n_ctx, p.zsplit, kZThreads);
   }
   if (last && p.gram_part != nullptr) {
-    // The tile's Gram share G[a][b] = sum over its rows of z[a] z[b] in fp64 (products of
-    // fp32 values are exact). Work items (row group, 4 x 4 block of G): each sums its rows
-    // in order into 16 registers, eight 16-byte shared-memory loads per row; the row-group
-    // partials are then added in row-group order. Rows past n_ctx hold zeros.
     const double* zs = reinterpret_cast<const double*>(sa);  // [128][mk]
-    const int mk = p.mk, nb4 = mk / 4, blocks = nb4 * nb4;
-    const int RG = gram_row_groups(mk), rows_per = 128 / RG;
-    double* gp = reinterpret_cast<double*>(sa) + 128 * mk;    // [RG][mk][mk]
-    for (int it = threadIdx.x; it < blocks * RG; it += kZThreads) {
-      const int rg = it / blocks, blk = it - rg * blocks;
-      const int ba = blk / nb4, bb = blk - ba * nb4;
-      double acc[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-      for (int t = rg * rows_per; t < (rg + 1) * rows_per; ++t) {
-        const double2* ra = reinterpret_cast<const double2*>(zs + t * mk + ba * 4);
-        const double2* rb = reinterpret_cast<const double2*>(zs + t * mk + bb * 4);
-        const double2 a01 = ra[0], a23 = ra[1], b01 = rb[0], b23 = rb[1];
-        const double va[4] = {a01.x, a01.y, a23.x, a23.y}, vb[4] = {b01.x, b01.y, b23.x, b23.y};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fma(va[i], vb[j], acc[i][j]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) gp[((int64_t)rg * mk + ba * 4 + i) * mk + bb * 4 + j] = acc[i][j];
-    }
-    __syncthreads();
-    double* g = p.gram_part + (int64_t)blockIdx.y * mk * mk;
-    for (int e = threadIdx.x; e < mk * mk; e += kZThreads) {
-      double sum = gp[e];
-      for (int rg = 1; rg < RG; ++rg) sum += gp[(int64_t)rg * mk * mk + e];
-      g[e] = sum;
-    }
+    gram_tile(zs, p.mk, reinterpret_cast<double*>(sa) + 128 * p.mk, p.gram_part + (int64_t)blockIdx.y * p.mk * p.mk,
+              kZThreads);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem_base, 64);
+}
+
+// Z computed outside this file (the estimator's stage 1 as extra columns of the LoRA x A^T
+// launch: fp32 [n_ctx][ld_z]) -> the per-tile Gram shares of the linear criteria or the
+// three-term bf16 split of the SwiGLU criterion, exactly as est_z_kernel's tail forms them from its
+// own Z. One CTA per 128-row tile; rows past n_ctx count as zeros.
+__global__ void __launch_bounds__(kZThreads) z_finish_kernel(const float* __restrict__ z, int64_t ld_z, int64_t n_ctx,
+                                                             int mk, int k, double* __restrict__ gram_part,
+                                                             __nv_bfloat16* __restrict__ zsplit) {
+  extern __shared__ __align__(16) uint8_t zsm[];
+  pdl_wait();
+  const int64_t row0 = (int64_t)blockIdx.x * 128;
+  if (gram_part) {
+    double* zs = reinterpret_cast<double*>(zsm);  // [128][mk], then the row-group partials
+    for (int e = threadIdx.x; e < 128 * mk; e += kZThreads) {
+      const int rr = e / mk, c = e - rr * mk;
+      const int64_t row = row0 + rr;
+      zs[e] = row < n_ctx ? (double)z[row * ld_z + c] : 0.0;
+    }
+    __syncthreads();
+    gram_tile(zs, mk, zs + 128 * mk, gram_part + (int64_t)blockIdx.x * mk * mk, kZThreads);
+  } else {
+    float* zr = reinterpret_cast<float*>(zsm);  // [128][mk + 1]
+    for (int e = threadIdx.x; e < 128 * mk; e += kZThreads) {
+      const int rr = e / mk, c = e - rr * mk;
+      const int64_t row = row0 + rr;
+      zr[rr * (mk + 1) + c] = row < n_ctx ? z[row * ld_z + c] : 0.f;
+    }
+    __syncthreads();
+    write_zsplit_k(k, zr, mk, row0, n_ctx, zsplit, kZThreads);
+  }
 }
 
 // ---- linear criteria from the Gram matrix
@@ -850,6 +891,28 @@ int est_scores(const double* gram_part, int n_parts, int mk, int k, int wb_fp32,
   else
     launch_kernel(est_scores_kernel<16>, grid, 256, smem, s, P);
   if (launch_failed("sl_estimator")) return 5;
+  note_launch();
+  return 0;
+}
+
+int z_finish(const float* z, int64_t ld_z, int64_t n_ctx, int mk, int k, double* gram_part, void* zsplit,
+             cudaStream_t s) {
+  if (n_ctx <= 0 || mk <= 0 || mk > 64 || mk % 4 || ld_z < mk || (!gram_part && !zsplit)) return 1;
+  if (!gram_part && (k != 4 && k != 8 && k != 16)) return 1;
+  const int64_t tiles = (n_ctx + 127) / 128;
+  if (tiles > 2147483647LL) return 1;
+  const size_t smem = gram_part ? (size_t)128 * mk * 8 + (size_t)gram_row_groups(mk) * mk * mk * 8
+                                : (size_t)128 * (mk + 1) * 4;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(z_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 64 * 8 + 64 * 64 * 8) !=
+        cudaSuccess)
+      return 5;
+    attr = true;
+  }
+  launch_kernel(z_finish_kernel, (unsigned)tiles, kZThreads, smem, s, z, ld_z, n_ctx, mk, k, gram_part,
+                static_cast<__nv_bfloat16*>(zsplit));
+  if (launch_failed("sl_est_tc")) return 5;
   note_launch();
   return 0;
 }

@@ -332,11 +332,16 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
       case EPI_XA: {
         float* o0 = reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + n0 + c0;
         __nv_bfloat16* o1 = reinterpret_cast<__nv_bfloat16*>(pr.out1) + orow * pr.ld1 + n0 + c0;
+        const int zc = pr.z_col0 > 0 ? pr.z_col0 - (n0 + c0) : 1 << 30;  // first Z column of the chunk
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i >= n) break;
-          o0[i] = pr.a0 * v[i];
-          o1[i] = __float2bfloat16_rn(pr.a1 * v[i]);
+          if (i >= zc) {
+            if (orow < pr.z_rows) reinterpret_cast<float*>(pr.out2)[orow * pr.ld2 + (i - zc)] = pr.a0 * v[i];
+          } else {
+            o0[i] = pr.a0 * v[i];
+            o1[i] = __float2bfloat16_rn(pr.a1 * v[i]);
+          }
         }
         break;
       }
@@ -399,9 +404,9 @@ __device__ void epilogue_partial(const Prob& pr, int m0, int ks, int r, uint32_t
 }
 
 struct RedProb {
-  int32_t M, N, ksplit, epi, beta, out_row0, col_split, pad_;
+  int32_t M, N, ksplit, epi, beta, out_row0, col_split, z_col0, z_rows, pad_;
   int* err;
-  int64_t ld0, ld1;
+  int64_t ld0, ld1, ld2;
   void* out0;
   void* out1;
   void* out2;
@@ -440,8 +445,12 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
     if (pr.row_map && !index_ok(orow, pr.M, pr.err, DEV_BAD_ROW_MAP)) continue;
     if (pr.col_map && !index_ok(ocol, pr.N, pr.err, DEV_BAD_COL_MAP)) continue;
     if (pr.epi == EPI_XA) {
-      reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + ocol] = pr.a0 * acc;
-      reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + ocol] = __float2bfloat16_rn(pr.a1 * acc);
+      if (pr.z_col0 > 0 && ocol >= pr.z_col0) {
+        if (orow < pr.z_rows) reinterpret_cast<float*>(pr.out2)[orow * pr.ld2 + (ocol - pr.z_col0)] = pr.a0 * acc;
+      } else {
+        reinterpret_cast<float*>(pr.out0)[orow * pr.ld0 + ocol] = pr.a0 * acc;
+        reinterpret_cast<__nv_bfloat16*>(pr.out1)[orow * pr.ld1 + ocol] = __float2bfloat16_rn(pr.a1 * acc);
+      }
     } else {
       float* d = pr.epi == EPI_F32_T ? f32t_out(pr, ocol) + orow : reinterpret_cast<float*>(pr.out0) + orow * pr.ld0 + ocol;
       *d = pr.a0 * acc + (pr.beta ? *d : 0.f);
@@ -1277,6 +1286,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
     q.col_split = pr.col_split; q.out2 = pr.out2;
     q.ld0 = pr.ld0; q.ld1 = pr.ld1; q.out0 = pr.out0; q.out1 = pr.out1; q.row_map = pr.row_map;
     q.col_map = pr.col_map; q.part = pr.part; q.a0 = pr.a0; q.a1 = pr.a1; q.err = err;
+    q.z_col0 = pr.z_col0; q.z_rows = pr.z_rows; q.ld2 = pr.ld2;
     maxmn = std::max<int64_t>(maxmn, (int64_t)pr.M * pr.N);
   }
   if (nred) {

@@ -36,7 +36,7 @@ constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 
 enum Epi : int32_t {
   EPI_BF16 = 0,     // out0 bf16 = a0 * acc
   EPI_F32 = 1,      // out0 fp32 = a0 * acc (+ out0 when beta)
-  EPI_XA = 2,       // out0 fp32 = a0 * acc, out1 bf16 = a1 * acc
+  EPI_XA = 2,       // out0 fp32 = a0 * acc, out1 bf16 = a1 * acc (columns < z_col0 when set; out2 fp32 past it)
   EPI_SWIGLU = 3,   // paired tile: g = acc[:, 0:128], u = acc[:, 128:256]; out0 g, out1 u, out2 h = SiLU(g) u
   EPI_DSWIGLU = 4,  // dh = acc; reads g (aux0), u (aux1); out0 dg = dh u SiLU'(g), out1 du = dh SiLU(g)
   EPI_F32_T = 5,    // out0[col, row] fp32 = a0 * acc (+ old when beta): transposed store
@@ -75,6 +75,8 @@ struct Prob {
   int32_t col_split;    // EPI_F32_T: output columns [j * col_split, (j + 1) * col_split) go to
                         // out_j (j < 3), column c - j * col_split; 0 = all columns to out0
   int32_t out_row0;     // first output row
+  int32_t z_col0;       // EPI_XA: columns >= z_col0 (> 0) go to out2 (fp32, ld ld2, column c - z_col0),
+  int32_t z_rows;       //   only for output rows < z_rows; 0: every column goes to out0 / out1
   int8_t omap[4];       // tensor maps (32 x 32 boxes) of out0..out2 (SwiGLU backward: dg, du, g, u)
                         // over rows [out_row0, out_row0 + M), for the epilogue's bulk tensor copies;
                         // -1: per-thread loads and stores

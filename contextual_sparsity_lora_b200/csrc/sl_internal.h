@@ -149,6 +149,11 @@ int est_z_tc(const void* x, int64_t n_ctx, int64_t d_in, int64_t ldx, int n_proj
 // written by est_z_tc) and the bf16 W_B of gate and up [k, F]; scores[F].
 int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, const void* wb_u, int64_t F,
                   float* scores, double* sumsq, int* err, cudaStream_t s);
+// Z (fp32 [n_ctx][ld_z], computed elsewhere) -> per-128-row-tile fp64 Gram shares
+// (gram_part [tiles][mk][mk]) or the three-term bf16 split for est_swiglu_tc (zsplit
+// [n_ctx][128], two projections of k columns each). One launch.
+int z_finish(const float* z, int64_t ld_z, int64_t n_ctx, int mk, int k, double* gram_part, void* zsplit,
+             cudaStream_t s);
 // out[mk][mk] = sum of n_parts Gram matrices in order; scores = sqrt(sumsq).
 int gram_sum(const double* parts, int n_parts, int mk, double* out, cudaStream_t s);
 int sqrt_scores(const double* sumsq, int64_t n, float* scores, cudaStream_t s);

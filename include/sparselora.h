@@ -301,6 +301,33 @@ SL_API sl_status sl_lora_fwd_bwd(sl_lora_mode mode, int32_t n_ad, const sl_linea
                           int32_t out_layout, const sl_channels* out_ch, float* const* dya, void* const* dya_s,
                           float* const* dA, float* const* dB, sl_workspace* ws, sl_stream stream);
 
+/* a1 fused into a6's forward: the estimator's stage 1 and the adapters' x A^T from one pass over
+ * x ([WT] "SVD Sparsity Estimator", Algorithm 1: Z = X_ctx W_A on the context tokens; the dense
+ * LoRA branch's x A^T reads the same rows). The stacked, transposed factors of the estimated
+ * projections that share x become extra rows of the skinny product's B operand, so x streams from
+ * memory once for both:
+ *   xa, xa_s exactly as sl_lora_fwd_bwd(SL_LORA_FWD) for the n_ad (<= 3) adapters sharing x
+ *   (natural layout, equal scales);
+ *   z: fp32 [n_ctx, ld_z] (ld_z >= n_proj k) = X_ctx [W_A^(1) ... W_A^(n_proj)] for the context rows
+ *   [0, n_ctx) of x (rows past n_ctx are not written).
+ *   w_a_t: bf16 [n_proj k, d_in] (ld ld_wat): row j k + c = column c of W_A^(j) (sl_prepare_weight
+ *   of each W_A [d_in, k] gives its k rows).
+ * Requires k <= 16, n_proj k <= 64 and a multiple of 4, sum of ranks + n_proj k <= 256. Sums over
+ * d_in run in a fixed order (z is run-to-run identical). Errors as sl_lora_fwd_bwd. */
+SL_API sl_status sl_lora_fwd_estimate(int32_t n_ad, const sl_linear* lin, const void* x, int64_t ldx, int64_t n_tok,
+                                      int64_t n_ctx, float* xa, void* xa_s, int64_t ld_xa, int32_t n_proj,
+                                      int32_t k, const void* w_a_t, int64_t ld_wat, float* z, int64_t ld_z,
+                                      sl_workspace* ws, sl_stream stream);
+
+/* a2 from the Z of sl_lora_fwd_estimate: the scores sl_svd_estimate gives for the same context rows
+ * and factors (same criteria, arguments and results; z: fp32 [n_ctx, ld_z], n_proj k columns).
+ * The linear criteria go through the fp64 Gram matrix of Z, the SwiGLU criterion through a
+ * three-term bf16 expansion of Z on the tensor cores (k in {4, 8, 16}). */
+SL_API sl_status sl_svd_scores_from_z(sl_criterion crit, int32_t n_proj, const void* const* w_b, const int64_t* d_out,
+                                      int32_t k, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                      const float* z, int64_t ld_z, int64_t n_ctx, float* scores, float* scores_v,
+                                      sl_workspace* ws, sl_stream stream);
+
 /* a4: sparse frozen branch forward plus the fused LoRA add ([WT] Algorithm 1, Figure 8;
  * "Preliminary: what channel sparsity means structurally").
  * Context rows go through the weight sliced to the kept channels; output rows through

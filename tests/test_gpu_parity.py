@@ -365,3 +365,64 @@ def test_swiglu_epilogues_elementwise_on_negative_gates(tile_rows):
         # 2e-2 relative, plus a floor for the fp32 accumulation error of dh where dh itself is ~0
         bad = live & (np.abs(got - want) > 2e-2 * np.abs(want) + 1e-4 * np.abs(fac) * rms)
         assert not bad.any(), f"{name}: {int(bad.sum())} elements outside tolerance"
+
+
+# ------------------------------------------------- stage 1 inside the LoRA forward, criteria from Z
+
+@pytest.mark.parametrize("T,C,D,crit,k,r", [(424, 300, 512, "qk", 8, 32), (424, 300, 512, "swiglu", 8, 32),
+                                            (300, 200, 64, "swiglu", 4, 16), (200, 130, 256, "qk", 16, 8),
+                                            (256, 0, 256, "swiglu", 8, 16)])
+def test_lora_fwd_estimate_and_scores_from_z(T, C, D, crit, k, r):
+    """sl_lora_fwd_estimate: x A^T of the adapters and Z = X_ctx W_A from one skinny product (split-K
+    and, at d_in = 64, the unsplit epilogue); sl_svd_scores_from_z: the criteria from that Z,
+    against the oracle's estimator on the same context rows (QK with GQA, SwiGLU)."""
+    gen = inputs.generator(81 + k)
+    hq, hkv, hd = 4, 2, 32
+    x = inputs.activations_student_t(T, D, 4, 0.01, 30.0, gen)
+    if crit == "qk":
+        outs = (hq * hd, hkv * hd, hkv * hd)
+    else:
+        outs = (384, 384)
+    fac = [inputs.spectral_weight(n, D, 0.5, k, gen, "cpu", torch.float64, torch.bfloat16) for n in outs]
+    ads = [inputs.lora_pair(n, D, r, 0.02, gen) for n in outs]
+    mk = len(outs) * k
+    xg = cu(x)
+    dev_ab = [(cu(a), cu(b)) for a, b in ads]
+    lins = [B.linear_desc(cu(torch.zeros(n, D)), a, b, 2.0, B.SL_SLICE_OUT) for (a, b), n in zip(dev_ab, outs)]
+    WA = [cu(f.W_A) for f in fac]
+    WB = [cu(f.W_B) for f in fac]
+    WAt = torch.empty(mk, D, device=DEV, dtype=torch.bfloat16)
+    for j, w in enumerate(WA):
+        B.sl_prepare_weight(w, WAt[j * k:(j + 1) * k])
+    R = r * len(outs)
+    xa = torch.full((T, R), float("nan"), device=DEV)
+    xa_s = torch.full((T, R), float("nan"), device=DEV, dtype=torch.bfloat16)
+    z = torch.full((max(C, 1), mk), float("nan"), device=DEV)
+    ws = B.Workspace()
+    B.sl_lora_fwd_estimate(ws, lins, xg, C, xa_s, xa, len(outs), k, WAt, z)
+    torch.cuda.synchronize()
+    X = oracle.f64(x)
+    want_xa = X @ np.concatenate([oracle.f64(a) for a, _ in ads], 0).T
+    assert rel_fro(xa, want_xa) < FP32_TOL
+    assert rel_fro(xa_s, 2.0 * want_xa) < BF16_TOL
+    if C == 0:
+        assert torch.isnan(z).all()  # no context rows: Z untouched
+        return
+    want_z = X[:C] @ np.concatenate([oracle.f64(f.W_A) for f in fac], 1)
+    assert rel_fro(z, want_z) < FP32_TOL
+    ctx = np.arange(T) < C
+    if crit == "qk":
+        s_qk = torch.empty(hkv * hd, device=DEV)
+        s_v = torch.empty(hkv * hd, device=DEV)
+        B.sl_svd_scores_from_z(ws, B.SL_CRIT_QK, WB, k, z, C, s_qk, scores_v=s_v, n_q_heads=hq, n_kv_heads=hkv,
+                               head_dim=hd)
+        sel = oracle.attn_select(x, ctx, (fac[0].W_A, fac[0].W_B), (fac[1].W_A, fac[1].W_B), (fac[2].W_A, fac[2].W_B),
+                                 hq, hkv, hd, 0.5)
+        assert rel_fro(s_qk, sel["s_qk"]) < FP32_TOL
+        assert rel_fro(s_v, sel["s_v"]) < FP32_TOL
+    else:
+        sc = torch.empty(outs[0], device=DEV)
+        B.sl_svd_scores_from_z(ws, B.SL_CRIT_SWIGLU_L2, WB, k, z, C, sc)
+        s_w, _ = oracle.ffn_select(x, ctx, (fac[0].W_A, fac[0].W_B), (fac[1].W_A, fac[1].W_B), 0.5)
+        assert rel_fro(sc, s_w) < FP32_TOL
+    assert ws.read_device_flag() == 0
