@@ -110,13 +110,34 @@ __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* v
   }
 }
 
+// 32 bf16 of row `lane` of a 64-byte-swizzled 32 x 32 box (as loaded by a bulk tensor copy).
+__device__ __forceinline__ void load_box_row(const uint8_t* box, int lane, float* v) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(box + lane * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w = s4[i ^ ((lane >> 1) & 3)];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __bfloat1622float2(h[j]);
+      v[8 * i + 2 * j] = f.x;
+      v[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+}
+
 // Bulk-store path of the bf16 epilogues: the warp's 32 rows x 32 columns of one output go
-// through one of the warp's two 2 KB shared-memory boxes (row-major bf16, lane = row) and
-// leave with one bulk tensor store issued by lane 0, so the warp moves on while the copy
-// drains and every write is a whole line. Rows and columns outside the problem are clipped
-// by the tensor map (it covers exactly the problem's M x N block). Lane 0 waits, before a
-// box is rewritten, until at most one of its bulk groups (the other box) is still reading.
+// through one of the warp's two 2 KB shared-memory boxes (lane = row of 64 bytes) and leave
+// with one bulk tensor store issued by lane 0, so the warp moves on while the copy drains and
+// every write is a whole line. The boxes use the tensor map's 64-byte swizzle: 16-byte chunk i of
+// row r sits at chunk position i ^ ((r / 2) % 4) (the boxes are 512-byte aligned), so one 16-byte
+// store of the warp touches every bank at most four times (four wavefronts for 512 bytes) instead
+// of sixteen with rows of 64 bytes side by side. Rows and columns outside the problem are
+// clipped by the tensor map (it covers exactly the problem's M x N block). Lane 0 waits, before
+// a box is rewritten, until at most one of its bulk groups (the other box) is still reading.
 // Warp-collective; the caller skips warps whose rows all lie outside the problem.
+__device__ __forceinline__ int swz64(int lane, int i) { return i ^ ((lane >> 1) & 3); }
+
 __device__ __forceinline__ void bulk_store_chunk(const CUtensorMap* map, uint8_t* bufs, int& sb, const float* v,
                                                  int col, int row0) {
   const int lane = threadIdx.x & 31;
@@ -126,8 +147,9 @@ __device__ __forceinline__ void bulk_store_chunk(const CUtensorMap* map, uint8_t
   uint4* d = reinterpret_cast<uint4*>(buf + lane * 64);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    d[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+    d[swz64(lane, i)] =
+        make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                   pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -210,14 +232,15 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
   auto chunk = [&](uint32_t (&raw)[32], int c0) {
     const int n = min(32, ncols - c0);
     if (pr.epi == EPI_BF16 && pr.col_map) {
-      // Scatter through a 32 x 33 shared-memory transpose: each store instruction then
+      // Scatter through a 32 x 32 shared-memory transpose (element (r, c) at r * 32 + (c ^ r): the
+      // row writes and the column reads both hit 32 different banks): each store instruction then
       // writes 32 columns of one row (a few sectors) instead of one column of 32 rows.
       // (The transpose buffer is also the bulk-store boxes: let pending bulk reads finish.)
       const int lane = r & 31;
       if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(raw[i]) * pr.a0;
+      for (int i = 0; i < 32; ++i) stage[lane * 32 + (i ^ lane)] = __uint_as_float(raw[i]) * pr.a0;
       __syncwarp();
       bool cv = lane < n;
       const int64_t ocol = cv ? (int64_t)pr.col_map[n0 + c0 + lane] : 0;
@@ -229,7 +252,7 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
         if (cv && row2 < pr.M) {
           const int64_t o2 = pr.row_map ? (int64_t)pr.row_map[row2] : (int64_t)pr.out_row0 + row2;
           if (!pr.row_map || index_ok(o2, pr.M, aw.err, DEV_BAD_ROW_MAP))
-            out[o2 * pr.ld0 + ocol] = __float2bfloat16_rn(stage[rr * 33 + lane]);
+            out[o2 * pr.ld0 + ocol] = __float2bfloat16_rn(stage[rr * 32 + (lane ^ rr)]);
         }
       }
       __syncwarp();
@@ -260,8 +283,8 @@ __device__ void epilogue_tile(const Prob& pr, const CUtensorMap* maps, int m0, i
       if (!mbar_wait(aw.bar, aw.phase, aw.abort, aw.err, DEV_TIMEOUT_EPILOGUE)) return;
       aw.pending = false;
       aw.phase ^= 1;
-      load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(bufs) + lane * 32, g, 32, true);
-      load_bf16_row(reinterpret_cast<const __nv_bfloat16*>(bufs + 2048) + lane * 32, u, 32, true);
+      load_box_row(bufs, lane, g);
+      load_box_row(bufs + 2048, lane, u);
       __syncwarp();
       float dg[32];
 #pragma unroll
@@ -483,7 +506,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // kEpiWarps x [32][33]
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBlockBytes);  // kEpiWarps x 4 KB
   uint64_t* aux_bars = bars + 24;  // one per epilogue warp (bytes 192..255 of the barrier block)
 
   const int warp = threadIdx.x >> 5;
@@ -633,7 +656,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       if (pr.ksplit > 1)
         epilogue_partial(pr, ti.tm * kBM, ti.ks, r, tb, half);
       else
-        epilogue_tile(pr, p.maps, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * 32 * 33, half,
+        epilogue_tile(pr, p.maps, ti.tm * kBM, ti.tn * pr.tile_cols, r, tb, epi_stage + (warp - 2) * (kEpiWarpBytes / 4), half,
                       sbuf, aw);
       __syncwarp();
       tc_fence_before();
@@ -712,7 +735,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBlockBytes);
   uint64_t* aux_bars = bars + 24;  // one per epilogue warp (bytes 192..255 of the barrier block)
 
   const int warp = threadIdx.x >> 5;
@@ -863,7 +886,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int h = 0; h < MH; ++h)
         epilogue_tile(pr, p.maps, ti.tm * C::kTileM + 128 * MH * (int)rank + 128 * h, ti.tn * pr.tile_cols, r,
-                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * 32 * 33, half, sbuf, aw);
+                      tb + (uint32_t)(h * kBN), epi_stage + (warp - 2) * (kEpiWarpBytes / 4), half, sbuf, aw);
       __syncwarp();
       tc_fence_before();
       mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
@@ -941,8 +964,9 @@ int GemmBuilder::map(const void* ptr, int64_t rows, int64_t cols, int64_t ld, in
   return nmaps++;
 }
 
-// Tensor map of a bf16 output block [rows, cols] (ld elements) for 32 x 32 bulk stores;
-// -1 when it cannot be encoded (the epilogue then stores per thread).
+// Tensor map of a bf16 output block [rows, cols] (ld elements) for 32 x 32 bulk stores (64-byte
+// swizzle, matching the epilogue's box layout); -1 when it cannot be encoded (the epilogue then
+// stores per thread).
 int GemmBuilder::map_out(void* ptr, int64_t rows, int64_t cols, int64_t ld) {
   if (nmaps >= kMaxMaps || !ptr || rows <= 0 || cols <= 0 || ld < cols || (reinterpret_cast<uintptr_t>(ptr) & 15) ||
       (ld % 8))
@@ -954,7 +978,7 @@ int GemmBuilder::map_out(void* ptr, int64_t rows, int64_t cols, int64_t ld) {
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   if (enc(&params.maps[nmaps], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, gdim, gstride, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -1;
   specs[nmaps] = MapSpec{ptr, rows, cols, ld, 32};

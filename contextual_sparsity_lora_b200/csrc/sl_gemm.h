@@ -30,8 +30,13 @@ constexpr int kEpiWarps = 8;       // two epilogue warps per TMEM lane quarter, 
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
 constexpr int kStageABytes = kBM * kBK * 2;
 constexpr int kStageBBytes = kBN * kBK * 2;
-constexpr int kEpiStageBytes = kEpiWarps * 32 * 33 * 4;  // per-epilogue-warp transpose buffers
-constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + 256 + kEpiStageBytes;
+// Per epilogue warp 4 KB of shared memory, 512-byte aligned: two 2 KB boxes of the bulk tensor
+// stores (32 x 32 bf16, 64-byte swizzle) or one 32 x 32 fp32 transpose tile (XOR layout).
+constexpr int kEpiWarpBytes = 4096;
+constexpr int kEpiStageBytes = kEpiWarps * kEpiWarpBytes;
+constexpr int kBarBlockBytes = 512;  // mbarriers and flags; the epilogue region follows, 512-byte aligned
+constexpr int kGemmSmemBytes = kStages * (kStageABytes + kStageBBytes) + 1024 + kBarBlockBytes + kEpiStageBytes;
+static_assert(kGemmSmemBytes <= 232448, "GEMM shared memory exceeds the opt-in limit");
 
 enum Epi : int32_t {
   EPI_BF16 = 0,     // out0 bf16 = a0 * acc
