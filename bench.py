@@ -180,10 +180,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples), "source": self.source}
 
 
-def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None, cfgs=None):
+def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None, cfgs=None, kept_rows="compact"):
     """The two blocks of one layer (LLaMA3-8B unless `cfgs` = (attention config, FFN config))
     plus their per-step inputs (context-first rows). dp: a blocks.DataParallel over the ranks
-    (one index set per global batch), or None."""
+    (one index set per global batch), or None. kept_rows: where the sliced products read the
+    kept weight rows (blocks.KEPT_ROWS)."""
     from contextual_sparsity_lora_b200 import blocks
     ac, fc = cfgs if cfgs else (inputs.LLAMA3_8B_ATTN, inputs.LLAMA3_8B_FFN)
     da = inputs.make_attn_inputs(ac, seed_w, device=device)
@@ -192,9 +193,9 @@ def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None, cfgs=None):
     C = int(da["ctx_mask"].sum())
     attn = blocks.AttnProjBlock(da["q"], da["k"], da["v"], da["o"], da["lora_q"], da["lora_k"], da["lora_v"],
                                 da["lora_o"], ac.lora_scale, ac.k, ac.n_q_heads, ac.n_kv_heads, ac.head_dim,
-                                ac.n_tok, C, ratio, device, dense=dense, dp=dp)
+                                ac.n_tok, C, ratio, device, dense=dense, dp=dp, kept_rows=kept_rows)
     ffn = blocks.FFNBlock(df["gate"], df["up"], df["down"], df["lora_gate"], df["lora_up"], df["lora_down"],
-                          fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense, dp=dp)
+                          fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense, dp=dp, kept_rows=kept_rows)
     if seed_x != seed_w:  # per-rank batches
         dx = inputs.make_attn_inputs(ac, seed_x, device=device)
         for key in ("x", "x_o", "dq", "dk", "dv", "dy"):
@@ -350,14 +351,16 @@ def stage_times(attn, ffn, s, reps, device, hbm_gbs, step_ms):
                                                           blk.z))
         a2 = graph_us(lambda: B.sl_svd_scores_from_z(blk.ws, crit, WB, blk.k, blk.z, C, sc, **kw))
         sel = graph_us(blk.choose)
-        comp = graph_us(blk.compact)
+        # kept weight rows: read in place by the sliced products (no launch), or compacted per step
+        comp = graph_us(blk.compact) if blk.kept_rows == "compact" else 0.0
         standalone = graph_us(lambda: blk.estimate(x))
         a1 = max(fused_us - lora_us, 0.0)
         fused_bytes = T * D * 2 + (sum(l.r for l in lins) + n_proj * blk.k) * D * 2
         out[name] = {"a1_marginal_us": a1, "lora_x_at_us": lora_us, "lora_x_at_with_z_us": fused_us,
                      "fused_launch_bytes": fused_bytes, "fused_launch_GBs": fused_bytes / (fused_us * 1e3),
                      "fused_launch_frac_of_hbm": fused_bytes / (fused_us * 1e3) / hbm_gbs,
-                     "a2_criterion_us": a2, "a3_select_us": sel, "compact_weights_us": comp,
+                     "a2_criterion_us": a2, "a3_select_us": sel, "kept_rows": blk.kept_rows,
+                     "compact_weights_us": comp,
                      "standalone_estimator_us": standalone}
         total += a1 + a2 + sel
     # criterion ablation variants (not on the step's path): the Wanda-style FFN criterion
@@ -929,6 +932,17 @@ def main():
                               "effective_tflops": d_fl["total"] / (d_ms / args.steps / 1e3) / 1e12}
         line["speedup_vs_dense_lora"] = line["dense_lora"]["ms_per_step"] / ms_step
         del d_attn, d_ffn, d_graph
+        # the same sparse step with the kept weight rows read in place by the GEMM's row-gather
+        # copies instead of the per-step compacted copy: context, not the headline
+        c_attn, c_ffn, _, _, _, _ = make_layer(args.ratio, 0, 1000 + rank, device, dp=dp, kept_rows="gather")
+        for _ in range(3):
+            run_step(c_attn, c_ffn, step_in)
+        c_graph, _ = capture_or_eager(lambda: run_step(c_attn, c_ffn, step_in), world)
+        c_ms = time_steps(c_graph, args.steps, max(args.warmup, 3), world, device)
+        line["kept_rows_gathered"] = {"ms_per_step": c_ms / args.steps, "value": world * T / (c_ms / args.steps / 1e3),
+                                      "unit": UNIT, "step_ms_ratio_to_compacted": c_ms / args.steps / ms_step,
+                                      "what": "kept weight rows read in place by tile::gather4 operand copies"}
+        del c_attn, c_ffn, c_graph
     if world == 1 and not args.no_model:
         from contextual_sparsity_lora_b200.model import layerwise_keep, llama3_8b_math10k_keep
         line["model_32_layers"] = model_measure(da, df, perm, C, ac, fc, device, layerwise_keep())

@@ -415,7 +415,8 @@ def sl_attention_bwd(ws: Workspace, q, k, v, o, d_o, lse, n_seq, n_q_heads, n_kv
 
 
 def sl_set_pair_tile_rows(rows: int):
-    """Tile height of the CTA-pair GEMM for later launches: 256, 512, or 0 (chosen per launch)."""
+    """Tile height of the CTA-pair GEMM for later launches: 256, 512, 128 (no CTA pairs: the
+    one-CTA kernel), or 0 (chosen per launch)."""
     _check("sl_set_pair_tile_rows", lib().sl_set_pair_tile_rows(int(rows)))
 
 

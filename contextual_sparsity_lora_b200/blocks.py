@@ -12,6 +12,12 @@ import torch
 from . import binding as B
 
 
+# Where the sliced products find the kept weight rows: in a compacted copy made once per step
+# ("compact", the default: the tiled operand loads of the copy outrun the row-gather copies), or
+# in place through sigma ("gather": tile::gather4 copies of four 128-byte rows each).
+KEPT_ROWS = ("compact", "gather")
+
+
 def _empty(shape, dtype, device):
     return torch.empty(*shape, dtype=dtype, device=device)
 
@@ -93,12 +99,19 @@ class FFNBlock:
     CRITERIA = ("svd", "wanda", "random")
 
     def __init__(self, gate, up, down, lora_gate, lora_up, lora_down, lora_scale, k, n_tok, n_ctx, ratio,
-                 device="cuda", dense=False, dp=None, criterion="svd", seed=0):
+                 device="cuda", dense=False, dp=None, criterion="svd", seed=0, kept_rows="compact"):
         """criterion: "svd" (SwiGLU L2 of the SVD estimate, the method's criterion), or the
         criterion ablation's alternatives "wanda" (Wanda-style channel scores of the frozen
-        gate/up weights) and "random" (uniform scores from a generator seeded with `seed`)."""
+        gate/up weights) and "random" (uniform scores from a generator seeded with `seed`).
+        kept_rows: "compact" (a compacted copy of the kept rows, rebuilt once per step and
+        shared by the forward and backward products; the faster form on B200) or "gather" (the
+        sliced products read the kept weight rows in place, through sigma, with the GEMM's
+        row-gather copies)."""
         if criterion not in self.CRITERIA:
             raise ValueError(f"criterion {criterion!r} not in {self.CRITERIA}")
+        if kept_rows not in KEPT_ROWS:
+            raise ValueError(f"kept_rows {kept_rows!r} not in {KEPT_ROWS}")
+        self.kept_rows = kept_rows
         if criterion != "svd" and dp is not None and dp.active:
             raise ValueError("the ablation criteria run on one rank")
         self.criterion = criterion
@@ -156,10 +169,13 @@ class FFNBlock:
             B.sl_prepare_weight(self.WAg, self.WAt[: self.k])
             B.sl_prepare_weight(self.WAu, self.WAt[self.k:])
             self.z = _empty((n_ctx, 2 * self.k), f32, device)
-        # kept rows of the sliced weights, rebuilt once per step and shared by the forward
-        # and backward calls (the weights themselves when nothing is dropped)
+        # kept rows of the sliced weights: read in place by the GEMM (None), or a compacted copy
+        # rebuilt once per step and shared by the forward and backward calls (the weights
+        # themselves when nothing is dropped)
         if self.dense:
             self.Wg_k, self.Wu_k, self.Wd_k = self.Wg, self.Wu, self.Wd_t
+        elif kept_rows == "gather":
+            self.Wg_k = self.Wu_k = self.Wd_k = None
         else:
             nk = self.n_keep
             self.Wg_k, self.Wu_k, self.Wd_k = (_empty((nk, D), bf, device) for _ in range(3))
@@ -208,9 +224,30 @@ class FFNBlock:
         B.sl_select_channels(self.scores, self.n_keep, self.sigma)
 
     def compact(self):
-        """The kept weight rows of gate, up (rows of W) and down (rows of W^T) for this step."""
+        """The kept weight rows of gate, up (rows of W) and down (rows of W^T) for this step
+        (nothing to do when the GEMM gathers them)."""
+        if self.Wg_k is None or self.dense:
+            return
         kept = self.sigma[: self.n_keep]
         B.sl_gather_rows_batch([self.Wg, self.Wu, self.Wd_t], [kept] * 3, [self.Wg_k, self.Wu_k, self.Wd_k])
+
+    def _compact_gu(self):
+        if self.Wg_k is not None:
+            kept = self.sigma[: self.n_keep]
+            B.sl_gather_rows_batch([self.Wg, self.Wu], [kept] * 2, [self.Wg_k, self.Wu_k])
+
+    def _compact_d(self):
+        """The down projection's kept rows, on the second stream when the block runs chains
+        concurrently (needed only by the down product); True when it forked."""
+        if self.Wd_k is None:
+            return False
+        kept = self.sigma[: self.n_keep]
+        if self.concurrent:
+            with self.side.fork():
+                B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+            return True
+        B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+        return False
 
     def select(self, x):
         """a1 + a2 + a3 on the context rows of x, then the kept weight rows."""
@@ -235,14 +272,8 @@ class FFNBlock:
             B.sl_svd_scores_from_z(self.ws, B.SL_CRIT_SWIGLU_L2, [self.WBg, self.WBu], self.k, self.z, C,
                                    self.scores)
             self.choose()
-            kept = self.sigma[: self.n_keep]
-            B.sl_gather_rows_batch([self.Wg, self.Wu], [kept] * 2, [self.Wg_k, self.Wu_k])
-            if self.concurrent:
-                with self.side.fork():
-                    B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
-                down_side = True
-            else:
-                B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+            self._compact_gu()
+            down_side = self._compact_d()
         elif not self.dense and (C > 0 or self.dp):
             if self.concurrent:  # x A^T of gate/up does not depend on the selection
                 with self.side.fork():
@@ -251,12 +282,9 @@ class FFNBlock:
                 lora_done = self.side.mark()
                 self.estimate(x)
                 self.choose()
-                kept = self.sigma[: self.n_keep]
-                B.sl_gather_rows_batch([self.Wg, self.Wu], [kept] * 2, [self.Wg_k, self.Wu_k])
-                with self.side.fork():  # down's kept rows are needed only by the down product
-                    B.sl_permute_rows(self.Wd_t, kept, self.Wd_k)
+                self._compact_gu()
+                down_side = self._compact_d()
                 torch.cuda.current_stream().wait_event(lora_done)
-                down_side = True
             else:
                 self.select(x)
                 B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [self.lin_g, self.lin_u], x, C, self.xa_s_gu,
@@ -309,12 +337,18 @@ class AttnProjBlock:
 
     def __init__(self, q, k, v, o, lora_q, lora_k, lora_v, lora_o, lora_scale, est_k, n_q_heads, n_kv_heads,
                  head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False, dp=None, qk_criterion="channel",
-                 vo_criterion="l2", seed=0):
+                 vo_criterion="l2", seed=0, kept_rows="compact"):
         """qk_criterion: "channel" (the method's QK norm per KV channel), or the criterion
         ablation's "head" (whole KV heads by the summed QK norm) and "random"; vo_criterion:
-        "l2" (the method's) or "random" (uniform scores from a generator seeded with `seed`)."""
+        "l2" (the method's) or "random" (uniform scores from a generator seeded with `seed`).
+        kept_rows: "compact" (a compacted copy per step, shared by forward and backward; the
+        faster form on B200) or "gather" (the sliced products read the kept weight rows in place
+        through sigma)."""
         if qk_criterion not in ("channel", "head", "random") or vo_criterion not in ("l2", "random"):
             raise ValueError(f"criteria {qk_criterion!r}, {vo_criterion!r}")
+        if kept_rows not in KEPT_ROWS:
+            raise ValueError(f"kept_rows {kept_rows!r} not in {KEPT_ROWS}")
+        self.kept_rows = kept_rows
         if (qk_criterion, vo_criterion) != ("channel", "l2") and dp is not None and dp.active:
             raise ValueError("the ablation criteria run on one rank")
         self.qk_criterion, self.vo_criterion = qk_criterion, vo_criterion
@@ -382,12 +416,15 @@ class AttnProjBlock:
                 B.sl_prepare_weight(self.WA[j], self.WAt[j * est_k:(j + 1) * est_k])
             self.z = _empty((n_ctx, 3 * est_k), f32, device)
         s = self.scale
-        # kept rows of the sliced weights (rows of W for q, k, v; rows of W^T for o), rebuilt
-        # once per step after the selection and shared by the forward and backward calls
+        # kept rows of the sliced weights (rows of W for q, k, v; rows of W^T for o): read in
+        # place by the GEMM (None), or a copy rebuilt once per step after the selection and
+        # shared by the forward and backward calls
         nq, nu = self.n_keep_qk * self.hpg, self.n_keep_qk
         nv, no = self.n_keep_vo, self.n_keep_vo * self.hpg
         if self.dense:
             self.W_k = {"q": self.Wq, "k": self.Wk, "v": self.Wv, "o": self.Wo_t}
+        elif kept_rows == "gather":
+            self.W_k = {n: None for n in "qkvo"}
         else:
             self.W_k = {"q": _empty((nq, D), bf, device), "k": _empty((nu, D), bf, device),
                         "v": _empty((nv, D), bf, device), "o": _empty((no, D), bf, device)}
@@ -471,7 +508,10 @@ class AttnProjBlock:
         self.lin, self.ch = (self._lin_dense, self._ch_dense) if self.dense else (self._lin_sparse, self._ch_sparse)
 
     def _kept_rows(self, names):
-        """The kept weight rows of the named projections (rows of W; for o, rows of W^T), one launch."""
+        """The kept weight rows of the named projections (rows of W; for o, rows of W^T), one
+        launch; nothing when the GEMM gathers them."""
+        if self.W_k[names[0]] is None or self.dense:
+            return
         src = {"q": (self.Wq, self.sig_q), "k": (self.Wk, self.sig_k), "v": (self.Wv, self.sig_v),
                "o": (self.Wo_t, self.sig_o)}
         B.sl_gather_rows_batch([src[n][0] for n in names], [src[n][1][: self.ch[n].n_keep] for n in names],

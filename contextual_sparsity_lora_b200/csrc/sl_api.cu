@@ -112,6 +112,13 @@ inline sl_status ws_check(sl_workspace* ws, size_t needed) {
 }
 
 inline int* err_word(sl_workspace* ws) { return static_cast<int*>(ws->ptr); }
+// The workspace header's zero row (64 bf16 zeros): the rows past the kept count of a gathered operand.
+inline const void* zero_row(sl_workspace* ws) { return static_cast<const char*>(ws->ptr) + kZeroRowOffsetBytes; }
+// Whether the GEMM engine can read the kept rows of a weight straight from it (tile::gather4
+// copies through sigma) instead of a compacted copy: the gathered rows' width (the K extent of a
+// K-major operand, the N extent of an MN-major one) is whole 64-column boxes and sigma is 16-byte
+// aligned.
+inline bool gather_ok(const sl_channels& c, int64_t row_width) { return row_width % 64 == 0 && al16(c.sigma); }
 
 inline sl_status from_builder(int rc) {
   switch (rc) {
@@ -760,7 +767,7 @@ sl_status sl_svd_scores_from_z(sl_criterion crit, int32_t n_proj, const void* co
   const int64_t tiles = (n_ctx + 127) / 128;
   const bool linear = crit != SL_CRIT_SWIGLU_L2;
   auto carve = [&](Carver& c, double** gp, uint16_t** zs) {
-    *gp = linear ? c.take<double>((size_t)tiles * mk * mk) : nullptr;
+    *gp = linear ? c.take<double>((size_t)(tiles + 1) * mk * mk) : nullptr;  // tile shares, then their sum
     *zs = linear ? nullptr : c.take<uint16_t>((size_t)n_ctx * 128);
   };
   double* gp;
@@ -773,16 +780,19 @@ sl_status sl_svd_scores_from_z(sl_criterion crit, int32_t n_proj, const void* co
   Carver c(ws->ptr);
   carve(c, &gp, &zs);
   cudaStream_t s = cs(stream);
-  if (int rc = z_finish(z, ld_z, n_ctx, mk, k, gp, zs, s)) return from_kernel(rc);
+  // linear criteria: the Gram matrix of the whole context is summed inside the same launch
+  double* gtot = linear ? gp + tiles * mk * mk : nullptr;
+  if (int rc = z_finish(z, ld_z, n_ctx, mk, k, gp, zs, err_word(ws) + kCounterOffsetInts, gtot, s))
+    return from_kernel(rc);
   int rc;
   if (!linear) {
     rc = est_swiglu_tc(zs, n_ctx, k, w_b[0], w_b[1], n_units, scores, nullptr, err_word(ws), s);
     return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
   }
   if (crit == SL_CRIT_L2)
-    rc = est_scores(gp, (int)tiles, mk, k, 0, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0, n_units, scores, s);
+    rc = est_scores(gtot, 1, mk, k, 0, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, w_b[0], 0, n_units, scores, s);
   else
-    rc = est_scores(gp, (int)tiles, mk, k, 0, w_b[0], w_b[1], 0, 1, n_q_heads, n_kv_heads, head_dim, scores,
+    rc = est_scores(gtot, 1, mk, k, 0, w_b[0], w_b[1], 0, 1, n_q_heads, n_kv_heads, head_dim, scores,
                     n_proj == 3 ? w_b[2] : nullptr, 2, n_proj == 3 ? d_out[2] : 0, n_proj == 3 ? scores_v : nullptr,
                     s);
   return from_kernel(rc);
@@ -811,9 +821,11 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   if (slice == SL_SLICE_OUT && epi == SL_EPI_NONE) {
     for (int i = 0; i < n_lin; ++i)
       if (!y[i] || ldy[i] < lin[i].d_out || ldy[i] % 8 || !al16(y[i])) return SL_ERR_ALIGNMENT;
+    bool gath[4];  // kept rows read by the GEMM through sigma, no compacted copy
+    for (int i = 0; i < n_lin; ++i) gath[i] = !lin[i].w_kept && gather_ok(ch[i], d_in);
     auto carve = [&](Carver& c, void** wc, void** bs) {
       for (int i = 0; i < n_lin; ++i) {
-        wc[i] = lin[i].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        wc[i] = lin[i].w_kept || gath[i] ? nullptr : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
         bs[i] = c.take<uint16_t>((size_t)lin[i].d_out * lin[i].r);
       }
     };
@@ -825,11 +837,11 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
     Carver c(ws->ptr);
     carve(c, wc, bs);
-    GatherBatch gat;  // kept weight rows (when not given) and sigma-ordered LoRA B, one launch
+    GatherBatch gat;  // sigma-ordered LoRA B (and kept weight rows that are neither given nor gathered), one launch
     for (int i = 0; i < n_lin; ++i) {
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
-      else
+      else if (!gath[i])
         gat.add(lin[i].w, d_in, lin[i].d_out, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
       gat.add(lin[i].lora_b, lin[i].r, lin[i].d_out, ch[i].sigma, lin[i].d_out, lin[i].r, bs[i], lin[i].r);
     }
@@ -842,10 +854,15 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       const int mxa = gb.map(static_cast<const uint16_t*>(xa_s) + koff, T, L.r, ld_xa, kBM);
       koff += L.r;
       if (C > 0) {
-        const int mwc = gb.map(wc[i], ch[i].n_keep, d_in, d_in, kBN);
         const int mbs = gb.map(bs[i], L.d_out, L.r, L.r, kBN);
         Prob* p = gb.add((int)C, (int)L.d_out, kBN, kBN);
-        gb.bsrc(gb.seg(p, mx, 0, 0, 0, 0, 0, (int)d_in, (int)ch[i].n_keep), mwc, 0, kBN, 0, kBN);
+        Seg* sg = gb.seg(p, mx, 0, 0, 0, 0, 0, (int)d_in, (int)ch[i].n_keep);
+        if (gath[i]) {
+          gb.bsrc(sg, gb.gmap(L.w, L.d_out, d_in, d_in), 0, kBN, 0, kBN);
+          gb.gather(sg, ch[i].sigma, ch[i].n_keep, L.d_out, d_in, zero_row(ws));
+        } else {
+          gb.bsrc(sg, gb.map(wc[i], ch[i].n_keep, d_in, d_in, kBN), 0, kBN, 0, kBN);
+        }
         gb.bsrc(gb.seg(p, mxa, 0, 0, 0, 0, 0, L.r, kBig), mbs, 0, kBN, 0, kBN);
         if (p) {
           p->epi = EPI_BF16;
@@ -878,9 +895,10 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     for (int i = 0; i < 3; ++i)
       if (!y[i] || ldy[i] < F || ldy[i] % 8 || !al16(y[i]) || ldy[i] != ldy[0]) return SL_ERR_ALIGNMENT;
     const int64_t nt = (F + 127) / 128;  // paired tiles: 128 channels each
+    const bool gath = !lin[0].w_kept && !lin[1].w_kept && gather_ok(ch[0], d_in);
     auto carve = [&](Carver& c, void** wc, void** pk) {
-      wc[0] = lin[0].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
-      wc[1] = lin[1].w_kept ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      wc[0] = lin[0].w_kept || gath ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
+      wc[1] = lin[1].w_kept || gath ? nullptr : c.take<uint16_t>((size_t)ch[0].n_keep * d_in);
       pk[0] = c.take<uint16_t>((size_t)nt * 256 * 64);  // sigma order
       pk[1] = c.take<uint16_t>((size_t)nt * 256 * 64);  // natural order
     };
@@ -897,7 +915,7 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     for (int i = 0; i < 2; ++i) {
       if (lin[i].w_kept)
         wc[i] = const_cast<void*>(lin[i].w_kept);
-      else
+      else if (!gath)
         gat.add(lin[i].w, d_in, lin[i].d_out, sig, ch[0].n_keep, d_in, wc[i], d_in);
     }
     // LoRA B operand of a paired tile t: rows 256 t + j = [B_gate[c_j] | 0], rows 256 t + 128 + j = [0 | B_up[c_j]]
@@ -912,11 +930,12 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     GemmBuilder gb;
     const int mx = gb.map(x, T, d_in, ldx, kBM);
     const int mxa = gb.map(xa_s, T, lin[0].r + lin[1].r, ld_xa, kBM);
-    auto add_prob = [&](int64_t M, int64_t row0, int mg, int mu, int mp, int n_limit) {
+    auto add_prob = [&](int64_t M, int64_t row0, int mg, int mu, int mp, int n_limit, bool gathered) {
       Prob* p = gb.add((int)M, (int)F, 128, kBN);
       Seg* sg = gb.seg(p, mx, 0, (int)row0, 0, 0, 0, (int)d_in, n_limit);
       gb.bsrc(sg, mg, 0, 128, 0, 128);
       gb.bsrc(sg, mu, 128, 128, 0, 128);
+      if (gathered) gb.gather(sg, sig, ch[0].n_keep, F, d_in, zero_row(ws));
       gb.bsrc(gb.seg(p, mxa, 0, (int)row0, 0, 0, 0, 64, kBig), mp, 0, kBN, 0, kBN);
       if (!p) return;
       p->epi = EPI_SWIGLU;
@@ -926,12 +945,17 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       p->ld0 = ldy[0];
       p->out_row0 = (int)row0;
     };
-    if (C > 0)
-      add_prob(C, 0, gb.map(wc[0], ch[0].n_keep, d_in, d_in, 128), gb.map(wc[1], ch[0].n_keep, d_in, d_in, 128),
-               gb.map(pk[0], nt * 256, 64, 64, kBN), (int)ch[0].n_keep);
+    if (C > 0) {
+      if (gath)
+        add_prob(C, 0, gb.gmap(lin[0].w, F, d_in, d_in), gb.gmap(lin[1].w, F, d_in, d_in),
+                 gb.map(pk[0], nt * 256, 64, 64, kBN), (int)ch[0].n_keep, true);
+      else
+        add_prob(C, 0, gb.map(wc[0], ch[0].n_keep, d_in, d_in, 128), gb.map(wc[1], ch[0].n_keep, d_in, d_in, 128),
+                 gb.map(pk[0], nt * 256, 64, 64, kBN), (int)ch[0].n_keep, false);
+    }
     if (O > 0)
       add_prob(O, C, gb.map(lin[0].w, F, d_in, d_in, 128), gb.map(lin[1].w, F, d_in, d_in, 128),
-               gb.map(pk[1], nt * 256, 64, 64, kBN), kBig);
+               gb.map(pk[1], nt * 256, 64, 64, kBN), kBig, false);
     return from_builder(gb.launch(err_word(ws), s));
   }
 
@@ -943,8 +967,9 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     const int64_t nk = ch[0].n_keep;
     const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
     const int64_t ldc = rup(nk, 8);
+    const bool gath = !L.w_kept && gather_ok(ch[0], L.d_out);
     auto carve = [&](Carver& c, void** wtc, void** xc) {
-      *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : c.take<uint16_t>((size_t)nk * L.d_out);
+      *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : gath ? nullptr : c.take<uint16_t>((size_t)nk * L.d_out);
       *xc = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * ldc) : nullptr;
     };
     void *wtc, *xc;
@@ -955,7 +980,7 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
     Carver c(ws->ptr);
     carve(c, &wtc, &xc);
-    if (!L.w_kept)
+    if (!L.w_kept && !gath)
       if (int rc = gather_rows_bf16(L.w_t, L.d_out, L.d_in, ch[0].sigma, nk, L.d_out, wtc, L.d_out, 0, err_word(ws), s))
         return from_kernel(rc);
     if (xc)
@@ -965,9 +990,14 @@ sl_status sl_sparse_linear_fwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     const int mb = gb.map(L.lora_b, L.d_out, L.r, L.r, kBN);
     if (C > 0) {
       const int ma = in_sig ? gb.map(x, C, nk, ldx, kBM) : gb.map(xc, C, nk, ldc, kBM);
-      const int mw = gb.map(wtc, nk, L.d_out, L.d_out, 64);
       Prob* p = gb.add((int)C, (int)L.d_out, kBN, kBN);
-      gb.bsrc(gb.seg(p, ma, 0, 0, 0, 1, 0, (int)nk, kBig), mw, 0, kBN, 0, kBN);
+      Seg* sg = gb.seg(p, ma, 0, 0, 0, 1, 0, (int)nk, kBig);
+      if (gath) {
+        gb.bsrc(sg, gb.gmap(L.w_t, L.d_in, L.d_out, L.d_out), 0, kBN, 0, kBN);
+        gb.gather(sg, ch[0].sigma, nk, L.d_in, L.d_out, zero_row(ws));
+      } else {
+        gb.bsrc(sg, gb.map(wtc, nk, L.d_out, L.d_out, 64), 0, kBN, 0, kBN);
+      }
       gb.bsrc(gb.seg(p, mxa, 0, 0, 0, 0, 0, L.r, kBig), mb, 0, kBN, 0, kBN);
       if (p) {
         p->epi = EPI_BF16;
@@ -1016,9 +1046,13 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     if (epi != SL_EPI_NONE) return SL_ERR_UNSUPPORTED;
     if (!dx || lddx < d_in || lddx % 8 || !al16(dx)) return SL_ERR_ALIGNMENT;
     const bool in_sig = in_layout == SL_LAYOUT_SIGMA;
+    bool gath[3];  // kept rows read by the GEMM through sigma, no compacted copy
+    for (int i = 0; i < n_lin; ++i) gath[i] = !lin[i].w_kept && gather_ok(ch[i], d_in);
     auto carve = [&](Carver& c, void** wc, void** dyc) {
       for (int i = 0; i < n_lin; ++i) {
-        wc[i] = lin[i].w_kept ? const_cast<void*>(lin[i].w_kept) : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
+        wc[i] = lin[i].w_kept ? const_cast<void*>(lin[i].w_kept)
+                : gath[i]     ? nullptr
+                              : c.take<uint16_t>((size_t)ch[i].n_keep * d_in);
         dyc[i] = (!in_sig && C > 0) ? c.take<uint16_t>((size_t)C * rup(ch[i].n_keep, 8)) : nullptr;
       }
     };
@@ -1032,7 +1066,8 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     carve(c, wc, dyc);
     GatherBatch gat;
     for (int i = 0; i < n_lin; ++i)
-      if (!lin[i].w_kept) gat.add(lin[i].w, d_in, lin[i].d_out, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
+      if (!lin[i].w_kept && !gath[i])
+        gat.add(lin[i].w, d_in, lin[i].d_out, ch[i].sigma, ch[i].n_keep, d_in, wc[i], d_in);
     if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
     for (int i = 0; i < n_lin; ++i) {
       if (dyc[i])
@@ -1050,8 +1085,13 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
       if (pc) {
         const int64_t nk = ch[i].n_keep;
         const int ma = dyc[i] ? gb.map(dyc[i], C, nk, rup(nk, 8), kBM) : gb.map(dy[i], C, nk, ld_dy[i], kBM);
-        const int mw = gb.map(wc[i], nk, d_in, d_in, 64);
-        gb.bsrc(gb.seg(pc, ma, 0, 0, 0, 1, 0, (int)nk, kBig), mw, 0, kBN, 0, kBN);
+        Seg* sg = gb.seg(pc, ma, 0, 0, 0, 1, 0, (int)nk, kBig);
+        if (gath[i]) {
+          gb.bsrc(sg, gb.gmap(L.w, L.d_out, d_in, d_in), 0, kBN, 0, kBN);
+          gb.gather(sg, ch[i].sigma, nk, L.d_out, d_in, zero_row(ws));
+        } else {
+          gb.bsrc(sg, gb.map(wc[i], nk, d_in, d_in, 64), 0, kBN, 0, kBN);
+        }
         gb.bsrc(gb.seg(pc, mya, 0, 0, 0, 1, 0, L.r, kBig), mam, 0, kBN, 0, kBN);
       }
       if (po) {
@@ -1086,8 +1126,9 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     if (!dx || lddx < d_in || lddx % 8 || !al16(dx)) return SL_ERR_ALIGNMENT;
   }
   const int64_t nk = ch[0].n_keep;
+  const bool gath = !L.w_kept && gather_ok(ch[0], L.d_out);
   auto carve = [&](Carver& c, void** wtc, void** at, void** ats) {
-    *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : c.take<uint16_t>((size_t)nk * L.d_out);
+    *wtc = L.w_kept ? const_cast<void*>(L.w_kept) : gath ? nullptr : c.take<uint16_t>((size_t)nk * L.d_out);
     *at = c.take<uint16_t>((size_t)d_in * L.r);
     *ats = c.take<uint16_t>((size_t)d_in * L.r);
   };
@@ -1101,8 +1142,8 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
   carve(c, &wtc, &at, &ats);
   if (int rc = transpose_bf16(L.lora_a, L.r, d_in, d_in, at, L.r, s)) return from_kernel(rc);
   {
-    GatherBatch gat;  // kept rows of W^T (when not given) and the permuted A^T, one launch
-    if (!L.w_kept) gat.add(L.w_t, L.d_out, L.d_in, ch[0].sigma, nk, L.d_out, wtc, L.d_out);
+    GatherBatch gat;  // the permuted A^T (and kept rows of W^T that are neither given nor gathered), one launch
+    if (!L.w_kept && !gath) gat.add(L.w_t, L.d_out, L.d_in, ch[0].sigma, nk, L.d_out, wtc, L.d_out);
     gat.add(at, L.r, d_in, ch[0].sigma, d_in, L.r, ats, L.r);
     if (int rc = gat.launch(err_word(ws), s)) return from_kernel(rc);
   }
@@ -1128,10 +1169,15 @@ sl_status sl_sparse_linear_bwd(int32_t n_lin, const sl_linear* lin, const sl_cha
     }
   };
   if (C > 0) {
-    const int mw = gb.map(wtc, nk, L.d_out, L.d_out, kBN);
     const int mat = gb.map(ats, d_in, L.r, L.r, kBN);
     Prob* p = gb.add((int)C, (int)d_in, kBN, kBN);
-    gb.bsrc(gb.seg(p, mdy, 0, 0, 0, 0, 0, (int)L.d_out, (int)nk), mw, 0, kBN, 0, kBN);
+    Seg* sg = gb.seg(p, mdy, 0, 0, 0, 0, 0, (int)L.d_out, (int)nk);
+    if (gath) {
+      gb.bsrc(sg, gb.gmap(L.w_t, L.d_in, L.d_out, L.d_out), 0, kBN, 0, kBN);
+      gb.gather(sg, ch[0].sigma, nk, L.d_in, L.d_out, zero_row(ws));
+    } else {
+      gb.bsrc(sg, gb.map(wtc, nk, L.d_out, L.d_out, kBN), 0, kBN, 0, kBN);
+    }
     gb.bsrc(gb.seg(p, mya, 0, 0, 0, 0, 0, L.r, kBig), mat, 0, kBN, 0, kBN);
     set_epi(p, 0, !swiglu && out_layout == SL_LAYOUT_NATURAL);
   }
@@ -1230,8 +1276,8 @@ sl_status sl_attention_bwd(const void* q, const void* k, const void* v, const vo
 }
 
 sl_status sl_set_pair_tile_rows(int32_t rows) {
-  if (rows != 0 && rows != 256 && rows != 512) return SL_ERR_INVALID_ARG;
-  set_forced_pair_mh(rows / 256);
+  if (rows != 0 && rows != 128 && rows != 256 && rows != 512) return SL_ERR_INVALID_ARG;
+  set_forced_pair_mh(rows == 128 ? -1 : rows / 256);
   return SL_OK;
 }
 

@@ -419,11 +419,15 @@ __global__ void __launch_bounds__(kZThreads, 1) est_z_kernel(const __grid_consta
 // Z computed outside this file (the estimator's stage 1 as extra columns of the LoRA x A^T
 // launch: fp32 [n_ctx][ld_z]) -> the per-tile Gram shares of the linear criteria or the
 // three-term bf16 split of the SwiGLU criterion, exactly as est_z_kernel's tail forms them from its
-// own Z. One CTA per 128-row tile; rows past n_ctx count as zeros.
+// own Z. One CTA per 128-row tile; rows past n_ctx count as zeros. With gram_total set, the last
+// CTA to finish (a ticket that it returns to zero) also adds the tile shares in tile order into
+// gram_total, the Gram matrix of the whole context.
 __global__ void __launch_bounds__(kZThreads) z_finish_kernel(const float* __restrict__ z, int64_t ld_z, int64_t n_ctx,
                                                              int mk, int k, double* __restrict__ gram_part,
-                                                             __nv_bfloat16* __restrict__ zsplit) {
+                                                             __nv_bfloat16* __restrict__ zsplit, int* ticket,
+                                                             double* __restrict__ gram_total) {
   extern __shared__ __align__(16) uint8_t zsm[];
+  __shared__ int s_last;
   pdl_wait();
   const int64_t row0 = (int64_t)blockIdx.x * 128;
   if (gram_part) {
@@ -435,6 +439,27 @@ __global__ void __launch_bounds__(kZThreads) z_finish_kernel(const float* __rest
     }
     __syncthreads();
     gram_tile(zs, mk, zs + 128 * mk, gram_part + (int64_t)blockIdx.x * mk * mk, kZThreads);
+    if (!gram_total) return;
+    __threadfence();  // this CTA's share is visible before its ticket
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int ne = mk * mk, n_parts = (int)gridDim.x;
+    for (int e = threadIdx.x; e < ne; e += kZThreads) {
+      double sum = 0.0;
+      for (int c0 = 0; c0 < n_parts; c0 += 8) {
+        double v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = c0 + u < n_parts ? __ldcg(gram_part + (int64_t)(c0 + u) * ne + e) : 0.0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (c0 + u < n_parts) sum += v[u];
+      }
+      gram_total[e] = sum;
+    }
+    if (threadIdx.x == 0) *ticket = 0;
   } else {
     float* zr = reinterpret_cast<float*>(zsm);  // [128][mk + 1]
     for (int e = threadIdx.x; e < 128 * mk; e += kZThreads) {
@@ -491,11 +516,29 @@ __device__ __forceinline__ double quad_form(const double* G, int mk, int k, cons
   return s > 0.0 ? s : 0.0;
 }
 
+constexpr int kScoreThreads = 128;
+
 template <int KMAX>
-__global__ void __launch_bounds__(256) est_scores_kernel(const __grid_constant__ ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads) est_scores_kernel(const __grid_constant__ ScoreParams p) {
   pdl_wait();
   extern __shared__ double gs[];  // [mk][mk], the Gram matrix of the whole context
   const int ne = p.mk * p.mk;
+  // The unit's W_B columns (the K column and the first four query heads' columns of a QK unit,
+  // or the channel's column) are requested first, so their latency overlaps the Gram sum's.
+  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool is_qk = u < p.n_qk, is_l2 = !is_qk && u < p.n_qk + p.n_l2;
+  float bk[KMAX], bq[4][KMAX];
+  int g = 0, d = 0;
+  if (is_qk) {
+    g = (int)(u / p.head_dim);
+    d = (int)(u % p.head_dim);
+    load_b<KMAX>(p.wb_k, p.wb_fp32, p.k, p.n_kv, u, bk);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (j < p.hpg) load_b<KMAX>(p.wb_q, p.wb_fp32, p.k, p.n_q, (int64_t)(g * p.hpg + j) * p.head_dim + d, bq[j]);
+  } else if (is_l2) {
+    load_b<KMAX>(p.wb_l2, p.wb_fp32, p.k, p.n_l2, u - p.n_qk, bk);
+  }
   // Sum of the per-tile matrices in tile order, eight loads in flight per step.
   for (int e = threadIdx.x; e < ne; e += blockDim.x) {
     double s = 0.0;
@@ -510,30 +553,24 @@ __global__ void __launch_bounds__(256) est_scores_kernel(const __grid_constant__
     gs[e] = s;
   }
   __syncthreads();
-  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (u >= p.n_qk + p.n_l2) return;
-  if (u < p.n_qk) {
-    const int g = (int)(u / p.head_dim), d = (int)(u % p.head_dim);
+  if (is_qk) {
     const double* Gq = gs + p.blk_q * p.k * p.mk + p.blk_q * p.k;
     const double* Gk = gs + p.blk_k * p.k * p.mk + p.blk_k * p.k;
-    float bk[KMAX], bn[KMAX];
-    load_b<KMAX>(p.wb_k, p.wb_fp32, p.k, p.n_kv, u, bk);
-    load_b<KMAX>(p.wb_q, p.wb_fp32, p.k, p.n_q, (int64_t)(g * p.hpg) * p.head_dim + d, bn);
-    double qs = 0.0;
-    for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h) {
-      float bc[KMAX];
+    double qs = 0.0;  // the group's query heads in ascending order
+    for (int h0 = 0; h0 < p.hpg; h0 += 4) {
+      if (h0 > 0) {
 #pragma unroll
-      for (int c = 0; c < KMAX; ++c) bc[c] = bn[c];
-      if (h + 1 < (g + 1) * p.hpg)  // the next head's column is in flight during this head's form
-        load_b<KMAX>(p.wb_q, p.wb_fp32, p.k, p.n_q, (int64_t)(h + 1) * p.head_dim + d, bn);
-      qs += sqrt(quad_form<KMAX>(Gq, p.mk, p.k, bc));
+        for (int j = 0; j < 4; ++j)
+          if (h0 + j < p.hpg)
+            load_b<KMAX>(p.wb_q, p.wb_fp32, p.k, p.n_q, (int64_t)(g * p.hpg + h0 + j) * p.head_dim + d, bq[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (h0 + j < p.hpg) qs += sqrt(quad_form<KMAX>(Gq, p.mk, p.k, bq[j]));
     }
     p.scores_qk[u] = (float)(qs * sqrt(quad_form<KMAX>(Gk, p.mk, p.k, bk)));
-  } else {
-    const int64_t i = u - p.n_qk;
-    float b[KMAX];
-    load_b<KMAX>(p.wb_l2, p.wb_fp32, p.k, p.n_l2, i, b);
-    p.scores_l2[i] = (float)sqrt(quad_form<KMAX>(gs + p.blk_l2 * p.k * p.mk + p.blk_l2 * p.k, p.mk, p.k, b));
+  } else if (is_l2) {
+    p.scores_l2[u - p.n_qk] = (float)sqrt(quad_form<KMAX>(gs + p.blk_l2 * p.k * p.mk + p.blk_l2 * p.k, p.mk, p.k, bk));
   }
 }
 
@@ -884,20 +921,21 @@ int est_scores(const double* gram_part, int n_parts, int mk, int k, int wb_fp32,
   }
   const int64_t units = P.n_qk + P.n_l2;
   if (units <= 0) return 1;
-  const unsigned grid = (unsigned)((units + 255) / 256);
+  const unsigned grid = (unsigned)((units + kScoreThreads - 1) / kScoreThreads);
   const size_t smem = (size_t)mk * mk * sizeof(double);
   if (k <= 8)
-    launch_kernel(est_scores_kernel<8>, grid, 256, smem, s, P);
+    launch_kernel(est_scores_kernel<8>, grid, kScoreThreads, smem, s, P);
   else
-    launch_kernel(est_scores_kernel<16>, grid, 256, smem, s, P);
+    launch_kernel(est_scores_kernel<16>, grid, kScoreThreads, smem, s, P);
   if (launch_failed("sl_estimator")) return 5;
   note_launch();
   return 0;
 }
 
 int z_finish(const float* z, int64_t ld_z, int64_t n_ctx, int mk, int k, double* gram_part, void* zsplit,
-             cudaStream_t s) {
+             int* ticket, double* gram_total, cudaStream_t s) {
   if (n_ctx <= 0 || mk <= 0 || mk > 64 || mk % 4 || ld_z < mk || (!gram_part && !zsplit)) return 1;
+  if (gram_total && (!gram_part || !ticket)) return 1;
   if (!gram_part && (k != 4 && k != 8 && k != 16)) return 1;
   const int64_t tiles = (n_ctx + 127) / 128;
   if (tiles > 2147483647LL) return 1;
@@ -911,7 +949,7 @@ int z_finish(const float* z, int64_t ld_z, int64_t n_ctx, int mk, int k, double*
     attr = true;
   }
   launch_kernel(z_finish_kernel, (unsigned)tiles, kZThreads, smem, s, z, ld_z, n_ctx, mk, k, gram_part,
-                static_cast<__nv_bfloat16*>(zsplit));
+                static_cast<__nv_bfloat16*>(zsplit), ticket, gram_total);
   if (launch_failed("sl_est_tc")) return 5;
   note_launch();
   return 0;

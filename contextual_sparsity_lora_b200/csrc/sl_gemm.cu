@@ -481,6 +481,74 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
   }
 }
 
+// ---- row-gathered B operands (Seg::gidx)
+//
+// A gathered segment reads its B rows straight from the full weight: B row q of the stage is
+// weight row gidx[q] (q < g_valid), fetched by tile::gather4 copies of four 128-byte rows
+// each, and a zero row from the zero map past the kept count. The producer warp's lanes
+// issue the copies of one group of four rows each.
+struct Rows4 {
+  int32_t r[4];
+  uint32_t m;  // bit i set: row i comes from the weight; clear: from the zero row
+};
+
+// Weight rows of B positions q .. q + 3 (q a multiple of 4, gidx 16-byte aligned).
+__device__ __forceinline__ Rows4 gather_rows4(const Seg& sg, int q, int* err) {
+  Rows4 o;
+  if (q + 3 < sg.g_valid) {
+    const int4 v = __ldg(reinterpret_cast<const int4*>(sg.gidx + q));
+    o.r[0] = v.x;
+    o.r[1] = v.y;
+    o.r[2] = v.z;
+    o.r[3] = v.w;
+    o.m = 15u;
+  } else {
+    o.m = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool v = q + i < sg.g_valid;
+      o.r[i] = v ? __ldg(sg.gidx + q + i) : 0;
+      o.m |= (uint32_t)v << i;
+    }
+  }
+#ifdef SL_DEBUG_BOUNDS
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (((o.m >> i) & 1u) && !index_ok(o.r[i], sg.g_rows, err, DEV_BAD_GATHER_ROW)) o.m &= ~(1u << i);
+#else
+  (void)err;
+#endif
+  return o;
+}
+
+// Four B rows at dst (512 bytes, 128-byte rows): one gather4 copy when all four come from the
+// weight or all from the zero row, else one single-row copy each. Every copy lands 512 bytes
+// on the stage barrier in total, whatever the mix.
+template <bool PAIR>
+__device__ __forceinline__ void gather_issue4(uint8_t* dst, const CUtensorMap* mw, const CUtensorMap* mz,
+                                              uint64_t* bar, int x, const Rows4& g) {
+  if (g.m == 15u) {
+    if (PAIR)
+      tma_gather4_pair(dst, mw, bar, x, g.r[0], g.r[1], g.r[2], g.r[3]);
+    else
+      tma_gather4(dst, mw, bar, x, g.r[0], g.r[1], g.r[2], g.r[3]);
+  } else if (g.m == 0u) {
+    if (PAIR)
+      tma_gather4_pair(dst, mz, bar, 0, 0, 0, 0, 0);
+    else
+      tma_gather4(dst, mz, bar, 0, 0, 0, 0, 0);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool w = (g.m >> i) & 1u;
+      if (PAIR)
+        tma_load_2d_pair(dst + 128 * i, w ? mw : mz, bar, w ? x : 0, w ? g.r[i] : 0);
+      else
+        tma_load_2d(dst + 128 * i, w ? mw : mz, bar, w ? x : 0, w ? g.r[i] : 0);
+    }
+  }
+}
+
 // The one-CTA kernel's stage ring holds B tiles of BROWS rows (or N columns): skinny
 // launches (the rank-r LoRA products, estimator stage 1) stage only the B rows they use
 // and keep 6 or 8 stages of A in flight instead of 4 in the same shared memory.
@@ -536,7 +604,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the prologue above overlaps the previous kernel's tail
 
-  if (warp == 0) {
+  if (warp == 0 && !p.any_gather) {
+    // No gathered B rows in this launch: lane 0 alone runs the producer loop.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -553,7 +622,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const int kb_lo = max(0, ti.kb0 - g), kb_hi = min(sg.nk, ti.kb1 - g);
           g += sg.nk;
           for (int kb = kb_lo; kb < kb_hi; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto plain_done;
             mbar_arrive_expect_tx(&full[stage], bytes);
             issued_mask |= 1u << stage;
             issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -584,11 +653,88 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           }
         }
       }
-    producer_done:
+    plain_done:
       // Every issued copy must land before the CTA may exit.
       for (int s = 0; s < C::kStages; ++s)
         if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
+  } else if (warp == 0) {
+    // The whole warp runs the loop (lanes issue the copies of gathered B rows); lane 0 waits
+    // on the ring, arms the stage and issues every other copy.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
+      const TileInfo ti = decode_tile(p, t);
+      const Prob& pr = p.probs[ti.prob];
+      const int n0 = ti.tn * pr.tile_cols;
+      int g = 0;  // k-blocks of earlier active segments
+      for (int s = 0; s < pr.nseg; ++s) {
+        const Seg& sg = pr.seg[s];
+        if (n0 >= sg.n_limit) continue;
+        const uint32_t bytes = seg_tx_bytes(sg);
+        const int kb_lo = max(0, ti.kb0 - g), kb_hi = min(sg.nk, ti.kb1 - g);
+        g += sg.nk;
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) goto producer_done;
+          uint8_t* sa = smem_a + stage * kStageABytes;
+          uint8_t* sb = smem_b + stage * C::kStageB;
+          const int kc = kb * kBK;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            issued_mask |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (!sg.a_mn) {
+              tma_load_2d(sa, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, sg.a_row0 + ti.tm * kBM);
+            } else {
+              tma_load_2d(sa, &p.maps[sg.a_map], &full[stage], sg.a_row0 + ti.tm * kBM, sg.a_k0 + kc);
+              tma_load_2d(sa + 8192, &p.maps[sg.a_map], &full[stage], sg.a_row0 + ti.tm * kBM + 64, sg.a_k0 + kc);
+            }
+          }
+          for (int i = 0; i < sg.nb; ++i) {
+            const BSrc& b = sg.b[i];
+            const int coord = b.row0 + b.row_step * ti.tn;
+            if (b.gather) {
+              const int ng = sg.b_mn ? 16 * (b.rows / 64) : b.rows / 4;  // groups of four rows
+              for (int q4 = lane; q4 < ng; q4 += 32) {
+                if (!sg.b_mn) {
+                  const Rows4 r = gather_rows4(sg, coord + 4 * q4, p.err);
+                  gather_issue4<false>(sb + b.tile_off * 128 + q4 * 512, &p.maps[b.map], &p.maps[sg.zmap], &full[stage],
+                                       sg.b_k0 + kc, r);
+                } else {
+                  const int c = q4 >> 4, x = coord + 64 * c;
+                  Rows4 r = gather_rows4(sg, sg.b_k0 + kc + 4 * (q4 & 15), p.err);
+                  if (x >= sg.g_cols) r.m = 0u;
+                  gather_issue4<false>(sb + (b.tile_off / 64 + c) * 8192 + (q4 & 15) * 512, &p.maps[b.map],
+                                       &p.maps[sg.zmap], &full[stage], x, r);
+                }
+              }
+            } else if (lane == 0) {
+              if (!sg.b_mn) {
+                tma_load_2d(sb + b.tile_off * 128, &p.maps[b.map], &full[stage], sg.b_k0 + kc, coord);
+              } else {
+                for (int c = 0; c < b.rows / 64; ++c)
+                  tma_load_2d(sb + (b.tile_off / 64 + c) * 8192, &p.maps[b.map], &full[stage], coord + 64 * c,
+                              sg.b_k0 + kc);
+              }
+            }
+          }
+          __syncwarp();
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  producer_done:
+    // Every issued copy must land before the CTA may exit.
+    if (lane == 0)
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0;
@@ -769,7 +915,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the prologue above overlaps the previous kernel's tail
 
-  if (warp == 0) {
+  if (warp == 0 && !p.any_gather) {
+    // No gathered B rows in this launch: lane 0 alone runs the producer loop.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -782,7 +929,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const Seg& sg = pr.seg[s];
           if (n0 >= sg.n_limit) continue;
           for (int kb = 0; kb < sg.nk; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto producer_done;
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) goto plain_done;
             if (leader) {
               mbar_arrive_expect_tx(&full[stage], 2u * (C::kStageA + kStageB2Bytes));
               issued_mask |= 1u << stage;
@@ -810,11 +957,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-    producer_done:
+    plain_done:
       // The even CTA's barriers count both CTAs' copies: wait for every stage it armed.
       for (int s = 0; s < C::kStages; ++s)
         if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
+  } else if (warp == 0) {
+    // The whole warp runs the loop (lanes issue the copies of gathered B rows, one group of
+    // four rows each); lane 0 waits on the ring, arms the stage (even CTA) and issues the
+    // copies of A and of plain B sources.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;
+    for (int t = cl; t < p.total_tiles; t += n_cl) {
+      if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
+      const TileInfo ti = decode_tile(p, t);
+      const Prob& pr = p.probs[ti.prob];
+      const int n0 = ti.tn * pr.tile_cols;
+      for (int s = 0; s < pr.nseg; ++s) {
+        const Seg& sg = pr.seg[s];
+        if (n0 >= sg.n_limit) continue;
+        // Gathered segment: this CTA stages 128 B rows (K-major: positions qb + j of the one
+        // source it loads) or two 64-column blocks of 64 K rows (MN-major).
+        const bool gat = sg.gidx != nullptr;
+        const BSrc& gb = sg.b[sg.nb == 1 ? 0 : (int)rank];
+        const int gcoord = gb.row0 + gb.row_step * ti.tn;
+        int gx = 0, gq = 0;
+        int gdst = 0;  // byte offset of this lane's four rows within the stage's B tile
+        Rows4 gr;
+        gr.m = 0u;
+        if (gat) {
+          if (!sg.b_mn) {
+            gq = gcoord + (gb.rows == 256 ? 128 * (int)rank : 0) + 4 * lane;
+            gdst = lane * 512;
+            gr = gather_rows4(sg, gq, p.err);  // the same rows for every k-block of the tile
+          } else {
+            gx = gcoord + 128 * (int)rank + 64 * (lane >> 4);
+            gq = sg.b_k0 + 4 * (lane & 15);
+            gdst = (lane >> 4) * 8192 + (lane & 15) * 512;
+            gr = gather_rows4(sg, gq, p.err);  // k-block 0; each later block's rows are loaded one ahead
+            if (gx >= sg.g_cols) gr.m = 0u;
+          }
+        }
+        for (int kb = 0; kb < sg.nk; ++kb) {
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) goto producer_done;
+          uint8_t* sa = smem_a + stage * C::kStageA;
+          uint8_t* sb = smem_b + stage * kStageB2Bytes;
+          const int kc = kb * kBK;
+          if (lane == 0) {
+            if (leader) {
+              mbar_arrive_expect_tx(&full[stage], 2u * (C::kStageA + kStageB2Bytes));
+              issued_mask |= 1u << stage;
+              issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            }
+            const int arow = sg.a_row0 + ti.tm * C::kTileM + 128 * MH * (int)rank;
+#pragma unroll
+            for (int h = 0; h < MH; ++h) {
+              uint8_t* sah = sa + h * kStageABytes;
+              if (!sg.a_mn) {
+                tma_load_2d_pair(sah, &p.maps[sg.a_map], &full[stage], sg.a_k0 + kc, arow + 128 * h);
+              } else {
+                tma_load_2d_pair(sah, &p.maps[sg.a_map], &full[stage], arow + 128 * h, sg.a_k0 + kc);
+                tma_load_2d_pair(sah + 8192, &p.maps[sg.a_map], &full[stage], arow + 128 * h + 64, sg.a_k0 + kc);
+              }
+            }
+            if (!gat) pair_b_loads(p, sg, ti.tn, rank, sb, &full[stage], kc);
+          }
+          if (gat) {
+            gather_issue4<true>(sb + gdst, &p.maps[gb.map], &p.maps[sg.zmap],
+                                &full[stage], sg.b_mn ? gx : sg.b_k0 + kc, gr);
+            if (sg.b_mn && kb + 1 < sg.nk) {
+              gr = gather_rows4(sg, gq + (kb + 1) * kBK, p.err);
+              if (gx >= sg.g_cols) gr.m = 0u;
+            }
+          }
+          __syncwarp();
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  producer_done:
+    // The even CTA's barriers count both CTAs' copies: wait for every stage it armed.
+    if (lane == 0)
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, p.err, DEV_TIMEOUT_DRAIN);
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       int stage = 0;
@@ -1023,7 +1254,7 @@ bool GemmBuilder::pair_eligible() const {
     const char* e = getenv("SL_GEMM_1CTA");
     return e && e[0] == '1';
   }();
-  if (disabled || nprob == 0) return false;
+  if (disabled || nprob == 0 || forced_pair_mh() < 0) return false;
   for (int i = 0; i < nprob; ++i) {
     const Prob& pr = params.probs[i];
     if (pr.ksplit > 1 || pr.n_mma != kBN) return false;
@@ -1112,6 +1343,26 @@ void GemmBuilder::bsrc(Seg* s, int map, int tile_off, int rows, int row0, int ro
   b.row_step = row_step;
 }
 
+void GemmBuilder::gather(Seg* s, const int32_t* idx, int64_t n_valid, int64_t g_rows, int64_t g_cols,
+                         const void* zero_row) {
+  if (!s || status != 0) return;
+  if (!idx || (reinterpret_cast<uintptr_t>(idx) & 15) || n_valid < 0 || n_valid > g_rows || g_rows <= 0 ||
+      g_rows > INT32_MAX || g_cols <= 0 || g_cols % 64 || g_cols > INT32_MAX || !zero_row || s->nb == 0) {
+    status = 2;
+    return;
+  }
+  if (zmap < 0) {
+    zmap = map(zero_row, 1, 64, 64, 1);
+    if (status != 0) return;
+  }
+  s->gidx = idx;
+  s->g_valid = (int32_t)n_valid;
+  s->g_rows = (int32_t)g_rows;
+  s->g_cols = (int32_t)g_cols;
+  s->zmap = (int16_t)zmap;
+  for (int i = 0; i < s->nb; ++i) s->b[i].gather = 1;
+}
+
 // Rows per CTA pair (256 or 512) for a pair-eligible launch: the one with the smaller
 // estimated makespan of the round-robin persistent schedule over `pairs` CTA pairs. Cost
 // of a tile in 64-wide k-block units of a 256 x 256 tile: a 512-row tile moves 1.5x the
@@ -1193,7 +1444,7 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
         if (sg.b_mn) continue;
         for (int b = 0; b < sg.nb; ++b) {
           BSrc& bs = sg.b[b];
-          if (bs.rows != 256) continue;
+          if (bs.rows != 256 || bs.gather) continue;
           if (remap[bs.map] < 0) {
             const MapSpec sp = specs[bs.map];
             remap[bs.map] = map(sp.ptr, sp.rows, sp.cols, sp.ld, 128);
@@ -1218,7 +1469,16 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
         const BSrc& bs = sg.b[b];
         if (bs.tile_off + bs.rows > kBN || bs.tile_off % 8) return 4;
         if (sg.b_mn && (bs.rows % 64 || bs.tile_off % 64)) return 4;
+        if (bs.gather) {
+          // a row-gather map over the segment's gathered tensor; group positions 16-byte aligned
+          const MapSpec& sp = specs[bs.map];
+          if (!sg.gidx || sp.box_rows != 1 || sp.cols != sg.g_cols || sp.rows != sg.g_rows || bs.rows % 4 ||
+              bs.row0 % 4 || bs.row_step % 4 || sg.b_k0 % 4)
+            return 4;
+          if (!sg.b_mn && sg.b_k0 + sg.nk * kBK > sg.g_cols) return 4;  // every K box inside the rows
+        }
       }
+      if (sg.gidx && pr.ksplit > 1) return 4;
     }
     if (!always) return 4;
     pr.tiles_m = pr.M > 0 ? (pr.M + tile_m - 1) / tile_m : 0;
@@ -1241,6 +1501,10 @@ int GemmBuilder::launch(int* err, cudaStream_t stream) {
   params.nprob = nprob;
   params.total_tiles = total;
   params.err = err;
+  params.any_gather = 0;
+  for (int i = 0; i < nprob; ++i)
+    for (int s = 0; s < params.probs[i].nseg; ++s)
+      if (params.probs[i].seg[s].gidx) params.any_gather = 1;
   if (total == 0) return 0;
   attach_output_maps();
   static int smem_set = 0;

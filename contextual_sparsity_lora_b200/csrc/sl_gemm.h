@@ -7,7 +7,9 @@
 // MN-major (M or N contiguous); a segment can be switched off for the output
 // tiles at or beyond a channel limit (the kept prefix of a channel-ordered
 // output). The B tile of a segment can be assembled from up to four sources
-// (e.g. the gate and up weights for the two halves of a paired SwiGLU tile).
+// (e.g. the gate and up weights for the two halves of a paired SwiGLU tile), and its rows can
+// be gathered through an index list straight from the full weight (tile::gather4 copies of
+// the kept rows; positions past the kept count read a zero row).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -22,8 +24,11 @@ constexpr int kMaxMaps = 48;
 constexpr int kMaxProbs = 12;
 constexpr int kMaxSegs = 6;
 constexpr int kMaxBSrc = 4;
-// Workspace header: error word at byte 0, split-tile finish counters from byte 256.
+// Workspace header: error word at byte 0, a zero row of 64 bf16 at bytes 128..255 (the zero
+// source of gathered B operands; cleared with the header and never written), split-tile finish
+// counters from byte 256.
 constexpr int kWorkspaceHeaderBytes = 65536;
+constexpr int kZeroRowOffsetBytes = 128;
 constexpr int kCounterOffsetInts = 64;
 constexpr int kMaxSplitCounters = (kWorkspaceHeaderBytes - 256) / 4;
 constexpr int kEpiWarps = 8;       // two epilogue warps per TMEM lane quarter, splitting the columns
@@ -51,7 +56,7 @@ struct BSrc {
   int16_t map;       // tensor map index
   int16_t tile_off;  // first row of the B tile (K-major) / first N column (MN-major) this source fills
   int16_t rows;      // rows (K-major, = box height) / N columns (MN-major, multiple of 64) it fills
-  int16_t pad_;
+  int16_t gather;    // 1: the map is a row-gather map (box 64 x 1) read through the segment's index list
   int32_t row0;      // coordinate of that first row / column for output tile 0
   int32_t row_step;  // coordinate advance per output tile along N
 };
@@ -64,6 +69,14 @@ struct Seg {
   int32_t nk;           // number of kBK blocks
   int32_t n_limit;      // segment runs only for tiles whose first output column < n_limit
   BSrc b[kMaxBSrc];
+  // Row gather of the B operand (sources with `gather` set): the B row at position q (the N
+  // coordinate for K-major B, the K coordinate for MN-major B) is row gidx[q] of the source's
+  // tensor when q < g_valid, and zero from the zero map `zmap` otherwise (and for MN-major
+  // column blocks at or past g_cols); g_rows = rows of the gathered tensors (checked in the
+  // debug build).
+  const int32_t* gidx;
+  int32_t g_valid, g_rows, g_cols;
+  int16_t zmap, pad_;
 };
 
 struct Prob {
@@ -101,6 +114,7 @@ struct GemmParams {
   CUtensorMap maps[kMaxMaps];
   Prob probs[kMaxProbs];
   int32_t nprob, total_tiles;
+  int32_t any_gather;   // some segment gathers its B rows (the producer warp's lanes issue those copies)
   int* err;
   int* counters;        // split-tile finish counters (zero between launches)
 };

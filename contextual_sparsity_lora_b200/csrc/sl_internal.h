@@ -110,13 +110,20 @@ struct GemmBuilder {
   // K is the segment's K extent; n_limit = output column limit (use N or more for "always").
   Seg* seg(Prob* pr, int a_map, int a_mn, int a_row0, int a_k0, int b_mn, int b_k0, int K, int n_limit);
   void bsrc(Seg* s, int map, int tile_off, int rows, int row0, int row_step);
+  // Row-gather map of a bf16 weight [rows, cols] (box 64 columns x 1 row) for gathered B sources.
+  int gmap(const void* ptr, int64_t rows, int64_t cols, int64_t ld) { return map(ptr, rows, cols, ld, 1); }
+  // Make every B source of `s` (all made from gmap() maps over [g_rows, g_cols] tensors) a row
+  // gather: B position q reads row idx[q] when q < n_valid, else the zero row. zero_row: 64 bf16
+  // zeros in device memory (the workspace's zero row). idx 16-byte aligned; g_cols % 64 == 0.
+  void gather(Seg* s, const int32_t* idx, int64_t n_valid, int64_t g_rows, int64_t g_cols, const void* zero_row);
+  int zmap = -1;  // the launch's zero-row map, made by the first gather()
   // Compute a skinny problem as `ksplit` K ranges; `part` holds ksplit * M * N floats.
   void split(Prob* pr, int ksplit, float* part);
   int launch(int* err, cudaStream_t stream);
 };
 
 // Forced CTA-pair tile height of the GEMM engine: 0 = chosen per launch, 1 = 256 rows,
-// 2 = 512 rows (sl_set_pair_tile_rows).
+// 2 = 512 rows, -1 = no CTA pairs (every launch on the one-CTA kernel) (sl_set_pair_tile_rows).
 void set_forced_pair_mh(int mh);
 int forced_pair_mh();
 
@@ -151,9 +158,11 @@ int est_swiglu_tc(const void* zsplit, int64_t n_ctx, int k, const void* wb_g, co
                   float* scores, double* sumsq, int* err, cudaStream_t s);
 // Z (fp32 [n_ctx][ld_z], computed elsewhere) -> per-128-row-tile fp64 Gram shares
 // (gram_part [tiles][mk][mk]) or the three-term bf16 split for est_swiglu_tc (zsplit
-// [n_ctx][128], two projections of k columns each). One launch.
+// [n_ctx][128], two projections of k columns each). One launch. gram_total (optional, with
+// gram_part): the shares summed in tile order by the launch's last CTA; ticket: a counter
+// that is zero between calls.
 int z_finish(const float* z, int64_t ld_z, int64_t n_ctx, int mk, int k, double* gram_part, void* zsplit,
-             cudaStream_t s);
+             int* ticket, double* gram_total, cudaStream_t s);
 // out[mk][mk] = sum of n_parts Gram matrices in order; scores = sqrt(sumsq).
 int gram_sum(const double* parts, int n_parts, int mk, double* out, cudaStream_t s);
 int sqrt_scores(const double* sumsq, int64_t n, float* scores, cudaStream_t s);

@@ -55,17 +55,33 @@ __device__ int block_exclusive_scan(int v, int* warp_sums) {
   return excl;
 }
 
-// Block-wide sum of one int per thread; `slot` alternates between calls so that one
-// barrier per call suffices (a slot is rewritten only two calls later, after every
-// thread has passed the barrier of the call in between).
-__device__ __forceinline__ int block_sum(int v, int (*red)[32], int& slot) {
+// Exclusive block scan of one int per thread (1024 threads) that also returns the block total.
+__device__ int block_exclusive_scan_total(int v, int* warp_sums, int* total_slot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = __reduce_add_sync(0xffffffffu, v);
-  if (lane == 0) red[slot][warp] = v;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
-  const int tot = __reduce_add_sync(0xffffffffu, red[slot][lane]);
-  slot ^= 1;
-  return tot;
+  if (warp == 0) {
+    const int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+    if (lane == 31) *total_slot = wi;
+  }
+  __syncthreads();
+  const int excl = warp_sums[warp] + incl - v;
+  total = *total_slot;
+  __syncthreads();
+  return excl;
 }
 
 __host__ __device__ inline int stage_words(int n, int n_wide) {
@@ -80,15 +96,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   // staging words for scores in / sigma out (and sigma_wide when it fits), then [n] kept flags
   extern __shared__ uint32_t sbuf[];
   uint8_t* keep = reinterpret_cast<uint8_t*>(sbuf + stage_words(n, n_wide));
-  __shared__ int red[2][32];
   __shared__ uint32_t s_or[32], s_and[32];
   __shared__ int warp_sums[32];
-  __shared__ int hist[256];
-  __shared__ int sel_state[2];
+  __shared__ int hist[4][256];  // one histogram per radix pass, all zeroed before the first
+  __shared__ int scan_total;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per = (n + kSelThreads - 1) / kSelThreads;  // <= PER
   const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
   for (int i = threadIdx.x; i < n; i += kSelThreads) sbuf[i] = __float_as_uint(scores[i]);
+  for (int i = threadIdx.x; i < 4 * 256; i += kSelThreads) (&hist[0][0])[i] = 0;
   __syncthreads();
 
   uint32_t key[PER];
@@ -125,55 +141,46 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     const int first = (top / 8) * 8;
     tmask = first + 8 < 32 ? ~((1u << (first + 8)) - 1u) : 0u;  // bytes above the first pass
     T &= tmask;
-    for (int shift = first; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
-      __syncthreads();
+    for (int shift = first, pass = 0; shift >= 0; shift -= 8, ++pass) {
 #pragma unroll
       for (int j = 0; j < PER; ++j)
-        if (i0 + j < i1 && (key[j] & tmask) == T) atomicAdd(&hist[(key[j] >> shift) & 255u], 1);
+        if (i0 + j < i1 && (key[j] & tmask) == T) atomicAdd(&hist[pass][(key[j] >> shift) & 255u], 1);
       __syncthreads();
-      if (warp == 0) {
-        // lane l holds bins 255 - 8 l .. 248 - 8 l (descending); counts from the top
-        int c[8], tot = 0;
+      // every warp reads the finished histogram and picks the same byte (no second barrier):
+      // lane l holds bins 255 - 8 l .. 248 - 8 l (descending), counts from the top
+      int c[8], tot = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          c[e] = hist[255 - 8 * lane - e];
-          tot += c[e];
-        }
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int nb = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += nb;
-        }
-        int above = incl - tot;  // matching keys whose byte lies above this lane's bins
-        int pick = -1, above_pick = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (pick < 0 && above < need && above + c[e] >= need) {
-            pick = 255 - 8 * lane - e;
-            above_pick = above;
-          }
-          above += c[e];
-        }
-        const unsigned who = __ballot_sync(0xffffffffu, pick >= 0);  // one lane holds the crossing
-        const int src = who ? __ffs(who) - 1 : 0;
-        pick = __shfl_sync(0xffffffffu, pick, src);
-        above_pick = __shfl_sync(0xffffffffu, above_pick, src);
-        if (lane == 0) {
-          sel_state[0] = pick < 0 ? 0 : pick;
-          sel_state[1] = above_pick;
-        }
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[pass][255 - 8 * lane - e];
+        tot += c[e];
       }
-      __syncthreads();
-      T |= (uint32_t)sel_state[0] << shift;
-      need -= sel_state[1];
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nb;
+      }
+      int above = incl - tot;  // matching keys whose byte lies above this lane's bins
+      int pick = -1, above_pick = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (pick < 0 && above < need && above + c[e] >= need) {
+          pick = 255 - 8 * lane - e;
+          above_pick = above;
+        }
+        above += c[e];
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, pick >= 0);  // one lane holds the crossing
+      const int src = who ? __ffs(who) - 1 : 0;
+      pick = __shfl_sync(0xffffffffu, pick, src);
+      above_pick = __shfl_sync(0xffffffffu, above_pick, src);
+      T |= (uint32_t)(pick < 0 ? 0 : pick) << shift;
+      need -= above_pick;
       tmask |= 255u << shift;
-      __syncthreads();  // sel_state and hist are rewritten by the next pass
     }
   }
-  int slot = 0;
-  // Keys above T are kept; keys equal to T fill the remaining places lowest index first.
+  // Keys above T are kept; keys equal to T fill the remaining places lowest index first. One
+  // exclusive scan of both per-thread counts, packed in the halves of an int (each <= 40960).
   int gt = 0, n_eq = 0;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
@@ -181,21 +188,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     gt += valid && key[j] > T ? 1 : 0;
     n_eq += valid && key[j] == T ? 1 : 0;
   }
-  const int take_eq = n_keep - block_sum(gt, red, slot);
-  int eq_rank = block_exclusive_scan(n_eq, warp_sums);
+  int total = 0;
+  const int packed = block_exclusive_scan_total(gt | (n_eq << 16), warp_sums, &scan_total, total);
+  const int take_eq = n_keep - (total & 0xffff);
+  int eq_rank = packed >> 16;
+  int kept_before = (packed & 0xffff) + min(eq_rank, take_eq);
   uint64_t kmask = 0;
-  int n_kept = 0;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     if (i0 + j >= i1) break;
     bool kp = key[j] > T;
     if (key[j] == T) kp = eq_rank++ < take_eq;
-    if (kp) {
-      kmask |= 1ull << j;
-      ++n_kept;
-    }
+    if (kp) kmask |= 1ull << j;
   }
-  int kept_before = block_exclusive_scan(n_kept, warp_sums);  // also orders the key reads before the reuse
   int drop_before = i0 - kept_before;
   const bool wide = hpg > 0 && sigma_wide != nullptr;
 #pragma unroll

@@ -91,9 +91,10 @@ typedef enum { SL_LORA_FWD = 0, SL_LORA_BWD = 1 } sl_lora_mode;
 
 /* Caller-owned scratch memory. When ptr is NULL or bytes < the size a call needs, the
  * call stores the size in `needed` and returns SL_ERR_WORKSPACE without launching.
- * The first 64 KiB are a header: the device error word (byte 0) and the finish counters
- * of split-K GEMM tiles (which the kernels return to zero). Zero the header once with
- * sl_workspace_init before first use. Calls that share a workspace must be ordered on
+ * The first 64 KiB are a header: the device error word (byte 0), a row of 64 bf16 zeros
+ * (bytes 128..255, the zero rows past the kept count of a gathered GEMM operand; never
+ * written) and the finish counters of split-K GEMM tiles (which the kernels return to
+ * zero). Zero the header once with sl_workspace_init before first use. Calls that share a workspace must be ordered on
  * one stream (they reuse the same scratch and counters). */
 typedef struct {
   void* ptr;
@@ -114,12 +115,18 @@ typedef struct {
   int32_t pad_;
   /* Optional (may be NULL): the kept rows of the sliced weight for the channel set passed
    * with the call, row-major and dense: SL_SLICE_OUT: w[sigma[j], :] for j < n_keep
-   * ([n_keep, d_in]); SL_SLICE_IN: w_t[sigma[j], :] ([n_keep, d_out]). The forward and
-   * the backward of one step use the same rows, so a caller that builds them once per
-   * step (sl_gather_rows_batch or sl_permute_rows with the first n_keep entries of sigma,
-   * several projections per launch with the former) saves both calls their
-   * own gather into the workspace. With keep ratio 1 and the identity sigma it is w
-   * (w_t) itself. The caller keeps it consistent with sigma; 16-byte aligned. */
+   * ([n_keep, d_in]); SL_SLICE_IN: w_t[sigma[j], :] ([n_keep, d_out]). With keep ratio 1
+   * and the identity sigma it is w (w_t) itself. The caller keeps it consistent with sigma;
+   * 16-byte aligned.
+   * A compacted copy given here is the faster form on B200: the forward and the backward
+   * of a step share it, and the GEMM stages it with tiled tensor copies.
+   * NULL: the sliced products read the kept rows in place, each GEMM operand tile assembled
+   * by row-gather tensor copies (tile::gather4, four 128-byte rows per copy) of w
+   * (SL_SLICE_OUT) or w_t (SL_SLICE_IN) through sigma, with no copy of the rows, as long as
+   * the gathered rows are whole 64-column boxes (d_in % 64 == 0 for SL_SLICE_OUT,
+   * d_out % 64 == 0 for SL_SLICE_IN) and sigma is 16-byte aligned; otherwise each call first
+   * gathers the kept rows into its workspace (sl_gather_rows_batch semantics). Every form
+   * gives the same result bit for bit. */
   const void* w_kept;
 } sl_linear;
 
@@ -412,10 +419,12 @@ SL_API sl_status sl_attention_bwd(const void* q, const void* k, const void* v, c
 /* Tile height of the CTA-pair tensor-core GEMM that runs the sliced products (a4, a5):
  * rows = 256 (each pair of SMs computes 256 x 256 output tiles with two accumulators, so a
  * tile's epilogue overlaps the next tile's products), 512 (512 x 256 tiles: a quarter fewer
- * operand bytes per FLOP, epilogue not overlapped), or 0 (the default: chosen per launch by
- * a makespan model of the persistent schedule). Process-wide; applies to launches issued
- * (or captured) after the call; changes how a product is tiled, never its result beyond
- * the fp32 summation order of the tile. Errors: SL_ERR_INVALID_ARG for any other value. */
+ * operand bytes per FLOP, epilogue not overlapped), 128 (no CTA pairs: every GEMM launch runs
+ * on the one-CTA kernel with 128-row tiles, the slower path kept for shapes the pair kernel
+ * does not take), or 0 (the default: chosen per launch by a makespan model of the persistent
+ * schedule). Process-wide; applies to launches issued (or captured) after the call; changes
+ * how a product is tiled, never its result beyond the fp32 summation order of the tile.
+ * Errors: SL_ERR_INVALID_ARG for any other value. */
 SL_API sl_status sl_set_pair_tile_rows(int32_t rows);
 
 /* w_t[d_in, d_out] = w^T for a frozen weight (once per weight). */
@@ -448,7 +457,8 @@ SL_API sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const i
  * --debug writes libsparselora_debug.so; the release library has none) checks, on the device,
  * every index it reads from a channel set (sigma), a row permutation or a gather list against the
  * extent it indexes, before the access that index drives: gathered weight rows against the source's
- * rows (src_rows above, d_out or d_in of a projection), gathered activation and LoRA columns
+ * rows (src_rows above, d_out or d_in of a projection; also the rows a sliced product gathers
+ * in place, which then read the zero row instead), gathered activation and LoRA columns
  * against their columns, scattered output columns and rows against the product's extent, dB rows
  * against the adapter's output channels. A failing check skips that access (nothing outside the
  * caller's buffers is read or written) and records a code, first writer wins: 0x101 row gather,

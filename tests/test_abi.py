@@ -202,10 +202,11 @@ def test_layer_and_optimizer_entries_reject_bad_arguments(lib):
 
 
 def test_pair_tile_rows_setting_host_side(lib):
-    """The tile-height setting accepts 0 (chosen per launch), 256 and 512, and nothing else."""
-    for rows in (256, 512, 0):
+    """The tile-height setting accepts 0 (chosen per launch), 128 (no CTA pairs), 256 and 512,
+    and nothing else."""
+    for rows in (128, 256, 512, 0):
         assert lib.sl_set_pair_tile_rows(rows) == B.SL_OK
-    for rows in (-1, 1, 128, 384, 1024):
+    for rows in (-1, 1, 64, 384, 1024):
         assert lib.sl_set_pair_tile_rows(rows) == B.SL_ERR_INVALID_ARG
     assert lib.sl_set_pair_tile_rows(0) == B.SL_OK
 
