@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-layer", action="store_true", help="skip the whole-decoder-layer measurement")
     ap.add_argument("--no-model", action="store_true", help="skip the 32-layer fine-tuning run")
     ap.add_argument("--no-sweep", action="store_true", help="skip the keep-ratio sweep and the LLaMA2-13B layer")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time only the causal GQA attention core at the LLaMA3-8B layer's shape and print it")
     ap.add_argument("--stages-only", action="store_true",
                     help="time only the selection stages (estimator, criterion, top-n, compaction) of both blocks "
                          "and print them; no step, no headline line")
@@ -248,12 +250,12 @@ def capture_graph(fn, warm=True):
 # launches of one step of this workload, from an ncu capture of one step's CTA-pair launches
 # (dram__bytes_read.sum + dram__bytes_write.sum: 3014.7 MB per step). Valid for the kernel
 # as captured; to be set to None when the kernel changes.
-PAIR_DRAM_BYTES_PER_LAUNCH = 3009.4e6 / 8
+PAIR_DRAM_BYTES_PER_LAUNCH = 3016.5e6 / 8
 PAIR_DRAM_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of the step's 8 launches"
 # SHA-256 (first 16 hex digits) of the sources that define gemm_pair_kernel, as they were when the
 # figure above was captured; when the sources differ the figure is stale and is reported as null.
 PAIR_DRAM_SOURCES = ("sl_gemm.cu", "sl_gemm.h", "sl_ptx.cuh", "sl_internal.h")
-PAIR_DRAM_SOURCE_SHA = "8fb721552cbb1aa7"
+PAIR_DRAM_SOURCE_SHA = "06f93c1d6d27ad72"
 
 
 def pair_sources_sha() -> str:
@@ -561,37 +563,59 @@ def full_layer_measure(attn, ffn, step_in, perm, ac, K, W, device):
             "layer": "RMSNorm, sparse q/k/v, attention, sparse o, residual, RMSNorm, sparse SwiGLU FFN, residual"}
 
 
-def attention_core_measure(layer, ac, K, W, device):
-    """The layer's attention core alone (sl_attention_fwd, sl_attention_bwd on the layer's own q, k,
-    v, o, do buffers after a step), each captured in a CUDA graph of 10 calls: device time per call
-    and TFLOP/s of the causal products (forward Q K^T and P V, backward the recomputed Q K^T, dO V^T,
-    P^T dO, dS^T Q and dS K: 2 and 5 products of 2 hd FLOP per visible (query, key) pair)."""
+def attention_core_times(ws, q, k, v, o, d_o, lse, dq, dk, dv, n_seq, S, hq, hkv, hd, K, W, device):
+    """sl_attention_fwd and sl_attention_bwd on the given buffers, each captured in a CUDA graph of
+    10 calls: device time per call and TFLOP/s of the causal products (forward Q K^T and P V,
+    backward the recomputed Q K^T, dO V^T, P^T dO, dS^T Q and dS K: 2 and 5 products of 2 hd FLOP
+    per visible (query, key) pair)."""
     from contextual_sparsity_lora_b200 import binding as B
-    at = layer.attn
-    n_seq, S = layer.n_seq, layer.S
-    pairs = n_seq * at.hq * S * (S + 1) / 2
+    pairs = n_seq * hq * S * (S + 1) / 2
 
     def fwd():
-        B.sl_attention_fwd(layer.ws, layer.q_nat, layer.k_nat, layer.v_nat, n_seq, at.hq, at.hkv, at.hd,
-                           layer.a_nat, layer.lse)
+        B.sl_attention_fwd(ws, q, k, v, n_seq, hq, hkv, hd, o, lse)
 
     def bwd():
-        B.sl_attention_bwd(layer.ws, layer.q_nat, layer.k_nat, layer.v_nat, layer.a_nat, layer.da_nat, layer.lse,
-                           n_seq, at.hq, at.hkv, at.hd, layer.dq_nat, layer.dk_nat, layer.dv_nat)
+        B.sl_attention_bwd(ws, q, k, v, o, d_o, lse, n_seq, hq, hkv, hd, dq, dk, dv)
 
     out = {"kernels": "attn_fwd_kernel, attn_bwd_kernel (tcgen05, TMEM accumulators)",
-           "shape": f"{n_seq} x {S} tokens, {at.hq} query / {at.hkv} key-value heads of {at.hd}, causal"}
+           "shape": f"{n_seq} x {S} tokens, {hq} query / {hkv} key-value heads of {hd}, causal"}
     peak = float(load_peaks()[0].get("bf16_tflops", 1590.0))
     for name, fn, n_prod in (("fwd", fwd, 2), ("bwd", bwd, 5)):
         fn()
         g = capture_graph(lambda: [fn() for _ in range(10)], warm=False)
         us = time_steps(g.replay, K, W, 1, device) / (10 * K) * 1e3
         del g
-        tf = n_prod * 2.0 * at.hd * pairs / (us * 1e-6) / 1e12
+        tf = n_prod * 2.0 * hd * pairs / (us * 1e-6) / 1e12
         out[f"{name}_us"] = us
         out[f"{name}_tflops"] = tf
         out[f"{name}_frac_of_bf16_peak"] = tf / peak
     return out
+
+
+def attention_core_measure(layer, ac, K, W, device):
+    """The layer's attention core alone, on the layer's own q, k, v, o, dO buffers after a step."""
+    at = layer.attn
+    return attention_core_times(layer.ws, layer.q_nat, layer.k_nat, layer.v_nat, layer.a_nat, layer.da_nat,
+                                layer.lse, layer.dq_nat, layer.dk_nat, layer.dv_nat, layer.n_seq, layer.S, at.hq,
+                                at.hkv, at.hd, K, W, device)
+
+
+def attention_only(device, K, W):
+    """The attention core alone at the LLaMA3-8B layer's shape (8 sequences of 512 tokens, 32
+    query and 8 key-value heads of 128) on seeded normal q, k, v and dO (about 0.1 GB on the
+    device): the small case for profiling the attention kernels."""
+    from contextual_sparsity_lora_b200 import binding as B
+    ac = inputs.LLAMA3_8B_ATTN
+    T, hq, hkv, hd = ac.n_tok, ac.n_q_heads, ac.n_kv_heads, ac.head_dim
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    rnd = lambda n: torch.randn(T, n, generator=g, device=device).to(torch.bfloat16)
+    q, k, v, d_o = rnd(hq * hd), rnd(hkv * hd), rnd(hkv * hd), rnd(hq * hd)
+    o, dq = torch.empty_like(q), torch.empty_like(q)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    lse = torch.empty(hq, T, device=device)
+    return attention_core_times(B.Workspace(device), q, k, v, o, d_o, lse, dq, dk, dv, ac.batch, ac.seq, hq, hkv, hd,
+                                K, W, device)
 
 
 def e2e_measure(attn, ffn, step_in, K, W, world, device, eager=False):
@@ -794,6 +818,14 @@ def main():
     from contextual_sparsity_lora_b200 import binding as B
     from contextual_sparsity_lora_b200 import blocks
     B.lib()
+    if args.attention_only:
+        if rank == 0:
+            print(json.dumps({"attention_core": attention_only(device, args.steps, max(args.warmup, 3))}))
+        barrier(world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     # N > 1: every rank takes its own 4096-token share of the global batch; the criterion
     # statistics and the LoRA gradients are summed over the ranks (NCCL all-reduce)
     dp = blocks.DataParallel() if world > 1 else None
