@@ -110,13 +110,19 @@ struct Prob {
   float* part;          // split-K partials [ksplit][N][M] fp32 (workspace, column-major)
 };
 
+constexpr int kMaxSlots = 4096;
+
 struct GemmParams {
   CUtensorMap maps[kMaxMaps];
   Prob probs[kMaxProbs];
   int32_t nprob, total_tiles;
   int32_t any_gather;   // some segment gathers its B rows (the producer warp's lanes issue those copies)
+  int32_t n_slots;      // CTA-pair launches: slots of the tile order below (0: tile t runs in slot t)
   int* err;
   int* counters;        // split-tile finish counters (zero between launches)
+  // Tile of each slot of the CTA-pair schedule (pair c runs slots c, c + pairs, ...), -1: none.
+  // The host balances the pairs' estimated work by longest-first assignment.
+  int16_t order[kMaxSlots];
 };
 
 }  // namespace sl
