@@ -1,11 +1,11 @@
-// Top-n channel selection over fp32 scores (one CTA of 1024 threads per call).
+// Top-n channel selection over fp32 scores (one CTA per call: 256 to 1024 threads by set size).
 //
 // Scores become order-preserving 32-bit keys (NaN lowest, -0 == +0), held in registers:
 // thread t owns the contiguous index range [t * per, (t + 1) * per). The n-th largest key
 // K* is found by radix selection a byte at a time from the most significant byte in which two
-// keys differ (a shared-memory histogram of 256 bins per pass, at most four passes). Every key
-// above K* is kept, and among keys equal to K*
-// the lowest indices are kept, so exactly n channels survive. The output is a permutation
+// keys differ (a shared-memory histogram of 256 bins per pass, at most four passes; one warp
+// picks each byte). Every key above K* is kept, and among keys equal to K* the lowest indices
+// are kept, so exactly n channels survive. The output is a permutation
 // sigma of [0, N): sigma[0, n) = kept channels ascending, sigma[n, N) = dropped channels
 // ascending. Optionally the selection over KV units (g, d) is expanded to the query side:
 // query channel (h, d) is kept iff unit (h / heads_per_group, d) is. Scores come in and
@@ -19,6 +19,7 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxN = 40960;
+constexpr int kSelMaxNWide = 16384;  // units of a selection with the query-side expansion
 constexpr int kSelStageWords = 40960;  // staging words for scores in / sigma out (160 KB)
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -28,57 +29,33 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan of one int per thread (1024 threads). Returns the thread's prefix.
-__device__ int block_exclusive_scan(int v, int* warp_sums) {
+// Exclusive block scan of one unsigned int per thread (NT threads, arithmetic modulo 2^32)
+// that also returns the block total.
+template <int NT>
+__device__ uint32_t block_exclusive_scan_total(uint32_t v, uint32_t* warp_sums, uint32_t* total_slot,
+                                               uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+  uint32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, incl, o);
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += n;
   }
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int w = warp_sums[lane];
-    int wi = w;
+    const uint32_t w = lane < NT / 32 ? warp_sums[lane] : 0u;
+    uint32_t wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int n = __shfl_up_sync(0xffffffffu, wi, o);
+      const uint32_t n = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += n;
     }
-    warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
-  }
-  __syncthreads();
-  const int excl = warp_sums[warp] + incl - v;
-  __syncthreads();
-  return excl;
-}
-
-// Exclusive block scan of one int per thread (1024 threads) that also returns the block total.
-__device__ int block_exclusive_scan_total(int v, int* warp_sums, int* total_slot, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int w = warp_sums[lane];
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
-    }
-    warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+    if (lane < NT / 32) warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
     if (lane == 31) *total_slot = wi;
   }
   __syncthreads();
-  const int excl = warp_sums[warp] + incl - v;
+  const uint32_t excl = warp_sums[warp] + incl - v;
   total = *total_slot;
   __syncthreads();
   return excl;
@@ -88,23 +65,26 @@ __host__ __device__ inline int stage_words(int n, int n_wide) {
   return n_wide <= kSelStageWords && n_wide > n ? n_wide : n;
 }
 
-template <int PER>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores, int n, int n_keep,
+template <int PER, int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const float* __restrict__ scores, int n, int n_keep,
                                                              int32_t* __restrict__ sigma, int hpg, int head_dim,
                                                              int n_wide, int32_t* __restrict__ sigma_wide) {
   pdl_wait();
-  // staging words for scores in / sigma out (and sigma_wide when it fits), then [n] kept flags
+  // staging words for scores in / sigma out (and sigma_wide when it fits), then, for the
+  // query-side expansion, kbu[n]: the kept units before each unit
   extern __shared__ uint32_t sbuf[];
-  uint8_t* keep = reinterpret_cast<uint8_t*>(sbuf + stage_words(n, n_wide));
+  uint16_t* kbu = reinterpret_cast<uint16_t*>(sbuf + stage_words(n, n_wide));
   __shared__ uint32_t s_or[32], s_and[32];
   __shared__ int warp_sums[32];
+  __shared__ uint32_t warp_sums_u[32];
   __shared__ int hist[4][256];  // one histogram per radix pass, all zeroed before the first
-  __shared__ int scan_total;
+  __shared__ int sel_state[2];
+  __shared__ uint32_t scan_total;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per = (n + kSelThreads - 1) / kSelThreads;  // <= PER
+  const int per = (n + NT - 1) / NT;  // <= PER
   const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
-  for (int i = threadIdx.x; i < n; i += kSelThreads) sbuf[i] = __float_as_uint(scores[i]);
-  for (int i = threadIdx.x; i < 4 * 256; i += kSelThreads) (&hist[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < n; i += NT) sbuf[i] = __float_as_uint(scores[i]);
+  for (int i = threadIdx.x; i < 4 * 256; i += NT) (&hist[0][0])[i] = 0;
   __syncthreads();
 
   uint32_t key[PER];
@@ -125,8 +105,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     s_and[warp] = kand;
   }
   __syncthreads();
-  const uint32_t bor = __reduce_or_sync(0xffffffffu, s_or[lane]);
-  const uint32_t band = __reduce_and_sync(0xffffffffu, s_and[lane]);
+  const uint32_t bor = __reduce_or_sync(0xffffffffu, lane < NT / 32 ? s_or[lane] : 0u);
+  const uint32_t band = __reduce_and_sync(0xffffffffu, lane < NT / 32 ? s_and[lane] : 0xffffffffu);
   // The n-th largest key K* by radix selection, 8 bits per pass from the byte holding the highest
   // bit in which two keys differ (every key shares the bits above it): per pass, a 256-bin
   // histogram of the next byte over the keys that match the bytes chosen so far; the chosen byte is
@@ -146,36 +126,43 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
       for (int j = 0; j < PER; ++j)
         if (i0 + j < i1 && (key[j] & tmask) == T) atomicAdd(&hist[pass][(key[j] >> shift) & 255u], 1);
       __syncthreads();
-      // every warp reads the finished histogram and picks the same byte (no second barrier):
-      // lane l holds bins 255 - 8 l .. 248 - 8 l (descending), counts from the top
-      int c[8], tot = 0;
+      if (warp == 0) {
+        // lane l holds bins 255 - 8 l .. 248 - 8 l (descending), counts from the top; one warp
+        // picks (all 32 warps doing it cost more issue slots than the extra barrier)
+        int c[8], tot = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = hist[pass][255 - 8 * lane - e];
-        tot += c[e];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += nb;
-      }
-      int above = incl - tot;  // matching keys whose byte lies above this lane's bins
-      int pick = -1, above_pick = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (pick < 0 && above < need && above + c[e] >= need) {
-          pick = 255 - 8 * lane - e;
-          above_pick = above;
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[pass][255 - 8 * lane - e];
+          tot += c[e];
         }
-        above += c[e];
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += nb;
+        }
+        int above = incl - tot;  // matching keys whose byte lies above this lane's bins
+        int pick = -1, above_pick = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (pick < 0 && above < need && above + c[e] >= need) {
+            pick = 255 - 8 * lane - e;
+            above_pick = above;
+          }
+          above += c[e];
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, pick >= 0);  // one lane holds the crossing
+        const int src = who ? __ffs(who) - 1 : 0;
+        pick = __shfl_sync(0xffffffffu, pick, src);
+        above_pick = __shfl_sync(0xffffffffu, above_pick, src);
+        if (lane == 0) {
+          sel_state[pass & 1] = pick < 0 ? 0 : pick;  // two slots: the next pass writes the other
+          warp_sums[pass & 1] = above_pick;
+        }
       }
-      const unsigned who = __ballot_sync(0xffffffffu, pick >= 0);  // one lane holds the crossing
-      const int src = who ? __ffs(who) - 1 : 0;
-      pick = __shfl_sync(0xffffffffu, pick, src);
-      above_pick = __shfl_sync(0xffffffffu, above_pick, src);
-      T |= (uint32_t)(pick < 0 ? 0 : pick) << shift;
-      need -= above_pick;
+      __syncthreads();
+      T |= (uint32_t)sel_state[pass & 1] << shift;
+      need -= warp_sums[pass & 1];
       tmask |= 255u << shift;
     }
   }
@@ -188,11 +175,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     gt += valid && key[j] > T ? 1 : 0;
     n_eq += valid && key[j] == T ? 1 : 0;
   }
-  int total = 0;
-  const int packed = block_exclusive_scan_total(gt | (n_eq << 16), warp_sums, &scan_total, total);
-  const int take_eq = n_keep - (total & 0xffff);
-  int eq_rank = packed >> 16;
-  int kept_before = (packed & 0xffff) + min(eq_rank, take_eq);
+  // (unsigned: the tied count reaches 40960 << 16, past the int range)
+  uint32_t total = 0;
+  const uint32_t packed = block_exclusive_scan_total<NT>((uint32_t)gt | ((uint32_t)n_eq << 16), warp_sums_u, &scan_total,
+                                                     total);
+  const int take_eq = n_keep - (int)(total & 0xffffu);
+  int eq_rank = (int)(packed >> 16);
+  int kept_before = (int)(packed & 0xffffu) + min(eq_rank, take_eq);
   uint64_t kmask = 0;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
@@ -208,6 +197,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     const int i = i0 + j;
     if (i >= i1) break;
     const bool kp = (kmask >> j) & 1ull;
+    if (wide) kbu[i] = (uint16_t)kept_before;
     // exactly n_keep keys are kept, so both ranges stay inside [0, n); the checks only
     // keep a broken invariant from writing past them
     if (kp) {
@@ -217,49 +207,52 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
       if (n_keep + drop_before < n) sbuf[n_keep + drop_before] = (uint32_t)i;
       ++drop_before;
     }
-    if (wide) keep[i] = kp;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kSelThreads) sigma[i] = (int32_t)sbuf[i];
+  for (int i = threadIdx.x; i < n; i += NT) sigma[i] = (int32_t)sbuf[i];
   if (!wide) return;
   __syncthreads();
-  // Query-side expansion: channel c = h * head_dim + d follows unit (h / hpg) * head_dim + d.
+  // Query-side expansion: channel (h, d) = h * head_dim + d follows unit u = (h / hpg) * head_dim
+  // + d. Kept query channels are ordered by head, then d; with kb(u) the kept units before u
+  // (kbu) and, for the KV head g of u, kg = kb(g * head_dim) and cnt = its kept units, channel
+  // (g * hpg + j, d) of a kept unit goes to hpg kg + j cnt + (kb(u) - kg), and of a dropped one to
+  // n_keep hpg + hpg (g hd - kg) + j (hd - cnt) + ((u - kb(u)) - (g hd - kg)): each unit places its
+  // hpg channels directly, no second scan.
   const int n_keep_w = n_keep * hpg;
   const bool staged = n_wide <= kSelStageWords;
-  const int perw = (n_wide + kSelThreads - 1) / kSelThreads;
-  const int w0 = min(n_wide, (int)threadIdx.x * perw), w1 = min(n_wide, w0 + perw);
-  auto unit_of = [&](int c) { return (c / head_dim / hpg) * head_dim + c % head_dim; };
-  int nk = 0;
-  for (int c = w0; c < w1; ++c) nk += keep[unit_of(c)];
-  int kb = block_exclusive_scan(nk, warp_sums);
-  int db = w0 - kb;
   uint32_t* out = staged ? sbuf : reinterpret_cast<uint32_t*>(sigma_wide);
-  for (int c = w0; c < w1; ++c) {
-    if (keep[unit_of(c)]) {
-      if (kb < n_keep_w) out[kb] = (uint32_t)c;
-      ++kb;
-    } else {
-      if (n_keep_w + db < n_wide) out[n_keep_w + db] = (uint32_t)c;
-      ++db;
+  for (int u = threadIdx.x; u < n; u += NT) {
+    const int g = u / head_dim, gb = g * head_dim;
+    const int kg = kbu[gb];
+    const int kend = gb + head_dim < n ? (int)kbu[gb + head_dim] : n_keep;
+    const int cnt = kend - kg;
+    const int ku = kbu[u];
+    const bool kept = (u + 1 < n ? (int)kbu[u + 1] : n_keep) > ku;
+    const int c0 = g * hpg * head_dim + (u - gb);
+    for (int j = 0; j < hpg; ++j) {
+      const int pos = kept ? hpg * kg + j * cnt + (ku - kg)
+                           : n_keep_w + hpg * (gb - kg) + j * (head_dim - cnt) + ((u - ku) - (gb - kg));
+      if (pos >= 0 && pos < n_wide) out[pos] = (uint32_t)(c0 + j * head_dim);
     }
   }
   if (!staged) return;
   __syncthreads();
-  for (int c = threadIdx.x; c < n_wide; c += kSelThreads) sigma_wide[c] = (int32_t)sbuf[c];
+  for (int c = threadIdx.x; c < n_wide; c += NT) sigma_wide[c] = (int32_t)sbuf[c];
 }
 
-template <int PER>
+template <int PER, int NT>
 void launch_select(const float* scores, int n, int n_keep, int32_t* sigma, int hpg, int head_dim, int n_wide,
                    int32_t* sigma_wide, cudaStream_t s) {
   if (!sigma_wide) n_wide = 0;
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(select_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kSelStageWords * 4 + kSelMaxN + 16);
+    cudaFuncSetAttribute(select_kernel<PER, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kSelStageWords * 4 + kSelMaxNWide * 2 + 16);
     attr = true;
   }
-  const size_t smem = (size_t)stage_words(n, sigma_wide ? n_wide : 0) * 4 + (sigma_wide ? ((size_t)n + 15) / 16 * 16 : 0);
-  launch_kernel(select_kernel<PER>, 1, kSelThreads, smem, s, scores, n, n_keep, sigma, hpg, head_dim, n_wide,
+  const size_t smem =
+      (size_t)stage_words(n, sigma_wide ? n_wide : 0) * 4 + (sigma_wide ? ((size_t)n * 2 + 15) / 16 * 16 : 0);
+  launch_kernel(select_kernel<PER, NT>, 1, NT, smem, s, scores, n, n_keep, sigma, hpg, head_dim, n_wide,
                 sigma_wide);
 }
 
@@ -327,17 +320,20 @@ __global__ void __launch_bounds__(kSelThreads) select_heads_kernel(const float* 
 int select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma, int heads_per_group, int head_dim,
                     int64_t n_wide, int32_t* sigma_wide, int64_t* n_keep_wide_out, cudaStream_t s) {
   if (n <= 0 || n > kSelMaxN || n_keep < 1 || n_keep > n) return 1;
-  if (sigma_wide && (heads_per_group <= 0 || head_dim <= 0 || n % head_dim || n_wide != n * heads_per_group))
+  if (sigma_wide && (heads_per_group <= 0 || head_dim <= 0 || n % head_dim || n_wide != n * heads_per_group ||
+                     n > kSelMaxNWide))
     return 1;
   const int hpg = sigma_wide ? heads_per_group : 0;
-  if (n <= kSelThreads)
-    launch_select<1>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
-  else if (n <= 4 * kSelThreads)
-    launch_select<4>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
-  else if (n <= 16 * kSelThreads)
-    launch_select<16>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  // Fewer, fuller threads for small sets: each block-wide phase (barrier, scan) then involves
+  // fewer warps.
+  if (n <= 1024)
+    launch_select<4, 256>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  else if (n <= 4096)
+    launch_select<8, 512>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+  else if (n <= 16384)
+    launch_select<16, 1024>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
   else
-    launch_select<40>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
+    launch_select<40, 1024>(scores, (int)n, (int)n_keep, sigma, hpg, head_dim, (int)n_wide, sigma_wide, s);
   if (n_keep_wide_out) *n_keep_wide_out = sigma_wide ? n_keep * heads_per_group : 0;
   if (launch_failed("sl_select")) return 5;
   note_launch();

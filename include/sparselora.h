@@ -229,7 +229,7 @@ SL_API sl_status sl_svd_scores_from_partials(sl_criterion crit, sl_dtype dtype, 
  * the n scores are KV units (g, d) with d < head_dim, and sigma_wide[n *
  * heads_per_group] receives the matching query-side set: channel (h, d) is kept iff
  * unit (h / heads_per_group, d) is (the kept count is n_keep * heads_per_group).
- * n <= 40960. */
+ * n <= 40960; n <= 16384 with the query-side set. */
 SL_API sl_status sl_select_channels(const float* scores, int64_t n, int64_t n_keep, int32_t* sigma,
                              int32_t heads_per_group, int32_t head_dim, int32_t* sigma_wide, sl_stream stream);
 

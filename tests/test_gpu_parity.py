@@ -269,6 +269,44 @@ def test_select_continuous_scores_bit_exact(n, n_keep):
     np.testing.assert_array_equal(got[n_keep:], oracle.complement(want, n))
 
 
+def test_select_all_equal_scores_at_the_size_limit():
+    """Every score equal at n = 40960: the threshold is that score and the tied count (40960)
+    exceeds 2^15, which a signed 16-bit half of a packed count would overflow; the lowest
+    n_keep indices are kept."""
+    n, n_keep = 40960, 20000
+    sc = torch.full((n,), 1.5, device=DEV)
+    sig = torch.empty(n, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(sc, n_keep, sig)
+    np.testing.assert_array_equal(sig.cpu().numpy(), np.arange(n))
+    s = np.full(n, 2.0, np.float32)
+    s[:5] = 3.0  # five above the tie, then 39955 tied
+    sig2 = torch.empty(n, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(torch.tensor(s, device=DEV), 35000, sig2)
+    want = oracle.select_top(s.astype(np.float64), 35000)
+    np.testing.assert_array_equal(sig2.cpu().numpy()[:35000], want)
+    np.testing.assert_array_equal(sig2.cpu().numpy()[35000:], oracle.complement(want, n))
+
+
+@pytest.mark.parametrize("hkv,hd,hpg,keep", [(8, 128, 4, 0.5), (8, 128, 4, 0.05), (2, 64, 8, 0.7), (40, 128, 1, 0.4),
+                                              (3, 96, 3, 0.33), (5, 8, 2, 1.0)])
+def test_select_query_side_set_bit_exact(hkv, hd, hpg, keep):
+    """The query-side set of a KV-unit selection (GQA expansion) against the oracle's expansion:
+    query channel (h, d) kept iff unit (h / hpg, d) is; kept then dropped, each ascending."""
+    n = hkv * hd
+    n_keep = max(1, int(round(keep * n)))
+    rng = np.random.default_rng(n + hpg)
+    s = (1.0 + rng.standard_normal(n) ** 2).astype(np.float32)
+    sig = torch.empty(n, dtype=torch.int32, device=DEV)
+    wide = torch.empty(n * hpg, dtype=torch.int32, device=DEV)
+    B.sl_select_channels(torch.tensor(s, device=DEV), n_keep, sig, hpg, hd, wide)
+    units = oracle.select_top(s.astype(np.float64), n_keep)
+    np.testing.assert_array_equal(sig.cpu().numpy()[:n_keep], units)
+    kept_q = oracle.expand_units(units, hkv * hpg, hkv, hd)
+    got = wide.cpu().numpy()
+    np.testing.assert_array_equal(got[: len(kept_q)], kept_q)
+    np.testing.assert_array_equal(got[len(kept_q):], oracle.complement(kept_q, n * hpg))
+
+
 def test_select_and_estimate_are_deterministic():
     T, C, D, F, k = 424, 300, 512, 1000, 8
     p = ffn_problem(T, C, D, F, 32, k, seed=11)
