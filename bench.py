@@ -195,7 +195,7 @@ def make_layer(ratio, seed_w, seed_x, device, dense=False, dp=None, cfgs=None, k
     C = int(da["ctx_mask"].sum())
     attn = blocks.AttnProjBlock(da["q"], da["k"], da["v"], da["o"], da["lora_q"], da["lora_k"], da["lora_v"],
                                 da["lora_o"], ac.lora_scale, ac.k, ac.n_q_heads, ac.n_kv_heads, ac.head_dim,
-                                ac.n_tok, C, ratio, device, dense=dense, dp=dp, kept_rows=kept_rows)
+                                ac.n_tok, C, ratio, device, dense=dense, dp=dp, kept_rows=kept_rows, io_layout="sigma")
     ffn = blocks.FFNBlock(df["gate"], df["up"], df["down"], df["lora_gate"], df["lora_up"], df["lora_down"],
                           fc.lora_scale, fc.k, fc.n_tok, C, ratio, device, dense=dense, dp=dp, kept_rows=kept_rows)
     if seed_x != seed_w:  # per-rank batches

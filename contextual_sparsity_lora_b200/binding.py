@@ -32,7 +32,7 @@ EXPORTED = ("sl_status_string", "sl_version", "sl_keep_count", "sl_workspace_ini
             "sl_svd_scores_from_partials", "sl_select_heads", "sl_wanda_scores", "sl_rmsnorm_fwd", "sl_rmsnorm_bwd",
             "sl_add_rows", "sl_adamw_step", "sl_gather_rows_batch", "sl_set_pair_tile_rows",
             "sl_debug_bounds_enabled", "sl_read_debug_flag", "sl_attention_fwd", "sl_attention_bwd",
-            "sl_lora_fwd_estimate", "sl_svd_scores_from_z")
+            "sl_lora_fwd_estimate", "sl_svd_scores_from_z", "sl_permute_rows_sigma")
 
 
 class SlWorkspaceC(ctypes.Structure):
@@ -133,6 +133,8 @@ def load(path):
     L.sl_profile_enable.argtypes = [c_int32]
     L.sl_profile_read.argtypes = [POINTER(c_int64), POINTER(c_int64), POINTER(c_double)]
     L.sl_permute_rows.argtypes = [P, c_int64, c_int64, P, c_int64, c_int64, P, c_int64, P]
+    L.sl_permute_rows_sigma.argtypes = [P, c_int64, c_int64, P, c_int64, c_int64, P, c_int64, c_int32, P, c_int64,
+                                        P]
     L.sl_gather_rows_batch.argtypes = [c_int32, P, P, P, P, P, P, P, P, P]
     L.sl_debug_bounds_enabled.restype = c_int32
     L.sl_lora_fwd_estimate.argtypes = [c_int32, POINTER(SlLinearC), P, c_int64, c_int64, c_int64, P, P, c_int64,
@@ -375,6 +377,16 @@ def sl_permute_rows(src, perm, dst):
     """dst[i, :] = src[perm[i], :] for i < perm.numel() (src may have more rows than dst)."""
     _check("sl_permute_rows", lib().sl_permute_rows(_ptr(src), src.stride(0), src.shape[0], _ptr(perm), perm.numel(),
                                                     src.shape[1], _ptr(dst), dst.stride(0), _stream()))
+
+
+def sl_permute_rows_sigma(src, perm, dst, sigma, n_ctx, to_sigma):
+    """Row permutation with the sigma-layout channel order on context rows: to_sigma, destination
+    rows i < n_ctx get dst[i, p] = src[perm[i], sigma[p]]; else source rows perm[i] < n_ctx are in
+    the sigma layout and dst[i, sigma[p]] = src[perm[i], p]; other rows are copied."""
+    _check("sl_permute_rows_sigma",
+           lib().sl_permute_rows_sigma(_ptr(src), src.stride(0), src.shape[0], _ptr(perm), perm.numel(), src.shape[1],
+                                       _ptr(sigma), int(n_ctx), 1 if to_sigma else 0, _ptr(dst), dst.stride(0),
+                                       _stream()))
 
 
 def sl_gather_rows_batch(srcs, perms, dsts):

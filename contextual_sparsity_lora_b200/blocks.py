@@ -337,18 +337,26 @@ class AttnProjBlock:
 
     def __init__(self, q, k, v, o, lora_q, lora_k, lora_v, lora_o, lora_scale, est_k, n_q_heads, n_kv_heads,
                  head_dim, n_tok, n_ctx, ratio, device="cuda", dense=False, dp=None, qk_criterion="channel",
-                 vo_criterion="l2", seed=0, kept_rows="compact"):
+                 vo_criterion="l2", seed=0, kept_rows="compact", io_layout="natural"):
         """qk_criterion: "channel" (the method's QK norm per KV channel), or the criterion
         ablation's "head" (whole KV heads by the summed QK norm) and "random"; vo_criterion:
         "l2" (the method's) or "random" (uniform scores from a generator seeded with `seed`).
         kept_rows: "compact" (a compacted copy per step, shared by forward and backward; the
         faster form on B200) or "gather" (the sliced products read the kept weight rows in place
-        through sigma)."""
+        through sigma). io_layout: the channel order of the context rows of q, k, v (outputs),
+        x_o (input), dx_o (output) and dq, dk, dv (inputs): "natural", or "sigma" (channel
+        sigma[p] in column p, the order the sliced products read and write, so no column scatter
+        or gather runs; sl_permute_rows_sigma converts while it reorders the rows, as the decoder
+        layer does)."""
         if qk_criterion not in ("channel", "head", "random") or vo_criterion not in ("l2", "random"):
             raise ValueError(f"criteria {qk_criterion!r}, {vo_criterion!r}")
         if kept_rows not in KEPT_ROWS:
             raise ValueError(f"kept_rows {kept_rows!r} not in {KEPT_ROWS}")
+        if io_layout not in ("natural", "sigma"):
+            raise ValueError(f"io_layout {io_layout!r}")
         self.kept_rows = kept_rows
+        self.io_layout = io_layout
+        self.lay = B.SL_LAYOUT_SIGMA if io_layout == "sigma" else B.SL_LAYOUT_NATURAL
         if (qk_criterion, vo_criterion) != ("channel", "l2") and dp is not None and dp.active:
             raise ValueError("the ablation criteria run on one rank")
         self.qk_criterion, self.vo_criterion = qk_criterion, vo_criterion
@@ -553,55 +561,78 @@ class AttnProjBlock:
         lq, lk, lv, lo = (self.lin[n] for n in "qkvo")
         sel = not self.dense and (C > 0 or self.dp is not None)
 
-        def lora_fwd(ws):  # x A^T for q, k, v and x_o A^T for o: independent of the selection
+        def o_lora(ws):
+            B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o, in_layout=self.lay,
+                              in_ch=self.ch["o"])
+
+        # x_o A^T does not depend on the selection in the natural layout; in the sigma layout x_o's
+        # context columns follow the v/o set, so it runs after the selection (beside the q/k/v
+        # products when the block runs chains concurrently)
+        early_o = self.lay == B.SL_LAYOUT_NATURAL or not sel
+
+        def qkv_lora(ws):
             B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
-            B.sl_lora_fwd_bwd(ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
 
         if sel and self.fold:
-            if self.concurrent:
-                with self.side.fork():  # x_o A^T does not depend on the selection
-                    B.sl_lora_fwd_bwd(self.side.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+            if self.concurrent and early_o:
+                with self.side.fork():
+                    o_lora(self.side.ws)
                 o_done = self.side.mark()
                 self._estimate_fused(x, self.ws)
                 self._choose_and_compact()
                 torch.cuda.current_stream().wait_event(o_done)
             else:
-                B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+                if early_o:
+                    o_lora(self.ws)
                 self._estimate_fused(x, self.ws)
                 self._choose_and_compact()
         elif sel and self.concurrent:
             with self.side.fork():
-                lora_fwd(self.side.ws)
+                qkv_lora(self.side.ws)
+                if early_o:
+                    o_lora(self.side.ws)
             self.select(x)
             self.side.join()
         else:
             if sel:
                 self.select(x)
-            lora_fwd(self.ws)
+            qkv_lora(self.ws)
+            if early_o:
+                o_lora(self.ws)
+        late_side = not early_o and self.concurrent
+        if late_side:
+            with self.side.fork():
+                o_lora(self.side.ws)
+        elif not early_o:
+            o_lora(self.ws)
         B.sl_sparse_linear_fwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, x, C,
-                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=B.SL_LAYOUT_NATURAL)
+                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=self.lay)
+        if late_side:
+            self.side.join()
         B.sl_sparse_linear_fwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, x_o, C, self.xa_s_o, [self.y],
-                               in_layout=B.SL_LAYOUT_NATURAL)
+                               in_layout=self.lay)
         return self.y
 
     def _o_backward(self, ws, dy):
         """o's LoRA gradients and its input gradient dx_o."""
         lo = self.lin["o"]
         C = self.n_ctx
-        B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, dy=[dy], dya=[self.dya["o"][0]],
-                          dya_s=[self.dya["o"][1]], dA=[self.dA["o"]], dB=[self.dB["o"]])
+        B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lo], self.x_o, C, self.xa_s_o, in_layout=self.lay, in_ch=self.ch["o"],
+                          dy=[dy], dya=[self.dya["o"][0]], dya_s=[self.dya["o"][1]], dA=[self.dA["o"]],
+                          dB=[self.dB["o"]])
         B.sl_sparse_linear_bwd(ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, [dy], C, [self.dya["o"][1]],
-                               dx=self.dx_o, out_layout=B.SL_LAYOUT_NATURAL)
+                               dx=self.dx_o, out_layout=self.lay)
 
     def _qkv_backward(self, ws, dq, dk, dv):
         """q, k, v LoRA gradients and dx."""
         lq, lk, lv = (self.lin[n] for n in "qkv")
         C = self.n_ctx
         B.sl_lora_fwd_bwd(ws, B.SL_LORA_BWD, [lq, lk, lv], self.x, C, self.xa_s_qkv, dy=[dq, dk, dv],
+                          out_layout=self.lay, out_ch=[self.ch[n] for n in "qkv"],
                           dya=[self.dya[n][0] for n in "qkv"], dya_s=[self.dya[n][1] for n in "qkv"],
                           dA=[self.dA[n] for n in "qkv"], dB=[self.dB[n] for n in "qkv"])
         B.sl_sparse_linear_bwd(ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, [dq, dk, dv], C,
-                               [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=B.SL_LAYOUT_NATURAL)
+                               [self.dya[n][1] for n in "qkv"], dx=self.dx, in_layout=self.lay)
 
     def backward(self, dy, dq, dk, dv):
         if self.concurrent:  # the o chain and the q/k/v chain are independent
@@ -618,7 +649,7 @@ class AttnProjBlock:
     # q/k/v and o: forward_qkv, forward_o, then backward_o, backward_qkv
 
     def forward_qkv(self, x):
-        """The selection on x's context rows and q, k, v (natural column layout)."""
+        """The selection on x's context rows and q, k, v (context rows in the block's io_layout)."""
         C = self.n_ctx
         self.x = x
         lq, lk, lv = (self.lin[n] for n in "qkv")
@@ -636,7 +667,7 @@ class AttnProjBlock:
                 self.select(x)
             B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lq, lk, lv], x, C, self.xa_s_qkv, xa=self.xa_qkv)
         B.sl_sparse_linear_fwd(self.ws, [lq, lk, lv], [self.ch[n] for n in "qkv"], B.SL_EPI_NONE, x, C,
-                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=B.SL_LAYOUT_NATURAL)
+                               self.xa_s_qkv, [self.q, self.kk, self.vv], out_layout=self.lay)
         return self.q, self.kk, self.vv
 
     def forward_o(self, x_o):
@@ -644,9 +675,10 @@ class AttnProjBlock:
         C = self.n_ctx
         self.x_o = x_o
         lo = self.lin["o"]
-        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o)
+        B.sl_lora_fwd_bwd(self.ws, B.SL_LORA_FWD, [lo], x_o, C, self.xa_s_o, xa=self.xa_o, in_layout=self.lay,
+                          in_ch=self.ch["o"])
         B.sl_sparse_linear_fwd(self.ws, [lo], [self.ch["o"]], B.SL_EPI_NONE, x_o, C, self.xa_s_o, [self.y],
-                               in_layout=B.SL_LAYOUT_NATURAL)
+                               in_layout=self.lay)
         return self.y
 
     def backward_o(self, dy):
@@ -656,6 +688,13 @@ class AttnProjBlock:
     def backward_qkv(self, dq, dk, dv):
         self._qkv_backward(self.ws, dq, dk, dv)
         return self.dx
+
+    def sigma_of(self, name):
+        """The channel set in force for projection `name` ("q", "k", "v", "o"): its sigma tensor
+        (the identity in dense steps)."""
+        if self.dense:
+            return self._ids["q" if name in "qo" else "kv"]
+        return {"q": self.sig_q, "k": self.sig_k, "v": self.sig_v, "o": self.sig_o}[name]
 
     def read_device_flag(self) -> int:
         """Device error word of both workspaces (0: no device-side timeout); synchronises."""

@@ -1295,6 +1295,19 @@ sl_status sl_permute_rows(const void* src, int64_t ld_src, int64_t src_rows, con
       gather_rows_bf16(src, ld_src, src_rows, perm, n_rows, n_cols, dst, ld_dst, 0, aux_debug_word(), cs(stream)));
 }
 
+sl_status sl_permute_rows_sigma(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm,
+                                int64_t n_rows, int64_t n_cols, const int32_t* sigma, int64_t n_ctx, int32_t to_sigma,
+                                void* dst, int64_t ld_dst, sl_stream stream) {
+  if (!src || !perm || !sigma || !dst) return SL_ERR_INVALID_ARG;
+  if (src_rows <= 0 || n_rows <= 0 || n_cols <= 0 || n_cols > kPermMaxCols || n_ctx < 0 || ld_src < n_cols ||
+      ld_dst < n_cols)
+    return SL_ERR_SHAPE;
+  if (n_cols % 8 || ld_src % 8 || ld_dst % 8 || !al16(src) || !al16(dst)) return SL_ERR_ALIGNMENT;
+  const int rc = permute_rows_sigma(src, ld_src, src_rows, perm, n_rows, n_cols, sigma, n_ctx, to_sigma ? 1 : 0, dst,
+                                    ld_dst, aux_debug_word(), cs(stream));
+  return rc == 2 ? SL_ERR_ALIGNMENT : from_kernel(rc);
+}
+
 sl_status sl_gather_rows_batch(int32_t n, const void* const* src, const int64_t* ld_src, const int64_t* src_rows,
                                const int32_t* const* perm, const int64_t* n_rows, const int64_t* n_cols,
                                void* const* dst, const int64_t* ld_dst, sl_stream stream) {

@@ -4,6 +4,8 @@
 // in 16-byte vectors where the layout allows it.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "sl_internal.h"
 
 namespace sl {
@@ -65,6 +67,60 @@ __global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t 
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
     const int64_t c = c0 + i, r = r0 + threadIdx.x;
     if (r < rows && c < cols) dst[c * ld_dst + r] = tile[threadIdx.x][i];
+  }
+}
+
+// Row permutation that also converts the channel order of context rows to or from the sigma
+// layout (context rows store channel sigma[p] in column p), one CTA per row in a grid-stride
+// loop: dst[i, :] = src[perm[i], :], except
+//   to_sigma, destination row i < n_ctx:       dst[i, p] = src[perm[i], sigma[p]]
+//   from the sigma layout, source row < n_ctx: dst[i, sigma[p]] = src[perm[i], p]
+// A context row goes through shared memory, so the global read and write stay contiguous
+// 16-byte vectors and only the shared-memory accesses follow sigma.
+constexpr int kPermThreads = 256;
+__global__ void __launch_bounds__(kPermThreads)
+    permute_rows_sigma_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t src_rows,
+                              const int32_t* __restrict__ perm, int64_t n_rows, int n_cols,
+                              const int32_t* __restrict__ sigma, int64_t n_ctx, int to_sigma,
+                              __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int* err) {
+  extern __shared__ __align__(16) __nv_bfloat16 rowbuf[];  // two rows of n_cols
+  pdl_wait();
+  __nv_bfloat16* a = rowbuf;
+  __nv_bfloat16* b = rowbuf + n_cols;
+  const int nv = n_cols / 8;
+  for (int64_t i = blockIdx.x; i < n_rows; i += gridDim.x) {
+    const int64_t sr = perm[i];
+    if (!index_ok(sr, src_rows, err, DEV_BAD_GATHER_ROW)) continue;  // the whole CTA skips the row
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + sr * ld_src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + i * ld_dst);
+    const bool ctx = to_sigma ? i < n_ctx : sr < n_ctx;
+    if (!ctx) {
+      for (int c = threadIdx.x; c < nv; c += kPermThreads) d4[c] = __ldg(s4 + c);
+      continue;
+    }
+    for (int c = threadIdx.x; c < nv; c += kPermThreads) reinterpret_cast<uint4*>(a)[c] = __ldg(s4 + c);
+    __syncthreads();
+    if (to_sigma) {
+      for (int v = threadIdx.x; v < nv; v += kPermThreads) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c0 = sigma[8 * v + 2 * k], c1 = sigma[8 * v + 2 * k + 1];
+          const __nv_bfloat16 lo = index_ok(c0, n_cols, err, DEV_BAD_GATHER_COL) ? a[c0] : __float2bfloat16(0.f);
+          const __nv_bfloat16 hi = index_ok(c1, n_cols, err, DEV_BAD_GATHER_COL) ? a[c1] : __float2bfloat16(0.f);
+          w[k] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        }
+        d4[v] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      for (int p = threadIdx.x; p < n_cols; p += kPermThreads) {
+        const int c = sigma[p];
+        if (index_ok(c, n_cols, err, DEV_BAD_GATHER_COL)) b[c] = a[p];
+      }
+      __syncthreads();
+      for (int c = threadIdx.x; c < nv; c += kPermThreads) d4[c] = reinterpret_cast<const uint4*>(b)[c];
+    }
+    __syncthreads();  // the row buffers are refilled for the next row
   }
 }
 
@@ -157,6 +213,32 @@ int* aux_debug_word() {
 #else
 int* aux_debug_word() { return nullptr; }
 #endif
+
+int permute_rows_sigma(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm, int64_t n_rows,
+                       int64_t n_cols, const int32_t* sigma, int64_t n_ctx, int to_sigma, void* dst, int64_t ld_dst,
+                       int* err, cudaStream_t s) {
+  if (n_rows <= 0) return 0;
+  if (n_cols <= 0 || n_cols > kPermMaxCols || n_cols % 8 || ld_src % 8 || ld_dst % 8 ||
+      (reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15))
+    return 2;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(permute_rows_sigma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * kPermMaxCols * 2) != cudaSuccess)
+      return 5;
+    attr = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = (unsigned)std::min<int64_t>(n_rows, (int64_t)sms * 8);
+  launch_kernel(permute_rows_sigma_kernel, grid, kPermThreads, (size_t)n_cols * 4, s,
+                static_cast<const __nv_bfloat16*>(src), ld_src, src_rows, perm, n_rows, (int)n_cols, sigma, n_ctx,
+                to_sigma, static_cast<__nv_bfloat16*>(dst), ld_dst, err);
+  if (launch_failed("sl_aux")) return 5;
+  note_launch();
+  return 0;
+}
 
 int add_f32(float* dst, const float* src, int64_t n, cudaStream_t s) {
   if (n <= 0) return 0;

@@ -266,6 +266,12 @@ struct GatherBatch {
   int launch(int* err, cudaStream_t s);  // one launch for every job added, then empty
 };
 // dst[t, j] = src[t, idx[j]] for t < n_rows, j < n_idx; src_cols: columns of src (debug checks).
+// Row permutation with the sigma-layout channel permutation of context rows (sl_permute_rows_sigma).
+// Returns 2 for a shape or alignment the kernel does not take.
+constexpr int64_t kPermMaxCols = 16384;
+int permute_rows_sigma(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm, int64_t n_rows,
+                       int64_t n_cols, const int32_t* sigma, int64_t n_ctx, int to_sigma, void* dst, int64_t ld_dst,
+                       int* err, cudaStream_t s);
 int gather_cols_bf16(const void* src, int64_t ld_src, int64_t src_cols, int64_t n_rows, const int32_t* idx,
                      int64_t n_idx, void* dst, int64_t ld_dst, int* err, cudaStream_t s);
 int transpose_bf16(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,

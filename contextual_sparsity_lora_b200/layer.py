@@ -9,7 +9,9 @@ computed with the sparse projections).
 RMSNorm, the residual adds, every projection and the causal grouped-query attention core
 (sl_attention_fwd / sl_attention_bwd, tcgen05 kernels) run in libsparselora's kernels. Rows are
 in context-first order like the blocks' (sl_permute_rows moves q, k, v to sequence order for the
-attention core and its output back). No rotary positional encoding: the pages do not say how it
+attention core and its output back; when the attention block keeps its interfaces in the sigma
+layout, sl_permute_rows_sigma also restores or applies the channel order of the context rows in
+the same pass). No rotary positional encoding: the pages do not say how it
 meets channel sparsity (a rotation mixes channel pairs that the selection may split)."""
 from __future__ import annotations
 
@@ -52,21 +54,32 @@ class DecoderLayer:
         self.dx2, self.dx = e(T, D), e(T, D)
         self.ws = B.Workspace(dev)  # the attention core's scratch (the dq accumulator) and error word
 
-    def _to_seq(self, src, dst):
-        B.sl_permute_rows(src, self.inv, dst)
+    def _to_seq(self, src, dst, name):
+        """Context-first rows -> sequence order; with the block's sigma layout, the context rows'
+        channels also return to natural order (projection `name`'s channel set)."""
+        at = self.attn
+        if at.io_layout == "sigma":
+            B.sl_permute_rows_sigma(src, self.inv, dst, at.sigma_of(name), at.n_ctx, to_sigma=False)
+        else:
+            B.sl_permute_rows(src, self.inv, dst)
 
-    def _to_cf(self, src, dst):
-        B.sl_permute_rows(src, self.perm, dst)
+    def _to_cf(self, src, dst, name):
+        """Sequence order -> context-first rows (in the block's sigma layout when it uses one)."""
+        at = self.attn
+        if at.io_layout == "sigma":
+            B.sl_permute_rows_sigma(src, self.perm, dst, at.sigma_of(name), at.n_ctx, to_sigma=True)
+        else:
+            B.sl_permute_rows(src, self.perm, dst)
 
     def forward(self, x):
         at = self.attn
         B.sl_rmsnorm_fwd(x, self.g1, self.eps, self.h1, self.rstd1)
         q, k, v = at.forward_qkv(self.h1)
-        for src, dst in ((q, self.q_nat), (k, self.k_nat), (v, self.v_nat)):
-            self._to_seq(src, dst)
+        for src, dst, name in ((q, self.q_nat, "q"), (k, self.k_nat, "k"), (v, self.v_nat, "v")):
+            self._to_seq(src, dst, name)
         B.sl_attention_fwd(self.ws, self.q_nat, self.k_nat, self.v_nat, self.n_seq, at.hq, at.hkv, at.hd, self.a_nat,
                            self.lse)
-        self._to_cf(self.a_nat, self.a_cf)
+        self._to_cf(self.a_nat, self.a_cf, "o")
         o = at.forward_o(self.a_cf)
         # x2 = x + o (the residual stream) and h2 = RMSNorm(x2) in one pass
         B.sl_rmsnorm_fwd(o, self.g2, self.eps, self.h2, self.rstd2, res=x, sum_out=self.x2)
@@ -80,11 +93,12 @@ class DecoderLayer:
         dh2 = self.ffn.backward(dy)
         B.sl_rmsnorm_bwd(dh2, self.x2, self.g2, self.rstd2, self.dx2, dres=dy)
         da_cf = at.backward_o(self.dx2)
-        self._to_seq(da_cf, self.da_nat)
+        self._to_seq(da_cf, self.da_nat, "o")
         B.sl_attention_bwd(self.ws, self.q_nat, self.k_nat, self.v_nat, self.a_nat, self.da_nat, self.lse, self.n_seq,
                            at.hq, at.hkv, at.hd, self.dq_nat, self.dk_nat, self.dv_nat)
-        for src, dst in ((self.dq_nat, self.dq_cf), (self.dk_nat, self.dk_cf), (self.dv_nat, self.dv_cf)):
-            self._to_cf(src, dst)
+        for src, dst, name in ((self.dq_nat, self.dq_cf, "q"), (self.dk_nat, self.dk_cf, "k"),
+                               (self.dv_nat, self.dv_cf, "v")):
+            self._to_cf(src, dst, name)
         dh1 = at.backward_qkv(self.dq_cf, self.dk_cf, self.dv_cf)
         B.sl_rmsnorm_bwd(dh1, self.x, self.g1, self.rstd1, self.dx, dres=self.dx2)
         return self.dx

@@ -85,7 +85,7 @@ class SparseLoRAModel:
             w = frozen["layers"][i] if "layers" in frozen else frozen
             lo = loras[i]
             attn = AttnProjBlock(w["q"], w["k"], w["v"], w["o"], lo["q"], lo["k"], lo["v"], lo["o"], lora_scale, est_k,
-                                 hq, hkv, hd, T, n_ctx, keep[i][0], device)
+                                 hq, hkv, hd, T, n_ctx, keep[i][0], device, io_layout="sigma")
             ffn = FFNBlock(w["gate"], w["up"], w["down"], lo["gate"], lo["up"], lo["down"], lora_scale, est_k, T, n_ctx,
                            keep[i][1], device)
             self.layers.append(DecoderLayer(attn, ffn, gammas[i][0], gammas[i][1], perm, n_seq, eps))

@@ -438,6 +438,25 @@ SL_API sl_status sl_prepare_weight(const void* w, int64_t d_out, int64_t d_in, v
 SL_API sl_status sl_permute_rows(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm,
                                  int64_t n_rows, int64_t n_cols, void* dst, int64_t ld_dst, sl_stream stream);
 
+/* Row permutation of a batch that also converts the channel order of its context rows to or
+ * from the sigma layout (the layout a block's sliced products read and write; see the top of
+ * this file), so that one pass does both: dst[i, :] = src[perm[i], :] for i < n_rows, n_cols
+ * bf16 columns, except on context rows:
+ *   to_sigma != 0: destination rows i < n_ctx store dst[i, p] = src[perm[i], sigma[p]];
+ *   to_sigma == 0: source rows perm[i] < n_ctx are in the sigma layout: dst[i, sigma[p]] =
+ *                  src[perm[i], p].
+ * The decoder layer uses it between sequence order (the attention core) and context-first order
+ * with the sigma layout (the attention block's q, k, v, x_o, dq, dk, dv): "SparseLoRA:
+ * Accelerating LLM Fine-Tuning with Contextual Sparsity", walkthrough, "Putting It All Together"
+ * and Figure 8 (context and output tokens of each sequence). sigma: a permutation of [0, n_cols)
+ * (sl_select_channels writes it; the debug build checks its entries and perm's). n_cols <= 16384,
+ * a multiple of 8, leading dimensions multiples of 8, 16-byte aligned bases; dst must not overlap
+ * src. Errors: SL_ERR_INVALID_ARG for a null pointer, SL_ERR_SHAPE for a non-positive size,
+ * n_cols > 16384 or a leading dimension below n_cols, SL_ERR_ALIGNMENT otherwise. */
+SL_API sl_status sl_permute_rows_sigma(const void* src, int64_t ld_src, int64_t src_rows, const int32_t* perm,
+                                       int64_t n_rows, int64_t n_cols, const int32_t* sigma, int64_t n_ctx,
+                                       int32_t to_sigma, void* dst, int64_t ld_dst, sl_stream stream);
+
 /* Up to 8 row gathers of bf16 rows in one launch: for each q < n, dst[q][i, :] =
  * src[q][perm[q][i], :] for i < n_rows[q], n_cols[q] columns, leading dimensions ld_src[q] and
  * ld_dst[q]; src[q] has src_rows[q] rows (every perm entry must lie in [0, src_rows[q]); the debug

@@ -238,3 +238,19 @@ def test_permute_rows_rejects_bad_arguments(lib):
     assert f(a, 64, 0, a, 4, 64, a, 64, None) == B.SL_ERR_SHAPE
     assert f(a, 64, 8, a, 0, 64, a, 64, None) == B.SL_ERR_SHAPE
     assert f(a, 32, 8, a, 4, 64, a, 64, None) == B.SL_ERR_SHAPE
+
+
+def test_permute_rows_sigma_rejects_bad_arguments(lib):
+    """sl_permute_rows_sigma(src, ld_src, src_rows, perm, n_rows, n_cols, sigma, n_ctx, to_sigma, dst,
+    ld_dst, stream): host checks only; nothing is launched."""
+    P = ctypes.c_void_p
+    f = lib.sl_permute_rows_sigma
+    a, odd = P(0x10000), P(0x10008)
+    assert f(None, 64, 8, a, 4, 64, a, 2, 1, a, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, 8, a, 4, 64, None, 2, 1, a, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, 8, a, 4, 64, a, 2, 1, None, 64, None) == B.SL_ERR_INVALID_ARG
+    assert f(a, 64, 0, a, 4, 64, a, 2, 1, a, 64, None) == B.SL_ERR_SHAPE
+    assert f(a, 64, 8, a, 4, 64, a, -1, 1, a, 64, None) == B.SL_ERR_SHAPE
+    assert f(a, 1 << 15, 8, a, 4, 16392, a, 2, 1, a, 1 << 15, None) == B.SL_ERR_SHAPE  # wider than 16384
+    assert f(a, 60, 8, a, 4, 60, a, 2, 1, a, 64, None) == B.SL_ERR_ALIGNMENT
+    assert f(odd, 64, 8, a, 4, 64, a, 2, 1, a, 64, None) == B.SL_ERR_ALIGNMENT

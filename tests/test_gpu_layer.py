@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def build(n_seq, S, n_out, D, hq, hkv, hd, F, r, k, ratio, seed):
+def build(n_seq, S, n_out, D, hq, hkv, hd, F, r, k, ratio, seed, io_layout="natural"):
     gen = inputs.generator(seed)
     Dq, Dkv = hq * hd, hkv * hd
     shapes = {"q": (Dq, D), "k": (Dkv, D), "v": (Dkv, D), "o": (D, Dq), "gate": (F, D), "up": (F, D), "down": (D, F)}
@@ -31,7 +31,7 @@ def build(n_seq, S, n_out, D, hq, hkv, hd, F, r, k, ratio, seed):
     perm = inputs.context_first_order(torch.from_numpy(ctx)).numpy()
     C = int(ctx.sum())
     attn = blocks.AttnProjBlock(w["q"], w["k"], w["v"], w["o"], lora["q"], lora["k"], lora["v"], lora["o"], 2.0, k,
-                                hq, hkv, hd, T, C, ratio, DEV)
+                                hq, hkv, hd, T, C, ratio, DEV, io_layout=io_layout)
     ffn = blocks.FFNBlock(w["gate"], w["up"], w["down"], lora["gate"], lora["up"], lora["down"], 2.0, k, T, C, ratio,
                           DEV)
     layer = DecoderLayer(attn, ffn, g1, g2, perm, n_seq)
@@ -39,9 +39,12 @@ def build(n_seq, S, n_out, D, hq, hkv, hd, F, r, k, ratio, seed):
                 ffn=ffn, heads=(hq, hkv, hd), n_seq=n_seq)
 
 
+@pytest.mark.parametrize("io_layout", ["natural", "sigma"])
 @pytest.mark.parametrize("n_seq,S,n_out,D,hq,hkv,hd,F", [(2, 64, 16, 256, 4, 2, 32, 512), (3, 40, 8, 128, 2, 2, 64, 264)])
-def test_decoder_layer_matches_oracle(n_seq, S, n_out, D, hq, hkv, hd, F):
-    p = build(n_seq, S, n_out, D, hq, hkv, hd, F, 16, 8, 0.5, seed=61)
+def test_decoder_layer_matches_oracle(n_seq, S, n_out, D, hq, hkv, hd, F, io_layout):
+    """Both interface layouts of the attention block: natural channels, or the sigma layout with
+    the layer's permutations converting the context rows' channel order."""
+    p = build(n_seq, S, n_out, D, hq, hkv, hd, F, 16, 8, 0.5, seed=61, io_layout=io_layout)
     perm = p["perm"]
     pt = torch.from_numpy(perm)
     x_cf = p["x"][pt].to(DEV).contiguous()

@@ -35,7 +35,7 @@ def test_decoder_layer_full_size(ac, fc, seqs):
     g1 = (1.0 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
     g2 = (1.0 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
     attn = blocks.AttnProjBlock(da["q"], da["k"], da["v"], da["o"], da["lora_q"], da["lora_k"], da["lora_v"],
-                                da["lora_o"], ac.lora_scale, ac.k, hq, hkv, hd, T, C, ac.ratio, DEV)
+                                da["lora_o"], ac.lora_scale, ac.k, hq, hkv, hd, T, C, ac.ratio, DEV, io_layout="sigma")
     ffn = blocks.FFNBlock(df["gate"], df["up"], df["down"], df["lora_gate"], df["lora_up"], df["lora_down"],
                           fc.lora_scale, fc.k, T, C, fc.ratio, DEV)
     p_np = perm.cpu().numpy()

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from contextual_sparsity_lora_b200 import binding as B
-from contextual_sparsity_lora_b200 import inputs
+from contextual_sparsity_lora_b200 import blocks, inputs
 from gpu_helpers import BF16_TOL, FP32_TOL, attn_problem, ffn_problem, rel_fro, unsigma
 
 pytestmark = pytest.mark.gpu
@@ -464,3 +464,70 @@ def test_lora_fwd_estimate_and_scores_from_z(T, C, D, crit, k, r):
         s_w, _ = oracle.ffn_select(x, ctx, (fac[0].W_A, fac[0].W_B), (fac[1].W_A, fac[1].W_B), 0.5)
         assert rel_fro(sc, s_w) < FP32_TOL
     assert ws.read_device_flag() == 0
+
+
+@pytest.mark.parametrize("to_sigma", [True, False])
+@pytest.mark.parametrize("n_cols", [8, 1024, 4096, 5120])
+def test_permute_rows_sigma_is_exact(to_sigma, n_cols):
+    """Row permutation with the context rows' channel order converted to or from the sigma
+    layout, against NumPy indexing (bit-exact: it only moves bf16 values)."""
+    n_rows, n_ctx = 300, 217
+    rng = np.random.default_rng(n_cols + int(to_sigma))
+    src = torch.randn(n_rows + 5, n_cols, device=DEV).to(torch.bfloat16)
+    perm = rng.permutation(n_rows).astype(np.int32)
+    sig = rng.permutation(n_cols).astype(np.int32)
+    dst = torch.full((n_rows, n_cols), 7.0, device=DEV, dtype=torch.bfloat16)
+    B.sl_permute_rows_sigma(src, torch.tensor(perm, device=DEV), dst, torch.tensor(sig, device=DEV), n_ctx, to_sigma)
+    s = src.float().cpu().numpy()
+    want = s[perm].copy()
+    for i in range(n_rows):
+        if to_sigma and i < n_ctx:
+            want[i] = s[perm[i]][sig]
+        elif not to_sigma and perm[i] < n_ctx:
+            want[i, sig] = s[perm[i]]
+    np.testing.assert_array_equal(dst.float().cpu().numpy(), want)
+
+
+def test_attention_block_sigma_layout_matches_natural():
+    """The attention block with its interfaces in the sigma layout against the natural layout on
+    the same inputs: q, k, v and dx_o equal after the layout conversion (the same GEMM tiles,
+    bulk instead of scattered stores); y, dx and the gradients within fp32 summation-order
+    rounding (x_o A^T over permuted channels, the fused LoRA backward's unordered sums)."""
+    T, C, D, hq, hkv, hd, r, k = 424, 300, 512, 8, 2, 64, 32, 8
+    a = attn_problem(T, C, D, hq, hkv, hd, r, k, seed=47)
+    w, lo = a["w"], a["lora"]
+    blks = {}
+    for lay in ("natural", "sigma"):
+        blks[lay] = blocks.AttnProjBlock(w["q"], w["k"], w["v"], w["o"], lo["q"], lo["k"], lo["v"], lo["o"], 2.0, k, hq,
+                                         hkv, hd, T, C, 0.5, DEV, io_layout=lay)
+    nb, sb = blks["natural"], blks["sigma"]
+    xg = cu(a["x"])
+    nb.forward_qkv(xg)
+    sb.forward_qkv(xg)
+    torch.cuda.synchronize()
+    for name in ("sig_q", "sig_k", "sig_v", "sig_o"):
+        assert torch.equal(getattr(nb, name), getattr(sb, name)), name
+    for t_n, t_s, name in ((nb.q, sb.q, "q"), (nb.kk, sb.kk, "k"), (nb.vv, sb.vv, "v")):
+        np.testing.assert_array_equal(oracle.f64(t_n), unsigma(t_s, sb.sigma_of(name), C))
+
+    def to_sig(t, name):  # natural -> sigma layout on the context rows
+        out = t.clone()
+        sig = sb.sigma_of(name).long()
+        out[:C] = t[:C][:, sig]
+        return out
+    x_o = cu(a["x_o"])
+    nb.forward_o(x_o)
+    sb.forward_o(to_sig(x_o, "o"))
+    dy = cu(a["dy"])
+    nb.backward_o(dy)
+    sb.backward_o(dy)
+    dq, dk, dv = cu(a["dq"]), cu(a["dk"]), cu(a["dv"])
+    nb.backward_qkv(dq, dk, dv)
+    sb.backward_qkv(to_sig(dq, "q"), to_sig(dk, "k"), to_sig(dv, "v"))
+    torch.cuda.synchronize()
+    assert nb.read_device_flag() == 0 and sb.read_device_flag() == 0
+    # x_o A^T sums the context rows' channels in another order in the sigma layout (permuted A)
+    assert rel_fro(sb.y, nb.y) < 1e-3
+    np.testing.assert_array_equal(oracle.f64(nb.dx_o), unsigma(sb.dx_o, sb.sigma_of("o"), C))
+    assert rel_fro(sb.dx, nb.dx) < 1e-3
+    assert rel_fro(sb.grads.flat, nb.grads.flat) < 1e-3
