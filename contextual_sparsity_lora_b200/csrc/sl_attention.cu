@@ -258,9 +258,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < 32; ++i)
           if (32 * c + i <= kmax) mj = fmaxf(mj, __uint_as_float(sv[c][i]));
-      const float m_new = fmaxf(m, mj);
+      // The running maximum moves only when a row's maximum grows by more than 2^8 in the
+      // exponential's scale: the exponentials then stay below 256 and O and l keep one common
+      // reference, so O is rescaled in TMEM rarely (after the first tiles almost never).
+      const float m_cand = fmaxf(m, mj);
+      const bool grow = m == -INFINITY || (m_cand - m) * p.scale_log2 > 8.0f;
+      const float m_new = grow ? m_cand : m;
       const float mb = m_new * p.scale_log2;
-      const float corr = (m == -INFINITY) ? 0.f : ex2(m * p.scale_log2 - mb);
+      const float corr = (m == -INFINITY) ? 0.f : (grow ? ex2(m * p.scale_log2 - mb) : 1.f);
       float rs = 0.f;
       uint32_t pw[4][16];
 #pragma unroll
