@@ -23,10 +23,13 @@
 // run the online softmax, one query row per thread (its TMEM lane): row maximum, exponentials,
 // rescaling of O in TMEM when the maximum grows, P (bf16) into shared memory for the P V MMA.
 // Backward: one CTA per (128-key tile, key/value head, sequence), looping over the query heads of
-// the group and the query tiles at or after the key tile: S^T and dP^T by MMA, P^T and dS^T by the
-// compute warps (one key row per thread), then dV += P^T dO, dK += dS^T Q and dQ = dS K by MMA;
-// dK and dV stay in TMEM for the whole loop and are stored once, dQ leaves every iteration through
-// fp32 reductions into a workspace accumulator (several key tiles add to the same query rows).
+// the group and the query tiles at or after the key tile: S^T and dP^T by MMA, P^T and dS^T by
+// eight compute warps (one key row per thread, half of the query columns per warp), then
+// dV += P^T dO, dK += dS^T Q and dQ = dS K by MMA. dO and Q have separate barriers, so the next
+// dO loads once dV has read this one and dP^T of the next iteration starts while dQ is drained.
+// dK and dV stay in TMEM for the whole loop and are stored once; dQ leaves TMEM every iteration
+// into shared-memory boxes (over P^T and dS^T, free by then) and reaches the workspace accumulator
+// through bulk tensor reductions (fp32 adds in L2; several key tiles add to the same query rows).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -40,8 +43,11 @@ namespace sl {
 namespace {
 
 constexpr int kAttnThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 softmax / epilogue
+constexpr int kBwdComputeThreads = 256;                   // backward: warps 2..9
+constexpr int kAttnBwdThreads = 64 + kBwdComputeThreads;  // warp 0 TMA, warp 1 MMA + TMEM
 constexpr int kTile = 128;           // tokens per tile (TMEM lanes)
 constexpr int kChunk = 128 * 64 * 2;  // one 128-token x 64-element bf16 tile chunk (16 KB)
+constexpr int kDqBox = 128 * 32 * 4;  // one 128-row x 32-element fp32 dQ box (16 KB)
 
 struct AttnFwdParams {
   CUtensorMap qmap, kmap, vmap;  // [head_dim, heads, seq_len, n_seq], boxes 64 x 1 x 128 x 1
@@ -55,6 +61,7 @@ struct AttnFwdParams {
 
 struct AttnBwdParams {
   CUtensorMap qmap, kmap, vmap, domap;
+  CUtensorMap dqmap;             // dq_acc as [head_dim, hq, seq_len, n_seq] fp32, boxes 32 x 1 x 128 x 1
   const float* lse;              // [hq][T]
   const float* delta;            // [hq][T]: sum_d dO O per query row
   float* dq_acc;                 // [T][hq * hd] fp32, zero on entry
@@ -125,7 +132,42 @@ __device__ __forceinline__ void st_swizzled_row32(uint8_t* tile, int r, int c0, 
   }
 }
 
-__device__ __forceinline__ void named_bar_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_bwd() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Barrier of the backward's compute warps that also returns whether `ok` holds in all of them.
+__device__ __forceinline__ bool bar_and_bwd(bool ok) {
+  uint32_t all;
+  asm volatile(
+      "{\n\t.reg .pred q, a;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred a, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, a;\n\t}"
+      : "=r"(all)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return all != 0;
+}
+
+// Writes row r of a 128-row x 32-element fp32 box (128-byte swizzle: 16-byte unit u of row r sits
+// at unit u ^ (r % 8)) from 32 raw fp32 values, each multiplied by `mul`.
+__device__ __forceinline__ void st_dq_box_row(uint8_t* box, int r, const uint32_t (&v)[32], float mul) {
+  uint8_t* row = box + r * 128;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<float4*>(row + ((u ^ (r & 7)) * 16)) =
+        make_float4(__uint_as_float(v[4 * u]) * mul, __uint_as_float(v[4 * u + 1]) * mul,
+                    __uint_as_float(v[4 * u + 2]) * mul, __uint_as_float(v[4 * u + 3]) * mul);
+}
+
+// Adds a shared-memory box to global memory through a 4-D tensor map (fp32 add in L2; elements
+// outside the tensor are skipped), tracked in the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* m, const void* smem_src, int32_t c0, int32_t c1,
+                                                  int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 
 // ------------------------------------------------------------------------------------ forward
 
@@ -364,14 +406,9 @@ __global__ void attn_dq_cast_kernel(const float* __restrict__ acc, int64_t T, in
   *reinterpret_cast<uint2*>(dq + t * ldq + c) = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
 }
 
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 // ----------------------------------------------------------------------------------- backward
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams p) {
+__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nd = p.nd;
@@ -381,18 +418,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_
   uint8_t* sdo = sq + nd * kChunk;     // dO_i
   uint8_t* spt = sdo + nd * kChunk;    // P^T: 2 chunks (128 queries)
   uint8_t* sdst = spt + 2 * kChunk;    // dS^T: 2 chunks
+  // P^T and dS^T are also the four dQ boxes (128 query rows x 32 fp32, 128-byte swizzle) once the
+  // MMAs of an iteration have read them
   float* s_lse = reinterpret_cast<float*>(sdst + 2 * kChunk);  // [128]
   float* s_delta = s_lse + 128;                                // [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_delta + 128);
   uint64_t* kv_full = bars;
-  uint64_t* qd_full = bars + 1;
-  uint64_t* qd_empty = bars + 2;
-  uint64_t* s_full = bars + 3;
-  uint64_t* p_full = bars + 4;
-  uint64_t* mma2_done = bars + 5;
-  uint64_t* dq_free = bars + 6;
-  uint64_t* drain = bars + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* do_full = bars + 3;
+  uint64_t* do_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* mma2_done = bars + 7;
+  uint64_t* dq_free = bars + 8;
+  uint64_t* drain = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -403,12 +444,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_
   const int64_t T = (int64_t)p.n_seq * p.S;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, kBwdComputeThreads);
     mbar_init(mma2_done, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, kBwdComputeThreads);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -435,19 +478,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_
         tma_load_4d(sk + c * kChunk, &p.kmap, kv_full, 64 * c, g, kt * kTile, b);
         tma_load_4d(sv + c * kChunk, &p.vmap, kv_full, 64 * c, g, kt * kTile, b);
       }
-      int issued = 0;
+      // dO and Q have one buffer each and separate barriers: dO_(i+1) loads as soon as dV_i has
+      // read dO_i, Q_(i+1) once dK_i has read Q_i
+      int issued_do = 0, issued_q = 0;
       for (int it = 0; it < n_it; ++it) {
-        if (it > 0 && !mbar_wait(qd_empty, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
-        mbar_arrive_expect_tx(qd_full, 2 * nd * kChunk);
         const int h = it_head(it), qt = it_qtile(it);
-        for (int c = 0; c < nd; ++c) {
-          tma_load_4d(sq + c * kChunk, &p.qmap, qd_full, 64 * c, h, qt * kTile, b);
-          tma_load_4d(sdo + c * kChunk, &p.domap, qd_full, 64 * c, h, qt * kTile, b);
-        }
-        issued = it + 1;
+        if (it > 0 && !mbar_wait(do_empty, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(do_full, nd * kChunk);
+        for (int c = 0; c < nd; ++c) tma_load_4d(sdo + c * kChunk, &p.domap, do_full, 64 * c, h, qt * kTile, b);
+        issued_do = it + 1;
+        if (it > 0 && !mbar_wait(q_empty, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(q_full, nd * kChunk);
+        for (int c = 0; c < nd; ++c) tma_load_4d(sq + c * kChunk, &p.qmap, q_full, 64 * c, h, qt * kTile, b);
+        issued_q = it + 1;
       }
       mbar_wait(kv_full, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
-      if (issued > 0) mbar_wait(qd_full, (issued - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      if (issued_do > 0) mbar_wait(do_full, (issued_do - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      if (issued_q > 0) mbar_wait(q_full, (issued_q - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -458,117 +505,141 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_bwd_kernel(const __grid_
       const uint32_t apt = smem_u32(spt), adst = smem_u32(sdst);
       bool ok = mbar_wait(kv_full, 0, abort_flag, p.err, DEV_TIMEOUT_MMA);
       for (int it = 0; ok && it < n_it; ++it) {
-        if (!mbar_wait(qd_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        // dP^T (columns 128..255) needs only dO: it may run while the previous dQ is drained
+        if (!mbar_wait(do_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < 4 * nd; ++t)
+          umma_bf16(tmem + 128, kmajor_desc(av, t), kmajor_desc(bdo, t), id_kq, t > 0 ? 1u : 0u);
+        if (!mbar_wait(q_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
         if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
         tc_fence_after();
-        for (int t = 0; t < 4 * nd; ++t) {
+        for (int t = 0; t < 4 * nd; ++t)
           umma_bf16(tmem, kmajor_desc(ak, t), kmajor_desc(bq, t), id_kq, t > 0 ? 1u : 0u);
-          umma_bf16(tmem + 128, kmajor_desc(av, t), kmajor_desc(bdo, t), id_kq, t > 0 ? 1u : 0u);
-        }
         umma_commit(s_full);
         if (!mbar_wait(p_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
         tc_fence_after();
-        for (int t = 0; t < 8; ++t) {
-          const uint32_t acc = (it > 0 || t > 0) ? 1u : 0u;
-          umma_bf16(tmem + t_dv, kmajor_desc(apt, t), mnmajor_desc(bdo, t), id_kd, acc);
-          umma_bf16(tmem + t_dk, kmajor_desc(adst, t), mnmajor_desc(bq, t), id_kd, acc);
+        for (int t = 0; t < 8; ++t)
+          umma_bf16(tmem + t_dv, kmajor_desc(apt, t), mnmajor_desc(bdo, t), id_kd, (it > 0 || t > 0) ? 1u : 0u);
+        umma_commit(do_empty);
+        for (int t = 0; t < 8; ++t)
+          umma_bf16(tmem + t_dk, kmajor_desc(adst, t), mnmajor_desc(bq, t), id_kd, (it > 0 || t > 0) ? 1u : 0u);
+        umma_commit(q_empty);
+        for (int t = 0; t < 8; ++t)
           umma_bf16(tmem, mnmajor_desc(adst, t), mnmajor_desc(ak, t), id_qd, t > 0 ? 1u : 0u);
-        }
         umma_commit(mma2_done);
-        umma_commit(qd_empty);
       }
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else {
+    // Eight compute warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 and handles one half of the
+    // columns (query columns of S^T / dP^T, head-dimension columns of dQ, dK or dV).
+    const int cw = warp - 2;
     const int quarter = warp & 3;
+    const int half = cw >> 2;
     const int r = quarter * 32 + lane;           // key row of the tile (S^T, dP^T, dV, dK) or query row (dQ)
     const int kpos = kt * kTile + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool lead = cw == 0 && lane == 0;      // issues the dQ reductions
     const float log2e = 1.4426950408889634f;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int h = it_head(it), qt = it_qtile(it);
       const int qpos_r = qt * kTile + r;
-      // this tile's LSE and delta (the previous iteration's readers passed the barrier below)
-      named_bar_compute();
-      s_lse[r] = qpos_r < p.S ? p.lse[(int64_t)h * T + (int64_t)b * p.S + qpos_r] * log2e : 0.f;
-      s_delta[r] = qpos_r < p.S ? p.delta[(int64_t)h * T + (int64_t)b * p.S + qpos_r] : 0.f;
-      named_bar_compute();
-      if (!mbar_wait(s_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
-      tc_fence_after();
-      // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S
-      const int cmin = kpos - qt * kTile;            // first visible query column
-      const int cmax = p.S - 1 - qt * kTile;         // last query column inside the sequence
-      for (int c = 0; c < 4; ++c) {
-        uint32_t st[32], dp[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_off + 32 * c, st);
-        tmem_ld32(tmem + lane_off + 128 + 32 * c, dp);
-        tmem_ld_wait_regs(st);
-        regs_after_wait(dp);
-        uint32_t pw[16], dw[16];
+      // The previous iteration's dQ reductions have read their boxes (P^T and dS^T are written
+      // below) and every reader of the previous LSE and delta is past this point. `ok` is the same
+      // in every compute thread here (combined at the end of each iteration).
+      if (lead) bulk_wait_read<0>();
+      named_bar_bwd();
+      if (!ok) break;
+      if (half == 0) {
+        s_lse[r] = qpos_r < p.S ? p.lse[(int64_t)h * T + (int64_t)b * p.S + qpos_r] * log2e : 0.f;
+        s_delta[r] = qpos_r < p.S ? p.delta[(int64_t)h * T + (int64_t)b * p.S + qpos_r] : 0.f;
+      }
+      named_bar_bwd();
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
+      if (ok) {
+        tc_fence_after();
+        // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S
+        const int cmin = kpos - qt * kTile;            // first visible query column
+        const int cmax = p.S - 1 - qt * kTile;         // last query column inside the sequence
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
+          uint32_t st[32], dp[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_off + 32 * c, st);
+          tmem_ld32(tmem + lane_off + 128 + 32 * c, dp);
+          tmem_ld_wait_regs(st);
+          regs_after_wait(dp);
+          uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pv[2], dv2[2];
+          for (int i = 0; i < 32; i += 2) {
+            float pv[2], dv2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 32 * c + i + e;
-            const bool vis = col >= cmin && col <= cmax && kpos < p.S;
-            const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - s_lse[col]) : 0.f;
-            pv[e] = pe;
-            dv2[e] = pe * (__uint_as_float(dp[i + e]) - s_delta[col]);
+            for (int e = 0; e < 2; ++e) {
+              const int col = 32 * c + i + e;
+              const bool vis = col >= cmin && col <= cmax && kpos < p.S;
+              const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - s_lse[col]) : 0.f;
+              pv[e] = pe;
+              dv2[e] = pe * (__uint_as_float(dp[i + e]) - s_delta[col]);
+            }
+            pw[i / 2] = pack2(pv[0], pv[1]);
+            dw[i / 2] = pack2(dv2[0], dv2[1]);
           }
-          pw[i / 2] = pack2(pv[0], pv[1]);
-          dw[i / 2] = pack2(dv2[0], dv2[1]);
+          st_swizzled_row32(spt, r, 32 * c, pw);
+          st_swizzled_row32(sdst, r, 32 * c, dw);
         }
-        st_swizzled_row32(spt, r, 32 * c, pw);
-        st_swizzled_row32(sdst, r, 32 * c, dw);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        ok = __all_sync(0xffffffffu, mbar_wait(mma2_done, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-      // dQ of this (head, query tile): lane r = query row qt * 128 + r
-      if (!mbar_wait(mma2_done, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
-      tc_fence_after();
-      const bool qok = qpos_r < p.S;
-      float* dqrow = p.dq_acc + ((int64_t)b * p.S + qpos_r) * ((int64_t)p.hq * p.hd) + (int64_t)h * p.hd;
-      for (int c = 0; c < 2 * nd; ++c) {
-        uint32_t v[32];
+      if (ok) {
+        // dQ of this (head, query tile), lane r = query row qt * 128 + r: out of TMEM (which the next
+        // S^T may then overwrite), scaled into the boxes, added to the accumulator by bulk reductions
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
         __syncwarp();
-        tmem_ld32(tmem + lane_off + 32 * c, v);
-        tmem_ld_wait_regs(v);
-        if (!qok || 32 * c >= p.hd) continue;
-        const int n = min(32, p.hd - 32 * c);
-        for (int i = 0; i < n; i += 4)
-          red_add_v4(dqrow + 32 * c + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
-                     __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
+        tmem_ld32(tmem + lane_off + 64 * half, v0);
+        tmem_ld32(tmem + lane_off + 64 * half + 32, v1);
+        tmem_ld_wait_regs(v0);
+        regs_after_wait(v1);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        st_dq_box_row(spt + (2 * half) * kDqBox, r, v0, p.scale);
+        st_dq_box_row(spt + (2 * half + 1) * kDqBox, r, v1, p.scale);
+        fence_proxy_async_smem();
       }
-      tc_fence_before();
-      mbar_arrive(dq_free);
+      ok = bar_and_bwd(ok);
+      if (ok && lead) {
+        for (int c = 0; c < 4 && 32 * c < p.hd; ++c)
+          tma_reduce_add_4d(&p.dqmap, spt + c * kDqBox, 32 * c, h, qt * kTile, b);
+        bulk_commit();
+      }
     }
-    // dK, dV of this key tile: the MMAs of the last iteration have completed (mma2_done); every lane
-    // takes part in the (warp-collective) loads, rows past the sequence store nothing
+    // the reductions have completed before the CTA ends (and before its shared memory is reused)
+    if (lead) bulk_wait_all();
+    // dK (half 1), dV (half 0) of this key tile: the MMAs of the last iteration have completed
+    // (mma2_done); every lane takes part in the (warp-collective) loads, rows past the sequence
+    // store nothing
     if (ok) {
       tc_fence_after();
       const bool kok = kpos < p.S;
       const int64_t row = (int64_t)b * p.S + kpos;
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* out = (which ? p.dk : p.dv) + row * p.ldkv + (int64_t)g * p.hd;
-        const float mul = which ? p.scale : 1.f;
-        for (int c = 0; c < 2 * nd; ++c) {
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(tmem + lane_off + (which ? t_dk : t_dv) + 32 * c, v);
-          tmem_ld_wait_regs(v);
-          if (!kok || 32 * c >= p.hd) continue;
-          uint32_t w[16];
+      const int which = half;
+      __nv_bfloat16* out = (which ? p.dk : p.dv) + row * p.ldkv + (int64_t)g * p.hd;
+      const float mul = which ? p.scale : 1.f;
+      for (int c = 0; c < 2 * nd; ++c) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + (which ? t_dk : t_dv) + 32 * c, v);
+        tmem_ld_wait_regs(v);
+        if (!kok || 32 * c >= p.hd) continue;
+        uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
-          uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
-          const int nv = min(32, p.hd - 32 * c) / 8;
-          for (int q = 0; q < nv; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
+        for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
+        uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
+        const int nv = min(32, p.hd - 32 * c) / 8;
+        for (int q = 0; q < nv; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
       }
     }
   }
@@ -610,6 +681,20 @@ bool head_map(CUtensorMap* m, const void* ptr, int64_t ld, int n_seq, int S, int
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [hd, heads, S, n_seq] view of the [n_seq * S, heads * hd] fp32 dQ accumulator; boxes of
+// 32 x 1 x 128 x 1 (128 bytes per row), 128-byte swizzle.
+bool dq_acc_map(CUtensorMap* m, float* ptr, int n_seq, int S, int heads, int hd) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)S, (cuuint64_t)n_seq};
+  cuuint64_t strides[3] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4, (cuuint64_t)S * heads * hd * 4};
+  cuuint32_t box[4] = {32, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -669,6 +754,7 @@ int attention_bwd(const void* q, const void* k, const void* v, const void* o, co
   const int64_t T = (int64_t)n_seq * S;
   float* dq_acc = static_cast<float*>(scratch);
   float* delta = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + ((T * hq * hd * 4 + 255) & ~int64_t(255)));
+  if (!dq_acc_map(&p.dqmap, dq_acc, n_seq, S, hq, hd)) return 2;
   if (cudaMemsetAsync(dq_acc, 0, (size_t)T * hq * hd * 4, s) != cudaSuccess) return 5;
   {
     const int64_t items = T * hq;
@@ -699,7 +785,7 @@ int attention_bwd(const void* q, const void* k, const void* v, const void* o, co
     attr = true;
   }
   const dim3 grid((unsigned)((S + kTile - 1) / kTile), (unsigned)hkv, (unsigned)n_seq);
-  launch_kernel(attn_bwd_kernel, grid, kAttnThreads, bwd_smem(), s, p);
+  launch_kernel(attn_bwd_kernel, grid, kAttnBwdThreads, bwd_smem(), s, p);
   if (launch_failed("sl_attention")) return 5;
   note_launch();
   // dQ: the dense [T, hq hd] accumulator to bf16 rows of leading dimension ldq
