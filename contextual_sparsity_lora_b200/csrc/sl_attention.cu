@@ -19,9 +19,10 @@
 //
 // Forward: one CTA per (128-query tile, query head, sequence). Warp 0 loads Q once and the K/V
 // tiles through a two-stage ring; warp 1 issues the MMAs (S into two alternating TMEM buffers, so
-// S of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-5
-// run the online softmax, one query row per thread (its TMEM lane): row maximum, exponentials,
-// rescaling of O in TMEM when the maximum grows, P (bf16) into shared memory for the P V MMA.
+// S of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-9
+// run the online softmax, one query row (its TMEM lane) and half of the key columns per thread:
+// row maximum, exponentials, rescaling of O in TMEM when the maximum grows, P (bf16) into shared
+// memory for the P V MMA.
 // Backward: one CTA per (128-key tile, key/value head, sequence), looping over the query heads of
 // the group and the query tiles at or after the key tile: S^T and dP^T by MMA, P^T and dS^T by
 // eight compute warps (one key row per thread, half of the query columns per warp), then
@@ -42,12 +43,12 @@ namespace sl {
 
 namespace {
 
-constexpr int kAttnThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 softmax / epilogue
+constexpr int kSoftThreads = 256;                   // forward: warps 2..9 softmax / epilogue
+constexpr int kAttnThreads = 64 + kSoftThreads;     // warp 0 TMA, warp 1 MMA + TMEM
 constexpr int kBwdComputeThreads = 256;                   // backward: warps 2..9
 constexpr int kAttnBwdThreads = 64 + kBwdComputeThreads;  // warp 0 TMA, warp 1 MMA + TMEM
 constexpr int kTile = 128;           // tokens per tile (TMEM lanes)
 constexpr int kChunk = 128 * 64 * 2;  // one 128-token x 64-element bf16 tile chunk (16 KB)
-constexpr int kDqBox = 128 * 32 * 4;  // one 128-row x 32-element fp32 dQ box (16 KB)
 
 struct AttnFwdParams {
   CUtensorMap qmap, kmap, vmap;  // [head_dim, heads, seq_len, n_seq], boxes 64 x 1 x 128 x 1
@@ -132,7 +133,19 @@ __device__ __forceinline__ void st_swizzled_row32(uint8_t* tile, int r, int c0, 
   }
 }
 
-__device__ __forceinline__ void named_bar_bwd() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Barrier of the forward's softmax warps that also returns whether `ok` holds in all of them.
+__device__ __forceinline__ bool bar_and_soft(bool ok) {
+  uint32_t all;
+  asm volatile(
+      "{\n\t.reg .pred q, a;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred a, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, a;\n\t}"
+      : "=r"(all)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return all != 0;
+}
 // Barrier of the backward's compute warps that also returns whether `ok` holds in all of them.
 __device__ __forceinline__ bool bar_and_bwd(bool ok) {
   uint32_t all;
@@ -147,8 +160,9 @@ __device__ __forceinline__ bool bar_and_bwd(bool ok) {
   return all != 0;
 }
 
-// Writes row r of a 128-row x 32-element fp32 box (128-byte swizzle: 16-byte unit u of row r sits
-// at unit u ^ (r % 8)) from 32 raw fp32 values, each multiplied by `mul`.
+// Writes row r of a box of 32-element fp32 rows (128-byte swizzle: 16-byte unit u of row r sits at
+// unit u ^ (r % 8); the box starts on a 1024-byte boundary) from 32 raw fp32 values, each
+// multiplied by `mul`.
 __device__ __forceinline__ void st_dq_box_row(uint8_t* box, int r, const uint32_t (&v)[32], float mul) {
   uint8_t* row = box + r * 128;
 #pragma unroll
@@ -178,7 +192,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   uint8_t* sq = smem;                          // Q: nd chunks
   uint8_t* skv = sq + nd * kChunk;             // stage s: K (nd chunks) then V (nd chunks)
   uint8_t* sp = skv + 2 * 2 * nd * kChunk;     // P: 2 chunks (128 keys)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sp + 2 * kChunk);
+  float* s_l = reinterpret_cast<float*>(sp + 2 * kChunk);  // [2][128]: the two halves' row sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_l + 256);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
@@ -201,9 +216,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
+      mbar_init(&s_free[s], kSoftThreads);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, kSoftThreads);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -275,31 +290,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else {
+    // Eight softmax warps: warp w holds query rows 32 (w % 4) .. + 31 (its TMEM lanes) and one half
+    // of the key columns of each S tile (exponentials, P) and of O (rescale, output). Both halves
+    // read the whole S row for its maximum, so they keep the same running maximum without an
+    // exchange; their partial row sums meet once, at the end.
+    const int cw = warp - 2;
     const int quarter = warp & 3;
+    const int half = cw >> 2;
     const int r = quarter * 32 + lane;               // query row in the tile = TMEM lane
     const int qpos = qt * kTile + r;                 // position in the sequence
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const int own0 = 64 * half, oth0 = 64 - own0;    // first key column of this half / the other
+    float m = -INFINITY, l = 0.f;                    // l: this half's share of the row sum
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       const int s = j & 1;
-      if (!mbar_wait(&s_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      uint32_t sv[4][32];
+      uint32_t so[2][32], sx[2][32];                 // this half's columns, the other half's
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128 * s + 32 * c, sv[c]);
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(tmem + lane_off + 128 * s + own0 + 32 * c, so[c]);
+        tmem_ld32(tmem + lane_off + 128 * s + oth0 + 32 * c, sx[c]);
+      }
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s_free[s]);
       // causal mask within the sequence: key k is visible to query q when k <= q and k < S
       const int kbase = j * kTile;
       const int kmax = min(qpos, p.S - 1) - kbase;   // last visible column of this tile
-      float mj = -INFINITY;
+      // (tiles wholly below the diagonal and inside the sequence, kmax >= 127, skip the masks)
+      const bool whole = kmax >= kTile - 1;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (whole) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * c + i <= kmax) mj = fmaxf(mj, __uint_as_float(sv[c][i]));
+          for (int i = 0; i < 32; ++i)
+            mx[i & 3] = fmaxf(mx[i & 3], fmaxf(__uint_as_float(so[c][i]), __uint_as_float(sx[c][i])));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (own0 + 32 * c + i <= kmax) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(so[c][i]));
+            if (oth0 + 32 * c + i <= kmax) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sx[c][i]));
+          }
+      }
+      const float mj = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // The running maximum moves only when a row's maximum grows by more than 2^8 in the
       // exponential's scale: the exponentials then stay below 256 and O and l keep one common
       // reference, so O is rescaled in TMEM rarely (after the first tiles almost never).
@@ -308,24 +349,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const float m_new = grow ? m_cand : m;
       const float mb = m_new * p.scale_log2;
       const float corr = (m == -INFINITY) ? 0.f : (grow ? ex2(m * p.scale_log2 - mb) : 1.f);
-      float rs = 0.f;
-      uint32_t pw[4][16];
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pw[2][16];
+      if (whole) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float e0 = (32 * c + i <= kmax) ? ex2(__uint_as_float(sv[c][i]) * p.scale_log2 - mb) : 0.f;
-          const float e1 = (32 * c + i + 1 <= kmax) ? ex2(__uint_as_float(sv[c][i + 1]) * p.scale_log2 - mb) : 0.f;
-          rs += e0 + e1;
-          pw[c][i / 2] = pack2(e0, e1);
-        }
-      l = l * corr + rs;
+          for (int i = 0; i < 32; i += 2) {
+            const float e0 = ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb);
+            const float e1 = ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb);
+            rs[(i >> 1) & 3] += e0 + e1;
+            pw[c][i / 2] = pack2(e0, e1);
+          }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int col = own0 + 32 * c + i;
+            const float e0 = (col <= kmax) ? ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb) : 0.f;
+            const float e1 = (col + 1 <= kmax) ? ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb) : 0.f;
+            rs[(i >> 1) & 3] += e0 + e1;
+            pw[c][i / 2] = pack2(e0, e1);
+          }
+      }
+      l = l * corr + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       if (j >= 1) {
-        // the previous P V has landed in O (and read P): rescale O when the maximum grew
-        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) { ok = false; break; }
+        // the previous P V has landed in O (and read P): rescale this half of O when the maximum grew
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
-          for (int c = 0; c < 2 * nd; ++c) {
+          for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
             uint32_t ov[32];
             __syncwarp();
             tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
@@ -338,18 +395,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) st_swizzled_row32(sp, r, 32 * c, pw[c]);
+      for (int c = 0; c < 2; ++c) st_swizzled_row32(sp, r, own0 + 32 * c, pw[c]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
       m = m_new;
     }
-    if (ok && mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE)) {
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
+    s_l[half * 128 + r] = l;
+    // every softmax thread reaches this barrier (the loop above only breaks, never returns)
+    ok = bar_and_soft(ok);
+    if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float lt = s_l[r] + s_l[128 + r];
+      const float inv = 1.f / lt;
       const bool store = qpos < p.S;
       __nv_bfloat16* orow = p.o + ((int64_t)b * p.S + qpos) * p.ldo + (int64_t)h * p.hd;
-      for (int c = 0; c < 2 * nd; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
         uint32_t ov[32];
         __syncwarp();
         tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
@@ -360,9 +422,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
         uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
         const int nv = min(32, p.hd - 32 * c) / 8;
-        for (int v = 0; v < nv; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          if (v < nv) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
-      if (store) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(l);
+      if (store && half == 0) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(lt);
     }
   }
   tc_fence_before();
@@ -376,22 +440,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 
 // --------------------------------------------------------------------------- backward pieces
 
-// delta[h][t] = sum_d dO[t, h hd + d] O[t, h hd + d]; one warp per (token, head).
+// delta[h][t] = sum_d dO[t, h hd + d] O[t, h hd + d], and the dQ accumulator's segment
+// [t][h hd, (h + 1) hd) set to zero (the backward adds into it); half a warp per (token, head),
+// eight elements (16 bytes) of each row per lane.
 __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ d_o,
-                                  int64_t ld, int64_t T, int hq, int hd, float* __restrict__ delta) {
+                                  int64_t ld, int64_t T, int hq, int hd, float* __restrict__ delta,
+                                  float* __restrict__ dq_acc) {
   pdl_wait();
-  const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (item >= T * hq) return;
-  const int64_t t = item / hq;
-  const int h = (int)(item % hq);
-  const __nv_bfloat16* a = o + t * ld + (int64_t)h * hd;
-  const __nv_bfloat16* c = d_o + t * ld + (int64_t)h * hd;
+  const int64_t item = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const int sub = threadIdx.x & 15;
+  const bool live = item < T * hq;
+  const int64_t t = live ? item / hq : 0;
+  const int h = live ? (int)(item % hq) : 0;
   float acc = 0.f;
-  for (int d = lane; d < hd; d += 32) acc += __bfloat162float(a[d]) * __bfloat162float(c[d]);
+  if (live) {
+    if (8 * sub < hd) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + t * ld + (int64_t)h * hd + 8 * sub);
+      const uint4 c = *reinterpret_cast<const uint4*>(d_o + t * ld + (int64_t)h * hd + 8 * sub);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) delta[(int64_t)h * T + t] = acc;
+      for (int k = 0; k < 4; ++k) {
+        const float2 fa = __bfloat1622float2(a2[k]), fc = __bfloat1622float2(c2[k]);
+        acc += fa.x * fc.x + fa.y * fc.y;
+      }
+    }
+    float* z = dq_acc + (t * hq + h) * (int64_t)hd;
+    for (int d = 4 * sub; d < hd; d += 64) *reinterpret_cast<float4*>(z + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int s = 8; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (live && sub == 0) delta[(int64_t)h * T + t] = acc;
 }
 
 // dq[t * ldq + c] = bf16(acc[t * n + c]) for a [T, n] fp32 accumulator (n % 4 == 0), four
@@ -418,11 +497,11 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
   uint8_t* sdo = sq + nd * kChunk;     // dO_i
   uint8_t* spt = sdo + nd * kChunk;    // P^T: 2 chunks (128 queries)
   uint8_t* sdst = spt + 2 * kChunk;    // dS^T: 2 chunks
-  // P^T and dS^T are also the four dQ boxes (128 query rows x 32 fp32, 128-byte swizzle) once the
-  // MMAs of an iteration have read them
-  float* s_lse = reinterpret_cast<float*>(sdst + 2 * kChunk);  // [128]
-  float* s_delta = s_lse + 128;                                // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_delta + 128);
+  // P^T and dS^T also hold the dQ boxes (32 query rows x 32 fp32 per warp and box, 128-byte
+  // swizzle) once the MMAs of an iteration have read them
+  float* s_lse = reinterpret_cast<float*>(sdst + 2 * kChunk);  // [2][128] by iteration parity
+  float* s_delta = s_lse + 256;                                // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_delta + 256);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = bars + 2;
@@ -540,26 +619,42 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
     const int r = quarter * 32 + lane;           // key row of the tile (S^T, dP^T, dV, dK) or query row (dQ)
     const int kpos = kt * kTile + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const bool lead = cw == 0 && lane == 0;      // issues the dQ reductions
     const float log2e = 1.4426950408889634f;
+    // This warp's dQ boxes: head-dimension columns 64 half .. + 31 over its rows of P^T chunk `half`,
+    // columns 64 half + 32 .. + 63 over its rows of dS^T chunk `half`: the same shared memory the
+    // warp itself rewrites next (P^T and dS^T rows r, columns 64 half .. + 63), so one wait of its
+    // own bulk reads orders the two.
+    uint8_t* box0 = spt + half * kChunk + quarter * 32 * 128;
+    uint8_t* box1 = sdst + half * kChunk + quarter * 32 * 128;
+    // LSE and delta of a query tile are staged in shared memory (two buffers by iteration parity),
+    // read from global memory one iteration ahead
+    float n_lse = 0.f, n_delta = 0.f;
+    auto fetch = [&](int it) {
+      const int qp = it_qtile(it) * kTile + r;
+      const int64_t at = (int64_t)it_head(it) * T + (int64_t)b * p.S + qp;
+      n_lse = qp < p.S ? p.lse[at] * log2e : 0.f;
+      n_delta = qp < p.S ? p.delta[at] : 0.f;
+    };
+    if (half == 0 && n_it > 0) fetch(0);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int h = it_head(it), qt = it_qtile(it);
-      const int qpos_r = qt * kTile + r;
-      // The previous iteration's dQ reductions have read their boxes (P^T and dS^T are written
-      // below) and every reader of the previous LSE and delta is past this point. `ok` is the same
-      // in every compute thread here (combined at the end of each iteration).
-      if (lead) bulk_wait_read<0>();
-      named_bar_bwd();
-      if (!ok) break;
+      float* lse_it = s_lse + (it & 1) * 128;
+      float* delta_it = s_delta + (it & 1) * 128;
       if (half == 0) {
-        s_lse[r] = qpos_r < p.S ? p.lse[(int64_t)h * T + (int64_t)b * p.S + qpos_r] * log2e : 0.f;
-        s_delta[r] = qpos_r < p.S ? p.delta[(int64_t)h * T + (int64_t)b * p.S + qpos_r] : 0.f;
+        lse_it[r] = n_lse;
+        delta_it[r] = n_delta;
       }
-      named_bar_bwd();
+      // this iteration's LSE and delta are visible; `ok` is the same in every compute thread
+      ok = bar_and_bwd(ok);
+      if (!ok) break;
+      if (half == 0 && it + 1 < n_it) fetch(it + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
       if (ok) {
         tc_fence_after();
+        // this warp's previous dQ reductions have read its boxes (rewritten below)
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
         // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S
         const int cmin = kpos - qt * kTile;            // first visible query column
         const int cmax = p.S - 1 - qt * kTile;         // last query column inside the sequence
@@ -578,9 +673,9 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
             for (int e = 0; e < 2; ++e) {
               const int col = 32 * c + i + e;
               const bool vis = col >= cmin && col <= cmax && kpos < p.S;
-              const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - s_lse[col]) : 0.f;
+              const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - lse_it[col]) : 0.f;
               pv[e] = pe;
-              dv2[e] = pe * (__uint_as_float(dp[i + e]) - s_delta[col]);
+              dv2[e] = pe * (__uint_as_float(dp[i + e]) - delta_it[col]);
             }
             pw[i / 2] = pack2(pv[0], pv[1]);
             dw[i / 2] = pack2(dv2[0], dv2[1]);
@@ -595,7 +690,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
       }
       if (ok) {
         // dQ of this (head, query tile), lane r = query row qt * 128 + r: out of TMEM (which the next
-        // S^T may then overwrite), scaled into the boxes, added to the accumulator by bulk reductions
+        // S^T may then overwrite), scaled into this warp's boxes, added to the accumulator by bulk
+        // reductions of 32 rows x 32 columns
         tc_fence_after();
         uint32_t v0[32], v1[32];
         __syncwarp();
@@ -605,19 +701,19 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
         regs_after_wait(v1);
         tc_fence_before();
         mbar_arrive(dq_free);
-        st_dq_box_row(spt + (2 * half) * kDqBox, r, v0, p.scale);
-        st_dq_box_row(spt + (2 * half + 1) * kDqBox, r, v1, p.scale);
+        st_dq_box_row(box0, lane, v0, p.scale);
+        st_dq_box_row(box1, lane, v1, p.scale);
         fence_proxy_async_smem();
-      }
-      ok = bar_and_bwd(ok);
-      if (ok && lead) {
-        for (int c = 0; c < 4 && 32 * c < p.hd; ++c)
-          tma_reduce_add_4d(&p.dqmap, spt + c * kDqBox, 32 * c, h, qt * kTile, b);
-        bulk_commit();
+        __syncwarp();
+        if (lane == 0 && 64 * half < p.hd) {
+          tma_reduce_add_4d(&p.dqmap, box0, 64 * half, h, qt * kTile + 32 * quarter, b);
+          if (64 * half + 32 < p.hd) tma_reduce_add_4d(&p.dqmap, box1, 64 * half + 32, h, qt * kTile + 32 * quarter, b);
+          bulk_commit();
+        }
       }
     }
     // the reductions have completed before the CTA ends (and before its shared memory is reused)
-    if (lead) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
     // dK (half 1), dV (half 0) of this key tile: the MMAs of the last iteration have completed
     // (mma2_done); every lane takes part in the (warp-collective) loads, rows past the sequence
     // store nothing
@@ -639,7 +735,9 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
         for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
         uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
         const int nv = min(32, p.hd - 32 * c) / 8;
-        for (int q = 0; q < nv; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nv) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
       }
     }
   }
@@ -685,13 +783,13 @@ bool head_map(CUtensorMap* m, const void* ptr, int64_t ld, int n_seq, int S, int
 }
 
 // [hd, heads, S, n_seq] view of the [n_seq * S, heads * hd] fp32 dQ accumulator; boxes of
-// 32 x 1 x 128 x 1 (128 bytes per row), 128-byte swizzle.
+// 32 x 1 x 32 x 1 (32 rows of 128 bytes: one warp's rows), 128-byte swizzle.
 bool dq_acc_map(CUtensorMap* m, float* ptr, int n_seq, int S, int heads, int hd) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)S, (cuuint64_t)n_seq};
   cuuint64_t strides[3] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4, (cuuint64_t)S * heads * hd * 4};
-  cuuint32_t box[4] = {32, 1, 128, 1};
+  cuuint32_t box[4] = {32, 1, 32, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -700,8 +798,8 @@ bool dq_acc_map(CUtensorMap* m, float* ptr, int n_seq, int S, int heads, int hd)
 
 // Shared memory of a launch: sized for head_dim 128 whatever the head dimension, which also keeps
 // one CTA per SM (each CTA allocates all 512 TMEM columns).
-int fwd_smem() { return 1024 + 2 * kChunk + 8 * kChunk + 2 * kChunk + 256; }
-int bwd_smem() { return 1024 + 8 * kChunk + 4 * kChunk + 2 * 128 * 4 + 256; }
+int fwd_smem() { return 1024 + 2 * kChunk + 8 * kChunk + 2 * kChunk + 1024 + 256; }
+int bwd_smem() { return 1024 + 8 * kChunk + 4 * kChunk + 2 * 256 * 4 + 256; }
 
 }  // namespace
 
@@ -755,11 +853,10 @@ int attention_bwd(const void* q, const void* k, const void* v, const void* o, co
   float* dq_acc = static_cast<float*>(scratch);
   float* delta = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + ((T * hq * hd * 4 + 255) & ~int64_t(255)));
   if (!dq_acc_map(&p.dqmap, dq_acc, n_seq, S, hq, hd)) return 2;
-  if (cudaMemsetAsync(dq_acc, 0, (size_t)T * hq * hd * 4, s) != cudaSuccess) return 5;
   {
     const int64_t items = T * hq;
-    launch_kernel(attn_delta_kernel, (unsigned)((items + 7) / 8), 256, 0, s, static_cast<const __nv_bfloat16*>(o),
-                  static_cast<const __nv_bfloat16*>(d_o), ldq, T, hq, hd, delta);
+    launch_kernel(attn_delta_kernel, (unsigned)((items + 15) / 16), 256, 0, s, static_cast<const __nv_bfloat16*>(o),
+                  static_cast<const __nv_bfloat16*>(d_o), ldq, T, hq, hd, delta, dq_acc);
     if (launch_failed("sl_attention")) return 5;
     note_launch();
   }

@@ -85,7 +85,8 @@ def run(n_seq, S, hq, hkv, hd, seed, heads=None):
 
 
 @pytest.mark.parametrize("n_seq,S,hq,hkv,hd", [(2, 64, 4, 2, 32), (3, 40, 2, 2, 64), (2, 300, 4, 1, 128),
-                                                (1, 257, 2, 2, 128), (2, 128, 6, 3, 96)])
+                                                (1, 257, 2, 2, 128), (2, 128, 6, 3, 96), (2, 200, 4, 2, 40),
+                                                (1, 130, 2, 1, 8)])
 def test_attention_matches_oracle(n_seq, S, hq, hkv, hd):
     run(n_seq, S, hq, hkv, hd, seed=S + hd)
 
