@@ -32,6 +32,7 @@
 // into shared-memory boxes (over P^T and dS^T, free by then) and reaches the workspace accumulator
 // through bulk tensor reductions (fp32 adds in L2; several key tiles add to the same query rows).
 #include <cuda_bf16.h>
+#include <type_traits>
 
 #include <algorithm>
 #include <cmath>
@@ -52,6 +53,7 @@ constexpr int kChunk = 128 * 64 * 2;  // one 128-token x 64-element bf16 tile ch
 
 struct AttnFwdParams {
   CUtensorMap qmap, kmap, vmap;  // [head_dim, heads, seq_len, n_seq], boxes 64 x 1 x 128 x 1
+  CUtensorMap omap;              // the same view of o (bulk stores of the output tile)
   __nv_bfloat16* o;
   int64_t ldo;
   float* lse;                    // [n_q_heads][n_seq * seq_len]
@@ -172,6 +174,16 @@ __device__ __forceinline__ void st_dq_box_row(uint8_t* box, int r, const uint32_
                     __uint_as_float(v[4 * u + 2]) * mul, __uint_as_float(v[4 * u + 3]) * mul);
 }
 
+// Bulk tensor store of a shared-memory box through a 4-D tensor map (elements outside the tensor
+// are not written), tracked in the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* smem_src, int32_t c0, int32_t c1,
+                                             int32_t c2, int32_t c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 // Adds a shared-memory box to global memory through a 4-D tensor map (fp32 add in L2; elements
 // outside the tensor are skipped), tracked in the issuing thread's bulk async-groups.
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* m, const void* smem_src, int32_t c0, int32_t c1,
@@ -195,14 +207,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   float* s_l = reinterpret_cast<float*>(sp + 2 * kChunk);  // [2][128]: the two halves' row sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_l + 256);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]: K of a stage is free once S has read it
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]: V of a stage is free once P V has read it
+  uint64_t* s_full = bars + 9;    // [2]
+  uint64_t* s_free = bars + 11;   // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* pv_done = bars + 14;
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -213,8 +227,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], kSoftThreads);
     }
@@ -238,22 +254,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, nd * kChunk);
       for (int c = 0; c < nd; ++c) tma_load_4d(sq + c * kChunk, &p.qmap, q_full, 64 * c, h, qt * kTile, b);
-      uint32_t issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      // K and V of a stage have their own barriers: K of tile j + 1 is loaded as soon as S has read
+      // K of tile j - 1, ahead of V of tile j (which waits for P V of tile j - 2)
+      auto load = [&](int j, bool is_v) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) break;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * nd * kChunk);
-        issued |= 1u << s;
-        uint8_t* st = skv + s * 2 * nd * kChunk;
-        for (int c = 0; c < nd; ++c) {
-          tma_load_4d(st + c * kChunk, &p.kmap, &kv_full[s], 64 * c, g, j * kTile, b);
-          tma_load_4d(st + (nd + c) * kChunk, &p.vmap, &kv_full[s], 64 * c, g, j * kTile, b);
+        uint64_t* empty = is_v ? &v_empty[s] : &k_empty[s];
+        uint64_t* full = is_v ? &v_full[s] : &k_full[s];
+        if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) return false;
+        mbar_arrive_expect_tx(full, nd * kChunk);
+        uint8_t* st = skv + s * 2 * nd * kChunk + (is_v ? nd * kChunk : 0);
+        for (int c = 0; c < nd; ++c)
+          tma_load_4d(st + c * kChunk, is_v ? &p.vmap : &p.kmap, full, 64 * c, g, j * kTile, b);
+        return true;
+      };
+      int nk = 0, nv = 0;  // K and V tiles issued
+      if (load(0, false)) nk = 1;
+      for (int j = 0; nk > j && j < n_kv; ++j) {
+        if (j + 1 < n_kv) {
+          if (!load(j + 1, false)) break;
+          nk = j + 2;
         }
+        if (!load(j, true)) break;
+        nv = j + 1;
       }
       // every copy lands before the CTA may exit
       mbar_wait(q_full, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
-      for (int j = max(0, n_kv - 2); j < n_kv; ++j)
-        if (issued & (1u << (j & 1))) mbar_wait(&kv_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      for (int j = max(0, nk - 2); j < nk; ++j) mbar_wait(&k_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      for (int j = max(0, nv - 2); j < nv; ++j) mbar_wait(&v_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -263,17 +290,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       bool ok = mbar_wait(q_full, 0, abort_flag, p.err, DEV_TIMEOUT_MMA);
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(p_full, j & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
+        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
         tc_fence_after();
         const uint32_t bv = smem_u32(skv + (j & 1) * 2 * nd * kChunk + nd * kChunk);
         for (int t = 0; t < 8; ++t)
           umma_bf16(tmem + 256, kmajor_desc(ap, t), mnmajor_desc(bv, t), id_pv, (j > 0 || t > 0) ? 1u : 0u);
         umma_commit(pv_done);
-        umma_commit(&kv_empty[j & 1]);
+        umma_commit(&v_empty[j & 1]);
         return true;
       };
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        if (!mbar_wait(&k_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
         if (j >= 2 && !mbar_wait(&s_free[s], ((j - 2) >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) {
           ok = false;
           break;
@@ -283,6 +311,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         for (int t = 0; t < 4 * nd; ++t)
           umma_bf16(tmem + 128 * s, kmajor_desc(aq, t), kmajor_desc(bk, t), id_s, t > 0 ? 1u : 0u);
         umma_commit(&s_full[s]);
+        umma_commit(&k_empty[s]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(n_kv - 1);
@@ -322,24 +351,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // causal mask within the sequence: key k is visible to query q when k <= q and k < S
       const int kbase = j * kTile;
       const int kmax = min(qpos, p.S - 1) - kbase;   // last visible column of this tile
-      // (tiles wholly below the diagonal and inside the sequence, kmax >= 127, skip the masks)
-      const bool whole = kmax >= kTile - 1;
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (whole) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            mx[i & 3] = fmaxf(mx[i & 3], fmaxf(__uint_as_float(so[c][i]), __uint_as_float(sx[c][i])));
-      } else {
+      // Masked scores become -inf (then their exponentials are 0); tiles wholly below the diagonal
+      // and inside the sequence (kmax >= 127) skip this. Column 0 is always visible (kmax >= 0).
+      if (kmax < kTile - 1) {
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (own0 + 32 * c + i <= kmax) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(so[c][i]));
-            if (oth0 + 32 * c + i <= kmax) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sx[c][i]));
+            if (own0 + 32 * c + i > kmax) so[c][i] = __float_as_uint(-INFINITY);
+            if (oth0 + 32 * c + i > kmax) sx[c][i] = __float_as_uint(-INFINITY);
           }
       }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          mx[i & 3] = fmaxf(mx[i & 3], fmaxf(__uint_as_float(so[c][i]), __uint_as_float(sx[c][i])));
       const float mj = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // The running maximum moves only when a row's maximum grows by more than 2^8 in the
       // exponential's scale: the exponentials then stay below 256 and O and l keep one common
@@ -351,28 +379,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const float corr = (m == -INFINITY) ? 0.f : (grow ? ex2(m * p.scale_log2 - mb) : 1.f);
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pw[2][16];
-      if (whole) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float e0 = ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb);
-            const float e1 = ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb);
-            rs[(i >> 1) & 3] += e0 + e1;
-            pw[c][i / 2] = pack2(e0, e1);
-          }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int col = own0 + 32 * c + i;
-            const float e0 = (col <= kmax) ? ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb) : 0.f;
-            const float e1 = (col + 1 <= kmax) ? ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb) : 0.f;
-            rs[(i >> 1) & 3] += e0 + e1;
-            pw[c][i / 2] = pack2(e0, e1);
-          }
-      }
+        for (int i = 0; i < 32; i += 2) {
+          const float e0 = ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb);
+          const float e1 = ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb);
+          rs[(i >> 1) & 3] += e0 + e1;
+          pw[c][i / 2] = pack2(e0, e1);
+        }
       l = l * corr + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       if (j >= 1) {
         // the previous P V has landed in O (and read P): rescale this half of O when the maximum grew
@@ -406,27 +421,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // every softmax thread reaches this barrier (the loop above only breaks, never returns)
     ok = bar_and_soft(ok);
     if (ok) {
+      // O / l as bf16 into the P tile (free: the last P V has completed), laid out like a loaded
+      // tile (128-byte swizzle, 64-column chunks), then out by bulk tensor stores (rows past the
+      // sequence and columns past head_dim are not written)
       tc_fence_after();
       const float lt = s_l[r] + s_l[128 + r];
       const float inv = 1.f / lt;
-      const bool store = qpos < p.S;
-      __nv_bfloat16* orow = p.o + ((int64_t)b * p.S + qpos) * p.ldo + (int64_t)h * p.hd;
       for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
         uint32_t ov[32];
         __syncwarp();
         tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
         tmem_ld_wait_regs(ov);
-        if (!store || 32 * c >= p.hd) continue;
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-        const int nv = min(32, p.hd - 32 * c) / 8;
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          if (v < nv) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        st_swizzled_row32(sp, r, 32 * c, w);
       }
-      if (store && half == 0) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(lt);
+      fence_proxy_async_smem();
+      if (qpos < p.S && half == 0) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(lt);
+    }
+    ok = bar_and_soft(ok);
+    if (ok && cw == 0 && lane == 0) {
+      for (int c = 0; c < nd; ++c) tma_store_4d(&p.omap, sp + c * kChunk, 64 * c, h, qt * kTile, b);
+      bulk_commit();
+      bulk_wait_all();
     }
   }
   tc_fence_before();
@@ -655,10 +673,13 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
         // this warp's previous dQ reductions have read its boxes (rewritten below)
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S
+        // visible (key r, query c) pairs: kpos <= qpos = qt * 128 + c, qpos < S, kpos < S; a warp
+        // whose rows all lie wholly above the diagonal and inside the sequence needs no masks (the
+        // choice is the same for the whole warp: the chunks below hold warp-collective TMEM loads)
         const int cmin = kpos - qt * kTile;            // first visible query column
         const int cmax = p.S - 1 - qt * kTile;         // last query column inside the sequence
-        for (int c = 2 * half; c < 2 * half + 2; ++c) {
+        const bool whole = __all_sync(0xffffffffu, cmin <= 0 && cmax >= kTile - 1 && kpos < p.S);
+        auto soft_chunk = [&](int c, auto masked) {
           uint32_t st[32], dp[32];
           __syncwarp();
           tmem_ld32(tmem + lane_off + 32 * c, st);
@@ -667,21 +688,32 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
           regs_after_wait(dp);
           uint32_t pw[16], dw[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pv[2], dv2[2];
+          for (int i = 0; i < 32; i += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse_it + 32 * c + i);
+            const float4 d4 = *reinterpret_cast<const float4*>(delta_it + 32 * c + i);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dv4[4];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = 32 * c + i + e;
-              const bool vis = col >= cmin && col <= cmax && kpos < p.S;
-              const float pe = vis ? ex2(__uint_as_float(st[i + e]) * p.scale_log2 - lse_it[col]) : 0.f;
+            for (int e = 0; e < 4; ++e) {
+              float pe = ex2(__uint_as_float(st[i + e]) * p.scale_log2 - lv[e]);
+              if (decltype(masked)::value) {
+                const int col = 32 * c + i + e;
+                pe = (col >= cmin && col <= cmax && kpos < p.S) ? pe : 0.f;
+              }
               pv[e] = pe;
-              dv2[e] = pe * (__uint_as_float(dp[i + e]) - delta_it[col]);
+              dv4[e] = pe * (__uint_as_float(dp[i + e]) - dl[e]);
             }
             pw[i / 2] = pack2(pv[0], pv[1]);
-            dw[i / 2] = pack2(dv2[0], dv2[1]);
+            pw[i / 2 + 1] = pack2(pv[2], pv[3]);
+            dw[i / 2] = pack2(dv4[0], dv4[1]);
+            dw[i / 2 + 1] = pack2(dv4[2], dv4[3]);
           }
           st_swizzled_row32(spt, r, 32 * c, pw);
           st_swizzled_row32(sdst, r, 32 * c, dw);
+        };
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
+          if (whole) soft_chunk(c, std::false_type{});
+          else soft_chunk(c, std::true_type{});
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -808,7 +840,7 @@ int attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int6
   AttnFwdParams p;
   memset(&p, 0, sizeof(p));
   if (!head_map(&p.qmap, q, ldq, n_seq, S, hq, hd) || !head_map(&p.kmap, k, ldkv, n_seq, S, hkv, hd) ||
-      !head_map(&p.vmap, v, ldkv, n_seq, S, hkv, hd))
+      !head_map(&p.vmap, v, ldkv, n_seq, S, hkv, hd) || !head_map(&p.omap, o, ldo, n_seq, S, hq, hd))
     return 2;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.ldo = ldo;
