@@ -220,8 +220,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest (most key tiles) first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // Blocks start in linear order (x fastest): the linear index runs over query tiles slowest and
+  // from the last tile down, so every CTA of the longest tiles (most key tiles) starts before any
+  // shorter one and the SMs that take the short tiles last finish together (longest first).
+  const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  const int per_qt = p.hq * p.n_seq;
+  const int qt = gridDim.x - 1 - lin / per_qt;
+  const int h = (lin % per_qt) % p.hq, b = (lin % per_qt) / p.hq;
   const int g = h / (p.hq / p.hkv);
   const int n_kv = qt + 1;
   if (threadIdx.x == 0) {
@@ -534,7 +539,12 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // Longest first, as in the forward: the linear block index runs over key tiles slowest and from
+  // the first key tile up (key tile kt loops over the query tiles at or after it).
+  const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  const int per_kt = p.hkv * p.n_seq;
+  const int kt = lin / per_kt;
+  const int g = (lin % per_kt) % p.hkv, b = (lin % per_kt) / p.hkv;
   const int hpg = p.hq / p.hkv;
   const int n_qt = (p.S + kTile - 1) / kTile;
   const int n_it = hpg * (n_qt - kt);  // (query head of the group, query tile >= kt)
