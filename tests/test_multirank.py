@@ -54,8 +54,8 @@ def test_single_rank_needs_no_process_group():
 
 def _dp_rank_main(rank, world, port, out):
     """Two ranks, each with half of the batch's sequences: the rank-local statistics of the
-    criteria (oracle), summed with the same collective the library's blocks use (an fp64
-    all-reduce), give every rank the scores and the index sets of the whole batch."""
+    criteria (oracle), summed by the blocks' own `DataParallel` object (the fp64 all-reduce the
+    library's blocks issue), give every rank the scores and the index sets of the whole batch."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
                       LOCAL_RANK=str(rank))
     sys.path.insert(0, ROOT)
@@ -64,9 +64,11 @@ def _dp_rank_main(rank, world, port, out):
     import torch.distributed as dist
 
     import oracle
-    from contextual_sparsity_lora_b200 import inputs
+    from contextual_sparsity_lora_b200 import blocks, inputs
 
     dist.init_process_group("gloo")
+    dp = blocks.DataParallel()
+    assert dp.world == world and dp.active
     gen = inputs.generator(3)
     D, F, hq, hkv, hd, k = 64, 96, 4, 2, 8, 8
     x = inputs.activations_student_t(8 * 16, D, 4, 0.03, 30.0, gen)  # 8 sequences of 16 tokens
@@ -85,7 +87,7 @@ def _dp_rank_main(rank, world, port, out):
 
     mine = np.arange(8 * 16) // 64 == rank  # rank r holds sequences 4r .. 4r + 3
     t = torch.tensor(stats(mine), dtype=torch.float64)
-    dist.all_reduce(t)  # sum over the ranks
+    dp.all_reduce(t)  # sum over the ranks
     s = t.numpy()
     f2, q2, k2, v2 = np.split(s, np.cumsum([F, hq * hd, hkv * hd]))
     s_ffn = np.sqrt(f2)
@@ -167,3 +169,59 @@ def test_reference_arm_under_two_ranks_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert res["group_left_0"] and res["group_left_1"], "both ranks destroy the process group"
+
+
+def _grad_rank_main(rank, world, port, out):
+    """One rank's LoRA gradients in a block's flat buffer, summed by `DataParallel` (the one
+    fp32 all-reduce per block after the backward)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+
+    from contextual_sparsity_lora_b200 import blocks
+
+    dist.init_process_group("gloo")
+    dp = blocks.DataParallel()
+    shapes = [(32, 100), (7, 9), (64, 32)]  # A of 32 x 100, an odd-sized block, B of 64 x 32
+    buf = blocks._GradBuffer(shapes, "cpu")
+    g = torch.Generator().manual_seed(100 + rank)
+    mine = [torch.randn(*sh, generator=g) for sh in shapes]
+    for v, m in zip(buf.views, mine):
+        v.copy_(m)
+    dp.all_reduce(buf.flat)
+    out[rank] = ([m.numpy() for m in mine], [v.clone().numpy() for v in buf.views], list(buf.offsets),
+                 [v.data_ptr() - buf.flat.data_ptr() for v in buf.views])
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_data_parallel_sums_the_flat_gradient_buffer():
+    import numpy as np
+
+    ctx_ = mp.get_context("spawn")
+    with ctx_.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_grad_rank_main, args=(2, _free_port(), out), nprocs=2, start_method="spawn", join=True)
+        res = dict(out)
+    mine0, got0, offsets, byte_offsets = res[0]
+    mine1, got1, _, _ = res[1]
+    for a, b, c, d in zip(mine0, mine1, got0, got1):
+        np.testing.assert_array_equal(c, d)  # every rank holds the same sums
+        np.testing.assert_allclose(c, a + b, rtol=1e-6, atol=1e-6)
+    # the views start on 64-element boundaries of the one flat buffer (one collective covers all)
+    assert all(o % 64 == 0 for o in offsets) and offsets == sorted(offsets)
+    assert byte_offsets == [4 * o for o in offsets]
+
+
+def test_data_parallel_without_a_process_group_is_one_rank():
+    import torch
+
+    from contextual_sparsity_lora_b200 import blocks
+
+    dp = blocks.DataParallel()
+    assert dp.world == 1 and not dp.active
+    t = torch.arange(5, dtype=torch.float64)
+    dp.all_reduce(t)  # no collective: unchanged
+    assert t.tolist() == [0.0, 1.0, 2.0, 3.0, 4.0]
