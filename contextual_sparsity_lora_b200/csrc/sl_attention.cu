@@ -17,14 +17,16 @@
 // dimension is the contraction (Q K^T, dO V^T) and MN-major when the tokens are (P V, P^T dO,
 // dS^T Q, dS K).
 //
-// Forward: one CTA per (128-query tile, query head, sequence). Warp 0 loads Q once and the K/V
-// tiles through a two-stage ring; warp 1 issues the MMAs (S into two alternating TMEM buffers, so
-// S of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-9
+// Forward: one CTA per (128-query tile, query head, sequence), the tiles with the most key tiles
+// started first. Warp 0 loads Q once and the K/V tiles through a two-stage ring (K and V of a
+// stage on their own barriers); warp 1 issues the MMAs (S into two alternating TMEM buffers, so S
+// of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-9
 // run the online softmax, one query row (its TMEM lane) and half of the key columns per thread:
 // row maximum, exponentials, rescaling of O in TMEM when the maximum grows, P (bf16) into shared
-// memory for the P V MMA.
-// Backward: one CTA per (128-key tile, key/value head, sequence), looping over the query heads of
-// the group and the query tiles at or after the key tile: S^T and dP^T by MMA, P^T and dS^T by
+// memory for the P V MMA; at the end O / l goes through the P tile to bulk tensor stores.
+// Backward: one CTA per (128-key tile, key/value head, sequence), the first key tiles (the most
+// query tiles) started first, looping over the query heads of the group and the query tiles at or
+// after the key tile: S^T and dP^T by MMA, P^T and dS^T by
 // eight compute warps (one key row per thread, half of the query columns per warp), then
 // dV += P^T dO, dK += dS^T Q and dQ = dS K by MMA. dO and Q have separate barriers, so the next
 // dO loads once dV has read this one and dP^T of the next iteration starts while dQ is drained.
