@@ -17,13 +17,15 @@
 // dimension is the contraction (Q K^T, dO V^T) and MN-major when the tokens are (P V, P^T dO,
 // dS^T Q, dS K).
 //
-// Forward: one CTA per (128-query tile, query head, sequence), the tiles with the most key tiles
-// started first. Warp 0 loads Q once and the K/V tiles through a two-stage ring (K and V of a
-// stage on their own barriers); warp 1 issues the MMAs (S into two alternating TMEM buffers, so S
-// of the next key tile is computed while the softmax of this one runs, then O += P V); warps 2-9
-// run the online softmax, one query row (its TMEM lane) and half of the key columns per thread:
-// row maximum, exponentials, rescaling of O in TMEM when the maximum grows, P (bf16) into shared
-// memory for the P V MMA; at the end O / l goes through the P tile to bulk tensor stores.
+// Forward: persistent CTAs (one per SM) over the units (128-query tile, query head, sequence), the
+// units with the most key tiles first. Warp 0 loads each unit's Q and the K/V tiles through a
+// two-stage ring (K and V of a stage on their own barriers; the ring runs on over unit
+// boundaries); warp 1 issues the MMAs (S into two alternating TMEM buffers, so S of the next key
+// tile, also the next unit's first, is computed while the softmax or the epilogue runs, then
+// O += P V into one of two accumulators by unit); warps 2-9 run the online softmax, one query row
+// (its TMEM lane) and half of the key columns per thread: row maximum, exponentials, rescaling of
+// O in TMEM when the maximum grows, P (bf16) into shared memory for the P V MMA; at a unit's end
+// O / l goes through a staging tile to bulk tensor stores.
 // Backward: one CTA per (128-key tile, key/value head, sequence), the first key tiles (the most
 // query tiles) started first, looping over the query heads of the group and the query tiles at or
 // after the key tile: S^T and dP^T by MMA, P^T and dS^T by
@@ -203,36 +205,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nd = p.nd;
-  uint8_t* sq = smem;                          // Q: nd chunks
-  uint8_t* skv = sq + nd * kChunk;             // stage s: K (nd chunks) then V (nd chunks)
+  uint8_t* sq = smem;                          // Q: nd chunks (room for 2)
+  uint8_t* skv = sq + 2 * kChunk;              // stage s: K (nd chunks) then V (nd chunks)
   uint8_t* sp = skv + 2 * 2 * nd * kChunk;     // P: 2 chunks (128 keys)
-  float* s_l = reinterpret_cast<float*>(sp + 2 * kChunk);  // [2][128]: the two halves' row sums
+  uint8_t* sob = sp + 2 * kChunk;              // O staging tile for the bulk stores: 2 chunks
+  float* s_l = reinterpret_cast<float*>(sob + 2 * kChunk);  // [2][128]: the two halves' row sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_l + 256);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]: K of a stage is free once S has read it
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]: V of a stage is free once P V has read it
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* s_free = bars + 11;   // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* pv_done = bars + 14;
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_empty = bars + 1;   // Q of a query tile is free once its last S has read it
+  uint64_t* k_full = bars + 2;    // [2]
+  uint64_t* k_empty = bars + 4;   // [2]: K of a stage is free once S has read it
+  uint64_t* v_full = bars + 6;    // [2]
+  uint64_t* v_empty = bars + 8;   // [2]: V of a stage is free once P V has read it
+  uint64_t* s_full = bars + 10;   // [2]
+  uint64_t* s_free = bars + 12;   // [2]
+  uint64_t* p_full = bars + 14;
+  uint64_t* pv_done = bars + 15;
+  uint64_t* o_free = bars + 16;   // [2]: an O accumulator is free once the epilogue has read it
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Blocks start in linear order (x fastest): the linear index runs over query tiles slowest and
-  // from the last tile down, so every CTA of the longest tiles (most key tiles) starts before any
-  // shorter one and the SMs that take the short tiles last finish together (longest first).
-  const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  // Persistent CTAs: unit u = (query tile, query head, sequence) runs over query tiles slowest and
+  // from the last tile down (the most key tiles first); CTA c takes units c, c + grid, ... Every
+  // role walks the same units; K/V stages, S buffers and P follow one tile counter over all of a
+  // CTA's units, the two O accumulators alternate by unit.
+  const int n_qt = (p.S + kTile - 1) / kTile;
   const int per_qt = p.hq * p.n_seq;
-  const int qt = gridDim.x - 1 - lin / per_qt;
-  const int h = (lin % per_qt) % p.hq, b = (lin % per_qt) / p.hq;
-  const int g = h / (p.hq / p.hkv);
-  const int n_kv = qt + 1;
+  const int n_units = n_qt * per_qt;
+  const int hpg = p.hq / p.hkv;
+  auto unit = [&](int u, int& qt, int& h, int& b) {
+    qt = n_qt - 1 - u / per_qt;
+    h = (u % per_qt) % p.hq;
+    b = (u % per_qt) / p.hq;
+  };
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -240,6 +250,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], kSoftThreads);
+      mbar_init(&o_free[s], kSoftThreads);
     }
     mbar_init(p_full, kSoftThreads);
     mbar_init(pv_done, 1);
@@ -254,74 +265,105 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S buffers at columns 0 and 128, O at 256
+  const uint32_t tmem = *tmem_slot;  // S buffers at columns 0 and 128, O accumulators at 256 and 384
   pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, nd * kChunk);
-      for (int c = 0; c < nd; ++c) tma_load_4d(sq + c * kChunk, &p.qmap, q_full, 64 * c, h, qt * kTile, b);
-      // K and V of a stage have their own barriers: K of tile j + 1 is loaded as soon as S has read
-      // K of tile j - 1, ahead of V of tile j (which waits for P V of tile j - 2)
-      auto load = [&](int j, bool is_v) -> bool {
-        const int s = j & 1;
+      // Loads in order: Q of a unit right before K of its first key tile (once the previous unit's
+      // last S has read Q), K of tile t + 1 ahead of V of tile t.
+      auto load_kv = [&](int t, bool is_v, int g, int kv, int b) -> bool {
+        const int s = t & 1;
         uint64_t* empty = is_v ? &v_empty[s] : &k_empty[s];
         uint64_t* full = is_v ? &v_full[s] : &k_full[s];
-        if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) return false;
+        if (!mbar_wait(empty, ((t >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) return false;
         mbar_arrive_expect_tx(full, nd * kChunk);
         uint8_t* st = skv + s * 2 * nd * kChunk + (is_v ? nd * kChunk : 0);
         for (int c = 0; c < nd; ++c)
-          tma_load_4d(st + c * kChunk, is_v ? &p.vmap : &p.kmap, full, 64 * c, g, j * kTile, b);
+          tma_load_4d(st + c * kChunk, is_v ? &p.vmap : &p.kmap, full, 64 * c, g, kv * kTile, b);
         return true;
       };
-      int nk = 0, nv = 0;  // K and V tiles issued
-      if (load(0, false)) nk = 1;
-      for (int j = 0; nk > j && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          if (!load(j + 1, false)) break;
-          nk = j + 2;
+      int nq = 0, nk = 0, nv = 0;  // Q, K and V tiles issued
+      int pg = 0, pkv = 0, pb = 0;   // the tile whose V is still to load (tile nv when nk > nv)
+      bool ok = true;
+      for (int u = blockIdx.x, i = 0; ok && u < n_units; u += gridDim.x, ++i) {
+        int qt, h, b;
+        unit(u, qt, h, b);
+        const int g = h / hpg;
+        for (int j = 0; j <= qt; ++j) {
+          if (j == 0) {
+            // the previous unit's last V first (its P V does not wait for this unit), then Q
+            if (nk > nv) {
+              if (!load_kv(nv, true, pg, pkv, pb)) { ok = false; break; }
+              ++nv;
+            }
+            if (i > 0 && !mbar_wait(q_empty, (i - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER)) { ok = false; break; }
+            mbar_arrive_expect_tx(q_full, nd * kChunk);
+            for (int c = 0; c < nd; ++c) tma_load_4d(sq + c * kChunk, &p.qmap, q_full, 64 * c, h, qt * kTile, b);
+            ++nq;
+          }
+          if (!load_kv(nk, false, g, j, b)) { ok = false; break; }
+          ++nk;
+          if (j > 0) {
+            if (!load_kv(nv, true, pg, pkv, pb)) { ok = false; break; }
+            ++nv;
+          }
+          pg = g;
+          pkv = j;
+          pb = b;
         }
-        if (!load(j, true)) break;
-        nv = j + 1;
       }
+      if (ok && nk > nv && load_kv(nv, true, pg, pkv, pb)) ++nv;
       // every copy lands before the CTA may exit
-      mbar_wait(q_full, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
-      for (int j = max(0, nk - 2); j < nk; ++j) mbar_wait(&k_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
-      for (int j = max(0, nv - 2); j < nv; ++j) mbar_wait(&v_full[j & 1], (j >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      for (int t = max(0, nk - 2); t < nk; ++t) mbar_wait(&k_full[t & 1], (t >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
+      for (int t = max(0, nv - 2); t < nv; ++t) mbar_wait(&v_full[t & 1], (t >> 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(128, 128, 0, 0);          // S = Q K^T: both K-major over d
       const uint32_t id_pv = idesc_bf16(128, 64 * nd, 0, 1);     // O += P V: P K-major, V MN-major
       const uint32_t aq = smem_u32(sq), ap = smem_u32(sp);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.err, DEV_TIMEOUT_MMA);
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(p_full, j & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
-        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
+      // P V of tile t (key tile j of the CTA's unit i) into the unit's O accumulator
+      auto issue_pv = [&](int t, int i, int j) -> bool {
+        if (!mbar_wait(p_full, t & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
+        if (!mbar_wait(&v_full[t & 1], (t >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) return false;
+        // the first P V of a unit overwrites its accumulator: the epilogue of unit i - 2 has read it
+        if (j == 0 && i >= 2 && !mbar_wait(&o_free[i & 1], ((i >> 1) & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_MMA))
+          return false;
         tc_fence_after();
-        const uint32_t bv = smem_u32(skv + (j & 1) * 2 * nd * kChunk + nd * kChunk);
-        for (int t = 0; t < 8; ++t)
-          umma_bf16(tmem + 256, kmajor_desc(ap, t), mnmajor_desc(bv, t), id_pv, (j > 0 || t > 0) ? 1u : 0u);
+        const uint32_t bv = smem_u32(skv + (t & 1) * 2 * nd * kChunk + nd * kChunk);
+        for (int k = 0; k < 8; ++k)
+          umma_bf16(tmem + 256 + 128 * (i & 1), kmajor_desc(ap, k), mnmajor_desc(bv, k), id_pv, (j > 0 || k > 0) ? 1u : 0u);
         umma_commit(pv_done);
-        umma_commit(&v_empty[j & 1]);
+        umma_commit(&v_empty[t & 1]);
         return true;
       };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&k_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&s_free[s], ((j - 2) >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) {
-          ok = false;
-          break;
+      bool ok = true;
+      int t = 0;
+      for (int u = blockIdx.x, i = 0; ok && u < n_units; u += gridDim.x, ++i) {
+        int qt, h, b;
+        unit(u, qt, h, b);
+        if (!mbar_wait(q_full, i & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+        for (int j = 0; j <= qt; ++j, ++t) {
+          const int s = t & 1;
+          if (!mbar_wait(&k_full[s], (t >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) { ok = false; break; }
+          if (t >= 2 && !mbar_wait(&s_free[s], ((t - 2) >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t bk = smem_u32(skv + s * 2 * nd * kChunk);
+          for (int k = 0; k < 4 * nd; ++k)
+            umma_bf16(tmem + 128 * s, kmajor_desc(aq, k), kmajor_desc(bk, k), id_s, k > 0 ? 1u : 0u);
+          umma_commit(&s_full[s]);
+          umma_commit(&k_empty[s]);
+          if (j == qt) umma_commit(q_empty);
+          if (j >= 1 && !issue_pv(t - 1, i, j - 1)) { ok = false; break; }
         }
-        tc_fence_after();
-        const uint32_t bk = smem_u32(skv + s * 2 * nd * kChunk);
-        for (int t = 0; t < 4 * nd; ++t)
-          umma_bf16(tmem + 128 * s, kmajor_desc(aq, t), kmajor_desc(bk, t), id_s, t > 0 ? 1u : 0u);
-        umma_commit(&s_full[s]);
-        umma_commit(&k_empty[s]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        // this unit's last P V before the next unit's first S: the epilogue needs it first
+        if (ok && !issue_pv(t - 1, i, qt)) ok = false;
       }
-      if (ok) issue_pv(n_kv - 1);
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN);
     }
@@ -329,130 +371,144 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // Eight softmax warps: warp w holds query rows 32 (w % 4) .. + 31 (its TMEM lanes) and one half
     // of the key columns of each S tile (exponentials, P) and of O (rescale, output). Both halves
     // read the whole S row for its maximum, so they keep the same running maximum without an
-    // exchange; their partial row sums meet once, at the end.
+    // exchange; their partial row sums meet once per unit, at its end.
     const int cw = warp - 2;
     const int quarter = warp & 3;
     const int half = cw >> 2;
     const int r = quarter * 32 + lane;               // query row in the tile = TMEM lane
-    const int qpos = qt * kTile + r;                 // position in the sequence
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int own0 = 64 * half, oth0 = 64 - own0;    // first key column of this half / the other
-    float m = -INFINITY, l = 0.f;                    // l: this half's share of the row sum
+    const bool storer = cw == 0 && lane == 0;        // issues the output tile's bulk stores
     bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int s = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t so[2][32], sx[2][32];                 // this half's columns, the other half's
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(tmem + lane_off + 128 * s + own0 + 32 * c, so[c]);
-        tmem_ld32(tmem + lane_off + 128 * s + oth0 + 32 * c, sx[c]);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[s]);
-      // causal mask within the sequence: key k is visible to query q when k <= q and k < S
-      const int kbase = j * kTile;
-      const int kmax = min(qpos, p.S - 1) - kbase;   // last visible column of this tile
-      // Masked scores become -inf (then their exponentials are 0); tiles wholly below the diagonal
-      // and inside the sequence (kmax >= 127) skip this. Column 0 is always visible (kmax >= 0).
-      if (kmax < kTile - 1) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (own0 + 32 * c + i > kmax) so[c][i] = __float_as_uint(-INFINITY);
-            if (oth0 + 32 * c + i > kmax) sx[c][i] = __float_as_uint(-INFINITY);
-          }
-      }
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          mx[i & 3] = fmaxf(mx[i & 3], fmaxf(__uint_as_float(so[c][i]), __uint_as_float(sx[c][i])));
-      const float mj = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      // The running maximum moves only when a row's maximum grows by more than 2^8 in the
-      // exponential's scale: the exponentials then stay below 256 and O and l keep one common
-      // reference, so O is rescaled in TMEM rarely (after the first tiles almost never).
-      const float m_cand = fmaxf(m, mj);
-      const bool grow = m == -INFINITY || (m_cand - m) * p.scale_log2 > 8.0f;
-      const float m_new = grow ? m_cand : m;
-      const float mb = m_new * p.scale_log2;
-      const float corr = (m == -INFINITY) ? 0.f : (grow ? ex2(m * p.scale_log2 - mb) : 1.f);
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pw[2][16];
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float e0 = ex2(__uint_as_float(so[c][i]) * p.scale_log2 - mb);
-          const float e1 = ex2(__uint_as_float(so[c][i + 1]) * p.scale_log2 - mb);
-          rs[(i >> 1) & 3] += e0 + e1;
-          pw[c][i / 2] = pack2(e0, e1);
-        }
-      l = l * corr + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-      if (j >= 1) {
-        // the previous P V has landed in O (and read P): rescale this half of O when the maximum grew
-        if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
+    int t = 0;
+    for (int u = blockIdx.x, i = 0; u < n_units; u += gridDim.x, ++i) {
+      int qt, h, b;
+      unit(u, qt, h, b);
+      const int qpos = qt * kTile + r;               // position in the sequence
+      const uint32_t o_tm = tmem + lane_off + 256 + 128 * (i & 1);
+      float m = -INFINITY, l = 0.f;                  // l: this half's share of the row sum
+      for (int j = 0; j <= qt && ok; ++j, ++t) {
+        const int s = t & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (t >> 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
-          for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
-            uint32_t ov[32];
-            __syncwarp();
-            tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
-            tmem_ld_wait_regs(ov);
+        uint32_t so[2][32], sx[2][32];               // this half's columns, the other half's
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-            tmem_st32(tmem + lane_off + 256 + 32 * c, ov);
-          }
-          tmem_st_wait();
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tmem + lane_off + 128 * s + own0 + 32 * c, so[c]);
+          tmem_ld32(tmem + lane_off + 128 * s + oth0 + 32 * c, sx[c]);
         }
-      }
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[s]);
+        // causal mask within the sequence: key k is visible to query q when k <= q and k < S
+        const int kbase = j * kTile;
+        const int kmax = min(qpos, p.S - 1) - kbase;  // last visible column of this tile
+        // Masked scores become -inf (then their exponentials are 0); tiles wholly below the
+        // diagonal and inside the sequence (kmax >= 127) skip this. Column 0 is always visible.
+        if (kmax < kTile - 1) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) st_swizzled_row32(sp, r, own0 + 32 * c, pw[c]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-      m = m_new;
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
-    s_l[half * 128 + r] = l;
-    // every softmax thread reaches this barrier (the loop above only breaks, never returns)
-    ok = bar_and_soft(ok);
-    if (ok) {
-      // O / l as bf16 into the P tile (free: the last P V has completed), laid out like a loaded
-      // tile (128-byte swizzle, 64-column chunks), then out by bulk tensor stores (rows past the
-      // sequence and columns past head_dim are not written)
-      tc_fence_after();
-      const float lt = s_l[r] + s_l[128 + r];
-      const float inv = 1.f / lt;
-      for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
-        uint32_t ov[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_off + 256 + 32 * c, ov);
-        tmem_ld_wait_regs(ov);
-        uint32_t w[16];
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) w[i / 2] = pack2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
-        st_swizzled_row32(sp, r, 32 * c, w);
+            for (int e = 0; e < 32; ++e) {
+              if (own0 + 32 * c + e > kmax) so[c][e] = __float_as_uint(-INFINITY);
+              if (oth0 + 32 * c + e > kmax) sx[c][e] = __float_as_uint(-INFINITY);
+            }
+        }
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            mx[e & 3] = fmaxf(mx[e & 3], fmaxf(__uint_as_float(so[c][e]), __uint_as_float(sx[c][e])));
+        const float mj = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        // The running maximum moves only when a row's maximum grows by more than 2^8 in the
+        // exponential's scale: the exponentials then stay below 256 and O and l keep one common
+        // reference, so O is rescaled in TMEM rarely (after the first tiles almost never).
+        const float m_cand = fmaxf(m, mj);
+        const bool grow = m == -INFINITY || (m_cand - m) * p.scale_log2 > 8.0f;
+        const float m_new = grow ? m_cand : m;
+        const float mb = m_new * p.scale_log2;
+        const float corr = (m == -INFINITY) ? 0.f : (grow ? ex2(m * p.scale_log2 - mb) : 1.f);
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pw[2][16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float e0 = ex2(__uint_as_float(so[c][e]) * p.scale_log2 - mb);
+            const float e1 = ex2(__uint_as_float(so[c][e + 1]) * p.scale_log2 - mb);
+            rs[(e >> 1) & 3] += e0 + e1;
+            pw[c][e / 2] = pack2(e0, e1);
+          }
+        l = l * corr + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+        if (j >= 1) {
+          // the previous P V has landed in O (and read P): rescale this half of O when the maximum
+          // grew (the first key tile of a unit: the previous unit's epilogue waited for its last P V)
+          if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, corr != 1.f)) {
+            for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
+              uint32_t ov[32];
+              __syncwarp();
+              tmem_ld32(o_tm + 32 * c, ov);
+              tmem_ld_wait_regs(ov);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+              tmem_st32(o_tm + 32 * c, ov);
+            }
+            tmem_st_wait();
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) st_swizzled_row32(sp, r, own0 + 32 * c, pw[c]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        m = m_new;
       }
-      fence_proxy_async_smem();
-      if (qpos < p.S && half == 0) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(lt);
+      // this unit's last P V (tile t - 1) has landed
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, abort_flag, p.err, DEV_TIMEOUT_EPILOGUE));
+      // the previous unit's bulk stores have read the staging tile (rewritten below)
+      if (storer) bulk_wait_read<0>();
+      s_l[half * 128 + r] = l;
+      // every softmax thread reaches both barriers of every unit (the loops only break)
+      ok = bar_and_soft(ok);
+      if (ok) {
+        // O / l as bf16 into the staging tile, laid out like a loaded tile (128-byte swizzle,
+        // 64-column chunks), then out by bulk tensor stores (rows past the sequence and columns
+        // past head_dim are not written); the accumulator is released as soon as it is read
+        tc_fence_after();
+        const float lt = s_l[r] + s_l[128 + r];
+        const float inv = 1.f / lt;
+        for (int c = 2 * half; c < 2 * half + 2 && c < 2 * nd; ++c) {
+          uint32_t ov[32];
+          __syncwarp();
+          tmem_ld32(o_tm + 32 * c, ov);
+          tmem_ld_wait_regs(ov);
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) w[e / 2] = pack2(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv);
+          st_swizzled_row32(sob, r, 32 * c, w);
+        }
+        tc_fence_before();
+        mbar_arrive(&o_free[i & 1]);
+        fence_proxy_async_smem();
+        if (qpos < p.S && half == 0) p.lse[(int64_t)h * p.n_seq * p.S + (int64_t)b * p.S + qpos] = m * p.scale + logf(lt);
+      }
+      ok = bar_and_soft(ok);
+      if (!ok) break;
+      if (storer) {
+        for (int c = 0; c < nd; ++c) tma_store_4d(&p.omap, sob + c * kChunk, 64 * c, h, qt * kTile, b);
+        bulk_commit();
+      }
     }
-    ok = bar_and_soft(ok);
-    if (ok && cw == 0 && lane == 0) {
-      for (int c = 0; c < nd; ++c) tma_store_4d(&p.omap, sp + c * kChunk, 64 * c, h, qt * kTile, b);
-      bulk_commit();
-      bulk_wait_all();
-    }
+    if (storer) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -842,7 +898,7 @@ bool dq_acc_map(CUtensorMap* m, float* ptr, int n_seq, int S, int heads, int hd)
 
 // Shared memory of a launch: sized for head_dim 128 whatever the head dimension, which also keeps
 // one CTA per SM (each CTA allocates all 512 TMEM columns).
-int fwd_smem() { return 1024 + 2 * kChunk + 8 * kChunk + 2 * kChunk + 1024 + 256; }
+int fwd_smem() { return 1024 + 2 * kChunk + 8 * kChunk + 2 * kChunk + 2 * kChunk + 1024 + 256; }
 int bwd_smem() { return 1024 + 8 * kChunk + 4 * kChunk + 2 * 256 * 4 + 256; }
 
 }  // namespace
@@ -873,7 +929,14 @@ int attention_fwd(const void* q, const void* k, const void* v, int64_t ldq, int6
       return 5;
     attr = true;
   }
-  const dim3 grid((unsigned)((S + kTile - 1) / kTile), (unsigned)hq, (unsigned)n_seq);
+  static int n_sm = 0;
+  if (!n_sm) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+      return 5;
+  }
+  const int64_t n_units = (int64_t)((S + kTile - 1) / kTile) * hq * n_seq;
+  const dim3 grid((unsigned)std::min<int64_t>(n_units, n_sm));
   launch_kernel(attn_fwd_kernel, grid, kAttnThreads, smem, s, p);
   if (launch_failed("sl_attention")) return 5;
   note_launch();
